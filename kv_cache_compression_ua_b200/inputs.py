@@ -1,0 +1,235 @@
+"""Seeded synthetic inputs for the Universal Attention hot path.
+
+This module is shared by the tests, the benchmark and the smoke check.  It draws
+random numbers and nothing else: it holds none of the method's arithmetic, so the
+oracle and the CUDA library can both consume its output without sharing code.
+
+Generator: counter-based splitmix64 (Steele, Lea & Flood, "Fast splittable
+pseudorandom number generators", OOPSLA 2014; finaliser constants as published there)
+over a per-tensor stream key.  Uniforms take the top 53 bits; normals use the
+Box-Muller transform.  Values are drawn in fp64 and rounded once to the workload's
+dtype (round-to-nearest-even, fp64 -> fp32 -> bf16), and both sides consume the
+rounded values.
+
+Workloads (shapes and value distributions of the pages' 1B/3B Llama3-style models at
+4k-16k context; no benchmark item is reproduced -- these synthetic tensors stand in for
+the pages' RULER / LongBench-E / Dolma inputs):
+  tiny_fp32      B1 T256 H1 Hkv1 d64 fp32; Q,K,V,G ~ N(0,1); a_q,a_k ~ N(-2,1); alpha 4, beta -2
+  prefill_1b     B8 T4096 H32 Hkv8 d64 bf16; alpha ~ U(2,6), beta ~ U(-3,-1) per KV head
+  prefill_1b_16k B1 T16384, 1B shapes; a_k bimodal 0.9 N(-1,0.5) + 0.1 N(-6,0.5)
+  decode_1b      B32, prefill as prefill_1b_16k, then 256 steps of fresh tokens
+  fwdbwd_3b      B4 T8192 H24 Hkv8 d128 bf16, as prefill_1b plus dO ~ N(0,1)
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+_M64 = np.uint64(0xFFFFFFFFFFFFFFFF)
+_GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_MUL1 = np.uint64(0xBF58476D1CE4E5B9)
+_MUL2 = np.uint64(0x94D049BB133111EB)
+
+
+def _mix(z: np.ndarray) -> np.ndarray:
+    z = (z ^ (z >> np.uint64(30))) * _MUL1
+    z = (z ^ (z >> np.uint64(27))) * _MUL2
+    return z ^ (z >> np.uint64(31))
+
+
+def _stream_key(seed: int, stream: int) -> np.uint64:
+    with np.errstate(over="ignore"):
+        z = np.array([(seed * 0x100000001B3 + stream * 0x632BE59BD9B4E019) & 0xFFFFFFFFFFFFFFFF],
+                     dtype=np.uint64)
+        return _mix(z + _GAMMA)[0]
+
+
+def _mix_ctr(key: np.uint64, ctr: np.ndarray) -> np.ndarray:
+    with np.errstate(over="ignore"):
+        return _mix(key + ctr * _GAMMA)
+
+
+def _u53(bits: np.ndarray) -> np.ndarray:
+    return (bits >> np.uint64(11)).astype(np.float64) * (1.0 / 9007199254740992.0)
+
+
+def _lin_index(full_shape, lead_lo, lead_n) -> np.ndarray:
+    """Linear (row-major) indices, within full_shape, of the box that takes lead_n[i]
+    entries from lead_lo[i] on each leading axis and all entries of the others."""
+    full_shape = tuple(int(s) for s in full_shape)
+    idx = np.zeros((), dtype=np.uint64)
+    for ax, size in enumerate(full_shape):
+        if ax < len(lead_n):
+            r = np.arange(lead_lo[ax], lead_lo[ax] + lead_n[ax], dtype=np.uint64)
+        else:
+            r = np.arange(size, dtype=np.uint64)
+        idx = idx[..., None] * np.uint64(size) + r
+    return idx
+
+
+def uniform(seed: int, stream: int, shape, lo=0.0, hi=1.0, box=None) -> np.ndarray:
+    """U(lo, hi) draws for `shape`; `box` = (lead_lo, lead_n) draws only that box of the
+    full shape, with the same values the full draw would give there."""
+    key = _stream_key(seed, stream)
+    lead_lo, lead_n = box if box is not None else ((), ())
+    lin = _lin_index(shape, lead_lo, lead_n)
+    u = _u53(_mix_ctr(key, lin + np.uint64(1)))
+    return lo + (hi - lo) * u
+
+
+def normal(seed: int, stream: int, shape, mean=0.0, std=1.0, box=None) -> np.ndarray:
+    """N(mean, std^2) draws by Box-Muller from the counter pair (2i+1, 2i+2)."""
+    key = _stream_key(seed, stream)
+    lead_lo, lead_n = box if box is not None else ((), ())
+    lin = _lin_index(shape, lead_lo, lead_n) * np.uint64(2)
+    u1 = 1.0 - _u53(_mix_ctr(key, lin + np.uint64(1)))     # (0, 1]
+    u2 = _u53(_mix_ctr(key, lin + np.uint64(2)))
+    z = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+    return mean + std * z
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """fp64 -> fp32 (RNE) -> bf16 (RNE), returned as float32 values."""
+    f = np.ascontiguousarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    u = (u + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)
+    out = u.astype(np.uint32).view(np.float32)
+    nan = np.isnan(f)
+    if nan.any():
+        out = out.copy()
+        out[nan] = np.nan
+    return out
+
+
+def to_dtype(x: np.ndarray, dtype: str) -> np.ndarray:
+    if dtype == "f32":
+        return np.ascontiguousarray(x, dtype=np.float32)
+    if dtype == "bf16":
+        return round_bf16(x)
+    raise ValueError(dtype)
+
+
+# stream ids, in the draw order Q, K, V, G, a_q, a_k, alpha, beta, dO
+S_Q, S_K, S_V, S_G, S_AQ, S_AK, S_ALPHA, S_BETA, S_DO = range(9)
+S_AK_MODE = 20       # Bernoulli selector of the bimodal a_k
+S_AK_SLOW = 21       # the slow mode's draws
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    B: int
+    T: int
+    H: int
+    Hkv: int
+    d: int
+    dtype: str              # "f32" | "bf16"
+    seed: int
+    theta: float = 500000.0
+    alpha_fixed: float | None = None
+    beta_fixed: float | None = None
+    bimodal_ak: bool = False
+    with_grad: bool = False
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.d))
+
+    @property
+    def G(self) -> int:
+        return self.H // self.Hkv
+
+    def resized(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS = {
+    "tiny_fp32": Workload("tiny_fp32", 1, 256, 1, 1, 64, "f32", 1001, alpha_fixed=4.0, beta_fixed=-2.0),
+    "prefill_1b": Workload("prefill_1b", 8, 4096, 32, 8, 64, "bf16", 1002),
+    "prefill_1b_16k": Workload("prefill_1b_16k", 1, 16384, 32, 8, 64, "bf16", 1003, bimodal_ak=True),
+    "decode_1b": Workload("decode_1b", 32, 16384, 32, 8, 64, "bf16", 1004, bimodal_ak=True),
+    "fwdbwd_3b": Workload("fwdbwd_3b", 4, 8192, 24, 8, 128, "bf16", 1005, with_grad=True),
+}
+
+DECODE_STEPS = 256
+DECODE_THRESHOLDS = (0.05, 0.15)
+
+
+def bimodal_ak(seed: int, shape, box=None, streams=(S_AK_MODE, S_AK, S_AK_SLOW)):
+    """a_k logits: with probability 0.1 from N(-6, 0.5) (slowly decaying keys),
+    otherwise from N(-1, 0.5)."""
+    s_mode, s_fast, s_slow = streams
+    sel = uniform(seed, s_mode, shape, box=box) < 0.1
+    fast = normal(seed, s_fast, shape, -1.0, 0.5, box=box)
+    slow = normal(seed, s_slow, shape, -6.0, 0.5, box=box)
+    return np.where(sel, slow, fast)
+
+
+PREFILL_NAMES = ("q", "k", "v", "g", "a_q", "a_k", "alpha", "beta", "d_o")
+
+
+def _draw(w: Workload, name: str, seed: int, full_shape, box):
+    if name in ("q", "k", "v", "g", "d_o"):
+        stream = {"q": S_Q, "k": S_K, "v": S_V, "g": S_G, "d_o": S_DO}[name]
+        return to_dtype(normal(seed, stream, full_shape, box=box), w.dtype)
+    if name == "a_q":
+        return normal(seed, S_AQ, full_shape, -2.0, 1.0, box=box).astype(np.float32)
+    if name == "a_k":
+        x = bimodal_ak(seed, full_shape, box=box) if w.bimodal_ak else \
+            normal(seed, S_AK, full_shape, -2.0, 1.0, box=box)
+        return x.astype(np.float32)
+    raise KeyError(name)
+
+
+def make_prefill_inputs(w: Workload, T: int | None = None, B: int | None = None,
+                        names=None, b0: int = 0) -> dict:
+    """Prefill inputs as float32 numpy arrays holding values already rounded to w.dtype.
+
+    The values are those of the full workload shape; B / T / b0 select the batches
+    b0 .. b0+B-1 and the leading T tokens of that full draw, so a reduced case holds
+    exactly a slice of the full one.  `names` limits which tensors are drawn."""
+    Bf, Tf, H, Hkv, d = w.B, w.T, w.H, w.Hkv, w.d
+    B = Bf - b0 if B is None else B
+    T = Tf if T is None else T
+    assert 0 <= b0 and b0 + B <= Bf and T <= Tf
+    names = [n for n in PREFILL_NAMES if (names is None or n in names)]
+    if not w.with_grad and "d_o" in names:
+        names.remove("d_o")
+    s = w.seed
+    out = {}
+    for n in names:
+        if n == "alpha":
+            out[n] = (np.full(Hkv, w.alpha_fixed) if w.alpha_fixed is not None
+                      else uniform(s, S_ALPHA, (Hkv,), 2.0, 6.0)).astype(np.float32)
+            continue
+        if n == "beta":
+            out[n] = (np.full(Hkv, w.beta_fixed) if w.beta_fixed is not None
+                      else uniform(s, S_BETA, (Hkv,), -3.0, -1.0)).astype(np.float32)
+            continue
+        heads = H if n in ("q", "g", "d_o") else Hkv
+        full = (Bf, Tf, heads, d) if n in ("q", "k", "v", "g", "d_o") else (Bf, Tf, heads)
+        arr = np.empty((B, T) + full[2:], dtype=np.float32)
+        for bi in range(B):            # one batch at a time keeps the fp64 temporaries small
+            arr[bi] = _draw(w, n, s, full, ((b0 + bi, 0), (1, T)))[0]
+        out[n] = arr
+    return out
+
+
+def make_decode_token(w: Workload, step: int, B: int | None = None) -> dict:
+    """Fresh token for decode step `step`: q, g [B,H,d], k, v [B,Hkv,d] ~ N(0,1);
+    a_q [B,Hkv] ~ N(-2,1); a_k as in the prefill (bimodal when the workload is)."""
+    B = w.B if B is None else B
+    s = w.seed * 7919 + 100003 * (step + 1)
+    box = ((0,), (B,))
+    out = {
+        "q": to_dtype(normal(s, S_Q, (w.B, w.H, w.d), box=box), w.dtype),
+        "k": to_dtype(normal(s, S_K, (w.B, w.Hkv, w.d), box=box), w.dtype),
+        "v": to_dtype(normal(s, S_V, (w.B, w.Hkv, w.d), box=box), w.dtype),
+        "g": to_dtype(normal(s, S_G, (w.B, w.H, w.d), box=box), w.dtype),
+        "a_q": normal(s, S_AQ, (w.B, w.Hkv), -2.0, 1.0, box=box).astype(np.float32),
+        "a_k": (bimodal_ak(s, (w.B, w.Hkv), box=box) if w.bimodal_ak else
+                normal(s, S_AK, (w.B, w.Hkv), -2.0, 1.0, box=box)).astype(np.float32),
+    }
+    return {n: np.ascontiguousarray(x) for n, x in out.items()}

@@ -1,0 +1,211 @@
+"""fp64 CPU oracle for Universal Attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference legs of
+``bench.py`` may import this package.  The CUDA library never calls it and shares no
+code with it.  The arithmetic lives in ``ua_oracle.c`` (plain C, fp64); this module only
+builds it with gcc and marshals numpy arrays through ctypes.
+
+Every function computes straight from the definitions written in the header of
+``ua_oracle.c`` (structure from the pages "A Self-Pruning Transformer: Extreme KV-Cache
+Compression with Universal Attention" (paperlayer.ai summary, §3, §4, §4.1, §4.2, App. C)
+and the ai4snews synopsis of the same paper (Fig. 1 caption, veto property, eviction
+paragraph)).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ua_oracle.c")
+_LIB = os.path.join(_HERE, "libua_oracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ua_oracle.c into libua_oracle.so next to it (gcc, -O2, IEEE fp64)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-fno-fast-math",
+               "-ffp-contract=off", _SRC, "-o", _LIB + ".tmp", "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        Dd = ctypes.c_double
+        lib.ora_prefill_fwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 4 + [I]
+        lib.ora_prefill_fwd.restype = I
+        lib.ora_lambda_bruteforce.argtypes = [I, I, I, I, P, P, P, P, P, P, I]
+        lib.ora_lambda_bruteforce.restype = I
+        lib.ora_decode_step.argtypes = ([I, I, I, I, I, Dd, Dd] + [P] * 6 + [P] * 8 +
+                                        [Dd, Dd, Dd, P, P, P, P, P, I])
+        lib.ora_decode_step.restype = I
+        lib.ora_compact_order.argtypes = [I, P, P]
+        lib.ora_compact_order.restype = I
+        lib.ora_prefill_bwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 8 + [I]
+        lib.ora_prefill_bwd.restype = I
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0,
+                want_lambda=False, unit_mask=None, row_mask=None, nthreads=None):
+    """Prefill forward of UA in fp64.
+
+    Shapes: q, g [B,T,H,d]; k, v [B,T,Hkv,d]; a_q, a_k [B,T,Hkv]; alpha, beta [Hkv].
+    Returns dict(o [B,T,H,d], lse [B,H,T], b_final [B,Hkv,T], lam [B,Hkv,T,T] or None).
+    Entries outside unit_mask / row_mask are left as NaN.
+    """
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(g)
+    a_q, a_k, alpha, beta = _f64(a_q), _f64(a_k), _f64(alpha), _f64(beta)
+    B, T, H, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.full((B, T, H, d), np.nan)
+    lse = np.full((B, H, T), np.nan)
+    bfin = np.full((B, Hkv, T), np.nan)
+    lam = np.zeros((B, Hkv, T, T)) if want_lambda else None
+    um = None if unit_mask is None else np.ascontiguousarray(np.asarray(unit_mask, np.uint8))
+    rm = None if row_mask is None else np.ascontiguousarray(np.asarray(row_mask, np.uint8))
+    rc = _load().ora_prefill_fwd(B, T, H, Hkv, d, float(scale), float(theta),
+                                 _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
+                                 _ptr(alpha), _ptr(beta), _ptr(um), _ptr(rm),
+                                 _ptr(o), _ptr(lse), _ptr(bfin), _ptr(lam),
+                                 nthreads or default_threads())
+    if rc != 0:
+        raise ValueError(f"ora_prefill_fwd rejected the shapes (code {rc})")
+    return {"o": o, "lse": lse, "b_final": bfin, "lam": lam}
+
+
+def lambda_bruteforce(k, a_q, a_k, alpha, beta, nthreads=None):
+    """Lambda [B,Hkv,T,T] from the O(T^3) direct sum (lower triangle; zeros above)."""
+    k, a_q, a_k, alpha, beta = _f64(k), _f64(a_q), _f64(a_k), _f64(alpha), _f64(beta)
+    B, T, Hkv, d = k.shape
+    lam = np.zeros((B, Hkv, T, T))
+    _load().ora_lambda_bruteforce(B, T, Hkv, d, _ptr(k), _ptr(a_q), _ptr(a_k), _ptr(alpha),
+                                  _ptr(beta), _ptr(lam), nthreads or default_threads())
+    return lam
+
+
+def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, d_o, *, scale=None, theta=500000.0,
+                unit_mask=None, nthreads=None):
+    """Analytic fp64 gradients of sum(dO * O).  Returns a dict keyed dq, dk, dv, dg,
+    da_q, da_k, dalpha, dbeta (same shapes as the inputs)."""
+    q, k, v, g, d_o = _f64(q), _f64(k), _f64(v), _f64(g), _f64(d_o)
+    a_q, a_k, alpha, beta = _f64(a_q), _f64(a_k), _f64(alpha), _f64(beta)
+    B, T, H, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = {n: np.full(x.shape, np.nan) for n, x in
+           (("dq", q), ("dk", k), ("dv", v), ("dg", g), ("da_q", a_q), ("da_k", a_k))}
+    out["dalpha"] = np.zeros(Hkv)
+    out["dbeta"] = np.zeros(Hkv)
+    um = None if unit_mask is None else np.ascontiguousarray(np.asarray(unit_mask, np.uint8))
+    rc = _load().ora_prefill_bwd(B, T, H, Hkv, d, float(scale), float(theta),
+                                 _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
+                                 _ptr(alpha), _ptr(beta), _ptr(d_o), _ptr(um),
+                                 _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                                 _ptr(out["dg"]), _ptr(out["da_q"]), _ptr(out["da_k"]),
+                                 _ptr(out["dalpha"]), _ptr(out["dbeta"]),
+                                 nthreads or default_threads())
+    if rc != 0:
+        raise ValueError(f"ora_prefill_bwd rejected the shapes (code {rc})")
+    return out
+
+
+class DecodeCache:
+    """fp64 oracle cache: per (b, KV head) slot arrays of raw key, value, a_k logit,
+    token position and running bias b, plus the kept count."""
+
+    def __init__(self, B, Hkv, d, cap):
+        self.B, self.Hkv, self.d, self.cap = B, Hkv, d, cap
+        self.k = np.zeros((B, Hkv, cap, d))
+        self.v = np.zeros((B, Hkv, cap, d))
+        self.ak = np.zeros((B, Hkv, cap))
+        self.pos = np.zeros((B, Hkv, cap))
+        self.b = np.zeros((B, Hkv, cap))
+        self.n = np.zeros((B, Hkv), dtype=np.int32)
+
+    def fill_from_prefill(self, k, v, a_k, b_final, logp=None):
+        """Load a prefill's keys/values/a_k with their final biases b_final (Lambda's last
+        row).  With logp given, keep only pairs with b >= logp (stable order)."""
+        k, v, a_k, b_final = _f64(k), _f64(v), _f64(a_k), _f64(b_final)
+        B, T, Hkv, d = k.shape
+        for b in range(B):
+            for h in range(Hkv):
+                keep = np.ones(T, bool) if logp is None else (b_final[b, h] >= logp)
+                idx = np.nonzero(keep)[0]
+                n = len(idx)
+                if n > self.cap:
+                    raise ValueError("capacity exceeded")
+                self.k[b, h, :n] = k[b, idx, h]
+                self.v[b, h, :n] = v[b, idx, h]
+                self.ak[b, h, :n] = a_k[b, idx, h]
+                self.pos[b, h, :n] = idx
+                self.b[b, h, :n] = b_final[b, h, idx]
+                self.n[b, h] = n
+
+
+def decode_step(cache: DecodeCache, q, k, v, g, a_q, a_k, alpha, beta, pos_t, p, *,
+                scale=None, theta=500000.0, band=1e-3, adopt_keep=None, nthreads=None):
+    """One decode step on the oracle cache (mutated in place).
+
+    q, g [B,H,d]; k, v [B,Hkv,d]; a_q, a_k [B,Hkv].  Returns dict(o [B,H,d],
+    evict [B,Hkv,cap] (over pre-step slots), in_band, kept_order [B,Hkv,cap] (old slot
+    index of each survivor in new order, -1 beyond), n_before)."""
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(g)
+    a_q, a_k, alpha, beta = _f64(a_q), _f64(a_k), _f64(alpha), _f64(beta)
+    B, H, d = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    logp = float(np.log(p)) if p > 0 else -np.inf
+    o = np.full((B, H, d), np.nan)
+    ev = np.zeros((B, Hkv, cache.cap), np.uint8)
+    inb = np.zeros((B, Hkv, cache.cap), np.uint8)
+    order = np.full((B, Hkv, cache.cap), -1, np.int64)
+    ak_ = None if adopt_keep is None else np.ascontiguousarray(np.asarray(adopt_keep, np.uint8))
+    n_before = cache.n.copy()
+    rc = _load().ora_decode_step(B, H, Hkv, d, cache.cap, float(scale), float(theta),
+                                 _ptr(cache.n), _ptr(cache.k), _ptr(cache.v), _ptr(cache.ak),
+                                 _ptr(cache.pos), _ptr(cache.b),
+                                 _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
+                                 _ptr(alpha), _ptr(beta), float(pos_t), logp, float(band),
+                                 _ptr(ak_), _ptr(o), _ptr(ev), _ptr(inb), _ptr(order),
+                                 nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"ora_decode_step failed (code {rc})")
+    return {"o": o, "evict": ev, "in_band": inb, "kept_order": order, "n_before": n_before}
+
+
+def compact_order(keep):
+    """Stable compaction order of a keep mask: kept slot indices, ascending."""
+    keep = np.ascontiguousarray(np.asarray(keep, np.uint8))
+    order = np.zeros(len(keep), np.int64)
+    n = _load().ora_compact_order(len(keep), _ptr(keep), _ptr(order))
+    return order[:n]
