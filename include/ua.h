@@ -1,0 +1,187 @@
+/*
+ * ua.h -- C ABI of libua, the B200 (sm_100a) Universal Attention hot path.
+ *
+ * Universal Attention (UA) is causal RoPE softmax attention whose logits carry an
+ * additive, content-aware decay bias Lambda, plus the inference-time self-pruning of
+ * the KV cache that Lambda drives.  Sources: "A Self-Pruning Transformer: Extreme
+ * KV-Cache Compression with Universal Attention" -- paperlayer.ai summary (§3 causal
+ * softmax attention and the FoX additive forget gate; §4 and §4.1 the three decay
+ * mechanisms and their geometric mean; §4.2 threshold-p eviction and the training
+ * kernels; App. C decay applied inside a fused online softmax; App. H the missing
+ * fused dynamic cache manager) and the ai4snews synopsis of the same paper (Fig. 1
+ * caption: L2-normalised keys, sigmoid output gate, geometric mean -> log space ->
+ * causal accumulation; the veto property; the eviction paragraph).
+ *
+ * The pages fix the structure, not the formulas.  This library computes, per KV head:
+ *   khat_j     = k_j / max(||k_j||, 1e-12)                   (keys L2-normalised)
+ *   r_q(l)     = softplus(a_q[l])      query-aware rate
+ *   r_k(j)     = softplus(a_k[j])      key-aware rate
+ *   r_sim(l,j) = softplus(alpha * <khat_l, khat_j> + beta)   similarity rate (pre-RoPE keys)
+ *   D[l,j]     = (r_q(l) r_k(j) r_sim(l,j))^(1/3)            geometric mean (veto: any 0 -> 0)
+ *   Lambda_ij  = -sum_{l=j+1..i} D[l,j]                      (Lambda_ii = 0, never positive)
+ *   O_i        = softmax_{j<=i}(scale * RoPE(q_i).RoPE(khat_j) + Lambda_ij) V  (.) sigmoid(G_i)
+ * RoPE pairs element m with m + d/2 ("rotate half"), frequency theta^(-2m/d), position =
+ * token index.  Query head h uses KV head h / (H/Hkv); a_q, a_k, alpha and beta belong
+ * to the KV head, so the G query heads of a group share one Lambda.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers to caller-owned memory; the library never
+ *     allocates or frees, and launches asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Nothing synchronises except ua_get_device_status.
+ *   - Tensors are dense, row-major, innermost dimension last, with the shapes written
+ *     beside each argument.  "act" means the activation dtype of the call: float32 for
+ *     UA_F32, bfloat16 for UA_BF16.  Decay logits and parameters are always float32.
+ *   - Every pointer must be 16-byte aligned (256-byte for the workspace).
+ *   - Host-detectable errors (NULL pointer, bad shape, unsupported head_dim, misaligned
+ *     pointer, workspace too small) return a status before anything is launched and leave
+ *     all outputs untouched.  Device-detectable errors (cache capacity exceeded) set a
+ *     device status word read back by ua_get_device_status; the affected outputs are then
+ *     unspecified.  No kernel traps.
+ */
+#ifndef UA_H_
+#define UA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    UA_OK = 0,
+    UA_ERR_INVALID_ARG = 1,   /* NULL pointer, non-positive size, H % Hkv != 0, ... */
+    UA_ERR_UNSUPPORTED = 2,   /* head_dim / group size / dtype outside what is compiled */
+    UA_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte (workspace: 256-byte) aligned */
+    UA_ERR_WORKSPACE = 4,     /* workspace smaller than the size query returned */
+    UA_ERR_CAPACITY = 5,      /* a cache would exceed its capacity (device status bit) */
+    UA_ERR_CUDA = 6,          /* a CUDA runtime call failed (launch error, ...) */
+    UA_ERR_TIMEOUT = 7        /* a bounded device-side wait gave up (device status bit) */
+} ua_status;
+
+typedef enum { UA_F32 = 0, UA_BF16 = 1 } ua_dtype;
+
+/* Problem shape of a prefill call.  d (head_dim) must be 64 or 128; H % Hkv == 0 and
+ * H / Hkv in {1, 2, 3, 4, 8}; T >= 1. */
+typedef struct {
+    int B, T, H, Hkv, d;
+    float scale;          /* logit scale, usually 1/sqrt(d); multiplies only QK^T */
+    double rope_theta;    /* RoPE base, e.g. 500000 */
+    ua_dtype dtype;       /* activation dtype of q, k, v, g, o (and gradients) */
+} ua_shape;
+
+/* ------------------------------------------------------------------ prefill forward
+ * Decay construction (§4, §4.1, Fig. 1) and biased causal attention with the decay
+ * applied inside the online softmax (App. C).  Lambda is never written to HBM except
+ * through the optional debug output.
+ *
+ * ua_prefill_workspace_size: bytes of device scratch ua_prefill_fwd needs for `shape`
+ * (rotated queries and keys, rates and the per-query-tile column prefixes of the decay).
+ */
+ua_status ua_prefill_workspace_size(const ua_shape* shape, size_t* bytes);
+
+/* q, g: [B,T,H,d] act;  k, v: [B,T,Hkv,d] act;  a_q, a_k: [B,T,Hkv] f32;
+ * alpha, beta: [Hkv] f32.
+ * Outputs: o [B,T,H,d] act (required);
+ *          lse [B,H,T] f32 natural-log row normaliser of the biased logits (or NULL);
+ *          b_final [B,Hkv,T] f32 = Lambda_{T-1,j}, the initial per-pair cache bias (or NULL);
+ *          lambda_dbg [B,Hkv,T,T] f32 full Lambda, zero above the diagonal (or NULL;
+ *          allowed only for T <= 1024).
+ * ws / ws_bytes: device workspace of at least ua_prefill_workspace_size bytes; its
+ * contents are scratch (overwritten). */
+ua_status ua_prefill_fwd(const ua_shape* shape, const void* q, const void* k, const void* v,
+                         const void* g, const float* a_q, const float* a_k, const float* alpha,
+                         const float* beta, void* o, float* lse, float* b_final, float* lambda_dbg,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ prefill backward
+ * Gradient of sum(dO * O) with respect to every input of ua_prefill_fwd (the backward of
+ * the custom training kernels, §4.2 and App. H; the decay is recomputed, not stored,
+ * App. C).  Needs the forward's o, lse and b_final.
+ * Outputs: dq, dg [B,T,H,d] act; dk, dv [B,T,Hkv,d] act; da_q, da_k [B,T,Hkv] f32;
+ * dalpha, dbeta [Hkv] f32 (summed over the batch).  All outputs are overwritten. */
+ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes);
+
+ua_status ua_prefill_bwd(const ua_shape* shape, const void* q, const void* k, const void* v,
+                         const void* g, const float* a_q, const float* a_k, const float* alpha,
+                         const float* beta, const void* o, const float* lse, const float* b_final,
+                         const void* d_o, void* dq, void* dk, void* dv, void* dg, float* da_q,
+                         float* da_k, float* dalpha, float* dbeta, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* ------------------------------------------------------------------ self-pruning cache
+ * One cache per (batch, KV head), structure of arrays, `capacity` slots each; slot s of
+ * (b, h) lives at index (b*Hkv + h)*capacity + s.  Slots [0, n_kept[b,h]) are live, in
+ * ascending token order.  The cache element type follows `dtype` (f32 or bf16).
+ *   khat  [B,Hkv,cap,d]  normalised key (pre-RoPE), used by the similarity rate
+ *   krope [B,Hkv,cap,d]  RoPE(khat, pos), used by the attention logit
+ *   v     [B,Hkv,cap,d]  value
+ *   bias  [B,Hkv,cap]    f32 running log-bias b_j (= Lambda_{t,j} at the current row t)
+ *   rk    [B,Hkv,cap]    f32 key-aware rate softplus(a_k[j])
+ *   pos   [B,Hkv,cap]    int32 token position
+ *   n_kept [B,Hkv]       int32 live slot count
+ * The pages keep a scalar bias per cached pair and evict a pair once exp(b_j) < p; b_j
+ * only decreases, so an evicted pair never returns (§4.2; ai4snews eviction paragraph). */
+typedef struct {
+    int B, Hkv, d, capacity;
+    ua_dtype dtype;
+    void* khat;
+    void* krope;
+    void* v;
+    float* bias;
+    float* rk;
+    int32_t* pos;
+    int32_t* n_kept;
+} ua_cache;
+
+/* Load a prefill into the cache: slot t <- token t for t < T (khat, krope, v from k and
+ * v; bias = b_final; rk = softplus(a_k); pos = t) and n_kept = T.  Requires T <= capacity.
+ * k, v: [B,T,Hkv,d] act; a_k [B,T,Hkv] f32; b_final [B,Hkv,T] f32. */
+ua_status ua_cache_fill(const ua_cache* cache, int T, const void* k, const void* v,
+                        const float* a_k, const float* b_final, double rope_theta, void* stream);
+
+/* Stable in-place compaction of every (b, KV head) cache.  A slot survives when
+ * keep[b,h,s] != 0 (keep: [B,Hkv,cap] uint8) or, with keep == NULL, when bias >= log p.
+ * Survivors keep their relative order.  kept_idx (optional, [B,Hkv,cap] int32) receives
+ * the old slot of each survivor in its new order; entries past the new n_kept are left
+ * untouched. */
+ua_status ua_cache_compact(const ua_cache* cache, const uint8_t* keep, float p,
+                           int32_t* kept_idx, void* stream);
+
+/* One decode step for all B sequences, the new token sitting at position pos_t:
+ *   1. each live pair j takes the new row's decay, b_j -= D[t,j];
+ *   2. it is evicted when b_j < log p (exp(b_j) < p); p = 0 evicts nothing;
+ *   3. the H query heads attend over the survivors plus the new token (bias 0) with
+ *      logits scale * RoPE(q).krope_j + b_j, and the result is gated by sigmoid(g);
+ *   4. survivors are compacted stably in place and the new token is appended (b = 0).
+ * All in one pass over the cache.  q, g: [B,H,d] act; k, v: [B,Hkv,d] act;
+ * a_q, a_k: [B,Hkv] f32; alpha, beta [Hkv] f32; o: [B,H,d] act (required).
+ * evict_bits (optional, [B,Hkv,ceil(cap/32)] uint32): bit s set when pre-step slot s was
+ * evicted (all words are written).  kept_idx (optional, [B,Hkv,cap] int32): pre-step
+ * slot of each survivor in new order, then -1 for the appended token.
+ * flags: reserved, pass 0.  Every cache call requires capacity <= 2^20 slots
+ * (UA_ERR_UNSUPPORTED otherwise).  If a cache is full (no pair evicted and n_kept == capacity)
+ * the step sets UA_ERR_CAPACITY in the device status word and that cache is left as it
+ * was after compaction, without the new token. */
+ua_status ua_decode_step(const ua_cache* cache, int H, const void* q, const void* k,
+                         const void* v, const void* g, const float* a_q, const float* a_k,
+                         const float* alpha, const float* beta, int pos_t, float p, float scale,
+                         double rope_theta, void* o, uint32_t* evict_bits, int32_t* kept_idx,
+                         int flags, void* stream);
+
+/* ------------------------------------------------------------------ status
+ * Synchronises `stream`, returns the device status word accumulated since the last call
+ * (0 = no error, else a ua_status code) in *code, and clears it. */
+ua_status ua_get_device_status(void* stream, int* code);
+
+/* Static, human-readable name of a status code. */
+const char* ua_status_string(ua_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int ua_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UA_H_ */

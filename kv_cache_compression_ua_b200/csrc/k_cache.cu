@@ -1,0 +1,435 @@
+// k_cache.cu -- the self-pruning KV cache: fill from a prefill, stable compaction, and the
+// fused decode step (bias update, eviction, attention, compaction, append) in one pass.
+//
+// The pages keep a scalar bias per cached key/value pair that the learned decay lowers at
+// every step, and evict a pair once exp(b_j) < p; b_j only decreases, so evicted pairs never
+// come back, and each head keeps its own, input-dependent number of pairs (paperlayer.ai
+// summary §4.2; ai4snews synopsis, eviction paragraph).  The pages report that their own
+// implementation lacked a fused dynamic cache manager and name specialised kernels for the
+// pruned cache as future work (paperlayer.ai summary §6, App. H) -- this file is that part.
+//
+// Layout: one structure-of-arrays cache per (batch, KV head), slots in ascending token
+// order.  An entry is read by a group of LPE lanes, each moving 16 bytes of khat, krope and v
+// (128-bit coalesced loads); dot products reduce across the group with shuffles.
+#include "ua_common.cuh"
+#include "ua_kernels.h"
+
+namespace ua {
+
+template <typename TC, int DH>
+struct EntryLayout {
+    static constexpr int VEC = Vec16<TC>::N;   // elements per 16-byte vector
+    static constexpr int LPE = DH / VEC;       // lanes per entry
+    static constexpr int EPW = 32 / LPE;       // entries per warp
+    static constexpr int NW = 8;               // warps per block
+    static constexpr int EPB = EPW * NW;       // entries per block pass
+};
+
+template <int LPE>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+    for (int o = LPE / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Block-wide stable compaction bookkeeping for one pass: returns the destination of this
+// lane's entry (valid only when keep) and the number of survivors in the pass.
+template <int LPE, int NW>
+__device__ __forceinline__ int pass_scan(bool keep, int warp, int lane, int* s_wcnt, int* total) {
+    const int grp_lane0 = (lane / LPE) * LPE;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep && (lane % LPE) == 0);
+    const int wpre = __popc(bal & ((1u << grp_lane0) - 1u));
+    if (lane == 0) s_wcnt[warp] = __popc(bal);
+    __syncthreads();
+    int bpre = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        const int c = s_wcnt[w];
+        bpre += (w < warp) ? c : 0;
+        tot += c;
+    }
+    *total = tot;
+    return bpre + wpre;
+}
+
+// ------------------------------------------------------------------ fill from a prefill
+// grid (T, B), 256 threads; warp per KV head.
+template <typename TC, int DH>
+__global__ void __launch_bounds__(256) k_cache_fill(FillParams p) {
+    const int t = blockIdx.x, b = blockIdx.y, T = p.T;
+    const CacheView& c = p.c;
+    constexpr int half = DH / 2;
+    __shared__ float s_cos[half], s_sin[half];
+    for (int m = threadIdx.x; m < half; m += blockDim.x) rope_cs((double)t, m, DH, p.theta, &s_cos[m], &s_sin[m]);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const TC* kin = static_cast<const TC*>(p.k);
+    const TC* vin = static_cast<const TC*>(p.v);
+    for (int h = warp; h < c.Hkv; h += 8) {
+        const size_t src = (((size_t)b * T + t) * c.Hkv + h) * DH;
+        const size_t slot = ((size_t)b * c.Hkv + h) * c.cap + t;
+        float x0[2] = {0.f, 0.f}, x1[2] = {0.f, 0.f};
+        float ss = 0.f;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int m = lane + 32 * r;
+            if (m < half) {
+                x0[r] = Elem<TC>::ld(kin + src + m);
+                x1[r] = Elem<TC>::ld(kin + src + m + half);
+                ss += x0[r] * x0[r] + x1[r] * x1[r];
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float den = fmaxf(sqrtf(ss), 1e-12f);
+        TC* kh = static_cast<TC*>(c.khat) + slot * DH;
+        TC* kr = static_cast<TC*>(c.krope) + slot * DH;
+        TC* vv = static_cast<TC*>(c.v) + slot * DH;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int m = lane + 32 * r;
+            if (m < half) {
+                const float a = x0[r] / den, bq = x1[r] / den;
+                Elem<TC>::st(kh + m, a);
+                Elem<TC>::st(kh + m + half, bq);
+                Elem<TC>::st(kr + m, a * s_cos[m] - bq * s_sin[m]);
+                Elem<TC>::st(kr + m + half, bq * s_cos[m] + a * s_sin[m]);
+            }
+        }
+        for (int x = lane; x < DH; x += 32) vv[x] = vin[src + x];
+        if (lane == 0) {
+            c.bias[slot] = p.bfinal[((size_t)b * c.Hkv + h) * T + t];
+            c.rk[slot] = softplus_f(p.a_k[((size_t)b * T + t) * c.Hkv + h]);
+            c.pos[slot] = t;
+            if (t == 0) c.n_kept[(size_t)b * c.Hkv + h] = T;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ compaction
+// grid (B*Hkv), 256 threads.
+template <typename TC, int DH>
+__global__ void __launch_bounds__(256) k_cache_compact(CompactParams p) {
+    using L = EntryLayout<TC, DH>;
+    __shared__ int s_wcnt[L::NW];
+    const CacheView& c = p.c;
+    const int unit = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = lane / L::LPE, gl = lane % L::LPE;
+    int n = c.n_kept[unit];
+    if (n < 0 || n > c.cap) {                 // corrupt count: never read past the cache
+        if (threadIdx.x == 0) raise_status(UA_ERR_CAPACITY);
+        n = n < 0 ? 0 : c.cap;
+    }
+    const size_t base = (size_t)unit * c.cap;
+    TC* khat = static_cast<TC*>(c.khat);
+    TC* krope = static_cast<TC*>(c.krope);
+    TC* vc = static_cast<TC*>(c.v);
+    int out = 0;
+    for (int c0 = 0; c0 < n; c0 += L::EPB) {
+        const int j = c0 + warp * L::EPW + grp;
+        const bool valid = j < n;
+        uint4 a = make_uint4(0, 0, 0, 0), bq = a, vv = a;
+        float bj = 0.f, rkj = 0.f;
+        int pj = 0;
+        bool keep = false;
+        if (valid) {
+            const size_t e = (base + j) * DH + gl * L::VEC;
+            a = *reinterpret_cast<const uint4*>(khat + e);
+            bq = *reinterpret_cast<const uint4*>(krope + e);
+            vv = *reinterpret_cast<const uint4*>(vc + e);
+            bj = c.bias[base + j];
+            rkj = c.rk[base + j];
+            pj = c.pos[base + j];
+            keep = p.keep ? (p.keep[base + j] != 0) : (bj >= p.logp);
+        }
+        int tot;
+        const int dst = out + pass_scan<L::LPE, L::NW>(keep, warp, lane, s_wcnt, &tot);
+        if (keep) {
+            if (dst != j) {
+                const size_t e = (base + dst) * DH + gl * L::VEC;
+                *reinterpret_cast<uint4*>(khat + e) = a;
+                *reinterpret_cast<uint4*>(krope + e) = bq;
+                *reinterpret_cast<uint4*>(vc + e) = vv;
+                if (gl == 0) {
+                    c.bias[base + dst] = bj;
+                    c.rk[base + dst] = rkj;
+                    c.pos[base + dst] = pj;
+                }
+            }
+            if (gl == 0 && p.kept_idx) p.kept_idx[base + dst] = j;
+        }
+        out += tot;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) c.n_kept[unit] = out;
+}
+
+// ------------------------------------------------------------------ decode step
+// grid (B*Hkv), 256 threads.  Dynamic shared memory: eviction bitmap (ceil(cap/32) words)
+// followed by the per-group softmax partials.
+template <typename TC, int DH, int G>
+__global__ void __launch_bounds__(256) k_decode(DecodeParams p) {
+    using L = EntryLayout<TC, DH>;
+    constexpr int VEC = L::VEC, LPE = L::LPE, EPB = L::EPB, NW = L::NW;
+    constexpr int half = DH / 2;
+    __shared__ float s_kt[DH], s_ktr[DH], s_vt[DH], s_q[G][DH], s_lt[G];
+    __shared__ float s_red[NW];
+    __shared__ int s_wcnt[NW];
+    extern __shared__ float dsm[];
+    const CacheView& c = p.c;
+    const int words = (c.cap + 31) / 32;
+    uint32_t* s_ev = reinterpret_cast<uint32_t*>(dsm);
+    float* s_m = dsm + ((words + 3) & ~3);          // [EPB][G]
+    float* s_l = s_m + EPB * G;                       // [EPB][G]
+    float* s_acc = s_l + EPB * G;                     // [EPB][G][DH]
+
+    const int unit = blockIdx.x, b = unit / c.Hkv, kvh = unit % c.Hkv;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = lane / LPE, gl = lane % LPE;
+    const int gidx = warp * L::EPW + grp;             // entry group index in the pass
+    const size_t base = (size_t)unit * c.cap;
+
+    // ---- new token: khat_t, RoPE(khat_t), v_t, RoPE(q_h), rates
+    const TC* kin = static_cast<const TC*>(p.k) + (size_t)unit * DH;
+    const TC* vin = static_cast<const TC*>(p.v) + (size_t)unit * DH;
+    float kx = 0.f;
+    if (tid < DH) {
+        kx = Elem<TC>::ld(kin + tid);
+        s_vt[tid] = Elem<TC>::ld(vin + tid);
+    }
+    float ss = kx * kx;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) s_red[warp] = ss;
+    for (int w = tid; w < words; w += blockDim.x) s_ev[w] = 0u;
+    __syncthreads();
+    float tot_ss = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) tot_ss += s_red[w];
+    const float den = fmaxf(sqrtf(tot_ss), 1e-12f);
+    if (tid < DH) s_kt[tid] = kx / den;
+    __syncthreads();
+    const TC* qin = static_cast<const TC*>(p.q) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
+    for (int e = tid; e < (G + 1) * half; e += blockDim.x) {
+        const int vecid = e / half, m = e % half;
+        float cs, sn;
+        rope_cs((double)p.pos_t, m, DH, p.theta, &cs, &sn);
+        if (vecid < G) {
+            const float x0 = Elem<TC>::ld(qin + vecid * DH + m), x1 = Elem<TC>::ld(qin + vecid * DH + m + half);
+            s_q[vecid][m] = x0 * cs - x1 * sn;
+            s_q[vecid][m + half] = x1 * cs + x0 * sn;
+        } else {
+            const float x0 = s_kt[m], x1 = s_kt[m + half];
+            s_ktr[m] = x0 * cs - x1 * sn;
+            s_ktr[m + half] = x1 * cs + x0 * sn;
+        }
+    }
+    __syncthreads();
+    if (tid < G) {
+        float a = 0.f;
+        for (int x = 0; x < DH; ++x) a = fmaf(s_q[tid][x], s_ktr[x], a);
+        s_lt[tid] = a * p.scale;                      // new token's own bias is 0
+    }
+    const float rq_t = softplus_f(p.a_q[unit]);
+    const float rk_t = softplus_f(p.a_k[unit]);
+    const float al = p.alpha[kvh], be = p.beta[kvh];
+
+    float kq[VEC], qh[G][VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        kq[e] = s_kt[gl * VEC + e];
+#pragma unroll
+        for (int h = 0; h < G; ++h) qh[h][e] = s_q[h][gl * VEC + e];
+    }
+    float m_h[G], l_h[G], acc[G][VEC];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        m_h[h] = -INFINITY;
+        l_h[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[h][e] = 0.f;
+    }
+
+    TC* khat = static_cast<TC*>(c.khat);
+    TC* krope = static_cast<TC*>(c.krope);
+    TC* vc = static_cast<TC*>(c.v);
+    int n = c.n_kept[unit];
+    if (n < 0 || n > c.cap) {                 // corrupt count: never read past the cache
+        if (tid == 0) raise_status(UA_ERR_CAPACITY);
+        n = n < 0 ? 0 : c.cap;
+    }
+    int out = 0;
+    for (int c0 = 0; c0 < n; c0 += EPB) {
+        const int j = c0 + gidx;
+        const bool valid = j < n;
+        uint4 ra = make_uint4(0, 0, 0, 0), rb = ra, rv = ra;
+        float bj = 0.f, rkj = 0.f;
+        int pj = 0;
+        if (valid) {
+            const size_t e = (base + j) * DH + gl * VEC;
+            ra = *reinterpret_cast<const uint4*>(khat + e);
+            rb = *reinterpret_cast<const uint4*>(krope + e);
+            rv = *reinterpret_cast<const uint4*>(vc + e);
+            bj = c.bias[base + j];
+            rkj = c.rk[base + j];
+            pj = c.pos[base + j];
+        }
+        float xa[VEC], xb[VEC], xv[VEC];
+        Vec16<TC>::unpack(ra, xa);
+        Vec16<TC>::unpack(rb, xb);
+        Vec16<TC>::unpack(rv, xv);
+        float sim = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) sim = fmaf(kq[e], xa[e], sim);
+        sim = group_sum<LPE>(sim);
+        const float D = decay_geo(rq_t, rkj, softplus_f(fmaf(al, sim, be)));
+        const float bnew = bj - D;
+        const bool keep = valid && (bnew >= p.logp);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float lg = 0.f;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) lg = fmaf(qh[h][e], xb[e], lg);
+            lg = group_sum<LPE>(lg);
+            if (keep) {
+                lg = fmaf(lg, p.scale, bnew);
+                const float mn = fmaxf(m_h[h], lg);
+                const float corr = expf(m_h[h] - mn);
+                const float pe = expf(lg - mn);
+                l_h[h] = l_h[h] * corr + pe;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc[h][e] = fmaf(pe, xv[e], acc[h][e] * corr);
+                m_h[h] = mn;
+            }
+        }
+        if (valid && !keep && gl == 0) atomicOr(&s_ev[j >> 5], 1u << (j & 31));
+        int tot;
+        const int dst = out + pass_scan<LPE, NW>(keep, warp, lane, s_wcnt, &tot);
+        if (keep) {
+            if (dst != j) {
+                const size_t e = (base + dst) * DH + gl * VEC;
+                *reinterpret_cast<uint4*>(khat + e) = ra;
+                *reinterpret_cast<uint4*>(krope + e) = rb;
+                *reinterpret_cast<uint4*>(vc + e) = rv;
+                if (gl == 0) {
+                    c.rk[base + dst] = rkj;
+                    c.pos[base + dst] = pj;
+                }
+            }
+            if (gl == 0) {
+                c.bias[base + dst] = bnew;
+                if (p.kept_idx) p.kept_idx[base + dst] = j;
+            }
+        }
+        out += tot;
+        __syncthreads();
+    }
+
+    // ---- merge the per-group online-softmax states, add the new token, gate, store
+    if (gl == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            s_m[gidx * G + h] = m_h[h];
+            s_l[gidx * G + h] = l_h[h];
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) s_acc[((size_t)gidx * G + h) * DH + gl * VEC + e] = acc[h][e];
+    __syncthreads();
+    const TC* gin = static_cast<const TC*>(p.g) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
+    TC* oout = static_cast<TC*>(p.o) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
+    for (int e = tid; e < G * DH; e += blockDim.x) {
+        const int h = e / DH, x = e % DH;
+        float M = s_lt[h];
+        for (int q = 0; q < EPB; ++q) M = fmaxf(M, s_m[q * G + h]);
+        float Ls = expf(s_lt[h] - M);
+        float A = Ls * s_vt[x];
+        for (int q = 0; q < EPB; ++q) {
+            const float w = expf(s_m[q * G + h] - M);
+            Ls = fmaf(s_l[q * G + h], w, Ls);
+            A = fmaf(s_acc[((size_t)q * G + h) * DH + x], w, A);
+        }
+        Elem<TC>::st(oout + e, A / Ls * sigmoid_f(Elem<TC>::ld(gin + e)));
+    }
+    // ---- eviction bits, append the new token
+    if (p.evict_bits)
+        for (int w = tid; w < words; w += blockDim.x) p.evict_bits[(size_t)unit * words + w] = s_ev[w];
+    if (out < c.cap) {
+        const size_t e = (base + out) * DH;
+        for (int x = tid; x < DH; x += blockDim.x) {
+            Elem<TC>::st(khat + e + x, s_kt[x]);
+            Elem<TC>::st(krope + e + x, s_ktr[x]);
+            Elem<TC>::st(vc + e + x, s_vt[x]);
+        }
+        if (tid == 0) {
+            c.bias[base + out] = 0.f;
+            c.rk[base + out] = rk_t;
+            c.pos[base + out] = p.pos_t;
+            c.n_kept[unit] = out + 1;
+            if (p.kept_idx) p.kept_idx[base + out] = -1;
+        }
+    } else if (tid == 0) {
+        c.n_kept[unit] = out;
+        raise_status(UA_ERR_CAPACITY);
+    }
+}
+
+// ------------------------------------------------------------------ launchers
+cudaError_t launch_cache_fill(const FillParams& p, bool bf16, cudaStream_t s) {
+    dim3 grid(p.T, p.c.B);
+    if (bf16) {
+        if (p.c.d == 64) k_cache_fill<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
+        else k_cache_fill<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
+    } else {
+        if (p.c.d == 64) k_cache_fill<float, 64><<<grid, 256, 0, s>>>(p);
+        else k_cache_fill<float, 128><<<grid, 256, 0, s>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cache_compact(const CompactParams& p, bool bf16, cudaStream_t s) {
+    dim3 grid(p.c.B * p.c.Hkv);
+    if (bf16) {
+        if (p.c.d == 64) k_cache_compact<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
+        else k_cache_compact<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
+    } else {
+        if (p.c.d == 64) k_cache_compact<float, 64><<<grid, 256, 0, s>>>(p);
+        else k_cache_compact<float, 128><<<grid, 256, 0, s>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+template <typename TC, int DH, int G>
+static cudaError_t decode_inst(const DecodeParams& p, cudaStream_t s) {
+    using L = EntryLayout<TC, DH>;
+    const int words = (p.c.cap + 31) / 32;
+    const size_t smem = sizeof(float) * ((size_t)((words + 3) & ~3) + 2 * L::EPB * G + (size_t)L::EPB * G * DH);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_decode<TC, DH, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    k_decode<TC, DH, G><<<p.c.B * p.c.Hkv, 256, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename TC, int DH>
+static cudaError_t decode_g(const DecodeParams& p, cudaStream_t s) {
+    switch (p.G) {
+        case 1: return decode_inst<TC, DH, 1>(p, s);
+        case 2: return decode_inst<TC, DH, 2>(p, s);
+        case 3: return decode_inst<TC, DH, 3>(p, s);
+        case 4: return decode_inst<TC, DH, 4>(p, s);
+        case 8: return decode_inst<TC, DH, 8>(p, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t s) {
+    if (bf16) return p.c.d == 64 ? decode_g<__nv_bfloat16, 64>(p, s) : decode_g<__nv_bfloat16, 128>(p, s);
+    return p.c.d == 64 ? decode_g<float, 64>(p, s) : decode_g<float, 128>(p, s);
+}
+
+}  // namespace ua

@@ -1,0 +1,338 @@
+// k_prefill_simt.cu -- token preparation, the decay boundary pass and the fused biased
+// attention forward, written as plain fp32 SIMT CUDA.  This is the exact-arithmetic path
+// (fp32 activations); bf16 activations take the tensor-core path in k_prefill_tc.cu.
+//
+// Structure followed (see ua.h for the formulas): keys L2-normalised and RoPE kept
+// (ai4snews synopsis, Fig. 1 caption); three rates combined by a geometric mean and
+// accumulated causally (paperlayer.ai summary §4, §4.1); the decay applied inside a fused
+// online softmax without materialising the T x T mask (paperlayer.ai summary App. C).
+// Lambda is built as a chunked scan: the boundary pass writes, for every query tile t and
+// key j, the column prefix Pb_t[j] = sum_{j<l<t*bq} D[l,j]; the attention kernel adds the
+// in-tile triangular cumulative sum on top.
+#include "ua_common.cuh"
+#include "ua_kernels.h"
+
+namespace ua {
+
+// ------------------------------------------------------------------ token preparation
+// grid (T, B), 256 threads.  Each warp takes one (query or key) head of token t at a time.
+template <typename TI, typename TW>
+__global__ void __launch_bounds__(256) k_prep(PrepParams p) {
+    const int t = blockIdx.x, b = blockIdx.y;
+    const int d = p.d, half = d / 2, T = p.T;
+    __shared__ float s_cos[64], s_sin[64];
+    for (int m = threadIdx.x; m < half; m += blockDim.x) rope_cs((double)t, m, d, p.theta, &s_cos[m], &s_sin[m]);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const TI* q = static_cast<const TI*>(p.q);
+    const TI* k = static_cast<const TI*>(p.k);
+    for (int hh = warp; hh < p.H + p.Hkv; hh += 8) {
+        const bool is_q = hh < p.H;
+        const int h = is_q ? hh : hh - p.H;
+        const TI* src = is_q ? q + (((size_t)b * T + t) * p.H + h) * d : k + (((size_t)b * T + t) * p.Hkv + h) * d;
+        float x0[2] = {0.f, 0.f}, x1[2] = {0.f, 0.f};
+        float ss = 0.f;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int m = lane + 32 * r;
+            if (m < half) {
+                x0[r] = Elem<TI>::ld(src + m);
+                x1[r] = Elem<TI>::ld(src + m + half);
+                ss += x0[r] * x0[r] + x1[r] * x1[r];
+            }
+        }
+        TW* dst_rot;
+        if (!is_q) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float den = fmaxf(sqrtf(ss), 1e-12f);
+            TW* dst_hat = static_cast<TW*>(p.kh) + (((size_t)b * p.Hkv + h) * T + t) * d;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int m = lane + 32 * r;
+                if (m < half) {
+                    x0[r] = x0[r] / den;
+                    x1[r] = x1[r] / den;
+                    Elem<TW>::st(dst_hat + m, x0[r]);
+                    Elem<TW>::st(dst_hat + m + half, x1[r]);
+                }
+            }
+            dst_rot = static_cast<TW*>(p.kr) + (((size_t)b * p.Hkv + h) * T + t) * d;
+        } else {
+            dst_rot = static_cast<TW*>(p.qr) + (((size_t)b * p.H + h) * T + t) * d;
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int m = lane + 32 * r;
+            if (m < half) {
+                const float c = s_cos[m], s = s_sin[m];
+                Elem<TW>::st(dst_rot + m, x0[r] * c - x1[r] * s);
+                Elem<TW>::st(dst_rot + m + half, x1[r] * c + x0[r] * s);
+            }
+        }
+    }
+    for (int h = threadIdx.x; h < p.Hkv; h += blockDim.x) {
+        const size_t src = ((size_t)b * T + t) * p.Hkv + h;
+        const size_t dst = ((size_t)b * p.Hkv + h) * T + t;
+        p.rq[dst] = softplus_f(p.a_q[src]);
+        p.rk[dst] = softplus_f(p.a_k[src]);
+    }
+}
+
+// ------------------------------------------------------------------ boundary pass
+// grid (ceil(T/128), Hkv, B), 128 threads; thread = key j, sweeping the rows l > j in
+// order.  At every query-tile boundary l = t*bq it writes the prefix sum so far.
+template <int DH>
+__global__ void __launch_bounds__(128) k_boundary_simt(BoundaryParams p) {
+    constexpr int RC = 32;
+    __shared__ float s_k[RC][DH];
+    __shared__ float s_rq[RC];
+    const int T = p.T;
+    const int kt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    const int j = kt * 128 + threadIdx.x;
+    const bool valid = j < T;
+    const size_t unit = (size_t)b * p.Hkv + kvh;
+    const float* kh = p.kh + unit * T * DH;
+    float kj[DH];
+#pragma unroll
+    for (int c = 0; c < DH; ++c) kj[c] = valid ? kh[(size_t)j * DH + c] : 0.f;
+    const float rkj = valid ? p.rk[unit * T + j] : 0.f;
+    const float al = p.alpha[kvh], be = p.beta[kvh];
+    float* pb = p.pb + unit * (size_t)p.nqt * T;
+    const int l0 = kt * 128;
+    if (valid)
+        for (int t = 0; t * p.bq < l0; ++t) pb[(size_t)t * T + j] = 0.f;
+    float acc = 0.f;
+    for (int c0 = l0; c0 < T; c0 += RC) {
+        __syncthreads();
+        const int nrow = min(RC, T - c0);
+        for (int e = threadIdx.x; e < RC * DH; e += 128) {
+            const int r = e / DH, c = e % DH;
+            s_k[r][c] = r < nrow ? kh[(size_t)(c0 + r) * DH + c] : 0.f;
+        }
+        if (threadIdx.x < RC) s_rq[threadIdx.x] = threadIdx.x < nrow ? p.rq[unit * T + c0 + threadIdx.x] : 0.f;
+        __syncthreads();
+        for (int r = 0; r < nrow; ++r) {
+            const int l = c0 + r;
+            if (valid && (l % p.bq) == 0) pb[(size_t)(l / p.bq) * T + j] = acc;
+            if (valid && l > j) {
+                float s = 0.f;
+#pragma unroll
+                for (int c = 0; c < DH; ++c) s = fmaf(s_k[r][c], kj[c], s);
+                acc += decay_geo(s_rq[r], rkj, softplus_f(fmaf(al, s, be)));
+            }
+        }
+    }
+    if (valid && p.bfinal) p.bfinal[unit * T + j] = -acc;
+}
+
+// ------------------------------------------------------------------ fused forward
+// grid (nqt, H, B), 256 threads = 16 x 16; 64 query rows x 64 keys per tile.  Thread
+// (ty, tx) owns rows ty + 16*rr and columns tx + 16*cc (rr, cc < 4), which keeps the
+// padded shared-memory reads conflict-free.
+template <int DH, typename TI>
+__global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
+    constexpr int BM = 64, BN = 64, LD = DH + 1, LP = BN + 1, ND = DH / 16;
+    extern __shared__ float sm[];
+    float* sQ = sm;
+    float* sKq = sQ + BM * LD;
+    float* sKh = sKq + BM * LD;
+    float* sKr = sKh + BN * LD;
+    float* sV = sKr + BN * LD;
+    float* sL = sV + BN * LD;
+    float* sP = sL + BM * LP;
+    float* sRq = sP + BM * LP;
+    float* sRk = sRq + BM;
+    float* sPb = sRk + BN;
+
+    const int T = p.T;
+    const int qt = gridDim.x - 1 - blockIdx.x;        // heaviest (last) query tiles first
+    const int h = blockIdx.y, b = blockIdx.z, kvh = h / p.G;
+    const int i0 = qt * BM;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const size_t unit = (size_t)b * p.Hkv + kvh;
+    const TI* vin = static_cast<const TI*>(p.v);
+    const bool write_lambda = p.lambda_dbg != nullptr && (h % p.G) == 0;
+
+    for (int e = tid; e < BM * DH; e += 256) {
+        const int r = e / DH, c = e % DH, i = i0 + r;
+        sQ[r * LD + c] = i < T ? p.qr[(((size_t)b * p.H + h) * T + i) * DH + c] : 0.f;
+        sKq[r * LD + c] = i < T ? p.kh[(unit * T + i) * DH + c] : 0.f;
+    }
+    for (int r = tid; r < BM; r += 256) sRq[r] = (i0 + r < T) ? p.rq[unit * T + i0 + r] : 0.f;
+
+    float m_r[4], l_r[4], acc[4][ND];
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+        m_r[rr] = -INFINITY;
+        l_r[rr] = 0.f;
+#pragma unroll
+        for (int dd = 0; dd < ND; ++dd) acc[rr][dd] = 0.f;
+    }
+    const float al = p.alpha[kvh], be = p.beta[kvh];
+
+    for (int kt = 0; kt <= qt; ++kt) {
+        const int j0 = kt * BN;
+        __syncthreads();
+        for (int e = tid; e < BN * DH; e += 256) {
+            const int c = e / DH, x = e % DH, j = j0 + c;
+            const bool ok = j < T;
+            sKh[c * LD + x] = ok ? p.kh[(unit * T + j) * DH + x] : 0.f;
+            sKr[c * LD + x] = ok ? p.kr[(unit * T + j) * DH + x] : 0.f;
+            sV[c * LD + x] = ok ? Elem<TI>::ld(vin + (((size_t)b * T + j) * p.Hkv + kvh) * DH + x) : 0.f;
+        }
+        for (int c = tid; c < BN; c += 256) {
+            const int j = j0 + c;
+            sRk[c] = j < T ? p.rk[unit * T + j] : 0.f;
+            sPb[c] = j < T ? p.pb[(unit * p.nqt + qt) * T + j] : 0.f;
+        }
+        __syncthreads();
+        // decay D[l = i0 + r, j = j0 + c]
+        {
+            float s[4][4];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) s[rr][cc] = 0.f;
+            for (int x = 0; x < DH; ++x) {
+                float a[4], bb[4];
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) a[rr] = sKq[(ty + 16 * rr) * LD + x];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) bb[cc] = sKh[(tx + 16 * cc) * LD + x];
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) s[rr][cc] = fmaf(a[rr], bb[cc], s[rr][cc]);
+            }
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int r = ty + 16 * rr, c = tx + 16 * cc;
+                    const int i = i0 + r, j = j0 + c;
+                    float D = 0.f;
+                    if (i > j && i < T && j < T) D = decay_geo(sRq[r], sRk[c], softplus_f(fmaf(al, s[rr][cc], be)));
+                    sL[r * LP + c] = D;
+                }
+        }
+        __syncthreads();
+        // in-tile causal accumulation on top of the boundary prefix
+        if (tid < BN) {
+            float a = sPb[tid];
+            for (int r = 0; r < BM; ++r) {
+                a += sL[r * LP + tid];
+                sL[r * LP + tid] = -a;
+            }
+        }
+        __syncthreads();
+        float sc[4][4];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) sc[rr][cc] = 0.f;
+        for (int x = 0; x < DH; ++x) {
+            float a[4], bb[4];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) a[rr] = sQ[(ty + 16 * rr) * LD + x];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) bb[cc] = sKr[(tx + 16 * cc) * LD + x];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) sc[rr][cc] = fmaf(a[rr], bb[cc], sc[rr][cc]);
+        }
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            const int r = ty + 16 * rr, i = i0 + r;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const int c = tx + 16 * cc, j = j0 + c;
+                const float lam = sL[r * LP + c];
+                if (write_lambda && i < T && j < T)
+                    p.lambda_dbg[(unit * T + i) * (size_t)T + j] = (j <= i) ? lam : 0.f;
+                sc[rr][cc] = (j <= i && j < T) ? fmaf(p.scale, sc[rr][cc], lam) : -INFINITY;
+                mx = fmaxf(mx, sc[rr][cc]);
+            }
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float m_new = fmaxf(m_r[rr], mx);
+            const float corr = expf(m_r[rr] - m_new);
+            float rs = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const float pe = expf(sc[rr][cc] - m_new);
+                rs += pe;
+                sP[r * LP + tx + 16 * cc] = pe;
+            }
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
+            l_r[rr] = l_r[rr] * corr + rs;
+            m_r[rr] = m_new;
+#pragma unroll
+            for (int dd = 0; dd < ND; ++dd) acc[rr][dd] *= corr;
+        }
+        __syncthreads();
+        for (int c = 0; c < BN; ++c) {
+            float pv[4], vv[ND];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) pv[rr] = sP[(ty + 16 * rr) * LP + c];
+#pragma unroll
+            for (int dd = 0; dd < ND; ++dd) vv[dd] = sV[c * LD + tx + 16 * dd];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                for (int dd = 0; dd < ND; ++dd) acc[rr][dd] = fmaf(pv[rr], vv[dd], acc[rr][dd]);
+        }
+    }
+    const TI* gin = static_cast<const TI*>(p.g);
+    TI* out = static_cast<TI*>(p.o);
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+        const int i = i0 + ty + 16 * rr;
+        if (i >= T) continue;
+        const float inv = 1.f / l_r[rr];
+#pragma unroll
+        for (int dd = 0; dd < ND; ++dd) {
+            const size_t off = (((size_t)b * T + i) * p.H + h) * DH + tx + 16 * dd;
+            Elem<TI>::st(out + off, acc[rr][dd] * inv * sigmoid_f(Elem<TI>::ld(gin + off)));
+        }
+        if (tx == 0 && p.lse) p.lse[((size_t)b * p.H + h) * T + i] = m_r[rr] + logf(l_r[rr]);
+    }
+}
+
+// ------------------------------------------------------------------ launchers
+cudaError_t launch_prep(const PrepParams& p, bool bf16_in, bool bf16_work, cudaStream_t s) {
+    dim3 grid(p.T, p.B);
+    if (bf16_in && bf16_work) k_prep<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, s>>>(p);
+    else if (bf16_in) k_prep<__nv_bfloat16, float><<<grid, 256, 0, s>>>(p);
+    else if (bf16_work) k_prep<float, __nv_bfloat16><<<grid, 256, 0, s>>>(p);
+    else k_prep<float, float><<<grid, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_boundary_simt(const BoundaryParams& p, cudaStream_t s) {
+    dim3 grid((p.T + 127) / 128, p.Hkv, p.B);
+    if (p.d == 64) k_boundary_simt<64><<<grid, 128, 0, s>>>(p);
+    else k_boundary_simt<128><<<grid, 128, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <int DH, typename TI>
+static cudaError_t fwd_simt_inst(const FwdParams& p, cudaStream_t s) {
+    constexpr int BM = 64, BN = 64, LD = DH + 1, LP = BN + 1;
+    const size_t smem = sizeof(float) * (size_t)(2 * BM * LD + 3 * BN * LD + 2 * BM * LP + BM + 2 * BN);
+    cudaError_t e = cudaFuncSetAttribute(k_fwd_simt<DH, TI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.nqt, p.H, p.B);
+    k_fwd_simt<DH, TI><<<grid, 256, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_simt(const FwdParams& p, bool bf16_act, cudaStream_t s) {
+    if (p.d == 64) return bf16_act ? fwd_simt_inst<64, __nv_bfloat16>(p, s) : fwd_simt_inst<64, float>(p, s);
+    return bf16_act ? fwd_simt_inst<128, __nv_bfloat16>(p, s) : fwd_simt_inst<128, float>(p, s);
+}
+
+}  // namespace ua

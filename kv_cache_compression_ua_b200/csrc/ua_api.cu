@@ -1,0 +1,233 @@
+// ua_api.cu -- the C ABI of libua: argument validation, workspace carving and launches.
+// Formulas, layouts and error behaviour are documented in include/ua.h.
+#include <math.h>
+#include <string.h>
+
+#include "ua_common.cuh"
+#include "ua_kernels.h"
+
+namespace ua {
+__device__ int g_status = 0;
+}
+
+using namespace ua;
+
+namespace {
+
+constexpr int kVersion = 100;   // 0.1.0
+constexpr int kBq = 64;         // query tile height of the SIMT attention path
+constexpr int kMaxCapacity = 1 << 20;   // decode keeps a capacity/32-word bitmap in shared memory
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool group_ok(int G) { return G == 1 || G == 2 || G == 3 || G == 4 || G == 8; }
+
+ua_status check_shape(const ua_shape* s) {
+    if (!s) return UA_ERR_INVALID_ARG;
+    if (s->B < 1 || s->T < 1 || s->H < 1 || s->Hkv < 1) return UA_ERR_INVALID_ARG;
+    if (s->H % s->Hkv != 0) return UA_ERR_INVALID_ARG;
+    if (!(s->rope_theta > 0.0) || !isfinite(s->scale)) return UA_ERR_INVALID_ARG;
+    if (s->d != 64 && s->d != 128) return UA_ERR_UNSUPPORTED;
+    if (!group_ok(s->H / s->Hkv)) return UA_ERR_UNSUPPORTED;
+    if (s->dtype != UA_F32 && s->dtype != UA_BF16) return UA_ERR_UNSUPPORTED;
+    return UA_OK;
+}
+
+// Workspace of the prefill forward: f32 rotated/normalised copies, rates, prefixes.
+struct FwdWs {
+    size_t qr, kh, kr, rq, rk, pb, total;
+};
+
+FwdWs fwd_ws_layout(const ua_shape* s) {
+    const size_t B = s->B, T = s->T, H = s->H, Hkv = s->Hkv, d = s->d;
+    const size_t nqt = (T + kBq - 1) / kBq;
+    FwdWs w;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = round_up(off + bytes, 256); return o; };
+    w.qr = take(B * H * T * d * 4);
+    w.kh = take(B * Hkv * T * d * 4);
+    w.kr = take(B * Hkv * T * d * 4);
+    w.rq = take(B * Hkv * T * 4);
+    w.rk = take(B * Hkv * T * 4);
+    w.pb = take(B * Hkv * nqt * T * 4);
+    w.total = off;
+    return w;
+}
+
+ua_status cuda_status(cudaError_t e) { return e == cudaSuccess ? UA_OK : UA_ERR_CUDA; }
+
+char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
+
+ua_status check_cache(const ua_cache* c) {
+    if (!c) return UA_ERR_INVALID_ARG;
+    if (c->B < 1 || c->Hkv < 1 || c->capacity < 1) return UA_ERR_INVALID_ARG;
+    if (c->capacity > kMaxCapacity) return UA_ERR_UNSUPPORTED;
+    if (c->d != 64 && c->d != 128) return UA_ERR_UNSUPPORTED;
+    if (c->dtype != UA_F32 && c->dtype != UA_BF16) return UA_ERR_UNSUPPORTED;
+    if (!c->khat || !c->krope || !c->v || !c->bias || !c->rk || !c->pos || !c->n_kept) return UA_ERR_INVALID_ARG;
+    const void* ps[] = {c->khat, c->krope, c->v, c->bias, c->rk, c->pos, c->n_kept};
+    for (const void* p : ps)
+        if (!aligned(p, 16)) return UA_ERR_ALIGNMENT;
+    return UA_OK;
+}
+
+CacheView view(const ua_cache* c) {
+    CacheView v;
+    v.B = c->B; v.Hkv = c->Hkv; v.d = c->d; v.cap = c->capacity;
+    v.khat = c->khat; v.krope = c->krope; v.v = c->v; v.bias = c->bias; v.rk = c->rk;
+    v.pos = c->pos; v.n_kept = c->n_kept;
+    return v;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ua_version(void) { return kVersion; }
+
+const char* ua_status_string(ua_status s) {
+    switch (s) {
+        case UA_OK: return "UA_OK";
+        case UA_ERR_INVALID_ARG: return "UA_ERR_INVALID_ARG";
+        case UA_ERR_UNSUPPORTED: return "UA_ERR_UNSUPPORTED";
+        case UA_ERR_ALIGNMENT: return "UA_ERR_ALIGNMENT";
+        case UA_ERR_WORKSPACE: return "UA_ERR_WORKSPACE";
+        case UA_ERR_CAPACITY: return "UA_ERR_CAPACITY";
+        case UA_ERR_CUDA: return "UA_ERR_CUDA";
+        case UA_ERR_TIMEOUT: return "UA_ERR_TIMEOUT";
+    }
+    return "UA_ERR_UNKNOWN";
+}
+
+ua_status ua_prefill_workspace_size(const ua_shape* shape, size_t* bytes) {
+    ua_status st = check_shape(shape);
+    if (st != UA_OK) return st;
+    if (!bytes) return UA_ERR_INVALID_ARG;
+    *bytes = fwd_ws_layout(shape).total;
+    return UA_OK;
+}
+
+ua_status ua_prefill_fwd(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
+                         const float* a_q, const float* a_k, const float* alpha, const float* beta,
+                         void* o, float* lse, float* b_final, float* lambda_dbg, void* ws, size_t ws_bytes,
+                         void* stream) {
+    ua_status st = check_shape(s);
+    if (st != UA_OK) return st;
+    if (!q || !k || !v || !g || !a_q || !a_k || !alpha || !beta || !o || !ws) return UA_ERR_INVALID_ARG;
+    const void* ps[] = {q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, lambda_dbg};
+    for (const void* p : ps)
+        if (p && !aligned(p, 16)) return UA_ERR_ALIGNMENT;
+    if (!aligned(ws, 256)) return UA_ERR_ALIGNMENT;
+    if (lambda_dbg && s->T > 1024) return UA_ERR_INVALID_ARG;
+    const FwdWs w = fwd_ws_layout(s);
+    if (ws_bytes < w.total) return UA_ERR_WORKSPACE;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const bool bf = s->dtype == UA_BF16;
+    const int nqt = (s->T + kBq - 1) / kBq;
+
+    PrepParams pp;
+    pp.B = s->B; pp.T = s->T; pp.H = s->H; pp.Hkv = s->Hkv; pp.d = s->d; pp.theta = s->rope_theta;
+    pp.q = q; pp.k = k; pp.a_q = a_q; pp.a_k = a_k;
+    pp.qr = at(ws, w.qr); pp.kh = at(ws, w.kh); pp.kr = at(ws, w.kr);
+    pp.rq = reinterpret_cast<float*>(at(ws, w.rq)); pp.rk = reinterpret_cast<float*>(at(ws, w.rk));
+    if ((st = cuda_status(launch_prep(pp, bf, false, cs))) != UA_OK) return st;
+
+    BoundaryParams bp;
+    bp.B = s->B; bp.T = s->T; bp.Hkv = s->Hkv; bp.d = s->d; bp.bq = kBq; bp.nqt = nqt;
+    bp.kh = reinterpret_cast<const float*>(pp.kh); bp.rq = pp.rq; bp.rk = pp.rk;
+    bp.alpha = alpha; bp.beta = beta;
+    bp.pb = reinterpret_cast<float*>(at(ws, w.pb)); bp.bfinal = b_final;
+    if ((st = cuda_status(launch_boundary_simt(bp, cs))) != UA_OK) return st;
+
+    if (lambda_dbg) {
+        const size_t n = (size_t)s->B * s->Hkv * s->T * s->T * sizeof(float);
+        if ((st = cuda_status(cudaMemsetAsync(lambda_dbg, 0, n, cs))) != UA_OK) return st;
+    }
+    FwdParams fp;
+    fp.B = s->B; fp.T = s->T; fp.H = s->H; fp.Hkv = s->Hkv; fp.d = s->d; fp.G = s->H / s->Hkv; fp.nqt = nqt;
+    fp.scale = s->scale;
+    fp.qr = reinterpret_cast<const float*>(pp.qr); fp.kh = reinterpret_cast<const float*>(pp.kh);
+    fp.kr = reinterpret_cast<const float*>(pp.kr);
+    fp.v = v; fp.g = g; fp.rq = pp.rq; fp.rk = pp.rk; fp.alpha = alpha; fp.beta = beta; fp.pb = bp.pb;
+    fp.o = o; fp.lse = lse; fp.lambda_dbg = lambda_dbg;
+    return cuda_status(launch_fwd_simt(fp, bf, cs));
+}
+
+ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes) {
+    ua_status st = check_shape(shape);
+    if (st != UA_OK) return st;
+    if (!bytes) return UA_ERR_INVALID_ARG;
+    *bytes = 0;
+    return UA_ERR_UNSUPPORTED;
+}
+
+ua_status ua_prefill_bwd(const ua_shape* s, const void*, const void*, const void*, const void*, const float*,
+                         const float*, const float*, const float*, const void*, const float*, const float*,
+                         const void*, void*, void*, void*, void*, float*, float*, float*, float*, void*, size_t,
+                         void*) {
+    ua_status st = check_shape(s);
+    if (st != UA_OK) return st;
+    return UA_ERR_UNSUPPORTED;
+}
+
+ua_status ua_cache_fill(const ua_cache* c, int T, const void* k, const void* v, const float* a_k,
+                        const float* b_final, double rope_theta, void* stream) {
+    ua_status st = check_cache(c);
+    if (st != UA_OK) return st;
+    if (T < 1 || !k || !v || !a_k || !b_final || !(rope_theta > 0.0)) return UA_ERR_INVALID_ARG;
+    if (T > c->capacity) return UA_ERR_CAPACITY;
+    const void* ps[] = {k, v, a_k, b_final};
+    for (const void* p : ps)
+        if (!aligned(p, 16)) return UA_ERR_ALIGNMENT;
+    FillParams fp;
+    fp.c = view(c); fp.T = T; fp.theta = rope_theta; fp.k = k; fp.v = v; fp.a_k = a_k; fp.bfinal = b_final;
+    return cuda_status(launch_cache_fill(fp, c->dtype == UA_BF16, static_cast<cudaStream_t>(stream)));
+}
+
+ua_status ua_cache_compact(const ua_cache* c, const uint8_t* keep, float p, int32_t* kept_idx, void* stream) {
+    ua_status st = check_cache(c);
+    if (st != UA_OK) return st;
+    if (!keep && !(p >= 0.f && p <= 1.f)) return UA_ERR_INVALID_ARG;
+    if ((keep && !aligned(keep, 16)) || (kept_idx && !aligned(kept_idx, 16))) return UA_ERR_ALIGNMENT;
+    CompactParams cp;
+    cp.c = view(c); cp.keep = keep; cp.logp = p > 0.f ? logf(p) : -INFINITY; cp.kept_idx = kept_idx;
+    return cuda_status(launch_cache_compact(cp, c->dtype == UA_BF16, static_cast<cudaStream_t>(stream)));
+}
+
+ua_status ua_decode_step(const ua_cache* c, int H, const void* q, const void* k, const void* v, const void* g,
+                         const float* a_q, const float* a_k, const float* alpha, const float* beta, int pos_t,
+                         float p, float scale, double rope_theta, void* o, uint32_t* evict_bits,
+                         int32_t* kept_idx, int flags, void* stream) {
+    ua_status st = check_cache(c);
+    if (st != UA_OK) return st;
+    if (H < 1 || H % c->Hkv != 0 || pos_t < 0 || flags != 0) return UA_ERR_INVALID_ARG;
+    if (!group_ok(H / c->Hkv)) return UA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !g || !a_q || !a_k || !alpha || !beta || !o) return UA_ERR_INVALID_ARG;
+    if (!(p >= 0.f && p <= 1.f) || !isfinite(scale) || !(rope_theta > 0.0)) return UA_ERR_INVALID_ARG;
+    const void* ps[] = {q, k, v, g, a_q, a_k, alpha, beta, o, evict_bits, kept_idx};
+    for (const void* x : ps)
+        if (x && !aligned(x, 16)) return UA_ERR_ALIGNMENT;
+    DecodeParams dp;
+    dp.c = view(c); dp.H = H; dp.G = H / c->Hkv; dp.pos_t = pos_t; dp.scale = scale;
+    dp.logp = p > 0.f ? logf(p) : -INFINITY; dp.theta = rope_theta;
+    dp.q = q; dp.k = k; dp.v = v; dp.g = g; dp.a_q = a_q; dp.a_k = a_k; dp.alpha = alpha; dp.beta = beta;
+    dp.o = o; dp.evict_bits = evict_bits; dp.kept_idx = kept_idx;
+    return cuda_status(launch_decode(dp, c->dtype == UA_BF16, static_cast<cudaStream_t>(stream)));
+}
+
+ua_status ua_get_device_status(void* stream, int* code) {
+    if (!code) return UA_ERR_INVALID_ARG;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    int host = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&host, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    const int zero = 0;
+    if (e == cudaSuccess) e = cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return UA_ERR_CUDA;
+    *code = host;
+    return UA_OK;
+}
+
+}  // extern "C"

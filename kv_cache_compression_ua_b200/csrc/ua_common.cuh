@@ -1,0 +1,93 @@
+// ua_common.cuh -- small device helpers shared by the libua kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ua.h"
+
+namespace ua {
+
+// Device status word: the first ua_status code a kernel raises sticks until
+// ua_get_device_status reads and clears it.  Defined in ua_api.cu.
+extern __device__ int g_status;
+
+__device__ __forceinline__ void raise_status(int code) { atomicCAS(&g_status, 0, code); }
+
+// ------------------------------------------------------------------ scalar math
+// softplus(x) = log(1 + e^x) in its overflow-free form.
+__device__ __forceinline__ float softplus_f(float x) {
+    return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
+}
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + expf(-x)); }
+
+// Geometric mean of the three decay rates (veto: a zero factor gives exactly zero).
+__device__ __forceinline__ float decay_geo(float rq, float rk, float rsim) {
+    return cbrtf(rq * rk * rsim);
+}
+
+// RoPE angle of pair m at position pos, in double precision (positions up to 1e6 keep
+// the angle accurate to ~1e-10 rad before the fp32 cos/sin are formed).
+__device__ __forceinline__ void rope_cs(double pos, int m, int d, double theta, float* c, float* s) {
+    double freq = pow(theta, -2.0 * (double)m / (double)d);
+    double sn, cs;
+    sincos(pos * freq, &sn, &cs);
+    *c = (float)cs;
+    *s = (float)sn;
+}
+
+// ------------------------------------------------------------------ element access
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float ld(const float* p) { return *p; }
+    static __device__ __forceinline__ void st(float* p, float x) { *p = x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ void st(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+};
+
+// 16-byte vector of activations <-> float registers.
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+    static constexpr int N = 4;
+    static __device__ __forceinline__ void ld(const float* p, float* x) {
+        float4 u = *reinterpret_cast<const float4*>(p);
+        x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+    }
+    static __device__ __forceinline__ void st(float* p, const float* x) {
+        *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    }
+    static __device__ __forceinline__ uint4 raw(const float* p) { return *reinterpret_cast<const uint4*>(p); }
+    static __device__ __forceinline__ void unpack(uint4 u, float* x) {
+        x[0] = __uint_as_float(u.x); x[1] = __uint_as_float(u.y);
+        x[2] = __uint_as_float(u.z); x[3] = __uint_as_float(u.w);
+    }
+};
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int N = 8;
+    static __device__ __forceinline__ void unpack(uint4 u, float* x) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    static __device__ __forceinline__ void ld(const __nv_bfloat16* p, float* x) {
+        unpack(*reinterpret_cast<const uint4*>(p), x);
+    }
+    static __device__ __forceinline__ uint4 raw(const __nv_bfloat16* p) { return *reinterpret_cast<const uint4*>(p); }
+    static __device__ __forceinline__ void st(__nv_bfloat16* p, const float* x) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+}  // namespace ua

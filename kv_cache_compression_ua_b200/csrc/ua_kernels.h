@@ -1,0 +1,147 @@
+// ua_kernels.h -- internal launch interface between ua_api.cu and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ua {
+
+// Token preparation: normalised keys, RoPE'd queries/keys, per-token rates.
+struct PrepParams {
+    int B, T, H, Hkv, d;
+    double theta;
+    const void* q;      // [B,T,H,d] act
+    const void* k;      // [B,T,Hkv,d] act
+    const float* a_q;   // [B,T,Hkv]
+    const float* a_k;   // [B,T,Hkv]
+    void* qr;           // [B,H,T,d] work type: RoPE(q)
+    void* kh;           // [B,Hkv,T,d] work type: khat
+    void* kr;           // [B,Hkv,T,d] work type: RoPE(khat)
+    float* rq;          // [B,Hkv,T] softplus(a_q)
+    float* rk;          // [B,Hkv,T] softplus(a_k)
+};
+
+// Boundary pass: per-query-tile column prefixes of the decay and the final biases.
+struct BoundaryParams {
+    int B, T, Hkv, d;
+    int bq;             // query tile height the prefixes are cut at
+    int nqt;            // ceil(T / bq)
+    const float* kh;    // [B,Hkv,T,d] f32
+    const float* rq;    // [B,Hkv,T]
+    const float* rk;    // [B,Hkv,T]
+    const float* alpha; // [Hkv]
+    const float* beta;  // [Hkv]
+    float* pb;          // [B,Hkv,nqt,T]: sum_{j < l < t*bq} D[l,j]  (>= 0)
+    float* bfinal;      // [B,Hkv,T] = -sum_{l > j} D[l,j], or NULL
+};
+
+// Fused biased attention (SIMT path).
+struct FwdParams {
+    int B, T, H, Hkv, d, G, nqt;
+    float scale;
+    const float* qr;    // [B,H,T,d]
+    const float* kh;    // [B,Hkv,T,d]
+    const float* kr;    // [B,Hkv,T,d]
+    const void* v;      // [B,T,Hkv,d] act
+    const void* g;      // [B,T,H,d] act
+    const float* rq;
+    const float* rk;
+    const float* alpha;
+    const float* beta;
+    const float* pb;    // [B,Hkv,nqt,T] with bq = 64
+    void* o;            // [B,T,H,d] act
+    float* lse;         // [B,H,T] or NULL
+    float* lambda_dbg;  // [B,Hkv,T,T] or NULL (pre-zeroed)
+};
+
+struct CacheView {
+    int B, Hkv, d, cap;
+    void* khat;
+    void* krope;
+    void* v;
+    float* bias;
+    float* rk;
+    int32_t* pos;
+    int32_t* n_kept;
+};
+
+struct FillParams {
+    CacheView c;
+    int T;
+    double theta;
+    const void* k;       // [B,T,Hkv,d] act
+    const void* v;       // [B,T,Hkv,d] act
+    const float* a_k;    // [B,T,Hkv]
+    const float* bfinal; // [B,Hkv,T]
+};
+
+struct CompactParams {
+    CacheView c;
+    const uint8_t* keep; // [B,Hkv,cap] or NULL
+    float logp;
+    int32_t* kept_idx;   // or NULL
+};
+
+struct DecodeParams {
+    CacheView c;
+    int H, G, pos_t;
+    float scale, logp;
+    double theta;
+    const void* q;       // [B,H,d] act
+    const void* k;       // [B,Hkv,d] act
+    const void* v;       // [B,Hkv,d] act
+    const void* g;       // [B,H,d] act
+    const float* a_q;    // [B,Hkv]
+    const float* a_k;    // [B,Hkv]
+    const float* alpha;
+    const float* beta;
+    void* o;             // [B,H,d] act
+    uint32_t* evict_bits;
+    int32_t* kept_idx;
+};
+
+// Backward (SIMT path).
+struct BwdParams {
+    int B, T, H, Hkv, d, G, nqt;
+    float scale;
+    const float* qr;     // [B,H,T,d]  RoPE(q)
+    const float* kh;     // [B,Hkv,T,d]
+    const float* kr;     // [B,Hkv,T,d]
+    const void* v;       // [B,T,Hkv,d] act
+    const void* g;       // [B,T,H,d] act
+    const void* o;       // [B,T,H,d] act
+    const void* d_o;     // [B,T,H,d] act
+    const float* a_q;    // [B,T,Hkv]
+    const float* a_k;    // [B,T,Hkv]
+    const float* rq;     // [B,Hkv,T]
+    const float* rk;     // [B,Hkv,T]
+    const float* alpha;
+    const float* beta;
+    const float* lse;    // [B,H,T]
+    const float* bfinal; // [B,Hkv,T]
+    float* delta;        // [B,H,T] rowwise dO.O
+    float* dqr;          // [B,H,T,d] f32 accum of dL/dRoPE(q)
+    float* dkh;          // [B,Hkv,T,d] f32 accum of dL/dkhat (similarity path + RoPE^T dkr)
+    float* dkr;          // [B,Hkv,T,d] f32 dL/dRoPE(khat)
+    float* dv32;         // [B,Hkv,T,d] f32 dL/dv
+    float* daq32;        // [B,Hkv,T] f32 accum (over key tiles)
+    float* dak32;        // [B,Hkv,T] f32
+    float* dab;          // [B*Hkv*nkt][2] per-CTA partial (dalpha, dbeta)
+    int nkt;
+    // outputs
+    double theta;
+    const void* k;       // raw keys for the normalisation Jacobian
+    void* dq; void* dk; void* dv; void* dg;
+    float* da_q; float* da_k; float* dalpha; float* dbeta;
+};
+
+cudaError_t launch_prep(const PrepParams& p, bool bf16_in, bool bf16_work, cudaStream_t s);
+cudaError_t launch_boundary_simt(const BoundaryParams& p, cudaStream_t s);
+cudaError_t launch_fwd_simt(const FwdParams& p, bool bf16_act, cudaStream_t s);
+cudaError_t launch_cache_fill(const FillParams& p, bool bf16, cudaStream_t s);
+cudaError_t launch_cache_compact(const CompactParams& p, bool bf16, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t s);
+cudaError_t launch_bwd_simt(const BwdParams& p, bool bf16_act, cudaStream_t s);
+
+}  // namespace ua

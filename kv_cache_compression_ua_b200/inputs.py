@@ -22,7 +22,9 @@ the pages' RULER / LongBench-E / Dolma inputs):
 """
 from __future__ import annotations
 
+import concurrent.futures as _cf
 import dataclasses
+import os
 
 import numpy as np
 
@@ -183,6 +185,10 @@ def _draw(w: Workload, name: str, seed: int, full_shape, box):
     raise KeyError(name)
 
 
+def _workers() -> int:
+    return max(1, min(32, os.cpu_count() or 1))
+
+
 def make_prefill_inputs(w: Workload, T: int | None = None, B: int | None = None,
                         names=None, b0: int = 0) -> dict:
     """Prefill inputs as float32 numpy arrays holding values already rounded to w.dtype.
@@ -211,8 +217,16 @@ def make_prefill_inputs(w: Workload, T: int | None = None, B: int | None = None,
         heads = H if n in ("q", "g", "d_o") else Hkv
         full = (Bf, Tf, heads, d) if n in ("q", "k", "v", "g", "d_o") else (Bf, Tf, heads)
         arr = np.empty((B, T) + full[2:], dtype=np.float32)
-        for bi in range(B):            # one batch at a time keeps the fp64 temporaries small
-            arr[bi] = _draw(w, n, s, full, ((b0 + bi, 0), (1, T)))[0]
+        # chunks of (one batch, up to 256 tokens) drawn on a thread pool: numpy releases the
+        # GIL in its ufuncs, and the fp64 temporaries stay small
+        chunks = [(bi, t0, min(256, T - t0)) for bi in range(B) for t0 in range(0, T, 256)]
+
+        def work(c, n=n, full=full, arr=arr):
+            bi, t0, nt = c
+            arr[bi, t0:t0 + nt] = _draw(w, n, s, full, ((b0 + bi, t0), (1, nt)))[0]
+
+        with _cf.ThreadPoolExecutor(max_workers=_workers()) as ex:
+            list(ex.map(work, chunks))
         out[n] = arr
     return out
 

@@ -1,0 +1,250 @@
+"""Thin Python binding of libua (include/ua.h): argument marshalling only.
+
+Every step of the Universal Attention hot path runs in libua's CUDA kernels; this module
+only turns torch CUDA tensors into device pointers, allocates outputs / workspaces with
+torch (device memory plumbing) and checks status codes.  There is no fallback: if libua.so
+is missing or a CUDA device is absent, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libua.so")
+
+UA_F32, UA_BF16 = 0, 1
+STATUS = {0: "UA_OK", 1: "UA_ERR_INVALID_ARG", 2: "UA_ERR_UNSUPPORTED", 3: "UA_ERR_ALIGNMENT",
+          4: "UA_ERR_WORKSPACE", 5: "UA_ERR_CAPACITY", 6: "UA_ERR_CUDA", 7: "UA_ERR_TIMEOUT"}
+
+
+class UAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        self.code = code
+
+
+class ua_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("d", ctypes.c_int), ("scale", ctypes.c_float), ("rope_theta", ctypes.c_double),
+                ("dtype", ctypes.c_int)]
+
+
+class ua_cache(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int), ("capacity", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("khat", ctypes.c_void_p), ("krope", ctypes.c_void_p),
+                ("v", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("rk", ctypes.c_void_p),
+                ("pos", ctypes.c_void_p), ("n_kept", ctypes.c_void_p)]
+
+
+EXPORTS = ("ua_prefill_workspace_size", "ua_prefill_fwd", "ua_prefill_bwd_workspace_size", "ua_prefill_bwd",
+           "ua_cache_fill", "ua_cache_compact", "ua_decode_step", "ua_get_device_status",
+           "ua_status_string", "ua_version")
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libua.so and declare its signatures.  Raises if the file is missing."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libua.so not found at {path}; build it with "
+                           "`python -m kv_cache_compression_ua_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, F, D, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_double, ctypes.c_size_t
+    SP = ctypes.POINTER(ua_shape)
+    CP = ctypes.POINTER(ua_cache)
+    lib.ua_prefill_workspace_size.argtypes = [SP, ctypes.POINTER(S)]
+    lib.ua_prefill_fwd.argtypes = [SP] + [P] * 8 + [P, P, P, P, P, S, P]
+    lib.ua_prefill_bwd_workspace_size.argtypes = [SP, ctypes.POINTER(S)]
+    lib.ua_prefill_bwd.argtypes = [SP] + [P] * 8 + [P, P, P, P] + [P] * 8 + [P, S, P]
+    lib.ua_cache_fill.argtypes = [CP, I, P, P, P, P, D, P]
+    lib.ua_cache_compact.argtypes = [CP, P, F, P, P]
+    lib.ua_decode_step.argtypes = [CP, I] + [P] * 8 + [I, F, F, D, P, P, P, I, P]
+    lib.ua_get_device_status.argtypes = [P, ctypes.POINTER(I)]
+    lib.ua_status_string.argtypes = [I]
+    lib.ua_status_string.restype = ctypes.c_char_p
+    lib.ua_version.argtypes = []
+    for n in EXPORTS:
+        if n not in ("ua_status_string", "ua_version"):
+            getattr(lib, n).restype = I
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise UAError(fn, code)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libua takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libua takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return UA_F32
+    if dt == torch.bfloat16:
+        return UA_BF16
+    raise ValueError(f"unsupported activation dtype {dt}")
+
+
+def make_shape(q: torch.Tensor, k: torch.Tensor, scale=None, theta=500000.0) -> ua_shape:
+    B, T, H, d = q.shape
+    Hkv = k.shape[2]
+    scale = float(d) ** -0.5 if scale is None else float(scale)
+    return ua_shape(B, T, H, Hkv, d, scale, float(theta), _dtype_code(q.dtype))
+
+
+def prefill_workspace_size(shape: ua_shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check("ua_prefill_workspace_size", load_library().ua_prefill_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns >= 512-byte aligned blocks
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0, want_lse=True,
+                want_bfinal=True, want_lambda=False, out=None, ws=None, stream=None):
+    """ua_prefill_fwd.  Returns dict(o, lse, b_final, lam) (absent outputs are None)."""
+    lib = load_library()
+    shape = make_shape(q, k, scale, theta)
+    B, T, H, d = q.shape
+    Hkv = k.shape[2]
+    dev = q.device
+    o = out if out is not None else torch.empty_like(q)
+    lse = torch.empty(B, H, T, dtype=torch.float32, device=dev) if want_lse else None
+    bfin = torch.empty(B, Hkv, T, dtype=torch.float32, device=dev) if want_bfinal else None
+    lam = torch.empty(B, Hkv, T, T, dtype=torch.float32, device=dev) if want_lambda else None
+    need = prefill_workspace_size(shape)
+    if ws is None or ws.numel() < need:
+        ws = alloc_workspace(need, dev)
+    rc = lib.ua_prefill_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
+                            _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(bfin), _ptr(lam),
+                            _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(stream))
+    _check("ua_prefill_fwd", rc)
+    return {"o": o, "lse": lse, "b_final": bfin, "lam": lam}
+
+
+def prefill_bwd_workspace_size(shape: ua_shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check("ua_prefill_bwd_workspace_size",
+           load_library().ua_prefill_bwd_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
+def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, d_o, *, scale=None, theta=500000.0,
+                ws=None, stream=None):
+    """ua_prefill_bwd.  Returns dict(dq, dk, dv, dg, da_q, da_k, dalpha, dbeta)."""
+    lib = load_library()
+    shape = make_shape(q, k, scale, theta)
+    dev = q.device
+    gr = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+          "dg": torch.empty_like(g), "da_q": torch.empty_like(a_q), "da_k": torch.empty_like(a_k),
+          "dalpha": torch.empty_like(alpha), "dbeta": torch.empty_like(beta)}
+    need = prefill_bwd_workspace_size(shape)
+    if ws is None or ws.numel() < need:
+        ws = alloc_workspace(need, dev)
+    rc = lib.ua_prefill_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
+                            _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(b_final), _ptr(d_o),
+                            _ptr(gr["dq"]), _ptr(gr["dk"]), _ptr(gr["dv"]), _ptr(gr["dg"]), _ptr(gr["da_q"]),
+                            _ptr(gr["da_k"]), _ptr(gr["dalpha"]), _ptr(gr["dbeta"]), _ptr(ws),
+                            ctypes.c_size_t(ws.numel()), _stream(stream))
+    _check("ua_prefill_bwd", rc)
+    return gr
+
+
+@dataclass
+class Cache:
+    """Device tensors of one self-pruning cache set (see ua_cache in ua.h)."""
+    B: int
+    Hkv: int
+    d: int
+    capacity: int
+    dtype: torch.dtype
+    khat: torch.Tensor
+    krope: torch.Tensor
+    v: torch.Tensor
+    bias: torch.Tensor
+    rk: torch.Tensor
+    pos: torch.Tensor
+    n_kept: torch.Tensor
+
+    @staticmethod
+    def empty(B, Hkv, d, capacity, dtype=torch.bfloat16, device="cuda"):
+        kw = dict(device=device)
+        return Cache(B, Hkv, d, capacity, dtype,
+                     torch.zeros(B, Hkv, capacity, d, dtype=dtype, **kw),
+                     torch.zeros(B, Hkv, capacity, d, dtype=dtype, **kw),
+                     torch.zeros(B, Hkv, capacity, d, dtype=dtype, **kw),
+                     torch.zeros(B, Hkv, capacity, dtype=torch.float32, **kw),
+                     torch.zeros(B, Hkv, capacity, dtype=torch.float32, **kw),
+                     torch.zeros(B, Hkv, capacity, dtype=torch.int32, **kw),
+                     torch.zeros(B, Hkv, dtype=torch.int32, **kw))
+
+    def struct(self) -> ua_cache:
+        return ua_cache(self.B, self.Hkv, self.d, self.capacity, _dtype_code(self.dtype),
+                        self.khat.data_ptr(), self.krope.data_ptr(), self.v.data_ptr(), self.bias.data_ptr(),
+                        self.rk.data_ptr(), self.pos.data_ptr(), self.n_kept.data_ptr())
+
+    def nbytes_per_entry(self) -> int:
+        return 3 * self.d * self.khat.element_size() + 12
+
+
+def cache_fill(cache: Cache, k, v, a_k, b_final, *, theta=500000.0, stream=None):
+    T = k.shape[1]
+    c = cache.struct()
+    _check("ua_cache_fill", load_library().ua_cache_fill(ctypes.byref(c), T, _ptr(k), _ptr(v), _ptr(a_k),
+                                                         _ptr(b_final), float(theta), _stream(stream)))
+
+
+def cache_compact(cache: Cache, p: float = 0.0, keep=None, kept_idx=None, stream=None):
+    c = cache.struct()
+    _check("ua_cache_compact", load_library().ua_cache_compact(ctypes.byref(c), _ptr(keep), float(p),
+                                                               _ptr(kept_idx), _stream(stream)))
+
+
+def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: float, *, scale=None,
+                theta=500000.0, out=None, evict_bits=None, kept_idx=None, stream=None):
+    """ua_decode_step for one token per sequence.  Returns o [B,H,d]."""
+    H = q.shape[1]
+    d = q.shape[2]
+    scale = float(d) ** -0.5 if scale is None else float(scale)
+    o = out if out is not None else torch.empty_like(q)
+    c = cache.struct()
+    rc = load_library().ua_decode_step(ctypes.byref(c), H, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q),
+                                       _ptr(a_k), _ptr(alpha), _ptr(beta), int(pos_t), float(p), scale,
+                                       float(theta), _ptr(o), _ptr(evict_bits), _ptr(kept_idx), 0,
+                                       _stream(stream))
+    _check("ua_decode_step", rc)
+    return o
+
+
+def get_device_status(stream=None) -> int:
+    code = ctypes.c_int(0)
+    _check("ua_get_device_status", load_library().ua_get_device_status(_stream(stream), ctypes.byref(code)))
+    return code.value
+
+
+def version() -> int:
+    return load_library().ua_version()

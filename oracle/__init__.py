@@ -151,14 +151,23 @@ class DecodeCache:
         self.b = np.zeros((B, Hkv, cap))
         self.n = np.zeros((B, Hkv), dtype=np.int32)
 
-    def fill_from_prefill(self, k, v, a_k, b_final, logp=None):
+    def fill_from_prefill(self, k, v, a_k, b_final, logp=None, adopt_keep=None, band=1e-3):
         """Load a prefill's keys/values/a_k with their final biases b_final (Lambda's last
-        row).  With logp given, keep only pairs with b >= logp (stable order)."""
+        row).  With logp given, keep only pairs with b >= logp (stable order); for pairs whose
+        bias lies within `band` of logp, adopt_keep[b, h, t] (if given) decides instead.
+        Returns the in-band mask [B,Hkv,T]."""
         k, v, a_k, b_final = _f64(k), _f64(v), _f64(a_k), _f64(b_final)
         B, T, Hkv, d = k.shape
+        in_band = np.zeros((B, Hkv, T), bool)
         for b in range(B):
             for h in range(Hkv):
-                keep = np.ones(T, bool) if logp is None else (b_final[b, h] >= logp)
+                if logp is None:
+                    keep = np.ones(T, bool)
+                else:
+                    keep = b_final[b, h] >= logp
+                    in_band[b, h] = np.abs(b_final[b, h] - logp) < band
+                    if adopt_keep is not None:
+                        keep = np.where(in_band[b, h], np.asarray(adopt_keep[b, h], bool), keep)
                 idx = np.nonzero(keep)[0]
                 n = len(idx)
                 if n > self.cap:
@@ -169,6 +178,7 @@ class DecodeCache:
                 self.pos[b, h, :n] = idx
                 self.b[b, h, :n] = b_final[b, h, idx]
                 self.n[b, h] = n
+        return in_band
 
 
 def decode_step(cache: DecodeCache, q, k, v, g, a_q, a_k, alpha, beta, pos_t, p, *,

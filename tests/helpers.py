@@ -1,0 +1,31 @@
+"""Shared test utilities: tolerances and comparisons (no method arithmetic)."""
+import numpy as np
+
+# Tolerances of the parity bar: fp32 outputs rel-L2 <= 1e-5 and max-abs <= 1e-4; bf16
+# outputs rel-L2 <= 5e-3 and max-abs <= 2e-2.  f32-typed outputs of a bf16 problem (lse,
+# b_final) use the bf16 bar with the max error taken relative to max(1, |ref|), because
+# their magnitude grows with T (b_final reaches -O(T)).
+TOL = {"f32": (1e-5, 1e-4), "bf16": (5e-3, 2e-2)}
+EVICT_BAND = 1e-3
+
+
+def rel_l2(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
+
+
+def assert_close(name, got, ref, dtype, relative_max=False):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    rl, ma = TOL[dtype]
+    r = rel_l2(got, ref)
+    err = np.abs(got - ref)
+    if relative_max:
+        err = err / np.maximum(1.0, np.abs(ref))
+    m = float(err.max()) if err.size else 0.0
+    assert r <= rl and m <= ma, f"{name}: rel-L2 {r:.3e} (<= {rl}), max-abs {m:.3e} (<= {ma})"
+    return r, m

@@ -1,0 +1,113 @@
+"""CPU checks of the C ABI: the library builds, loads, exports every symbol that
+include/ua.h declares, and rejects bad arguments on the host (before any launch)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from kv_cache_compression_ua_b200 import build as ua_build
+from kv_cache_compression_ua_b200 import ua
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ua_build.build()
+    return ua.load_library()
+
+
+def declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "ua.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(ua_[a-z_]+)\s*\(", txt)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ("ua_prefill_fwd", "ua_prefill_bwd", "ua_decode_step", "ua_cache_compact"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", ua.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (ua_[a-z_]+)\b", out))
+    missing = [n for n in declared_symbols() if n not in exported]
+    assert not missing, missing
+    for n in declared_symbols():
+        assert hasattr(lib, n)
+    assert set(ua.EXPORTS) == set(declared_symbols())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.ua_version() >= 100
+    assert lib.ua_status_string(0) == b"UA_OK"
+    assert lib.ua_status_string(5) == b"UA_ERR_CAPACITY"
+
+
+def _shape(**kw):
+    s = dict(B=1, T=128, H=4, Hkv=2, d=64, scale=0.125, rope_theta=5e5, dtype=ua.UA_BF16)
+    s.update(kw)
+    return ua.ua_shape(**s)
+
+
+FAKE = 0x7f0000000000          # aligned, never dereferenced: validation fails first
+
+
+def _fwd(lib, shape, ptrs=None, ws=FAKE, ws_bytes=1 << 40):
+    P = ctypes.c_void_p
+    p = [P(FAKE)] * 8 if ptrs is None else ptrs
+    return lib.ua_prefill_fwd(ctypes.byref(shape), *p, P(FAKE), None, None, None, P(ws),
+                              ctypes.c_size_t(ws_bytes), None)
+
+
+@pytest.mark.parametrize("kw,code", [(dict(d=96), 2), (dict(H=6, Hkv=4), 1), (dict(T=0), 1),
+                                     (dict(H=12, Hkv=2), 2), (dict(dtype=7), 2), (dict(rope_theta=0.0), 1)])
+def test_prefill_rejects_bad_shapes(lib, kw, code):
+    assert _fwd(lib, _shape(**kw)) == code
+
+
+def test_prefill_rejects_null_misaligned_and_small_workspace(lib):
+    P = ctypes.c_void_p
+    ptrs = [P(FAKE)] * 8
+    ptrs[2] = None
+    assert _fwd(lib, _shape(), ptrs) == 1
+    ptrs = [P(FAKE)] * 8
+    ptrs[0] = P(FAKE + 2)
+    assert _fwd(lib, _shape(), ptrs) == 3
+    assert _fwd(lib, _shape(), ws=FAKE + 16) == 3
+    need = ctypes.c_size_t(0)
+    assert lib.ua_prefill_workspace_size(ctypes.byref(_shape()), ctypes.byref(need)) == 0
+    assert need.value > 0
+    assert _fwd(lib, _shape(), ws_bytes=need.value - 1) == 4
+
+
+def test_lambda_debug_limited_to_small_T(lib):
+    P = ctypes.c_void_p
+    shape = _shape(T=2048)
+    rc = lib.ua_prefill_fwd(ctypes.byref(shape), *([P(FAKE)] * 8), P(FAKE), None, None, P(FAKE), P(FAKE),
+                            ctypes.c_size_t(1 << 40), None)
+    assert rc == 1
+
+
+def test_cache_calls_reject_bad_arguments(lib):
+    P = ctypes.c_void_p
+    c = ua.ua_cache(2, 2, 64, 100, ua.UA_BF16, *([FAKE] * 7))
+    # capacity too small for the fill
+    assert lib.ua_cache_fill(ctypes.byref(c), 101, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 5e5, None) == 5
+    # bad p without a mask
+    assert lib.ua_cache_compact(ctypes.byref(c), None, ctypes.c_float(1.5), None, None) == 1
+    # misaligned cache array
+    c2 = ua.ua_cache(2, 2, 64, 100, ua.UA_BF16, *([FAKE] * 6 + [FAKE + 4]))
+    assert lib.ua_cache_compact(ctypes.byref(c2), None, ctypes.c_float(0.1), None, None) == 3
+    # decode: group size 5 unsupported, flags must be 0, head_dim 80 unsupported
+    args = [P(FAKE)] * 8
+    assert lib.ua_decode_step(ctypes.byref(c), 10, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
+                              P(FAKE), None, None, 0, None) == 2
+    assert lib.ua_decode_step(ctypes.byref(c), 8, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
+                              P(FAKE), None, None, 1, None) == 1
+    c3 = ua.ua_cache(2, 2, 80, 100, ua.UA_BF16, *([FAKE] * 7))
+    assert lib.ua_decode_step(ctypes.byref(c3), 8, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
+                              P(FAKE), None, None, 0, None) == 2

@@ -1,0 +1,127 @@
+"""GPU parity of ua_prefill_fwd against the fp64 oracle (through the C ABI).
+
+Small cases compare every output element; the full-size workloads compare sampled
+(batch, KV-head) units and rows, which the oracle computes one by one."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_compression_ua_b200 import inputs as I
+from kv_cache_compression_ua_b200 import ua
+from helpers import TOL, assert_close
+
+pytestmark = pytest.mark.gpu
+
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def to_dev(x, w):
+    out = {}
+    for n, a in x.items():
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        dt = TORCH_DT[w.dtype] if n in ("q", "k", "v", "g", "d_o") else torch.float32
+        out[n] = t.to("cuda").to(dt).contiguous()
+    return out
+
+
+def run_gpu(w, x, want_lambda=False):
+    d = to_dev({k: v for k, v in x.items() if k != "d_o"}, w)
+    r = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
+                       scale=w.scale, theta=w.theta, want_lambda=want_lambda)
+    torch.cuda.synchronize()
+    return {k: (None if v is None else v.float().cpu().numpy()) for k, v in r.items()}
+
+
+def oracle_inputs(x):
+    return {k: v for k, v in x.items() if k != "d_o"}
+
+
+def test_tiny_fp32_full_parity_and_bruteforce_lambda():
+    w = I.WORKLOADS["tiny_fp32"]
+    x = I.make_prefill_inputs(w)
+    g = run_gpu(w, x, want_lambda=True)
+    r = oracle.prefill_fwd(**oracle_inputs(x), scale=w.scale, theta=w.theta, want_lambda=True)
+    lb = oracle.lambda_bruteforce(x["k"], x["a_q"], x["a_k"], x["alpha"], x["beta"])
+    assert_close("o", g["o"], r["o"], "f32")
+    assert_close("lse", g["lse"], r["lse"], "f32")
+    assert_close("b_final", g["b_final"], r["b_final"], "f32")
+    assert_close("lambda vs brute force", g["lam"], lb, "f32")
+
+
+SMALL = [
+    # (B, T, H, Hkv, d, dtype)
+    (2, 1, 4, 2, 64, "bf16"),
+    (2, 63, 4, 2, 64, "bf16"),
+    (2, 65, 4, 1, 64, "bf16"),
+    (1, 200, 8, 2, 64, "bf16"),
+    (2, 333, 4, 4, 64, "bf16"),
+    (1, 300, 6, 2, 128, "bf16"),
+    (1, 257, 8, 1, 128, "bf16"),
+    (1, 130, 2, 2, 64, "f32"),
+    (1, 190, 6, 2, 128, "f32"),
+]
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,d,dtype", SMALL)
+def test_small_shapes_full_parity(B, T, H, Hkv, d, dtype):
+    w = I.Workload("small", B, T, H, Hkv, d, dtype, 77 + T)
+    x = I.make_prefill_inputs(w)
+    g = run_gpu(w, x, want_lambda=True)
+    r = oracle.prefill_fwd(**oracle_inputs(x), scale=w.scale, theta=w.theta, want_lambda=True)
+    assert_close("o", g["o"], r["o"], dtype)
+    assert_close("lse", g["lse"], r["lse"], dtype, relative_max=True)
+    assert_close("b_final", g["b_final"], r["b_final"], dtype, relative_max=True)
+    tri = np.tril(np.ones((T, T), bool))
+    assert_close("lambda", g["lam"][..., tri], r["lam"][..., tri], dtype, relative_max=True)
+    assert np.all(g["lam"][..., ~tri] == 0.0)
+
+
+def test_veto_gives_plain_attention_and_zero_bias():
+    w = I.Workload("veto", 2, 150, 4, 2, 64, "bf16", 5)
+    x = I.make_prefill_inputs(w)
+    x["a_k"][:] = -1e4
+    g = run_gpu(w, x, want_lambda=True)
+    assert np.all(g["b_final"] == 0.0) and np.all(g["lam"] == 0.0)
+    r = oracle.prefill_fwd(**oracle_inputs(x), scale=w.scale, theta=w.theta)
+    assert_close("o", g["o"], r["o"], "bf16")
+
+
+def sampled_rows(T, n_rand=24, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = {0, 1, 63, 64, 127, 128, 129, T // 2, T - 129, T - 128, T - 65, T - 64, T - 1}
+    rows |= set(int(a) for a in rng.integers(0, T, n_rand))
+    return sorted(r for r in rows if 0 <= r < T)
+
+
+def check_sampled(w, units, seed):
+    x = I.make_prefill_inputs(w)
+    g = run_gpu(w, x)
+    T, Hkv, G = w.T, w.Hkv, w.G
+    rows = sampled_rows(T, seed=seed)
+    rm = np.zeros(T, np.uint8)
+    rm[rows] = 1
+    um = np.zeros(w.B * Hkv, np.uint8)
+    for b, h in units:
+        um[b * Hkv + h] = 1
+    r = oracle.prefill_fwd(**oracle_inputs(x), scale=w.scale, theta=w.theta, unit_mask=um, row_mask=rm)
+    for b, h in units:
+        hs = slice(h * G, (h + 1) * G)
+        assert_close(f"o[{b},{h}]", g["o"][b][rows][:, hs], r["o"][b][rows][:, hs], w.dtype)
+        assert_close(f"lse[{b},{h}]", g["lse"][b, hs][:, rows], r["lse"][b, hs][:, rows], w.dtype,
+                     relative_max=True)
+        assert_close(f"b_final[{b},{h}]", g["b_final"][b, h], r["b_final"][b, h], w.dtype, relative_max=True)
+    assert np.all(np.isfinite(g["o"]))
+    return g, r
+
+
+@pytest.mark.slow
+def test_prefill_1b_full_size_sampled():
+    w = I.WORKLOADS["prefill_1b"]
+    check_sampled(w, [(0, 0), (3, 5), (7, 7)], seed=1)
+
+
+@pytest.mark.slow
+def test_prefill_1b_16k_full_size_sampled():
+    w = I.WORKLOADS["prefill_1b_16k"]
+    check_sampled(w, [(0, 0), (0, 7)], seed=2)
