@@ -1,0 +1,435 @@
+"""Benchmark of the Universal Attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one UA prefill forward (token preparation, decay boundary pass, fused biased
+attention) over the 1B-shaped workload B=8, T=4096, H=32, Hkv=8, d=64 in bf16, inputs
+resident in HBM (they total ~335 MB, larger than the 126 MB L2, so no flush is needed).
+`value` is whole-job algorithmic TFLOP/s, F = B*T(T+1)/2*(H*4d + Hkv*2d) per step and GPU.
+The line also carries the decode workload (B=32, 16k prefill, 256 steps at p=0.15 and 0.05,
+tokens/s and HBM GB/s), the roofline of the dominant kernel, an end-to-end number through
+the public API with host buffers, and the fp64 oracle timed on the host cores.
+
+Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no collective on the
+data path); time is the max over ranks.  --impl reference times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_compression_ua_b200 import inputs as I  # noqa: E402
+
+METRIC = "UA prefill TFLOP/s & decode tok/s; % of BF16 TC peak / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def fwd_flops(w) -> float:
+    """Algorithmic forward FLOPs, counted once: per causal (i, j) pair and batch, H*4d for
+    QK^T and PV of every query head plus Hkv*2d for the key-key similarity."""
+    return w.B * w.T * (w.T + 1) / 2 * (w.H * 4 * w.d + w.Hkv * 2 * w.d)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during a region."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+
+def oracle_sample(w, n_units: int, nthreads: int):
+    """Time the fp64 oracle on n_units (batch, KV-head) units of workload w at full T, all
+    rows and heads; returns (seconds, algorithmic FLOPs of the sample, description)."""
+    import oracle
+    b_needed = max(1, math.ceil(n_units / w.Hkv))
+    x = I.make_prefill_inputs(w, B=b_needed)
+    um = np.zeros(b_needed * w.Hkv, np.uint8)
+    um[:n_units] = 1
+    oracle._load()
+    t0 = time.perf_counter()
+    oracle.prefill_fwd(**{k: v for k, v in x.items() if k != "d_o"}, scale=w.scale, theta=w.theta,
+                       unit_mask=um, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    flops = n_units * w.T * (w.T + 1) / 2 * (w.G * 4 * w.d + 2 * w.d)
+    desc = (f"{n_units} of the {w.B * w.Hkv} (batch, KV-head) units of {w.name} at full T={w.T}, "
+            f"all rows and {w.G} query heads each, fp64, {nthreads} threads")
+    return dt, flops, desc
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = I.WORKLOADS[args.workload]
+    cores = os.cpu_count() or 1
+    n_units = cores
+    times = []
+    flops = None
+    desc = None
+    for it in range(args.warmup + args.steps):
+        dt, flops, desc = oracle_sample(w, n_units, cores)
+        if it >= args.warmup:
+            times.append(dt)
+    tot = sum(times)
+    val = flops * len(times) / tot / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w),
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": desc, "value": val,
+                             "unit": "TFLOP/s"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "Hkv": w.Hkv, "head_dim": w.d,
+            "dtype": w.dtype, "rope_theta": w.theta, "l2": "inputs (~335 MB) larger than the 126 MB L2, no flush",
+            "parallelism": "weak: one batch per GPU"}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def device_inputs(w, rank):
+    wr = w.resized(seed=w.seed + 7919 * rank)
+    return I.make_prefill_inputs_torch(wr, "cuda")
+
+
+def bench_prefill(args, world, rank, local, peaks, peaks_kind):
+    from kv_cache_compression_ua_b200 import ua
+    w = I.WORKLOADS[args.workload]
+    x = device_inputs(w, rank)
+    out = torch.empty_like(x["q"])
+    shape = ua.make_shape(x["q"], x["k"], w.scale, w.theta)
+    ws = ua.alloc_workspace(ua.prefill_workspace_size(shape), "cuda")
+    lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32, device="cuda")
+    bfin = torch.empty(w.B, w.Hkv, w.T, dtype=torch.float32, device="cuda")
+
+    def step():
+        ua.prefill_fwd(x["q"], x["k"], x["v"], x["g"], x["a_q"], x["a_k"], x["alpha"], x["beta"],
+                       scale=w.scale, theta=w.theta, out=out, ws=ws, want_lse=False, want_bfinal=False)
+
+    # lse / b_final are outputs of the same call; the timed step writes O only and one
+    # extra call checks the full-output path is also healthy
+    ua.prefill_fwd(x["q"], x["k"], x["v"], x["g"], x["a_q"], x["a_k"], x["alpha"], x["beta"],
+                   scale=w.scale, theta=w.theta, out=out, ws=ws)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ua.profile_reset()
+    ua.profile_enable(True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ua.profile_enable(False)
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world)
+    prof = ua.profile_read()
+    assert ua.get_device_status() == 0
+    F = fwd_flops(w)
+    value = F * world * args.steps / (ms_max * 1e-3) / 1e12
+
+    # dominant kernel roofline (algorithmic FLOPs per launch / measured launch duration)
+    top = max(prof.items(), key=lambda kv: kv[1][1])
+    name, (launches, tot_ms) = top
+    per_launch_ms = tot_ms / launches
+    peak_t = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    achieved = F / (per_launch_ms * 1e-3) / 1e12
+    roofline = {"kernel": name, "bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+                "frac": achieved / peak_t, "traffic": None,
+                "peak_source": f"{peaks_kind} bf16 burst (MEASURED_PEAKS.json)" if peaks_kind == "measured"
+                else "fallback 1590 TF/s", "per_launch_ms": per_launch_ms,
+                "share_of_step": tot_ms / sum(v[1] for v in prof.values())}
+    kernels = {k: {"launches": v[0], "total_ms": v[1], "ms_per_launch": v[1] / v[0]} for k, v in prof.items()}
+    gpu_launches = sum(v[0] for v in prof.values())
+    return w, x, value, ms_max / args.steps, roofline, kernels, gpu_launches, clk.summary(), step
+
+
+def bench_e2e(args, w, x):
+    """Public API with host buffers: pinned host inputs copied in, prefill, O copied out."""
+    from kv_cache_compression_ua_b200 import ua
+    host = {n: t.cpu().pin_memory() for n, t in x.items()}
+    dev = {n: torch.empty_like(t) for n, t in x.items()}
+    o_host = torch.empty(x["q"].shape, dtype=x["q"].dtype).pin_memory()
+    out = torch.empty_like(x["q"])
+    shape = ua.make_shape(x["q"], x["k"], w.scale, w.theta)
+    ws = ua.alloc_workspace(ua.prefill_workspace_size(shape), "cuda")
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def step():
+        for n in host:
+            dev[n].copy_(host[n], non_blocking=True)
+        ua.prefill_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["a_q"], dev["a_k"], dev["alpha"],
+                       dev["beta"], scale=w.scale, theta=w.theta, out=out, ws=ws, want_lse=False,
+                       want_bfinal=False)
+        o_host.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 10))
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    return {"value": fwd_flops(w) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n}
+
+
+def bench_decode(args, peaks, peaks_kind):
+    """Decode workload: B=32 caches prefilled (on the GPU) from a 16k-token draw, compacted at
+    p, then 256 single-token steps captured in one CUDA graph and replayed."""
+    from kv_cache_compression_ua_b200 import ua
+    w = I.WORKLOADS["decode_1b"]
+    steps = I.DECODE_STEPS
+    T0 = w.T
+    x = I.make_prefill_inputs_torch(w, "cuda", names=["k", "v", "a_q", "a_k", "alpha", "beta"])
+    q0 = torch.zeros(w.B, T0, w.H, w.d, dtype=torch.bfloat16, device="cuda")
+    r = ua.prefill_fwd(q0, x["k"], x["v"], q0, x["a_q"], x["a_k"], x["alpha"], x["beta"],
+                       scale=w.scale, theta=w.theta, want_lse=False)
+    del q0
+    bfinal = r["b_final"]
+    del r
+    torch.cuda.empty_cache()
+    toks = [I.make_decode_token(w, s) for s in range(steps)]
+    tok = {n: torch.from_numpy(np.stack([t[n] for t in toks])).to("cuda").to(
+        torch.bfloat16 if n in ("q", "k", "v", "g") else torch.float32).contiguous() for n in toks[0]}
+    res = {}
+    cap = T0 + steps + 1
+    entry_bytes = 3 * w.d * 2 + 12
+    for p in list(I.DECODE_THRESHOLDS) + [0.0]:
+        cache = ua.Cache.empty(w.B, w.Hkv, w.d, cap, torch.bfloat16)
+        ua.cache_fill(cache, x["k"], x["v"], x["a_k"], bfinal, theta=w.theta)
+        ua.cache_compact(cache, p)
+        snap = {n: getattr(cache, n).clone() for n in ("khat", "krope", "v", "bias", "rk", "pos", "n_kept")}
+        n0 = cache.n_kept.clone()
+        o = torch.empty(steps, w.B, w.H, w.d, dtype=torch.bfloat16, device="cuda")
+
+        def restore():
+            for n, t in snap.items():
+                getattr(cache, n).copy_(t)
+
+        def run_all(stream=None):
+            for s in range(steps):
+                ua.decode_step(cache, tok["q"][s], tok["k"][s], tok["v"][s], tok["g"][s], tok["a_q"][s],
+                               tok["a_k"][s], x["alpha"], x["beta"], T0 + s, p, scale=w.scale, theta=w.theta,
+                               out=o[s], stream=stream)
+
+        # kept counts per step (for the byte count): one eager pass
+        counts = [n0.sum().item()]
+        for s in range(steps):
+            ua.decode_step(cache, tok["q"][s], tok["k"][s], tok["v"][s], tok["g"][s], tok["a_q"][s],
+                           tok["a_k"][s], x["alpha"], x["beta"], T0 + s, p, scale=w.scale, theta=w.theta,
+                           out=o[s])
+            counts.append(cache.n_kept.sum().item())
+        assert ua.get_device_status() == 0
+        final_kept = counts[-1]
+        restore()
+        g = torch.cuda.CUDAGraph()
+        s_cap = torch.cuda.Stream()
+        s_cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s_cap):
+            run_all(s_cap)           # warm-up on the capture stream
+        torch.cuda.current_stream().wait_stream(s_cap)
+        torch.cuda.synchronize()
+        restore()
+        with torch.cuda.graph(g, stream=s_cap):
+            run_all(s_cap)
+        times = []
+        for it in range(3 + 5):
+            restore()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            if it >= 3:
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        # algorithmic bytes: every live entry read once per step (khat, krope, v, bias, rk,
+        # pos), its bias written back, the appended token written, and the token's q/k/v/g/o
+        tok_bytes = w.B * (3 * w.H * w.d * 2 + 2 * w.Hkv * w.d * 2 + 2 * w.Hkv * 4)
+        bytes_total = sum(counts[s] * entry_bytes + counts[s + 1] * 4 + w.B * w.Hkv * entry_bytes + tok_bytes
+                          for s in range(steps))
+        gbs = bytes_total / (ms * 1e-3) / 1e9
+        retained = final_kept / (w.B * w.Hkv * (T0 + steps))
+        key = f"p={p:g}" if p > 0 else "p=0 (no eviction, supplementary)"
+        res[key] = {"tokens_per_s": w.B * steps / (ms * 1e-3), "ms_per_256_steps": ms,
+                    "us_per_step": 1e3 * ms / steps, "hbm_gbs": gbs,
+                    "hbm_frac": gbs / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+                    "retained_fraction": retained, "kept_entries_after": final_kept,
+                    "mean_kept_per_head": float(np.mean(counts)) / (w.B * w.Hkv),
+                    "cache_MB_after": final_kept * entry_bytes / 1e6,
+                    "compression_x": 1.0 / retained if retained > 0 else None}
+        del g, cache, snap
+        torch.cuda.empty_cache()
+    res["peak_source"] = f"{peaks_kind} HBM copy bandwidth"
+    res["workload"] = f"decode_1b: B={w.B}, 16k prefill, {steps} steps, graph-captured"
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_1b")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup() if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    from kv_cache_compression_ua_b200 import build as ua_build
+    if rank == 0 and not os.path.exists(os.path.join(ROOT, "kv_cache_compression_ua_b200", "libua.so")):
+        ua_build.build()
+    barrier(world)
+    peaks, peaks_kind = load_peaks()
+    w, x, value, ms_step, roofline, kernels, launches, clocks, _ = bench_prefill(
+        args, world, rank, local, peaks, peaks_kind)
+    e2e = bench_e2e(args, w, x)
+    del x
+    torch.cuda.empty_cache()
+    decode = None
+    if not args.no_decode and world == 1:
+        decode = bench_decode(args, peaks, peaks_kind)
+    cpu = None
+    if not args.no_cpu and rank == 0 and world == 1:
+        cores = os.cpu_count() or 1
+        dt, fl, desc = oracle_sample(w, cores, cores)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": workload_config(w), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clocks, "kernels": kernels, "decode": decode}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -56,7 +56,9 @@ typedef enum {
     UA_ERR_WORKSPACE = 4,     /* workspace smaller than the size query returned */
     UA_ERR_CAPACITY = 5,      /* a cache would exceed its capacity (device status bit) */
     UA_ERR_CUDA = 6,          /* a CUDA runtime call failed (launch error, ...) */
-    UA_ERR_TIMEOUT = 7        /* a bounded device-side wait gave up (device status bit) */
+    UA_ERR_TIMEOUT = 7,       /* a bounded device-side wait gave up (device status bit) */
+    UA_ERR_RANGE = 8          /* a softmax row normaliser under- or overflowed on the bf16
+                                 tensor-core path (device status bit; see ua_prefill_fwd) */
 } ua_status;
 
 typedef enum { UA_F32 = 0, UA_BF16 = 1 } ua_dtype;
@@ -88,7 +90,15 @@ ua_status ua_prefill_workspace_size(const ua_shape* shape, size_t* bytes);
  *          lambda_dbg [B,Hkv,T,T] f32 full Lambda, zero above the diagonal (or NULL;
  *          allowed only for T <= 1024).
  * ws / ws_bytes: device workspace of at least ua_prefill_workspace_size bytes; its
- * contents are scratch (overwritten). */
+ * contents are scratch (overwritten).
+ *
+ * Paths: bf16 problems with d = 64 and H/Hkv <= 4 run on the tensor cores (tcgen05/TMEM/
+ * TMA).  That path shifts every softmax row by the a-priori bound scale*||q_i|| (the keys
+ * are unit vectors and Lambda <= 0, so no logit exceeds it) instead of a running maximum; a
+ * row whose true maximum lies more than ~87 below that bound (scale*||q_i|| > ~43) would
+ * underflow, and then UA_ERR_RANGE is raised in the device status word.  All other problems,
+ * and every call that asks for lambda_dbg, run the fp32 SIMT path, which uses a running
+ * maximum. */
 ua_status ua_prefill_fwd(const ua_shape* shape, const void* q, const void* k, const void* v,
                          const void* g, const float* a_q, const float* a_k, const float* alpha,
                          const float* beta, void* o, float* lse, float* b_final, float* lambda_dbg,
@@ -173,6 +183,23 @@ ua_status ua_decode_step(const ua_cache* cache, int H, const void* q, const void
  * Synchronises `stream`, returns the device status word accumulated since the last call
  * (0 = no error, else a ua_status code) in *code, and clears it. */
 ua_status ua_get_device_status(void* stream, int* code);
+
+/* ------------------------------------------------------------------ kernel timing
+ * Optional tracing for measurement: while enabled, every libua kernel launch is bracketed
+ * by two CUDA events recorded on its stream (about a microsecond of overhead per launch; at
+ * most 8192 launches are recorded between resets).  ua_profile_read synchronises on the
+ * recorded events and returns, per kernel name, the number of launches and their summed
+ * duration in milliseconds; it returns UA_ERR_CAPACITY if launches were dropped.  `name`
+ * points to a static string owned by the library. */
+typedef struct {
+    const char* name;
+    int launches;
+    double total_ms;
+} ua_kernel_time;
+
+ua_status ua_profile_enable(int enable);
+ua_status ua_profile_reset(void);
+ua_status ua_profile_read(ua_kernel_time* out, int max_entries, int* n_entries);
 
 /* Static, human-readable name of a status code. */
 const char* ua_status_string(ua_status s);

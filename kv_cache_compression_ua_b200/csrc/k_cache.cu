@@ -13,6 +13,7 @@
 // (128-bit coalesced loads); dot products reduce across the group with shuffles.
 #include "ua_common.cuh"
 #include "ua_kernels.h"
+#include "ua_profile.h"
 
 namespace ua {
 
@@ -380,6 +381,7 @@ __global__ void __launch_bounds__(256) k_decode(DecodeParams p) {
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_cache_fill(const FillParams& p, bool bf16, cudaStream_t s) {
     dim3 grid(p.T, p.c.B);
+    UA_PROFILE("k_cache_fill", s);
     if (bf16) {
         if (p.c.d == 64) k_cache_fill<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
         else k_cache_fill<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
@@ -392,6 +394,7 @@ cudaError_t launch_cache_fill(const FillParams& p, bool bf16, cudaStream_t s) {
 
 cudaError_t launch_cache_compact(const CompactParams& p, bool bf16, cudaStream_t s) {
     dim3 grid(p.c.B * p.c.Hkv);
+    UA_PROFILE("k_cache_compact", s);
     if (bf16) {
         if (p.c.d == 64) k_cache_compact<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
         else k_cache_compact<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
@@ -411,6 +414,7 @@ static cudaError_t decode_inst(const DecodeParams& p, cudaStream_t s) {
         cudaError_t e = cudaFuncSetAttribute(k_decode<TC, DH, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
+    UA_PROFILE("k_decode", s);
     k_decode<TC, DH, G><<<p.c.B * p.c.Hkv, 256, smem, s>>>(p);
     return cudaGetLastError();
 }

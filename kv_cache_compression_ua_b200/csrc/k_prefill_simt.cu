@@ -11,6 +11,7 @@
 // in-tile triangular cumulative sum on top.
 #include "ua_common.cuh"
 #include "ua_kernels.h"
+#include "ua_profile.h"
 
 namespace ua {
 
@@ -42,6 +43,12 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p) {
             }
         }
         TW* dst_rot;
+        if (is_q && p.mq) {
+            float sq = ss;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            if (lane == 0) p.mq[((size_t)b * p.H + h) * p.Tp + t] = p.mq_scale * sqrtf(sq);
+        }
         if (!is_q) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -74,8 +81,14 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p) {
     for (int h = threadIdx.x; h < p.Hkv; h += blockDim.x) {
         const size_t src = ((size_t)b * T + t) * p.Hkv + h;
         const size_t dst = ((size_t)b * p.Hkv + h) * T + t;
-        p.rq[dst] = softplus_f(p.a_q[src]);
-        p.rk[dst] = softplus_f(p.a_k[src]);
+        const float sq = softplus_f(p.a_q[src]), sk = softplus_f(p.a_k[src]);
+        if (p.rq) p.rq[dst] = sq;
+        if (p.rk) p.rk[dst] = sk;
+        if (p.lq2) {
+            const size_t dp = ((size_t)b * p.Hkv + h) * p.Tp + t;
+            p.lq2[dp] = log2f(sq) * (1.f / 3.f);      // log2(0) = -inf keeps the veto
+            p.lk2[dp] = log2f(sk) * (1.f / 3.f);
+        }
     }
 }
 
@@ -305,6 +318,7 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_prep(const PrepParams& p, bool bf16_in, bool bf16_work, cudaStream_t s) {
     dim3 grid(p.T, p.B);
+    UA_PROFILE("k_prep", s);
     if (bf16_in && bf16_work) k_prep<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, s>>>(p);
     else if (bf16_in) k_prep<__nv_bfloat16, float><<<grid, 256, 0, s>>>(p);
     else if (bf16_work) k_prep<float, __nv_bfloat16><<<grid, 256, 0, s>>>(p);
@@ -314,6 +328,7 @@ cudaError_t launch_prep(const PrepParams& p, bool bf16_in, bool bf16_work, cudaS
 
 cudaError_t launch_boundary_simt(const BoundaryParams& p, cudaStream_t s) {
     dim3 grid((p.T + 127) / 128, p.Hkv, p.B);
+    UA_PROFILE("k_boundary_simt", s);
     if (p.d == 64) k_boundary_simt<64><<<grid, 128, 0, s>>>(p);
     else k_boundary_simt<128><<<grid, 128, 0, s>>>(p);
     return cudaGetLastError();
@@ -326,6 +341,7 @@ static cudaError_t fwd_simt_inst(const FwdParams& p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(k_fwd_simt<DH, TI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.nqt, p.H, p.B);
+    UA_PROFILE("k_fwd_simt", s);
     k_fwd_simt<DH, TI><<<grid, 256, smem, s>>>(p);
     return cudaGetLastError();
 }

@@ -34,7 +34,7 @@ ua_status check_shape(const ua_shape* s) {
     return UA_OK;
 }
 
-// Workspace of the prefill forward: f32 rotated/normalised copies, rates, prefixes.
+// Workspace of the SIMT prefill forward: f32 rotated/normalised copies, rates, prefixes.
 struct FwdWs {
     size_t qr, kh, kr, rq, rk, pb, total;
 };
@@ -53,6 +53,44 @@ FwdWs fwd_ws_layout(const ua_shape* s) {
     w.pb = take(B * Hkv * nqt * T * 4);
     w.total = off;
     return w;
+}
+
+// Workspace of the tensor-core prefill forward: bf16 rotated/normalised copies (TMA
+// sources), log2-rates and row bounds (rows padded to Tp), prefixes at 128-row query tiles.
+struct TcWs {
+    size_t qr, kh, kr, lq2, lk2, mq, pb, total;
+    int Tp, nqt;
+};
+
+TcWs tc_ws_layout(const ua_shape* s) {
+    const size_t B = s->B, T = s->T, H = s->H, Hkv = s->Hkv, d = s->d;
+    TcWs w;
+    w.Tp = (int)round_up(T, 4);
+    w.nqt = (int)((T + 127) / 128);
+    const size_t Tp = w.Tp;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = round_up(off + bytes, 1024); return o; };
+    w.qr = take(B * H * T * d * 2);
+    w.kh = take(B * Hkv * T * d * 2);
+    w.kr = take(B * Hkv * T * d * 2);
+    w.lq2 = take(B * Hkv * Tp * 4);
+    w.lk2 = take(B * Hkv * Tp * 4);
+    w.mq = take(B * H * Tp * 4);
+    w.pb = take(B * Hkv * (size_t)w.nqt * Tp * 4);
+    w.total = off;
+    return w;
+}
+
+bool use_tc(const ua_shape* s) { return s->dtype == UA_BF16 && fwd_tc_supported(s->d, s->H / s->Hkv); }
+
+size_t prefill_ws_bytes(const ua_shape* s) {
+    size_t n = fwd_ws_layout(s).total;
+    if (use_tc(s)) {
+        const size_t t = tc_ws_layout(s).total;
+        // the debug Lambda output (T <= 1024) runs the SIMT path, so small T reserve both
+        n = s->T <= 1024 ? (n > t ? n : t) : t;
+    }
+    return n;
 }
 
 ua_status cuda_status(cudaError_t e) { return e == cudaSuccess ? UA_OK : UA_ERR_CUDA; }
@@ -96,6 +134,7 @@ const char* ua_status_string(ua_status s) {
         case UA_ERR_CAPACITY: return "UA_ERR_CAPACITY";
         case UA_ERR_CUDA: return "UA_ERR_CUDA";
         case UA_ERR_TIMEOUT: return "UA_ERR_TIMEOUT";
+        case UA_ERR_RANGE: return "UA_ERR_RANGE";
     }
     return "UA_ERR_UNKNOWN";
 }
@@ -104,29 +143,20 @@ ua_status ua_prefill_workspace_size(const ua_shape* shape, size_t* bytes) {
     ua_status st = check_shape(shape);
     if (st != UA_OK) return st;
     if (!bytes) return UA_ERR_INVALID_ARG;
-    *bytes = fwd_ws_layout(shape).total;
+    *bytes = prefill_ws_bytes(shape);
     return UA_OK;
 }
 
-ua_status ua_prefill_fwd(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
-                         const float* a_q, const float* a_k, const float* alpha, const float* beta,
-                         void* o, float* lse, float* b_final, float* lambda_dbg, void* ws, size_t ws_bytes,
-                         void* stream) {
-    ua_status st = check_shape(s);
-    if (st != UA_OK) return st;
-    if (!q || !k || !v || !g || !a_q || !a_k || !alpha || !beta || !o || !ws) return UA_ERR_INVALID_ARG;
-    const void* ps[] = {q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, lambda_dbg};
-    for (const void* p : ps)
-        if (p && !aligned(p, 16)) return UA_ERR_ALIGNMENT;
-    if (!aligned(ws, 256)) return UA_ERR_ALIGNMENT;
-    if (lambda_dbg && s->T > 1024) return UA_ERR_INVALID_ARG;
+static ua_status prefill_fwd_simt(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
+                                  const float* a_q, const float* a_k, const float* alpha, const float* beta,
+                                  void* o, float* lse, float* b_final, float* lambda_dbg, void* ws,
+                                  cudaStream_t cs) {
+    ua_status st;
     const FwdWs w = fwd_ws_layout(s);
-    if (ws_bytes < w.total) return UA_ERR_WORKSPACE;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const bool bf = s->dtype == UA_BF16;
     const int nqt = (s->T + kBq - 1) / kBq;
-
     PrepParams pp;
+    memset(&pp, 0, sizeof(pp));
     pp.B = s->B; pp.T = s->T; pp.H = s->H; pp.Hkv = s->Hkv; pp.d = s->d; pp.theta = s->rope_theta;
     pp.q = q; pp.k = k; pp.a_q = a_q; pp.a_k = a_k;
     pp.qr = at(ws, w.qr); pp.kh = at(ws, w.kh); pp.kr = at(ws, w.kr);
@@ -152,6 +182,54 @@ ua_status ua_prefill_fwd(const ua_shape* s, const void* q, const void* k, const 
     fp.v = v; fp.g = g; fp.rq = pp.rq; fp.rk = pp.rk; fp.alpha = alpha; fp.beta = beta; fp.pb = bp.pb;
     fp.o = o; fp.lse = lse; fp.lambda_dbg = lambda_dbg;
     return cuda_status(launch_fwd_simt(fp, bf, cs));
+}
+
+static ua_status prefill_fwd_tc(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
+                                const float* a_q, const float* a_k, const float* alpha, const float* beta,
+                                void* o, float* lse, float* b_final, void* ws, cudaStream_t cs) {
+    ua_status st;
+    const TcWs w = tc_ws_layout(s);
+    PrepParams pp;
+    memset(&pp, 0, sizeof(pp));
+    pp.B = s->B; pp.T = s->T; pp.H = s->H; pp.Hkv = s->Hkv; pp.d = s->d; pp.theta = s->rope_theta;
+    pp.q = q; pp.k = k; pp.a_q = a_q; pp.a_k = a_k;
+    pp.qr = at(ws, w.qr); pp.kh = at(ws, w.kh); pp.kr = at(ws, w.kr);
+    pp.rq = nullptr; pp.rk = nullptr;
+    pp.Tp = w.Tp; pp.mq_scale = s->scale * 1.4426950408889634f;
+    pp.lq2 = reinterpret_cast<float*>(at(ws, w.lq2)); pp.lk2 = reinterpret_cast<float*>(at(ws, w.lk2));
+    pp.mq = reinterpret_cast<float*>(at(ws, w.mq));
+    if ((st = cuda_status(launch_prep(pp, true, true, cs))) != UA_OK) return st;
+
+    BoundaryParams bp;
+    memset(&bp, 0, sizeof(bp));
+    bp.B = s->B; bp.T = s->T; bp.Hkv = s->Hkv; bp.d = s->d; bp.bq = 128; bp.nqt = w.nqt;
+    bp.alpha = alpha; bp.beta = beta;
+    bp.pb = reinterpret_cast<float*>(at(ws, w.pb)); bp.bfinal = b_final;
+    if ((st = cuda_status(launch_boundary_tc(bp, pp.kh, pp.lq2, pp.lk2, w.Tp, cs))) != UA_OK) return st;
+
+    FwdTcLaunch L;
+    L.B = s->B; L.T = s->T; L.Tp = w.Tp; L.H = s->H; L.Hkv = s->Hkv; L.nqt = w.nqt; L.scale = s->scale;
+    L.kh = pp.kh; L.kr = pp.kr; L.qr = pp.qr; L.v = v; L.lq2 = pp.lq2; L.lk2 = pp.lk2; L.mq = pp.mq; L.pb = bp.pb;
+    L.alpha = alpha; L.beta = beta; L.g = g; L.o = o; L.lse = lse;
+    return cuda_status(launch_fwd_tc(L, cs));
+}
+
+ua_status ua_prefill_fwd(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
+                         const float* a_q, const float* a_k, const float* alpha, const float* beta,
+                         void* o, float* lse, float* b_final, float* lambda_dbg, void* ws, size_t ws_bytes,
+                         void* stream) {
+    ua_status st = check_shape(s);
+    if (st != UA_OK) return st;
+    if (!q || !k || !v || !g || !a_q || !a_k || !alpha || !beta || !o || !ws) return UA_ERR_INVALID_ARG;
+    const void* ps[] = {q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, lambda_dbg};
+    for (const void* p : ps)
+        if (p && !aligned(p, 16)) return UA_ERR_ALIGNMENT;
+    if (!aligned(ws, 256)) return UA_ERR_ALIGNMENT;
+    if (lambda_dbg && s->T > 1024) return UA_ERR_INVALID_ARG;
+    if (ws_bytes < prefill_ws_bytes(s)) return UA_ERR_WORKSPACE;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (use_tc(s) && !lambda_dbg) return prefill_fwd_tc(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, ws, cs);
+    return prefill_fwd_simt(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, lambda_dbg, ws, cs);
 }
 
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes) {

@@ -18,8 +18,14 @@ struct PrepParams {
     void* qr;           // [B,H,T,d] work type: RoPE(q)
     void* kh;           // [B,Hkv,T,d] work type: khat
     void* kr;           // [B,Hkv,T,d] work type: RoPE(khat)
-    float* rq;          // [B,Hkv,T] softplus(a_q)
-    float* rk;          // [B,Hkv,T] softplus(a_k)
+    float* rq;          // [B,Hkv,T] softplus(a_q), or NULL
+    float* rk;          // [B,Hkv,T] softplus(a_k), or NULL
+    // tensor-core path extras (NULL when unused); rows padded to Tp
+    int Tp;
+    float mq_scale;     // scale * log2(e)
+    float* lq2;         // [B*Hkv][Tp] log2(softplus(a_q)) / 3
+    float* lk2;         // [B*Hkv][Tp] log2(softplus(a_k)) / 3
+    float* mq;          // [B*H][Tp]  scale * ||q|| * log2(e): bound of every logit of the row
 };
 
 // Boundary pass: per-query-tile column prefixes of the decay and the final biases.
@@ -135,6 +141,29 @@ struct BwdParams {
     void* dq; void* dk; void* dv; void* dg;
     float* da_q; float* da_k; float* dalpha; float* dbeta;
 };
+
+struct FwdTcLaunch {
+    int B, T, Tp, H, Hkv, nqt;
+    float scale;
+    const void* kh;      // [B*Hkv][T][64] bf16 khat
+    const void* kr;      // [B*Hkv][T][64] bf16 RoPE(khat)
+    const void* qr;      // [B*H][T][64] bf16 RoPE(q)
+    const void* v;       // [B,T,Hkv,64] bf16 (caller's layout)
+    const float* lq2;
+    const float* lk2;
+    const float* mq;
+    const float* pb;     // [B*Hkv][nqt][Tp], query tiles of 128
+    const float* alpha;
+    const float* beta;
+    const void* g;
+    void* o;
+    float* lse;
+};
+
+bool fwd_tc_supported(int d, int G);
+cudaError_t launch_boundary_tc(const BoundaryParams& bp, const void* kh_bf16, const float* lq2, const float* lk2,
+                               int Tp, cudaStream_t s);
+cudaError_t launch_fwd_tc(const FwdTcLaunch& L, cudaStream_t s);
 
 cudaError_t launch_prep(const PrepParams& p, bool bf16_in, bool bf16_work, cudaStream_t s);
 cudaError_t launch_boundary_simt(const BoundaryParams& p, cudaStream_t s);

@@ -247,3 +247,104 @@ def make_decode_token(w: Workload, step: int, B: int | None = None) -> dict:
                 normal(s, S_AK, (w.B, w.Hkv), -2.0, 1.0, box=box)).astype(np.float32),
     }
     return {n: np.ascontiguousarray(x) for n, x in out.items()}
+
+
+# --------------------------------------------------------------------------- torch twin
+# The same counter-based draws evaluated with torch int64 ops (uint64 arithmetic emulated
+# by wrapping int64 multiply/add and masked right shifts), for large benchmark inputs made
+# directly on the device.  Integer stages are bit-identical to the numpy path; the fp64
+# Box-Muller stage may differ in the last ulp on a GPU, so parity tests use the numpy path.
+
+def _i64(c: int) -> int:
+    c &= 0xFFFFFFFFFFFFFFFF
+    return c - (1 << 64) if c >= (1 << 63) else c
+
+
+def _t_srl(x, s: int):
+    import torch
+    return (x >> s) & ((1 << (64 - s)) - 1)
+
+
+def _t_mix(z):
+    z = (z ^ _t_srl(z, 30)) * _i64(0xBF58476D1CE4E5B9)
+    z = (z ^ _t_srl(z, 27)) * _i64(0x94D049BB133111EB)
+    return z ^ _t_srl(z, 31)
+
+
+def _t_u53(bits):
+    import torch
+    return _t_srl(bits, 11).to(torch.float64) * (1.0 / 9007199254740992.0)
+
+
+def _t_lin(full_shape, lead_lo, lead_n, device):
+    import torch
+    idx = torch.zeros((), dtype=torch.int64, device=device)
+    for ax, size in enumerate(full_shape):
+        if ax < len(lead_n):
+            r = torch.arange(lead_lo[ax], lead_lo[ax] + lead_n[ax], dtype=torch.int64, device=device)
+        else:
+            r = torch.arange(size, dtype=torch.int64, device=device)
+        idx = idx[..., None] * size + r
+    return idx
+
+
+def _t_uniform(seed, stream, shape, lo, hi, box, device):
+    key = _i64(int(_stream_key(seed, stream)))
+    lead_lo, lead_n = box
+    lin = _t_lin(shape, lead_lo, lead_n, device)
+    return lo + (hi - lo) * _t_u53(_t_mix(key + (lin + 1) * _i64(0x9E3779B97F4A7C15)))
+
+
+def _t_normal(seed, stream, shape, mean, std, box, device):
+    import torch
+    key = _i64(int(_stream_key(seed, stream)))
+    lead_lo, lead_n = box
+    lin = _t_lin(shape, lead_lo, lead_n, device) * 2
+    g = _i64(0x9E3779B97F4A7C15)
+    u1 = 1.0 - _t_u53(_t_mix(key + (lin + 1) * g))
+    u2 = _t_u53(_t_mix(key + (lin + 2) * g))
+    return mean + std * torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * np.pi * u2)
+
+
+def make_prefill_inputs_torch(w: Workload, device, T: int | None = None, B: int | None = None,
+                              names=None, b0: int = 0) -> dict:
+    """make_prefill_inputs evaluated with torch on `device` (activations in bf16/f32, decay
+    logits f32).  For benchmark-size inputs; see the note above on the last fp64 ulp."""
+    import torch
+    Bf, Tf, H, Hkv, d = w.B, w.T, w.H, w.Hkv, w.d
+    B = Bf - b0 if B is None else B
+    T = Tf if T is None else T
+    names = [n for n in PREFILL_NAMES if (names is None or n in names)]
+    if not w.with_grad and "d_o" in names:
+        names.remove("d_o")
+    act = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    s = w.seed
+    out = {}
+    for n in names:
+        if n in ("alpha", "beta"):
+            x = make_prefill_inputs(w, names=[n])[n]
+            out[n] = torch.from_numpy(x).to(device)
+            continue
+        heads = H if n in ("q", "g", "d_o") else Hkv
+        full = (Bf, Tf, heads, d) if n in ("q", "k", "v", "g", "d_o") else (Bf, Tf, heads)
+        dt = act if len(full) == 4 else torch.float32
+        arr = torch.empty((B, T) + full[2:], dtype=dt, device=device)
+        step = max(1, (1 << 24) // max(1, int(np.prod(full[2:]))))
+        for bi in range(B):
+            for t0 in range(0, T, step):
+                nt = min(step, T - t0)
+                box = ((b0 + bi, t0), (1, nt))
+                if n in ("q", "k", "v", "g", "d_o"):
+                    stream = {"q": S_Q, "k": S_K, "v": S_V, "g": S_G, "d_o": S_DO}[n]
+                    x = _t_normal(s, stream, full, 0.0, 1.0, box, device)
+                elif n == "a_q":
+                    x = _t_normal(s, S_AQ, full, -2.0, 1.0, box, device)
+                elif w.bimodal_ak:
+                    sel = _t_uniform(s, S_AK_MODE, full, 0.0, 1.0, box, device) < 0.1
+                    x = torch.where(sel, _t_normal(s, S_AK_SLOW, full, -6.0, 0.5, box, device),
+                                    _t_normal(s, S_AK, full, -1.0, 0.5, box, device))
+                else:
+                    x = _t_normal(s, S_AK, full, -2.0, 1.0, box, device)
+                arr[bi, t0:t0 + nt] = x[0].to(torch.float32).to(dt)
+        out[n] = arr
+    return out

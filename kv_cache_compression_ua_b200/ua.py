@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_PKG, "libua.so")
 
 UA_F32, UA_BF16 = 0, 1
 STATUS = {0: "UA_OK", 1: "UA_ERR_INVALID_ARG", 2: "UA_ERR_UNSUPPORTED", 3: "UA_ERR_ALIGNMENT",
-          4: "UA_ERR_WORKSPACE", 5: "UA_ERR_CAPACITY", 6: "UA_ERR_CUDA", 7: "UA_ERR_TIMEOUT"}
+          4: "UA_ERR_WORKSPACE", 5: "UA_ERR_CAPACITY", 6: "UA_ERR_CUDA", 7: "UA_ERR_TIMEOUT",
+          8: "UA_ERR_RANGE"}
 
 
 class UAError(RuntimeError):
@@ -42,7 +43,11 @@ class ua_cache(ctypes.Structure):
 
 EXPORTS = ("ua_prefill_workspace_size", "ua_prefill_fwd", "ua_prefill_bwd_workspace_size", "ua_prefill_bwd",
            "ua_cache_fill", "ua_cache_compact", "ua_decode_step", "ua_get_device_status",
-           "ua_status_string", "ua_version")
+           "ua_profile_enable", "ua_profile_reset", "ua_profile_read", "ua_status_string", "ua_version")
+
+
+class ua_kernel_time(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int), ("total_ms", ctypes.c_double)]
 
 _lib = None
 
@@ -67,6 +72,9 @@ def load_library(path: str = LIB_PATH):
     lib.ua_cache_compact.argtypes = [CP, P, F, P, P]
     lib.ua_decode_step.argtypes = [CP, I] + [P] * 8 + [I, F, F, D, P, P, P, I, P]
     lib.ua_get_device_status.argtypes = [P, ctypes.POINTER(I)]
+    lib.ua_profile_enable.argtypes = [I]
+    lib.ua_profile_reset.argtypes = []
+    lib.ua_profile_read.argtypes = [ctypes.POINTER(ua_kernel_time), I, ctypes.POINTER(I)]
     lib.ua_status_string.argtypes = [I]
     lib.ua_status_string.restype = ctypes.c_char_p
     lib.ua_version.argtypes = []
@@ -244,6 +252,22 @@ def get_device_status(stream=None) -> int:
     code = ctypes.c_int(0)
     _check("ua_get_device_status", load_library().ua_get_device_status(_stream(stream), ctypes.byref(code)))
     return code.value
+
+
+def profile_enable(on: bool = True):
+    _check("ua_profile_enable", load_library().ua_profile_enable(1 if on else 0))
+
+
+def profile_reset():
+    _check("ua_profile_reset", load_library().ua_profile_reset())
+
+
+def profile_read() -> dict:
+    """{kernel name: (launches, total_ms)} for the launches recorded since the last reset."""
+    arr = (ua_kernel_time * 64)()
+    n = ctypes.c_int(0)
+    _check("ua_profile_read", load_library().ua_profile_read(arr, 64, ctypes.byref(n)))
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n.value)}
 
 
 def version() -> int:

@@ -77,6 +77,61 @@ def test_small_shapes_full_parity(B, T, H, Hkv, d, dtype):
     assert np.all(g["lam"][..., ~tri] == 0.0)
 
 
+TC_SHAPES = [
+    # (B, T, H, Hkv): bf16, d = 64 -> tensor-core path
+    (1, 1, 4, 1),
+    (2, 63, 4, 2),
+    (1, 128, 4, 1),
+    (2, 129, 8, 2),
+    (1, 200, 2, 2),
+    (1, 333, 6, 2),
+    (2, 517, 4, 4),
+    (1, 1000, 4, 1),
+]
+
+
+def kernels_ran(fn):
+    ua.profile_reset()
+    ua.profile_enable(True)
+    try:
+        out = fn()
+        torch.cuda.synchronize()
+    finally:
+        ua.profile_enable(False)
+    return out, set(ua.profile_read())
+
+
+@pytest.mark.parametrize("B,T,H,Hkv", TC_SHAPES)
+def test_tensor_core_path_full_parity(B, T, H, Hkv):
+    w = I.Workload("tc", B, T, H, Hkv, 64, "bf16", 500 + T + H)
+    x = I.make_prefill_inputs(w)
+    g, names = kernels_ran(lambda: run_gpu(w, x))
+    assert "k_fwd_tc" in names and "k_boundary_tc" in names, names
+    assert ua.get_device_status() == 0
+    r = oracle.prefill_fwd(**oracle_inputs(x), scale=w.scale, theta=w.theta)
+    assert_close("o", g["o"], r["o"], "bf16")
+    assert_close("lse", g["lse"], r["lse"], "bf16", relative_max=True)
+    assert_close("b_final", g["b_final"], r["b_final"], "bf16", relative_max=True)
+
+
+def test_tensor_core_path_veto_and_plain_attention():
+    w = I.Workload("tcveto", 1, 300, 4, 1, 64, "bf16", 17)
+    x = I.make_prefill_inputs(w)
+    x["a_q"][:] = -1e4
+    g, names = kernels_ran(lambda: run_gpu(w, x))
+    assert "k_fwd_tc" in names
+    assert np.all(g["b_final"] == 0.0)
+    r = oracle.prefill_fwd(**oracle_inputs(x), scale=w.scale, theta=w.theta)
+    assert_close("o", g["o"], r["o"], "bf16")
+
+
+def test_debug_lambda_runs_exact_path():
+    w = I.Workload("dbg", 1, 100, 4, 1, 64, "bf16", 18)
+    x = I.make_prefill_inputs(w)
+    _, names = kernels_ran(lambda: run_gpu(w, x, want_lambda=True))
+    assert "k_fwd_simt" in names and "k_fwd_tc" not in names
+
+
 def test_veto_gives_plain_attention_and_zero_bias():
     w = I.Workload("veto", 2, 150, 4, 2, 64, "bf16", 5)
     x = I.make_prefill_inputs(w)
@@ -118,10 +173,12 @@ def check_sampled(w, units, seed):
 @pytest.mark.slow
 def test_prefill_1b_full_size_sampled():
     w = I.WORKLOADS["prefill_1b"]
-    check_sampled(w, [(0, 0), (3, 5), (7, 7)], seed=1)
+    (_, _), names = kernels_ran(lambda: check_sampled(w, [(0, 0), (3, 5), (7, 7)], seed=1))
+    assert "k_fwd_tc" in names
 
 
 @pytest.mark.slow
 def test_prefill_1b_16k_full_size_sampled():
     w = I.WORKLOADS["prefill_1b_16k"]
-    check_sampled(w, [(0, 0), (0, 7)], seed=2)
+    (_, _), names = kernels_ran(lambda: check_sampled(w, [(0, 0), (0, 7)], seed=2))
+    assert "k_fwd_tc" in names
