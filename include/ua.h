@@ -104,6 +104,28 @@ ua_status ua_prefill_fwd(const ua_shape* shape, const void* q, const void* k, co
                          const float* beta, void* o, float* lse, float* b_final, float* lambda_dbg,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ allocation-free forward
+ * No counterpart on the pages: this is a deployment convenience of this library.
+ * Same computation and arguments as ua_prefill_fwd, minus lambda_dbg and the workspace.
+ * For callers that cannot allocate device memory (a plug-in inside a host application that
+ * owns the whole GPU memory pool, or a caller that cannot afford cudaMalloc's latency and
+ * synchronisation): the scratch lives in a fixed 32 MiB array inside the library, which
+ * every device that loads the library keeps until the process exits.
+ *   - Problems whose ua_prefill_workspace_size exceeds ua_prefill_noalloc_max_scratch()
+ *     (32 MiB; e.g. one 4096-token sequence of the 1B shape fits) return UA_ERR_WORKSPACE.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the one array: calls that overlap on the GPU (different streams,
+ *     without ordering between them) race on it and give undefined results.  Serialise them.
+ *   - Nothing is allocated or freed; no state carries over between calls (every byte of the
+ *     scratch a call reads was written earlier in the same call). */
+ua_status ua_prefill_fwd_noalloc(const ua_shape* shape, const void* q, const void* k, const void* v,
+                                 const void* g, const float* a_q, const float* a_k, const float* alpha,
+                                 const float* beta, void* o, float* lse, float* b_final, void* stream);
+
+/* Size in bytes of the array ua_prefill_fwd_noalloc uses (the largest workspace it serves). */
+size_t ua_prefill_noalloc_max_scratch(void);
+
 /* ------------------------------------------------------------------ prefill backward
  * Gradient of sum(dO * O) with respect to every input of ua_prefill_fwd (the backward of
  * the custom training kernels, §4.2 and App. H; the decay is recomputed, not stored,

@@ -3,6 +3,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "ua_common.cuh"
 #include "ua_kernels.h"
 
@@ -231,6 +233,58 @@ ua_status ua_prefill_fwd(const ua_shape* s, const void* q, const void* k, const 
     if (use_tc(s) && !lambda_dbg) return prefill_fwd_tc(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, ws, cs);
     return prefill_fwd_simt(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, lambda_dbg, ws, cs);
 }
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free prefill forward.  Some callers cannot allocate device memory at all: a
+// plug-in whose host application (an inference server, a game engine) has already carved
+// the whole GPU into its own memory pool and forbids further cudaMalloc calls, or a caller
+// that must not pay cudaMalloc's latency and device-wide synchronisation.  Such callers use
+// ua_prefill_fwd_noalloc, whose scratch is this fixed file-scope device array instead of a
+// caller workspace.  Every device that loads the library holds the array until exit.
+namespace {
+constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;   // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device, resolved once per device.  The array's
+// host-side symbol is only a handle and must never be handed to a kernel.
+ua_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return UA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return UA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return UA_OK;
+}
+}  // namespace
+
+ua_status ua_prefill_fwd_noalloc(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
+                                 const float* a_q, const float* a_k, const float* alpha, const float* beta,
+                                 void* o, float* lse, float* b_final, void* stream) {
+    ua_status st = check_shape(s);
+    if (st != UA_OK) return st;
+    if (!q || !k || !v || !g || !a_q || !a_k || !alpha || !beta || !o) return UA_ERR_INVALID_ARG;
+    const void* ps[] = {q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final};
+    for (const void* p : ps)
+        if (p && !aligned(p, 16)) return UA_ERR_ALIGNMENT;
+    if (prefill_ws_bytes(s) > kNoAllocScratchBytes) return UA_ERR_WORKSPACE;
+    void* ws = nullptr;
+    if ((st = noalloc_scratch(&ws)) != UA_OK) return st;
+    // Every part of the scratch is written before it is read within a call, so nothing has
+    // to be cleared between calls.
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (use_tc(s)) return prefill_fwd_tc(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, ws, cs);
+    return prefill_fwd_simt(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, nullptr, ws, cs);
+}
+
+size_t ua_prefill_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
 
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes) {
     ua_status st = check_shape(shape);

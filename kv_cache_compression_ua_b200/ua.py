@@ -43,7 +43,8 @@ class ua_cache(ctypes.Structure):
 
 EXPORTS = ("ua_prefill_workspace_size", "ua_prefill_fwd", "ua_prefill_bwd_workspace_size", "ua_prefill_bwd",
            "ua_cache_fill", "ua_cache_compact", "ua_decode_step", "ua_get_device_status",
-           "ua_profile_enable", "ua_profile_reset", "ua_profile_read", "ua_status_string", "ua_version")
+           "ua_profile_enable", "ua_profile_reset", "ua_profile_read", "ua_status_string", "ua_version",
+           "ua_prefill_fwd_noalloc", "ua_prefill_noalloc_max_scratch")
 
 
 class ua_kernel_time(ctypes.Structure):
@@ -75,11 +76,14 @@ def load_library(path: str = LIB_PATH):
     lib.ua_profile_enable.argtypes = [I]
     lib.ua_profile_reset.argtypes = []
     lib.ua_profile_read.argtypes = [ctypes.POINTER(ua_kernel_time), I, ctypes.POINTER(I)]
+    lib.ua_prefill_fwd_noalloc.argtypes = [SP] + [P] * 8 + [P, P, P, P]
+    lib.ua_prefill_noalloc_max_scratch.argtypes = []
+    lib.ua_prefill_noalloc_max_scratch.restype = S
     lib.ua_status_string.argtypes = [I]
     lib.ua_status_string.restype = ctypes.c_char_p
     lib.ua_version.argtypes = []
     for n in EXPORTS:
-        if n not in ("ua_status_string", "ua_version"):
+        if n not in ("ua_status_string", "ua_version", "ua_prefill_noalloc_max_scratch"):
             getattr(lib, n).restype = I
     if path == LIB_PATH:
         _lib = lib
@@ -152,6 +156,25 @@ def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0
                             _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(stream))
     _check("ua_prefill_fwd", rc)
     return {"o": o, "lse": lse, "b_final": bfin, "lam": lam}
+
+
+def prefill_fwd_noalloc(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0, want_lse=True,
+                        want_bfinal=True, out=None, stream=None):
+    """ua_prefill_fwd_noalloc: the prefill forward using the library's fixed internal scratch
+    instead of a workspace (for callers that cannot allocate device memory)."""
+    lib = load_library()
+    shape = make_shape(q, k, scale, theta)
+    B, T, H, d = q.shape
+    Hkv = k.shape[2]
+    dev = q.device
+    o = out if out is not None else torch.empty_like(q)
+    lse = torch.empty(B, H, T, dtype=torch.float32, device=dev) if want_lse else None
+    bfin = torch.empty(B, Hkv, T, dtype=torch.float32, device=dev) if want_bfinal else None
+    rc = lib.ua_prefill_fwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q),
+                                    _ptr(a_k), _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(bfin),
+                                    _stream(stream))
+    _check("ua_prefill_fwd_noalloc", rc)
+    return {"o": o, "lse": lse, "b_final": bfin}
 
 
 def prefill_bwd_workspace_size(shape: ua_shape) -> int:
