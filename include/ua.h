@@ -129,9 +129,11 @@ size_t ua_prefill_noalloc_max_scratch(void);
 /* ------------------------------------------------------------------ prefill backward
  * Gradient of sum(dO * O) with respect to every input of ua_prefill_fwd (the backward of
  * the custom training kernels, §4.2 and App. H; the decay is recomputed, not stored,
- * App. C).  Needs the forward's o, lse and b_final.
+ * App. C).  Needs the forward's o and lse (natural-log row normalisers); b_final may be NULL
+ * and is not read (the decay prefixes are recomputed).  d_o: [B,T,H,d] act.
  * Outputs: dq, dg [B,T,H,d] act; dk, dv [B,T,Hkv,d] act; da_q, da_k [B,T,Hkv] f32;
- * dalpha, dbeta [Hkv] f32 (summed over the batch).  All outputs are overwritten. */
+ * dalpha, dbeta [Hkv] f32 (summed over the batch).  All outputs are overwritten; the result
+ * is deterministic (no atomics).  Runs as fp32 SIMT kernels. */
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes);
 
 ua_status ua_prefill_bwd(const ua_shape* shape, const void* q, const void* k, const void* v,

@@ -286,21 +286,90 @@ ua_status ua_prefill_fwd_noalloc(const ua_shape* s, const void* q, const void* k
 
 size_t ua_prefill_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
 
+// Workspace of the backward: the f32 token preparation and decay prefixes of the SIMT
+// forward, then f32 gradient intermediates.
+struct BwdWs {
+    FwdWs f;
+    size_t delta, dpb, dqr, dkh, dkh_rows, dkr, dv32, daq, dak, dab, total;
+    int nqt, nkt;
+};
+
+BwdWs bwd_ws_layout(const ua_shape* s) {
+    BwdWs w;
+    w.f = fwd_ws_layout(s);
+    const size_t B = s->B, T = s->T, H = s->H, Hkv = s->Hkv, d = s->d;
+    w.nqt = (int)((T + kBq - 1) / kBq);
+    w.nkt = (int)((T + 31) / 32);
+    size_t off = w.f.total;
+    auto take = [&](size_t bytes) { size_t o = off; off = round_up(off + bytes, 256); return o; };
+    w.delta = take(B * H * T * 4);
+    w.dpb = take(B * Hkv * (size_t)w.nqt * T * 4);
+    w.dqr = take(B * H * T * d * 4);
+    w.dkh = take(B * Hkv * T * d * 4);
+    w.dkh_rows = take(B * Hkv * T * d * 4);
+    w.dkr = take(B * Hkv * T * d * 4);
+    w.dv32 = take(B * Hkv * T * d * 4);
+    w.daq = take(B * Hkv * T * 4);
+    w.dak = take(B * Hkv * T * 4);
+    w.dab = take(B * Hkv * (size_t)w.nkt * 2 * 4);
+    w.total = off;
+    return w;
+}
+
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes) {
     ua_status st = check_shape(shape);
     if (st != UA_OK) return st;
     if (!bytes) return UA_ERR_INVALID_ARG;
-    *bytes = 0;
-    return UA_ERR_UNSUPPORTED;
+    *bytes = bwd_ws_layout(shape).total;
+    return UA_OK;
 }
 
-ua_status ua_prefill_bwd(const ua_shape* s, const void*, const void*, const void*, const void*, const float*,
-                         const float*, const float*, const float*, const void*, const float*, const float*,
-                         const void*, void*, void*, void*, void*, float*, float*, float*, float*, void*, size_t,
-                         void*) {
+ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
+                         const float* a_q, const float* a_k, const float* alpha, const float* beta, const void* o,
+                         const float* lse, const float* b_final, const void* d_o, void* dq, void* dk, void* dv,
+                         void* dg, float* da_q, float* da_k, float* dalpha, float* dbeta, void* ws, size_t ws_bytes,
+                         void* stream) {
     ua_status st = check_shape(s);
     if (st != UA_OK) return st;
-    return UA_ERR_UNSUPPORTED;
+    (void)b_final;   // the backward recomputes the decay prefixes; b_final is not read
+    const void* need[] = {q, k, v, g, a_q, a_k, alpha, beta, o, lse, d_o, dq, dk, dv, dg, da_q, da_k, dalpha, dbeta, ws};
+    for (const void* p : need)
+        if (!p) return UA_ERR_INVALID_ARG;
+    for (const void* p : need)
+        if (!aligned(p, 16)) return UA_ERR_ALIGNMENT;
+    if (!aligned(ws, 256)) return UA_ERR_ALIGNMENT;
+    const BwdWs w = bwd_ws_layout(s);
+    if (ws_bytes < w.total) return UA_ERR_WORKSPACE;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const bool bf = s->dtype == UA_BF16;
+
+    PrepParams pp;
+    memset(&pp, 0, sizeof(pp));
+    pp.B = s->B; pp.T = s->T; pp.H = s->H; pp.Hkv = s->Hkv; pp.d = s->d; pp.theta = s->rope_theta;
+    pp.q = q; pp.k = k; pp.a_q = a_q; pp.a_k = a_k;
+    pp.qr = at(ws, w.f.qr); pp.kh = at(ws, w.f.kh); pp.kr = at(ws, w.f.kr);
+    pp.rq = reinterpret_cast<float*>(at(ws, w.f.rq)); pp.rk = reinterpret_cast<float*>(at(ws, w.f.rk));
+    if ((st = cuda_status(launch_prep(pp, bf, false, cs))) != UA_OK) return st;
+    BoundaryParams bp;
+    bp.B = s->B; bp.T = s->T; bp.Hkv = s->Hkv; bp.d = s->d; bp.bq = kBq; bp.nqt = w.nqt;
+    bp.kh = reinterpret_cast<const float*>(pp.kh); bp.rq = pp.rq; bp.rk = pp.rk; bp.alpha = alpha; bp.beta = beta;
+    bp.pb = reinterpret_cast<float*>(at(ws, w.f.pb)); bp.bfinal = nullptr;
+    if ((st = cuda_status(launch_boundary_simt(bp, cs))) != UA_OK) return st;
+
+    BwdParams p;
+    p.B = s->B; p.T = s->T; p.H = s->H; p.Hkv = s->Hkv; p.d = s->d; p.G = s->H / s->Hkv; p.nqt = w.nqt; p.nkt = w.nkt;
+    p.scale = s->scale; p.theta = s->rope_theta;
+    p.qr = reinterpret_cast<const float*>(pp.qr); p.kh = reinterpret_cast<const float*>(pp.kh);
+    p.kr = reinterpret_cast<const float*>(pp.kr); p.rq = pp.rq; p.rk = pp.rk; p.pb = bp.pb;
+    p.k = k; p.v = v; p.g = g; p.o = o; p.d_o = d_o; p.a_q = a_q; p.a_k = a_k; p.alpha = alpha; p.beta = beta;
+    p.lse = lse;
+    p.delta = reinterpret_cast<float*>(at(ws, w.delta)); p.dpb = reinterpret_cast<float*>(at(ws, w.dpb));
+    p.dqr = reinterpret_cast<float*>(at(ws, w.dqr)); p.dkh = reinterpret_cast<float*>(at(ws, w.dkh));
+    p.dkh_rows = reinterpret_cast<float*>(at(ws, w.dkh_rows)); p.dkr = reinterpret_cast<float*>(at(ws, w.dkr));
+    p.dv32 = reinterpret_cast<float*>(at(ws, w.dv32)); p.daq32 = reinterpret_cast<float*>(at(ws, w.daq));
+    p.dak32 = reinterpret_cast<float*>(at(ws, w.dak)); p.dab = reinterpret_cast<float*>(at(ws, w.dab));
+    p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.da_q = da_q; p.da_k = da_k; p.dalpha = dalpha; p.dbeta = dbeta;
+    return cuda_status(launch_bwd_simt(p, bf, cs));
 }
 
 ua_status ua_cache_fill(const ua_cache* c, int T, const void* k, const void* v, const float* a_k,

@@ -107,37 +107,38 @@ struct DecodeParams {
     int32_t* kept_idx;
 };
 
-// Backward (SIMT path).
+// Backward (SIMT path).  Inputs from the f32 token preparation and boundary pass (query
+// tiles of 64 rows); f32 intermediates in the workspace; outputs in the caller's layouts.
 struct BwdParams {
-    int B, T, H, Hkv, d, G, nqt;
+    int B, T, H, Hkv, d, G, nqt, nkt;
     float scale;
+    double theta;
     const float* qr;     // [B,H,T,d]  RoPE(q)
-    const float* kh;     // [B,Hkv,T,d]
-    const float* kr;     // [B,Hkv,T,d]
-    const void* v;       // [B,T,Hkv,d] act
-    const void* g;       // [B,T,H,d] act
-    const void* o;       // [B,T,H,d] act
-    const void* d_o;     // [B,T,H,d] act
-    const float* a_q;    // [B,T,Hkv]
-    const float* a_k;    // [B,T,Hkv]
+    const float* kh;     // [B,Hkv,T,d] khat
+    const float* kr;     // [B,Hkv,T,d] RoPE(khat)
     const float* rq;     // [B,Hkv,T]
     const float* rk;     // [B,Hkv,T]
+    const float* pb;     // [B,Hkv,nqt,T] decay prefixes
+    const void* k;       // [B,T,Hkv,d] act (raw keys, for the normalisation Jacobian)
+    const void* v;
+    const void* g;
+    const void* o;
+    const void* d_o;
+    const float* a_q;
+    const float* a_k;
     const float* alpha;
     const float* beta;
     const float* lse;    // [B,H,T]
-    const float* bfinal; // [B,Hkv,T]
-    float* delta;        // [B,H,T] rowwise dO.O
-    float* dqr;          // [B,H,T,d] f32 accum of dL/dRoPE(q)
-    float* dkh;          // [B,Hkv,T,d] f32 accum of dL/dkhat (similarity path + RoPE^T dkr)
-    float* dkr;          // [B,Hkv,T,d] f32 dL/dRoPE(khat)
-    float* dv32;         // [B,Hkv,T,d] f32 dL/dv
-    float* daq32;        // [B,Hkv,T] f32 accum (over key tiles)
-    float* dak32;        // [B,Hkv,T] f32
-    float* dab;          // [B*Hkv*nkt][2] per-CTA partial (dalpha, dbeta)
-    int nkt;
-    // outputs
-    double theta;
-    const void* k;       // raw keys for the normalisation Jacobian
+    float* delta;        // [B,H,T]
+    float* dpb;          // [B,Hkv,nqt,T] suffix sums of dLambda per query tile
+    float* dqr;          // [B,H,T,d]
+    float* dkh;          // [B,Hkv,T,d] key-side similarity gradient
+    float* dkh_rows;     // [B,Hkv,T,d] row-side similarity gradient
+    float* dkr;          // [B,Hkv,T,d]
+    float* dv32;         // [B,Hkv,T,d]
+    float* daq32;        // [B,Hkv,T]
+    float* dak32;        // [B,Hkv,T]
+    float* dab;          // [B*Hkv*nkt][2]
     void* dq; void* dk; void* dv; void* dg;
     float* da_q; float* da_k; float* dalpha; float* dbeta;
 };

@@ -17,7 +17,10 @@ def rel_l2(got, ref):
     return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
 
 
-def assert_close(name, got, ref, dtype, relative_max=False):
+def assert_close(name, got, ref, dtype, relative_max=False, tensor_scale=False):
+    """relative_max: log-domain outputs, errors measured against max(1, |ref|) elementwise.
+    tensor_scale: gradients, whose max error is measured against max(1, max |ref|) of the
+    whole tensor (a bf16 output carries ~2^-9 relative rounding whatever its magnitude)."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
@@ -31,6 +34,8 @@ def assert_close(name, got, ref, dtype, relative_max=False):
     err = np.abs(got - ref)
     if relative_max:
         err = err / np.maximum(1.0, np.abs(ref))
+    elif tensor_scale and ref.size:
+        err = err / max(1.0, float(np.abs(ref).max()))
     m = float(err.max()) if err.size else 0.0
     assert r <= rl and m <= ma, f"{name}: rel-L2 {r:.3e} (<= {rl}), max-abs {m:.3e} (<= {ma})"
     return r, m
