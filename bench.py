@@ -31,6 +31,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from kv_cache_compression_ua_b200 import dist  # noqa: E402
 from kv_cache_compression_ua_b200 import inputs as I  # noqa: E402
 
 METRIC = "UA prefill TFLOP/s & decode tok/s; % of BF16 TC peak / HBM roofline"
@@ -111,33 +112,6 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                             device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    return world, rank, local
-
-
-def barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
-
-
-def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
-
-
 # ----------------------------------------------------------------------------- oracle (CPU)
 
 def oracle_sample(w, n_units: int, nthreads: int):
@@ -193,7 +167,7 @@ def workload_config(w):
 # ----------------------------------------------------------------------------- our arm
 
 def device_inputs(w, rank):
-    wr = w.resized(seed=w.seed + 7919 * rank)
+    wr = w.resized(seed=dist.rank_seed(w.seed, rank))
     return I.make_prefill_inputs_torch(wr, "cuda")
 
 
@@ -218,7 +192,7 @@ def bench_prefill(args, world, rank, local, peaks, peaks_kind):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    barrier(world)
+    dist.barrier(world)
     stream = torch.cuda.current_stream()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ua.profile_reset()
@@ -231,9 +205,9 @@ def bench_prefill(args, world, rank, local, peaks, peaks_kind):
         ev1.record(stream)
         torch.cuda.synchronize()
     ua.profile_enable(False)
-    barrier(world)
+    dist.barrier(world)
     ms = ev0.elapsed_time(ev1)
-    ms_max = max_over_ranks(ms, world)
+    ms_max = dist.max_over_ranks(ms, world)
     prof = ua.profile_read()
     assert ua.get_device_status() == 0
     F = fwd_flops(w)
@@ -312,7 +286,7 @@ def bench_decode(args, peaks, peaks_kind):
     res = {}
     cap = T0 + steps + 1
     entry_bytes = 3 * w.d * 2 + 12
-    for p in list(I.DECODE_THRESHOLDS) + [0.0]:
+    for p in (list(I.DECODE_THRESHOLDS) + [0.0] if args.decode_p is None else [args.decode_p]):
         cache = ua.Cache.empty(w.B, w.Hkv, w.d, cap, torch.bfloat16)
         ua.cache_fill(cache, x["k"], x["v"], x["a_k"], bfinal, theta=w.theta)
         ua.cache_compact(cache, p)
@@ -384,6 +358,47 @@ def bench_decode(args, peaks, peaks_kind):
     return res
 
 
+def bwd_flops(w) -> float:
+    """Algorithmic backward FLOPs, counted once: per causal pair and batch, H*10d (the S, dP,
+    dV, dK and dQ products of every query head) plus Hkv*6d (the key-key similarity, and its
+    two gradient products)."""
+    return w.B * w.T * (w.T + 1) / 2 * (w.H * 10 * w.d + w.Hkv * 6 * w.d)
+
+
+def bench_fwdbwd(args):
+    """3B layer forward + backward (B=4, T=8192, H=24, Hkv=8, d=128, bf16)."""
+    from kv_cache_compression_ua_b200 import ua
+    w = I.WORKLOADS["fwdbwd_3b"]
+    x = I.make_prefill_inputs_torch(w, "cuda")
+    args_in = (x["q"], x["k"], x["v"], x["g"], x["a_q"], x["a_k"], x["alpha"], x["beta"])
+    shape = ua.make_shape(x["q"], x["k"], w.scale, w.theta)
+    wsf = ua.alloc_workspace(ua.prefill_workspace_size(shape), "cuda")
+    wsb = ua.alloc_workspace(ua.prefill_bwd_workspace_size(shape), "cuda")
+    f = ua.prefill_fwd(*args_in, scale=w.scale, theta=w.theta, ws=wsf)
+    ua.prefill_bwd(*args_in, f["o"], f["lse"], f["b_final"], x["d_o"], scale=w.scale, theta=w.theta, ws=wsb)
+    torch.cuda.synchronize()
+    n = 3
+    ua.profile_reset()
+    ua.profile_enable(True)
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    e[0].record()
+    for _ in range(n):
+        f = ua.prefill_fwd(*args_in, scale=w.scale, theta=w.theta, ws=wsf)
+    e[1].record()
+    for _ in range(n):
+        ua.prefill_bwd(*args_in, f["o"], f["lse"], f["b_final"], x["d_o"], scale=w.scale, theta=w.theta, ws=wsb)
+    e[2].record()
+    torch.cuda.synchronize()
+    ua.profile_enable(False)
+    prof = ua.profile_read()
+    assert ua.get_device_status() == 0
+    fms, bms = e[0].elapsed_time(e[1]) / n, e[1].elapsed_time(e[2]) / n
+    return {"workload": "fwdbwd_3b: B=4 T=8192 H=24 Hkv=8 d=128 bf16", "fwd_ms": fms, "bwd_ms": bms,
+            "fwd_tflops": fwd_flops(w) / (fms * 1e-3) / 1e12, "bwd_tflops": bwd_flops(w) / (bms * 1e-3) / 1e12,
+            "fwd_bwd_tflops": (fwd_flops(w) + bwd_flops(w)) / ((fms + bms) * 1e-3) / 1e12,
+            "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / v[0]} for k, v in prof.items()}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -393,18 +408,19 @@ def main():
     ap.add_argument("--workload", default="prefill_1b")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--decode-p", type=float, default=None, help="run the decode section at this p only")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    world, rank, local = dist_setup() if args.impl == "ours" else (
-        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    world, rank, local = dist.init("nccl") if args.impl == "ours" else dist.env_world()
     if args.impl == "reference":
         run_reference(args, world, rank)
         return
     from kv_cache_compression_ua_b200 import build as ua_build
     if rank == 0 and not os.path.exists(os.path.join(ROOT, "kv_cache_compression_ua_b200", "libua.so")):
         ua_build.build()
-    barrier(world)
+    dist.barrier(world)
     peaks, peaks_kind = load_peaks()
     w, x, value, ms_step, roofline, kernels, launches, clocks, _ = bench_prefill(
         args, world, rank, local, peaks, peaks_kind)
@@ -414,6 +430,10 @@ def main():
     decode = None
     if not args.no_decode and world == 1:
         decode = bench_decode(args, peaks, peaks_kind)
+    fwdbwd = None
+    if not args.no_bwd and world == 1:
+        torch.cuda.empty_cache()
+        fwdbwd = bench_fwdbwd(args)
     cpu = None
     if not args.no_cpu and rank == 0 and world == 1:
         cores = os.cpu_count() or 1
@@ -425,10 +445,10 @@ def main():
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": workload_config(w), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches, "clocks": clocks, "kernels": kernels, "decode": decode}
+                "gpu_launches": launches, "clocks": clocks, "kernels": kernels, "decode": decode,
+                "fwdbwd_3b": fwdbwd}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        torch.distributed.destroy_process_group()
+    dist.finalize(world)
 
 
 if __name__ == "__main__":
