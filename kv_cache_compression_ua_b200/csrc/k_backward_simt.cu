@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(256) k_bwd_post(Ctx c, BwdParams p) {
     const int t = blockIdx.x, b = blockIdx.y;
     const int d = c.d, half = d / 2, T = c.T;
     __shared__ float s_cos[64], s_sin[64];
-    for (int m = threadIdx.x; m < half; m += blockDim.x) rope_cs((double)t, m, d, p.theta, &s_cos[m], &s_sin[m]);
+    for (int m = threadIdx.x; m < half; m += blockDim.x) rope_cs((double)t, p.rf.f[m], &s_cos[m], &s_sin[m]);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     TI* dq = static_cast<TI*>(p.dq);

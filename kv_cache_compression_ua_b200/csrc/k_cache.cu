@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(256) k_cache_fill(FillParams p) {
     const CacheView& c = p.c;
     constexpr int half = DH / 2;
     __shared__ float s_cos[half], s_sin[half];
-    for (int m = threadIdx.x; m < half; m += blockDim.x) rope_cs((double)t, m, DH, p.theta, &s_cos[m], &s_sin[m]);
+    for (int m = threadIdx.x; m < half; m += blockDim.x) rope_cs((double)t, p.rf.f[m], &s_cos[m], &s_sin[m]);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const TC* kin = static_cast<const TC*>(p.k);
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(256) k_decode(DecodeParams p) {
     for (int e = tid; e < (G + 1) * half; e += blockDim.x) {
         const int vecid = e / half, m = e % half;
         float cs, sn;
-        rope_cs((double)p.pos_t, m, DH, p.theta, &cs, &sn);
+        rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
         if (vecid < G) {
             const float x0 = Elem<TC>::ld(qin + vecid * DH + m), x1 = Elem<TC>::ld(qin + vecid * DH + m + half);
             s_q[vecid][m] = x0 * cs - x1 * sn;

@@ -16,69 +16,92 @@
 namespace ua {
 
 // ------------------------------------------------------------------ token preparation
-// grid (T, B), 256 threads.  Each warp takes one (query or key) head of token t at a time.
-template <typename TI, typename TW>
+// 8 consecutive activations <-> float registers (16-byte bf16 or 2 x 16-byte f32 accesses).
+template <typename T> struct Vec8;
+template <> struct Vec8<__nv_bfloat16> {
+    static __device__ __forceinline__ void ld(const __nv_bfloat16* p, float* x) { Vec16<__nv_bfloat16>::ld(p, x); }
+    static __device__ __forceinline__ void st(__nv_bfloat16* p, const float* x) { Vec16<__nv_bfloat16>::st(p, x); }
+};
+template <> struct Vec8<float> {
+    static __device__ __forceinline__ void ld(const float* p, float* x) {
+        Vec16<float>::ld(p, x);
+        Vec16<float>::ld(p + 4, x + 4);
+    }
+    static __device__ __forceinline__ void st(float* p, const float* x) {
+        Vec16<float>::st(p, x);
+        Vec16<float>::st(p + 4, x + 4);
+    }
+};
+
+// grid (ceil(T/TB), B), 256 threads.  A task is one 8-element chunk c of one (query or key)
+// head of one token: elements 8c..8c+7 of the first half and their RoPE partners d/2 + 8c...;
+// the CH = d/16 tasks of a head sit on consecutive lanes, which reduce the head's norm.
+template <typename TI, typename TW, int DH>
 __global__ void __launch_bounds__(256) k_prep(PrepParams p) {
-    const int t = blockIdx.x, b = blockIdx.y;
-    const int d = p.d, half = d / 2, T = p.T;
-    __shared__ float s_cos[64], s_sin[64];
-    for (int m = threadIdx.x; m < half; m += blockDim.x) rope_cs((double)t, m, d, p.theta, &s_cos[m], &s_sin[m]);
+    constexpr int TB = 4, HALF = DH / 2, CH = HALF / 8;
+    __shared__ float s_cos[TB][HALF], s_sin[TB][HALF];
+    const int t0 = blockIdx.x * TB, b = blockIdx.y, T = p.T;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < TB * HALF; e += blockDim.x) {
+        const int tk = e / HALF, m = e % HALF;
+        rope_cs((double)(t0 + tk), p.rf.f[m], &s_cos[tk][m], &s_sin[tk][m]);
+    }
     __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nh = p.H + p.Hkv;
+    const int ntask = TB * nh * CH;
     const TI* q = static_cast<const TI*>(p.q);
     const TI* k = static_cast<const TI*>(p.k);
-    for (int hh = warp; hh < p.H + p.Hkv; hh += 8) {
+    for (int base = 0; base < ntask; base += blockDim.x) {
+        const int task = base + tid;
+        const int c = task % CH, hh = (task / CH) % nh, tk = task / (CH * nh);
+        const int t = t0 + tk;
+        const bool valid = task < ntask && t < T;
         const bool is_q = hh < p.H;
         const int h = is_q ? hh : hh - p.H;
-        const TI* src = is_q ? q + (((size_t)b * T + t) * p.H + h) * d : k + (((size_t)b * T + t) * p.Hkv + h) * d;
-        float x0[2] = {0.f, 0.f}, x1[2] = {0.f, 0.f};
+        float x0[8], x1[8];
+        if (valid) {
+            const TI* src = is_q ? q + (((size_t)b * T + t) * p.H + h) * DH : k + (((size_t)b * T + t) * p.Hkv + h) * DH;
+            Vec8<TI>::ld(src + 8 * c, x0);
+            Vec8<TI>::ld(src + HALF + 8 * c, x1);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x0[e] = x1[e] = 0.f;
+        }
         float ss = 0.f;
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int m = lane + 32 * r;
-            if (m < half) {
-                x0[r] = Elem<TI>::ld(src + m);
-                x1[r] = Elem<TI>::ld(src + m + half);
-                ss += x0[r] * x0[r] + x1[r] * x1[r];
-            }
-        }
+        for (int e = 0; e < 8; ++e) ss = fmaf(x0[e], x0[e], fmaf(x1[e], x1[e], ss));
+#pragma unroll
+        for (int o = CH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (!valid) continue;
         TW* dst_rot;
-        if (is_q && p.mq) {
-            float sq = ss;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-            if (lane == 0) p.mq[((size_t)b * p.H + h) * p.Tp + t] = p.mq_scale * sqrtf(sq);
-        }
-        if (!is_q) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            const float den = fmaxf(sqrtf(ss), 1e-12f);
-            TW* dst_hat = static_cast<TW*>(p.kh) + (((size_t)b * p.Hkv + h) * T + t) * d;
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int m = lane + 32 * r;
-                if (m < half) {
-                    x0[r] = x0[r] / den;
-                    x1[r] = x1[r] / den;
-                    Elem<TW>::st(dst_hat + m, x0[r]);
-                    Elem<TW>::st(dst_hat + m + half, x1[r]);
-                }
-            }
-            dst_rot = static_cast<TW*>(p.kr) + (((size_t)b * p.Hkv + h) * T + t) * d;
+        if (is_q) {
+            if (p.mq && c == 0) p.mq[((size_t)b * p.H + h) * p.Tp + t] = p.mq_scale * sqrtf(ss);
+            dst_rot = static_cast<TW*>(p.qr) + (((size_t)b * p.H + h) * T + t) * DH;
         } else {
-            dst_rot = static_cast<TW*>(p.qr) + (((size_t)b * p.H + h) * T + t) * d;
-        }
+            const float den = fmaxf(sqrtf(ss), 1e-12f);
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int m = lane + 32 * r;
-            if (m < half) {
-                const float c = s_cos[m], s = s_sin[m];
-                Elem<TW>::st(dst_rot + m, x0[r] * c - x1[r] * s);
-                Elem<TW>::st(dst_rot + m + half, x1[r] * c + x0[r] * s);
+            for (int e = 0; e < 8; ++e) {
+                x0[e] = x0[e] / den;
+                x1[e] = x1[e] / den;
             }
+            TW* dst_hat = static_cast<TW*>(p.kh) + (((size_t)b * p.Hkv + h) * T + t) * DH;
+            Vec8<TW>::st(dst_hat + 8 * c, x0);
+            Vec8<TW>::st(dst_hat + HALF + 8 * c, x1);
+            dst_rot = static_cast<TW*>(p.kr) + (((size_t)b * p.Hkv + h) * T + t) * DH;
         }
+        float y0[8], y1[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float cs = s_cos[tk][8 * c + e], sn = s_sin[tk][8 * c + e];
+            y0[e] = x0[e] * cs - x1[e] * sn;
+            y1[e] = x1[e] * cs + x0[e] * sn;
+        }
+        Vec8<TW>::st(dst_rot + 8 * c, y0);
+        Vec8<TW>::st(dst_rot + HALF + 8 * c, y1);
     }
-    for (int h = threadIdx.x; h < p.Hkv; h += blockDim.x) {
+    for (int e = tid; e < TB * p.Hkv; e += blockDim.x) {
+        const int tk = e / p.Hkv, h = e % p.Hkv, t = t0 + tk;
+        if (t >= T) continue;
         const size_t src = ((size_t)b * T + t) * p.Hkv + h;
         const size_t dst = ((size_t)b * p.Hkv + h) * T + t;
         const float sq = softplus_f(p.a_q[src]), sk = softplus_f(p.a_k[src]);
@@ -316,13 +339,19 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
 }
 
 // ------------------------------------------------------------------ launchers
+template <int DH>
+static void prep_inst(const PrepParams& p, bool bf16_in, bool bf16_work, cudaStream_t s) {
+    dim3 grid((p.T + 3) / 4, p.B);
+    if (bf16_in && bf16_work) k_prep<__nv_bfloat16, __nv_bfloat16, DH><<<grid, 256, 0, s>>>(p);
+    else if (bf16_in) k_prep<__nv_bfloat16, float, DH><<<grid, 256, 0, s>>>(p);
+    else if (bf16_work) k_prep<float, __nv_bfloat16, DH><<<grid, 256, 0, s>>>(p);
+    else k_prep<float, float, DH><<<grid, 256, 0, s>>>(p);
+}
+
 cudaError_t launch_prep(const PrepParams& p, bool bf16_in, bool bf16_work, cudaStream_t s) {
-    dim3 grid(p.T, p.B);
     UA_PROFILE("k_prep", s);
-    if (bf16_in && bf16_work) k_prep<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, s>>>(p);
-    else if (bf16_in) k_prep<__nv_bfloat16, float><<<grid, 256, 0, s>>>(p);
-    else if (bf16_work) k_prep<float, __nv_bfloat16><<<grid, 256, 0, s>>>(p);
-    else k_prep<float, float><<<grid, 256, 0, s>>>(p);
+    if (p.d == 64) prep_inst<64>(p, bf16_in, bf16_work, s);
+    else prep_inst<128>(p, bf16_in, bf16_work, s);
     return cudaGetLastError();
 }
 

@@ -97,6 +97,13 @@ size_t prefill_ws_bytes(const ua_shape* s) {
 
 ua_status cuda_status(cudaError_t e) { return e == cudaSuccess ? UA_OK : UA_ERR_CUDA; }
 
+// RoPE frequencies theta^(-2m/d), m < d/2, in double precision.
+RopeFreq rope_freq(double theta, int d) {
+    RopeFreq r;
+    for (int m = 0; m < 64; ++m) r.f[m] = (m < d / 2) ? pow(theta, -2.0 * (double)m / (double)d) : 0.0;
+    return r;
+}
+
 char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
 
 ua_status check_cache(const ua_cache* c) {
@@ -163,6 +170,7 @@ static ua_status prefill_fwd_simt(const ua_shape* s, const void* q, const void* 
     pp.q = q; pp.k = k; pp.a_q = a_q; pp.a_k = a_k;
     pp.qr = at(ws, w.qr); pp.kh = at(ws, w.kh); pp.kr = at(ws, w.kr);
     pp.rq = reinterpret_cast<float*>(at(ws, w.rq)); pp.rk = reinterpret_cast<float*>(at(ws, w.rk));
+    pp.rf = rope_freq(s->rope_theta, s->d);
     if ((st = cuda_status(launch_prep(pp, bf, false, cs))) != UA_OK) return st;
 
     BoundaryParams bp;
@@ -200,6 +208,7 @@ static ua_status prefill_fwd_tc(const ua_shape* s, const void* q, const void* k,
     pp.Tp = w.Tp; pp.mq_scale = s->scale * 1.4426950408889634f;
     pp.lq2 = reinterpret_cast<float*>(at(ws, w.lq2)); pp.lk2 = reinterpret_cast<float*>(at(ws, w.lk2));
     pp.mq = reinterpret_cast<float*>(at(ws, w.mq));
+    pp.rf = rope_freq(s->rope_theta, s->d);
     if ((st = cuda_status(launch_prep(pp, true, true, cs))) != UA_OK) return st;
 
     BoundaryParams bp;
@@ -349,6 +358,7 @@ ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const 
     pp.q = q; pp.k = k; pp.a_q = a_q; pp.a_k = a_k;
     pp.qr = at(ws, w.f.qr); pp.kh = at(ws, w.f.kh); pp.kr = at(ws, w.f.kr);
     pp.rq = reinterpret_cast<float*>(at(ws, w.f.rq)); pp.rk = reinterpret_cast<float*>(at(ws, w.f.rk));
+    pp.rf = rope_freq(s->rope_theta, s->d);
     if ((st = cuda_status(launch_prep(pp, bf, false, cs))) != UA_OK) return st;
     BoundaryParams bp;
     bp.B = s->B; bp.T = s->T; bp.Hkv = s->Hkv; bp.d = s->d; bp.bq = kBq; bp.nqt = w.nqt;
@@ -358,7 +368,7 @@ ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const 
 
     BwdParams p;
     p.B = s->B; p.T = s->T; p.H = s->H; p.Hkv = s->Hkv; p.d = s->d; p.G = s->H / s->Hkv; p.nqt = w.nqt; p.nkt = w.nkt;
-    p.scale = s->scale; p.theta = s->rope_theta;
+    p.scale = s->scale; p.theta = s->rope_theta; p.rf = pp.rf;
     p.qr = reinterpret_cast<const float*>(pp.qr); p.kh = reinterpret_cast<const float*>(pp.kh);
     p.kr = reinterpret_cast<const float*>(pp.kr); p.rq = pp.rq; p.rk = pp.rk; p.pb = bp.pb;
     p.k = k; p.v = v; p.g = g; p.o = o; p.d_o = d_o; p.a_q = a_q; p.a_k = a_k; p.alpha = alpha; p.beta = beta;
@@ -383,6 +393,7 @@ ua_status ua_cache_fill(const ua_cache* c, int T, const void* k, const void* v, 
         if (!aligned(p, 16)) return UA_ERR_ALIGNMENT;
     FillParams fp;
     fp.c = view(c); fp.T = T; fp.theta = rope_theta; fp.k = k; fp.v = v; fp.a_k = a_k; fp.bfinal = b_final;
+    fp.rf = rope_freq(rope_theta, c->d);
     return cuda_status(launch_cache_fill(fp, c->dtype == UA_BF16, static_cast<cudaStream_t>(stream)));
 }
 
@@ -411,7 +422,7 @@ ua_status ua_decode_step(const ua_cache* c, int H, const void* q, const void* k,
         if (x && !aligned(x, 16)) return UA_ERR_ALIGNMENT;
     DecodeParams dp;
     dp.c = view(c); dp.H = H; dp.G = H / c->Hkv; dp.pos_t = pos_t; dp.scale = scale;
-    dp.logp = p > 0.f ? logf(p) : -INFINITY; dp.theta = rope_theta;
+    dp.logp = p > 0.f ? logf(p) : -INFINITY; dp.theta = rope_theta; dp.rf = rope_freq(rope_theta, c->d);
     dp.q = q; dp.k = k; dp.v = v; dp.g = g; dp.a_q = a_q; dp.a_k = a_k; dp.alpha = alpha; dp.beta = beta;
     dp.o = o; dp.evict_bits = evict_bits; dp.kept_idx = kept_idx;
     return cuda_status(launch_decode(dp, c->dtype == UA_BF16, static_cast<cudaStream_t>(stream)));

@@ -27,14 +27,20 @@ __device__ __forceinline__ float decay_geo(float rq, float rk, float rsim) {
     return cbrtf(rq * rk * rsim);
 }
 
-// RoPE angle of pair m at position pos, in double precision (positions up to 1e6 keep
-// the angle accurate to ~1e-10 rad before the fp32 cos/sin are formed).
-__device__ __forceinline__ void rope_cs(double pos, int m, int d, double theta, float* c, float* s) {
-    double freq = pow(theta, -2.0 * (double)m / (double)d);
-    double sn, cs;
-    sincos(pos * freq, &sn, &cs);
-    *c = (float)cs;
-    *s = (float)sn;
+// RoPE frequencies theta^(-2m/d), computed on the host in double precision (m < d/2 <= 64).
+struct RopeFreq {
+    double f[64];
+};
+
+// cos / sin of the RoPE angle pos * f.  The angle is formed in double precision and reduced
+// to [-pi, pi] with a two-constant Cody-Waite split of 2*pi (exact to ~1e-16 relative for the
+// positions used here), then the fp32 sincosf of the reduced angle is taken.
+__device__ __forceinline__ void rope_cs(double pos, double f, float* c, float* s) {
+    const double a = pos * f;
+    const double k = rint(a * 0.15915494309189535);            // 1 / (2 pi)
+    double r = fma(-k, 6.283185307179586, a);                   // 2 pi, high part
+    r = fma(-k, 2.4492935982947064e-16, r);                     // 2 pi, low part
+    sincosf((float)r, s, c);
 }
 
 // ------------------------------------------------------------------ element access

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "ua_common.cuh"
+
 namespace ua {
 
 // Token preparation: normalised keys, RoPE'd queries/keys, per-token rates.
@@ -26,6 +28,7 @@ struct PrepParams {
     float* lq2;         // [B*Hkv][Tp] log2(softplus(a_q)) / 3
     float* lk2;         // [B*Hkv][Tp] log2(softplus(a_k)) / 3
     float* mq;          // [B*H][Tp]  scale * ||q|| * log2(e): bound of every logit of the row
+    RopeFreq rf;
 };
 
 // Boundary pass: per-query-tile column prefixes of the decay and the final biases.
@@ -76,6 +79,7 @@ struct FillParams {
     CacheView c;
     int T;
     double theta;
+    RopeFreq rf;
     const void* k;       // [B,T,Hkv,d] act
     const void* v;       // [B,T,Hkv,d] act
     const float* a_k;    // [B,T,Hkv]
@@ -94,6 +98,7 @@ struct DecodeParams {
     int H, G, pos_t;
     float scale, logp;
     double theta;
+    RopeFreq rf;
     const void* q;       // [B,H,d] act
     const void* k;       // [B,Hkv,d] act
     const void* v;       // [B,Hkv,d] act
@@ -113,6 +118,7 @@ struct BwdParams {
     int B, T, H, Hkv, d, G, nqt, nkt;
     float scale;
     double theta;
+    RopeFreq rf;
     const float* qr;     // [B,H,T,d]  RoPE(q)
     const float* kh;     // [B,Hkv,T,d] khat
     const float* kr;     // [B,Hkv,T,d] RoPE(khat)
