@@ -323,7 +323,7 @@ struct Smem {
     alignas(16) float pb[128];                   // boundary prefix of the key tile at this query tile
     alignas(16) float tot[2][NWG][128];          // per-quarter column sums (without the key factor)
     alignas(8) uint64_t qfull, khfull, khempty, krfull, krempty, vfull[2], vempty[2], xsfull[NSLOT], xsempty[NSLOT],
-        pfull[2], pempty[2], ofull, cfull[2];
+        pfull[2], pempty[2], ofull, cfull[2][NWG];
     uint32_t tmem;
     int abort;
 };
@@ -377,7 +377,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             mbar_init(&S.vempty[i], 1);
             mbar_init(&S.pfull[i], 4 * NWG);
             mbar_init(&S.pempty[i], 1);
-            mbar_init(&S.cfull[i], 4 * NWG);
+            for (int w = 0; w < NWG; ++w) mbar_init(&S.cfull[i][w], 4);   // the four warps of quarter w
         }
         for (int w = 0; w < NSLOT; ++w) {
             mbar_init(&S.xsfull[w], 1);
@@ -588,11 +588,17 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 for (int pc = 0; pc < 2; ++pc) {
                     uint32_t x[16];
                     slot_read(pc, x);
+                    float lv[16];
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4) {
+                        const float4 t4 = *reinterpret_cast<const float4*>(lqh + pc * 16 + e);
+                        lv[e] = t4.x; lv[e + 1] = t4.y; lv[e + 2] = t4.z; lv[e + 3] = t4.w;
+                    }
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const int r = pc * 16 + e;
                         const float dq = ex2f(fmaf(log2_softplus_poly(fmaf(al, __uint_as_float(x[e]), be)),
-                                                   0.33333334f, lqh[r]));
+                                                   0.33333334f, lv[e]));
                         c += (!diag || qt * 128 + r0 + r > j) ? dq : 0.f;
                         lam[r] = c;
                     }
@@ -600,10 +606,13 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 S.tot[kt & 1][wg][jl] = c;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&S.cfull[kt & 1]);
-            if (!mbar_wait(&S.cfull[kt & 1], (kt >> 1) & 1, abort)) { ok = false; break; }
+            if (lane == 0) mbar_arrive(&S.cfull[kt & 1][wg]);
             float above = 0.f;                           // sum over the quarters above this one
-            for (int w = 0; w < wg; ++w) above += S.tot[kt & 1][w][jl];
+            for (int w = 0; w < wg; ++w) {
+                if (!mbar_wait(&S.cfull[kt & 1][w], (kt >> 1) & 1, abort)) { ok = false; break; }
+                above += S.tot[kt & 1][w][jl];
+            }
+            if (!ok) break;
             // Lambda in log2 units: -(Pb + r_k^(1/3) * (above + partial sum)) * log2(e)
             const float ka = -rk3 * kLog2e, kb = -fmaf(rk3, above, pbj) * kLog2e;
 #pragma unroll
@@ -624,12 +633,15 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                     for (int cc = 0; cc < 2; ++cc) {
                         const int ck = pc * 2 + cc;
                         uint32_t w4[4];
+                        const float4 m0 = *reinterpret_cast<const float4*>(mqh + ck * 8);
+                        const float4 m1 = *reinterpret_cast<const float4*>(mqh + ck * 8 + 4);
+                        const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
                         for (int e = 0; e < 8; e += 2) {
                             const int r = ck * 8 + e;
                             const int xe = cc * 8 + e;
-                            float p0 = ex2f(fmaf(__uint_as_float(x[xe]), sl, lam[r] - mqh[r]));
-                            float p1 = ex2f(fmaf(__uint_as_float(x[xe + 1]), sl, lam[r + 1] - mqh[r + 1]));
+                            float p0 = ex2f(fmaf(__uint_as_float(x[xe]), sl, lam[r] - mv[e]));
+                            float p1 = ex2f(fmaf(__uint_as_float(x[xe + 1]), sl, lam[r + 1] - mv[e + 1]));
                             if (diag) {
                                 const int i = qt * 128 + r0 + r;
                                 p0 = (j < T && j <= i) ? p0 : 0.f;
