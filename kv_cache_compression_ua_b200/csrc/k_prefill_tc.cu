@@ -1,5 +1,6 @@
-// k_prefill_tc.cu -- tensor-core (tcgen05 / TMEM / TMA) kernels of the bf16 prefill:
-// the decay boundary pass and the fused biased attention forward.
+// k_prefill_tc.cu -- tensor-core (tcgen05 / TMEM / TMA) kernel of the bf16 prefill: the
+// fused biased attention forward, with the decay boundary prefixes carried between query
+// tiles inside the same launch.
 //
 // Decay structure (see ua.h for the formulas): L2-normalised keys, three rates combined by
 // a geometric mean, log space, causal accumulation into Lambda (ai4snews synopsis, Fig. 1
@@ -90,211 +91,13 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
 
 }  // namespace
 
-// ================================================================ boundary pass
-// grid (ceil(T/128) key tiles, Hkv, B); 192 threads: warps 0-3 decay (one key per thread,
-// TMEM lanes 0-127), warp 4 TMA producer, warp 5 MMA issuer.  For key tile kt it sweeps the
-// query tiles t = kt .. nqt-1: X^T = Khat_k * Khat_t^T (M=128 keys, N=128 rows) into one of
-// two TMEM buffers, and each thread sums D over its row of X^T.
-namespace bnd {
-constexpr int NS = 3;   // query-tile stages
-template <int NB>
-struct Smem {
-    alignas(1024) uint8_t a[NB][16384];         // Khat of the key tile (NB 64-column boxes)
-    alignas(1024) uint8_t b[NS][NB][16384];     // Khat of the query tile
-    alignas(16) float lq[NS][128];              // lq2 of the query tile rows
-    alignas(8) uint64_t full[NS], empty[NS], tfull[2], tempty[2], abar;
-    uint32_t tmem;
-    int abort;
-};
-}  // namespace bnd
-
-struct BoundaryTcParams {
-    int B, T, Tp, Hkv, d, nqt;
-    const float* lk2;    // [B*Hkv][Tp]
-    const float* alpha;
-    const float* beta;
-    float* pb;           // [B*Hkv][nqt][Tp]
-    float* bfinal;       // [B*Hkv][T] or NULL
-};
-
-template <int DH>
-__global__ void __launch_bounds__(192, 2)
-k_boundary_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_lq,
-              BoundaryTcParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    constexpr int NB = DH / 64;                  // 64-column boxes per tile
-    using SM = bnd::Smem<NB>;
-    SM& S = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int KSTEPS = DH / 16;
-    constexpr uint32_t IDESC = idesc_bf16(128, 128, 0, 0);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-    const int unit = b * p.Hkv + kvh;
-    const int T = p.T;
-    const int ntile = p.nqt - kt;                // query tiles kt .. nqt-1
-    volatile int* abort = &S.abort;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < bnd::NS; ++s) {
-            mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], 1 + 4);       // MMA commit + 4 decay warps (lq reads)
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.tfull[i], 1);
-            mbar_init(&S.tempty[i], 4);
-        }
-        mbar_init(&S.abar, 1);
-        S.abort = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(&S.tmem, 256);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = S.tmem;
-
-    if (warp == 4) {
-        const bool leader = elect_one();
-        if (leader) {
-            prefetch_tmap(&tm_kh);
-            prefetch_tmap(&tm_lq);
-            mbar_expect_tx(&S.abar, NB * 16384);
-            for (int bx = 0; bx < NB; ++bx) tma_load_3d(S.a[bx], &tm_kh, &S.abar, bx * 64, kt * 128, unit);
-        }
-        __syncwarp();
-        for (int it = 0; it < ntile; ++it) {
-            const int s = it % bnd::NS;
-            if (it >= bnd::NS && !mbar_wait(&S.empty[s], ((it / bnd::NS) - 1) & 1, abort)) break;
-            const int t = kt + it;
-            if (leader) {
-                mbar_expect_tx(&S.full[s], NB * 16384 + 512);
-                for (int bx = 0; bx < NB; ++bx) tma_load_3d(S.b[s][bx], &tm_kh, &S.full[s], bx * 64, t * 128, unit);
-                tma_load_2d(S.lq[s], &tm_lq, &S.full[s], t * 128, unit);
-            }
-            __syncwarp();
-        }
-    } else if (warp == 5) {
-        const bool leader = elect_one();
-        if (mbar_wait(&S.abar, 0, abort)) {
-            uint64_t da[KSTEPS];
-#pragma unroll
-            for (int kk = 0; kk < KSTEPS; ++kk) da[kk] = kmajor_desc(smem_u32(S.a[0]), kk);
-            for (int it = 0; it < ntile; ++it) {
-                const int s = it % bnd::NS, buf = it & 1;
-                if (!mbar_wait(&S.full[s], (it / bnd::NS) & 1, abort)) break;
-                if (it >= 2 && !mbar_wait(&S.tempty[buf], ((it >> 1) - 1) & 1, abort)) break;
-                tc_fence_after();
-                if (leader) {
-                    const uint32_t b0 = smem_u32(S.b[s][0]);
-#pragma unroll
-                    for (int kk = 0; kk < KSTEPS; ++kk)
-                        umma_f16(tmem + buf * 128, da[kk], kmajor_desc(b0, kk), IDESC, kk > 0);
-                    umma_commit(&S.empty[s]);
-                    umma_commit(&S.tfull[buf]);
-                }
-                __syncwarp();
-            }
-        }
-    } else {
-        // decay warps: thread owns key j
-        const int jl = warp * 32 + lane;
-        const int j = kt * 128 + jl;
-        const bool jvalid = j < T;
-        const float al = p.alpha[kvh], be = p.beta[kvh];
-        float* pb = p.pb + (size_t)unit * p.nqt * p.Tp;
-        if (jvalid)
-            for (int t = 0; t < kt; ++t) pb[(size_t)t * p.Tp + j] = 0.f;
-        const float rk3 = jvalid ? ex2f(p.lk2[(size_t)unit * p.Tp + j]) : 0.f;   // r_k(j)^(1/3)
-        float acc = 0.f;
-        for (int it = 0; it < ntile; ++it) {
-            const int s = it % bnd::NS, buf = it & 1;
-            const int t = kt + it;
-            if (!mbar_wait(&S.tfull[buf], (it >> 1) & 1, abort)) break;
-            if (!mbar_wait(&S.full[s], (it / bnd::NS) & 1, abort)) break;   // lq of this stage landed
-            tc_fence_after();
-            // rows l of this tile need masking only on the diagonal tile (l > j) and past T
-            const bool masked = (t == kt) || (t * 128 + 128 > T);
-            float tile = 0.f;
-            const uint32_t xcol = tmem + ((uint32_t)(warp * 32) << 16) + buf * 128;
-            const float* lq = S.lq[s];
-            uint32_t ra[16], rb[16];
-            auto chunk = [&](const uint32_t (&x)[16], int ch) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int l = t * 128 + ch * 16 + e;
-                    const float dq = ex2f(fmaf(log2_softplus_poly(fmaf(al, __uint_as_float(x[e]), be)), 0.33333334f,
-                                               lq[ch * 16 + e]));
-                    tile += (!masked || (l > j && l < T)) ? dq : 0.f;
-                }
-            };
-            tmem_ld16_async(xcol, ra);
-#pragma unroll 1
-            for (int cp = 0; cp < 4; ++cp) {
-                tmem_wait16(ra);
-                tmem_ld16_async(xcol + (2 * cp + 1) * 16, rb);
-                chunk(ra, 2 * cp);
-                tmem_wait16(rb);
-                if (cp < 3) tmem_ld16_async(xcol + (2 * cp + 2) * 16, ra);
-                chunk(rb, 2 * cp + 1);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&S.tempty[buf]);
-                mbar_arrive(&S.empty[s]);
-            }
-            if (jvalid) pb[(size_t)t * p.Tp + j] = acc;
-            acc = fmaf(rk3, tile, acc);
-        }
-        if (jvalid && p.bfinal && !*abort) p.bfinal[(size_t)unit * T + j] = -acc;
-    }
-
-    __syncthreads();
-    if (*abort && threadIdx.x == 0) drain_pause(10000000ull);
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 256);
-    }
-}
-
-// ================================================================ launchers
-
-size_t boundary_tc_smem(int d) { return (d == 64 ? sizeof(bnd::Smem<1>) : sizeof(bnd::Smem<2>)) + 1024; }
-
-cudaError_t launch_boundary_tc(const BoundaryParams& bp, const void* kh_bf16, const float* lq2, const float* lk2,
-                               int Tp, cudaStream_t s) {
-    CUtensorMap tm_kh, tm_lq;
-    if (!map_rows_bf16(&tm_kh, kh_bf16, bp.d, bp.T, bp.B * bp.Hkv)) return cudaErrorInvalidValue;
-    if (!map_vec_f32(&tm_lq, lq2, bp.T, Tp, bp.B * bp.Hkv)) return cudaErrorInvalidValue;
-    BoundaryTcParams p;
-    p.B = bp.B; p.T = bp.T; p.Tp = Tp; p.Hkv = bp.Hkv; p.d = bp.d; p.nqt = bp.nqt;
-    p.lk2 = lk2; p.alpha = bp.alpha; p.beta = bp.beta; p.pb = bp.pb; p.bfinal = bp.bfinal;
-    const size_t smem = boundary_tc_smem(bp.d);
-    dim3 grid((bp.T + 127) / 128, bp.Hkv, bp.B);
-    UA_PROFILE("k_boundary_tc", s);
-    if (bp.d == 64) {
-        cudaError_t e = cudaFuncSetAttribute(k_boundary_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        k_boundary_tc<64><<<grid, 192, smem, s>>>(tm_kh, tm_lq, p);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(k_boundary_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        k_boundary_tc<128><<<grid, 192, smem, s>>>(tm_kh, tm_lq, p);
-    }
-    return cudaGetLastError();
-}
-
-
 // ================================================================ fused forward
-// grid (nqt, Hkv, B): one CTA per (batch, KV head, 128-row query tile) serving all G query
-// heads of the group, so the decay tile is built once for the G heads.  576 threads:
+// One CTA per (batch, KV head, 128-row query tile) serving all G query heads of the group,
+// so the decay tile is built once for the G heads.  608 threads:
 //   warps 0-15  decay/softmax: warpgroup w = warp/4 owns query rows 32w .. 32w+31 of the
 //               tile; while streaming key tiles, thread = key j (TMEM lane)
-//   warp 16     TMA producer (lane 0), warp 17 MMA issuer (lane 0)
+//   warp 16     TMA producer, warp 17 MMA issuer (one elected lane issues for each)
+//   warp 18     boundary look-back: fetches Pb of each key tile from the previous query tile
 // Per key tile kt <= qt:
 //   X^T = Khat_k Khat_q^T and S_h^T = Krope_k Qrope_h^T are computed one 32-row quarter per
 //   warpgroup into that warpgroup's 32-column TMEM slot.  Each thread turns X^T into D and
@@ -305,6 +108,14 @@ cudaError_t launch_boundary_tc(const BoundaryParams& bp, const void* kh_bf16, co
 //   the P tile.  M_i = scale*||q_i||*log2e bounds every logit of row i (keys are unit
 //   vectors, Lambda <= 0), so no running maximum and no rescaling are needed.  O_h += P V and
 //   l_h += P 1 run on the tensor cores with accumulators in TMEM.
+// Boundary prefixes without a separate pass: Pb(qt, kt)[j], the sum of D[l, j] over the rows
+// l > j of the query tiles before qt, equals Pb(qt-1, kt) plus the column total of tile qt-1.
+// The bottom quarter of each CTA holds exactly that inclusive prefix after its carry exchange
+// and publishes it to global memory (release: fence, then a per-(tile, key tile) counter);
+// the next query tile's look-back warp acquires it.  CTAs draw work tickets from a counter in
+// query-tile-major order, so a CTA only ever waits on CTAs with lower tickets, which are
+// already running: the chain always makes progress.  The last query tile writes b_final =
+// -(its inclusive prefix) = Lambda_{T-1, j}.
 namespace fwd {
 constexpr int NWG = 4;   // decay warpgroups (32 query rows each)
 constexpr int NSLOT = 3; // TMEM ring of 64-column half tiles (each half serves a pair of warpgroups)
@@ -320,11 +131,12 @@ struct Smem {
     alignas(16) float lq[128];                   // lq2 of the query rows
     alignas(16) float mq[G][128];                // row bound M_i (log2 units) per head
     alignas(16) float lk[128];                   // lk2 of the key tile
-    alignas(16) float pb[128];                   // boundary prefix of the key tile at this query tile
+    alignas(16) float pb[2][128];                // boundary prefix Pb of the key tile, two stages
     alignas(16) float tot[2][NWG][128];          // per-quarter column sums (without the key factor)
     alignas(8) uint64_t qfull, khfull, khempty, krfull, krempty, vfull[2], vempty[2], xsfull[NSLOT], xsempty[NSLOT],
-        pfull[2], pempty[2], ofull, cfull[2][NWG];
+        pfull[2], pempty[2], ofull, cfull[2][NWG], pbfull[2], pbempty[2];
     uint32_t tmem;
+    int ticket;
     int abort;
 };
 }  // namespace fwd
@@ -337,14 +149,39 @@ struct FwdTcParams {
     const void* g;       // [B,T,H,64] bf16
     void* o;             // [B,T,H,64] bf16
     float* lse;          // [B,H,T] or NULL
+    float* pincl;        // [B*Hkv*nqt][Tp] inclusive column prefixes published per query tile
+    unsigned* flags;     // [B*Hkv][nqt][nqt] publication counters; flags[B*Hkv*nqt*nqt] = ticket
+    float* b_final;      // [B*Hkv][T] or NULL
+    int nunits;          // B * Hkv
 };
 
+// Wait (all lanes of the warp) until *f >= target, with acquire semantics for every lane.
+__device__ __forceinline__ bool wait_counter(const unsigned* f, unsigned target, volatile int* abort, int lane) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 0;; ++it) {
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+        if (__all_sync(0xffffffffu, v >= target)) return true;
+        if ((it & 63u) == 63u) {
+            const bool stop = __shfl_sync(0xffffffffu, (int)(*abort != 0 || globaltimer() - t0 > kWaitLimitNs), 0);
+            if (stop) {
+                if (lane == 0 && !*abort) {
+                    raise_status(UA_ERR_TIMEOUT);
+                    *abort = 1;
+                }
+                return false;
+            }
+        }
+        __nanosleep(64);
+    }
+}
+
 template <int G>
-__global__ void __launch_bounds__(576, 1)
+__global__ void __launch_bounds__(608, 1)
 k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_kr,
          const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_v,
          const __grid_constant__ CUtensorMap tm_lq, const __grid_constant__ CUtensorMap tm_lk,
-         const __grid_constant__ CUtensorMap tm_mq, const __grid_constant__ CUtensorMap tm_pb, FwdTcParams p) {
+         const __grid_constant__ CUtensorMap tm_mq, FwdTcParams p) {
     constexpr int DH = 64;
     constexpr int NWG = fwd::NWG;
     constexpr uint32_t ID_XS = idesc_bf16(128, 64, 0, 0);
@@ -359,11 +196,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
     SM& S = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = gridDim.x - 1 - blockIdx.x;          // heaviest query tiles first
-    const int kvh = blockIdx.y, b = blockIdx.z;
-    const int unit = b * p.Hkv + kvh;
     const int T = p.T;
-    const int ntile = qt + 1;
     volatile int* abort = &S.abort;
 
     if (threadIdx.x == 0) {
@@ -378,6 +211,8 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             mbar_init(&S.pfull[i], 4 * NWG);
             mbar_init(&S.pempty[i], 1);
             for (int w = 0; w < NWG; ++w) mbar_init(&S.cfull[i][w], 4);   // the four warps of quarter w
+            mbar_init(&S.pbfull[i], 1);
+            mbar_init(&S.pbempty[i], 4 * NWG);
         }
         for (int w = 0; w < NSLOT; ++w) {
             mbar_init(&S.xsfull[w], 1);
@@ -385,6 +220,9 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
         }
         mbar_init(&S.ofull, 1);
         S.abort = 0;
+        // Work tickets go out in launch order, query tile major: every CTA a tile waits on
+        // (same KV unit, lower query tile) holds a lower ticket and is already resident.
+        S.ticket = (int)atomicAdd(p.flags + (size_t)p.nunits * p.nqt * p.nqt, 1u);
         fence_barrier_init();
     }
     if (warp == 16) {
@@ -401,13 +239,16 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem;
+    const int qt = S.ticket / p.nunits, unit = S.ticket % p.nunits;
+    const int kvh = unit % p.Hkv, b = unit / p.Hkv;
+    const int ntile = qt + 1;
 
     if (warp == 16) {
         // ------------------------------------------------ TMA producer (warp-uniform, one lane issues)
         const bool leader = elect_one();
         if (leader) {
-            const CUtensorMap* maps[8] = {&tm_kh, &tm_kr, &tm_q, &tm_v, &tm_lq, &tm_lk, &tm_mq, &tm_pb};
-            for (int m = 0; m < 8; ++m) prefetch_tmap(maps[m]);
+            const CUtensorMap* maps[7] = {&tm_kh, &tm_kr, &tm_q, &tm_v, &tm_lq, &tm_lk, &tm_mq};
+            for (int m = 0; m < 7; ++m) prefetch_tmap(maps[m]);
             mbar_expect_tx(&S.qfull, 16384 * (1 + G) + 512 * (1 + G));
             tma_load_3d(S.kq, &tm_kh, &S.qfull, 0, qt * 128, unit);
             for (int h = 0; h < G; ++h) tma_load_3d(S.q[h], &tm_q, &S.qfull, 0, qt * 128, b * p.H + kvh * G + h);
@@ -418,10 +259,9 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
         for (int kt = 0; kt < ntile; ++kt) {
             if (kt >= 1 && !mbar_wait(&S.khempty, (kt - 1) & 1, abort)) break;
             if (leader) {
-                mbar_expect_tx(&S.khfull, 16384 + 2 * 512);
+                mbar_expect_tx(&S.khfull, 16384 + 512);
                 tma_load_3d(S.kh, &tm_kh, &S.khfull, 0, kt * 128, unit);
                 tma_load_2d(S.lk, &tm_lk, &S.khfull, kt * 128, unit);
-                tma_load_2d(S.pb, &tm_pb, &S.khfull, kt * 128, unit * p.nqt + qt);
             }
             __syncwarp();
             const int sv = kt & 1;
@@ -437,6 +277,23 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 tma_load_3d(S.kr, &tm_kr, &S.krfull, 0, kt * 128, unit);
             }
             __syncwarp();
+        }
+    } else if (warp == 18) {
+        // ------------------------------------------------ boundary prefixes (look-back)
+        // Pb of key tile kt at this query tile = the inclusive prefix the previous query tile
+        // published for kt (zero on the diagonal): lane l fetches keys 4l .. 4l+3.
+        for (int kt = 0; kt < ntile; ++kt) {
+            const int sb = kt & 1;
+            if (kt >= 2 && !mbar_wait(&S.pbempty[sb], ((kt >> 1) - 1) & 1, abort)) break;
+            float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (kt < qt) {
+                const size_t row = (size_t)unit * p.nqt + (qt - 1);
+                if (!wait_counter(p.flags + row * p.nqt + kt, 4u, abort, lane)) break;
+                v4 = __ldcg(reinterpret_cast<const float4*>(p.pincl + row * p.Tp + (size_t)kt * 128) + lane);
+            }
+            *reinterpret_cast<float4*>(&S.pb[sb][lane * 4]) = v4;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.pbfull[sb]);
         }
     } else if (warp == 17) {
         // ------------------------------------------------ MMA issuer (warp-uniform, one lane issues)
@@ -574,9 +431,9 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
         for (int kt = 0; ok && kt < ntile; ++kt) {
             const int j = kt * 128 + jl;
             const bool diag = (kt == qt);                // only the diagonal tile needs masks
+            const bool tailq = qt * 128 + 128 > T;       // ... and, for the column totals, the last one
             if (!mbar_wait(&S.khfull, kt & 1, abort)) { ok = false; break; }
             const float rk3 = ex2f(S.lk[jl]);            // r_k(j)^(1/3); 0 when vetoed
-            const float pbj = S.pb[jl];
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.khempty);
             // ---- decay over this quarter's 32 rows (without the key factor), scanned down the column
@@ -599,7 +456,8 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                         const int r = pc * 16 + e;
                         const float dq = ex2f(fmaf(log2_softplus_poly(fmaf(al, __uint_as_float(x[e]), be)),
                                                    0.33333334f, lv[e]));
-                        c += (!diag || qt * 128 + r0 + r > j) ? dq : 0.f;
+                        const int row = qt * 128 + r0 + r;
+                        c += (!(diag || tailq) || (row > j && row < T)) ? dq : 0.f;
                         lam[r] = c;
                     }
                 }
@@ -613,6 +471,26 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 above += S.tot[kt & 1][w][jl];
             }
             if (!ok) break;
+            if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) { ok = false; break; }
+            const float pbj = S.pb[kt & 1][jl];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
+            if (wg == NWG - 1) {
+                // the bottom quarter holds the column total of this query tile: publish the
+                // inclusive prefix for the next query tile, or, on the last one, b_final
+                const float pinc = fmaf(rk3, above + lam[31], pbj);
+                if (qt == p.nqt - 1) {
+                    if (p.b_final && j < T) p.b_final[(size_t)unit * T + j] = -pinc;
+                } else {
+                    const size_t row = (size_t)unit * p.nqt + qt;
+                    __stcg(p.pincl + row * p.Tp + j, pinc);
+                    __syncwarp();
+                    if (lane == 0) {
+                        __threadfence();
+                        atomicAdd(p.flags + row * p.nqt + kt, 1u);
+                    }
+                }
+            }
             // Lambda in log2 units: -(Pb + r_k^(1/3) * (above + partial sum)) * log2(e)
             const float ka = -rk3 * kLog2e, kb = -fmaf(rk3, above, pbj) * kLog2e;
 #pragma unroll
@@ -717,14 +595,13 @@ static cudaError_t fwd_tc_inst(const CUtensorMap* m, const FwdTcParams& p, cudaS
     const size_t smem = fwd_tc_smem(G);
     cudaError_t e = cudaFuncSetAttribute(k_fwd_tc<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.nqt, p.Hkv, p.B);
     UA_PROFILE("k_fwd_tc", s);
-    k_fwd_tc<G><<<grid, 576, smem, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], p);
+    k_fwd_tc<G><<<p.nqt * p.nunits, 608, smem, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_fwd_tc(const FwdTcLaunch& L, cudaStream_t s) {
-    CUtensorMap m[8];
+    CUtensorMap m[7];
     const int BH = L.B * L.H, BK = L.B * L.Hkv;
     if (!map_rows_bf16(&m[0], L.kh, 64, L.T, BK)) return cudaErrorInvalidValue;
     if (!map_rows_bf16(&m[1], L.kr, 64, L.T, BK)) return cudaErrorInvalidValue;
@@ -733,11 +610,11 @@ cudaError_t launch_fwd_tc(const FwdTcLaunch& L, cudaStream_t s) {
     if (!map_vec_f32(&m[4], L.lq2, L.T, L.Tp, BK)) return cudaErrorInvalidValue;
     if (!map_vec_f32(&m[5], L.lk2, L.T, L.Tp, BK)) return cudaErrorInvalidValue;
     if (!map_vec_f32(&m[6], L.mq, L.T, L.Tp, BH)) return cudaErrorInvalidValue;
-    if (!map_vec_f32(&m[7], L.pb, L.T, L.Tp, BK * L.nqt)) return cudaErrorInvalidValue;
     FwdTcParams p;
     p.B = L.B; p.T = L.T; p.Tp = L.Tp; p.H = L.H; p.Hkv = L.Hkv; p.nqt = L.nqt;
     p.scale_log2e = L.scale * kLog2e;
     p.alpha = L.alpha; p.beta = L.beta; p.g = L.g; p.o = L.o; p.lse = L.lse;
+    p.pincl = L.pincl; p.flags = L.flags; p.b_final = L.b_final; p.nunits = BK;
     switch (L.H / L.Hkv) {
         case 1: return fwd_tc_inst<1>(m, p, s);
         case 2: return fwd_tc_inst<2>(m, p, s);

@@ -60,7 +60,7 @@ FwdWs fwd_ws_layout(const ua_shape* s) {
 // Workspace of the tensor-core prefill forward: bf16 rotated/normalised copies (TMA
 // sources), log2-rates and row bounds (rows padded to Tp), prefixes at 128-row query tiles.
 struct TcWs {
-    size_t qr, kh, kr, lq2, lk2, mq, pb, total;
+    size_t qr, kh, kr, lq2, lk2, mq, pb, flags, flags_bytes, total;
     int Tp, nqt;
 };
 
@@ -79,6 +79,8 @@ TcWs tc_ws_layout(const ua_shape* s) {
     w.lk2 = take(B * Hkv * Tp * 4);
     w.mq = take(B * H * Tp * 4);
     w.pb = take(B * Hkv * (size_t)w.nqt * Tp * 4);
+    w.flags_bytes = (B * Hkv * (size_t)w.nqt * w.nqt + 4) * 4;
+    w.flags = take(w.flags_bytes);
     w.total = off;
     return w;
 }
@@ -211,17 +213,14 @@ static ua_status prefill_fwd_tc(const ua_shape* s, const void* q, const void* k,
     pp.rf = rope_freq(s->rope_theta, s->d);
     if ((st = cuda_status(launch_prep(pp, true, true, cs))) != UA_OK) return st;
 
-    BoundaryParams bp;
-    memset(&bp, 0, sizeof(bp));
-    bp.B = s->B; bp.T = s->T; bp.Hkv = s->Hkv; bp.d = s->d; bp.bq = 128; bp.nqt = w.nqt;
-    bp.alpha = alpha; bp.beta = beta;
-    bp.pb = reinterpret_cast<float*>(at(ws, w.pb)); bp.bfinal = b_final;
-    if ((st = cuda_status(launch_boundary_tc(bp, pp.kh, pp.lq2, pp.lk2, w.Tp, cs))) != UA_OK) return st;
-
+    // the fused forward zeroes its publication counters and ticket itself (stream-ordered)
+    if ((st = cuda_status(cudaMemsetAsync(at(ws, w.flags), 0, w.flags_bytes, cs))) != UA_OK) return st;
     FwdTcLaunch L;
     L.B = s->B; L.T = s->T; L.Tp = w.Tp; L.H = s->H; L.Hkv = s->Hkv; L.nqt = w.nqt; L.scale = s->scale;
-    L.kh = pp.kh; L.kr = pp.kr; L.qr = pp.qr; L.v = v; L.lq2 = pp.lq2; L.lk2 = pp.lk2; L.mq = pp.mq; L.pb = bp.pb;
-    L.alpha = alpha; L.beta = beta; L.g = g; L.o = o; L.lse = lse;
+    L.kh = pp.kh; L.kr = pp.kr; L.qr = pp.qr; L.v = v; L.lq2 = pp.lq2; L.lk2 = pp.lk2; L.mq = pp.mq;
+    L.pincl = reinterpret_cast<float*>(at(ws, w.pb));
+    L.flags = reinterpret_cast<unsigned*>(at(ws, w.flags));
+    L.alpha = alpha; L.beta = beta; L.g = g; L.o = o; L.lse = lse; L.b_final = b_final;
     return cuda_status(launch_fwd_tc(L, cs));
 }
 

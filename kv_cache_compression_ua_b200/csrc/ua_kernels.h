@@ -159,17 +159,17 @@ struct FwdTcLaunch {
     const float* lq2;
     const float* lk2;
     const float* mq;
-    const float* pb;     // [B*Hkv][nqt][Tp], query tiles of 128
+    float* pincl;        // [B*Hkv][nqt][Tp]: per query tile, the inclusive column prefix it publishes
+    unsigned* flags;     // [B*Hkv][nqt][nqt] publication counters, then one ticket counter (zeroed here)
     const float* alpha;
     const float* beta;
     const void* g;
     void* o;
     float* lse;
+    float* b_final;      // [B*Hkv][T] or NULL
 };
 
 bool fwd_tc_supported(int d, int G);
-cudaError_t launch_boundary_tc(const BoundaryParams& bp, const void* kh_bf16, const float* lq2, const float* lk2,
-                               int Tp, cudaStream_t s);
 cudaError_t launch_fwd_tc(const FwdTcLaunch& L, cudaStream_t s);
 
 cudaError_t launch_prep(const PrepParams& p, bool bf16_in, bool bf16_work, cudaStream_t s);

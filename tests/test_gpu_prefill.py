@@ -106,7 +106,7 @@ def test_tensor_core_path_full_parity(B, T, H, Hkv):
     w = I.Workload("tc", B, T, H, Hkv, 64, "bf16", 500 + T + H)
     x = I.make_prefill_inputs(w)
     g, names = kernels_ran(lambda: run_gpu(w, x))
-    assert "k_fwd_tc" in names and "k_boundary_tc" in names, names
+    assert "k_fwd_tc" in names and "k_boundary_tc" not in names, names   # boundary prefixes fused
     assert ua.get_device_status() == 0
     r = oracle.prefill_fwd(**oracle_inputs(x), scale=w.scale, theta=w.theta)
     assert_close("o", g["o"], r["o"], "bf16")
