@@ -93,11 +93,12 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
 
 // ================================================================ fused forward
 // One CTA per (batch, KV head, 128-row query tile) serving all G query heads of the group,
-// so the decay tile is built once for the G heads.  608 threads:
+// so the decay tile is built once for the G heads.  640 threads:
 //   warps 0-15  decay/softmax: warpgroup w = warp/4 owns query rows 32w .. 32w+31 of the
 //               tile; while streaming key tiles, thread = key j (TMEM lane)
 //   warp 16     TMA producer, warp 17 MMA issuer (one elected lane issues for each)
 //   warp 18     boundary look-back: fetches Pb of each key tile from the previous query tile
+//   warp 19     publisher: stores this tile's inclusive prefixes and releases their counters
 // Per key tile kt <= qt:
 //   X^T = Khat_k Khat_q^T and S_h^T = Krope_k Qrope_h^T are computed one 32-row quarter per
 //   warpgroup into that warpgroup's 32-column TMEM slot.  Each thread turns X^T into D and
@@ -111,7 +112,8 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
 // Boundary prefixes without a separate pass: Pb(qt, kt)[j], the sum of D[l, j] over the rows
 // l > j of the query tiles before qt, equals Pb(qt-1, kt) plus the column total of tile qt-1.
 // The bottom quarter of each CTA holds exactly that inclusive prefix after its carry exchange
-// and publishes it to global memory (release: fence, then a per-(tile, key tile) counter);
+// and hands it to the publisher warp, which stores it to global memory and releases it
+// (fence, then a per-(tile, key tile) counter);
 // the next query tile's look-back warp acquires it.  CTAs draw work tickets from a counter in
 // query-tile-major order, so a CTA only ever waits on CTAs with lower tickets, which are
 // already running: the chain always makes progress.  The last query tile writes b_final =
@@ -132,9 +134,10 @@ struct Smem {
     alignas(16) float mq[G][128];                // row bound M_i (log2 units) per head
     alignas(16) float lk[128];                   // lk2 of the key tile
     alignas(16) float pb[2][128];                // boundary prefix Pb of the key tile, two stages
+    alignas(16) float pinc[2][128];              // inclusive prefix handed to the publisher warp
     alignas(16) float tot[2][NWG][128];          // per-quarter column sums (without the key factor)
     alignas(8) uint64_t qfull, khfull, khempty, krfull, krempty, vfull[2], vempty[2], xsfull[NSLOT], xsempty[NSLOT],
-        pfull[2], pempty[2], ofull, cfull[2][NWG], pbfull[2], pbempty[2];
+        pfull[2], pempty[2], ofull, cfull[2][NWG], pbfull[2], pbempty[2], pubfull[2], pubempty[2];
     uint32_t tmem;
     int ticket;
     int abort;
@@ -177,7 +180,7 @@ __device__ __forceinline__ bool wait_counter(const unsigned* f, unsigned target,
 }
 
 template <int G>
-__global__ void __launch_bounds__(608, 1)
+__global__ void __launch_bounds__(640, 1)
 k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_kr,
          const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_v,
          const __grid_constant__ CUtensorMap tm_lq, const __grid_constant__ CUtensorMap tm_lk,
@@ -213,6 +216,8 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             for (int w = 0; w < NWG; ++w) mbar_init(&S.cfull[i][w], 4);   // the four warps of quarter w
             mbar_init(&S.pbfull[i], 1);
             mbar_init(&S.pbempty[i], 4 * NWG);
+            mbar_init(&S.pubfull[i], 4);                // the four warps of the bottom quarter
+            mbar_init(&S.pubempty[i], 1);
         }
         for (int w = 0; w < NSLOT; ++w) {
             mbar_init(&S.xsfull[w], 1);
@@ -288,12 +293,31 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
             if (kt < qt) {
                 const size_t row = (size_t)unit * p.nqt + (qt - 1);
-                if (!wait_counter(p.flags + row * p.nqt + kt, 4u, abort, lane)) break;
+                if (!wait_counter(p.flags + row * p.nqt + kt, 1u, abort, lane)) break;
                 v4 = __ldcg(reinterpret_cast<const float4*>(p.pincl + row * p.Tp + (size_t)kt * 128) + lane);
             }
             *reinterpret_cast<float4*>(&S.pb[sb][lane * 4]) = v4;
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.pbfull[sb]);
+        }
+    } else if (warp == 19) {
+        // ------------------------------------------------ publisher of the inclusive prefixes
+        // Takes the bottom quarter's prefixes from shared memory, stores them, fences (each
+        // lane its own stores) and bumps the (tile, key tile) counter, so the costly fence
+        // never stalls a decay warp.
+        if (qt < p.nqt - 1) {
+            for (int kt = 0; kt < ntile; ++kt) {
+                const int sb = kt & 1;
+                if (!mbar_wait(&S.pubfull[sb], (kt >> 1) & 1, abort)) break;
+                const float4 v4 = *reinterpret_cast<const float4*>(&S.pinc[sb][lane * 4]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.pubempty[sb]);
+                const size_t row = (size_t)unit * p.nqt + qt;
+                __stcg(reinterpret_cast<float4*>(p.pincl + row * p.Tp + (size_t)kt * 128) + lane, v4);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicAdd(p.flags + row * p.nqt + kt, 1u);
+            }
         }
     } else if (warp == 17) {
         // ------------------------------------------------ MMA issuer (warp-uniform, one lane issues)
@@ -482,13 +506,11 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 if (qt == p.nqt - 1) {
                     if (p.b_final && j < T) p.b_final[(size_t)unit * T + j] = -pinc;
                 } else {
-                    const size_t row = (size_t)unit * p.nqt + qt;
-                    __stcg(p.pincl + row * p.Tp + j, pinc);
+                    const int sb = kt & 1;
+                    if (kt >= 2 && !mbar_wait(&S.pubempty[sb], ((kt >> 1) - 1) & 1, abort)) { ok = false; break; }
+                    S.pinc[sb][jl] = pinc;
                     __syncwarp();
-                    if (lane == 0) {
-                        __threadfence();
-                        atomicAdd(p.flags + row * p.nqt + kt, 1u);
-                    }
+                    if (lane == 0) mbar_arrive(&S.pubfull[sb]);
                 }
             }
             // Lambda in log2 units: -(Pb + r_k^(1/3) * (above + partial sum)) * log2(e)
@@ -596,7 +618,7 @@ static cudaError_t fwd_tc_inst(const CUtensorMap* m, const FwdTcParams& p, cudaS
     cudaError_t e = cudaFuncSetAttribute(k_fwd_tc<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     UA_PROFILE("k_fwd_tc", s);
-    k_fwd_tc<G><<<p.nqt * p.nunits, 608, smem, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
+    k_fwd_tc<G><<<p.nqt * p.nunits, 640, smem, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
     return cudaGetLastError();
 }
 
