@@ -330,28 +330,21 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             // one use = two 64-row halves (pair 0: rows 0-63, pair 1: rows 64-127), each into the
             // next slot of the ring: D = A_tile (128 keys) x (rows of the half)^T
             uint32_t nh = 0;                             // half-uses issued
-            auto issue_use = [&](uint32_t a_tile, uint32_t b_tile) -> bool {
-                uint64_t da[4], db[4];
+            // one half-use: rows 64*pr .. 64*pr+63 of the query tile into the next ring slot,
+            // D = A_tile (128 keys) x (rows of the half)^T
+            auto issue_half = [&](uint32_t a_tile, uint32_t b_tile, int pr) -> bool {
+                const uint32_t slot = nh % NSLOT;
+                if (nh >= NSLOT && !mbar_wait(&S.xsempty[slot], ((nh / NSLOT) - 1) & 1, abort)) return false;
+                tc_fence_after();
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    da[kk] = kmajor_desc(a_tile, kk);
-                    db[kk] = kmajor_desc(b_tile, kk);
+                    for (int kk = 0; kk < 4; ++kk)   // half pr starts 64 rows = 8192 B (512 in desc units) further
+                        umma_f16(tmem + COL_XS + slot * 64, kmajor_desc(a_tile, kk),
+                                 kmajor_desc(b_tile, kk) + (uint64_t)(pr * 512), ID_XS, kk > 0);
+                    umma_commit(&S.xsfull[slot]);
                 }
-#pragma unroll
-                for (int pr = 0; pr < 2; ++pr) {
-                    const uint32_t slot = nh % NSLOT;
-                    if (nh >= NSLOT && !mbar_wait(&S.xsempty[slot], ((nh / NSLOT) - 1) & 1, abort)) return false;
-                    tc_fence_after();
-                    if (leader) {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)   // half pr starts 64 rows = 8192 B (512 in desc units) further
-                            umma_f16(tmem + COL_XS + slot * 64, da[kk], db[kk] + (uint64_t)(pr * 512), ID_XS, kk > 0);
-                        umma_commit(&S.xsfull[slot]);
-                    }
-                    __syncwarp();
-                    ++nh;
-                }
-                ++use;
+                __syncwarp();
+                ++nh;
                 return true;
             };
             // descriptors of the two P tiles and the two V stages, k-step 0; k-step kk adds 128 (2048 B)
@@ -378,35 +371,52 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 return true;
             };
             const uint32_t akh = smem_u32(S.kh), akr = smem_u32(S.kr);
+            // Issue order: the upper half (rows 0-63) of each use goes out one step early, ahead of
+            // the PV that waits for every warpgroup, so the upper warpgroups never wait for the
+            // slowest quarter to get their next S.
             if (ok) ok = mbar_wait(&S.khfull, 0, abort);
             if (ok) {
                 tc_fence_after();
-                ok = issue_use(akh, akq);                            // X of the first key tile
+                ok = issue_half(akh, akq, 0) && issue_half(akh, akq, 1);   // X of the first key tile
+            }
+            if (ok) {
                 if (leader) umma_commit(&S.khempty);
                 __syncwarp();
+                ok = mbar_wait(&S.krfull, 0, abort);
+            }
+            if (ok) {
+                tc_fence_after();
+                ok = issue_half(akr, smem_u32(S.q[0]), 0);
             }
             for (int kt = 0; ok && kt < ntile; ++kt) {
                 const int sv = kt & 1;
-                if (!mbar_wait(&S.krfull, kt & 1, abort)) { ok = false; break; }
-                tc_fence_after();
                 for (int h = 0; h < G && ok; ++h) {
-                    if (!issue_use(akr, smem_u32(S.q[h]))) { ok = false; break; }
+                    if (!issue_half(akr, smem_u32(S.q[h]), 1)) { ok = false; break; }
                     if (h == G - 1) {
                         if (leader) umma_commit(&S.krempty);           // last reader of Krope
                         __syncwarp();
                     }
-                    if (h == 1 && !mbar_wait(&S.vfull[sv], (kt >> 1) & 1, abort)) { ok = false; break; }
-                    if (h >= 1 && !issue_pv(h - 1, sv, kt == 0)) { ok = false; break; }
-                    if (h == G - 1 && kt + 1 < ntile) {
-                        // run ahead: X of the next key tile before the last PV of this one
+                    if (h + 1 < G) {
+                        if (!issue_half(akr, smem_u32(S.q[h + 1]), 0)) { ok = false; break; }
+                    } else if (kt + 1 < ntile) {
                         if (!mbar_wait(&S.khfull, (kt + 1) & 1, abort)) { ok = false; break; }
                         tc_fence_after();
-                        if (!issue_use(akh, akq)) { ok = false; break; }
-                        if (leader) umma_commit(&S.khempty);
-                        __syncwarp();
+                        if (!issue_half(akh, akq, 0)) { ok = false; break; }
+                    }
+                    if (h >= 1) {
+                        if (h == 1 && !mbar_wait(&S.vfull[sv], (kt >> 1) & 1, abort)) { ok = false; break; }
+                        if (!issue_pv(h - 1, sv, kt == 0)) { ok = false; break; }
                     }
                 }
                 if (!ok) break;
+                if (kt + 1 < ntile) {
+                    if (!issue_half(akh, akq, 1)) { ok = false; break; }
+                    if (leader) umma_commit(&S.khempty);
+                    __syncwarp();
+                    if (!mbar_wait(&S.krfull, (kt + 1) & 1, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    if (!issue_half(akr, smem_u32(S.q[0]), 0)) { ok = false; break; }
+                }
                 if (G == 1 && !mbar_wait(&S.vfull[sv], (kt >> 1) & 1, abort)) { ok = false; break; }
                 if (!issue_pv(G - 1, sv, kt == 0)) { ok = false; break; }
                 if (leader) {
