@@ -107,7 +107,8 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
 //   above it.  Lambda (log2 units) stays in registers for the quarter's 32 rows.  For each
 //   head, P = 2^(S*scale*log2e + Lambda - M_i) is written MN-major (rows i contiguous) into
 //   the P tile.  M_i = scale*||q_i||*log2e bounds every logit of row i (keys are unit
-//   vectors, Lambda <= 0), so no running maximum and no rescaling are needed.  O_h += P V and
+//   vectors, Lambda <= 0); the shift is the largest M_i of the thread's 32 rows, so no
+//   running maximum, no rescaling and no per-element bound are needed.  O_h += P V and
 //   l_h += P 1 run on the tensor cores with accumulators in TMEM.
 // Boundary prefixes without a separate pass: Pb(qt, kt)[j], the sum of D[l, j] over the rows
 // l > j of the query tiles before qt, equals Pb(qt-1, kt) plus the column total of tile qt-1.
@@ -130,18 +131,30 @@ struct Smem {
     alignas(1024) uint8_t v[2][16384];           // V of the key tile, two stages
     alignas(1024) uint8_t p[2][32768];           // P tiles, MN-major SW128 [2 row blocks][16 k groups][8][128 B]
     alignas(1024) uint8_t ones[1024];            // all-ones bf16 operand for the row sums
-    alignas(16) float lq[128];                   // lq2 of the query rows
-    alignas(16) float mq[G][128];                // row bound M_i (log2 units) per head
-    alignas(16) float lk[128];                   // lk2 of the key tile
+    alignas(128) float lq[128];                   // lq2 of the query rows
+    alignas(128) float mq[G][128];               // row bound M_i (log2 units) per head
+    alignas(128) float lk[128];                   // lk2 of the key tile
     alignas(16) float pb[2][128];                // boundary prefix Pb of the key tile, two stages
     alignas(16) float pinc[2][128];              // inclusive prefix handed to the publisher warp
     alignas(16) float tot[2][NWG][128];          // per-quarter column sums (without the key factor)
+    float shift[4 * NWG][G];                     // per decay warp and head: max M_i over its quarter
     alignas(8) uint64_t qfull, khfull, khempty, krfull, krempty, vfull[2], vempty[2], xsfull[NSLOT], xsempty[NSLOT],
         pfull[2], pempty[2], ofull, cfull[2][NWG], pbfull[2], pbempty[2], pubfull[2], pubempty[2];
     uint32_t tmem;
     int ticket;
     int abort;
 };
+// TMA writes only to 128-byte aligned shared memory (the swizzled tiles need 1024)
+#define UA_TMA_DST(G_, m, a) static_assert(offsetof(Smem<G_>, m) % (a) == 0, "TMA destination alignment")
+#define UA_TMA_DSTS(G_) UA_TMA_DST(G_, kq, 1024); UA_TMA_DST(G_, q, 1024); UA_TMA_DST(G_, kh, 1024); \
+    UA_TMA_DST(G_, kr, 1024); UA_TMA_DST(G_, v, 1024); UA_TMA_DST(G_, lq, 128); UA_TMA_DST(G_, mq, 128); \
+    UA_TMA_DST(G_, lk, 128)
+UA_TMA_DSTS(1);
+UA_TMA_DSTS(2);
+UA_TMA_DSTS(3);
+UA_TMA_DSTS(4);
+#undef UA_TMA_DSTS
+#undef UA_TMA_DST
 }  // namespace fwd
 
 struct FwdTcParams {
@@ -438,6 +451,18 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
         const int r0 = wg * 32;                          // first row of this quarter
         uint32_t use = 0, p_use = 0;
         bool ok = mbar_wait(&S.qfull, 0, abort);
+        // Softmax shift of this quarter: the largest row bound M_i of its 32 rows, one value per
+        // head (each warp keeps its own copy), so no per-element bound is loaded.  Every logit
+        // of the quarter's rows is below it; the shift cancels in O / l and lse adds it back.
+        if (ok) {
+            for (int h = 0; h < G; ++h) {
+                float m = S.mq[h][r0 + lane];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0) S.shift[warp][h] = m;
+            }
+            __syncwarp();
+        }
         // this thread's 32 rows of column jl in a P tile: row block r0/64, chunks (r0%64)/8 + c
         const uint32_t pcol_off = (r0 >> 6) * 16384 + (jl >> 3) * 1024 + (jl & 7) * 128;
         const int ck0 = (r0 & 63) >> 3, sw = jl & 7;
@@ -530,7 +555,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             // ---- per head: P = 2^(S*scale*log2e + Lambda - M_i), causally masked
             for (int h = 0; h < G && ok; ++h) {
                 if (!slot_wait()) { ok = false; break; }
-                const float* mqh = S.mq[h] + r0;
+                const float shh = S.shift[warp][h];
                 // this P tile must be free: the PV of its previous use (two uses back) has completed
                 const uint32_t pbuf = p_use & 1;
                 if (p_use >= 2 && !mbar_wait(&S.pempty[pbuf], ((p_use >> 1) - 1) & 1, abort)) { ok = false; break; }
@@ -543,15 +568,12 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                     for (int cc = 0; cc < 2; ++cc) {
                         const int ck = pc * 2 + cc;
                         uint32_t w4[4];
-                        const float4 m0 = *reinterpret_cast<const float4*>(mqh + ck * 8);
-                        const float4 m1 = *reinterpret_cast<const float4*>(mqh + ck * 8 + 4);
-                        const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
                         for (int e = 0; e < 8; e += 2) {
                             const int r = ck * 8 + e;
                             const int xe = cc * 8 + e;
-                            float p0 = ex2f(fmaf(__uint_as_float(x[xe]), sl, lam[r] - mv[e]));
-                            float p1 = ex2f(fmaf(__uint_as_float(x[xe + 1]), sl, lam[r + 1] - mv[e + 1]));
+                            float p0 = ex2f(fmaf(__uint_as_float(x[xe]), sl, lam[r] - shh));
+                            float p1 = ex2f(fmaf(__uint_as_float(x[xe + 1]), sl, lam[r + 1] - shh));
                             if (diag) {
                                 const int i = qt * 128 + r0 + r;
                                 p0 = (j < T && j <= i) ? p0 : 0.f;
@@ -595,7 +617,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                         Vec16<__nv_bfloat16>::st(oi + c8 * 8, ov);
                     }
                     if (p.lse && wg == 0)
-                        p.lse[((size_t)b * p.H + hq) * T + i] = (S.mq[h][jl] + lg2f(l)) * 0.6931471805599453f;
+                        p.lse[((size_t)b * p.H + hq) * T + i] = (S.shift[4 * wq][h] + lg2f(l)) * 0.6931471805599453f;
                 }
             }
         }
