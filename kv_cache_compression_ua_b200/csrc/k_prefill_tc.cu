@@ -96,9 +96,11 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
 // so the decay tile is built once for the G heads.  640 threads:
 //   warps 0-15  decay/softmax: warpgroup w = warp/4 owns query rows 32w .. 32w+31 of the
 //               tile; while streaming key tiles, thread = key j (TMEM lane)
-//   warp 16     TMA producer, warp 17 MMA issuer (one elected lane issues for each)
-//   warp 18     boundary look-back: fetches Pb of each key tile from the previous query tile
-//   warp 19     publisher: stores this tile's inclusive prefixes and releases their counters
+//   warp 16     TMA producer
+//   warp 17     MMA issuer of the S/X ring, warp 19 MMA issuer of the PV products (one
+//               elected lane issues in each)
+//   warp 18     boundary look-back (fetches Pb of each key tile from the previous query tile)
+//               and publisher (stores this tile's inclusive prefixes, releases their counters)
 // Per key tile kt <= qt:
 //   X^T = Khat_k Khat_q^T and S_h^T = Krope_k Qrope_h^T are computed one 32-row quarter per
 //   warpgroup into that warpgroup's 32-column TMEM slot.  Each thread turns X^T into D and
@@ -113,8 +115,8 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
 // Boundary prefixes without a separate pass: Pb(qt, kt)[j], the sum of D[l, j] over the rows
 // l > j of the query tiles before qt, equals Pb(qt-1, kt) plus the column total of tile qt-1.
 // The bottom quarter of each CTA holds exactly that inclusive prefix after its carry exchange
-// and hands it to the publisher warp, which stores it to global memory and releases it
-// (fence, then a per-(tile, key tile) counter);
+// and hands it to warp 18, which stores it to global memory and releases it (fence, then a
+// per-(tile, key tile) counter);
 // the next query tile's look-back warp acquires it.  CTAs draw work tickets from a counter in
 // query-tile-major order, so a CTA only ever waits on CTAs with lower tickets, which are
 // already running: the chain always makes progress.  The last query tile writes b_final =
@@ -297,51 +299,58 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             __syncwarp();
         }
     } else if (warp == 18) {
-        // ------------------------------------------------ boundary prefixes (look-back)
-        // Pb of key tile kt at this query tile = the inclusive prefix the previous query tile
-        // published for kt (zero on the diagonal): lane l fetches keys 4l .. 4l+3.
-        for (int kt = 0; kt < ntile; ++kt) {
+        // ------------------------------------------------ boundary look-back and publisher
+        // fetch(kt): Pb of key tile kt at this query tile = the inclusive prefix the previous
+        // query tile published for kt (zero on the diagonal); lane l fetches keys 4l .. 4l+3.
+        // publish(kt): takes the bottom quarter's inclusive prefix from shared memory, stores
+        // it, fences (each lane its own stores) and bumps the (tile, key tile) counter, so the
+        // costly fence never stalls a decay warp or an MMA issuer.
+        auto fetch = [&](int kt) -> bool {
             const int sb = kt & 1;
-            if (kt >= 2 && !mbar_wait(&S.pbempty[sb], ((kt >> 1) - 1) & 1, abort)) break;
+            if (kt >= 2 && !mbar_wait(&S.pbempty[sb], ((kt >> 1) - 1) & 1, abort)) return false;
             float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
             if (kt < qt) {
                 const size_t row = (size_t)unit * p.nqt + (qt - 1);
-                if (!wait_counter(p.flags + row * p.nqt + kt, 1u, abort, lane)) break;
+                if (!wait_counter(p.flags + row * p.nqt + kt, 1u, abort, lane)) return false;
                 v4 = __ldcg(reinterpret_cast<const float4*>(p.pincl + row * p.Tp + (size_t)kt * 128) + lane);
             }
             *reinterpret_cast<float4*>(&S.pb[sb][lane * 4]) = v4;
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.pbfull[sb]);
+            return true;
+        };
+        auto publish = [&](int kt) -> bool {
+            const int sb = kt & 1;
+            if (!mbar_wait(&S.pubfull[sb], (kt >> 1) & 1, abort)) return false;
+            const float4 v4 = *reinterpret_cast<const float4*>(&S.pinc[sb][lane * 4]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.pubempty[sb]);
+            const size_t row = (size_t)unit * p.nqt + qt;
+            __stcg(reinterpret_cast<float4*>(p.pincl + row * p.Tp + (size_t)kt * 128) + lane, v4);
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicAdd(p.flags + row * p.nqt + kt, 1u);
+            return true;
+        };
+        // Pb of tile kt is fetched before the prefix of tile kt is published (the decay warps
+        // need the former to form the latter), two stages ahead.
+        bool ok = true;
+        for (int kt = 0; ok && kt < ntile && kt < 2; ++kt) ok = fetch(kt);
+        for (int kt = 0; ok && kt < ntile; ++kt) {
+            if (qt < p.nqt - 1) ok = publish(kt);
+            if (ok && kt + 2 < ntile) ok = fetch(kt + 2);
         }
-    } else if (warp == 19) {
-        // ------------------------------------------------ publisher of the inclusive prefixes
-        // Takes the bottom quarter's prefixes from shared memory, stores them, fences (each
-        // lane its own stores) and bumps the (tile, key tile) counter, so the costly fence
-        // never stalls a decay warp.
-        if (qt < p.nqt - 1) {
-            for (int kt = 0; kt < ntile; ++kt) {
-                const int sb = kt & 1;
-                if (!mbar_wait(&S.pubfull[sb], (kt >> 1) & 1, abort)) break;
-                const float4 v4 = *reinterpret_cast<const float4*>(&S.pinc[sb][lane * 4]);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.pubempty[sb]);
-                const size_t row = (size_t)unit * p.nqt + qt;
-                __stcg(reinterpret_cast<float4*>(p.pincl + row * p.Tp + (size_t)kt * 128) + lane, v4);
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) atomicAdd(p.flags + row * p.nqt + kt, 1u);
-            }
-        }
-    } else if (warp == 17) {
-        // ------------------------------------------------ MMA issuer (warp-uniform, one lane issues)
-        {
-            const bool leader = elect_one();
-            uint32_t use = 0, p_use = 0;                 // slot uses (same for all quarters), P uses
-            bool ok = mbar_wait(&S.qfull, 0, abort);
-            const uint64_t d_ones = smem_desc(smem_u32(S.ones), 256, 128, kSwizzleNone);
-            const uint32_t akq = smem_u32(S.kq);
-            // one use = two 64-row halves (pair 0: rows 0-63, pair 1: rows 64-127), each into the
-            // next slot of the ring: D = A_tile (128 keys) x (rows of the half)^T
+    } else if (warp == 17 || warp == 19) {
+        // ------------------------------------------------ MMA issuers (warp-uniform, one lane issues)
+        // Two independent in-order streams, each in its own warp (a commit tracks only its own
+        // thread's MMAs): warp 17 the S/X ring (X of a key tile, then S of each head, each as
+        // two 64-row halves), warp 19 the PV products.  A ring half never waits behind a PV
+        // that waits for the slowest warpgroup, and vice versa.
+        const bool leader = elect_one();
+        bool ok = true;
+        if (warp == 17) {
+            ok = mbar_wait(&S.qfull, 0, abort);
+            const uint32_t akq = smem_u32(S.kq), akh = smem_u32(S.kh), akr = smem_u32(S.kr);
             uint32_t nh = 0;                             // half-uses issued
             // one half-use: rows 64*pr .. 64*pr+63 of the query tile into the next ring slot,
             // D = A_tile (128 keys) x (rows of the half)^T
@@ -360,78 +369,49 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 ++nh;
                 return true;
             };
+            for (int kt = 0; ok && kt < ntile; ++kt) {
+                if (!mbar_wait(&S.khfull, kt & 1, abort)) break;
+                tc_fence_after();
+                if (!issue_half(akh, akq, 0) || !issue_half(akh, akq, 1)) break;
+                if (leader) umma_commit(&S.khempty);       // X done: Khat of this key tile is free
+                __syncwarp();
+                if (!mbar_wait(&S.krfull, kt & 1, abort)) break;
+                tc_fence_after();
+                for (int h = 0; h < G && ok; ++h)
+                    ok = issue_half(akr, smem_u32(S.q[h]), 0) && issue_half(akr, smem_u32(S.q[h]), 1);
+                if (!ok) break;
+                if (leader) umma_commit(&S.krempty);       // last reader of Krope
+                __syncwarp();
+            }
+        } else {
+            const uint64_t d_ones = smem_desc(smem_u32(S.ones), 256, 128, kSwizzleNone);
             // descriptors of the two P tiles and the two V stages, k-step 0; k-step kk adds 128 (2048 B)
             const uint64_t dpa = smem_desc(smem_u32(S.p[0]), 16384, 1024, kSwizzle128B);
             const uint64_t dpb = smem_desc(smem_u32(S.p[1]), 16384, 1024, kSwizzle128B);
             const uint64_t dva = smem_desc(smem_u32(S.v[0]), 16384, 1024, kSwizzle128B);
             const uint64_t dvb = smem_desc(smem_u32(S.v[1]), 16384, 1024, kSwizzle128B);
-            auto issue_pv = [&](int h, int sv, bool first_tile) -> bool {
-                const uint32_t pbuf = p_use & 1;
-                if (!mbar_wait(&S.pfull[pbuf], (p_use >> 1) & 1, abort)) return false;
-                tc_fence_after();
-                if (leader) {
-                    const uint64_t dp = pbuf ? dpb : dpa, dv = sv ? dvb : dva;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t acc = (!first_tile || kk > 0) ? 1u : 0u;
-                        umma_f16(tmem + COL_O + h * DH, dp + (uint64_t)(kk * 128), dv + (uint64_t)(kk * 128), ID_PV, acc);
-                        umma_f16(tmem + COL_L + h * 16, dp + (uint64_t)(kk * 128), d_ones, ID_L, acc);
-                    }
-                    umma_commit(&S.pempty[pbuf]);
-                }
-                __syncwarp();
-                ++p_use;
-                return true;
-            };
-            const uint32_t akh = smem_u32(S.kh), akr = smem_u32(S.kr);
-            // Issue order: the upper half (rows 0-63) of each use goes out one step early, ahead of
-            // the PV that waits for every warpgroup, so the upper warpgroups never wait for the
-            // slowest quarter to get their next S.
-            if (ok) ok = mbar_wait(&S.khfull, 0, abort);
-            if (ok) {
-                tc_fence_after();
-                ok = issue_half(akh, akq, 0) && issue_half(akh, akq, 1);   // X of the first key tile
-            }
-            if (ok) {
-                if (leader) umma_commit(&S.khempty);
-                __syncwarp();
-                ok = mbar_wait(&S.krfull, 0, abort);
-            }
-            if (ok) {
-                tc_fence_after();
-                ok = issue_half(akr, smem_u32(S.q[0]), 0);
-            }
+            uint32_t p_use = 0;
             for (int kt = 0; ok && kt < ntile; ++kt) {
                 const int sv = kt & 1;
+                if (!mbar_wait(&S.vfull[sv], (kt >> 1) & 1, abort)) break;
                 for (int h = 0; h < G && ok; ++h) {
-                    if (!issue_half(akr, smem_u32(S.q[h]), 1)) { ok = false; break; }
-                    if (h == G - 1) {
-                        if (leader) umma_commit(&S.krempty);           // last reader of Krope
-                        __syncwarp();
+                    const uint32_t pbuf = p_use & 1;
+                    if (!mbar_wait(&S.pfull[pbuf], (p_use >> 1) & 1, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    if (leader) {
+                        const uint64_t dp = pbuf ? dpb : dpa, dv = sv ? dvb : dva;
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
+                            umma_f16(tmem + COL_O + h * DH, dp + (uint64_t)(kk * 128), dv + (uint64_t)(kk * 128), ID_PV, acc);
+                            umma_f16(tmem + COL_L + h * 16, dp + (uint64_t)(kk * 128), d_ones, ID_L, acc);
+                        }
+                        umma_commit(&S.pempty[pbuf]);
                     }
-                    if (h + 1 < G) {
-                        if (!issue_half(akr, smem_u32(S.q[h + 1]), 0)) { ok = false; break; }
-                    } else if (kt + 1 < ntile) {
-                        if (!mbar_wait(&S.khfull, (kt + 1) & 1, abort)) { ok = false; break; }
-                        tc_fence_after();
-                        if (!issue_half(akh, akq, 0)) { ok = false; break; }
-                    }
-                    if (h >= 1) {
-                        if (h == 1 && !mbar_wait(&S.vfull[sv], (kt >> 1) & 1, abort)) { ok = false; break; }
-                        if (!issue_pv(h - 1, sv, kt == 0)) { ok = false; break; }
-                    }
+                    __syncwarp();
+                    ++p_use;
                 }
                 if (!ok) break;
-                if (kt + 1 < ntile) {
-                    if (!issue_half(akh, akq, 1)) { ok = false; break; }
-                    if (leader) umma_commit(&S.khempty);
-                    __syncwarp();
-                    if (!mbar_wait(&S.krfull, (kt + 1) & 1, abort)) { ok = false; break; }
-                    tc_fence_after();
-                    if (!issue_half(akr, smem_u32(S.q[0]), 0)) { ok = false; break; }
-                }
-                if (G == 1 && !mbar_wait(&S.vfull[sv], (kt >> 1) & 1, abort)) { ok = false; break; }
-                if (!issue_pv(G - 1, sv, kt == 0)) { ok = false; break; }
                 if (leader) {
                     umma_commit(&S.vempty[sv]);
                     if (kt == ntile - 1) umma_commit(&S.ofull);
