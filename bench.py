@@ -40,6 +40,16 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # ----------------------------------------------------------------------------- helpers
 
+MUFU_PER_CLK_SM = 16   # transcendental (exp2/log2) results per clock per SM: 4 per SM sub-partition
+N_SM = 148
+
+
+def mufu_ops(w) -> float:
+    """Algorithmic transcendental ops of the bf16 forward: per causal (i, j) pair, 3 per KV head
+    for the decay element and 1 per query head for the softmax numerator."""
+    return w.B * w.T * (w.T + 1) / 2 * (3 * w.Hkv + w.H)
+
+
 def fwd_flops(w) -> float:
     """Algorithmic forward FLOPs, counted once: per causal (i, j) pair and batch, H*4d for
     QK^T and PV of every query head plus Hkv*2d for the key-key similarity."""
@@ -213,20 +223,36 @@ def bench_prefill(args, world, rank, local, peaks, peaks_kind):
     F = fwd_flops(w)
     value = F * world * args.steps / (ms_max * 1e-3) / 1e12
 
-    # dominant kernel roofline (algorithmic FLOPs per launch / measured launch duration)
+    # dominant kernel roofline (algorithmic work per launch / measured launch duration)
     top = max(prof.items(), key=lambda kv: kv[1][1])
     name, (launches, tot_ms) = top
     per_launch_ms = tot_ms / launches
     peak_t = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    achieved = F / (per_launch_ms * 1e-3) / 1e12
-    roofline = {"kernel": name, "bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                "frac": achieved / peak_t, "traffic": None,
-                "peak_source": f"{peaks_kind} bf16 burst (MEASURED_PEAKS.json)" if peaks_kind == "measured"
-                else "fallback 1590 TF/s", "per_launch_ms": per_launch_ms,
-                "share_of_step": tot_ms / sum(v[1] for v in prof.values())}
+    achieved_t = F / (per_launch_ms * 1e-3) / 1e12
+    tensor = {"achieved": achieved_t, "peak": peak_t, "unit": "TFLOP/s", "frac": achieved_t / peak_t,
+              "peak_source": f"{peaks_kind} bf16 burst (MEASURED_PEAKS.json)" if peaks_kind == "measured"
+              else "fallback 1590 TF/s"}
+    clocks = clk.summary()
+    if name == "k_fwd_tc":
+        # The fused forward is bound by the exp2/log2 unit, not the tensor pipe: each causal
+        # (i, j) pair of a KV head needs 3 transcendental ops for the decay element (softplus:
+        # exp and log; cube root: exp of a third of the log) and 1 exp per query head for P.
+        mhz = clocks.get("sm_mhz") or 1965.0
+        peak_a = MUFU_PER_CLK_SM * N_SM * mhz * 1e6 / 1e9
+        achieved_a = mufu_ops(w) / (per_launch_ms * 1e-3) / 1e9
+        roofline = {"kernel": name, "bound": "alu", "achieved": achieved_a, "peak": peak_a,
+                    "unit": "Gop/s (exp2/log2)", "frac": achieved_a / peak_a, "traffic": None,
+                    "peak_source": f"{MUFU_PER_CLK_SM} exp2/log2 results per clock per SM x {N_SM} SMs x "
+                                   f"{mhz:.0f} MHz (median SM clock sampled during the timed region)",
+                    "tensor": tensor}
+    else:
+        roofline = {"kernel": name, "bound": "tensor", "achieved": achieved_t, "peak": peak_t,
+                    "unit": "TFLOP/s", "frac": achieved_t / peak_t, "traffic": None,
+                    "peak_source": tensor["peak_source"]}
+    roofline.update({"per_launch_ms": per_launch_ms, "share_of_step": tot_ms / sum(v[1] for v in prof.values())})
     kernels = {k: {"launches": v[0], "total_ms": v[1], "ms_per_launch": v[1] / v[0]} for k, v in prof.items()}
     gpu_launches = sum(v[0] for v in prof.values())
-    return w, x, value, ms_max / args.steps, roofline, kernels, gpu_launches, clk.summary(), step
+    return w, x, value, ms_max / args.steps, roofline, kernels, gpu_launches, clocks, step
 
 
 def bench_e2e(args, w, x):
