@@ -216,6 +216,7 @@ def bench_prefill(args, world, rank, local, peaks, peaks_kind):
         torch.cuda.synchronize()
     ua.profile_enable(False)
     dist.barrier(world)
+    tiles, skipped = ua.prefill_tile_stats(shape, ws)
     ms = ev0.elapsed_time(ev1)
     ms_max = dist.max_over_ranks(ms, world)
     prof = ua.profile_read()
@@ -228,7 +229,10 @@ def bench_prefill(args, world, rank, local, peaks, peaks_kind):
     name, (launches, tot_ms) = top
     per_launch_ms = tot_ms / launches
     peak_t = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    achieved_t = F / (per_launch_ms * 1e-3) / 1e12
+    # Tiles whose probabilities all underflow skip their QK^T and PV products (an exactly zero
+    # contribution): `value` counts the dense algorithmic FLOPs, the roofline what executed.
+    f_skip = skipped * 128 * 128 * (w.H // w.Hkv) * 4 * w.d
+    achieved_t = (F - f_skip) / (per_launch_ms * 1e-3) / 1e12
     tensor = {"achieved": achieved_t, "peak": peak_t, "unit": "TFLOP/s", "frac": achieved_t / peak_t,
               "peak_source": f"{peaks_kind} bf16 burst (MEASURED_PEAKS.json)" if peaks_kind == "measured"
               else "fallback 1590 TF/s"}
@@ -239,7 +243,9 @@ def bench_prefill(args, world, rank, local, peaks, peaks_kind):
         # exp and log; cube root: exp of a third of the log) and 1 exp per query head for P.
         mhz = clocks.get("sm_mhz") or 1965.0
         peak_a = MUFU_PER_CLK_SM * N_SM * mhz * 1e6 / 1e9
-        achieved_a = mufu_ops(w) / (per_launch_ms * 1e-3) / 1e9
+        # executed transcendental ops: the softmax exps of skipped tiles are not evaluated
+        ops = mufu_ops(w) - skipped * 128 * 128 * (w.H // w.Hkv)
+        achieved_a = ops / (per_launch_ms * 1e-3) / 1e9
         roofline = {"kernel": name, "bound": "alu", "achieved": achieved_a, "peak": peak_a,
                     "unit": "Gop/s (exp2/log2)", "frac": achieved_a / peak_a, "traffic": None,
                     "peak_source": f"{MUFU_PER_CLK_SM} exp2/log2 results per clock per SM x {N_SM} SMs x "
@@ -250,6 +256,8 @@ def bench_prefill(args, world, rank, local, peaks, peaks_kind):
                     "unit": "TFLOP/s", "frac": achieved_t / peak_t, "traffic": None,
                     "peak_source": tensor["peak_source"]}
     roofline.update({"per_launch_ms": per_launch_ms, "share_of_step": tot_ms / sum(v[1] for v in prof.values())})
+    roofline["tiles"] = {"causal": tiles, "softmax_skipped": skipped,
+                         "executed_tflops": (F - f_skip) * world * args.steps / (ms_max * 1e-3) / 1e12}
     kernels = {k: {"launches": v[0], "total_ms": v[1], "ms_per_launch": v[1] / v[0]} for k, v in prof.items()}
     gpu_launches = sum(v[0] for v in prof.values())
     return w, x, value, ms_max / args.steps, roofline, kernels, gpu_launches, clocks, step

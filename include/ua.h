@@ -96,7 +96,12 @@ ua_status ua_prefill_workspace_size(const ua_shape* shape, size_t* bytes);
  * TMA).  That path shifts every softmax row by the a-priori bound scale*||q_i|| (the keys
  * are unit vectors and Lambda <= 0, so no logit exceeds it) instead of a running maximum; a
  * row whose true maximum lies more than ~87 below that bound (scale*||q_i|| > ~43) would
- * underflow, and then UA_ERR_RANGE is raised in the device status word.  All other problems,
+ * underflow, and then UA_ERR_RANGE is raised in the device status word.  The same path skips
+ * the softmax and PV work of every 128 x 128 (query tile, key tile) whose decay prefix
+ * makes all its probabilities underflow to exactly 0 in fp32 (Lambda only decreases down a
+ * key column, so the prefix above the tile bounds the whole tile); the decay of the tile is
+ * still evaluated, so b_final and all outputs are identical to the unskipped computation
+ * (see ua_prefill_tile_stats).  All other problems,
  * and every call that asks for lambda_dbg, run the fp32 SIMT path, which uses a running
  * maximum. */
 ua_status ua_prefill_fwd(const ua_shape* shape, const void* q, const void* k, const void* v,
@@ -125,6 +130,16 @@ ua_status ua_prefill_fwd_noalloc(const ua_shape* shape, const void* q, const voi
 
 /* Size in bytes of the array ua_prefill_fwd_noalloc uses (the largest workspace it serves). */
 size_t ua_prefill_noalloc_max_scratch(void);
+
+/* ------------------------------------------------------------------ prefill tile statistics
+ * No counterpart on the pages: a measurement aid for the tile skipping described at
+ * ua_prefill_fwd.  Synchronises `stream` and reports, for the most recent ua_prefill_fwd
+ * (without lambda_dbg) that used workspace `ws` for `shape`, the number of causal
+ * 128 x 128 tiles, B*Hkv*n*(n+1)/2 with n = ceil(T/128), in *tiles, and how many of them
+ * skipped the softmax in *skipped.  Problems that run the fp32 SIMT path report
+ * *skipped = 0.  Not available for the allocation-free entry point. */
+ua_status ua_prefill_tile_stats(const ua_shape* shape, const void* ws, size_t ws_bytes,
+                                unsigned long long* tiles, unsigned long long* skipped, void* stream);
 
 /* ------------------------------------------------------------------ prefill backward
  * Gradient of sum(dO * O) with respect to every input of ua_prefill_fwd (the backward of

@@ -23,6 +23,10 @@ using namespace tc;
 
 namespace {
 constexpr float kLog2e = 1.4426950408889634f;
+// A (query tile, key tile) is skipped when Pb*log2(e) >= kSkipLog2 for all its keys: then every
+// exponent S*scale*log2e + Lambda - shift of the tile is <= -126 (S*scale*log2e - shift <= 0 up to
+// bf16 rounding of the operands, Lambda <= -Pb), so ex2.approx.ftz returns exactly 0 for every P.
+constexpr float kSkipLog2 = 128.f;
 
 // --------------------------------------------------------------- tensor maps (host)
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -137,6 +141,7 @@ struct Smem {
     alignas(128) float mq[G][128];               // row bound M_i (log2 units) per head
     alignas(128) float lk[128];                   // lk2 of the key tile
     alignas(16) float pb[2][128];                // boundary prefix Pb of the key tile, two stages
+    int pbskip[2];                               // 1: every P of this (query tile, key tile) underflows
     alignas(16) float pinc[2][128];              // inclusive prefix handed to the publisher warp
     alignas(16) float tot[2][NWG][128];          // per-quarter column sums (without the key factor)
     float shift[4 * NWG][G];                     // per decay warp and head: max M_i over its quarter
@@ -230,7 +235,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             mbar_init(&S.pempty[i], 1);
             for (int w = 0; w < NWG; ++w) mbar_init(&S.cfull[i][w], 4);   // the four warps of quarter w
             mbar_init(&S.pbfull[i], 1);
-            mbar_init(&S.pbempty[i], 4 * NWG);
+            mbar_init(&S.pbempty[i], 4 * NWG + 2);      // decay warps and both MMA issuers
             mbar_init(&S.pubfull[i], 4);                // the four warps of the bottom quarter
             mbar_init(&S.pubempty[i], 1);
         }
@@ -309,12 +314,21 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             const int sb = kt & 1;
             if (kt >= 2 && !mbar_wait(&S.pbempty[sb], ((kt >> 1) - 1) & 1, abort)) return false;
             float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            int skip = 0;
             if (kt < qt) {
                 const size_t row = (size_t)unit * p.nqt + (qt - 1);
                 if (!wait_counter(p.flags + row * p.nqt + kt, 1u, abort, lane)) return false;
                 v4 = __ldcg(reinterpret_cast<const float4*>(p.pincl + row * p.Tp + (size_t)kt * 128) + lane);
+                float mn = fminf(fminf(v4.x, v4.y), fminf(v4.z, v4.w));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                skip = (mn * kLog2e >= kSkipLog2) ? 1 : 0;
             }
             *reinterpret_cast<float4*>(&S.pb[sb][lane * 4]) = v4;
+            if (lane == 0) {
+                S.pbskip[sb] = skip;
+                if (skip) atomicAdd(p.flags + (size_t)p.nunits * p.nqt * p.nqt + 1, 1u);
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.pbfull[sb]);
             return true;
@@ -375,9 +389,13 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 if (!issue_half(akh, akq, 0) || !issue_half(akh, akq, 1)) break;
                 if (leader) umma_commit(&S.khempty);       // X done: Khat of this key tile is free
                 __syncwarp();
+                if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) break;
+                const bool skip = S.pbskip[kt & 1] != 0;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
                 if (!mbar_wait(&S.krfull, kt & 1, abort)) break;
                 tc_fence_after();
-                for (int h = 0; h < G && ok; ++h)
+                for (int h = 0; h < G && ok && !skip; ++h)
                     ok = issue_half(akr, smem_u32(S.q[h]), 0) && issue_half(akr, smem_u32(S.q[h]), 1);
                 if (!ok) break;
                 if (leader) umma_commit(&S.krempty);       // last reader of Krope
@@ -391,10 +409,15 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             const uint64_t dva = smem_desc(smem_u32(S.v[0]), 16384, 1024, kSwizzle128B);
             const uint64_t dvb = smem_desc(smem_u32(S.v[1]), 16384, 1024, kSwizzle128B);
             uint32_t p_use = 0;
+            bool first = true;                           // no PV issued yet: the first one initialises O
             for (int kt = 0; ok && kt < ntile; ++kt) {
                 const int sv = kt & 1;
+                if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) break;
+                const bool skip = S.pbskip[kt & 1] != 0;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
                 if (!mbar_wait(&S.vfull[sv], (kt >> 1) & 1, abort)) break;
-                for (int h = 0; h < G && ok; ++h) {
+                for (int h = 0; h < G && ok && !skip; ++h) {
                     const uint32_t pbuf = p_use & 1;
                     if (!mbar_wait(&S.pfull[pbuf], (p_use >> 1) & 1, abort)) { ok = false; break; }
                     tc_fence_after();
@@ -402,7 +425,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                         const uint64_t dp = pbuf ? dpb : dpa, dv = sv ? dvb : dva;
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
+                            const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
                             umma_f16(tmem + COL_O + h * DH, dp + (uint64_t)(kk * 128), dv + (uint64_t)(kk * 128), ID_PV, acc);
                             umma_f16(tmem + COL_L + h * 16, dp + (uint64_t)(kk * 128), d_ones, ID_L, acc);
                         }
@@ -412,6 +435,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                     ++p_use;
                 }
                 if (!ok) break;
+                if (!skip) first = false;
                 if (leader) {
                     umma_commit(&S.vempty[sv]);
                     if (kt == ntile - 1) umma_commit(&S.ofull);
@@ -512,6 +536,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             if (!ok) break;
             if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) { ok = false; break; }
             const float pbj = S.pb[kt & 1][jl];
+            const bool skip = S.pbskip[kt & 1] != 0;
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
             if (wg == NWG - 1) {
@@ -528,6 +553,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                     if (lane == 0) mbar_arrive(&S.pubfull[sb]);
                 }
             }
+            if (skip) continue;                          // every P of this tile is exactly 0
             // Lambda in log2 units: -(Pb + r_k^(1/3) * (above + partial sum)) * log2(e)
             const float ka = -rk3 * kLog2e, kb = -fmaf(rk3, above, pbj) * kLog2e;
 #pragma unroll

@@ -427,6 +427,28 @@ ua_status ua_decode_step(const ua_cache* c, int H, const void* q, const void* k,
     return cuda_status(launch_decode(dp, c->dtype == UA_BF16, static_cast<cudaStream_t>(stream)));
 }
 
+ua_status ua_prefill_tile_stats(const ua_shape* s, const void* ws, size_t ws_bytes, unsigned long long* tiles,
+                                unsigned long long* skipped, void* stream) {
+    if (!s || !tiles || !skipped) return UA_ERR_INVALID_ARG;
+    if (s->B <= 0 || s->T <= 0 || s->Hkv <= 0) return UA_ERR_INVALID_ARG;
+    const unsigned long long n = (unsigned long long)((s->T + 127) / 128);
+    *tiles = (unsigned long long)s->B * s->Hkv * n * (n + 1) / 2;
+    *skipped = 0;
+    if (!use_tc(s)) return UA_OK;
+    const TcWs w = tc_ws_layout(s);
+    if (!ws) return UA_ERR_INVALID_ARG;
+    if (ws_bytes < w.total) return UA_ERR_WORKSPACE;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    unsigned host = 0;
+    const size_t off = w.flags + ((size_t)s->B * s->Hkv * w.nqt * w.nqt + 1) * sizeof(unsigned);
+    cudaError_t e = cudaMemcpyAsync(&host, static_cast<const uint8_t*>(ws) + off, sizeof(unsigned),
+                                    cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return UA_ERR_CUDA;
+    *skipped = host;
+    return UA_OK;
+}
+
 ua_status ua_get_device_status(void* stream, int* code) {
     if (!code) return UA_ERR_INVALID_ARG;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);

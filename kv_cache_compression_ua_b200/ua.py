@@ -44,7 +44,7 @@ class ua_cache(ctypes.Structure):
 EXPORTS = ("ua_prefill_workspace_size", "ua_prefill_fwd", "ua_prefill_bwd_workspace_size", "ua_prefill_bwd",
            "ua_cache_fill", "ua_cache_compact", "ua_decode_step", "ua_get_device_status",
            "ua_profile_enable", "ua_profile_reset", "ua_profile_read", "ua_status_string", "ua_version",
-           "ua_prefill_fwd_noalloc", "ua_prefill_noalloc_max_scratch")
+           "ua_prefill_fwd_noalloc", "ua_prefill_noalloc_max_scratch", "ua_prefill_tile_stats")
 
 
 class ua_kernel_time(ctypes.Structure):
@@ -78,6 +78,8 @@ def load_library(path: str = LIB_PATH):
     lib.ua_profile_read.argtypes = [ctypes.POINTER(ua_kernel_time), I, ctypes.POINTER(I)]
     lib.ua_prefill_fwd_noalloc.argtypes = [SP] + [P] * 8 + [P, P, P, P]
     lib.ua_prefill_noalloc_max_scratch.argtypes = []
+    lib.ua_prefill_tile_stats.argtypes = [SP, P, S, ctypes.POINTER(ctypes.c_ulonglong),
+                                          ctypes.POINTER(ctypes.c_ulonglong), P]
     lib.ua_prefill_noalloc_max_scratch.restype = S
     lib.ua_status_string.argtypes = [I]
     lib.ua_status_string.restype = ctypes.c_char_p
@@ -156,6 +158,15 @@ def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0
                             _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(stream))
     _check("ua_prefill_fwd", rc)
     return {"o": o, "lse": lse, "b_final": bfin, "lam": lam}
+
+
+def prefill_tile_stats(shape: ua_shape, ws: torch.Tensor, stream=None) -> tuple:
+    """ua_prefill_tile_stats: (causal tiles, tiles whose softmax was skipped) of the last
+    ua_prefill_fwd that used `ws` for `shape`."""
+    tiles, skipped = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+    _check("ua_prefill_tile_stats", load_library().ua_prefill_tile_stats(
+        ctypes.byref(shape), _ptr(ws), ws.numel(), ctypes.byref(tiles), ctypes.byref(skipped), _stream(stream)))
+    return tiles.value, skipped.value
 
 
 def prefill_fwd_noalloc(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0, want_lse=True,

@@ -114,6 +114,42 @@ def test_tensor_core_path_full_parity(B, T, H, Hkv):
     assert_close("b_final", g["b_final"], r["b_final"], "bf16", relative_max=True)
 
 
+SKIP_SHAPES = [
+    # (B, T, H, Hkv, rate shift): strong decay, so most off-diagonal tiles underflow
+    (1, 1000, 4, 1, 4.0),
+    (2, 700, 8, 2, 3.0),
+    (1, 1100, 4, 2, 2.0),
+]
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,shift", SKIP_SHAPES)
+def test_tensor_core_underflow_tile_skipping_is_exact(B, T, H, Hkv, shift):
+    """Rates shifted up (stronger decay): the tensor-core path skips the softmax of tiles whose
+    decay prefix underflows every probability.  Skipping must occur, and every output must
+    still match the oracle as the dense computation does (b_final included: the decay of a
+    skipped tile is still evaluated)."""
+    w = I.Workload("skip", B, T, H, Hkv, 64, "bf16", 700 + T)
+    x = I.make_prefill_inputs(w)
+    x["a_q"] = x["a_q"] + shift
+    x["a_k"] = x["a_k"] + shift
+    d = to_dev(oracle_inputs(x), w)
+    shape = ua.make_shape(d["q"], d["k"], w.scale, w.theta)
+    ws = ua.alloc_workspace(ua.prefill_workspace_size(shape), "cuda")
+    r_gpu = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
+                           scale=w.scale, theta=w.theta, ws=ws)
+    tiles, skipped = ua.prefill_tile_stats(shape, ws)
+    assert ua.get_device_status() == 0
+    n = (T + 127) // 128
+    assert tiles == B * Hkv * n * (n + 1) // 2
+    off_diag = B * Hkv * n * (n - 1) // 2
+    assert skipped >= max(1, off_diag // 8), (skipped, off_diag)
+    g = {k: v.float().cpu().numpy() for k, v in r_gpu.items() if v is not None}
+    r = oracle.prefill_fwd(**oracle_inputs(x), scale=w.scale, theta=w.theta)
+    assert_close("o", g["o"], r["o"], "bf16")
+    assert_close("lse", g["lse"], r["lse"], "bf16", relative_max=True)
+    assert_close("b_final", g["b_final"], r["b_final"], "bf16", relative_max=True)
+
+
 def test_tensor_core_path_veto_and_plain_attention():
     w = I.Workload("tcveto", 1, 300, 4, 1, 64, "bf16", 17)
     x = I.make_prefill_inputs(w)
