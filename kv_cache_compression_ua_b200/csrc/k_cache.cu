@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(256) k_cache_compact(CompactParams p) {
 // grid (B*Hkv), 256 threads.  Dynamic shared memory: eviction bitmap (ceil(cap/32) words)
 // followed by the per-group softmax partials.
 template <typename TC, int DH, int G>
-__global__ void __launch_bounds__(256) k_decode(DecodeParams p) {
+__global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) {
     using L = EntryLayout<TC, DH>;
     constexpr int VEC = L::VEC, LPE = L::LPE, EPB = L::EPB, NW = L::NW;
     constexpr int half = DH / 2;
@@ -190,15 +190,45 @@ __global__ void __launch_bounds__(256) k_decode(DecodeParams p) {
     const int grp = lane / LPE, gl = lane % LPE;
     const int gidx = warp * L::EPW + grp;             // entry group index in the pass
     const size_t base = (size_t)unit * c.cap;
+    TC* khat = static_cast<TC*>(c.khat);
+    TC* krope = static_cast<TC*>(c.krope);
+    TC* vc = static_cast<TC*>(c.v);
 
-    // ---- new token: khat_t, RoPE(khat_t), v_t, RoPE(q_h), rates
+    // ---- Every load that depends on no other goes out first (the live count, the new token,
+    // its gate and the rates), so a step over a pruned, tiny cache does not pay a chain of
+    // memory round trips before its arithmetic.  (Prefetching the first pass of cache entries
+    // as well was measured slower: the registers it holds cost occupancy.)
+    int n = c.n_kept[unit];
     const TC* kin = static_cast<const TC*>(p.k) + (size_t)unit * DH;
     const TC* vin = static_cast<const TC*>(p.v) + (size_t)unit * DH;
-    float kx = 0.f;
+    const TC* qin = static_cast<const TC*>(p.q) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
+    const TC* gin = static_cast<const TC*>(p.g) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
+    constexpr int QE = (G * half + 255) / 256, GE = (G * DH + 255) / 256;
+    float kx = 0.f, vx = 0.f;
     if (tid < DH) {
         kx = Elem<TC>::ld(kin + tid);
-        s_vt[tid] = Elem<TC>::ld(vin + tid);
+        vx = Elem<TC>::ld(vin + tid);
     }
+    float qa[QE], qb[QE], gv[GE];
+#pragma unroll
+    for (int r = 0; r < QE; ++r) {
+        const int e = tid + 256 * r;
+        qa[r] = qb[r] = 0.f;
+        if (e < G * half) {
+            const int vecid = e / half, m = e % half;
+            qa[r] = Elem<TC>::ld(qin + vecid * DH + m);
+            qb[r] = Elem<TC>::ld(qin + vecid * DH + m + half);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < GE; ++r) {
+        const int e = tid + 256 * r;
+        gv[r] = e < G * DH ? Elem<TC>::ld(gin + e) : 0.f;
+    }
+    const float aq_t = p.a_q[unit], ak_t = p.a_k[unit];
+    const float al = p.alpha[kvh], be = p.beta[kvh];
+
+    // ---- new token: khat_t, RoPE(khat_t), v_t, RoPE(q_h), rates
     float ss = kx * kx;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -209,22 +239,28 @@ __global__ void __launch_bounds__(256) k_decode(DecodeParams p) {
 #pragma unroll
     for (int w = 0; w < NW; ++w) tot_ss += s_red[w];
     const float den = fmaxf(sqrtf(tot_ss), 1e-12f);
-    if (tid < DH) s_kt[tid] = kx / den;
+    if (tid < DH) {
+        s_kt[tid] = kx / den;
+        s_vt[tid] = vx;
+    }
     __syncthreads();
-    const TC* qin = static_cast<const TC*>(p.q) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
-    for (int e = tid; e < (G + 1) * half; e += blockDim.x) {
-        const int vecid = e / half, m = e % half;
+#pragma unroll
+    for (int r = 0; r < QE; ++r) {
+        const int e = tid + 256 * r;
+        if (e < G * half) {
+            const int vecid = e / half, m = e % half;
+            float cs, sn;
+            rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
+            s_q[vecid][m] = qa[r] * cs - qb[r] * sn;
+            s_q[vecid][m + half] = qb[r] * cs + qa[r] * sn;
+        }
+    }
+    for (int m = tid; m < half; m += blockDim.x) {
         float cs, sn;
         rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
-        if (vecid < G) {
-            const float x0 = Elem<TC>::ld(qin + vecid * DH + m), x1 = Elem<TC>::ld(qin + vecid * DH + m + half);
-            s_q[vecid][m] = x0 * cs - x1 * sn;
-            s_q[vecid][m + half] = x1 * cs + x0 * sn;
-        } else {
-            const float x0 = s_kt[m], x1 = s_kt[m + half];
-            s_ktr[m] = x0 * cs - x1 * sn;
-            s_ktr[m + half] = x1 * cs + x0 * sn;
-        }
+        const float x0 = s_kt[m], x1 = s_kt[m + half];
+        s_ktr[m] = x0 * cs - x1 * sn;
+        s_ktr[m + half] = x1 * cs + x0 * sn;
     }
     __syncthreads();
     if (tid < G) {
@@ -232,9 +268,8 @@ __global__ void __launch_bounds__(256) k_decode(DecodeParams p) {
         for (int x = 0; x < DH; ++x) a = fmaf(s_q[tid][x], s_ktr[x], a);
         s_lt[tid] = a * p.scale;                      // new token's own bias is 0
     }
-    const float rq_t = softplus_f(p.a_q[unit]);
-    const float rk_t = softplus_f(p.a_k[unit]);
-    const float al = p.alpha[kvh], be = p.beta[kvh];
+    const float rq_t = softplus_f(aq_t);
+    const float rk_t = softplus_f(ak_t);
 
     float kq[VEC], qh[G][VEC];
 #pragma unroll
@@ -252,10 +287,6 @@ __global__ void __launch_bounds__(256) k_decode(DecodeParams p) {
         for (int e = 0; e < VEC; ++e) acc[h][e] = 0.f;
     }
 
-    TC* khat = static_cast<TC*>(c.khat);
-    TC* krope = static_cast<TC*>(c.krope);
-    TC* vc = static_cast<TC*>(c.v);
-    int n = c.n_kept[unit];
     if (n < 0 || n > c.cap) {                 // corrupt count: never read past the cache
         if (tid == 0) raise_status(UA_ERR_CAPACITY);
         n = n < 0 ? 0 : c.cap;
@@ -340,9 +371,11 @@ __global__ void __launch_bounds__(256) k_decode(DecodeParams p) {
 #pragma unroll
         for (int e = 0; e < VEC; ++e) s_acc[((size_t)gidx * G + h) * DH + gl * VEC + e] = acc[h][e];
     __syncthreads();
-    const TC* gin = static_cast<const TC*>(p.g) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     TC* oout = static_cast<TC*>(p.o) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
-    for (int e = tid; e < G * DH; e += blockDim.x) {
+#pragma unroll
+    for (int r = 0; r < GE; ++r) {
+        const int e = tid + 256 * r;
+        if (e >= G * DH) break;
         const int h = e / DH, x = e % DH;
         float M = s_lt[h];
         for (int q = 0; q < EPB; ++q) M = fmaxf(M, s_m[q * G + h]);
@@ -353,7 +386,7 @@ __global__ void __launch_bounds__(256) k_decode(DecodeParams p) {
             Ls = fmaf(s_l[q * G + h], w, Ls);
             A = fmaf(s_acc[((size_t)q * G + h) * DH + x], w, A);
         }
-        Elem<TC>::st(oout + e, A / Ls * sigmoid_f(Elem<TC>::ld(gin + e)));
+        Elem<TC>::st(oout + e, A / Ls * sigmoid_f(gv[r]));
     }
     // ---- eviction bits, append the new token
     if (p.evict_bits)
