@@ -125,6 +125,49 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
 // query-tile-major order, so a CTA only ever waits on CTAs with lower tickets, which are
 // already running: the chain always makes progress.  The last query tile writes b_final =
 // -(its inclusive prefix) = Lambda_{T-1, j}.
+// 16 rows of one key column of the decay tile: D (without the key factor) from the
+// similarity x and the row's lq2, scanned into c; lam[r] = the running sum after row r.
+// MASK: only rows rlo <= r < rhi accumulate (the causal diagonal and the sequence end).
+template <bool MASK>
+__device__ __forceinline__ void decay16(const uint32_t (&x)[16], const float (&lv)[16], int pc, int rlo, int rhi,
+                                        float al, float be, float& c, float (&lam)[32]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const int r = pc * 16 + e;
+        const float dq = ex2f(fmaf(log2_softplus_poly(fmaf(al, __uint_as_float(x[e]), be)), 0.33333334f, lv[e]));
+        if (MASK) c += (r >= rlo && r < rhi) ? dq : 0.f;
+        else c += dq;
+        lam[r] = c;
+    }
+}
+
+// 16 rows of one key column of P for one head: P = 2^(S*scale*log2e + Lambda - shift), packed
+// to bf16 and stored MN-major into the P tile (two 16-byte chunks of 8 rows).  MASK: only
+// rows r >= rlo of a valid key are kept (the causal diagonal, keys past the sequence end).
+template <bool MASK>
+__device__ __forceinline__ void probs16(const uint32_t (&x)[16], int pc, float sl, const float (&lam)[32], float shh,
+                                        bool jvalid, int rlo, uint8_t* pcol, int ck0, int sw) {
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+        const int ck = pc * 2 + cc;
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            const int r = ck * 8 + e;
+            const int xe = cc * 8 + e;
+            float p0 = ex2f(fmaf(__uint_as_float(x[xe]), sl, lam[r] - shh));
+            float p1 = ex2f(fmaf(__uint_as_float(x[xe + 1]), sl, lam[r + 1] - shh));
+            if (MASK) {
+                p0 = (jvalid && r >= rlo) ? p0 : 0.f;
+                p1 = (jvalid && r + 1 >= rlo) ? p1 : 0.f;
+            }
+            __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+            w4[e >> 1] = *reinterpret_cast<uint32_t*>(&pr);
+        }
+        *reinterpret_cast<uint4*>(pcol + (((ck0 + ck) ^ sw) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+}
+
 namespace fwd {
 constexpr int NWG = 4;   // decay warpgroups (32 query rows each)
 constexpr int NSLOT = 3; // TMEM ring of 64-column half tiles (each half serves a pair of warpgroups)
@@ -504,6 +547,11 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             {
                 if (!slot_wait()) { ok = false; break; }
                 float c = 0.f;
+                // rows r of the quarter that accumulate: row > j on the diagonal tile, row < T on
+                // the last query tile (uniform per tile, so the common tile runs unmasked)
+                const bool masked = diag || tailq;
+                const int rlo = diag ? j - (qt * 128 + r0) + 1 : 0;
+                const int rhi = tailq ? T - (qt * 128 + r0) : 32;
 #pragma unroll
                 for (int pc = 0; pc < 2; ++pc) {
                     uint32_t x[16];
@@ -514,15 +562,8 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                         const float4 t4 = *reinterpret_cast<const float4*>(lqh + pc * 16 + e);
                         lv[e] = t4.x; lv[e + 1] = t4.y; lv[e + 2] = t4.z; lv[e + 3] = t4.w;
                     }
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int r = pc * 16 + e;
-                        const float dq = ex2f(fmaf(log2_softplus_poly(fmaf(al, __uint_as_float(x[e]), be)),
-                                                   0.33333334f, lv[e]));
-                        const int row = qt * 128 + r0 + r;
-                        c += (!(diag || tailq) || (row > j && row < T)) ? dq : 0.f;
-                        lam[r] = c;
-                    }
+                    if (masked) decay16<true>(x, lv, pc, rlo, rhi, al, be, c, lam);
+                    else decay16<false>(x, lv, pc, rlo, rhi, al, be, c, lam);
                 }
                 S.tot[kt & 1][wg][jl] = c;
             }
@@ -566,31 +607,13 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 const uint32_t pbuf = p_use & 1;
                 if (p_use >= 2 && !mbar_wait(&S.pempty[pbuf], ((p_use >> 1) - 1) & 1, abort)) { ok = false; break; }
                 uint8_t* pcol = S.p[pbuf] + pcol_off;
+                const int rlo = j - (qt * 128 + r0);      // first row of the quarter with i >= j
 #pragma unroll
                 for (int pc = 0; pc < 2; ++pc) {
                     uint32_t x[16];
                     slot_read(pc, x);
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        const int ck = pc * 2 + cc;
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int e = 0; e < 8; e += 2) {
-                            const int r = ck * 8 + e;
-                            const int xe = cc * 8 + e;
-                            float p0 = ex2f(fmaf(__uint_as_float(x[xe]), sl, lam[r] - shh));
-                            float p1 = ex2f(fmaf(__uint_as_float(x[xe + 1]), sl, lam[r + 1] - shh));
-                            if (diag) {
-                                const int i = qt * 128 + r0 + r;
-                                p0 = (j < T && j <= i) ? p0 : 0.f;
-                                p1 = (j < T && j <= i + 1) ? p1 : 0.f;
-                            }
-                            __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-                            w4[e >> 1] = *reinterpret_cast<uint32_t*>(&pr);
-                        }
-                        *reinterpret_cast<uint4*>(pcol + (((ck0 + ck) ^ sw) << 4)) =
-                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    }
+                    if (diag) probs16<true>(x, pc, sl, lam, shh, j < T, rlo, pcol, ck0, sw);
+                    else probs16<false>(x, pc, sl, lam, shh, true, 0, pcol, ck0, sw);
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
