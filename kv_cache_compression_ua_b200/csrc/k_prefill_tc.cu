@@ -23,6 +23,7 @@ using namespace tc;
 
 namespace {
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kCbrtLn2 = 0.8849970445005177f;   // (ln 2)^(1/3): the decay evaluated in log2 units
 // A (query tile, key tile) is skipped when Pb*log2(e) >= kSkipLog2 for all its keys: then every
 // exponent S*scale*log2e + Lambda - shift of the tile is <= -126 (S*scale*log2e - shift <= 0 up to
 // bf16 rounding of the operands, Lambda <= -Pb), so ex2.approx.ftz returns exactly 0 for every P.
@@ -125,27 +126,30 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
 // query-tile-major order, so a CTA only ever waits on CTAs with lower tickets, which are
 // already running: the chain always makes progress.  The last query tile writes b_final =
 // -(its inclusive prefix) = Lambda_{T-1, j}.
-// 16 rows of one key column of the decay tile: D (without the key factor) from the
-// similarity x and the row's lq2, scanned into c; lam[r] = the running sum after row r.
-// MASK: only rows rlo <= r < rhi accumulate (the causal diagonal and the sequence end).
+// 16 rows of one key column of the decay tile: D / (r_k^(1/3) (ln 2)^(1/3)) from the
+// similarity x and the row's lq2 = log2(r_q)/3, scanned into c; lam[r] = the running sum
+// after row r.  al2, be2 = alpha, beta times log2(e), so the softplus runs in log2 units
+// (its 1/ln 2 factor is returned to the key factor).  MASK: only rows rlo <= r < rhi
+// accumulate (the causal diagonal and the sequence end).
 template <bool MASK>
 __device__ __forceinline__ void decay16(const uint32_t (&x)[16], const float (&lv)[16], int pc, int rlo, int rhi,
-                                        float al, float be, float& c, float (&lam)[32]) {
+                                        float al2, float be2, float& c, float (&lam)[32]) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         const int r = pc * 16 + e;
-        const float dq = ex2f(fmaf(log2_softplus_poly(fmaf(al, __uint_as_float(x[e]), be)), 0.33333334f, lv[e]));
+        const float dq = ex2f(fmaf(log2_softplus_over_ln2(fmaf(al2, __uint_as_float(x[e]), be2)), 0.33333334f, lv[e]));
         if (MASK) c += (r >= rlo && r < rhi) ? dq : 0.f;
         else c += dq;
         lam[r] = c;
     }
 }
 
-// 16 rows of one key column of P for one head: P = 2^(S*scale*log2e + Lambda - shift), packed
+// 16 rows of one key column of P for one head: P = 2^(S*scale*log2e + lam), lam = Lambda*log2e
+// - shift, packed
 // to bf16 and stored MN-major into the P tile (two 16-byte chunks of 8 rows).  MASK: only
 // rows r >= rlo of a valid key are kept (the causal diagonal, keys past the sequence end).
 template <bool MASK>
-__device__ __forceinline__ void probs16(const uint32_t (&x)[16], int pc, float sl, const float (&lam)[32], float shh,
+__device__ __forceinline__ void probs16(const uint32_t (&x)[16], int pc, float sl, const float (&lam)[32],
                                         bool jvalid, int rlo, uint8_t* pcol, int ck0, int sw) {
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
@@ -155,8 +159,8 @@ __device__ __forceinline__ void probs16(const uint32_t (&x)[16], int pc, float s
         for (int e = 0; e < 8; e += 2) {
             const int r = ck * 8 + e;
             const int xe = cc * 8 + e;
-            float p0 = ex2f(fmaf(__uint_as_float(x[xe]), sl, lam[r] - shh));
-            float p1 = ex2f(fmaf(__uint_as_float(x[xe + 1]), sl, lam[r + 1] - shh));
+            float p0 = ex2f(fmaf(__uint_as_float(x[xe]), sl, lam[r]));
+            float p1 = ex2f(fmaf(__uint_as_float(x[xe + 1]), sl, lam[r + 1]));
             if (MASK) {
                 p0 = (jvalid && r >= rlo) ? p0 : 0.f;
                 p1 = (jvalid && r + 1 >= rlo) ? p1 : 0.f;
@@ -187,7 +191,7 @@ struct Smem {
     int pbskip[2];                               // 1: every P of this (query tile, key tile) underflows
     alignas(16) float pinc[2][128];              // inclusive prefix handed to the publisher warp
     alignas(16) float tot[2][NWG][128];          // per-quarter column sums (without the key factor)
-    float shift[4 * NWG][G];                     // per decay warp and head: max M_i over its quarter
+    float shift[4 * NWG];                        // per decay warp: max M_i over its quarter and the G heads
     alignas(8) uint64_t qfull, khfull, khempty, krfull, krempty, vfull[2], vempty[2], xsfull[NSLOT], xsempty[NSLOT],
         pfull[2], pempty[2], ofull, cfull[2][NWG], pbfull[2], pbempty[2], pubfull[2], pubempty[2];
     uint32_t tmem;
@@ -498,18 +502,18 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
         const int r0 = wg * 32;                          // first row of this quarter
         uint32_t use = 0, p_use = 0;
         bool ok = mbar_wait(&S.qfull, 0, abort);
-        // Softmax shift of this quarter: the largest row bound M_i of its 32 rows, one value per
-        // head (each warp keeps its own copy), so no per-element bound is loaded.  Every logit
-        // of the quarter's rows is below it; the shift cancels in O / l and lse adds it back.
+        // Softmax shift of this quarter: the largest row bound M_i of its 32 rows over the G
+        // heads (each warp keeps its own copy).  Every logit of the quarter's rows is below it;
+        // it is folded into Lambda once per tile, cancels in O / l, and lse adds it back.
         if (ok) {
-            for (int h = 0; h < G; ++h) {
-                float m = S.mq[h][r0 + lane];
+            float m = S.mq[0][r0 + lane];
+            for (int h = 1; h < G; ++h) m = fmaxf(m, S.mq[h][r0 + lane]);
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                if (lane == 0) S.shift[warp][h] = m;
-            }
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) S.shift[warp] = m;
             __syncwarp();
         }
+        const float al2 = al * kLog2e, be2 = be * kLog2e;
         // this thread's 32 rows of column jl in a P tile: row block r0/64, chunks (r0%64)/8 + c
         const uint32_t pcol_off = (r0 >> 6) * 16384 + (jl >> 3) * 1024 + (jl & 7) * 128;
         const int ck0 = (r0 & 63) >> 3, sw = jl & 7;
@@ -539,7 +543,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             const bool diag = (kt == qt);                // only the diagonal tile needs masks
             const bool tailq = qt * 128 + 128 > T;       // ... and, for the column totals, the last one
             if (!mbar_wait(&S.khfull, kt & 1, abort)) { ok = false; break; }
-            const float rk3 = ex2f(S.lk[jl]);            // r_k(j)^(1/3); 0 when vetoed
+            const float rk3 = ex2f(S.lk[jl]) * kCbrtLn2; // r_k(j)^(1/3) (ln 2)^(1/3); 0 when vetoed
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.khempty);
             // ---- decay over this quarter's 32 rows (without the key factor), scanned down the column
@@ -562,8 +566,8 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                         const float4 t4 = *reinterpret_cast<const float4*>(lqh + pc * 16 + e);
                         lv[e] = t4.x; lv[e + 1] = t4.y; lv[e + 2] = t4.z; lv[e + 3] = t4.w;
                     }
-                    if (masked) decay16<true>(x, lv, pc, rlo, rhi, al, be, c, lam);
-                    else decay16<false>(x, lv, pc, rlo, rhi, al, be, c, lam);
+                    if (masked) decay16<true>(x, lv, pc, rlo, rhi, al2, be2, c, lam);
+                    else decay16<false>(x, lv, pc, rlo, rhi, al2, be2, c, lam);
                 }
                 S.tot[kt & 1][wg][jl] = c;
             }
@@ -595,14 +599,13 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 }
             }
             if (skip) continue;                          // every P of this tile is exactly 0
-            // Lambda in log2 units: -(Pb + r_k^(1/3) * (above + partial sum)) * log2(e)
-            const float ka = -rk3 * kLog2e, kb = -fmaf(rk3, above, pbj) * kLog2e;
+            // lam = Lambda in log2 units minus the shift: -(Pb + r_k^(1/3) * (above + partial sum)) * log2(e) - shift
+            const float ka = -rk3 * kLog2e, kb = -fmaf(rk3, above, pbj) * kLog2e - S.shift[warp];
 #pragma unroll
             for (int r = 0; r < 32; ++r) lam[r] = fmaf(lam[r], ka, kb);
             // ---- per head: P = 2^(S*scale*log2e + Lambda - M_i), causally masked
             for (int h = 0; h < G && ok; ++h) {
                 if (!slot_wait()) { ok = false; break; }
-                const float shh = S.shift[warp][h];
                 // this P tile must be free: the PV of its previous use (two uses back) has completed
                 const uint32_t pbuf = p_use & 1;
                 if (p_use >= 2 && !mbar_wait(&S.pempty[pbuf], ((p_use >> 1) - 1) & 1, abort)) { ok = false; break; }
@@ -612,8 +615,8 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 for (int pc = 0; pc < 2; ++pc) {
                     uint32_t x[16];
                     slot_read(pc, x);
-                    if (diag) probs16<true>(x, pc, sl, lam, shh, j < T, rlo, pcol, ck0, sw);
-                    else probs16<false>(x, pc, sl, lam, shh, true, 0, pcol, ck0, sw);
+                    if (diag) probs16<true>(x, pc, sl, lam, j < T, rlo, pcol, ck0, sw);
+                    else probs16<false>(x, pc, sl, lam, true, 0, pcol, ck0, sw);
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
@@ -646,7 +649,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                         Vec16<__nv_bfloat16>::st(oi + c8 * 8, ov);
                     }
                     if (p.lse && wg == 0)
-                        p.lse[((size_t)b * p.H + hq) * T + i] = (S.shift[4 * wq][h] + lg2f(l)) * 0.6931471805599453f;
+                        p.lse[((size_t)b * p.H + hq) * T + i] = (S.shift[4 * wq] + lg2f(l)) * 0.6931471805599453f;
                 }
             }
         }

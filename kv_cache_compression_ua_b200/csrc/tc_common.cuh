@@ -257,26 +257,23 @@ __device__ __forceinline__ float lg2f(float x) {
     return y;
 }
 
-// log1p(e) for e in [0, 1] as e * q(e), q a degree-7 polynomial approximating log1p(e)/e,
-// fitted for this library by iteratively reweighted (Lawson) least squares on Chebyshev
-// nodes; maximum relative error 3.5e-7 when evaluated in fp32 by Horner's rule.  Runs on the
-// FMA pipe instead of the transcendental unit.
-__device__ __forceinline__ float log1p_unit(float e) {
-    float q = -0.0087831942f;
-    q = fmaf(q, e, 0.044944093f);
-    q = fmaf(q, e, -0.10885743f);
-    q = fmaf(q, e, 0.17825474f);
-    q = fmaf(q, e, -0.24523574f);
-    q = fmaf(q, e, 0.33280173f);
-    q = fmaf(q, e, -0.49997699f);
-    q = fmaf(q, e, 0.99999982f);
-    return e * q;
-}
-
-// log2(softplus(x)) = log2(max(x, 0) + log1p(exp(-|x|))): two transcendental-unit ops.
-__device__ __forceinline__ float log2_softplus_poly(float x) {
-    const float e = ex2f(-fabsf(x) * 1.4426950408889634f);
-    return lg2f(fmaxf(x, 0.f) + log1p_unit(e));
+// Softplus in log2 units.  For t2 = t * log2(e):
+//   log2(softplus(t) / ln 2) = log2(max(t2, 0) + log2(1 + 2^-|t2|)),
+// with log2(1 + e) for e in [0, 1] evaluated as e * q(e) on the FMA pipe: q is a degree-7
+// polynomial approximating log2(1 + e) / e, fitted for this library by iteratively reweighted
+// (Lawson) least squares on Chebyshev nodes; maximum relative error 3.3e-7 evaluated in fp32 by
+// Horner's rule.  Two transcendental-unit ops (one exp2, one log2).
+__device__ __forceinline__ float log2_softplus_over_ln2(float t2) {
+    const float e = ex2f(-fabsf(t2));
+    float q = -0.012319492176175117f;
+    q = fmaf(q, e, 0.06360796093940735f);
+    q = fmaf(q, e, -0.15535196661949158f);
+    q = fmaf(q, e, 0.2560097873210907f);
+    q = fmaf(q, e, -0.35339486598968506f);
+    q = fmaf(q, e, 0.48006370663642883f);
+    q = fmaf(q, e, -0.7213100790977478f);
+    q = fmaf(q, e, 1.4426947832107544f);
+    return lg2f(fmaf(e, q, fmaxf(t2, 0.f)));
 }
 
 
