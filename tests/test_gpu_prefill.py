@@ -150,6 +150,25 @@ def test_tensor_core_underflow_tile_skipping_is_exact(B, T, H, Hkv, shift):
     assert_close("b_final", g["b_final"], r["b_final"], "bf16", relative_max=True)
 
 
+def test_tensor_core_shared_shift_with_unequal_head_norms():
+    """The tensor-core path shifts every row of a 32-row quarter by the largest a-priori bound
+    over those rows and the G heads of the group.  Heads with very different query norms (one
+    head 6x, one 0.25x) and rows with tiny norms must still match the oracle."""
+    w = I.Workload("shift", 1, 600, 4, 1, 64, "bf16", 77)
+    x = I.make_prefill_inputs(w)
+    q = x["q"].astype(np.float64)
+    q[:, :, 0] *= 6.0
+    q[:, :, 2] *= 0.25
+    q[:, ::7, :] *= 1e-3                                  # some rows with almost no signal
+    x["q"] = I.round_bf16(q).astype(np.float32)
+    g, names = kernels_ran(lambda: run_gpu(w, x))
+    assert "k_fwd_tc" in names
+    assert ua.get_device_status() == 0
+    r = oracle.prefill_fwd(**oracle_inputs(x), scale=w.scale, theta=w.theta)
+    assert_close("o", g["o"], r["o"], "bf16")
+    assert_close("lse", g["lse"], r["lse"], "bf16", relative_max=True)
+
+
 def test_tensor_core_path_veto_and_plain_attention():
     w = I.Workload("tcveto", 1, 300, 4, 1, 64, "bf16", 17)
     x = I.make_prefill_inputs(w)
