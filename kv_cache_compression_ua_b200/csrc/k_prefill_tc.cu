@@ -183,17 +183,18 @@ struct Smem {
     alignas(1024) uint8_t kr[16384];             // Krope of the key tile  (used by the S of all heads)
     alignas(1024) uint8_t v[2][16384];           // V of the key tile, two stages
     alignas(1024) uint8_t p[2][32768];           // P tiles, MN-major SW128 [2 row blocks][16 k groups][8][128 B]
-    alignas(1024) uint8_t ones[1024];            // all-ones bf16 operand for the row sums
+    alignas(1024) uint8_t ones[512];             // all-ones bf16 operand for the row sums (N 16 x K 16)
     alignas(128) float lq[128];                   // lq2 of the query rows
     alignas(128) float mq[G][128];               // row bound M_i (log2 units) per head
     alignas(128) float lk[128];                   // lk2 of the key tile
     alignas(16) float pb[2][128];                // boundary prefix Pb of the key tile, two stages
-    int pbskip[2];                               // 1: every P of this (query tile, key tile) underflows
+    int pbskip[2];                               // 0: compute; 1: every P underflows (skip the softmax);
+                                                 // 2: also skip the decay (no b_final requested)
     alignas(16) float pinc[2][128];              // inclusive prefix handed to the publisher warp
-    alignas(16) float tot[2][NWG][128];          // per-quarter column sums (without the key factor)
+    alignas(16) float tot[3][NWG][128];          // per-quarter column sums (without the key factor), ring of 3
     float shift[4 * NWG];                        // per decay warp: max M_i over its quarter and the G heads
     alignas(8) uint64_t qfull, khfull, khempty, krfull, krempty, vfull[2], vempty[2], xsfull[NSLOT], xsempty[NSLOT],
-        pfull[2], pempty[2], ofull, cfull[2][NWG], pbfull[2], pbempty[2], pubfull[2], pubempty[2];
+        pfull[2], pempty[2], ofull, cfull[3][NWG], pbfull[2], pbempty[2], pubfull[2], pubempty[2];
     uint32_t tmem;
     int ticket;
     int abort;
@@ -246,7 +247,10 @@ __device__ __forceinline__ bool wait_counter(const unsigned* f, unsigned target,
     }
 }
 
-template <int G>
+// EARLY: no b_final is requested, so the decay of a tile whose softmax is skipped is not needed
+// either (the key tile is then neither loaded nor touched); a separate instantiation keeps the
+// other mode's hot loops free of that bookkeeping.
+template <int G, bool EARLY>
 __global__ void __launch_bounds__(640, 1)
 k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_kr,
          const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_v,
@@ -280,9 +284,9 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             mbar_init(&S.vempty[i], 1);
             mbar_init(&S.pfull[i], 4 * NWG);
             mbar_init(&S.pempty[i], 1);
-            for (int w = 0; w < NWG; ++w) mbar_init(&S.cfull[i][w], 4);   // the four warps of quarter w
             mbar_init(&S.pbfull[i], 1);
-            mbar_init(&S.pbempty[i], 4 * NWG + 2);      // decay warps and both MMA issuers
+            // decay warps and both MMA issuers; the producer too when tiles can go unloaded
+            mbar_init(&S.pbempty[i], 4 * NWG + 2 + (EARLY ? 1 : 0));
             mbar_init(&S.pubfull[i], 4);                // the four warps of the bottom quarter
             mbar_init(&S.pubempty[i], 1);
         }
@@ -290,6 +294,8 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             mbar_init(&S.xsfull[w], 1);
             mbar_init(&S.xsempty[w], 8);                 // the two warpgroups of a pair
         }
+        for (int i = 0; i < 3; ++i)
+            for (int w = 0; w < NWG; ++w) mbar_init(&S.cfull[i][w], 4);   // the four warps of quarter w
         mbar_init(&S.ofull, 1);
         S.abort = 0;
         // Work tickets go out in launch order, query tile major: every CTA a tile waits on
@@ -300,7 +306,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
     if (warp == 16) {
         // all-ones operand (bf16 1.0 = 0x3F80); any layout of it reads as ones
         uint32_t* o32 = reinterpret_cast<uint32_t*>(S.ones);
-        for (int i = lane; i < 256; i += 32) o32[i] = 0x3F803F80u;
+        for (int i = lane; i < 128; i += 32) o32[i] = 0x3F803F80u;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 0) {
@@ -328,27 +334,41 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             for (int h = 0; h < G; ++h) tma_load_2d(S.mq[h], &tm_mq, &S.qfull, qt * 128, b * p.H + kvh * G + h);
         }
         __syncwarp();
+        // Key tiles whose decay is skipped (code 2) are not loaded at all; nk counts the loaded
+        // ones, and every role that takes part in the key-tile hand-offs counts the same.
+        // (That can only happen when no b_final is requested; otherwise every tile is loaded and
+        // the producer runs ahead without looking at the codes.)
+        constexpr bool early = EARLY;
+        uint32_t nk = 0;
         for (int kt = 0; kt < ntile; ++kt) {
-            if (kt >= 1 && !mbar_wait(&S.khempty, (kt - 1) & 1, abort)) break;
+            if (early) {
+                if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) break;
+                const int code = S.pbskip[kt & 1];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
+                if (code == 2) continue;
+            }
+            if (nk >= 1 && !mbar_wait(&S.khempty, (nk - 1) & 1, abort)) break;
             if (leader) {
                 mbar_expect_tx(&S.khfull, 16384 + 512);
                 tma_load_3d(S.kh, &tm_kh, &S.khfull, 0, kt * 128, unit);
                 tma_load_2d(S.lk, &tm_lk, &S.khfull, kt * 128, unit);
             }
             __syncwarp();
-            const int sv = kt & 1;
-            if (kt >= 2 && !mbar_wait(&S.vempty[sv], ((kt >> 1) - 1) & 1, abort)) break;
+            const int sv = nk & 1;
+            if (nk >= 2 && !mbar_wait(&S.vempty[sv], ((nk >> 1) - 1) & 1, abort)) break;
             if (leader) {
                 mbar_expect_tx(&S.vfull[sv], 16384);
                 tma_load_4d(S.v[sv], &tm_v, &S.vfull[sv], 0, kvh, kt * 128, b);
             }
             __syncwarp();
-            if (kt >= 1 && !mbar_wait(&S.krempty, (kt - 1) & 1, abort)) break;
+            if (nk >= 1 && !mbar_wait(&S.krempty, (nk - 1) & 1, abort)) break;
             if (leader) {
                 mbar_expect_tx(&S.krfull, 16384);
                 tma_load_3d(S.kr, &tm_kr, &S.krfull, 0, kt * 128, unit);
             }
             __syncwarp();
+            ++nk;
         }
     } else if (warp == 18) {
         // ------------------------------------------------ boundary look-back and publisher
@@ -369,7 +389,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 float mn = fminf(fminf(v4.x, v4.y), fminf(v4.z, v4.w));
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                skip = (mn * kLog2e >= kSkipLog2) ? 1 : 0;
+                skip = (mn * kLog2e >= kSkipLog2) ? (EARLY ? 2 : 1) : 0;
             }
             *reinterpret_cast<float4*>(&S.pb[sb][lane * 4]) = v4;
             if (lane == 0) {
@@ -380,12 +400,23 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             if (lane == 0) mbar_arrive(&S.pbfull[sb]);
             return true;
         };
+        // A tile whose decay is skipped adds nothing to the prefix it passes on: Pb itself
+        // (a lower bound of the true prefix, already past the skip threshold, so every later
+        // query tile skips this key tile too).  Other tiles' prefixes come from the bottom
+        // quarter through pinc, counted by npub.
+        uint32_t npub = 0;
         auto publish = [&](int kt) -> bool {
-            const int sb = kt & 1;
-            if (!mbar_wait(&S.pubfull[sb], (kt >> 1) & 1, abort)) return false;
-            const float4 v4 = *reinterpret_cast<const float4*>(&S.pinc[sb][lane * 4]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.pubempty[sb]);
+            float4 v4;
+            if (S.pbskip[kt & 1] == 2) {
+                v4 = *reinterpret_cast<const float4*>(&S.pb[kt & 1][lane * 4]);
+            } else {
+                const int sb = npub & 1;
+                if (!mbar_wait(&S.pubfull[sb], (npub >> 1) & 1, abort)) return false;
+                v4 = *reinterpret_cast<const float4*>(&S.pinc[sb][lane * 4]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.pubempty[sb]);
+                ++npub;
+            }
             const size_t row = (size_t)unit * p.nqt + qt;
             __stcg(reinterpret_cast<float4*>(p.pincl + row * p.Tp + (size_t)kt * 128) + lane, v4);
             __threadfence();
@@ -430,23 +461,35 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 ++nh;
                 return true;
             };
+            constexpr bool early = EARLY;               // decay-skipped tiles possible
+            uint32_t nk = 0;                             // key tiles loaded (code != 2)
             for (int kt = 0; ok && kt < ntile; ++kt) {
-                if (!mbar_wait(&S.khfull, kt & 1, abort)) break;
+                int code = 0;
+                auto take_code = [&]() -> bool {
+                    if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) return false;
+                    code = S.pbskip[kt & 1];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
+                    return true;
+                };
+                // the skip code before X when a tile may be neither loaded nor needed, else after
+                if (early && !take_code()) break;
+                if (code == 2) continue;
+                if (!mbar_wait(&S.khfull, nk & 1, abort)) break;
                 tc_fence_after();
                 if (!issue_half(akh, akq, 0) || !issue_half(akh, akq, 1)) break;
                 if (leader) umma_commit(&S.khempty);       // X done: Khat of this key tile is free
                 __syncwarp();
-                if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) break;
-                const bool skip = S.pbskip[kt & 1] != 0;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
-                if (!mbar_wait(&S.krfull, kt & 1, abort)) break;
+                if (!early && !take_code()) break;
+                const bool skip = code != 0;
+                if (!mbar_wait(&S.krfull, nk & 1, abort)) break;
                 tc_fence_after();
                 for (int h = 0; h < G && ok && !skip; ++h)
                     ok = issue_half(akr, smem_u32(S.q[h]), 0) && issue_half(akr, smem_u32(S.q[h]), 1);
                 if (!ok) break;
                 if (leader) umma_commit(&S.krempty);       // last reader of Krope
                 __syncwarp();
+                ++nk;
             }
         } else {
             const uint64_t d_ones = smem_desc(smem_u32(S.ones), 256, 128, kSwizzleNone);
@@ -455,15 +498,17 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             const uint64_t dpb = smem_desc(smem_u32(S.p[1]), 16384, 1024, kSwizzle128B);
             const uint64_t dva = smem_desc(smem_u32(S.v[0]), 16384, 1024, kSwizzle128B);
             const uint64_t dvb = smem_desc(smem_u32(S.v[1]), 16384, 1024, kSwizzle128B);
-            uint32_t p_use = 0;
+            uint32_t p_use = 0, nk = 0;                 // P uses; key tiles loaded (code != 2)
             bool first = true;                           // no PV issued yet: the first one initialises O
             for (int kt = 0; ok && kt < ntile; ++kt) {
-                const int sv = kt & 1;
                 if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) break;
-                const bool skip = S.pbskip[kt & 1] != 0;
+                const int code = S.pbskip[kt & 1];
+                const bool skip = code != 0;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
-                if (!mbar_wait(&S.vfull[sv], (kt >> 1) & 1, abort)) break;
+                if (code == 2) continue;
+                const int sv = nk & 1;
+                if (!mbar_wait(&S.vfull[sv], (nk >> 1) & 1, abort)) break;   // V stage protocol, used or not
                 for (int h = 0; h < G && ok && !skip; ++h) {
                     const uint32_t pbuf = p_use & 1;
                     if (!mbar_wait(&S.pfull[pbuf], (p_use >> 1) & 1, abort)) { ok = false; break; }
@@ -488,6 +533,7 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                     if (kt == ntile - 1) umma_commit(&S.ofull);
                 }
                 __syncwarp();
+                ++nk;
             }
         }
     } else {
@@ -501,6 +547,9 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
         const float sl = p.scale_log2e;
         const int r0 = wg * 32;                          // first row of this quarter
         uint32_t use = 0, p_use = 0;
+        uint32_t nd = 0, npub = 0, nk = 0;               // tiles whose decay ran / whose prefix went to
+                                                         // warp 18 / key tiles loaded
+        constexpr bool early = EARLY;                   // decay-skipped tiles possible
         bool ok = mbar_wait(&S.qfull, 0, abort);
         // Softmax shift of this quarter: the largest row bound M_i of its 32 rows over the G
         // heads (each warp keeps its own copy).  Every logit of the quarter's rows is below it;
@@ -542,12 +591,29 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             const int j = kt * 128 + jl;
             const bool diag = (kt == qt);                // only the diagonal tile needs masks
             const bool tailq = qt * 128 + 128 > T;       // ... and, for the column totals, the last one
-            if (!mbar_wait(&S.khfull, kt & 1, abort)) { ok = false; break; }
+            // Pb and the skip code of this tile (staged by warp 18 two tiles ahead): before the
+            // decay when the decay itself may be skipped (no b_final requested), else after it,
+            // where Pb is first needed
+            int code = 0;
+            float pbj = 0.f;
+            auto take_pb = [&]() -> bool {
+                if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) return false;
+                pbj = S.pb[kt & 1][jl];
+                code = S.pbskip[kt & 1];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
+                return true;
+            };
+            if (early && !take_pb()) { ok = false; break; }
+            if (code == 2) continue;                     // nothing of this tile is needed or loaded
+            if (!mbar_wait(&S.khfull, nk & 1, abort)) { ok = false; break; }
             const float rk3 = ex2f(S.lk[jl]) * kCbrtLn2; // r_k(j)^(1/3) (ln 2)^(1/3); 0 when vetoed
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.khempty);
+            ++nk;
             // ---- decay over this quarter's 32 rows (without the key factor), scanned down the column
             float lam[32];
+            float tot_above = 0.f;
             {
                 if (!slot_wait()) { ok = false; break; }
                 float c = 0.f;
@@ -569,21 +635,27 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                     if (masked) decay16<true>(x, lv, pc, rlo, rhi, al2, be2, c, lam);
                     else decay16<false>(x, lv, pc, rlo, rhi, al2, be2, c, lam);
                 }
-                S.tot[kt & 1][wg][jl] = c;
+                // Carry across quarters through a ring of three buffers.  Buffer nd % 3 was last
+                // read for decay tile nd - 3; this tile's Pb wait (before the decay, or the one
+                // of the tile before, after its decay) implies that every warp has passed its Pb
+                // arrival of a later tile, which follows its reads of those totals.
+                const int tb = nd % 3;
+                const uint32_t tph = (nd / 3) & 1;
+                S.tot[tb][wg][jl] = c;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.cfull[tb][wg]);
+                float above = 0.f;                       // sum over the quarters above this one
+                for (int w = 0; w < wg && ok; ++w) {
+                    if (!mbar_wait(&S.cfull[tb][w], tph, abort)) { ok = false; break; }
+                    above += S.tot[tb][w][jl];
+                }
+                if (!ok) break;
+                ++nd;
+                tot_above = above;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.cfull[kt & 1][wg]);
-            float above = 0.f;                           // sum over the quarters above this one
-            for (int w = 0; w < wg; ++w) {
-                if (!mbar_wait(&S.cfull[kt & 1][w], (kt >> 1) & 1, abort)) { ok = false; break; }
-                above += S.tot[kt & 1][w][jl];
-            }
-            if (!ok) break;
-            if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) { ok = false; break; }
-            const float pbj = S.pb[kt & 1][jl];
-            const bool skip = S.pbskip[kt & 1] != 0;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
+            const float above = tot_above;
+            if (!early && !take_pb()) { ok = false; break; }
+            const bool skip = code != 0;
             if (wg == NWG - 1) {
                 // the bottom quarter holds the column total of this query tile: publish the
                 // inclusive prefix for the next query tile, or, on the last one, b_final
@@ -591,11 +663,12 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 if (qt == p.nqt - 1) {
                     if (p.b_final && j < T) p.b_final[(size_t)unit * T + j] = -pinc;
                 } else {
-                    const int sb = kt & 1;
-                    if (kt >= 2 && !mbar_wait(&S.pubempty[sb], ((kt >> 1) - 1) & 1, abort)) { ok = false; break; }
+                    const int sb = npub & 1;
+                    if (npub >= 2 && !mbar_wait(&S.pubempty[sb], ((npub >> 1) - 1) & 1, abort)) { ok = false; break; }
                     S.pinc[sb][jl] = pinc;
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.pubfull[sb]);
+                    ++npub;
                 }
             }
             if (skip) continue;                          // every P of this tile is exactly 0
@@ -676,14 +749,19 @@ size_t fwd_tc_smem(int G) {
 
 bool fwd_tc_supported(int d, int G) { return d == 64 && G >= 1 && G <= 4; }
 
-template <int G>
-static cudaError_t fwd_tc_inst(const CUtensorMap* m, const FwdTcParams& p, cudaStream_t s) {
+template <int G, bool EARLY>
+static cudaError_t fwd_tc_launch(const CUtensorMap* m, const FwdTcParams& p, cudaStream_t s) {
     const size_t smem = fwd_tc_smem(G);
-    cudaError_t e = cudaFuncSetAttribute(k_fwd_tc<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_fwd_tc<G, EARLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     UA_PROFILE("k_fwd_tc", s);
-    k_fwd_tc<G><<<p.nqt * p.nunits, 640, smem, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
+    k_fwd_tc<G, EARLY><<<p.nqt * p.nunits, 640, smem, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
     return cudaGetLastError();
+}
+
+template <int G>
+static cudaError_t fwd_tc_inst(const CUtensorMap* m, const FwdTcParams& p, cudaStream_t s) {
+    return p.b_final ? fwd_tc_launch<G, false>(m, p, s) : fwd_tc_launch<G, true>(m, p, s);
 }
 
 cudaError_t launch_fwd_tc(const FwdTcLaunch& L, cudaStream_t s) {

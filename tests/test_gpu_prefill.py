@@ -148,6 +148,15 @@ def test_tensor_core_underflow_tile_skipping_is_exact(B, T, H, Hkv, shift):
     assert_close("o", g["o"], r["o"], "bf16")
     assert_close("lse", g["lse"], r["lse"], "bf16", relative_max=True)
     assert_close("b_final", g["b_final"], r["b_final"], "bf16", relative_max=True)
+    # Without b_final the decay of the skipped tiles is skipped as well; o and lse must be
+    # bit-identical to the run above (those tiles contribute exactly zero either way).
+    r2 = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
+                        scale=w.scale, theta=w.theta, ws=ws, want_bfinal=False)
+    _, skipped2 = ua.prefill_tile_stats(shape, ws)
+    assert ua.get_device_status() == 0
+    assert skipped2 == skipped
+    assert torch.equal(r2["o"], r_gpu["o"])
+    assert torch.equal(r2["lse"], r_gpu["lse"])
 
 
 def test_tensor_core_shared_shift_with_unequal_head_norms():
