@@ -99,9 +99,10 @@ ua_status ua_prefill_workspace_size(const ua_shape* shape, size_t* bytes);
  * underflow, and then UA_ERR_RANGE is raised in the device status word.  The same path skips
  * the softmax and PV work of every 128 x 128 (query tile, key tile) whose decay prefix
  * makes all its probabilities underflow to exactly 0 in fp32 (Lambda only decreases down a
- * key column, so the prefix above the tile bounds the whole tile); the decay of the tile is
- * still evaluated, so b_final and all outputs are identical to the unskipped computation
- * (see ua_prefill_tile_stats).  All other problems,
+ * key column, so the prefix above the tile bounds the whole tile).  When b_final is requested
+ * the decay of such a tile is still evaluated (b_final stays exact); when b_final is NULL the
+ * tile is skipped entirely.  Either way every requested output is identical to the unskipped
+ * computation (see ua_prefill_tile_stats).  All other problems,
  * and every call that asks for lambda_dbg, run the fp32 SIMT path, which uses a running
  * maximum. */
 ua_status ua_prefill_fwd(const ua_shape* shape, const void* q, const void* k, const void* v,
