@@ -41,6 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ----------------------------------------------------------------------------- helpers
 
 MUFU_PER_CLK_SM = 16   # transcendental (exp2/log2) results per clock per SM: 4 per SM sub-partition
+# DRAM bytes (read + written) per launch of the dominant kernel, from the ncu capture summarised
+# in profiles/k_fwd_tc_prefill_1b.md; valid only for the kernel version that capture was taken of
+TRAFFIC_BYTES = {"k_fwd_tc": 926.0e6 + 149.4e6}
 N_SM = 148
 
 
@@ -244,7 +247,8 @@ def bench_prefill(args, world, rank, local, peaks, peaks_kind):
         ops = mufu_ops(w) - skipped * 128 * 128 * (w.H // w.Hkv)
         achieved_a = ops / (per_launch_ms * 1e-3) / 1e9
         roofline = {"kernel": name, "bound": "alu", "achieved": achieved_a, "peak": peak_a,
-                    "unit": "Gop/s (exp2/log2)", "frac": achieved_a / peak_a, "traffic": None,
+                    "unit": "Gop/s (exp2/log2)", "frac": achieved_a / peak_a,
+                    "traffic": TRAFFIC_BYTES.get(name) if w.name == "prefill_1b" else None,
                     "peak_source": f"{MUFU_PER_CLK_SM} exp2/log2 results per clock per SM x {N_SM} SMs x "
                                    f"{mhz:.0f} MHz (median SM clock sampled during the timed region)",
                     "tensor": tensor}
