@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     using L = EntryLayout<TC, DH>;
     constexpr int VEC = L::VEC, LPE = L::LPE, EPB = L::EPB, NW = L::NW;
     constexpr int half = DH / 2;
-    __shared__ float s_kt[DH], s_ktr[DH], s_vt[DH], s_q[G][DH], s_lt[G];
+    __shared__ float s_kt[DH], s_ktr[DH], s_vt[DH], s_q[G][DH], s_lt[G], s_g[G * DH];
     __shared__ float s_red[NW];
     __shared__ int s_wcnt[NW];
     extern __shared__ float dsm[];
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         kx = Elem<TC>::ld(kin + tid);
         vx = Elem<TC>::ld(vin + tid);
     }
-    float qa[QE], qb[QE], gv[GE];
+    float qa[QE], qb[QE];
 #pragma unroll
     for (int r = 0; r < QE; ++r) {
         const int e = tid + 256 * r;
@@ -220,10 +220,11 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
             qb[r] = Elem<TC>::ld(qin + vecid * DH + m + half);
         }
     }
+    // the gate goes to shared memory: loaded now, held in no register through the entry loop
 #pragma unroll
     for (int r = 0; r < GE; ++r) {
         const int e = tid + 256 * r;
-        gv[r] = e < G * DH ? Elem<TC>::ld(gin + e) : 0.f;
+        if (e < G * DH) s_g[e] = Elem<TC>::ld(gin + e);
     }
     const float aq_t = p.a_q[unit], ak_t = p.a_k[unit];
     const float al = p.alpha[kvh], be = p.beta[kvh];
@@ -386,7 +387,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
             Ls = fmaf(s_l[q * G + h], w, Ls);
             A = fmaf(s_acc[((size_t)q * G + h) * DH + x], w, A);
         }
-        Elem<TC>::st(oout + e, A / Ls * sigmoid_f(gv[r]));
+        Elem<TC>::st(oout + e, A / Ls * sigmoid_f(s_g[e]));
     }
     // ---- eviction bits, append the new token
     if (p.evict_bits)

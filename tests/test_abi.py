@@ -111,3 +111,25 @@ def test_cache_calls_reject_bad_arguments(lib):
     c3 = ua.ua_cache(2, 2, 80, 100, ua.UA_BF16, *([FAKE] * 7))
     assert lib.ua_decode_step(ctypes.byref(c3), 8, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
                               P(FAKE), None, None, 0, None) == 2
+
+
+def test_tile_stats_host_logic(lib):
+    """ua_prefill_tile_stats: argument checks, and the tile count for problems that run the fp32
+    SIMT path (no device access: nothing is skipped there)."""
+    import ctypes
+    tiles, skipped = ctypes.c_ulonglong(7), ctypes.c_ulonglong(7)
+    s = _shape(B=2, T=300, H=4, Hkv=2, d=64, dtype=ua.UA_F32)
+    assert lib.ua_prefill_tile_stats(ctypes.byref(s), None, 0, ctypes.byref(tiles), ctypes.byref(skipped),
+                                     None) == 0
+    n = (300 + 127) // 128
+    assert tiles.value == 2 * 2 * n * (n + 1) // 2 and skipped.value == 0
+    assert lib.ua_prefill_tile_stats(ctypes.byref(s), None, 0, None, ctypes.byref(skipped), None) == 1
+    bad = _shape(B=0)
+    assert lib.ua_prefill_tile_stats(ctypes.byref(bad), None, 0, ctypes.byref(tiles), ctypes.byref(skipped),
+                                     None) == 1
+    # the tensor-core path needs the workspace it ran on
+    tc = _shape(B=1, T=300, H=4, Hkv=1, d=64, dtype=ua.UA_BF16)
+    assert lib.ua_prefill_tile_stats(ctypes.byref(tc), None, 0, ctypes.byref(tiles), ctypes.byref(skipped),
+                                     None) == 1
+    assert lib.ua_prefill_tile_stats(ctypes.byref(tc), ctypes.c_void_p(256), 16, ctypes.byref(tiles),
+                                     ctypes.byref(skipped), None) == 4
