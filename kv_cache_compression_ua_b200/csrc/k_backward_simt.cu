@@ -114,6 +114,7 @@ struct Ctx {
     const float *qr, *kh, *kr;
     const void *v, *g, *o, *d_o;
     const float *aq, *ak, *rq, *rk, *alpha, *beta, *lse, *delta, *pb;
+    const float* qmax;   // [B,Hkv,nqt] tile row bounds, or NULL (no skipping)
     float *dpb, *dqr, *dkh_rows, *dkh_keys, *dkr, *dv32, *daq32, *dak32, *dab;
 };
 
@@ -247,7 +248,15 @@ __global__ void __launch_bounds__(NT) k_bwd_keys(Ctx c) {
             t.colv[BN + tid] = j < T ? c.pb[(unit * c.nqt + qt) * T + j] : 0.f;
             if (j < T) c.dpb[(unit * c.nqt + qt) * T + j] = sdl;   // sum of dLambda over rows >= 64(qt+1)
         }
-        __syncthreads();
+        // Nothing of this (query tile, key tile) reaches any gradient when every probability
+        // underflows (then dS = dLambda = 0 here) and the later query tiles fed no dLambda into
+        // these keys (then dD = 0 here too): skip it.
+        if (c.qmax) {
+            const float thr = kSimtSkipMargin + 2.f * c.qmax[unit * c.nqt + qt];
+            if (__syncthreads_and(tid >= BN || (t.colv[BN + tid] >= thr && sdl == 0.f))) continue;
+        } else {
+            __syncthreads();
+        }
         decay_tile<DH>(t, i0, j0, T, al, be, ty, tx, tid);
         for (int hh = 0; hh < c.G; ++hh) {
             const int h = kvh * c.G + hh;
@@ -412,7 +421,13 @@ __global__ void __launch_bounds__(NT) k_bwd_rows(Ctx c) {
             t.colv[BN + tid] = j < T ? c.pb[(unit * c.nqt + qt) * T + j] : 0.f;
             t.colv[3 * BN + tid] = j < T ? c.dpb[(unit * c.nqt + qt) * T + j] : 0.f;
         }
-        __syncthreads();
+        // as in the key pass: no probability survives and no dLambda arrives from later rows
+        if (c.qmax) {
+            const float thr = kSimtSkipMargin + 2.f * c.qmax[unit * c.nqt + qt];
+            if (__syncthreads_and(tid >= BN || (t.colv[BN + tid] >= thr && t.colv[3 * BN + tid] == 0.f))) continue;
+        } else {
+            __syncthreads();
+        }
         decay_tile<DH>(t, i0, j0, T, al, be, ty, tx, tid);
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) {
@@ -622,7 +637,7 @@ static cudaError_t bwd_inst(const BwdParams& p, cudaStream_t s) {
     c.B = p.B; c.T = p.T; c.H = p.H; c.Hkv = p.Hkv; c.d = p.d; c.G = p.G; c.nqt = p.nqt; c.scale = p.scale;
     c.qr = p.qr; c.kh = p.kh; c.kr = p.kr; c.v = p.v; c.g = p.g; c.o = p.o; c.d_o = p.d_o;
     c.aq = p.a_q; c.ak = p.a_k; c.rq = p.rq; c.rk = p.rk; c.alpha = p.alpha; c.beta = p.beta; c.lse = p.lse;
-    c.delta = p.delta; c.pb = p.pb; c.dpb = p.dpb; c.dqr = p.dqr; c.dkh_rows = p.dkh_rows; c.dkh_keys = p.dkh;
+    c.delta = p.delta; c.pb = p.pb; c.qmax = p.qmax; c.dpb = p.dpb; c.dqr = p.dqr; c.dkh_rows = p.dkh_rows; c.dkh_keys = p.dkh;
     c.dkr = p.dkr; c.dv32 = p.dv32; c.daq32 = p.daq32; c.dak32 = p.dak32; c.dab = p.dab;
     const size_t smem = tiles_bytes<DH>();
     cudaError_t e;

@@ -115,6 +115,33 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p) {
     }
 }
 
+// ------------------------------------------------------------------ tile row bounds
+// grid (nqt, B*Hkv), 256 threads: the largest scale*||q_i|| over the 64 rows of a query tile and
+// the G heads of a KV group.
+__global__ void __launch_bounds__(256) k_tile_qmax(TileQmaxParams p) {
+    const int qt = blockIdx.x, unit = blockIdx.y, b = unit / p.Hkv, kvh = unit % p.Hkv, G = p.H / p.Hkv;
+    __shared__ float red[8];
+    float m = 0.f;
+    for (int e = threadIdx.x; e < 64 * G; e += blockDim.x) {
+        const int hh = e / 64, i = qt * 64 + e % 64;
+        if (i < p.T) m = fmaxf(m, p.mq[((size_t)b * p.H + kvh * G + hh) * p.T + i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+        p.qmax[(size_t)unit * p.nqt + qt] = m;
+    }
+}
+
+cudaError_t launch_tile_qmax(const TileQmaxParams& p, cudaStream_t s) {
+    UA_PROFILE("k_tile_qmax", s);
+    k_tile_qmax<<<dim3(p.nqt, p.B * p.Hkv), 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ boundary pass
 // grid (ceil(T/128), Hkv, B), 128 threads; thread = key j, sweeping the rows l > j in
 // order.  At every query-tile boundary l = t*bq it writes the prefix sum so far.
@@ -207,20 +234,26 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
     }
     const float al = p.alpha[kvh], be = p.beta[kvh];
 
+    // tiles whose probabilities all underflow are skipped (not when the debug Lambda is written)
+    const bool can_skip = p.qmax != nullptr && p.lambda_dbg == nullptr;
+    const float thr = can_skip ? kSimtSkipMargin + 2.f * p.qmax[unit * p.nqt + qt] : 0.f;
     for (int kt = 0; kt <= qt; ++kt) {
         const int j0 = kt * BN;
         __syncthreads();
+        for (int c = tid; c < BN; c += 256) {
+            const int j = j0 + c;
+            sRk[c] = j < T ? p.rk[unit * T + j] : 0.f;
+            sPb[c] = j < T ? p.pb[(unit * p.nqt + qt) * T + j] : 0.f;
+        }
+        if (__syncthreads_and(!can_skip || tid >= BN || sPb[tid] >= thr)) {
+            if (can_skip) continue;
+        }
         for (int e = tid; e < BN * DH; e += 256) {
             const int c = e / DH, x = e % DH, j = j0 + c;
             const bool ok = j < T;
             sKh[c * LD + x] = ok ? p.kh[(unit * T + j) * DH + x] : 0.f;
             sKr[c * LD + x] = ok ? p.kr[(unit * T + j) * DH + x] : 0.f;
             sV[c * LD + x] = ok ? Elem<TI>::ld(vin + (((size_t)b * T + j) * p.Hkv + kvh) * DH + x) : 0.f;
-        }
-        for (int c = tid; c < BN; c += 256) {
-            const int j = j0 + c;
-            sRk[c] = j < T ? p.rk[unit * T + j] : 0.f;
-            sPb[c] = j < T ? p.pb[(unit * p.nqt + qt) * T + j] : 0.f;
         }
         __syncthreads();
         // decay D[l = i0 + r, j = j0 + c]

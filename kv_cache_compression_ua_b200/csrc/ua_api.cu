@@ -38,7 +38,7 @@ ua_status check_shape(const ua_shape* s) {
 
 // Workspace of the SIMT prefill forward: f32 rotated/normalised copies, rates, prefixes.
 struct FwdWs {
-    size_t qr, kh, kr, rq, rk, pb, total;
+    size_t qr, kh, kr, rq, rk, pb, mq, qmax, total;
 };
 
 FwdWs fwd_ws_layout(const ua_shape* s) {
@@ -53,6 +53,8 @@ FwdWs fwd_ws_layout(const ua_shape* s) {
     w.rq = take(B * Hkv * T * 4);
     w.rk = take(B * Hkv * T * 4);
     w.pb = take(B * Hkv * nqt * T * 4);
+    w.mq = take(B * H * T * 4);
+    w.qmax = take(B * Hkv * nqt * 4);
     w.total = off;
     return w;
 }
@@ -173,7 +175,12 @@ static ua_status prefill_fwd_simt(const ua_shape* s, const void* q, const void* 
     pp.qr = at(ws, w.qr); pp.kh = at(ws, w.kh); pp.kr = at(ws, w.kr);
     pp.rq = reinterpret_cast<float*>(at(ws, w.rq)); pp.rk = reinterpret_cast<float*>(at(ws, w.rk));
     pp.rf = rope_freq(s->rope_theta, s->d);
+    pp.mq = reinterpret_cast<float*>(at(ws, w.mq)); pp.Tp = s->T; pp.mq_scale = s->scale;
     if ((st = cuda_status(launch_prep(pp, bf, false, cs))) != UA_OK) return st;
+    TileQmaxParams tq;
+    tq.B = s->B; tq.T = s->T; tq.H = s->H; tq.Hkv = s->Hkv; tq.nqt = nqt; tq.mq = pp.mq;
+    tq.qmax = reinterpret_cast<float*>(at(ws, w.qmax));
+    if ((st = cuda_status(launch_tile_qmax(tq, cs))) != UA_OK) return st;
 
     BoundaryParams bp;
     bp.B = s->B; bp.T = s->T; bp.Hkv = s->Hkv; bp.d = s->d; bp.bq = kBq; bp.nqt = nqt;
@@ -192,6 +199,7 @@ static ua_status prefill_fwd_simt(const ua_shape* s, const void* q, const void* 
     fp.qr = reinterpret_cast<const float*>(pp.qr); fp.kh = reinterpret_cast<const float*>(pp.kh);
     fp.kr = reinterpret_cast<const float*>(pp.kr);
     fp.v = v; fp.g = g; fp.rq = pp.rq; fp.rk = pp.rk; fp.alpha = alpha; fp.beta = beta; fp.pb = bp.pb;
+    fp.qmax = tq.qmax;
     fp.o = o; fp.lse = lse; fp.lambda_dbg = lambda_dbg;
     return cuda_status(launch_fwd_simt(fp, bf, cs));
 }
@@ -358,7 +366,12 @@ ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const 
     pp.qr = at(ws, w.f.qr); pp.kh = at(ws, w.f.kh); pp.kr = at(ws, w.f.kr);
     pp.rq = reinterpret_cast<float*>(at(ws, w.f.rq)); pp.rk = reinterpret_cast<float*>(at(ws, w.f.rk));
     pp.rf = rope_freq(s->rope_theta, s->d);
+    pp.mq = reinterpret_cast<float*>(at(ws, w.f.mq)); pp.Tp = s->T; pp.mq_scale = s->scale;
     if ((st = cuda_status(launch_prep(pp, bf, false, cs))) != UA_OK) return st;
+    TileQmaxParams tq;
+    tq.B = s->B; tq.T = s->T; tq.H = s->H; tq.Hkv = s->Hkv; tq.nqt = w.nqt; tq.mq = pp.mq;
+    tq.qmax = reinterpret_cast<float*>(at(ws, w.f.qmax));
+    if ((st = cuda_status(launch_tile_qmax(tq, cs))) != UA_OK) return st;
     BoundaryParams bp;
     bp.B = s->B; bp.T = s->T; bp.Hkv = s->Hkv; bp.d = s->d; bp.bq = kBq; bp.nqt = w.nqt;
     bp.kh = reinterpret_cast<const float*>(pp.kh); bp.rq = pp.rq; bp.rk = pp.rk; bp.alpha = alpha; bp.beta = beta;
@@ -369,7 +382,7 @@ ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const 
     p.B = s->B; p.T = s->T; p.H = s->H; p.Hkv = s->Hkv; p.d = s->d; p.G = s->H / s->Hkv; p.nqt = w.nqt; p.nkt = w.nkt;
     p.scale = s->scale; p.theta = s->rope_theta; p.rf = pp.rf;
     p.qr = reinterpret_cast<const float*>(pp.qr); p.kh = reinterpret_cast<const float*>(pp.kh);
-    p.kr = reinterpret_cast<const float*>(pp.kr); p.rq = pp.rq; p.rk = pp.rk; p.pb = bp.pb;
+    p.kr = reinterpret_cast<const float*>(pp.kr); p.rq = pp.rq; p.rk = pp.rk; p.pb = bp.pb; p.qmax = tq.qmax;
     p.k = k; p.v = v; p.g = g; p.o = o; p.d_o = d_o; p.a_q = a_q; p.a_k = a_k; p.alpha = alpha; p.beta = beta;
     p.lse = lse;
     p.delta = reinterpret_cast<float*>(at(ws, w.delta)); p.dpb = reinterpret_cast<float*>(at(ws, w.dpb));

@@ -59,10 +59,25 @@ struct FwdParams {
     const float* alpha;
     const float* beta;
     const float* pb;    // [B,Hkv,nqt,T] with bq = 64
+    const float* qmax;  // [B,Hkv,nqt] largest scale*||q_i|| of each query tile and group, or NULL
     void* o;            // [B,T,H,d] act
     float* lse;         // [B,H,T] or NULL
     float* lambda_dbg;  // [B,Hkv,T,T] or NULL (pre-zeroed)
 };
+
+// A 64-row query tile and a key tile of the SIMT paths contribute exactly nothing (every
+// probability underflows to 0 in fp32, expf below -103.98) when min_j Pb[j] exceeds
+// 2 * max_i scale*||q_i|| by this much: the logit of (i, j) is at most scale*||q_i|| - Pb[j]
+// and row i's normaliser at least its diagonal logit, -scale*||q_i||.
+constexpr float kSimtSkipMargin = 105.f;
+
+// qmax[unit][t] = max over the 64 rows of query tile t and the G heads of the group of mq.
+struct TileQmaxParams {
+    int B, T, H, Hkv, nqt;
+    const float* mq;    // [B,H,T] scale*||q_i||
+    float* qmax;        // [B,Hkv,nqt]
+};
+cudaError_t launch_tile_qmax(const TileQmaxParams& p, cudaStream_t s);
 
 struct CacheView {
     int B, Hkv, d, cap;
@@ -122,6 +137,7 @@ struct BwdParams {
     const float* qr;     // [B,H,T,d]  RoPE(q)
     const float* kh;     // [B,Hkv,T,d] khat
     const float* kr;     // [B,Hkv,T,d] RoPE(khat)
+    const float* qmax;   // [B,Hkv,nqt] tile row bounds (see TileQmaxParams), or NULL
     const float* rq;     // [B,Hkv,T]
     const float* rk;     // [B,Hkv,T]
     const float* pb;     // [B,Hkv,nqt,T] decay prefixes
