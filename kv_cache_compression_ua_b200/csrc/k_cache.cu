@@ -293,9 +293,29 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         n = n < 0 ? 0 : c.cap;
     }
     int out = 0;
+    const bool multi_pass = n > 4 * EPB;   // block-uniform
     for (int c0 = 0; c0 < n; c0 += EPB) {
         const int j = c0 + gidx;
         const bool valid = j < n;
+        // long caches: ask L2 for the entries of the next two passes now (no registers held);
+        // one lane per entry covers its whole 128-byte row; a cache of four passes or fewer skips this
+        if (multi_pass && gl == 0) {
+#pragma unroll
+            for (int ahead = 1; ahead <= 2; ++ahead) {
+                const int jn = j + ahead * EPB;
+                if (jn < n) {
+                    const size_t e = (base + jn) * DH;
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(khat + e));
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(krope + e));
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(vc + e));
+                    if ((jn & 31) == 0) {
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(c.bias + base + jn));
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(c.rk + base + jn));
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(c.pos + base + jn));
+                    }
+                }
+            }
+        }
         uint4 ra = make_uint4(0, 0, 0, 0), rb = ra, rv = ra;
         float bj = 0.f, rkj = 0.f;
         int pj = 0;
