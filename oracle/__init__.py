@@ -44,16 +44,16 @@ def _load():
         P = ctypes.c_void_p
         I = ctypes.c_int
         Dd = ctypes.c_double
-        lib.ora_prefill_fwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 4 + [I]
+        lib.ora_prefill_fwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 4 + [I, I]
         lib.ora_prefill_fwd.restype = I
-        lib.ora_lambda_bruteforce.argtypes = [I, I, I, I, P, P, P, P, P, P, I]
+        lib.ora_lambda_bruteforce.argtypes = [I, I, I, I, P, P, P, P, P, P, I, I]
         lib.ora_lambda_bruteforce.restype = I
         lib.ora_decode_step.argtypes = ([I, I, I, I, I, Dd, Dd] + [P] * 6 + [P] * 8 +
-                                        [Dd, Dd, Dd, P, P, P, P, P, I])
+                                        [Dd, Dd, Dd, P, P, P, P, P, I, I])
         lib.ora_decode_step.restype = I
         lib.ora_compact_order.argtypes = [I, P, P]
         lib.ora_compact_order.restype = I
-        lib.ora_prefill_bwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 8 + [I]
+        lib.ora_prefill_bwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 8 + [I, I]
         lib.ora_prefill_bwd.restype = I
         _lib = lib
     return _lib
@@ -71,8 +71,13 @@ def default_threads() -> int:
     return max(1, os.cpu_count() or 1)
 
 
+# Variant bits (the ablations; 0 = the method itself): a set bit 0 / 1 / 2 switches the
+# query / key / similarity decay mechanism off; bit 3 RMS-normalises the queries.
+VAR_NO_Q, VAR_NO_K, VAR_NO_SIM, VAR_QNORM = 1, 2, 4, 8
+
+
 def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0,
-                want_lambda=False, unit_mask=None, row_mask=None, nthreads=None):
+                want_lambda=False, unit_mask=None, row_mask=None, variant=0, nthreads=None):
     """Prefill forward of UA in fp64.
 
     Shapes: q, g [B,T,H,d]; k, v [B,T,Hkv,d]; a_q, a_k [B,T,Hkv]; alpha, beta [Hkv].
@@ -94,25 +99,28 @@ def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0
     rc = _load().ora_prefill_fwd(B, T, H, Hkv, d, float(scale), float(theta),
                                  _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
                                  _ptr(alpha), _ptr(beta), _ptr(um), _ptr(rm),
-                                 _ptr(o), _ptr(lse), _ptr(bfin), _ptr(lam),
+                                 _ptr(o), _ptr(lse), _ptr(bfin), _ptr(lam), int(variant),
                                  nthreads or default_threads())
     if rc != 0:
         raise ValueError(f"ora_prefill_fwd rejected the shapes (code {rc})")
     return {"o": o, "lse": lse, "b_final": bfin, "lam": lam}
 
 
-def lambda_bruteforce(k, a_q, a_k, alpha, beta, nthreads=None):
+def lambda_bruteforce(k, a_q, a_k, alpha, beta, variant=0, nthreads=None):
     """Lambda [B,Hkv,T,T] from the O(T^3) direct sum (lower triangle; zeros above)."""
     k, a_q, a_k, alpha, beta = _f64(k), _f64(a_q), _f64(a_k), _f64(alpha), _f64(beta)
     B, T, Hkv, d = k.shape
     lam = np.zeros((B, Hkv, T, T))
-    _load().ora_lambda_bruteforce(B, T, Hkv, d, _ptr(k), _ptr(a_q), _ptr(a_k), _ptr(alpha),
-                                  _ptr(beta), _ptr(lam), nthreads or default_threads())
+    rc = _load().ora_lambda_bruteforce(B, T, Hkv, d, _ptr(k), _ptr(a_q), _ptr(a_k), _ptr(alpha),
+                                       _ptr(beta), _ptr(lam), int(variant),
+                                       nthreads or default_threads())
+    if rc != 0:
+        raise ValueError(f"ora_lambda_bruteforce rejected the variant (code {rc})")
     return lam
 
 
 def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, d_o, *, scale=None, theta=500000.0,
-                unit_mask=None, nthreads=None):
+                unit_mask=None, variant=0, nthreads=None):
     """Analytic fp64 gradients of sum(dO * O).  Returns a dict keyed dq, dk, dv, dg,
     da_q, da_k, dalpha, dbeta (same shapes as the inputs)."""
     q, k, v, g, d_o = _f64(q), _f64(k), _f64(v), _f64(g), _f64(d_o)
@@ -131,7 +139,7 @@ def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, d_o, *, scale=None, theta=500
                                  _ptr(alpha), _ptr(beta), _ptr(d_o), _ptr(um),
                                  _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
                                  _ptr(out["dg"]), _ptr(out["da_q"]), _ptr(out["da_k"]),
-                                 _ptr(out["dalpha"]), _ptr(out["dbeta"]),
+                                 _ptr(out["dalpha"]), _ptr(out["dbeta"]), int(variant),
                                  nthreads or default_threads())
     if rc != 0:
         raise ValueError(f"ora_prefill_bwd rejected the shapes (code {rc})")
@@ -182,7 +190,7 @@ class DecodeCache:
 
 
 def decode_step(cache: DecodeCache, q, k, v, g, a_q, a_k, alpha, beta, pos_t, p, *,
-                scale=None, theta=500000.0, band=1e-3, adopt_keep=None, nthreads=None):
+                scale=None, theta=500000.0, band=1e-3, adopt_keep=None, variant=0, nthreads=None):
     """One decode step on the oracle cache (mutated in place).
 
     q, g [B,H,d]; k, v [B,Hkv,d]; a_q, a_k [B,Hkv].  Returns dict(o [B,H,d],
@@ -207,7 +215,7 @@ def decode_step(cache: DecodeCache, q, k, v, g, a_q, a_k, alpha, beta, pos_t, p,
                                  _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
                                  _ptr(alpha), _ptr(beta), float(pos_t), logp, float(band),
                                  _ptr(ak_), _ptr(o), _ptr(ev), _ptr(inb), _ptr(order),
-                                 nthreads or default_threads())
+                                 int(variant), nthreads or default_threads())
     if rc != 0:
         raise RuntimeError(f"ora_decode_step failed (code {rc})")
     return {"o": o, "evict": ev, "in_band": inb, "kept_order": order, "n_before": n_before}

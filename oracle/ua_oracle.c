@@ -33,6 +33,14 @@
  *   a_q, a_k    : [B, T, Hkv]       alpha, beta : [Hkv]
  *   lse         : [B, H, T]         b_final : [B, Hkv, T]     lambda : [B, Hkv, T, T]
  * Query head h reads KV head h / (H / Hkv); decay parameters belong to the KV head.
+ *
+ * Variants (the ablations of [S1] §5.4 with Table 3 and App. E with Table 6; [S3]
+ * interpretation paragraph), selected by a `variant` bit field, 0 = the method above:
+ *   bit 0 / 1 / 2 set: the query / key / similarity mechanism is switched off, and D is
+ *     the geometric mean of the rates left on: (prod of the n active rates)^(1/n).
+ *     All three off is rejected.
+ *   bit 3 set: queries are RMS-normalised per head before RoPE (Qwen3-style query norm,
+ *     unit gain): q' = q / sqrt(mean(q^2) + 1e-6).  Keys keep their L2 normalisation.
  */
 #include <math.h>
 #include <pthread.h>
@@ -88,6 +96,42 @@ static void rope(const double* x, int d, double pos, double theta, double sign, 
  * veto property: a zero rate in any factor gives exactly zero). */
 static double decay_rate(double rq, double rk, double rsim) { return cbrt(rq * rk * rsim); }
 
+/* Variant bits (see the header). */
+enum { VAR_NO_Q = 1, VAR_NO_K = 2, VAR_NO_SIM = 4, VAR_QNORM = 8, VAR_ALL = 15 };
+
+static int n_active(int variant) {
+    return !(variant & VAR_NO_Q) + !(variant & VAR_NO_K) + !(variant & VAR_NO_SIM);
+}
+
+/* Geometric mean of the rates whose mechanisms are on ([S1] §5.4, App. E: the ablations
+ * drop mechanisms from the combination).  With all three on this is decay_rate. */
+static double decay_active(double rq, double rk, double rsim, int variant) {
+    if (!(variant & (VAR_NO_Q | VAR_NO_K | VAR_NO_SIM))) return decay_rate(rq, rk, rsim);
+    double prod = 1.0;
+    if (!(variant & VAR_NO_Q)) prod *= rq;
+    if (!(variant & VAR_NO_K)) prod *= rk;
+    if (!(variant & VAR_NO_SIM)) prod *= rsim;
+    return n_active(variant) == 2 ? sqrt(prod) : prod;
+}
+
+/* Qwen3-style query normalisation ([S1] App. E): RMS norm over the head dimension with
+ * unit gain and eps 1e-6.  Returns the factor 1/sqrt(mean(x^2) + eps). */
+static double rms_normalise(const double* x, int d, double* out) {
+    double r = 1.0 / sqrt(dot(x, x, d) / (double)d + 1e-6);
+    for (int c = 0; c < d; ++c) out[c] = x[c] * r;
+    return r;
+}
+
+/* RoPE of a query, RMS-normalised first when the variant asks for it. */
+static void rope_query(const double* q, int d, double pos, double theta, int variant,
+                       double* tmp, double* out) {
+    if (variant & VAR_QNORM) {
+        rms_normalise(q, d, tmp);
+        q = tmp;
+    }
+    rope(q, d, pos, theta, 1.0, out);
+}
+
 /* ------------------------------------------------------------------ tiny thread pool */
 
 typedef void (*unit_fn)(void* ctx, int unit);
@@ -131,6 +175,7 @@ typedef struct {
     const uint8_t* unit_mask; /* [B*Hkv] or NULL = all units */
     const uint8_t* row_mask;  /* [T] or NULL = all rows get attention outputs */
     double *o, *lse, *bfinal, *lambda;
+    int variant;
 } fwd_ctx;
 
 static void fwd_unit(void* vctx, int unit) {
@@ -147,6 +192,7 @@ static void fwd_unit(void* vctx, int unit) {
     double* lam = (double*)malloc(sizeof(double) * (size_t)T);   /* row i of Lambda */
     double* srow = (double*)malloc(sizeof(double) * (size_t)T);
     double* qrot = (double*)malloc(sizeof(double) * (size_t)d);
+    double* qtmp = (double*)malloc(sizeof(double) * (size_t)d);
     double* acc = (double*)malloc(sizeof(double) * (size_t)d);
 
     for (int t = 0; t < T; ++t) {
@@ -162,7 +208,7 @@ static void fwd_unit(void* vctx, int unit) {
         for (int j = 0; j < i; ++j) {
             double sim = dot(khat + (size_t)i * d, khat + (size_t)j * d, d);
             double rsim = softplus(alpha * sim + beta);
-            lam[j] -= decay_rate(rq_i, rk[j], rsim);
+            lam[j] -= decay_active(rq_i, rk[j], rsim, c->variant);
         }
         lam[i] = 0.0;
         if (c->lambda) {
@@ -173,7 +219,7 @@ static void fwd_unit(void* vctx, int unit) {
         for (int hh = 0; hh < G; ++hh) {
             int h = kvh * G + hh;
             const double* qi = c->q + (((size_t)b * T + i) * H + h) * d;
-            rope(qi, d, (double)i, c->theta, 1.0, qrot);
+            rope_query(qi, d, (double)i, c->theta, c->variant, qtmp, qrot);
             double m = -INFINITY;
             for (int j = 0; j <= i; ++j) {
                 srow[j] = c->scale * dot(qrot, krot + (size_t)j * d, d) + lam[j];
@@ -197,7 +243,7 @@ static void fwd_unit(void* vctx, int unit) {
         double* bf = c->bfinal + ((size_t)b * Hkv + kvh) * T;
         for (int j = 0; j < T; ++j) bf[j] = lam[j];
     }
-    free(khat); free(krot); free(rk); free(lam); free(srow); free(qrot); free(acc);
+    free(khat); free(krot); free(rk); free(lam); free(srow); free(qrot); free(qtmp); free(acc);
 }
 
 /* Prefill forward.  Outputs that are NULL are skipped.  Only units with unit_mask set
@@ -206,10 +252,12 @@ int ora_prefill_fwd(int B, int T, int H, int Hkv, int d, double scale, double th
                     const double* q, const double* k, const double* v, const double* g,
                     const double* aq, const double* ak, const double* alpha, const double* beta,
                     const uint8_t* unit_mask, const uint8_t* row_mask,
-                    double* o, double* lse, double* bfinal, double* lambda, int nthreads) {
+                    double* o, double* lse, double* bfinal, double* lambda, int variant,
+                    int nthreads) {
     if (B < 1 || T < 1 || H < 1 || Hkv < 1 || d < 2 || (d & 1) || H % Hkv) return 1;
+    if ((variant & ~VAR_ALL) || n_active(variant) == 0) return 1;
     fwd_ctx c = {B, T, H, Hkv, d, scale, theta, q, k, v, g, aq, ak, alpha, beta,
-                 unit_mask, row_mask, o, lse, bfinal, lambda};
+                 unit_mask, row_mask, o, lse, bfinal, lambda, variant};
     run_units(fwd_unit, &c, B * Hkv, nthreads);
     return 0;
 }
@@ -220,6 +268,7 @@ typedef struct {
     int B, T, Hkv, d;
     const double *k, *aq, *ak, *alpha, *beta;
     double* lambda;
+    int variant;
 } brute_ctx;
 
 static void brute_unit(void* vctx, int unit) {
@@ -239,7 +288,7 @@ static void brute_unit(void* vctx, int unit) {
                     double rq = softplus(c->aq[((size_t)b * T + l) * Hkv + kvh]);
                     double rk = softplus(c->ak[((size_t)b * T + j) * Hkv + kvh]);
                     double rsim = softplus(c->alpha[kvh] * dot(kl, kj, d) + c->beta[kvh]);
-                    s -= decay_rate(rq, rk, rsim);
+                    s -= decay_active(rq, rk, rsim, c->variant);
                 }
             }
             c->lambda[(((size_t)b * Hkv + kvh) * T + i) * (size_t)T + j] = s;
@@ -251,8 +300,9 @@ static void brute_unit(void* vctx, int unit) {
 /* O(T^3 d) Lambda straight from its definition (tiny T only). */
 int ora_lambda_bruteforce(int B, int T, int Hkv, int d, const double* k, const double* aq,
                           const double* ak, const double* alpha, const double* beta,
-                          double* lambda, int nthreads) {
-    brute_ctx c = {B, T, Hkv, d, k, aq, ak, alpha, beta, lambda};
+                          double* lambda, int variant, int nthreads) {
+    if ((variant & ~VAR_ALL) || n_active(variant) == 0) return 1;
+    brute_ctx c = {B, T, Hkv, d, k, aq, ak, alpha, beta, lambda, variant};
     run_units(brute_unit, &c, B * Hkv, nthreads);
     return 0;
 }
@@ -284,6 +334,7 @@ typedef struct {
     double* o;
     uint8_t *evict, *in_band;
     int64_t* kept_order;
+    int variant;
 } dec_ctx;
 
 static void dec_unit(void* vctx, int unit) {
@@ -297,6 +348,7 @@ static void dec_unit(void* vctx, int unit) {
     double* kj_hat = (double*)malloc(sizeof(double) * (size_t)d);
     double* kj_rot = (double*)malloc(sizeof(double) * (size_t)d);
     double* qrot = (double*)malloc(sizeof(double) * (size_t)d);
+    double* qtmp = (double*)malloc(sizeof(double) * (size_t)d);
     double* acc = (double*)malloc(sizeof(double) * (size_t)d);
     double* logits = (double*)malloc(sizeof(double) * (size_t)(n + 1));
     uint8_t* keep = (uint8_t*)malloc((size_t)(n + 1));
@@ -313,7 +365,7 @@ static void dec_unit(void* vctx, int unit) {
         l2_normalise(c->kc + (base + j) * d, d, kj_hat);
         double rsim = softplus(alpha * dot(kt_hat, kj_hat, d) + beta);
         double rk = softplus(c->akc[base + j]);
-        c->bc[base + j] -= decay_rate(rq_t, rk, rsim);
+        c->bc[base + j] -= decay_active(rq_t, rk, rsim, c->variant);
         double bj = c->bc[base + j];
         keep[j] = bj >= c->logp;
         int inb = fabs(bj - c->logp) < c->band;
@@ -324,7 +376,7 @@ static void dec_unit(void* vctx, int unit) {
     /* 3: attention of the G query heads over survivors + the new token */
     for (int hh = 0; hh < G; ++hh) {
         int h = kvh * G + hh;
-        rope(c->q + ((size_t)b * H + h) * d, d, c->pos_t, c->theta, 1.0, qrot);
+        rope_query(c->q + ((size_t)b * H + h) * d, d, c->pos_t, c->theta, c->variant, qtmp, qrot);
         double m = -INFINITY;
         for (int j = 0; j < n; ++j) {
             if (!keep[j]) continue;
@@ -372,7 +424,7 @@ static void dec_unit(void* vctx, int unit) {
     } else {
         c->n_kept[unit] = -1; /* capacity exceeded */
     }
-    free(kt_hat); free(kt_rot); free(kj_hat); free(kj_rot); free(qrot); free(acc);
+    free(kt_hat); free(kt_rot); free(kj_hat); free(kj_rot); free(qrot); free(qtmp); free(acc);
     free(logits); free(keep);
 }
 
@@ -382,11 +434,12 @@ int ora_decode_step(int B, int H, int Hkv, int d, int cap, double scale, double 
                     const double* aq, const double* ak, const double* alpha, const double* beta,
                     double pos_t, double logp, double band, const uint8_t* adopt_keep,
                     double* o, uint8_t* evict, uint8_t* in_band, int64_t* kept_order,
-                    int nthreads) {
+                    int variant, int nthreads) {
     if (H % Hkv) return 1;
+    if ((variant & ~VAR_ALL) || n_active(variant) == 0) return 1;
     dec_ctx c = {B, H, Hkv, d, cap, scale, theta, logp, band, pos_t, n_kept, kc, vc, akc,
                  posc, bc, q, k, v, g, aq, ak, alpha, beta, adopt_keep, o, evict, in_band,
-                 kept_order};
+                 kept_order, variant};
     run_units(dec_unit, &c, B * Hkv, nthreads);
     for (int u = 0; u < B * Hkv; ++u)
         if (n_kept[u] < 0) return 2;
@@ -416,6 +469,10 @@ int ora_compact_order(int n, const uint8_t* keep, int64_t* order) {
  *   dX = w sigmoid(X)/softplus(X), X = alpha c + beta, c = <khat_l, khat_j>
  *   d alpha += dX c;  d beta += dX;  dkhat_l += alpha dX khat_j;  dkhat_j += alpha dX khat_l
  *   then dq = RoPE^T dqrot, dkhat += RoPE^T dkrot, dk = (dkhat - khat <khat,dkhat>)/||k||.
+ * Variants: with n mechanisms on, D = (product of the active rates)^(1/n), so
+ *   w = dD * D / n, and the a_q / a_k / (alpha, beta, khat-similarity) terms appear only
+ *   for the mechanisms that are on.  With the query norm q' = r q, r = 1/sqrt(mean(q^2)+eps):
+ *   dq = r (dq' - q' <q', dq'> / d), dq' = RoPE^T dqrot.
  * Lambda and dLambda are held as packed lower-triangular T x T matrices per unit.
  * dalpha / dbeta are summed over the batch: [Hkv].
  */
@@ -426,6 +483,7 @@ typedef struct {
     const uint8_t* unit_mask;
     double *dq, *dk, *dv, *dg, *daq, *dak;
     double *dalpha_u, *dbeta_u; /* per unit partials [B*Hkv] */
+    int variant;
 } bwd_ctx;
 
 static size_t tri(int i, int j) { return (size_t)i * (size_t)(i + 1) / 2 + (size_t)j; }
@@ -453,6 +511,7 @@ static void bwd_unit(void* vctx, int unit) {
     double* qrot = (double*)calloc((size_t)d, sizeof(double));
     double* dqrot = (double*)calloc((size_t)d, sizeof(double));
     double* tmp = (double*)calloc((size_t)d, sizeof(double));
+    double* qn = (double*)calloc((size_t)d, sizeof(double));
     double* A = (double*)calloc((size_t)d, sizeof(double));
     double* dA = (double*)calloc((size_t)d, sizeof(double));
     double* P = (double*)calloc((size_t)T, sizeof(double));
@@ -470,7 +529,7 @@ static void bwd_unit(void* vctx, int unit) {
         for (int j = 0; j < i; ++j) {
             double rsim = softplus(alpha * dot(khat + (size_t)i * d, khat + (size_t)j * d, d) + beta);
             double prev = (i - 1 >= j) ? lam[tri(i - 1, j)] : 0.0;
-            lam[tri(i, j)] = prev - decay_rate(rq[i], rk[j], rsim);
+            lam[tri(i, j)] = prev - decay_active(rq[i], rk[j], rsim, c->variant);
         }
     }
     /* attention part, head by head, row by row */
@@ -480,7 +539,7 @@ static void bwd_unit(void* vctx, int unit) {
             const double* qi = c->q + (((size_t)b * T + i) * H + h) * d;
             const double* gi = c->g + (((size_t)b * T + i) * H + h) * d;
             const double* doi = c->dout + (((size_t)b * T + i) * H + h) * d;
-            rope(qi, d, (double)i, c->theta, 1.0, qrot);
+            rope_query(qi, d, (double)i, c->theta, c->variant, qn, qrot);
             double m = -INFINITY;
             for (int j = 0; j <= i; ++j) {
                 P[j] = s * dot(qrot, krot + (size_t)j * d, d) + lam[tri(i, j)];
@@ -518,6 +577,12 @@ static void bwd_unit(void* vctx, int unit) {
             }
             double* dqi = c->dq + (((size_t)b * T + i) * H + h) * d;
             rope(dqrot, d, (double)i, c->theta, -1.0, dqi);
+            if (c->variant & VAR_QNORM) {
+                /* back through q' = r q: qn holds q' from rope_query */
+                double r = rms_normalise(qi, d, qn);
+                double pr = dot(qn, dqi, d);
+                for (int x = 0; x < d; ++x) dqi[x] = r * (dqi[x] - qn[x] * pr / (double)d);
+            }
         }
     }
     /* dD[l,j] = -sum_{i>=l} dLambda_ij, then through the geometric mean and softplus */
@@ -529,12 +594,14 @@ static void bwd_unit(void* vctx, int unit) {
             double dD = -suffix;
             double cs = dot(khat + (size_t)l * d, khat + (size_t)j * d, d);
             double X = alpha * cs + beta;
-            double D = decay_rate(rq[l], rk[j], softplus(X));
+            double D = decay_active(rq[l], rk[j], softplus(X), c->variant);
             if (D == 0.0) continue;
-            double w = dD * D / 3.0;
-            daq[l] += w * sig_over_softplus(c->aq[((size_t)b * T + l) * Hkv + kvh]);
-            dak[j] += w * sig_over_softplus(c->ak[((size_t)b * T + j) * Hkv + kvh]);
-            double dX = w * sig_over_softplus(X);
+            double w = dD * D / (double)n_active(c->variant);
+            if (!(c->variant & VAR_NO_Q))
+                daq[l] += w * sig_over_softplus(c->aq[((size_t)b * T + l) * Hkv + kvh]);
+            if (!(c->variant & VAR_NO_K))
+                dak[j] += w * sig_over_softplus(c->ak[((size_t)b * T + j) * Hkv + kvh]);
+            double dX = (c->variant & VAR_NO_SIM) ? 0.0 : w * sig_over_softplus(X);
             dal += dX * cs;
             dbe += dX;
             for (int x = 0; x < d; ++x) {
@@ -565,7 +632,7 @@ static void bwd_unit(void* vctx, int unit) {
 
     free(khat); free(knorm); free(krot); free(rq); free(rk); free(lam); free(dlam);
     free(dkhat); free(dkrot); free(dvl); free(daq); free(dak); free(qrot); free(dqrot);
-    free(tmp); free(A); free(dA); free(P); free(dP);
+    free(tmp); free(qn); free(A); free(dA); free(P); free(dP);
 }
 
 int ora_prefill_bwd(int B, int T, int H, int Hkv, int d, double scale, double theta,
@@ -573,12 +640,13 @@ int ora_prefill_bwd(int B, int T, int H, int Hkv, int d, double scale, double th
                     const double* aq, const double* ak, const double* alpha, const double* beta,
                     const double* dout, const uint8_t* unit_mask,
                     double* dq, double* dk, double* dv, double* dg, double* daq, double* dak,
-                    double* dalpha, double* dbeta, int nthreads) {
+                    double* dalpha, double* dbeta, int variant, int nthreads) {
     if (B < 1 || T < 1 || H < 1 || Hkv < 1 || d < 2 || (d & 1) || H % Hkv) return 1;
+    if ((variant & ~VAR_ALL) || n_active(variant) == 0) return 1;
     double* dal_u = (double*)calloc((size_t)B * Hkv, sizeof(double));
     double* dbe_u = (double*)calloc((size_t)B * Hkv, sizeof(double));
     bwd_ctx c = {B, T, H, Hkv, d, scale, theta, q, k, v, g, aq, ak, alpha, beta, dout,
-                 unit_mask, dq, dk, dv, dg, daq, dak, dal_u, dbe_u};
+                 unit_mask, dq, dk, dv, dg, daq, dak, dal_u, dbe_u, variant};
     run_units(bwd_unit, &c, B * Hkv, nthreads);
     for (int h = 0; h < Hkv; ++h) {
         dalpha[h] = 0.0;
