@@ -63,6 +63,21 @@ typedef enum {
 
 typedef enum { UA_F32 = 0, UA_BF16 = 1 } ua_dtype;
 
+/* Variant bits: the ablations of "A Self-Pruning Transformer: Extreme KV-Cache Compression
+ * with Universal Attention" (paperlayer.ai summary, §5.4 with Table 3 and App. E with
+ * Table 6; ai4snews synopsis, interpretation paragraph).  0 is the method itself.
+ *   UA_VAR_NO_QUERY_DECAY / UA_VAR_NO_KEY_DECAY / UA_VAR_NO_SIM_DECAY switch one decay
+ *     mechanism off; the decay rate is then the geometric mean of the rates left on,
+ *     D = (product of the n active rates)^(1/n).  Switching all three off is
+ *     UA_ERR_INVALID_ARG.
+ *   UA_VAR_QUERY_NORM RMS-normalises every query head before RoPE (Qwen3-style query norm
+ *     with unit gain): q' = q / sqrt(mean(q^2) + 1e-6).  Keys keep their L2 normalisation.
+ * Any other bit is UA_ERR_INVALID_ARG. */
+#define UA_VAR_NO_QUERY_DECAY 1
+#define UA_VAR_NO_KEY_DECAY 2
+#define UA_VAR_NO_SIM_DECAY 4
+#define UA_VAR_QUERY_NORM 8
+
 /* Problem shape of a prefill call.  d (head_dim) must be 64 or 128; H % Hkv == 0 and
  * H / Hkv in {1, 2, 3, 4, 8}; T >= 1. */
 typedef struct {
@@ -70,6 +85,7 @@ typedef struct {
     float scale;          /* logit scale, usually 1/sqrt(d); multiplies only QK^T */
     double rope_theta;    /* RoPE base, e.g. 500000 */
     ua_dtype dtype;       /* activation dtype of q, k, v, g, o (and gradients) */
+    int variant;          /* UA_VAR_* bits, 0 = Universal Attention as published */
 } ua_shape;
 
 /* ------------------------------------------------------------------ prefill forward
@@ -102,9 +118,10 @@ ua_status ua_prefill_workspace_size(const ua_shape* shape, size_t* bytes);
  * key column, so the prefix above the tile bounds the whole tile).  When b_final is requested
  * the decay of such a tile is still evaluated (b_final stays exact); when b_final is NULL the
  * tile is skipped entirely.  Either way every requested output is identical to the unskipped
- * computation (see ua_prefill_tile_stats).  All other problems,
- * and every call that asks for lambda_dbg, run the fp32 SIMT path, which uses a running
- * maximum. */
+ * computation (see ua_prefill_tile_stats).  The tensor-core path computes the
+ * three-rate geometric mean only; it takes UA_VAR_QUERY_NORM, but a shape with a decay
+ * mechanism switched off runs the SIMT path.  All other problems, and every call that asks
+ * for lambda_dbg, run the fp32 SIMT path, which uses a running maximum. */
 ua_status ua_prefill_fwd(const ua_shape* shape, const void* q, const void* k, const void* v,
                          const void* g, const float* a_q, const float* a_k, const float* alpha,
                          const float* beta, void* o, float* lse, float* b_final, float* lambda_dbg,
@@ -209,7 +226,8 @@ ua_status ua_cache_compact(const ua_cache* cache, const uint8_t* keep, float p,
  * evict_bits (optional, [B,Hkv,ceil(cap/32)] uint32): bit s set when pre-step slot s was
  * evicted (all words are written).  kept_idx (optional, [B,Hkv,cap] int32): pre-step
  * slot of each survivor in new order, then -1 for the appended token.
- * flags: reserved, pass 0.  Every cache call requires capacity <= 2^20 slots
+ * flags: UA_VAR_* bits, which must equal the variant of the prefill that filled the cache
+ * (0 = the method itself; the cache stores softplus(a_k) whatever the variant).  Every cache call requires capacity <= 2^20 slots
  * (UA_ERR_UNSUPPORTED otherwise).  If a cache is full (no pair evicted and n_kept == capacity)
  * the step sets UA_ERR_CAPACITY in the device status word and that cache is left as it
  * was after compaction, without the new token. */

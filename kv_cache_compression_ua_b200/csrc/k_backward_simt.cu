@@ -116,12 +116,15 @@ struct Ctx {
     const float *aq, *ak, *rq, *rk, *alpha, *beta, *lse, *delta, *pb;
     const float* qmax;   // [B,Hkv,nqt] tile row bounds, or NULL (no skipping)
     float *dpb, *dqr, *dkh_rows, *dkh_keys, *dkr, *dv32, *daq32, *dak32, *dab;
+    int variant;         // UA_VAR_* bits
+    float inv_n;         // 1 / number of decay mechanisms on (1/3 for the method itself)
 };
 
 // Decay tile D[l, j] and Lambda for query tile starting at i0 and key tile at j0.  Needs
 // khq/khk/rowv(rq)/colv(rk, pb) loaded; leaves D and L filled.
 template <int DH>
-__device__ void decay_tile(const Tiles<DH>& t, int i0, int j0, int T, float al, float be, int ty, int tx, int tid) {
+__device__ void decay_tile(const Tiles<DH>& t, int i0, int j0, int T, float al, float be, int variant, int ty, int tx,
+                           int tid) {
     constexpr int LP = BN + 1;
     float acc[4][2];
     tile_dots<DH>(t.khq, t.khk, ty, tx, acc);
@@ -131,7 +134,7 @@ __device__ void decay_tile(const Tiles<DH>& t, int i0, int j0, int T, float al, 
         for (int cc = 0; cc < 2; ++cc) {
             const int r = ty + 16 * rr, c = tx + 16 * cc, i = i0 + r, j = j0 + c;
             float D = 0.f;
-            if (i > j && i < T && j < T) D = decay_geo(t.rowv[r], t.colv[c], softplus_f(fmaf(al, acc[rr][cc], be)));
+            if (i > j && i < T && j < T) D = decay_var(t.rowv[r], t.colv[c], fmaf(al, acc[rr][cc], be), variant);
             t.D[r * LP + c] = D;
         }
     __syncthreads();
@@ -210,6 +213,7 @@ __global__ void __launch_bounds__(NT) k_bwd_keys(Ctx c) {
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const size_t unit = (size_t)b * c.Hkv + kvh;
     const float al = c.alpha[kvh], be = c.beta[kvh];
+    const bool sim_on = !(c.variant & kVarNoSim);   // similarity mechanism on: dX terms exist
     const TI* vin = static_cast<const TI*>(c.v);
     const TI* gin = static_cast<const TI*>(c.g);
     const TI* doin = static_cast<const TI*>(c.d_o);
@@ -224,7 +228,8 @@ __global__ void __launch_bounds__(NT) k_bwd_keys(Ctx c) {
     if (tid < BN) {
         const int j = j0 + tid;
         t.colv[tid] = j < T ? c.rk[unit * T + j] : 0.f;
-        t.colv[2 * BN + tid] = j < T ? sig_over_sp(c.ak[((size_t)b * T + j) * c.Hkv + kvh]) : 0.f;
+        // d log r_k / d a_k; zero when the key mechanism is off (r_k is then the constant 1)
+        t.colv[2 * BN + tid] = j < T && !(c.variant & kVarNoK) ? sig_over_sp(c.ak[((size_t)b * T + j) * c.Hkv + kvh]) : 0.f;
     }
     // key accumulators: thread owns key kc = tid / 8 and dims (tid % 8) + 8 m
     const int kc = tid >> 3, kd = tid & 7;
@@ -257,7 +262,7 @@ __global__ void __launch_bounds__(NT) k_bwd_keys(Ctx c) {
         } else {
             __syncthreads();
         }
-        decay_tile<DH>(t, i0, j0, T, al, be, ty, tx, tid);
+        decay_tile<DH>(t, i0, j0, T, al, be, c.variant, ty, tx, tid);
         for (int hh = 0; hh < c.G; ++hh) {
             const int h = kvh * c.G + hh;
             __syncthreads();
@@ -298,8 +303,8 @@ __global__ void __launch_bounds__(NT) k_bwd_keys(Ctx c) {
                 sdl += t.dL[r * LP + tid];
                 const int i = i0 + r;
                 const float D = t.D[r * LP + tid];
-                // w = dD * D / 3 with dD = -sdl; stored in dS for the dX pass below
-                t.dS[r * LP + tid] = (i > j && D > 0.f) ? -sdl * D * (1.f / 3.f) : 0.f;
+                // w = dD * D / n with dD = -sdl (n mechanisms on); stored in dS for the dX pass below
+                t.dS[r * LP + tid] = (i > j && D > 0.f) ? -sdl * D * c.inv_n : 0.f;
             }
         }
         __syncthreads();
@@ -313,7 +318,7 @@ __global__ void __launch_bounds__(NT) k_bwd_keys(Ctx c) {
                     const int r = ty + 16 * rr, cl = tx + 16 * cc;
                     const float w = t.dS[r * LP + cl];
                     const float X = fmaf(al, acc[rr][cc], be);
-                    const float dX = w != 0.f ? w * sig_over_sp(X) : 0.f;
+                    const float dX = w != 0.f && sim_on ? w * sig_over_sp(X) : 0.f;
                     dal = fmaf(dX, acc[rr][cc], dal);
                     dbe += dX;
                     t.P[r * LP + cl] = dX;                // reuse P for dX
@@ -383,6 +388,7 @@ __global__ void __launch_bounds__(NT) k_bwd_rows(Ctx c) {
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const size_t unit = (size_t)b * c.Hkv + kvh;
     const float al = c.alpha[kvh], be = c.beta[kvh];
+    const bool sim_on = !(c.variant & kVarNoSim);   // similarity mechanism on: dX terms exist
     const TI* vin = static_cast<const TI*>(c.v);
     const TI* gin = static_cast<const TI*>(c.g);
     const TI* doin = static_cast<const TI*>(c.d_o);
@@ -391,7 +397,7 @@ __global__ void __launch_bounds__(NT) k_bwd_rows(Ctx c) {
     if (tid < BM) {
         const int i = i0 + tid;
         t.rowv[tid] = i < T ? c.rq[unit * T + i] : 0.f;
-        t.rowv[3 * BM + tid] = i < T ? sig_over_sp(c.aq[((size_t)b * T + i) * c.Hkv + kvh]) : 0.f;
+        t.rowv[3 * BM + tid] = i < T && !(c.variant & kVarNoQ) ? sig_over_sp(c.aq[((size_t)b * T + i) * c.Hkv + kvh]) : 0.f;
     }
     float aQ[G][4][ND], aKh[4][ND], daq[4];
 #pragma unroll
@@ -428,7 +434,7 @@ __global__ void __launch_bounds__(NT) k_bwd_rows(Ctx c) {
         } else {
             __syncthreads();
         }
-        decay_tile<DH>(t, i0, j0, T, al, be, ty, tx, tid);
+        decay_tile<DH>(t, i0, j0, T, al, be, c.variant, ty, tx, tid);
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) {
             const int h = kvh * G + hh;
@@ -470,7 +476,7 @@ __global__ void __launch_bounds__(NT) k_bwd_rows(Ctx c) {
                 sd += t.dL[r * LP + tid];
                 const int i = i0 + r;
                 const float D = t.D[r * LP + tid];
-                t.dS[r * LP + tid] = (i > j && D > 0.f) ? -sd * D * (1.f / 3.f) : 0.f;   // w
+                t.dS[r * LP + tid] = (i > j && D > 0.f) ? -sd * D * c.inv_n : 0.f;   // w
             }
         }
         __syncthreads();
@@ -484,7 +490,7 @@ __global__ void __launch_bounds__(NT) k_bwd_rows(Ctx c) {
                     const int r = ty + 16 * rr, cl = tx + 16 * cc;
                     const float w = t.dS[r * LP + cl];
                     const float X = fmaf(al, acc[rr][cc], be);
-                    t.P[r * LP + cl] = w != 0.f ? w * sig_over_sp(X) : 0.f;   // dX
+                    t.P[r * LP + cl] = w != 0.f && sim_on ? w * sig_over_sp(X) : 0.f;   // dX
                 }
         }
         __syncthreads();
@@ -532,13 +538,49 @@ __global__ void __launch_bounds__(256) k_bwd_post(Ctx c, BwdParams p) {
     for (int hh = warp; hh < c.H + c.Hkv; hh += 8) {
         const bool is_q = hh < c.H;
         const int h = is_q ? hh : hh - c.H;
-        if (is_q) {
+        if (is_q && !(p.variant & kVarQNorm)) {
             const float* src = c.dqr + (((size_t)b * c.H + h) * T + t) * d;
             TI* dst = dq + (((size_t)b * T + t) * c.H + h) * d;
             for (int m = lane; m < half; m += 32) {
                 const float x0 = src[m], x1 = src[m + half], cs = s_cos[m], sn = s_sin[m];
                 Elem<TI>::st(dst + m, x0 * cs + x1 * sn);          // rotation by -angle
                 Elem<TI>::st(dst + m + half, x1 * cs - x0 * sn);
+            }
+        } else if (is_q) {
+            // query norm q' = r q, r = 1/sqrt(mean(q^2) + eps):  dq = r (dq' - q' <q', dq'> / d),
+            // dq' = RoPE^T dqrot
+            const float* src = c.dqr + (((size_t)b * c.H + h) * T + t) * d;
+            const TI* qraw = static_cast<const TI*>(p.q) + (((size_t)b * T + t) * c.H + h) * d;
+            TI* dst = dq + (((size_t)b * T + t) * c.H + h) * d;
+            float y0[2] = {0.f, 0.f}, y1[2] = {0.f, 0.f}, q0[2] = {0.f, 0.f}, q1[2] = {0.f, 0.f};
+            float ss = 0.f, qy = 0.f;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int m = lane + 32 * u;
+                if (m < half) {
+                    const float x0 = src[m], x1 = src[m + half], cs = s_cos[m], sn = s_sin[m];
+                    y0[u] = x0 * cs + x1 * sn;
+                    y1[u] = x1 * cs - x0 * sn;
+                    q0[u] = Elem<TI>::ld(qraw + m);
+                    q1[u] = Elem<TI>::ld(qraw + m + half);
+                    ss += q0[u] * q0[u] + q1[u] * q1[u];
+                    qy += q0[u] * y0[u] + q1[u] * y1[u];
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                qy += __shfl_xor_sync(0xffffffffu, qy, o);
+            }
+            const float r = 1.f / sqrtf(ss / (float)d + kQNormEps);
+            const float k = r * r * qy / (float)d;        // <q', dq'> / d, divided by r once more
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int m = lane + 32 * u;
+                if (m < half) {
+                    Elem<TI>::st(dst + m, r * (y0[u] - q0[u] * k));
+                    Elem<TI>::st(dst + m + half, r * (y1[u] - q1[u] * k));
+                }
             }
         } else {
             const size_t u = (size_t)b * c.Hkv + h;
@@ -639,6 +681,7 @@ static cudaError_t bwd_inst(const BwdParams& p, cudaStream_t s) {
     c.aq = p.a_q; c.ak = p.a_k; c.rq = p.rq; c.rk = p.rk; c.alpha = p.alpha; c.beta = p.beta; c.lse = p.lse;
     c.delta = p.delta; c.pb = p.pb; c.qmax = p.qmax; c.dpb = p.dpb; c.dqr = p.dqr; c.dkh_rows = p.dkh_rows; c.dkh_keys = p.dkh;
     c.dkr = p.dkr; c.dv32 = p.dv32; c.daq32 = p.daq32; c.dak32 = p.dak32; c.dab = p.dab;
+    c.variant = p.variant; c.inv_n = var_inv_n(p.variant);
     const size_t smem = tiles_bytes<DH>();
     cudaError_t e;
     {

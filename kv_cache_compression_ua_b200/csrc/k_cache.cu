@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     using L = EntryLayout<TC, DH>;
     constexpr int VEC = L::VEC, LPE = L::LPE, EPB = L::EPB, NW = L::NW;
     constexpr int half = DH / 2;
-    __shared__ float s_kt[DH], s_ktr[DH], s_vt[DH], s_q[G][DH], s_lt[G], s_g[G * DH];
+    __shared__ float s_kt[DH], s_ktr[DH], s_vt[DH], s_q[G][DH], s_lt[G], s_g[G * DH], s_qn[G];
     __shared__ float s_red[NW];
     __shared__ int s_wcnt[NW];
     extern __shared__ float dsm[];
@@ -264,13 +264,23 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         s_ktr[m + half] = x1 * cs + x0 * sn;
     }
     __syncthreads();
+    if (p.variant & kVarQNorm) {                  // query RMS norm (RoPE keeps the norm)
+        if (tid < G) {
+            float qq = 0.f;
+            for (int x = 0; x < DH; ++x) qq = fmaf(s_q[tid][x], s_q[tid][x], qq);
+            s_qn[tid] = 1.f / sqrtf(qq * (1.f / DH) + kQNormEps);
+        }
+        __syncthreads();
+        for (int e = tid; e < G * DH; e += blockDim.x) s_q[e / DH][e % DH] *= s_qn[e / DH];
+        __syncthreads();
+    }
     if (tid < G) {
         float a = 0.f;
         for (int x = 0; x < DH; ++x) a = fmaf(s_q[tid][x], s_ktr[x], a);
         s_lt[tid] = a * p.scale;                      // new token's own bias is 0
     }
-    const float rq_t = softplus_f(aq_t);
-    const float rk_t = softplus_f(ak_t);
+    const float rq_t = (p.variant & kVarNoQ) ? 1.f : softplus_f(aq_t);
+    const float rk_t = softplus_f(ak_t);          // stored in the cache as is
 
     float kq[VEC], qh[G][VEC];
 #pragma unroll
@@ -336,7 +346,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
 #pragma unroll
         for (int e = 0; e < VEC; ++e) sim = fmaf(kq[e], xa[e], sim);
         sim = group_sum<LPE>(sim);
-        const float D = decay_geo(rq_t, rkj, softplus_f(fmaf(al, sim, be)));
+        const float D = decay_var(rq_t, (p.variant & kVarNoK) ? 1.f : rkj, fmaf(al, sim, be), p.variant);
         const float bnew = bj - D;
         const bool keep = valid && (bnew >= p.logp);
 #pragma unroll

@@ -75,6 +75,15 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p) {
         if (!valid) continue;
         TW* dst_rot;
         if (is_q) {
+            if (p.variant & kVarQNorm) {              // Qwen3-style RMS norm, unit gain
+                const float r = 1.f / sqrtf(ss * (1.f / DH) + kQNormEps);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    x0[e] *= r;
+                    x1[e] *= r;
+                }
+                ss *= r * r;
+            }
             if (p.mq && c == 0) p.mq[((size_t)b * p.H + h) * p.Tp + t] = p.mq_scale * sqrtf(ss);
             dst_rot = static_cast<TW*>(p.qr) + (((size_t)b * p.H + h) * T + t) * DH;
         } else {
@@ -104,7 +113,9 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p) {
         if (t >= T) continue;
         const size_t src = ((size_t)b * T + t) * p.Hkv + h;
         const size_t dst = ((size_t)b * p.Hkv + h) * T + t;
-        const float sq = softplus_f(p.a_q[src]), sk = softplus_f(p.a_k[src]);
+        // a switched-off mechanism contributes the neutral rate 1 to the geometric mean
+        const float sq = (p.variant & kVarNoQ) ? 1.f : softplus_f(p.a_q[src]);
+        const float sk = (p.variant & kVarNoK) ? 1.f : softplus_f(p.a_k[src]);
         if (p.rq) p.rq[dst] = sq;
         if (p.rk) p.rk[dst] = sk;
         if (p.lq2) {
@@ -182,7 +193,7 @@ __global__ void __launch_bounds__(128) k_boundary_simt(BoundaryParams p) {
                 float s = 0.f;
 #pragma unroll
                 for (int c = 0; c < DH; ++c) s = fmaf(s_k[r][c], kj[c], s);
-                acc += decay_geo(s_rq[r], rkj, softplus_f(fmaf(al, s, be)));
+                acc += decay_var(s_rq[r], rkj, fmaf(al, s, be), p.variant);
             }
         }
     }
@@ -281,7 +292,7 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
                     const int r = ty + 16 * rr, c = tx + 16 * cc;
                     const int i = i0 + r, j = j0 + c;
                     float D = 0.f;
-                    if (i > j && i < T && j < T) D = decay_geo(sRq[r], sRk[c], softplus_f(fmaf(al, s[rr][cc], be)));
+                    if (i > j && i < T && j < T) D = decay_var(sRq[r], sRk[c], fmaf(al, s[rr][cc], be), p.variant);
                     sL[r * LP + c] = D;
                 }
         }

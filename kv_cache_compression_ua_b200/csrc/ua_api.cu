@@ -25,6 +25,9 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool group_ok(int G) { return G == 1 || G == 2 || G == 3 || G == 4 || G == 8; }
 
+// Known bits only, and at least one decay mechanism left on.
+bool variant_ok(int v) { return (v & ~(kVarMech | kVarQNorm)) == 0 && (v & kVarMech) != kVarMech; }
+
 ua_status check_shape(const ua_shape* s) {
     if (!s) return UA_ERR_INVALID_ARG;
     if (s->B < 1 || s->T < 1 || s->H < 1 || s->Hkv < 1) return UA_ERR_INVALID_ARG;
@@ -33,6 +36,7 @@ ua_status check_shape(const ua_shape* s) {
     if (s->d != 64 && s->d != 128) return UA_ERR_UNSUPPORTED;
     if (!group_ok(s->H / s->Hkv)) return UA_ERR_UNSUPPORTED;
     if (s->dtype != UA_F32 && s->dtype != UA_BF16) return UA_ERR_UNSUPPORTED;
+    if (!variant_ok(s->variant)) return UA_ERR_INVALID_ARG;
     return UA_OK;
 }
 
@@ -87,7 +91,11 @@ TcWs tc_ws_layout(const ua_shape* s) {
     return w;
 }
 
-bool use_tc(const ua_shape* s) { return s->dtype == UA_BF16 && fwd_tc_supported(s->d, s->H / s->Hkv); }
+// The tensor-core forward evaluates the three-rate geometric mean only (its decay runs in
+// log2 units with the cube root folded in); a shape with a mechanism switched off runs SIMT.
+bool use_tc(const ua_shape* s) {
+    return s->dtype == UA_BF16 && fwd_tc_supported(s->d, s->H / s->Hkv) && (s->variant & kVarMech) == 0;
+}
 
 size_t prefill_ws_bytes(const ua_shape* s) {
     size_t n = fwd_ws_layout(s).total;
@@ -176,6 +184,7 @@ static ua_status prefill_fwd_simt(const ua_shape* s, const void* q, const void* 
     pp.rq = reinterpret_cast<float*>(at(ws, w.rq)); pp.rk = reinterpret_cast<float*>(at(ws, w.rk));
     pp.rf = rope_freq(s->rope_theta, s->d);
     pp.mq = reinterpret_cast<float*>(at(ws, w.mq)); pp.Tp = s->T; pp.mq_scale = s->scale;
+    pp.variant = s->variant;
     if ((st = cuda_status(launch_prep(pp, bf, false, cs))) != UA_OK) return st;
     TileQmaxParams tq;
     tq.B = s->B; tq.T = s->T; tq.H = s->H; tq.Hkv = s->Hkv; tq.nqt = nqt; tq.mq = pp.mq;
@@ -186,7 +195,7 @@ static ua_status prefill_fwd_simt(const ua_shape* s, const void* q, const void* 
     bp.B = s->B; bp.T = s->T; bp.Hkv = s->Hkv; bp.d = s->d; bp.bq = kBq; bp.nqt = nqt;
     bp.kh = reinterpret_cast<const float*>(pp.kh); bp.rq = pp.rq; bp.rk = pp.rk;
     bp.alpha = alpha; bp.beta = beta;
-    bp.pb = reinterpret_cast<float*>(at(ws, w.pb)); bp.bfinal = b_final;
+    bp.pb = reinterpret_cast<float*>(at(ws, w.pb)); bp.bfinal = b_final; bp.variant = s->variant;
     if ((st = cuda_status(launch_boundary_simt(bp, cs))) != UA_OK) return st;
 
     if (lambda_dbg) {
@@ -200,7 +209,7 @@ static ua_status prefill_fwd_simt(const ua_shape* s, const void* q, const void* 
     fp.kr = reinterpret_cast<const float*>(pp.kr);
     fp.v = v; fp.g = g; fp.rq = pp.rq; fp.rk = pp.rk; fp.alpha = alpha; fp.beta = beta; fp.pb = bp.pb;
     fp.qmax = tq.qmax;
-    fp.o = o; fp.lse = lse; fp.lambda_dbg = lambda_dbg;
+    fp.o = o; fp.lse = lse; fp.lambda_dbg = lambda_dbg; fp.variant = s->variant;
     return cuda_status(launch_fwd_simt(fp, bf, cs));
 }
 
@@ -219,6 +228,7 @@ static ua_status prefill_fwd_tc(const ua_shape* s, const void* q, const void* k,
     pp.lq2 = reinterpret_cast<float*>(at(ws, w.lq2)); pp.lk2 = reinterpret_cast<float*>(at(ws, w.lk2));
     pp.mq = reinterpret_cast<float*>(at(ws, w.mq));
     pp.rf = rope_freq(s->rope_theta, s->d);
+    pp.variant = s->variant;   // the query norm only: use_tc excludes the mechanism bits
     if ((st = cuda_status(launch_prep(pp, true, true, cs))) != UA_OK) return st;
 
     // the fused forward zeroes its publication counters and ticket itself (stream-ordered)
@@ -367,6 +377,7 @@ ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const 
     pp.rq = reinterpret_cast<float*>(at(ws, w.f.rq)); pp.rk = reinterpret_cast<float*>(at(ws, w.f.rk));
     pp.rf = rope_freq(s->rope_theta, s->d);
     pp.mq = reinterpret_cast<float*>(at(ws, w.f.mq)); pp.Tp = s->T; pp.mq_scale = s->scale;
+    pp.variant = s->variant;
     if ((st = cuda_status(launch_prep(pp, bf, false, cs))) != UA_OK) return st;
     TileQmaxParams tq;
     tq.B = s->B; tq.T = s->T; tq.H = s->H; tq.Hkv = s->Hkv; tq.nqt = w.nqt; tq.mq = pp.mq;
@@ -375,7 +386,7 @@ ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const 
     BoundaryParams bp;
     bp.B = s->B; bp.T = s->T; bp.Hkv = s->Hkv; bp.d = s->d; bp.bq = kBq; bp.nqt = w.nqt;
     bp.kh = reinterpret_cast<const float*>(pp.kh); bp.rq = pp.rq; bp.rk = pp.rk; bp.alpha = alpha; bp.beta = beta;
-    bp.pb = reinterpret_cast<float*>(at(ws, w.f.pb)); bp.bfinal = nullptr;
+    bp.pb = reinterpret_cast<float*>(at(ws, w.f.pb)); bp.bfinal = nullptr; bp.variant = s->variant;
     if ((st = cuda_status(launch_boundary_simt(bp, cs))) != UA_OK) return st;
 
     BwdParams p;
@@ -391,6 +402,7 @@ ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const 
     p.dv32 = reinterpret_cast<float*>(at(ws, w.dv32)); p.daq32 = reinterpret_cast<float*>(at(ws, w.daq));
     p.dak32 = reinterpret_cast<float*>(at(ws, w.dak)); p.dab = reinterpret_cast<float*>(at(ws, w.dab));
     p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.da_q = da_q; p.da_k = da_k; p.dalpha = dalpha; p.dbeta = dbeta;
+    p.q = q; p.variant = s->variant;
     return cuda_status(launch_bwd_simt(p, bf, cs));
 }
 
@@ -425,7 +437,7 @@ ua_status ua_decode_step(const ua_cache* c, int H, const void* q, const void* k,
                          int32_t* kept_idx, int flags, void* stream) {
     ua_status st = check_cache(c);
     if (st != UA_OK) return st;
-    if (H < 1 || H % c->Hkv != 0 || pos_t < 0 || flags != 0) return UA_ERR_INVALID_ARG;
+    if (H < 1 || H % c->Hkv != 0 || pos_t < 0 || !variant_ok(flags)) return UA_ERR_INVALID_ARG;
     if (!group_ok(H / c->Hkv)) return UA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !g || !a_q || !a_k || !alpha || !beta || !o) return UA_ERR_INVALID_ARG;
     if (!(p >= 0.f && p <= 1.f) || !isfinite(scale) || !(rope_theta > 0.0)) return UA_ERR_INVALID_ARG;
@@ -436,7 +448,7 @@ ua_status ua_decode_step(const ua_cache* c, int H, const void* q, const void* k,
     dp.c = view(c); dp.H = H; dp.G = H / c->Hkv; dp.pos_t = pos_t; dp.scale = scale;
     dp.logp = p > 0.f ? logf(p) : -INFINITY; dp.theta = rope_theta; dp.rf = rope_freq(rope_theta, c->d);
     dp.q = q; dp.k = k; dp.v = v; dp.g = g; dp.a_q = a_q; dp.a_k = a_k; dp.alpha = alpha; dp.beta = beta;
-    dp.o = o; dp.evict_bits = evict_bits; dp.kept_idx = kept_idx;
+    dp.o = o; dp.evict_bits = evict_bits; dp.kept_idx = kept_idx; dp.variant = flags;
     return cuda_status(launch_decode(dp, c->dtype == UA_BF16, static_cast<cudaStream_t>(stream)));
 }
 

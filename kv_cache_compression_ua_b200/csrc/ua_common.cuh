@@ -27,6 +27,27 @@ __device__ __forceinline__ float decay_geo(float rq, float rk, float rsim) {
     return cbrtf(rq * rk * rsim);
 }
 
+// Variant bits of ua_shape.variant (the ablations; 0 = the method itself).
+constexpr int kVarNoQ = 1, kVarNoK = 2, kVarNoSim = 4, kVarQNorm = 8;
+constexpr int kVarMech = kVarNoQ | kVarNoK | kVarNoSim;
+constexpr float kQNormEps = 1e-6f;
+
+// Decay rate of a variant: the geometric mean of the rates whose mechanisms are on.
+// rq and rk arrive as 1 when their mechanism is off; x is the similarity logit
+// alpha * <khat_l, khat_j> + beta, whose softplus enters only when that mechanism is on.
+__device__ __forceinline__ float decay_var(float rq, float rk, float x, int variant) {
+    const int off = variant & kVarMech;
+    if (off == 0) return decay_geo(rq, rk, softplus_f(x));
+    const float prod = rq * rk * ((off & kVarNoSim) ? 1.f : softplus_f(x));
+    return __popc(off) == 1 ? sqrtf(prod) : prod;     // two rates on, or one
+}
+
+// 1 / number of mechanisms on: the exponent of the geometric mean, d log D / d log r.
+__host__ __device__ __forceinline__ float var_inv_n(int variant) {
+    const int n = 3 - (((variant & kVarNoQ) != 0) + ((variant & kVarNoK) != 0) + ((variant & kVarNoSim) != 0));
+    return n == 3 ? 1.f / 3.f : (n == 2 ? 0.5f : 1.f);
+}
+
 // RoPE frequencies theta^(-2m/d), computed on the host in double precision (m < d/2 <= 64).
 struct RopeFreq {
     double f[64];

@@ -29,6 +29,7 @@ struct PrepParams {
     float* lk2;         // [B*Hkv][Tp] log2(softplus(a_k)) / 3
     float* mq;          // [B*H][Tp]  scale * ||q|| * log2(e): bound of every logit of the row
     RopeFreq rf;
+    int variant;        // UA_VAR_* bits: query norm; rq / rk = 1 for a switched-off mechanism
 };
 
 // Boundary pass: per-query-tile column prefixes of the decay and the final biases.
@@ -43,6 +44,7 @@ struct BoundaryParams {
     const float* beta;  // [Hkv]
     float* pb;          // [B,Hkv,nqt,T]: sum_{j < l < t*bq} D[l,j]  (>= 0)
     float* bfinal;      // [B,Hkv,T] = -sum_{l > j} D[l,j], or NULL
+    int variant;        // UA_VAR_* bits (decay_var)
 };
 
 // Fused biased attention (SIMT path).
@@ -63,6 +65,7 @@ struct FwdParams {
     void* o;            // [B,T,H,d] act
     float* lse;         // [B,H,T] or NULL
     float* lambda_dbg;  // [B,Hkv,T,T] or NULL (pre-zeroed)
+    int variant;        // UA_VAR_* bits (decay_var)
 };
 
 // A 64-row query tile and a key tile of the SIMT paths contribute exactly nothing (every
@@ -125,6 +128,7 @@ struct DecodeParams {
     void* o;             // [B,H,d] act
     uint32_t* evict_bits;
     int32_t* kept_idx;
+    int variant;         // UA_VAR_* bits
 };
 
 // Backward (SIMT path).  Inputs from the f32 token preparation and boundary pass (query
@@ -163,6 +167,8 @@ struct BwdParams {
     float* dab;          // [B*Hkv*nkt][2]
     void* dq; void* dk; void* dv; void* dg;
     float* da_q; float* da_k; float* dalpha; float* dbeta;
+    const void* q;       // [B,T,H,d] act (raw queries, for the query-norm Jacobian)
+    int variant;         // UA_VAR_* bits
 };
 
 struct FwdTcLaunch {

@@ -31,7 +31,11 @@ class UAError(RuntimeError):
 class ua_shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("Hkv", ctypes.c_int),
                 ("d", ctypes.c_int), ("scale", ctypes.c_float), ("rope_theta", ctypes.c_double),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("variant", ctypes.c_int)]
+
+
+# ua_shape.variant bits (UA_VAR_* in ua.h); 0 is the method itself.
+VAR_NO_QUERY_DECAY, VAR_NO_KEY_DECAY, VAR_NO_SIM_DECAY, VAR_QUERY_NORM = 1, 2, 4, 8
 
 
 class ua_cache(ctypes.Structure):
@@ -120,11 +124,11 @@ def _dtype_code(dt: torch.dtype) -> int:
     raise ValueError(f"unsupported activation dtype {dt}")
 
 
-def make_shape(q: torch.Tensor, k: torch.Tensor, scale=None, theta=500000.0) -> ua_shape:
+def make_shape(q: torch.Tensor, k: torch.Tensor, scale=None, theta=500000.0, variant=0) -> ua_shape:
     B, T, H, d = q.shape
     Hkv = k.shape[2]
     scale = float(d) ** -0.5 if scale is None else float(scale)
-    return ua_shape(B, T, H, Hkv, d, scale, float(theta), _dtype_code(q.dtype))
+    return ua_shape(B, T, H, Hkv, d, scale, float(theta), _dtype_code(q.dtype), int(variant))
 
 
 def prefill_workspace_size(shape: ua_shape) -> int:
@@ -139,10 +143,11 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0, want_lse=True,
-                want_bfinal=True, want_lambda=False, out=None, ws=None, stream=None):
-    """ua_prefill_fwd.  Returns dict(o, lse, b_final, lam) (absent outputs are None)."""
+                want_bfinal=True, want_lambda=False, out=None, ws=None, variant=0, stream=None):
+    """ua_prefill_fwd (variant: VAR_* bits).  Returns dict(o, lse, b_final, lam) (absent
+    outputs are None)."""
     lib = load_library()
-    shape = make_shape(q, k, scale, theta)
+    shape = make_shape(q, k, scale, theta, variant)
     B, T, H, d = q.shape
     Hkv = k.shape[2]
     dev = q.device
@@ -170,11 +175,11 @@ def prefill_tile_stats(shape: ua_shape, ws: torch.Tensor, stream=None) -> tuple:
 
 
 def prefill_fwd_noalloc(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0, want_lse=True,
-                        want_bfinal=True, out=None, stream=None):
+                        want_bfinal=True, out=None, variant=0, stream=None):
     """ua_prefill_fwd_noalloc: the prefill forward using the library's fixed internal scratch
     instead of a workspace (for callers that cannot allocate device memory)."""
     lib = load_library()
-    shape = make_shape(q, k, scale, theta)
+    shape = make_shape(q, k, scale, theta, variant)
     B, T, H, d = q.shape
     Hkv = k.shape[2]
     dev = q.device
@@ -196,10 +201,11 @@ def prefill_bwd_workspace_size(shape: ua_shape) -> int:
 
 
 def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, d_o, *, scale=None, theta=500000.0,
-                ws=None, stream=None):
-    """ua_prefill_bwd.  Returns dict(dq, dk, dv, dg, da_q, da_k, dalpha, dbeta)."""
+                ws=None, variant=0, stream=None):
+    """ua_prefill_bwd (variant: the forward's VAR_* bits).  Returns dict(dq, dk, dv, dg,
+    da_q, da_k, dalpha, dbeta)."""
     lib = load_library()
-    shape = make_shape(q, k, scale, theta)
+    shape = make_shape(q, k, scale, theta, variant)
     dev = q.device
     gr = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
           "dg": torch.empty_like(g), "da_q": torch.empty_like(a_q), "da_k": torch.empty_like(a_k),
@@ -267,8 +273,9 @@ def cache_compact(cache: Cache, p: float = 0.0, keep=None, kept_idx=None, stream
 
 
 def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: float, *, scale=None,
-                theta=500000.0, out=None, evict_bits=None, kept_idx=None, stream=None):
-    """ua_decode_step for one token per sequence.  Returns o [B,H,d]."""
+                theta=500000.0, out=None, evict_bits=None, kept_idx=None, variant=0, stream=None):
+    """ua_decode_step for one token per sequence (variant: the prefill's VAR_* bits).
+    Returns o [B,H,d]."""
     H = q.shape[1]
     d = q.shape[2]
     scale = float(d) ** -0.5 if scale is None else float(scale)
@@ -276,7 +283,7 @@ def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: 
     c = cache.struct()
     rc = load_library().ua_decode_step(ctypes.byref(c), H, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q),
                                        _ptr(a_k), _ptr(alpha), _ptr(beta), int(pos_t), float(p), scale,
-                                       float(theta), _ptr(o), _ptr(evict_bits), _ptr(kept_idx), 0,
+                                       float(theta), _ptr(o), _ptr(evict_bits), _ptr(kept_idx), int(variant),
                                        _stream(stream))
     _check("ua_decode_step", rc)
     return o

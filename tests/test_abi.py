@@ -84,6 +84,25 @@ def test_prefill_rejects_null_misaligned_and_small_workspace(lib):
     assert _fwd(lib, _shape(), ws_bytes=need.value - 1) == 4
 
 
+@pytest.mark.parametrize("variant,code", [(16, 1), (7, 1), (15, 1), (-8, 1), (1, 0), (6, 0), (8, 0), (11, 0)])
+def test_variant_bits_validated(lib, variant, code):
+    need = ctypes.c_size_t(0)
+    s = _shape(variant=variant)
+    assert lib.ua_prefill_workspace_size(ctypes.byref(s), ctypes.byref(need)) == code
+    assert lib.ua_prefill_bwd_workspace_size(ctypes.byref(s), ctypes.byref(need)) == code
+    if code:
+        assert _fwd(lib, s) == code
+
+
+def test_mechanism_variants_leave_the_tensor_core_path(lib):
+    # a mechanism switched off runs the SIMT path: no tensor-core tile statistics
+    tiles, skipped = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+    s = _shape(T=512, variant=ua.VAR_NO_SIM_DECAY)
+    assert lib.ua_prefill_tile_stats(ctypes.byref(s), None, ctypes.c_size_t(0), ctypes.byref(tiles),
+                                     ctypes.byref(skipped), None) == 0
+    assert tiles.value == 4 * 5 // 2 * 2 and skipped.value == 0
+
+
 def test_lambda_debug_limited_to_small_T(lib):
     P = ctypes.c_void_p
     shape = _shape(T=2048)
@@ -102,12 +121,13 @@ def test_cache_calls_reject_bad_arguments(lib):
     # misaligned cache array
     c2 = ua.ua_cache(2, 2, 64, 100, ua.UA_BF16, *([FAKE] * 6 + [FAKE + 4]))
     assert lib.ua_cache_compact(ctypes.byref(c2), None, ctypes.c_float(0.1), None, None) == 3
-    # decode: group size 5 unsupported, flags must be 0, head_dim 80 unsupported
+    # decode: group size 5 unsupported, flags must be valid variant bits, head_dim 80 unsupported
     args = [P(FAKE)] * 8
     assert lib.ua_decode_step(ctypes.byref(c), 10, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
                               P(FAKE), None, None, 0, None) == 2
-    assert lib.ua_decode_step(ctypes.byref(c), 8, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
-                              P(FAKE), None, None, 1, None) == 1
+    for bad in (16, 7, 15, -1):   # unknown bit; all three decay mechanisms off
+        assert lib.ua_decode_step(ctypes.byref(c), 8, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
+                                  P(FAKE), None, None, bad, None) == 1
     c3 = ua.ua_cache(2, 2, 80, 100, ua.UA_BF16, *([FAKE] * 7))
     assert lib.ua_decode_step(ctypes.byref(c3), 8, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
                               P(FAKE), None, None, 0, None) == 2

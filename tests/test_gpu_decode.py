@@ -33,14 +33,14 @@ _ORACLE_BFINAL = {}
 _INPUTS = {}
 
 
-def oracle_bfinal(w, T0, b):
+def oracle_bfinal(w, T0, b, variant=0):
     """Oracle b_final of batch b (all KV heads), memoised across thresholds."""
-    key = (repr(w), T0, b)
+    key = (repr(w), T0, b, variant)
     if key not in _ORACLE_BFINAL:
         xb = I.make_prefill_inputs(w, T=T0, B=1, b0=b)
         rm = np.zeros(T0, np.uint8)          # only b_final is needed
         ro = oracle.prefill_fwd(**{k: v for k, v in xb.items() if k != "d_o"}, scale=w.scale, theta=w.theta,
-                                row_mask=rm)
+                                row_mask=rm, variant=variant)
         _ORACLE_BFINAL[key] = (xb, ro["b_final"])
     return _ORACLE_BFINAL[key]
 
@@ -48,8 +48,8 @@ def oracle_bfinal(w, T0, b):
 class Lockstep:
     """GPU cache and oracle cache for batches `b_sel` of workload w, prefilled to T0."""
 
-    def __init__(self, w, T0, steps, p, b_sel=None, zero_prefill_q=False):
-        self.w, self.T0, self.steps, self.p = w, T0, steps, p
+    def __init__(self, w, T0, steps, p, b_sel=None, zero_prefill_q=False, variant=0):
+        self.w, self.T0, self.steps, self.p, self.variant = w, T0, steps, p, variant
         self.cap = T0 + steps + 1
         Bg = w.B
         key = (repr(w), T0, zero_prefill_q)
@@ -64,7 +64,7 @@ class Lockstep:
             d["q"] = torch.zeros(Bg, T0, w.H, w.d, dtype=adt, device="cuda")
             d["g"] = torch.zeros(Bg, T0, w.H, w.d, dtype=adt, device="cuda")
         r = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
-                           scale=w.scale, theta=w.theta, want_lse=False)
+                           scale=w.scale, theta=w.theta, want_lse=False, variant=variant)
         self.gb_final = r["b_final"].cpu().numpy()
         self.cache = ua.Cache.empty(Bg, w.Hkv, w.d, self.cap, adt)
         ua.cache_fill(self.cache, d["k"], d["v"], d["a_k"], r["b_final"], theta=w.theta)
@@ -77,7 +77,7 @@ class Lockstep:
         self.b_sel = list(range(Bg)) if b_sel is None else list(b_sel)
         self.ora = []
         for b in self.b_sel:
-            xb, ob_final = oracle_bfinal(w, T0, b)
+            xb, ob_final = oracle_bfinal(w, T0, b, variant)
             ro = {"b_final": ob_final}
             assert_close(f"b_final[b={b}]", self.gb_final[b], ro["b_final"][0], w.dtype, relative_max=True)
             gpu_keep = np.zeros((1, w.Hkv, T0), bool)
@@ -108,7 +108,7 @@ class Lockstep:
         kept = torch.full((w.B, w.Hkv, self.cap), -7, dtype=torch.int32, device="cuda")
         o = ua.decode_step(self.cache, t["q"], t["k"], t["v"], t["g"], t["a_q"], t["a_k"], self.alpha,
                            self.beta, pos_t, self.p, scale=w.scale, theta=w.theta, evict_bits=ev,
-                           kept_idx=kept)
+                           kept_idx=kept, variant=self.variant)
         assert ua.get_device_status() == 0
         o = o.float().cpu().numpy()
         ev = ev.cpu().numpy().view(np.uint32)
@@ -128,7 +128,8 @@ class Lockstep:
             ro = oracle.decode_step(oc, tok["q"][b:b + 1], tok["k"][b:b + 1], tok["v"][b:b + 1],
                                     tok["g"][b:b + 1], tok["a_q"][b:b + 1], tok["a_k"][b:b + 1],
                                     self.alpha.cpu().numpy(), self.beta.cpu().numpy(), pos_t, self.p,
-                                    scale=w.scale, theta=w.theta, band=EVICT_BAND, adopt_keep=gpu_keep)
+                                    scale=w.scale, theta=w.theta, band=EVICT_BAND, adopt_keep=gpu_keep,
+                                    variant=self.variant)
             inb = ro["in_band"].astype(bool)
             mism = (ro["evict"].astype(bool) != gpu_ev) & ~inb
             assert not mism.any(), f"step {s}: eviction differs outside the band at {np.argwhere(mism)[:5]}"
@@ -153,6 +154,26 @@ def test_small_lockstep(dtype, d, H, Hkv, p):
     w = I.Workload("dec_small", 3, 400, H, Hkv, d, dtype, 4242, bimodal_ak=True)
     ls = Lockstep(w, T0=400, steps=40, p=p)
     for s in range(40):
+        ls.step(s)
+
+
+NQ, NK, NS, QN = ua.VAR_NO_QUERY_DECAY, ua.VAR_NO_KEY_DECAY, ua.VAR_NO_SIM_DECAY, ua.VAR_QUERY_NORM
+
+
+@pytest.mark.parametrize("variant,dtype,d,H,Hkv,p", [(NQ, "bf16", 64, 8, 2, 0.15), (NK | NS, "bf16", 64, 8, 2, 0.05),
+                                                    (QN | NS, "f32", 64, 4, 2, 0.15), (QN, "bf16", 128, 6, 2, 0.15),
+                                                    (NQ | NK, "f32", 64, 4, 4, 0.15)])
+def test_variant_lockstep(variant, dtype, d, H, Hkv, p):
+    """Ablation variants (decay mechanisms switched off, query norm) through fill, compaction
+    and 24 decode steps, in lockstep with the oracle's variant.
+
+    The similarity-only variant runs in f32: a bf16 cache holds the unit keys rounded to 8
+    mantissa bits, and with the similarity rate alone (no cube or square root to divide its
+    relative error) that rounding reaches the bias at full strength and accumulates over the
+    steps, past the 1e-3 band that eviction decisions are compared within."""
+    w = I.Workload("dec_var", 2, 300, H, Hkv, d, dtype, 4300 + variant, bimodal_ak=True)
+    ls = Lockstep(w, T0=300, steps=24, p=p, variant=variant)
+    for s in range(24):
         ls.step(s)
 
 

@@ -1,0 +1,128 @@
+"""GPU parity of the ablation variants (ua_shape.variant) against the fp64 oracle: decay
+mechanisms switched off from the geometric mean, and the Qwen3-style query norm ("A
+Self-Pruning Transformer: Extreme KV-Cache Compression with Universal Attention",
+paperlayer.ai summary, §5.4 with Table 3 and App. E with Table 6).
+
+Forward on the fp32 SIMT path for every mechanism subset; bf16 with a mechanism switched
+off must leave the tensor-core path for the SIMT one, while the query norm stays on the
+tensor cores; backward on both activation dtypes, with the gradient of every switched-off
+mechanism exactly zero."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_compression_ua_b200 import inputs as I
+from kv_cache_compression_ua_b200 import ua
+from helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+NQ, NK, NS, QN = ua.VAR_NO_QUERY_DECAY, ua.VAR_NO_KEY_DECAY, ua.VAR_NO_SIM_DECAY, ua.VAR_QUERY_NORM
+MECH_SUBSETS = [NQ, NK, NS, NQ | NK, NQ | NS, NK | NS]
+
+
+def to_dev(x, dtype):
+    return {n: torch.from_numpy(np.ascontiguousarray(a)).cuda().to(
+        TORCH_DT[dtype] if n in ("q", "k", "v", "g", "d_o") else torch.float32).contiguous() for n, a in x.items()}
+
+
+def kernels_ran(fn):
+    ua.profile_reset()
+    ua.profile_enable(True)
+    try:
+        out = fn()
+        torch.cuda.synchronize()
+    finally:
+        ua.profile_enable(False)
+    return out, set(ua.profile_read())
+
+
+def run_fwd(w, x, variant, want_lambda=False):
+    d = to_dev({k: v for k, v in x.items() if k != "d_o"}, w.dtype)
+    r = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
+                       scale=w.scale, theta=w.theta, want_lambda=want_lambda, variant=variant)
+    torch.cuda.synchronize()
+    return {k: (None if v is None else v.float().cpu().numpy()) for k, v in r.items()}
+
+
+def ora_fwd(w, x, variant, want_lambda=False):
+    return oracle.prefill_fwd(**{k: v for k, v in x.items() if k != "d_o"}, scale=w.scale, theta=w.theta,
+                              want_lambda=want_lambda, variant=variant)
+
+
+@pytest.mark.parametrize("variant", MECH_SUBSETS + [QN, QN | NS])
+def test_fp32_forward_every_variant(variant):
+    w = I.Workload("var", 2, 190, 4, 2, 64, "f32", 900 + variant)
+    x = I.make_prefill_inputs(w)
+    g = run_fwd(w, x, variant, want_lambda=True)
+    r = ora_fwd(w, x, variant, want_lambda=True)
+    assert_close("o", g["o"], r["o"], "f32")
+    # log-domain outputs against max(1, |ref|): with one or two mechanisms the decay per step is
+    # no longer damped by the cube root and b_final reaches O(100) here (key only: -(i-j) r_k(j)),
+    # where a 190-term fp32 sum carries ~1e-6 relative rounding, i.e. ~1e-4 absolute
+    assert_close("lse", g["lse"], r["lse"], "f32", relative_max=True)
+    assert_close("b_final", g["b_final"], r["b_final"], "f32", relative_max=True)
+    tri = np.tril(np.ones((w.T, w.T), bool))
+    assert_close("lambda", g["lam"][..., tri], r["lam"][..., tri], "f32", relative_max=True)
+    # the variant matters: the method itself gives a different Lambda or output
+    r0 = ora_fwd(w, x, 0, want_lambda=True)
+    assert np.max(np.abs(r0["o"] - r["o"])) > 1e-3
+
+
+@pytest.mark.parametrize("variant,d", [(NS, 64), (NQ | NK, 64), (NK, 128)])
+def test_bf16_mechanism_variant_runs_simt_path(variant, d):
+    w = I.Workload("var", 2, 333, 8, 2, d, "bf16", 950 + variant)
+    x = I.make_prefill_inputs(w)
+    g, names = kernels_ran(lambda: run_fwd(w, x, variant))
+    assert "k_fwd_simt" in names and "k_fwd_tc" not in names, names
+    assert ua.get_device_status() == 0
+    r = ora_fwd(w, x, variant)
+    assert_close("o", g["o"], r["o"], "bf16")
+    assert_close("lse", g["lse"], r["lse"], "bf16", relative_max=True)
+    assert_close("b_final", g["b_final"], r["b_final"], "bf16", relative_max=True)
+
+
+@pytest.mark.parametrize("B,T,H,Hkv", [(2, 129, 8, 2), (1, 517, 4, 1), (1, 1000, 4, 4)])
+def test_bf16_query_norm_stays_on_tensor_cores(B, T, H, Hkv):
+    w = I.Workload("var", B, T, H, Hkv, 64, "bf16", 970 + T)
+    x = I.make_prefill_inputs(w)
+    x["q"] = x["q"] * 3.0          # the norm removes the scale; without it logits would triple
+    g, names = kernels_ran(lambda: run_fwd(w, x, QN))
+    assert "k_fwd_tc" in names and "k_fwd_simt" not in names, names
+    assert ua.get_device_status() == 0
+    r = ora_fwd(w, x, QN)
+    assert_close("o", g["o"], r["o"], "bf16")
+    assert_close("lse", g["lse"], r["lse"], "bf16", relative_max=True)
+    assert_close("b_final", g["b_final"], r["b_final"], "bf16", relative_max=True)
+
+
+GRADS = ("dq", "dk", "dv", "dg", "da_q", "da_k", "dalpha", "dbeta")
+OFF_GRADS = {NQ: ("da_q",), NK: ("da_k",), NS: ("dalpha", "dbeta")}
+
+
+@pytest.mark.parametrize("variant,dtype,d", [(NQ, "f32", 64), (NS, "f32", 64), (NK | NS, "f32", 128),
+                                             (NQ | NK, "f32", 64), (QN, "f32", 64), (QN | NQ, "bf16", 64),
+                                             (QN | NK, "bf16", 128), (NS, "bf16", 64)])
+def test_backward_every_variant(variant, dtype, d):
+    w = I.Workload("varbwd", 1, 97, 4, 2, d, dtype, 990 + variant, with_grad=True)
+    x = I.make_prefill_inputs(w)
+    dv = to_dev(x, dtype)
+    f = ua.prefill_fwd(dv["q"], dv["k"], dv["v"], dv["g"], dv["a_q"], dv["a_k"], dv["alpha"], dv["beta"],
+                       scale=w.scale, theta=w.theta, variant=variant)
+    gr = ua.prefill_bwd(dv["q"], dv["k"], dv["v"], dv["g"], dv["a_q"], dv["a_k"], dv["alpha"], dv["beta"],
+                        f["o"], f["lse"], f["b_final"], dv["d_o"], scale=w.scale, theta=w.theta, variant=variant)
+    torch.cuda.synchronize()
+    assert ua.get_device_status() == 0
+    g = {k: v.float().cpu().numpy() for k, v in gr.items()}
+    r = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta, variant=variant)
+    off = set()
+    for bit, names in OFF_GRADS.items():
+        if variant & bit:
+            off |= set(names)
+    for n in GRADS:
+        assert np.all(np.isfinite(g[n])), n
+        if n in off:
+            assert np.all(g[n] == 0.0), n          # a switched-off mechanism has no gradient
+            continue
+        assert_close(n, g[n], r[n], dtype, tensor_scale=True)
