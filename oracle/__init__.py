@@ -44,7 +44,7 @@ def _load():
         P = ctypes.c_void_p
         I = ctypes.c_int
         Dd = ctypes.c_double
-        lib.ora_prefill_fwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 4 + [I, I]
+        lib.ora_prefill_fwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 4 + [I, Dd, I]
         lib.ora_prefill_fwd.restype = I
         lib.ora_lambda_bruteforce.argtypes = [I, I, I, I, P, P, P, P, P, P, I, I]
         lib.ora_lambda_bruteforce.restype = I
@@ -77,10 +77,11 @@ VAR_NO_Q, VAR_NO_K, VAR_NO_SIM, VAR_QNORM = 1, 2, 4, 8
 
 
 def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0,
-                want_lambda=False, unit_mask=None, row_mask=None, variant=0, nthreads=None):
+                want_lambda=False, unit_mask=None, row_mask=None, variant=0, prune_p=0.0, nthreads=None):
     """Prefill forward of UA in fp64.
 
     Shapes: q, g [B,T,H,d]; k, v [B,T,Hkv,d]; a_q, a_k [B,T,Hkv]; alpha, beta [Hkv].
+    prune_p > 0: chunked pruned prefill (128-token chunks, threshold p); 0 = dense.
     Returns dict(o [B,T,H,d], lse [B,H,T], b_final [B,Hkv,T], lam [B,Hkv,T,T] or None).
     Entries outside unit_mask / row_mask are left as NaN.
     """
@@ -100,6 +101,7 @@ def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0
                                  _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
                                  _ptr(alpha), _ptr(beta), _ptr(um), _ptr(rm),
                                  _ptr(o), _ptr(lse), _ptr(bfin), _ptr(lam), int(variant),
+                                 float(np.log(prune_p)) if prune_p > 0 else -np.inf,
                                  nthreads or default_threads())
     if rc != 0:
         raise ValueError(f"ora_prefill_fwd rejected the shapes (code {rc})")

@@ -41,6 +41,13 @@
  *     All three off is rejected.
  *   bit 3 set: queries are RMS-normalised per head before RoPE (Qwen3-style query norm,
  *     unit gain): q' = q / sqrt(mean(q^2) + 1e-6).  Keys keep their L2 normalisation.
+ *
+ * Chunked pruned prefill ([S1] §5: prefill pruning proceeds in chunks of 128 tokens), when
+ * prune_logp > -inf: before the chunk that starts at row c (c a multiple of 128, c > 0), every
+ * pair j < c whose bias Lambda_{c-1,j} is below log p is evicted for good (Lambda only
+ * decreases down a column, so it would never come back).  A row of that chunk attends over
+ * the surviving pairs and every pair of its own chunk, with the same biases as before.
+ * Lambda and b_final do not change; with prune_logp = -inf (p = 0) nothing is evicted.
  */
 #include <math.h>
 #include <pthread.h>
@@ -176,6 +183,7 @@ typedef struct {
     const uint8_t* row_mask;  /* [T] or NULL = all rows get attention outputs */
     double *o, *lse, *bfinal, *lambda;
     int variant;
+    double prune_logp;        /* log p of the chunked prefill pruning, -inf = dense */
 } fwd_ctx;
 
 static void fwd_unit(void* vctx, int unit) {
@@ -194,6 +202,8 @@ static void fwd_unit(void* vctx, int unit) {
     double* qrot = (double*)malloc(sizeof(double) * (size_t)d);
     double* qtmp = (double*)malloc(sizeof(double) * (size_t)d);
     double* acc = (double*)malloc(sizeof(double) * (size_t)d);
+    double* lamb = (double*)malloc(sizeof(double) * (size_t)T);  /* Lambda at the last chunk boundary */
+    int cs = 0;                                                  /* first row of the current chunk */
 
     for (int t = 0; t < T; ++t) {
         const double* kt = c->k + (((size_t)b * T + t) * Hkv + kvh) * d;
@@ -203,6 +213,11 @@ static void fwd_unit(void* vctx, int unit) {
     }
 
     for (int i = 0; i < T; ++i) {
+        if (i > 0 && i % 128 == 0) {
+            /* chunk boundary: lam still holds row i-1, the biases the eviction decides on */
+            cs = i;
+            for (int j = 0; j < i; ++j) lamb[j] = lam[j];
+        }
         /* Causal accumulation, column prefix form: Lambda_ij = Lambda_{i-1,j} - D[i,j]. */
         double rq_i = softplus(c->aq[((size_t)b * T + i) * Hkv + kvh]);
         for (int j = 0; j < i; ++j) {
@@ -222,12 +237,18 @@ static void fwd_unit(void* vctx, int unit) {
             rope_query(qi, d, (double)i, c->theta, c->variant, qtmp, qrot);
             double m = -INFINITY;
             for (int j = 0; j <= i; ++j) {
+                /* evicted at the chunk boundary: no longer in the cache */
+                if (j < cs && !(lamb[j] >= c->prune_logp)) {
+                    srow[j] = -INFINITY;
+                    continue;
+                }
                 srow[j] = c->scale * dot(qrot, krot + (size_t)j * d, d) + lam[j];
                 if (srow[j] > m) m = srow[j];
             }
             double l = 0.0;
             for (int x = 0; x < d; ++x) acc[x] = 0.0;
             for (int j = 0; j <= i; ++j) {
+                if (srow[j] == -INFINITY) continue;
                 double p = exp(srow[j] - m);
                 l += p;
                 const double* vj = c->v + (((size_t)b * T + j) * Hkv + kvh) * d;
@@ -244,6 +265,7 @@ static void fwd_unit(void* vctx, int unit) {
         for (int j = 0; j < T; ++j) bf[j] = lam[j];
     }
     free(khat); free(krot); free(rk); free(lam); free(srow); free(qrot); free(qtmp); free(acc);
+    free(lamb);
 }
 
 /* Prefill forward.  Outputs that are NULL are skipped.  Only units with unit_mask set
@@ -253,11 +275,12 @@ int ora_prefill_fwd(int B, int T, int H, int Hkv, int d, double scale, double th
                     const double* aq, const double* ak, const double* alpha, const double* beta,
                     const uint8_t* unit_mask, const uint8_t* row_mask,
                     double* o, double* lse, double* bfinal, double* lambda, int variant,
-                    int nthreads) {
+                    double prune_logp, int nthreads) {
     if (B < 1 || T < 1 || H < 1 || Hkv < 1 || d < 2 || (d & 1) || H % Hkv) return 1;
     if ((variant & ~VAR_ALL) || n_active(variant) == 0) return 1;
+    if (isnan(prune_logp) || prune_logp > 0.0) return 1;
     fwd_ctx c = {B, T, H, Hkv, d, scale, theta, q, k, v, g, aq, ak, alpha, beta,
-                 unit_mask, row_mask, o, lse, bfinal, lambda, variant};
+                 unit_mask, row_mask, o, lse, bfinal, lambda, variant, prune_logp};
     run_units(fwd_unit, &c, B * Hkv, nthreads);
     return 0;
 }
