@@ -86,6 +86,8 @@ typedef struct {
     double rope_theta;    /* RoPE base, e.g. 500000 */
     ua_dtype dtype;       /* activation dtype of q, k, v, g, o (and gradients) */
     int variant;          /* UA_VAR_* bits, 0 = Universal Attention as published */
+    float prune_p;        /* chunked pruned prefill threshold p in [0, 1]; 0 = dense prefill
+                             (see ua_prefill_fwd); must be 0 for the backward */
 } ua_shape;
 
 /* ------------------------------------------------------------------ prefill forward
@@ -121,7 +123,15 @@ ua_status ua_prefill_workspace_size(const ua_shape* shape, size_t* bytes);
  * computation (see ua_prefill_tile_stats).  The tensor-core path computes the
  * three-rate geometric mean only; it takes UA_VAR_QUERY_NORM, but a shape with a decay
  * mechanism switched off runs the SIMT path.  All other problems, and every call that asks
- * for lambda_dbg, run the fp32 SIMT path, which uses a running maximum. */
+ * for lambda_dbg, run the fp32 SIMT path, which uses a running maximum.
+ *
+ * Chunked pruned prefill (shape->prune_p = p > 0; paperlayer.ai summary §5: prefill pruning
+ * proceeds in chunks of 128 tokens): before the chunk that starts at token c (c a multiple of
+ * 128), every pair j < c whose bias Lambda_{c-1,j} is below log p is evicted, and the rows of
+ * that chunk and of every later one attend over the surviving pairs and their own chunk only
+ * (the biases themselves are unchanged).  b_final and lambda_dbg are the same as for the dense
+ * prefill, so filling a cache with b_final and compacting it at p keeps exactly the pairs that
+ * survive the last chunk; o and lse change.  Key tiles evicted as a whole are skipped. */
 ua_status ua_prefill_fwd(const ua_shape* shape, const void* q, const void* k, const void* v,
                          const void* g, const float* a_q, const float* a_k, const float* alpha,
                          const float* beta, void* o, float* lse, float* b_final, float* lambda_dbg,
@@ -166,7 +176,8 @@ ua_status ua_prefill_tile_stats(const ua_shape* shape, const void* ws, size_t ws
  * and is not read (the decay prefixes are recomputed).  d_o: [B,T,H,d] act.
  * Outputs: dq, dg [B,T,H,d] act; dk, dv [B,T,Hkv,d] act; da_q, da_k [B,T,Hkv] f32;
  * dalpha, dbeta [Hkv] f32 (summed over the batch).  All outputs are overwritten; the result
- * is deterministic (no atomics).  Runs as fp32 SIMT kernels. */
+ * is deterministic (no atomics).  Runs as fp32 SIMT kernels.  Training is dense: a shape
+ * with prune_p != 0 is UA_ERR_INVALID_ARG. */
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes);
 
 ua_status ua_prefill_bwd(const ua_shape* shape, const void* q, const void* k, const void* v,

@@ -218,6 +218,7 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
     float* sRq = sP + BM * LP;
     float* sRk = sRq + BM;
     float* sPb = sRk + BN;
+    float* sEv = sPb + BN;                            // 1: key evicted at this chunk's boundary
 
     const int T = p.T;
     const int qt = gridDim.x - 1 - blockIdx.x;        // heaviest (last) query tiles first
@@ -248,17 +249,24 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
     // tiles whose probabilities all underflow are skipped (not when the debug Lambda is written)
     const bool can_skip = p.qmax != nullptr && p.lambda_dbg == nullptr;
     const float thr = can_skip ? kSimtSkipMargin + 2.f * p.qmax[unit * p.nqt + qt] : 0.f;
+    // Chunked pruned prefill: the 128-row chunk of this tile starts at query tile qt & ~1, and a
+    // key before it is evicted when its bias there, -Pb, is below log p (Pb > prune_thr).
+    const int qchunk = qt & ~1;
     for (int kt = 0; kt <= qt; ++kt) {
         const int j0 = kt * BN;
+        const bool pruned_tile = kt < qchunk && p.prune_thr < INFINITY;
         __syncthreads();
         for (int c = tid; c < BN; c += 256) {
             const int j = j0 + c;
             sRk[c] = j < T ? p.rk[unit * T + j] : 0.f;
             sPb[c] = j < T ? p.pb[(unit * p.nqt + qt) * T + j] : 0.f;
+            sEv[c] = (pruned_tile && j < T && p.pb[(unit * p.nqt + qchunk) * T + j] > p.prune_thr) ? 1.f : 0.f;
         }
-        if (__syncthreads_and(!can_skip || tid >= BN || sPb[tid] >= thr)) {
-            if (can_skip) continue;
-        }
+        // skip when every key underflows, or (no debug Lambda to write) every key is evicted;
+        // thread tid < BN votes on the entries it wrote itself
+        if (__syncthreads_and(tid >= BN || (can_skip && sPb[tid] >= thr) ||
+                              (pruned_tile && p.lambda_dbg == nullptr && sEv[tid] != 0.f)))
+            continue;
         for (int e = tid; e < BN * DH; e += 256) {
             const int c = e / DH, x = e % DH, j = j0 + c;
             const bool ok = j < T;
@@ -332,17 +340,20 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
                 const float lam = sL[r * LP + c];
                 if (write_lambda && i < T && j < T)
                     p.lambda_dbg[(unit * T + i) * (size_t)T + j] = (j <= i) ? lam : 0.f;
-                sc[rr][cc] = (j <= i && j < T) ? fmaf(p.scale, sc[rr][cc], lam) : -INFINITY;
+                sc[rr][cc] = (j <= i && j < T && sEv[c] == 0.f) ? fmaf(p.scale, sc[rr][cc], lam) : -INFINITY;
                 mx = fmaxf(mx, sc[rr][cc]);
             }
 #pragma unroll
             for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             const float m_new = fmaxf(m_r[rr], mx);
-            const float corr = expf(m_r[rr] - m_new);
+            // a row that has seen no visible key yet (every key so far evicted by the chunked
+            // pruning) keeps m = -inf; subtracting 0 then gives exp(-inf) = 0, not a NaN
+            const float m_use = m_new == -INFINITY ? 0.f : m_new;
+            const float corr = expf(m_r[rr] - m_use);
             float rs = 0.f;
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-                const float pe = expf(sc[rr][cc] - m_new);
+                const float pe = expf(sc[rr][cc] - m_use);
                 rs += pe;
                 sP[r * LP + tx + 16 * cc] = pe;
             }
@@ -410,7 +421,7 @@ cudaError_t launch_boundary_simt(const BoundaryParams& p, cudaStream_t s) {
 template <int DH, typename TI>
 static cudaError_t fwd_simt_inst(const FwdParams& p, cudaStream_t s) {
     constexpr int BM = 64, BN = 64, LD = DH + 1, LP = BN + 1;
-    const size_t smem = sizeof(float) * (size_t)(2 * BM * LD + 3 * BN * LD + 2 * BM * LP + BM + 2 * BN);
+    const size_t smem = sizeof(float) * (size_t)(2 * BM * LD + 3 * BN * LD + 2 * BM * LP + BM + 3 * BN);
     cudaError_t e = cudaFuncSetAttribute(k_fwd_simt<DH, TI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.nqt, p.H, p.B);

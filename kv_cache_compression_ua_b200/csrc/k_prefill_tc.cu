@@ -224,6 +224,7 @@ struct FwdTcParams {
     unsigned* flags;     // [B*Hkv][nqt][nqt] publication counters; flags[B*Hkv*nqt*nqt] = ticket
     float* b_final;      // [B*Hkv][T] or NULL
     int nunits;          // B * Hkv
+    float prune_thr;     // chunked pruned prefill: keys with Pb > prune_thr are evicted; +inf = dense
 };
 
 // Wait (all lanes of the warp) until *f >= target, with acquire semantics for every lane.
@@ -389,7 +390,10 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 float mn = fminf(fminf(v4.x, v4.y), fminf(v4.z, v4.w));
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                skip = (mn * kLog2e >= kSkipLog2) ? (EARLY ? 2 : 1) : 0;
+                // every P underflows, or (chunked pruned prefill, the chunk being this query
+                // tile) every key was evicted at the chunk boundary.  Either stays true for every
+                // later query tile, so the lower-bound prefix that code 2 publishes is enough.
+                skip = (mn * kLog2e >= kSkipLog2 || mn > p.prune_thr) ? (EARLY ? 2 : 1) : 0;
             }
             *reinterpret_cast<float4*>(&S.pb[sb][lane * 4]) = v4;
             if (lane == 0) {
@@ -676,6 +680,10 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
             const float ka = -rk3 * kLog2e, kb = -fmaf(rk3, above, pbj) * kLog2e - S.shift[warp];
 #pragma unroll
             for (int r = 0; r < 32; ++r) lam[r] = fmaf(lam[r], ka, kb);
+            if (!diag && pbj > p.prune_thr) {            // key evicted at this chunk's boundary
+#pragma unroll
+                for (int r = 0; r < 32; ++r) lam[r] = -INFINITY;
+            }
             // ---- per head: P = 2^(S*scale*log2e + Lambda - M_i), causally masked
             for (int h = 0; h < G && ok; ++h) {
                 if (!slot_wait()) { ok = false; break; }
@@ -778,7 +786,7 @@ cudaError_t launch_fwd_tc(const FwdTcLaunch& L, cudaStream_t s) {
     p.B = L.B; p.T = L.T; p.Tp = L.Tp; p.H = L.H; p.Hkv = L.Hkv; p.nqt = L.nqt;
     p.scale_log2e = L.scale * kLog2e;
     p.alpha = L.alpha; p.beta = L.beta; p.g = L.g; p.o = L.o; p.lse = L.lse;
-    p.pincl = L.pincl; p.flags = L.flags; p.b_final = L.b_final; p.nunits = BK;
+    p.pincl = L.pincl; p.flags = L.flags; p.b_final = L.b_final; p.nunits = BK; p.prune_thr = L.prune_thr;
     switch (L.H / L.Hkv) {
         case 1: return fwd_tc_inst<1>(m, p, s);
         case 2: return fwd_tc_inst<2>(m, p, s);

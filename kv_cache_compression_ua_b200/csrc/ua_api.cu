@@ -37,8 +37,12 @@ ua_status check_shape(const ua_shape* s) {
     if (!group_ok(s->H / s->Hkv)) return UA_ERR_UNSUPPORTED;
     if (s->dtype != UA_F32 && s->dtype != UA_BF16) return UA_ERR_UNSUPPORTED;
     if (!variant_ok(s->variant)) return UA_ERR_INVALID_ARG;
+    if (!(s->prune_p >= 0.f && s->prune_p <= 1.f)) return UA_ERR_INVALID_ARG;
     return UA_OK;
 }
+
+// Chunked pruned prefill: a key is evicted when its boundary prefix Pb exceeds -log p.
+float prune_thr(const ua_shape* s) { return s->prune_p > 0.f ? -logf(s->prune_p) : INFINITY; }
 
 // Workspace of the SIMT prefill forward: f32 rotated/normalised copies, rates, prefixes.
 struct FwdWs {
@@ -209,7 +213,7 @@ static ua_status prefill_fwd_simt(const ua_shape* s, const void* q, const void* 
     fp.kr = reinterpret_cast<const float*>(pp.kr);
     fp.v = v; fp.g = g; fp.rq = pp.rq; fp.rk = pp.rk; fp.alpha = alpha; fp.beta = beta; fp.pb = bp.pb;
     fp.qmax = tq.qmax;
-    fp.o = o; fp.lse = lse; fp.lambda_dbg = lambda_dbg; fp.variant = s->variant;
+    fp.o = o; fp.lse = lse; fp.lambda_dbg = lambda_dbg; fp.variant = s->variant; fp.prune_thr = prune_thr(s);
     return cuda_status(launch_fwd_simt(fp, bf, cs));
 }
 
@@ -238,7 +242,7 @@ static ua_status prefill_fwd_tc(const ua_shape* s, const void* q, const void* k,
     L.kh = pp.kh; L.kr = pp.kr; L.qr = pp.qr; L.v = v; L.lq2 = pp.lq2; L.lk2 = pp.lk2; L.mq = pp.mq;
     L.pincl = reinterpret_cast<float*>(at(ws, w.pb));
     L.flags = reinterpret_cast<unsigned*>(at(ws, w.flags));
-    L.alpha = alpha; L.beta = beta; L.g = g; L.o = o; L.lse = lse; L.b_final = b_final;
+    L.alpha = alpha; L.beta = beta; L.g = g; L.o = o; L.lse = lse; L.b_final = b_final; L.prune_thr = prune_thr(s);
     return cuda_status(launch_fwd_tc(L, cs));
 }
 
@@ -345,7 +349,7 @@ BwdWs bwd_ws_layout(const ua_shape* s) {
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes) {
     ua_status st = check_shape(shape);
     if (st != UA_OK) return st;
-    if (!bytes) return UA_ERR_INVALID_ARG;
+    if (!bytes || shape->prune_p != 0.f) return UA_ERR_INVALID_ARG;   // training is dense
     *bytes = bwd_ws_layout(shape).total;
     return UA_OK;
 }
@@ -357,6 +361,7 @@ ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const 
                          void* stream) {
     ua_status st = check_shape(s);
     if (st != UA_OK) return st;
+    if (s->prune_p != 0.f) return UA_ERR_INVALID_ARG;   // training is dense
     (void)b_final;   // the backward recomputes the decay prefixes; b_final is not read
     const void* need[] = {q, k, v, g, a_q, a_k, alpha, beta, o, lse, d_o, dq, dk, dv, dg, da_q, da_k, dalpha, dbeta, ws};
     for (const void* p : need)

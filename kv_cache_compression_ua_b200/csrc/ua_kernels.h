@@ -66,6 +66,8 @@ struct FwdParams {
     float* lse;         // [B,H,T] or NULL
     float* lambda_dbg;  // [B,Hkv,T,T] or NULL (pre-zeroed)
     int variant;        // UA_VAR_* bits (decay_var)
+    float prune_thr;    // chunked pruned prefill: a key whose Pb at its chunk boundary exceeds
+                        // this (-log p) is evicted; +inf = dense
 };
 
 // A 64-row query tile and a key tile of the SIMT paths contribute exactly nothing (every
@@ -189,6 +191,7 @@ struct FwdTcLaunch {
     void* o;
     float* lse;
     float* b_final;      // [B*Hkv][T] or NULL
+    float prune_thr;     // chunked pruned prefill (chunks = the 128-row query tiles): -log p, +inf = dense
 };
 
 bool fwd_tc_supported(int d, int G);

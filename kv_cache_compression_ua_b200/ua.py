@@ -31,7 +31,7 @@ class UAError(RuntimeError):
 class ua_shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("Hkv", ctypes.c_int),
                 ("d", ctypes.c_int), ("scale", ctypes.c_float), ("rope_theta", ctypes.c_double),
-                ("dtype", ctypes.c_int), ("variant", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("variant", ctypes.c_int), ("prune_p", ctypes.c_float)]
 
 
 # ua_shape.variant bits (UA_VAR_* in ua.h); 0 is the method itself.
@@ -124,11 +124,11 @@ def _dtype_code(dt: torch.dtype) -> int:
     raise ValueError(f"unsupported activation dtype {dt}")
 
 
-def make_shape(q: torch.Tensor, k: torch.Tensor, scale=None, theta=500000.0, variant=0) -> ua_shape:
+def make_shape(q: torch.Tensor, k: torch.Tensor, scale=None, theta=500000.0, variant=0, prune_p=0.0) -> ua_shape:
     B, T, H, d = q.shape
     Hkv = k.shape[2]
     scale = float(d) ** -0.5 if scale is None else float(scale)
-    return ua_shape(B, T, H, Hkv, d, scale, float(theta), _dtype_code(q.dtype), int(variant))
+    return ua_shape(B, T, H, Hkv, d, scale, float(theta), _dtype_code(q.dtype), int(variant), float(prune_p))
 
 
 def prefill_workspace_size(shape: ua_shape) -> int:
@@ -143,11 +143,11 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0, want_lse=True,
-                want_bfinal=True, want_lambda=False, out=None, ws=None, variant=0, stream=None):
-    """ua_prefill_fwd (variant: VAR_* bits).  Returns dict(o, lse, b_final, lam) (absent
-    outputs are None)."""
+                want_bfinal=True, want_lambda=False, out=None, ws=None, variant=0, prune_p=0.0, stream=None):
+    """ua_prefill_fwd (variant: VAR_* bits; prune_p > 0: chunked pruned prefill).  Returns
+    dict(o, lse, b_final, lam) (absent outputs are None)."""
     lib = load_library()
-    shape = make_shape(q, k, scale, theta, variant)
+    shape = make_shape(q, k, scale, theta, variant, prune_p)
     B, T, H, d = q.shape
     Hkv = k.shape[2]
     dev = q.device
@@ -175,11 +175,11 @@ def prefill_tile_stats(shape: ua_shape, ws: torch.Tensor, stream=None) -> tuple:
 
 
 def prefill_fwd_noalloc(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0, want_lse=True,
-                        want_bfinal=True, out=None, variant=0, stream=None):
+                        want_bfinal=True, out=None, variant=0, prune_p=0.0, stream=None):
     """ua_prefill_fwd_noalloc: the prefill forward using the library's fixed internal scratch
     instead of a workspace (for callers that cannot allocate device memory)."""
     lib = load_library()
-    shape = make_shape(q, k, scale, theta, variant)
+    shape = make_shape(q, k, scale, theta, variant, prune_p)
     B, T, H, d = q.shape
     Hkv = k.shape[2]
     dev = q.device

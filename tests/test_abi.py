@@ -94,6 +94,18 @@ def test_variant_bits_validated(lib, variant, code):
         assert _fwd(lib, s) == code
 
 
+@pytest.mark.parametrize("prune_p,code", [(-0.1, 1), (1.5, 1), (float("nan"), 1), (0.0, 0), (0.15, 0), (1.0, 0)])
+def test_prune_threshold_validated(lib, prune_p, code):
+    need = ctypes.c_size_t(0)
+    s = _shape(prune_p=prune_p)
+    assert lib.ua_prefill_workspace_size(ctypes.byref(s), ctypes.byref(need)) == code
+    if code:
+        assert _fwd(lib, s) == code
+    # training is dense: the backward refuses any pruning threshold
+    bwd_code = 0 if prune_p == 0.0 else 1
+    assert lib.ua_prefill_bwd_workspace_size(ctypes.byref(s), ctypes.byref(need)) == bwd_code
+
+
 def test_mechanism_variants_leave_the_tensor_core_path(lib):
     # a mechanism switched off runs the SIMT path: no tensor-core tile statistics
     tiles, skipped = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
