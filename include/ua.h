@@ -78,6 +78,9 @@ typedef enum { UA_F32 = 0, UA_BF16 = 1 } ua_dtype;
 #define UA_VAR_NO_SIM_DECAY 4
 #define UA_VAR_QUERY_NORM 8
 
+/* Decode-step flag: defer compaction (see ua_decode_step). */
+#define UA_DECODE_DEFER_COMPACT 256
+
 /* Problem shape of a prefill call.  d (head_dim) must be 64 or 128; H % Hkv == 0 and
  * H / Hkv in {1, 2, 3, 4, 8}; T >= 1. */
 typedef struct {
@@ -238,7 +241,13 @@ ua_status ua_cache_compact(const ua_cache* cache, const uint8_t* keep, float p,
  * evicted (all words are written).  kept_idx (optional, [B,Hkv,cap] int32): pre-step
  * slot of each survivor in new order, then -1 for the appended token.
  * flags: UA_VAR_* bits, which must equal the variant of the prefill that filled the cache
- * (0 = the method itself; the cache stores softplus(a_k) whatever the variant).  Every cache call requires capacity <= 2^20 slots
+ * (0 = the method itself; the cache stores softplus(a_k) whatever the variant), plus
+ * optionally UA_DECODE_DEFER_COMPACT: step 4 then moves nothing.  Every pair stays in its slot
+ * with its updated bias, the new token is appended at slot n_kept, and evicted pairs (b < log p,
+ * which never rises again) are left in place, excluded from attention by their bias, until a
+ * ua_cache_compact(p) removes them; evict_bits then marks every pair with b < log p and
+ * kept_idx (if given) holds s at slot s.  The outputs and the compacted cache are those of the
+ * step-by-step compaction; deferring trades the per-step moves for cache slots.  Every cache call requires capacity <= 2^20 slots
  * (UA_ERR_UNSUPPORTED otherwise).  If a cache is full (no pair evicted and n_kept == capacity)
  * the step sets UA_ERR_CAPACITY in the device status word and that cache is left as it
  * was after compaction, without the new token. */

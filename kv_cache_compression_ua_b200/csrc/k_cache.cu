@@ -169,8 +169,12 @@ __global__ void __launch_bounds__(256) k_cache_compact(CompactParams p) {
 // ------------------------------------------------------------------ decode step
 // grid (B*Hkv), 256 threads.  Dynamic shared memory: eviction bitmap (ceil(cap/32) words)
 // followed by the per-group softmax partials.
-template <typename TC, int DH, int G>
+// DEFER: deferred compaction (UA_DECODE_DEFER_COMPACT).  VAR: an ablation variant is set; without
+// it the variant is the constant 0 and every variant branch folds away.  Both are separate
+// instantiations so that the method's own per-step path keeps its registers and instructions.
+template <typename TC, int DH, int G, bool DEFER, bool VAR>
 __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) {
+    const int variant = VAR ? p.variant : 0;
     using L = EntryLayout<TC, DH>;
     constexpr int VEC = L::VEC, LPE = L::LPE, EPB = L::EPB, NW = L::NW;
     constexpr int half = DH / 2;
@@ -264,7 +268,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         s_ktr[m + half] = x1 * cs + x0 * sn;
     }
     __syncthreads();
-    if (p.variant & kVarQNorm) {                  // query RMS norm (RoPE keeps the norm)
+    if (variant & kVarQNorm) {                    // query RMS norm (RoPE keeps the norm)
         if (tid < G) {
             float qq = 0.f;
             for (int x = 0; x < DH; ++x) qq = fmaf(s_q[tid][x], s_q[tid][x], qq);
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         for (int x = 0; x < DH; ++x) a = fmaf(s_q[tid][x], s_ktr[x], a);
         s_lt[tid] = a * p.scale;                      // new token's own bias is 0
     }
-    const float rq_t = (p.variant & kVarNoQ) ? 1.f : softplus_f(aq_t);
+    const float rq_t = (variant & kVarNoQ) ? 1.f : softplus_f(aq_t);
     const float rk_t = softplus_f(ak_t);          // stored in the cache as is
 
     float kq[VEC], qh[G][VEC];
@@ -346,7 +350,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
 #pragma unroll
         for (int e = 0; e < VEC; ++e) sim = fmaf(kq[e], xa[e], sim);
         sim = group_sum<LPE>(sim);
-        const float D = decay_var(rq_t, (p.variant & kVarNoK) ? 1.f : rkj, fmaf(al, sim, be), p.variant);
+        const float D = decay_var(rq_t, (variant & kVarNoK) ? 1.f : rkj, fmaf(al, sim, be), variant);
         const float bnew = bj - D;
         const bool keep = valid && (bnew >= p.logp);
 #pragma unroll
@@ -367,6 +371,14 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
             }
         }
         if (valid && !keep && gl == 0) atomicOr(&s_ev[j >> 5], 1u << (j & 31));
+        if (DEFER) {                              // every pair keeps its slot
+            if (valid && gl == 0) {
+                c.bias[base + j] = bnew;
+                if (p.kept_idx) p.kept_idx[base + j] = j;
+            }
+            __syncthreads();
+            continue;
+        }
         int tot;
         const int dst = out + pass_scan<LPE, NW>(keep, warp, lane, s_wcnt, &tot);
         if (keep) {
@@ -389,6 +401,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         __syncthreads();
     }
 
+    if (DEFER) out = n;                           // append after every pair, evicted ones included
     // ---- merge the per-group online-softmax states, add the new token, gate, store
     if (gl == 0) {
 #pragma unroll
@@ -469,18 +482,26 @@ cudaError_t launch_cache_compact(const CompactParams& p, bool bf16, cudaStream_t
     return cudaGetLastError();
 }
 
+template <typename TC, int DH, int G, bool DEFER, bool VAR>
+static cudaError_t decode_launch(const DecodeParams& p, size_t smem, cudaStream_t s) {
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_decode<TC, DH, G, DEFER, VAR>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    UA_PROFILE("k_decode", s);
+    k_decode<TC, DH, G, DEFER, VAR><<<p.c.B * p.c.Hkv, 256, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
 template <typename TC, int DH, int G>
 static cudaError_t decode_inst(const DecodeParams& p, cudaStream_t s) {
     using L = EntryLayout<TC, DH>;
     const int words = (p.c.cap + 31) / 32;
     const size_t smem = sizeof(float) * ((size_t)((words + 3) & ~3) + 2 * L::EPB * G + (size_t)L::EPB * G * DH);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k_decode<TC, DH, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    UA_PROFILE("k_decode", s);
-    k_decode<TC, DH, G><<<p.c.B * p.c.Hkv, 256, smem, s>>>(p);
-    return cudaGetLastError();
+    if (p.variant != 0)
+        return p.defer ? decode_launch<TC, DH, G, true, true>(p, smem, s) : decode_launch<TC, DH, G, false, true>(p, smem, s);
+    return p.defer ? decode_launch<TC, DH, G, true, false>(p, smem, s) : decode_launch<TC, DH, G, false, false>(p, smem, s);
 }
 
 template <typename TC, int DH>

@@ -442,7 +442,9 @@ ua_status ua_decode_step(const ua_cache* c, int H, const void* q, const void* k,
                          int32_t* kept_idx, int flags, void* stream) {
     ua_status st = check_cache(c);
     if (st != UA_OK) return st;
-    if (H < 1 || H % c->Hkv != 0 || pos_t < 0 || !variant_ok(flags)) return UA_ERR_INVALID_ARG;
+    const int defer = flags & UA_DECODE_DEFER_COMPACT;
+    if (H < 1 || H % c->Hkv != 0 || pos_t < 0 || !variant_ok(flags & ~UA_DECODE_DEFER_COMPACT))
+        return UA_ERR_INVALID_ARG;
     if (!group_ok(H / c->Hkv)) return UA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !g || !a_q || !a_k || !alpha || !beta || !o) return UA_ERR_INVALID_ARG;
     if (!(p >= 0.f && p <= 1.f) || !isfinite(scale) || !(rope_theta > 0.0)) return UA_ERR_INVALID_ARG;
@@ -453,7 +455,8 @@ ua_status ua_decode_step(const ua_cache* c, int H, const void* q, const void* k,
     dp.c = view(c); dp.H = H; dp.G = H / c->Hkv; dp.pos_t = pos_t; dp.scale = scale;
     dp.logp = p > 0.f ? logf(p) : -INFINITY; dp.theta = rope_theta; dp.rf = rope_freq(rope_theta, c->d);
     dp.q = q; dp.k = k; dp.v = v; dp.g = g; dp.a_q = a_q; dp.a_k = a_k; dp.alpha = alpha; dp.beta = beta;
-    dp.o = o; dp.evict_bits = evict_bits; dp.kept_idx = kept_idx; dp.variant = flags;
+    dp.o = o; dp.evict_bits = evict_bits; dp.kept_idx = kept_idx;
+    dp.variant = flags & ~UA_DECODE_DEFER_COMPACT; dp.defer = defer ? 1 : 0;
     return cuda_status(launch_decode(dp, c->dtype == UA_BF16, static_cast<cudaStream_t>(stream)));
 }
 

@@ -131,6 +131,7 @@ struct DecodeParams {
     uint32_t* evict_bits;
     int32_t* kept_idx;
     int variant;         // UA_VAR_* bits
+    int defer;           // 1: no compaction (pairs stay in their slots; append at n_kept)
 };
 
 // Backward (SIMT path).  Inputs from the f32 token preparation and boundary pass (query

@@ -36,6 +36,7 @@ class ua_shape(ctypes.Structure):
 
 # ua_shape.variant bits (UA_VAR_* in ua.h); 0 is the method itself.
 VAR_NO_QUERY_DECAY, VAR_NO_KEY_DECAY, VAR_NO_SIM_DECAY, VAR_QUERY_NORM = 1, 2, 4, 8
+DECODE_DEFER_COMPACT = 256      # ua_decode_step flag: leave evicted pairs in place
 
 
 class ua_cache(ctypes.Structure):
@@ -273,9 +274,10 @@ def cache_compact(cache: Cache, p: float = 0.0, keep=None, kept_idx=None, stream
 
 
 def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: float, *, scale=None,
-                theta=500000.0, out=None, evict_bits=None, kept_idx=None, variant=0, stream=None):
-    """ua_decode_step for one token per sequence (variant: the prefill's VAR_* bits).
-    Returns o [B,H,d]."""
+                theta=500000.0, out=None, evict_bits=None, kept_idx=None, variant=0, defer_compact=False,
+                stream=None):
+    """ua_decode_step for one token per sequence (variant: the prefill's VAR_* bits;
+    defer_compact: leave evicted pairs in place until cache_compact).  Returns o [B,H,d]."""
     H = q.shape[1]
     d = q.shape[2]
     scale = float(d) ** -0.5 if scale is None else float(scale)
@@ -283,7 +285,8 @@ def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: 
     c = cache.struct()
     rc = load_library().ua_decode_step(ctypes.byref(c), H, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q),
                                        _ptr(a_k), _ptr(alpha), _ptr(beta), int(pos_t), float(p), scale,
-                                       float(theta), _ptr(o), _ptr(evict_bits), _ptr(kept_idx), int(variant),
+                                       float(theta), _ptr(o), _ptr(evict_bits), _ptr(kept_idx),
+                                       int(variant) | (DECODE_DEFER_COMPACT if defer_compact else 0),
                                        _stream(stream))
     _check("ua_decode_step", rc)
     return o

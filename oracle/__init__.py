@@ -49,7 +49,7 @@ def _load():
         lib.ora_lambda_bruteforce.argtypes = [I, I, I, I, P, P, P, P, P, P, I, I]
         lib.ora_lambda_bruteforce.restype = I
         lib.ora_decode_step.argtypes = ([I, I, I, I, I, Dd, Dd] + [P] * 6 + [P] * 8 +
-                                        [Dd, Dd, Dd, P, P, P, P, P, I, I])
+                                        [Dd, Dd, Dd, P, P, P, P, P, I, I, I])
         lib.ora_decode_step.restype = I
         lib.ora_compact_order.argtypes = [I, P, P]
         lib.ora_compact_order.restype = I
@@ -190,9 +190,24 @@ class DecodeCache:
                 self.n[b, h] = n
         return in_band
 
+    def compact(self, p):
+        """Stable compaction of every slot list by b >= log p (after deferred decode steps)."""
+        logp = float(np.log(p)) if p > 0 else -np.inf
+        for b in range(self.B):
+            for h in range(self.Hkv):
+                n = int(self.n[b, h])
+                idx = compact_order(self.b[b, h, :n] >= logp)
+                m = len(idx)
+                for arr in (self.k, self.v):
+                    arr[b, h, :m] = arr[b, h, idx]
+                for arr in (self.ak, self.pos, self.b):
+                    arr[b, h, :m] = arr[b, h, idx]
+                self.n[b, h] = m
+
 
 def decode_step(cache: DecodeCache, q, k, v, g, a_q, a_k, alpha, beta, pos_t, p, *,
-                scale=None, theta=500000.0, band=1e-3, adopt_keep=None, variant=0, nthreads=None):
+                scale=None, theta=500000.0, band=1e-3, adopt_keep=None, variant=0, defer=False,
+                nthreads=None):
     """One decode step on the oracle cache (mutated in place).
 
     q, g [B,H,d]; k, v [B,Hkv,d]; a_q, a_k [B,Hkv].  Returns dict(o [B,H,d],
@@ -217,7 +232,7 @@ def decode_step(cache: DecodeCache, q, k, v, g, a_q, a_k, alpha, beta, pos_t, p,
                                  _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
                                  _ptr(alpha), _ptr(beta), float(pos_t), logp, float(band),
                                  _ptr(ak_), _ptr(o), _ptr(ev), _ptr(inb), _ptr(order),
-                                 int(variant), nthreads or default_threads())
+                                 int(variant), int(bool(defer)), nthreads or default_threads())
     if rc != 0:
         raise RuntimeError(f"ora_decode_step failed (code {rc})")
     return {"o": o, "evict": ev, "in_band": inb, "kept_order": order, "n_before": n_before}

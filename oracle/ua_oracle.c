@@ -346,6 +346,11 @@ int ora_lambda_bruteforce(int B, int T, int Hkv, int d, const double* k, const d
  * `band` of log p the oracle takes this decision instead of its own, so that two
  * implementations whose roundings differ near the threshold stay in lockstep.
  * in_band (optional out) flags those pairs.
+ *
+ * defer != 0 (deferred compaction): step 4 moves nothing.  Every pair keeps its slot and its
+ * updated bias, evicted ones included (their bias stays below log p: it only decreases), and the
+ * new token goes to slot n.  kept_order then holds s at slot s.  Step 3 attends over the same
+ * pairs either way, since an evicted pair's bias never rises back above log p.
  */
 typedef struct {
     int B, H, Hkv, d, cap;
@@ -358,6 +363,7 @@ typedef struct {
     uint8_t *evict, *in_band;
     int64_t* kept_order;
     int variant;
+    int defer;
 } dec_ctx;
 
 static void dec_unit(void* vctx, int unit) {
@@ -383,7 +389,8 @@ static void dec_unit(void* vctx, int unit) {
     double rq_t = softplus(c->aq[(size_t)b * Hkv + kvh]);
     const double alpha = c->alpha[kvh], beta = c->beta[kvh];
 
-    /* 1-2: bias update and eviction decision */
+    /* 1-2: bias update and eviction decision (a pair left in place by a deferred compaction
+     * already has b < log p and stays evicted) */
     for (int j = 0; j < n; ++j) {
         l2_normalise(c->kc + (base + j) * d, d, kj_hat);
         double rsim = softplus(alpha * dot(kt_hat, kj_hat, d) + beta);
@@ -423,9 +430,14 @@ static void dec_unit(void* vctx, int unit) {
         double* oh = c->o + ((size_t)b * H + h) * d;
         for (int x = 0; x < d; ++x) oh[x] = acc[x] / l * sigmoid(gh[x]);
     }
-    /* 4: stable compaction, then append */
+    /* 4: stable compaction (or none, deferred), then append */
     int w = 0;
-    for (int j = 0; j < n; ++j) {
+    if (c->defer) {
+        for (int j = 0; j < n; ++j)
+            if (c->kept_order) c->kept_order[base + j] = j;
+        w = n;
+    }
+    for (int j = 0; j < n && !c->defer; ++j) {
         if (!keep[j]) continue;
         if (c->kept_order) c->kept_order[base + w] = j;
         if (w != j) {
@@ -457,12 +469,12 @@ int ora_decode_step(int B, int H, int Hkv, int d, int cap, double scale, double 
                     const double* aq, const double* ak, const double* alpha, const double* beta,
                     double pos_t, double logp, double band, const uint8_t* adopt_keep,
                     double* o, uint8_t* evict, uint8_t* in_band, int64_t* kept_order,
-                    int variant, int nthreads) {
+                    int variant, int defer, int nthreads) {
     if (H % Hkv) return 1;
     if ((variant & ~VAR_ALL) || n_active(variant) == 0) return 1;
     dec_ctx c = {B, H, Hkv, d, cap, scale, theta, logp, band, pos_t, n_kept, kc, vc, akc,
                  posc, bc, q, k, v, g, aq, ak, alpha, beta, adopt_keep, o, evict, in_band,
-                 kept_order, variant};
+                 kept_order, variant, defer};
     run_units(dec_unit, &c, B * Hkv, nthreads);
     for (int u = 0; u < B * Hkv; ++u)
         if (n_kept[u] < 0) return 2;

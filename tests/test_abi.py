@@ -137,7 +137,7 @@ def test_cache_calls_reject_bad_arguments(lib):
     args = [P(FAKE)] * 8
     assert lib.ua_decode_step(ctypes.byref(c), 10, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
                               P(FAKE), None, None, 0, None) == 2
-    for bad in (16, 7, 15, -1):   # unknown bit; all three decay mechanisms off
+    for bad in (16, 7, 15, -1, 512, 256 | 7, 256 | 16):   # unknown bits; all three decay mechanisms off
         assert lib.ua_decode_step(ctypes.byref(c), 8, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
                                   P(FAKE), None, None, bad, None) == 1
     c3 = ua.ua_cache(2, 2, 80, 100, ua.UA_BF16, *([FAKE] * 7))

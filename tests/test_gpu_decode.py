@@ -253,3 +253,67 @@ def test_decode_1b_full_size_sampled(p):
     ls = Lockstep(w, T0=w.T, steps=I.DECODE_STEPS, p=p, b_sel=[0, w.B - 1], zero_prefill_q=True)
     for s in range(I.DECODE_STEPS):
         ls.step(s)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_deferred_compaction_matches_step_by_step(dtype):
+    """UA_DECODE_DEFER_COMPACT: pairs stay in place (evicted ones excluded by their bias) and one
+    ua_cache_compact(p) at the end gives the cache of step-by-step compaction.  Both GPU caches
+    take the same decisions; outputs and biases agree within the parity bars (the two kernel
+    instantiations may round the decay differently), slots and positions exactly."""
+    w = I.Workload("dec_defer", 2, 300, 8, 2, 64, dtype, 4500, bimodal_ak=True)
+    T0, steps, p = 300, 24, 0.15
+    adt = TORCH_DT[dtype]
+    x = I.make_prefill_inputs(w, T=T0)
+    d = {n: dev(a, adt if n in ("k", "v", "q", "g") else torch.float32) for n, a in x.items() if n != "d_o"}
+    r = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
+                       scale=w.scale, theta=w.theta, want_lse=False)
+    cap = T0 + steps + 1
+    caches = []
+    for _ in range(2):
+        c = ua.Cache.empty(w.B, w.Hkv, w.d, cap, adt)
+        ua.cache_fill(c, d["k"], d["v"], d["a_k"], r["b_final"], theta=w.theta)
+        ua.cache_compact(c, p)
+        caches.append(c)
+    eager, lazy = caches
+    words = (cap + 31) // 32
+    n_evicted = 0
+    for s in range(steps):
+        tok = I.make_decode_token(w, s)
+        t = {n: dev(a, adt if n in ("q", "k", "v", "g") else torch.float32) for n, a in tok.items()}
+        n_lazy = lazy.n_kept.cpu().numpy()
+        ev_e = torch.zeros(w.B, w.Hkv, words, dtype=torch.int32, device="cuda")
+        ev_l = torch.zeros_like(ev_e)
+        kept = torch.full((w.B, w.Hkv, cap), -7, dtype=torch.int32, device="cuda")
+        args = (t["q"], t["k"], t["v"], t["g"], t["a_q"], t["a_k"], d["alpha"], d["beta"], T0 + s, p)
+        o_e = ua.decode_step(eager, *args, scale=w.scale, theta=w.theta, evict_bits=ev_e)
+        o_l = ua.decode_step(lazy, *args, scale=w.scale, theta=w.theta, evict_bits=ev_l, kept_idx=kept,
+                             defer_compact=True)
+        assert ua.get_device_status() == 0
+        assert_close(f"o step {s}", o_l.float().cpu().numpy(), o_e.float().cpu().numpy(), dtype)
+        np.testing.assert_array_equal(lazy.n_kept.cpu().numpy(), n_lazy + 1)
+        kept = kept.cpu().numpy()
+        ev_l = ev_l.cpu().numpy().view(np.uint32)
+        ev_e = ev_e.cpu().numpy().view(np.uint32)
+        pos_l, pos_e, n_e = lazy.pos.cpu().numpy(), eager.pos.cpu().numpy(), eager.n_kept.cpu().numpy()
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                m = n_lazy[b, h]
+                np.testing.assert_array_equal(kept[b, h, :m], np.arange(m))
+                assert kept[b, h, m] == -1
+                live = ~unpack_bits(ev_l[b, h], m)          # pairs with b >= log p after this step
+                np.testing.assert_array_equal(pos_l[b, h, :m][live], pos_e[b, h, :n_e[b, h] - 1])
+        n_evicted += int(sum(bin(int(v)).count("1") for v in ev_e.ravel()))
+    assert n_evicted > 0
+    ua.cache_compact(lazy, p)
+    np.testing.assert_array_equal(lazy.n_kept.cpu().numpy(), eager.n_kept.cpu().numpy())
+    n_e = eager.n_kept.cpu().numpy()
+    for name in ("pos", "bias", "rk", "khat", "krope", "v"):
+        a, b_ = getattr(lazy, name).float().cpu().numpy(), getattr(eager, name).float().cpu().numpy()
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                m = n_e[b, h]
+                if name == "bias":
+                    assert_close("bias", a[b, h, :m], b_[b, h, :m], "f32", relative_max=True)
+                else:
+                    np.testing.assert_array_equal(a[b, h, :m], b_[b, h, :m], err_msg=name)

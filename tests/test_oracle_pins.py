@@ -344,3 +344,40 @@ def test_backward_vetoed_decay_has_zero_decay_grads():
     gr = oracle.prefill_bwd(**x, d_o=rng.standard_normal(x["q"].shape))
     assert np.all(gr["da_k"] == 0) and np.all(gr["dalpha"] == 0) and np.all(gr["dbeta"] == 0)
     assert np.all(np.isfinite(gr["dq"])) and np.all(np.isfinite(gr["dk"]))
+
+
+def test_deferred_compaction_equals_step_by_step():
+    """Deferred compaction (pairs left in place, compacted once at the end) attends over the same
+    pairs in the same order as step-by-step compaction: an evicted pair's bias never rises back
+    above log p (paperlayer.ai summary, §4.2: the bias is monotone), so outputs agree bit for bit
+    and the compacted cache is the same."""
+    T0, n, p = 16, 20, 0.15
+    w, x = small_case(T=T0 + n, B=2, H=4, Hkv=2, d=16, seed=13)
+    pre = oracle.prefill_fwd(**{k: (v[:, :T0] if v.ndim >= 3 else v) for k, v in x.items()})
+    caches = []
+    for _ in range(2):
+        c = oracle.DecodeCache(w.B, w.Hkv, w.d, T0 + n + 1)
+        c.fill_from_prefill(x["k"][:, :T0], x["v"][:, :T0], x["a_k"][:, :T0], pre["b_final"], logp=math.log(p))
+        caches.append(c)
+    eager, lazy = caches
+    n_evicted = 0
+    for t in range(T0, T0 + n):
+        args = (x["q"][:, t], x["k"][:, t], x["v"][:, t], x["g"][:, t], x["a_q"][:, t], x["a_k"][:, t],
+                x["alpha"], x["beta"], t, p)
+        n0 = lazy.n.copy()
+        re = oracle.decode_step(eager, *args)
+        rl = oracle.decode_step(lazy, *args, defer=True)
+        np.testing.assert_array_equal(rl["o"], re["o"])
+        assert np.all(lazy.n == n0 + 1)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                assert list(rl["kept_order"][b, h, :n0[b, h]]) == list(range(n0[b, h]))
+        n_evicted += int(re["evict"].sum())
+    lazy.compact(p)
+    assert n_evicted > 0
+    np.testing.assert_array_equal(lazy.n, eager.n)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            m = eager.n[b, h]
+            for name in ("k", "v", "ak", "pos", "b"):
+                np.testing.assert_array_equal(getattr(lazy, name)[b, h, :m], getattr(eager, name)[b, h, :m])
