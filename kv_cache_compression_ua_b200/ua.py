@@ -112,6 +112,44 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+F32 = (torch.float32,)
+I32 = (torch.int32,) + ((torch.uint32,) if hasattr(torch, "uint32") else ())
+MASK = (torch.uint8, torch.bool)
+
+
+def _need(name, t, n, dtypes):
+    """Refuse a tensor the library would read or write past its end, or in another element type
+    (the C ABI takes bare pointers, so this is the last place such a mistake can be caught)."""
+    if t is None:
+        return
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
+    if t.numel() < n:
+        raise ValueError(f"{name}: {t.numel()} elements, the call needs {n}")
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out):
+    """Checks the prefill arguments against q [B,T,H,d] and k [B,T,Hkv,d]; returns the sizes."""
+    B, T, H, d = q.shape
+    if k.dim() != 4 or (k.shape[0], k.shape[1], k.shape[3]) != (B, T, d):
+        raise ValueError(f"k: shape {tuple(k.shape)}, expected [{B}, {T}, Hkv, {d}]")
+    Hkv = k.shape[2]
+    act = (q.dtype,)
+    _need("k", k, B * T * Hkv * d, act)
+    _need("v", v, B * T * Hkv * d, act)
+    _need("g", g, B * T * H * d, act)
+    _need("a_q", a_q, B * T * Hkv, F32)
+    _need("a_k", a_k, B * T * Hkv, F32)
+    _need("alpha", alpha, Hkv, F32)
+    _need("beta", beta, Hkv, F32)
+    _need("out", out, B * T * H * d, act)
+    return B, T, H, Hkv, d
+
+
 def _stream(stream):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
@@ -148,20 +186,19 @@ def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0
     """ua_prefill_fwd (variant: VAR_* bits; prune_p > 0: chunked pruned prefill).  Returns
     dict(o, lse, b_final, lam) (absent outputs are None)."""
     lib = load_library()
+    B, T, H, Hkv, d = _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out)
     shape = make_shape(q, k, scale, theta, variant, prune_p)
-    B, T, H, d = q.shape
-    Hkv = k.shape[2]
     dev = q.device
     o = out if out is not None else torch.empty_like(q)
     lse = torch.empty(B, H, T, dtype=torch.float32, device=dev) if want_lse else None
     bfin = torch.empty(B, Hkv, T, dtype=torch.float32, device=dev) if want_bfinal else None
     lam = torch.empty(B, Hkv, T, T, dtype=torch.float32, device=dev) if want_lambda else None
     need = prefill_workspace_size(shape)
-    if ws is None or ws.numel() < need:
+    if ws is None or _nbytes(ws) < need:
         ws = alloc_workspace(need, dev)
     rc = lib.ua_prefill_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
                             _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(bfin), _ptr(lam),
-                            _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(stream))
+                            _ptr(ws), ctypes.c_size_t(_nbytes(ws)), _stream(stream))
     _check("ua_prefill_fwd", rc)
     return {"o": o, "lse": lse, "b_final": bfin, "lam": lam}
 
@@ -171,7 +208,7 @@ def prefill_tile_stats(shape: ua_shape, ws: torch.Tensor, stream=None) -> tuple:
     ua_prefill_fwd that used `ws` for `shape`."""
     tiles, skipped = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
     _check("ua_prefill_tile_stats", load_library().ua_prefill_tile_stats(
-        ctypes.byref(shape), _ptr(ws), ws.numel(), ctypes.byref(tiles), ctypes.byref(skipped), _stream(stream)))
+        ctypes.byref(shape), _ptr(ws), _nbytes(ws), ctypes.byref(tiles), ctypes.byref(skipped), _stream(stream)))
     return tiles.value, skipped.value
 
 
@@ -180,9 +217,8 @@ def prefill_fwd_noalloc(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=
     """ua_prefill_fwd_noalloc: the prefill forward using the library's fixed internal scratch
     instead of a workspace (for callers that cannot allocate device memory)."""
     lib = load_library()
+    B, T, H, Hkv, d = _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out)
     shape = make_shape(q, k, scale, theta, variant, prune_p)
-    B, T, H, d = q.shape
-    Hkv = k.shape[2]
     dev = q.device
     o = out if out is not None else torch.empty_like(q)
     lse = torch.empty(B, H, T, dtype=torch.float32, device=dev) if want_lse else None
@@ -206,19 +242,24 @@ def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, d_o, *, scal
     """ua_prefill_bwd (variant: the forward's VAR_* bits).  Returns dict(dq, dk, dv, dg,
     da_q, da_k, dalpha, dbeta)."""
     lib = load_library()
+    B, T, H, Hkv, d = _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, None)
+    _need("o", o, B * T * H * d, (q.dtype,))
+    _need("d_o", d_o, B * T * H * d, (q.dtype,))
+    _need("lse", lse, B * H * T, F32)
+    _need("b_final", b_final, B * Hkv * T, F32)
     shape = make_shape(q, k, scale, theta, variant)
     dev = q.device
     gr = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
           "dg": torch.empty_like(g), "da_q": torch.empty_like(a_q), "da_k": torch.empty_like(a_k),
           "dalpha": torch.empty_like(alpha), "dbeta": torch.empty_like(beta)}
     need = prefill_bwd_workspace_size(shape)
-    if ws is None or ws.numel() < need:
+    if ws is None or _nbytes(ws) < need:
         ws = alloc_workspace(need, dev)
     rc = lib.ua_prefill_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
                             _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(b_final), _ptr(d_o),
                             _ptr(gr["dq"]), _ptr(gr["dk"]), _ptr(gr["dv"]), _ptr(gr["dg"]), _ptr(gr["da_q"]),
                             _ptr(gr["da_k"]), _ptr(gr["dalpha"]), _ptr(gr["dbeta"]), _ptr(ws),
-                            ctypes.c_size_t(ws.numel()), _stream(stream))
+                            ctypes.c_size_t(_nbytes(ws)), _stream(stream))
     _check("ua_prefill_bwd", rc)
     return gr
 
@@ -252,6 +293,13 @@ class Cache:
                      torch.zeros(B, Hkv, dtype=torch.int32, **kw))
 
     def struct(self) -> ua_cache:
+        n = self.B * self.Hkv * self.capacity
+        for name in ("khat", "krope", "v"):
+            _need(f"cache.{name}", getattr(self, name), n * self.d, (self.dtype,))
+        _need("cache.bias", self.bias, n, F32)
+        _need("cache.rk", self.rk, n, F32)
+        _need("cache.pos", self.pos, n, I32)
+        _need("cache.n_kept", self.n_kept, self.B * self.Hkv, I32)
         return ua_cache(self.B, self.Hkv, self.d, self.capacity, _dtype_code(self.dtype),
                         self.khat.data_ptr(), self.krope.data_ptr(), self.v.data_ptr(), self.bias.data_ptr(),
                         self.rk.data_ptr(), self.pos.data_ptr(), self.n_kept.data_ptr())
@@ -261,13 +309,23 @@ class Cache:
 
 
 def cache_fill(cache: Cache, k, v, a_k, b_final, *, theta=500000.0, stream=None):
+    if k.dim() != 4 or (k.shape[0], k.shape[2], k.shape[3]) != (cache.B, cache.Hkv, cache.d):
+        raise ValueError(f"k: shape {tuple(k.shape)}, expected [{cache.B}, T, {cache.Hkv}, {cache.d}]")
     T = k.shape[1]
+    n = cache.B * T * cache.Hkv
+    _need("k", k, n * cache.d, (cache.dtype,))
+    _need("v", v, n * cache.d, (cache.dtype,))
+    _need("a_k", a_k, n, F32)
+    _need("b_final", b_final, n, F32)
     c = cache.struct()
     _check("ua_cache_fill", load_library().ua_cache_fill(ctypes.byref(c), T, _ptr(k), _ptr(v), _ptr(a_k),
                                                          _ptr(b_final), float(theta), _stream(stream)))
 
 
 def cache_compact(cache: Cache, p: float = 0.0, keep=None, kept_idx=None, stream=None):
+    n = cache.B * cache.Hkv * cache.capacity
+    _need("keep", keep, n, MASK)
+    _need("kept_idx", kept_idx, n, I32)
     c = cache.struct()
     _check("ua_cache_compact", load_library().ua_cache_compact(ctypes.byref(c), _ptr(keep), float(p),
                                                                _ptr(kept_idx), _stream(stream)))
@@ -278,8 +336,21 @@ def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: 
                 stream=None):
     """ua_decode_step for one token per sequence (variant: the prefill's VAR_* bits;
     defer_compact: leave evicted pairs in place until cache_compact).  Returns o [B,H,d]."""
-    H = q.shape[1]
-    d = q.shape[2]
+    B, H, d = q.shape
+    if (B, d) != (cache.B, cache.d):
+        raise ValueError(f"q: shape {tuple(q.shape)}, expected [{cache.B}, H, {cache.d}]")
+    Hkv, act = cache.Hkv, (cache.dtype,)
+    _need("q", q, B * H * d, act)
+    _need("k", k, B * Hkv * d, act)
+    _need("v", v, B * Hkv * d, act)
+    _need("g", g, B * H * d, act)
+    _need("a_q", a_q, B * Hkv, F32)
+    _need("a_k", a_k, B * Hkv, F32)
+    _need("alpha", alpha, Hkv, F32)
+    _need("beta", beta, Hkv, F32)
+    _need("out", out, B * H * d, act)
+    _need("evict_bits", evict_bits, B * Hkv * ((cache.capacity + 31) // 32), I32)
+    _need("kept_idx", kept_idx, B * Hkv * cache.capacity, I32)
     scale = float(d) ** -0.5 if scale is None else float(scale)
     o = out if out is not None else torch.empty_like(q)
     c = cache.struct()

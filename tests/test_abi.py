@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 from kv_cache_compression_ua_b200 import build as ua_build
 from kv_cache_compression_ua_b200 import ua
@@ -165,3 +166,65 @@ def test_tile_stats_host_logic(lib):
                                      None) == 1
     assert lib.ua_prefill_tile_stats(ctypes.byref(tc), ctypes.c_void_p(256), 16, ctypes.byref(tiles),
                                      ctypes.byref(skipped), None) == 4
+
+
+# --------------------------------------------------------------------------- Python binding checks
+# The binding refuses, before any CUDA call, tensors the library would read or write past their
+# end or in another element type.  CPU tensors with the right sizes get through these checks
+# and stop at the device check, which is how the tests tell the two apart.
+
+def _prefill_args(B=1, T=8, H=4, Hkv=2, d=64, act=torch.bfloat16):
+    f = torch.float32
+    return dict(q=torch.zeros(B, T, H, d, dtype=act), k=torch.zeros(B, T, Hkv, d, dtype=act),
+                v=torch.zeros(B, T, Hkv, d, dtype=act), g=torch.zeros(B, T, H, d, dtype=act),
+                a_q=torch.zeros(B, T, Hkv, dtype=f), a_k=torch.zeros(B, T, Hkv, dtype=f),
+                alpha=torch.zeros(Hkv, dtype=f), beta=torch.zeros(Hkv, dtype=f))
+
+
+def _call_fwd(**over):
+    a = _prefill_args()
+    a.update(over)
+    return ua.prefill_fwd(a["q"], a["k"], a["v"], a["g"], a["a_q"], a["a_k"], a["alpha"], a["beta"])
+
+
+def test_binding_passes_well_formed_prefill_arguments(lib):
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        _call_fwd()
+
+
+@pytest.mark.parametrize("name,bad,msg", [
+    ("a_q", torch.zeros(1, 8, dtype=torch.float32), "a_q"),                   # [B,T] instead of [B,T,Hkv]
+    ("alpha", torch.zeros(2, dtype=torch.bfloat16), "alpha"),                 # wrong element type
+    ("v", torch.zeros(1, 8, 2, 32, dtype=torch.bfloat16), "v"),               # half the head dim
+    ("g", torch.zeros(1, 8, 4, 64, dtype=torch.float32), "g"),                # other activation type
+    ("k", torch.zeros(1, 7, 2, 64, dtype=torch.bfloat16), "k: shape"),        # T differs from q
+])
+def test_binding_refuses_undersized_or_mistyped_prefill_arguments(lib, name, bad, msg):
+    with pytest.raises(ValueError, match=msg):
+        _call_fwd(**{name: bad})
+
+
+def test_binding_refuses_bad_cache_and_decode_arguments(lib):
+    c = ua.Cache.empty(2, 2, 64, 40, torch.bfloat16, device="cpu")
+    f = torch.float32
+    q = torch.zeros(2, 4, 64, dtype=torch.bfloat16)
+    kv = torch.zeros(2, 2, 64, dtype=torch.bfloat16)
+    a = torch.zeros(2, 2, dtype=f)
+    ab = torch.zeros(2, dtype=f)
+    with pytest.raises(ValueError, match="CUDA tensors"):          # well formed
+        ua.decode_step(c, q, kv, kv, q, a, a, ab, ab, 40, 0.1)
+    with pytest.raises(ValueError, match="evict_bits"):
+        ua.decode_step(c, q, kv, kv, q, a, a, ab, ab, 40, 0.1, evict_bits=torch.zeros(2, 2, 1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="kept_idx"):
+        ua.decode_step(c, q, kv, kv, q, a, a, ab, ab, 40, 0.1, kept_idx=torch.zeros(2, 2, 40, dtype=torch.int64))
+    with pytest.raises(ValueError, match="q: shape"):
+        ua.decode_step(c, torch.zeros(3, 4, 64, dtype=torch.bfloat16), kv, kv, q, a, a, ab, ab, 40, 0.1)
+    with pytest.raises(ValueError, match="a_k"):
+        ua.decode_step(c, q, kv, kv, q, a, torch.zeros(2, dtype=f), ab, ab, 40, 0.1)
+    with pytest.raises(ValueError, match="keep"):
+        ua.cache_compact(c, keep=torch.zeros(2, 2, 40, dtype=torch.int32))
+    with pytest.raises(ValueError, match="k: shape"):
+        ua.cache_fill(c, torch.zeros(2, 10, 2, 128, dtype=torch.bfloat16), kv, a, a)
+    c.bias = torch.zeros(2, 2, 40, dtype=torch.float64)
+    with pytest.raises(ValueError, match="cache.bias"):
+        ua.cache_compact(c, 0.1)
