@@ -325,7 +325,10 @@ def bench_e2e(args, w, x):
 
 def bench_decode(args, peaks, peaks_kind):
     """Decode workload: B=32 caches prefilled (on the GPU) from a 16k-token draw, compacted at
-    p, then 256 single-token steps captured in one CUDA graph and replayed."""
+    p, then 256 single-token steps captured in one CUDA graph and replayed.  Besides the
+    workload's thresholds, two supplementary cases: p = 0 (no eviction, the longest caches)
+    and a retention-matched draw (the slow mode of a_k moved so that the prefill keeps the
+    pages' 16k average share of the keys, 1/21.38 at p = 0.15)."""
     from kv_cache_compression_ua_b200 import ua
     w = I.WORKLOADS["decode_1b"]
     steps = I.DECODE_STEPS
@@ -334,19 +337,38 @@ def bench_decode(args, peaks, peaks_kind):
     q0 = torch.zeros(w.B, T0, w.H, w.d, dtype=torch.bfloat16, device="cuda")
     r = ua.prefill_fwd(q0, x["k"], x["v"], q0, x["a_q"], x["a_k"], x["alpha"], x["beta"],
                        scale=w.scale, theta=w.theta, want_lse=False)
-    del q0
     bfinal = r["b_final"]
     del r
+    # Supplementary retention-matched workload: the same draws with the slow mode of a_k moved
+    # so that the cache kept after the prefill holds the pages' 16k average share of the keys.
+    retained = args.decode_p is None
+    if retained:
+        wr = w.resized(ak_slow_mean=I.DECODE_RETAINED_AK_SLOW_MEAN)
+        ak_r = I.make_prefill_inputs_torch(wr, "cuda", names=["a_k"])["a_k"]
+        r = ua.prefill_fwd(q0, x["k"], x["v"], q0, x["a_q"], ak_r, x["alpha"], x["beta"],
+                           scale=w.scale, theta=w.theta, want_lse=False)
+        bfinal_r = r["b_final"]
+        del r
+    del q0
     torch.cuda.empty_cache()
     toks = [I.make_decode_token(w, s) for s in range(steps)]
     tok = {n: torch.from_numpy(np.stack([t[n] for t in toks])).to("cuda").to(
         torch.bfloat16 if n in ("q", "k", "v", "g") else torch.float32).contiguous() for n in toks[0]}
+    ps = list(I.DECODE_THRESHOLDS) + [0.0] if args.decode_p is None else [args.decode_p]
+    configs = [(f"p={p:g}" if p > 0 else "p=0 (no eviction, supplementary)", p, x["a_k"], bfinal, tok)
+               for p in ps]
+    if retained:
+        tok_r = dict(tok)
+        tok_r["a_k"] = torch.from_numpy(np.stack([I.make_decode_token(wr, s)["a_k"] for s in range(steps)])).to(
+            "cuda").to(torch.float32).contiguous()
+        configs.append((f"p={I.DECODE_RETAINED_P:g}, retention-matched (supplementary)", I.DECODE_RETAINED_P,
+                        ak_r, bfinal_r, tok_r))
     res = {}
     cap = T0 + steps + 1
     entry_bytes = 3 * w.d * 2 + 12
-    for p in (list(I.DECODE_THRESHOLDS) + [0.0] if args.decode_p is None else [args.decode_p]):
+    for key, p, ak, bf, tk in configs:
         cache = ua.Cache.empty(w.B, w.Hkv, w.d, cap, torch.bfloat16)
-        ua.cache_fill(cache, x["k"], x["v"], x["a_k"], bfinal, theta=w.theta)
+        ua.cache_fill(cache, x["k"], x["v"], ak, bf, theta=w.theta)
         ua.cache_compact(cache, p)
         snap = {n: getattr(cache, n).clone() for n in ("khat", "krope", "v", "bias", "rk", "pos", "n_kept")}
         n0 = cache.n_kept.clone()
@@ -358,15 +380,15 @@ def bench_decode(args, peaks, peaks_kind):
 
         def run_all(stream=None):
             for s in range(steps):
-                ua.decode_step(cache, tok["q"][s], tok["k"][s], tok["v"][s], tok["g"][s], tok["a_q"][s],
-                               tok["a_k"][s], x["alpha"], x["beta"], T0 + s, p, scale=w.scale, theta=w.theta,
+                ua.decode_step(cache, tk["q"][s], tk["k"][s], tk["v"][s], tk["g"][s], tk["a_q"][s],
+                               tk["a_k"][s], x["alpha"], x["beta"], T0 + s, p, scale=w.scale, theta=w.theta,
                                out=o[s], stream=stream)
 
         # kept counts per step (for the byte count): one eager pass
         counts = [n0.sum().item()]
         for s in range(steps):
-            ua.decode_step(cache, tok["q"][s], tok["k"][s], tok["v"][s], tok["g"][s], tok["a_q"][s],
-                           tok["a_k"][s], x["alpha"], x["beta"], T0 + s, p, scale=w.scale, theta=w.theta,
+            ua.decode_step(cache, tk["q"][s], tk["k"][s], tk["v"][s], tk["g"][s], tk["a_q"][s],
+                           tk["a_k"][s], x["alpha"], x["beta"], T0 + s, p, scale=w.scale, theta=w.theta,
                            out=o[s])
             counts.append(cache.n_kept.sum().item())
         assert ua.get_device_status() == 0
@@ -400,15 +422,16 @@ def bench_decode(args, peaks, peaks_kind):
         bytes_total = sum(counts[s] * entry_bytes + counts[s + 1] * 4 + w.B * w.Hkv * entry_bytes + tok_bytes
                           for s in range(steps))
         gbs = bytes_total / (ms * 1e-3) / 1e9
-        retained = final_kept / (w.B * w.Hkv * (T0 + steps))
-        key = f"p={p:g}" if p > 0 else "p=0 (no eviction, supplementary)"
+        kept_frac = final_kept / (w.B * w.Hkv * (T0 + steps))
         res[key] = {"tokens_per_s": w.B * steps / (ms * 1e-3), "ms_per_256_steps": ms,
                     "us_per_step": 1e3 * ms / steps, "hbm_gbs": gbs,
                     "hbm_frac": gbs / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
-                    "retained_fraction": retained, "kept_entries_after": final_kept,
+                    "retained_fraction": kept_frac, "kept_entries_after": final_kept,
                     "mean_kept_per_head": float(np.mean(counts)) / (w.B * w.Hkv),
                     "cache_MB_after": final_kept * entry_bytes / 1e6,
-                    "compression_x": 1.0 / retained if retained > 0 else None}
+                    "compression_x": 1.0 / kept_frac if kept_frac > 0 else None}
+        if ak is not x["a_k"]:
+            res[key]["ak_slow_mean"] = I.DECODE_RETAINED_AK_SLOW_MEAN
         del g, cache, snap
         torch.cuda.empty_cache()
     res["peak_source"] = f"{peaks_kind} HBM copy bandwidth"
