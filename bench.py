@@ -127,6 +127,19 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- oracle (CPU)
 
+def cpu_model() -> str:
+    """The host CPU's model name (for the CPU-baseline record)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 def oracle_sample(w, n_units: int, nthreads: int):
     """Time the fp64 oracle on n_units (batch, KV-head) units of workload w at full T, all
     rows and heads; returns (seconds, algorithmic FLOPs of the sample, description)."""
@@ -165,8 +178,8 @@ def run_reference(args, world, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(w),
-            "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": desc, "value": val,
-                             "unit": "TFLOP/s"},
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "cpu_model": cpu_model(), "sample": desc,
+                             "value": val, "unit": "TFLOP/s"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -519,8 +532,8 @@ def main():
     if not args.no_cpu and rank == 0 and world == 1:
         cores = os.cpu_count() or 1
         dt, fl, desc = oracle_sample(w, cores, cores)
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
-               "seconds": dt}
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
+               "sample": desc, "seconds": dt}
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
