@@ -532,8 +532,10 @@ def main():
     if not args.no_cpu and rank == 0 and world == 1:
         cores = os.cpu_count() or 1
         dt, fl, desc = oracle_sample(w, cores, cores)
+        dt1, fl1, desc1 = oracle_sample(w, 1, 1)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
-               "sample": desc, "seconds": dt}
+               "sample": desc, "seconds": dt,
+               "single_core": {"value": fl1 / dt1 / 1e12, "unit": "TFLOP/s", "sample": desc1, "seconds": dt1}}
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
