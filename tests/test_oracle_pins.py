@@ -381,3 +381,32 @@ def test_deferred_compaction_equals_step_by_step():
             m = eager.n[b, h]
             for name in ("k", "v", "ak", "pos", "b"):
                 np.testing.assert_array_equal(getattr(lazy, name)[b, h, :m], getattr(eager, name)[b, h, :m])
+
+
+@pytest.mark.parametrize("shift", [1, 37, 100000])
+def test_rope_relative_position_invariance(shift):
+    """RoPE makes a logit depend on the positions only through their difference: moving every
+    cached pair and the new token by the same offset leaves every decode output and bias
+    unchanged (to fp64 rounding of the rotations).  A rotation applied with opposite senses to
+    queries and keys would make the logit depend on the sum instead, and fail this."""
+    T0, n, p = 24, 8, 0.15
+    w, x = small_case(T=T0 + n, B=2, H=4, Hkv=2, d=16, seed=29)
+    pre = {k: (v[:, :T0] if v.ndim >= 2 else v) for k, v in x.items()}
+    r = oracle.prefill_fwd(**pre)
+    caches = []
+    for _ in range(2):
+        c = oracle.DecodeCache(w.B, w.Hkv, w.d, T0 + n + 1)
+        c.fill_from_prefill(pre["k"], pre["v"], pre["a_k"], r["b_final"], logp=math.log(p))
+        caches.append(c)
+    base, moved = caches
+    moved.pos += shift
+    for t in range(T0, T0 + n):
+        args = (x["q"][:, t], x["k"][:, t], x["v"][:, t], x["g"][:, t], x["a_q"][:, t], x["a_k"][:, t],
+                x["alpha"], x["beta"])
+        a = oracle.decode_step(base, *args, t, p)
+        b = oracle.decode_step(moved, *args, t + shift, p)
+        np.testing.assert_allclose(b["o"], a["o"], atol=1e-9, rtol=0)
+        np.testing.assert_array_equal(b["evict"], a["evict"])
+    np.testing.assert_array_equal(moved.n, base.n)
+    np.testing.assert_array_equal(moved.pos - shift, base.pos)
+    np.testing.assert_array_equal(moved.b, base.b)
