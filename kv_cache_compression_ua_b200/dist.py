@@ -1,8 +1,10 @@
 """Host-side plumbing for running the UA hot path on several GPUs of one node.
 
 The (batch, KV head) units are independent in prefill and decode, so ranks never exchange
-data on the hot path (weak scaling: every rank runs its own batch).  The only collectives are
-timing ones: a barrier around the timed region and the max of the per-rank times.
+data on the hot path (weak scaling: every rank runs its own batch).  The collectives are a
+barrier around the timed region, the max of the per-rank times, and, for a data-parallel
+backward, the sum of the decay parameters' gradients (the only gradients shared by the
+ranks' batches).
 """
 from __future__ import annotations
 
@@ -53,6 +55,19 @@ def max_over_ranks(x: float, world: int) -> float:
     t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def allreduce_decay_param_grads(dalpha: torch.Tensor, dbeta: torch.Tensor, world: int):
+    """Data-parallel backward: each rank's ua_prefill_bwd sums dalpha and dbeta [Hkv] over its
+    own batch; the model's gradient is their sum over the ranks, taken in place with one
+    all-reduce of 2*Hkv floats.  Every other gradient belongs to the rank's own tokens."""
+    if world == 1:
+        return
+    buf = torch.cat([dalpha.reshape(-1), dbeta.reshape(-1)])
+    torch.distributed.all_reduce(buf, op=torch.distributed.ReduceOp.SUM)
+    n = dalpha.numel()
+    dalpha.copy_(buf[:n].view_as(dalpha))
+    dbeta.copy_(buf[n:].view_as(dbeta))
 
 
 def finalize(world: int):
