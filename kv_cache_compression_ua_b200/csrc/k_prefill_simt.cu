@@ -156,8 +156,10 @@ cudaError_t launch_tile_qmax(const TileQmaxParams& p, cudaStream_t s) {
 // ------------------------------------------------------------------ boundary pass
 // grid (ceil(T/128), Hkv, B), 128 threads; thread = key j, sweeping the rows l > j in
 // order.  At every query-tile boundary l = t*bq it writes the prefix sum so far.
-template <int DH>
+// VAR: an ablation variant is set (without it the variant is the constant 0 and folds away).
+template <int DH, bool VAR>
 __global__ void __launch_bounds__(128) k_boundary_simt(BoundaryParams p) {
+    const int variant = VAR ? p.variant : 0;
     constexpr int RC = 32;
     __shared__ float s_k[RC][DH];
     __shared__ float s_rq[RC];
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(128) k_boundary_simt(BoundaryParams p) {
                 float s = 0.f;
 #pragma unroll
                 for (int c = 0; c < DH; ++c) s = fmaf(s_k[r][c], kj[c], s);
-                acc += decay_var(s_rq[r], rkj, fmaf(al, s, be), p.variant);
+                acc += decay_var(s_rq[r], rkj, fmaf(al, s, be), variant);
             }
         }
     }
@@ -204,8 +206,12 @@ __global__ void __launch_bounds__(128) k_boundary_simt(BoundaryParams p) {
 // grid (nqt, H, B), 256 threads = 16 x 16; 64 query rows x 64 keys per tile.  Thread
 // (ty, tx) owns rows ty + 16*rr and columns tx + 16*cc (rr, cc < 4), which keeps the
 // padded shared-memory reads conflict-free.
-template <int DH, typename TI>
+// FULL: an ablation variant or the chunked pruning is on.  Without it both fold away at
+// compile time, so the method's own forward carries neither branch.
+template <int DH, typename TI, bool FULL>
 __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
+    const int variant = FULL ? p.variant : 0;
+    const float prune_thr = FULL ? p.prune_thr : INFINITY;
     constexpr int BM = 64, BN = 64, LD = DH + 1, LP = BN + 1, ND = DH / 16;
     extern __shared__ float sm[];
     float* sQ = sm;
@@ -254,13 +260,13 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
     const int qchunk = qt & ~1;
     for (int kt = 0; kt <= qt; ++kt) {
         const int j0 = kt * BN;
-        const bool pruned_tile = kt < qchunk && p.prune_thr < INFINITY;
+        const bool pruned_tile = FULL && kt < qchunk && prune_thr < INFINITY;
         __syncthreads();
         for (int c = tid; c < BN; c += 256) {
             const int j = j0 + c;
             sRk[c] = j < T ? p.rk[unit * T + j] : 0.f;
             sPb[c] = j < T ? p.pb[(unit * p.nqt + qt) * T + j] : 0.f;
-            sEv[c] = (pruned_tile && j < T && p.pb[(unit * p.nqt + qchunk) * T + j] > p.prune_thr) ? 1.f : 0.f;
+            sEv[c] = (pruned_tile && j < T && p.pb[(unit * p.nqt + qchunk) * T + j] > prune_thr) ? 1.f : 0.f;
         }
         // skip when every key underflows, or (no debug Lambda to write) every key is evicted;
         // thread tid < BN votes on the entries it wrote itself
@@ -300,7 +306,7 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
                     const int r = ty + 16 * rr, c = tx + 16 * cc;
                     const int i = i0 + r, j = j0 + c;
                     float D = 0.f;
-                    if (i > j && i < T && j < T) D = decay_var(sRq[r], sRk[c], fmaf(al, s[rr][cc], be), p.variant);
+                    if (i > j && i < T && j < T) D = decay_var(sRq[r], sRk[c], fmaf(al, s[rr][cc], be), variant);
                     sL[r * LP + c] = D;
                 }
         }
@@ -340,7 +346,7 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
                 const float lam = sL[r * LP + c];
                 if (write_lambda && i < T && j < T)
                     p.lambda_dbg[(unit * T + i) * (size_t)T + j] = (j <= i) ? lam : 0.f;
-                sc[rr][cc] = (j <= i && j < T && sEv[c] == 0.f) ? fmaf(p.scale, sc[rr][cc], lam) : -INFINITY;
+                sc[rr][cc] = (j <= i && j < T && (!FULL || sEv[c] == 0.f)) ? fmaf(p.scale, sc[rr][cc], lam) : -INFINITY;
                 mx = fmaxf(mx, sc[rr][cc]);
             }
 #pragma unroll
@@ -413,21 +419,33 @@ cudaError_t launch_prep(const PrepParams& p, bool bf16_in, bool bf16_work, cudaS
 cudaError_t launch_boundary_simt(const BoundaryParams& p, cudaStream_t s) {
     dim3 grid((p.T + 127) / 128, p.Hkv, p.B);
     UA_PROFILE("k_boundary_simt", s);
-    if (p.d == 64) k_boundary_simt<64><<<grid, 128, 0, s>>>(p);
-    else k_boundary_simt<128><<<grid, 128, 0, s>>>(p);
+    if (p.variant != 0) {
+        if (p.d == 64) k_boundary_simt<64, true><<<grid, 128, 0, s>>>(p);
+        else k_boundary_simt<128, true><<<grid, 128, 0, s>>>(p);
+    } else {
+        if (p.d == 64) k_boundary_simt<64, false><<<grid, 128, 0, s>>>(p);
+        else k_boundary_simt<128, false><<<grid, 128, 0, s>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+template <int DH, typename TI, bool FULL>
+static cudaError_t fwd_simt_launch(const FwdParams& p, cudaStream_t s) {
+    constexpr int BM = 64, BN = 64, LD = DH + 1, LP = BN + 1;
+    const size_t smem = sizeof(float) * (size_t)(2 * BM * LD + 3 * BN * LD + 2 * BM * LP + BM + 3 * BN);
+    cudaError_t e = cudaFuncSetAttribute(k_fwd_simt<DH, TI, FULL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.nqt, p.H, p.B);
+    UA_PROFILE("k_fwd_simt", s);
+    k_fwd_simt<DH, TI, FULL><<<grid, 256, smem, s>>>(p);
     return cudaGetLastError();
 }
 
 template <int DH, typename TI>
 static cudaError_t fwd_simt_inst(const FwdParams& p, cudaStream_t s) {
-    constexpr int BM = 64, BN = 64, LD = DH + 1, LP = BN + 1;
-    const size_t smem = sizeof(float) * (size_t)(2 * BM * LD + 3 * BN * LD + 2 * BM * LP + BM + 3 * BN);
-    cudaError_t e = cudaFuncSetAttribute(k_fwd_simt<DH, TI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(p.nqt, p.H, p.B);
-    UA_PROFILE("k_fwd_simt", s);
-    k_fwd_simt<DH, TI><<<grid, 256, smem, s>>>(p);
-    return cudaGetLastError();
+    const bool full = p.variant != 0 || p.prune_thr < INFINITY;
+    return full ? fwd_simt_launch<DH, TI, true>(p, s) : fwd_simt_launch<DH, TI, false>(p, s);
 }
 
 cudaError_t launch_fwd_simt(const FwdParams& p, bool bf16_act, cudaStream_t s) {
