@@ -31,7 +31,10 @@
  *   - Tensors are dense, row-major, innermost dimension last, with the shapes written
  *     beside each argument.  "act" means the activation dtype of the call: float32 for
  *     UA_F32, bfloat16 for UA_BF16.  Decay logits and parameters are always float32.
- *   - Every pointer must be 16-byte aligned (256-byte for the workspace).
+ *   - Every pointer must be 16-byte aligned (256-byte for the workspace) and address at
+ *     least the elements its shape implies: the library cannot see a buffer's extent, so an
+ *     undersized one is read or written past its end (the Python binding checks extents and
+ *     element types before calling).
  *   - Host-detectable errors (NULL pointer, bad shape, unsupported head_dim, misaligned
  *     pointer, workspace too small) return a status before anything is launched and leave
  *     all outputs untouched.  Device-detectable errors (cache capacity exceeded) set a
