@@ -228,3 +228,22 @@ def test_binding_refuses_bad_cache_and_decode_arguments(lib):
     c.bias = torch.zeros(2, 2, 40, dtype=torch.float64)
     with pytest.raises(ValueError, match="cache.bias"):
         ua.cache_compact(c, 0.1)
+
+
+def test_binding_constants_match_the_header():
+    txt = open(os.path.join(ROOT, "include", "ua.h")).read()
+    defines = {n: int(v) for n, v in re.findall(r"#define\s+(UA_[A-Z_]+)\s+(\d+)", txt)}
+    assert defines["UA_VAR_NO_QUERY_DECAY"] == ua.VAR_NO_QUERY_DECAY
+    assert defines["UA_VAR_NO_KEY_DECAY"] == ua.VAR_NO_KEY_DECAY
+    assert defines["UA_VAR_NO_SIM_DECAY"] == ua.VAR_NO_SIM_DECAY
+    assert defines["UA_VAR_QUERY_NORM"] == ua.VAR_QUERY_NORM
+    assert defines["UA_DECODE_DEFER_COMPACT"] == ua.DECODE_DEFER_COMPACT
+    assert re.search(r"UA_F32\s*=\s*0", txt) and re.search(r"UA_BF16\s*=\s*1", txt)
+    assert (ua.UA_F32, ua.UA_BF16) == (0, 1)
+    # the shape struct's fields, in order, as the binding lays them out
+    body = re.search(r"typedef struct \{(.*?)\} ua_shape;", re.sub(r"/\*.*?\*/", "", txt, flags=re.S), re.S).group(1)
+    fields = re.findall(r"(\w+)\s*[,;]", body)
+    assert fields == [f for f, _ in ua.ua_shape._fields_], fields
+    body = re.search(r"typedef struct \{(.*?)\} ua_cache;", re.sub(r"/\*.*?\*/", "", txt, flags=re.S), re.S).group(1)
+    fields = re.findall(r"(\w+)\s*[,;]", body)
+    assert fields == [f for f, _ in ua.ua_cache._fields_], fields
