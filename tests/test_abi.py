@@ -241,9 +241,9 @@ def test_binding_constants_match_the_header():
     assert re.search(r"UA_F32\s*=\s*0", txt) and re.search(r"UA_BF16\s*=\s*1", txt)
     assert (ua.UA_F32, ua.UA_BF16) == (0, 1)
     # the shape struct's fields, in order, as the binding lays them out
-    body = re.search(r"typedef struct \{(.*?)\} ua_shape;", re.sub(r"/\*.*?\*/", "", txt, flags=re.S), re.S).group(1)
+    body = re.search(r"typedef struct \{([^{}]*)\} ua_shape;", re.sub(r"/\*.*?\*/", "", txt, flags=re.S), re.S).group(1)
     fields = re.findall(r"(\w+)\s*[,;]", body)
     assert fields == [f for f, _ in ua.ua_shape._fields_], fields
-    body = re.search(r"typedef struct \{(.*?)\} ua_cache;", re.sub(r"/\*.*?\*/", "", txt, flags=re.S), re.S).group(1)
+    body = re.search(r"typedef struct \{([^{}]*)\} ua_cache;", re.sub(r"/\*.*?\*/", "", txt, flags=re.S), re.S).group(1)
     fields = re.findall(r"(\w+)\s*[,;]", body)
     assert fields == [f for f, _ in ua.ua_cache._fields_], fields
