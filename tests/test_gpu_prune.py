@@ -37,12 +37,12 @@ def kernels_ran(fn):
     return out, set(ua.profile_read())
 
 
-def run(w, x, p, want_bfinal=True, want_lambda=False):
+def run(w, x, p, want_bfinal=True, want_lambda=False, variant=0):
     d = {n: torch.from_numpy(np.ascontiguousarray(a)).cuda().to(
         TORCH_DT[w.dtype] if n in ("q", "k", "v", "g") else torch.float32).contiguous() for n, a in x.items()}
     r = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
                        scale=w.scale, theta=w.theta, want_bfinal=want_bfinal, want_lambda=want_lambda,
-                       prune_p=p)
+                       prune_p=p, variant=variant)
     torch.cuda.synchronize()
     return {k: (None if v is None else v.float().cpu().numpy()) for k, v in r.items()}
 
@@ -69,10 +69,10 @@ def check(w, g, r, lam, p, dense_bfinal=None):
         assert_close("b_final", g["b_final"], dense_bfinal, w.dtype, relative_max=True)
 
 
-def oracle_pair(w, x, p):
+def oracle_pair(w, x, p, variant=0):
     xo = {k: v for k, v in x.items() if k != "d_o"}
-    r = oracle.prefill_fwd(**xo, scale=w.scale, theta=w.theta, prune_p=p, want_lambda=True)
-    dense = oracle.prefill_fwd(**xo, scale=w.scale, theta=w.theta)
+    r = oracle.prefill_fwd(**xo, scale=w.scale, theta=w.theta, prune_p=p, want_lambda=True, variant=variant)
+    dense = oracle.prefill_fwd(**xo, scale=w.scale, theta=w.theta, variant=variant)
     assert np.max(np.abs(dense["o"] - r["o"])) > 1e-3                  # pruning changed something
     return r, dense
 
@@ -133,4 +133,18 @@ def test_bf16_d128_runs_simt_path():
     r, dense = oracle_pair(w, x, 0.15)
     g, names = kernels_ran(lambda: run(w, x, 0.15))
     assert "k_fwd_simt" in names
+    check(w, g, r, r["lam"], 0.15, dense["b_final"])
+
+
+@pytest.mark.parametrize("dtype,variant,kernel", [("bf16", ua.VAR_QUERY_NORM, "k_fwd_tc"),
+                                                  ("f32", ua.VAR_NO_KEY_DECAY, "k_fwd_simt")])
+def test_pruning_with_a_variant(dtype, variant, kernel):
+    """The chunked pruning and an ablation variant together: the variant changes the prep and
+    the decay, the pruning acts on the resulting prefixes."""
+    w = I.Workload("prune_var", 1, 640, 8, 2, 64, dtype, 1600 + variant)
+    x = I.make_prefill_inputs(w)
+    r, dense = oracle_pair(w, x, 0.15, variant)
+    g, names = kernels_ran(lambda: run(w, x, 0.15, variant=variant))
+    assert kernel in names, names
+    assert ua.get_device_status() == 0
     check(w, g, r, r["lam"], 0.15, dense["b_final"])
