@@ -244,3 +244,33 @@ def compact_order(keep):
     order = np.zeros(len(keep), np.int64)
     n = _load().ora_compact_order(len(keep), _ptr(keep), _ptr(order))
     return order[:n]
+
+
+# ----------------------------------------------------------------------------- per-query-head decay
+# The alternative reading of which head the decay parameters belong to (per query head rather
+# than per KV head; an ablation direction of "A Self-Pruning Transformer: Extreme KV-Cache
+# Compression with Universal Attention", paperlayer.ai summary App. E): a_q, a_k [B,T,H] and
+# alpha, beta [H], every query head with its own rates and its own Lambda over its group's
+# shared keys, each head evicting for itself.  That is multi-head UA on K and V repeated over
+# the G query heads of each group, so these wrappers only repeat the keys and values (and sum
+# their gradients back over the copies); all the arithmetic is the functions above.
+
+def _repeat_kv(x, G):
+    return np.repeat(_f64(x), G, axis=2)
+
+
+def prefill_fwd_per_head(q, k, v, g, a_q, a_k, alpha, beta, **kw):
+    """Prefill forward with per-query-head decay.  a_q, a_k [B,T,H]; alpha, beta [H].
+    Returns as prefill_fwd, with b_final [B,H,T] (and lam [B,H,T,T])."""
+    G = np.shape(q)[2] // np.shape(k)[2]
+    return prefill_fwd(q, _repeat_kv(k, G), _repeat_kv(v, G), g, a_q, a_k, alpha, beta, **kw)
+
+
+def prefill_bwd_per_head(q, k, v, g, a_q, a_k, alpha, beta, d_o, **kw):
+    """Gradients of the per-query-head forward; dk, dv are summed over each group's heads."""
+    B, T, Hkv, d = np.shape(k)
+    G = np.shape(q)[2] // Hkv
+    r = prefill_bwd(q, _repeat_kv(k, G), _repeat_kv(v, G), g, a_q, a_k, alpha, beta, d_o, **kw)
+    r["dk"] = r["dk"].reshape(B, T, Hkv, G, d).sum(axis=3)
+    r["dv"] = r["dv"].reshape(B, T, Hkv, G, d).sum(axis=3)
+    return r

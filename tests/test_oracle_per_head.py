@@ -1,0 +1,88 @@
+"""Per-query-head decay in the oracle (the alternative to decay parameters per KV head).
+
+Pins: rates that are equal across the heads of a group reproduce the per-KV-head results;
+with G = 1 the two readings coincide; the gradients (dk and dv summed over the group's
+heads) equal central differences of the per-head forward; distinct per-head rates give
+distinct heads."""
+import numpy as np
+import pytest
+
+import oracle
+from kv_cache_compression_ua_b200 import inputs as I
+
+
+def case(T=24, B=2, H=4, Hkv=2, d=8, seed=3):
+    w = I.Workload("ph", B, T, H, Hkv, d, "f32", seed, with_grad=True)
+    return w, {k: v.astype(np.float64) for k, v in I.make_prefill_inputs(w).items()}
+
+
+def per_head(x, G, rng=None):
+    """Rates per query head: each KV head's repeated over its group, perturbed if rng is given."""
+    y = dict(x)
+    for n in ("a_q", "a_k"):
+        y[n] = np.repeat(x[n], G, axis=2)
+    for n in ("alpha", "beta"):
+        y[n] = np.repeat(x[n], G)
+    if rng is not None:
+        for n in ("a_q", "a_k", "alpha", "beta"):
+            y[n] = y[n] + 0.3 * rng.standard_normal(y[n].shape)
+    return y
+
+
+def test_shared_rates_reproduce_the_per_kv_head_decay():
+    w, x = case()
+    G = w.H // w.Hkv
+    xo = {k: v for k, v in x.items() if k != "d_o"}
+    ref = oracle.prefill_fwd(**xo, want_lambda=True)
+    got = oracle.prefill_fwd_per_head(**{k: v for k, v in per_head(x, G).items() if k != "d_o"}, want_lambda=True)
+    np.testing.assert_allclose(got["o"], ref["o"], atol=1e-12, rtol=0)
+    np.testing.assert_allclose(got["lse"], ref["lse"], atol=1e-12, rtol=0)
+    np.testing.assert_array_equal(got["b_final"], np.repeat(ref["b_final"], G, axis=1))
+    np.testing.assert_array_equal(got["lam"], np.repeat(ref["lam"], G, axis=1))
+
+
+def test_single_head_groups_coincide():
+    w, x = case(H=2, Hkv=2)
+    xo = {k: v for k, v in x.items() if k != "d_o"}
+    a = oracle.prefill_fwd(**xo)
+    b = oracle.prefill_fwd_per_head(**xo)
+    for n in ("o", "lse", "b_final"):
+        np.testing.assert_array_equal(a[n], b[n])
+
+
+def test_distinct_rates_give_distinct_heads():
+    w, x = case()
+    G = w.H // w.Hkv
+    y = per_head(x, G, np.random.default_rng(1))
+    r = oracle.prefill_fwd_per_head(**{k: v for k, v in y.items() if k != "d_o"})
+    s = oracle.prefill_fwd_per_head(**{k: v for k, v in per_head(x, G).items() if k != "d_o"})
+    assert np.max(np.abs(r["b_final"][:, 0] - r["b_final"][:, 1])) > 1e-3   # heads of one group differ
+    assert np.max(np.abs(r["o"] - s["o"])) > 1e-3
+
+
+def _loss(y, d_o):
+    r = oracle.prefill_fwd_per_head(**{k: v for k, v in y.items() if k != "d_o"}, nthreads=1)
+    return float(np.sum(r["o"] * d_o))
+
+
+def test_per_head_backward_matches_central_differences():
+    w, x = case(T=7, B=1, H=4, Hkv=2, d=8, seed=9)
+    G = w.H // w.Hkv
+    y = per_head(x, G, np.random.default_rng(2))
+    d_o = y["d_o"]
+    gr = oracle.prefill_bwd_per_head(**y, nthreads=1)
+    names = {"q": "dq", "k": "dk", "v": "dv", "g": "dg", "a_q": "da_q", "a_k": "da_k",
+             "alpha": "dalpha", "beta": "dbeta"}
+    for name, gname in names.items():
+        base = y[name]
+        fd = np.zeros_like(base)
+        it = np.nditer(base, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            h = 1e-6 * max(1.0, abs(base[idx]))
+            yp = dict(y); yp[name] = base.copy(); yp[name][idx] += h
+            ym = dict(y); ym[name] = base.copy(); ym[name][idx] -= h
+            fd[idx] = (_loss(yp, d_o) - _loss(ym, d_o)) / (2 * h)
+        assert gr[gname].shape == base.shape, gname
+        err = np.max(np.abs(fd - gr[gname]))
+        assert err <= 1e-6 * (1.0 + np.max(np.abs(fd))), (name, err)
