@@ -69,14 +69,43 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during a region."""
+    """SM clocks and throttle reasons sampled during a region: through NVML every 2 ms when the
+    library is there (a short timed region still gets dozens of samples), else nvidia-smi every
+    200 ms."""
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.nvml = None
+        self.stop = threading.Event()
+
+    def _nvml_loop(self):
+        import pynvml as N
+        h = N.nvmlDeviceGetHandleByIndex(self.gpu)
+        mx = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+        bits = [0x8, 0x40, 0x20, 0x4]   # hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
+        while not self.stop.is_set():
+            try:
+                sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+                r = N.nvmlDeviceGetCurrentClocksEventReasons(h) if hasattr(
+                    N, "nvmlDeviceGetCurrentClocksEventReasons") else N.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                flags = ["Active" if r & b else "Not Active" for b in bits]
+                self.lines.append(", ".join([str(sm), str(mx), "0"] + flags))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = threading.Thread(target=self._nvml_loop, daemon=True)
+            self.nvml.start()
+            time.sleep(0.02)
+            return self
+        except Exception:
+            self.nvml = None
         q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
              "clocks_event_reasons.sw_power_cap")
@@ -96,6 +125,11 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *a):
+        if self.nvml is not None:
+            time.sleep(0.01)
+            self.stop.set()
+            self.nvml.join(timeout=5)
+            return
         if self.proc is not None:
             time.sleep(0.25)
             self.proc.terminate()
@@ -122,7 +156,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvml, 2 ms" if self.nvml is not None else "nvidia-smi, 200 ms"}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)
@@ -211,7 +245,7 @@ def bench_prefill(args, world, rank, local, peaks, peaks_kind):
         # the whole forward contract: O, the row normalisers (for a backward) and b_final (the
         # initial biases of the self-pruning cache)
         ua.prefill_fwd(x["q"], x["k"], x["v"], x["g"], x["a_q"], x["a_k"], x["alpha"], x["beta"],
-                       scale=w.scale, theta=w.theta, out=out, ws=ws)
+                       scale=w.scale, theta=w.theta, out=out, lse=lse, b_final=bfin, ws=ws)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -279,18 +313,22 @@ def bench_prefill(args, world, rank, local, peaks, peaks_kind):
 
 def bench_e2e(args, w, x):
     """Public API with host buffers: every step copies its inputs in from pinned host memory,
-    runs the prefill and copies O out.  Steps are pipelined the way a serving loop would run
+    runs the prefill and copies its outputs (O, lse, b_final) out.  Steps are pipelined the way a serving loop would run
     them: two device buffer sets and three streams (copy in, compute, copy out), so step n's
     inputs travel while step n-1 computes and step n-2's output travels back."""
     from kv_cache_compression_ua_b200 import ua
     host = {n: t.cpu().pin_memory() for n, t in x.items()}
     dev = [{n: torch.empty_like(t) for n, t in x.items()} for _ in range(2)]
     out = [torch.empty_like(x["q"]) for _ in range(2)]
+    lse = [torch.empty(w.B, w.H, w.T, dtype=torch.float32, device="cuda") for _ in range(2)]
+    bfin = [torch.empty(w.B, w.Hkv, w.T, dtype=torch.float32, device="cuda") for _ in range(2)]
     o_host = [torch.empty(x["q"].shape, dtype=x["q"].dtype).pin_memory() for _ in range(2)]
+    lse_host = [torch.empty(lse[0].shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    bfin_host = [torch.empty(bfin[0].shape, dtype=torch.float32).pin_memory() for _ in range(2)]
     shape = ua.make_shape(x["q"], x["k"], w.scale, w.theta)
     ws = ua.alloc_workspace(ua.prefill_workspace_size(shape), "cuda")
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o_host[0].numel() * o_host[0].element_size()
+    d2h = sum(t[0].numel() * t[0].element_size() for t in (o_host, lse_host, bfin_host))
     s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()
     in_done = [ev(), ev()]      # inputs of buffer set i are on the device
@@ -311,11 +349,14 @@ def bench_e2e(args, w, x):
             s_run.wait_event(out_done[b])                # out[b] has been copied back
             d = dev[b]
             ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
-                           scale=w.scale, theta=w.theta, out=out[b], ws=ws, stream=s_run)
+                           scale=w.scale, theta=w.theta, out=out[b], lse=lse[b], b_final=bfin[b], ws=ws,
+                           stream=s_run)
             run_done[b].record(s_run)
         with torch.cuda.stream(s_out):
             s_out.wait_event(run_done[b])
             o_host[b].copy_(out[b], non_blocking=True)
+            lse_host[b].copy_(lse[b], non_blocking=True)
+            bfin_host[b].copy_(bfin[b], non_blocking=True)
             out_done[b].record(s_out)
 
     for i in range(2):
@@ -452,6 +493,76 @@ def bench_decode(args, peaks, peaks_kind):
     return res
 
 
+def time_prefill(w, x, steps, warmup, prune_p=0.0, want_bfinal=True):
+    """Device time of `steps` prefill forwards of workload w (inputs x resident in HBM), with the
+    per-kernel launch times and the tile statistics of the last call."""
+    from kv_cache_compression_ua_b200 import ua
+    out = torch.empty_like(x["q"])
+    shape = ua.make_shape(x["q"], x["k"], w.scale, w.theta, prune_p=prune_p)
+    ws = ua.alloc_workspace(ua.prefill_workspace_size(shape), "cuda")
+    lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32, device="cuda")
+    bfin = torch.empty(w.B, w.Hkv, w.T, dtype=torch.float32, device="cuda") if want_bfinal else None
+
+    def step():
+        ua.prefill_fwd(x["q"], x["k"], x["v"], x["g"], x["a_q"], x["a_k"], x["alpha"], x["beta"],
+                       scale=w.scale, theta=w.theta, out=out, lse=lse, b_final=bfin, want_bfinal=want_bfinal,
+                       ws=ws, prune_p=prune_p)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ua.profile_reset()
+    ua.profile_enable(True)
+    ev0.record()
+    for _ in range(steps):
+        step()
+    ev1.record()
+    torch.cuda.synchronize()
+    ua.profile_enable(False)
+    prof = ua.profile_read()
+    tiles, skipped = ua.prefill_tile_stats(shape, ws)
+    assert ua.get_device_status() == 0
+    return ev0.elapsed_time(ev1) / steps, prof, tiles, skipped
+
+
+def bench_prefill_more(args, peaks, peaks_kind, mhz):
+    """The other prefill configurations: the 16k-token long-context prefill (B=1, bimodal a_k,
+    b_final emitted) and the chunked pruned prefill of the 1B workload at p = 0.05 and 0.15
+    (128-token chunks), each with the roofline of its fused kernel."""
+    res = {}
+    peak_t = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_a = MUFU_PER_CLK_SM * N_SM * (mhz or 1965.0) * 1e6 / 1e9
+    cases = [("prefill_1b_16k", 0.0)] + [("prefill_1b", p) for p in I.DECODE_THRESHOLDS]
+    for wname, p in cases:
+        w = I.WORKLOADS[wname]
+        x = I.make_prefill_inputs_torch(w, "cuda")
+        steps = max(10, min(args.steps, 50))
+        ms, prof, tiles, skipped = time_prefill(w, x, steps, 3, prune_p=p)
+        F = fwd_flops(w)
+        G = w.H // w.Hkv
+        entry = {"workload": f"{wname}: B={w.B} T={w.T} H={w.H} Hkv={w.Hkv} d={w.d} bf16"
+                             + (f", chunked pruned prefill p={p:g} (128-token chunks)" if p > 0 else ""),
+                 "ms_per_step": ms, "tflops_dense_equiv": F / (ms * 1e-3) / 1e12,
+                 "tokens_per_s": w.B * w.T / (ms * 1e-3), "steps": steps,
+                 "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / v[0]} for k, v in prof.items()},
+                 "tiles": {"causal": tiles, "softmax_skipped": skipped}}
+        if "k_fwd_tc" in prof:
+            kms = prof["k_fwd_tc"][1] / prof["k_fwd_tc"][0]
+            f_exec = F - skipped * 128 * 128 * G * 4 * w.d
+            ops = mufu_ops(w) - skipped * 128 * 128 * G
+            entry["roofline"] = {
+                "kernel": "k_fwd_tc", "bound": "alu", "per_launch_ms": kms,
+                "achieved": ops / (kms * 1e-3) / 1e9, "peak": peak_a, "unit": "Gop/s (exp2/log2)",
+                "frac": ops / (kms * 1e-3) / 1e9 / peak_a,
+                "tensor": {"achieved": f_exec / (kms * 1e-3) / 1e12, "peak": peak_t, "unit": "TFLOP/s",
+                           "frac": f_exec / (kms * 1e-3) / 1e12 / peak_t,
+                           "dense_equiv_frac": F / (kms * 1e-3) / 1e12 / peak_t}}
+        res[f"{wname}" + (f"_pruned_p{p:g}" if p > 0 else "")] = entry
+        del x
+        torch.cuda.empty_cache()
+    return res
+
+
 def bwd_flops(w) -> float:
     """Algorithmic backward FLOPs, counted once: per causal pair and batch, H*10d (the S, dP,
     dV, dK and dQ products of every query head) plus Hkv*6d (the key-key similarity, and its
@@ -496,13 +607,14 @@ def bench_fwdbwd(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_1b")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-more", action="store_true", help="skip the 16k and chunked-pruned prefill lines")
     ap.add_argument("--decode-p", type=float, default=None, help="run the decode section at this p only")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -524,6 +636,9 @@ def main():
     decode = None
     if not args.no_decode and world == 1:
         decode = bench_decode(args, peaks, peaks_kind)
+    more = None
+    if not args.no_more and world == 1:
+        more = bench_prefill_more(args, peaks, peaks_kind, clocks.get("sm_mhz"))
     fwdbwd = None
     if not args.no_bwd and world == 1:
         torch.cuda.empty_cache()
@@ -541,8 +656,8 @@ def main():
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": workload_config(w), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches, "clocks": clocks, "kernels": kernels, "decode": decode,
-                "fwdbwd_3b": fwdbwd}
+                "gpu_launches": launches, "clocks": clocks, "kernels": kernels, "prefill_more": more,
+                "decode": decode, "fwdbwd_3b": fwdbwd}
         print(json.dumps(line), flush=True)
     dist.finalize(world)
 

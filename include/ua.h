@@ -265,6 +265,18 @@ ua_status ua_decode_step(const ua_cache* cache, int H, const void* q, const void
  * (0 = no error, else a ua_status code) in *code, and clears it. */
 ua_status ua_get_device_status(void* stream, int* code);
 
+/* ------------------------------------------------------------------ bounded waits
+ * No counterpart on the pages: a robustness aid.  Every device-side wait of the tensor-core
+ * kernels (an mbarrier phase, another CTA's published decay prefix) gives up after a limit of
+ * %globaltimer nanoseconds, records UA_ERR_TIMEOUT in the device status word and tears the CTA
+ * down (abort flag, a 10 ms pause for copies in flight, TMEM freed), so a stuck wait can never
+ * hang the GPU.  ua_set_wait_limit_ns sets that limit on the current device (synchronously, for
+ * every later launch; UA_WAIT_LIMIT_DEFAULT_NS = 2 s, far above any legitimate wait).  A limit
+ * of 0 makes every wait that has to spin give up at its first check: that exercises the timeout
+ * path, after which the outputs of the call are unspecified; restore the default afterwards. */
+#define UA_WAIT_LIMIT_DEFAULT_NS 2000000000ull
+ua_status ua_set_wait_limit_ns(unsigned long long ns);
+
 /* ------------------------------------------------------------------ kernel timing
  * Optional tracing for measurement: while enabled, every libua kernel launch is bracketed
  * by two CUDA events recorded on its stream (about a microsecond of overhead per launch; at

@@ -235,7 +235,7 @@ __device__ __forceinline__ bool wait_counter(const unsigned* f, unsigned target,
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
         if (__all_sync(0xffffffffu, v >= target)) return true;
         if ((it & 63u) == 63u) {
-            const bool stop = __shfl_sync(0xffffffffu, (int)(*abort != 0 || globaltimer() - t0 > kWaitLimitNs), 0);
+            const bool stop = __shfl_sync(0xffffffffu, (int)(*abort != 0 || globaltimer() - t0 > wait_limit_ns()), 0);
             if (stop) {
                 if (lane == 0 && !*abort) {
                     raise_status(UA_ERR_TIMEOUT);

@@ -2,9 +2,9 @@
 // bounded waits, TMA tile loads, tcgen05 (TMEM allocation, UMMA issue/commit, TMEM loads),
 // shared-memory matrix descriptors, and fast exp2/log2.
 //
-// Every wait is bounded by a wall-clock limit read from %globaltimer; on expiry the waiter
-// records UA_ERR_TIMEOUT in the device status word and sets the CTA's abort flag, and all
-// roles leave their loops, drain and release TMEM instead of hanging.
+// Every wait is bounded by a wall-clock limit read from %globaltimer (2 s by default); on
+// expiry the waiter records UA_ERR_TIMEOUT in the device status word and sets the CTA's abort
+// flag, and all roles leave their loops, drain and release TMEM instead of hanging.
 #pragma once
 
 #include <cuda.h>
@@ -15,7 +15,11 @@
 namespace ua {
 namespace tc {
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: far above any legitimate wait
+// Current wait limit (2 s unless a caller lowered it to exercise the timeout path); read only on
+// the slow path of a wait, after it has already spun.
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+    return *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -74,7 +78,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         if (mbar_try(bar, parity)) return true;
         if ((it & 255u) == 0) {
             if (*abort) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
+            if (globaltimer() - t0 > wait_limit_ns()) {
                 raise_status(UA_ERR_TIMEOUT);
                 *abort = 1;
                 return false;

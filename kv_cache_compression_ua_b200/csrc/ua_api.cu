@@ -10,6 +10,7 @@
 
 namespace ua {
 __device__ int g_status = 0;
+__device__ unsigned long long g_wait_limit_ns = UA_WAIT_LIMIT_DEFAULT_NS;
 }
 
 using namespace ua;
@@ -479,6 +480,12 @@ ua_status ua_prefill_tile_stats(const ua_shape* s, const void* ws, size_t ws_byt
     if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
     if (e != cudaSuccess) return UA_ERR_CUDA;
     *skipped = host;
+    return UA_OK;
+}
+
+ua_status ua_set_wait_limit_ns(unsigned long long ns) {
+    // synchronous copy to the current device's symbol: every later launch sees the new limit
+    if (cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns)) != cudaSuccess) return UA_ERR_CUDA;
     return UA_OK;
 }
 

@@ -15,6 +15,10 @@ extern __device__ int g_status;
 
 __device__ __forceinline__ void raise_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// Limit of every bounded device-side wait, in ns of %globaltimer (ua_set_wait_limit_ns; default
+// UA_WAIT_LIMIT_DEFAULT_NS).  Defined in ua_api.cu.
+extern __device__ unsigned long long g_wait_limit_ns;
+
 // ------------------------------------------------------------------ scalar math
 // softplus(x) = log(1 + e^x) in its overflow-free form.
 __device__ __forceinline__ float softplus_f(float x) {

@@ -7,6 +7,7 @@ is missing or a CUDA device is absent, the first call raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from dataclasses import dataclass
@@ -49,7 +50,8 @@ class ua_cache(ctypes.Structure):
 EXPORTS = ("ua_prefill_workspace_size", "ua_prefill_fwd", "ua_prefill_bwd_workspace_size", "ua_prefill_bwd",
            "ua_cache_fill", "ua_cache_compact", "ua_decode_step", "ua_get_device_status",
            "ua_profile_enable", "ua_profile_reset", "ua_profile_read", "ua_status_string", "ua_version",
-           "ua_prefill_fwd_noalloc", "ua_prefill_noalloc_max_scratch", "ua_prefill_tile_stats")
+           "ua_prefill_fwd_noalloc", "ua_prefill_noalloc_max_scratch", "ua_prefill_tile_stats",
+           "ua_set_wait_limit_ns")
 
 
 class ua_kernel_time(ctypes.Structure):
@@ -86,6 +88,7 @@ def load_library(path: str = LIB_PATH):
     lib.ua_prefill_tile_stats.argtypes = [SP, P, S, ctypes.POINTER(ctypes.c_ulonglong),
                                           ctypes.POINTER(ctypes.c_ulonglong), P]
     lib.ua_prefill_noalloc_max_scratch.restype = S
+    lib.ua_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     lib.ua_status_string.argtypes = [I]
     lib.ua_status_string.restype = ctypes.c_char_p
     lib.ua_version.argtypes = []
@@ -110,6 +113,20 @@ def _ptr(t):
     if not t.is_contiguous():
         raise ValueError("libua takes contiguous tensors")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _same_device(dev, **tensors):
+    """Every tensor of a call must live on the device the call runs on: the library launches on
+    the current device, so a tensor elsewhere would be reached through peer memory or not at all."""
+    for name, t in tensors.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name}: on {t.device}, the call runs on {dev}")
+
+
+def _on(dev):
+    """Make `dev` current for the call (the library resolves per-device state on the current device).
+    A tensor off the GPU is refused by _ptr inside the block."""
+    return torch.cuda.device(dev) if dev.type == "cuda" else contextlib.nullcontext()
 
 
 F32 = (torch.float32,)
@@ -147,6 +164,7 @@ def _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out):
     _need("alpha", alpha, Hkv, F32)
     _need("beta", beta, Hkv, F32)
     _need("out", out, B * T * H * d, act)
+    _same_device(q.device, k=k, v=v, g=g, a_q=a_q, a_k=a_k, alpha=alpha, beta=beta, out=out)
     return B, T, H, Hkv, d
 
 
@@ -182,23 +200,33 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0, want_lse=True,
-                want_bfinal=True, want_lambda=False, out=None, ws=None, variant=0, prune_p=0.0, stream=None):
-    """ua_prefill_fwd (variant: VAR_* bits; prune_p > 0: chunked pruned prefill).  Returns
-    dict(o, lse, b_final, lam) (absent outputs are None)."""
+                want_bfinal=True, want_lambda=False, out=None, lse=None, b_final=None, ws=None, variant=0,
+                prune_p=0.0, stream=None):
+    """ua_prefill_fwd (variant: VAR_* bits; prune_p > 0: chunked pruned prefill).  out, lse and
+    b_final may be given as preallocated outputs.  Returns dict(o, lse, b_final, lam) (absent
+    outputs are None)."""
     lib = load_library()
     B, T, H, Hkv, d = _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out)
+    _need("lse", lse, B * H * T, F32)
+    _need("b_final", b_final, B * Hkv * T, F32)
     shape = make_shape(q, k, scale, theta, variant, prune_p)
     dev = q.device
+    _same_device(dev, lse=lse, b_final=b_final)
     o = out if out is not None else torch.empty_like(q)
-    lse = torch.empty(B, H, T, dtype=torch.float32, device=dev) if want_lse else None
-    bfin = torch.empty(B, Hkv, T, dtype=torch.float32, device=dev) if want_bfinal else None
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, T, dtype=torch.float32, device=dev)
+    if b_final is None and want_bfinal:
+        b_final = torch.empty(B, Hkv, T, dtype=torch.float32, device=dev)
+    bfin = b_final
     lam = torch.empty(B, Hkv, T, T, dtype=torch.float32, device=dev) if want_lambda else None
     need = prefill_workspace_size(shape)
     if ws is None or _nbytes(ws) < need:
         ws = alloc_workspace(need, dev)
-    rc = lib.ua_prefill_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
-                            _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(bfin), _ptr(lam),
-                            _ptr(ws), ctypes.c_size_t(_nbytes(ws)), _stream(stream))
+    _same_device(dev, ws=ws)
+    with _on(dev):
+        rc = lib.ua_prefill_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
+                                _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(bfin), _ptr(lam),
+                                _ptr(ws), ctypes.c_size_t(_nbytes(ws)), _stream(stream))
     _check("ua_prefill_fwd", rc)
     return {"o": o, "lse": lse, "b_final": bfin, "lam": lam}
 
@@ -223,9 +251,10 @@ def prefill_fwd_noalloc(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=
     o = out if out is not None else torch.empty_like(q)
     lse = torch.empty(B, H, T, dtype=torch.float32, device=dev) if want_lse else None
     bfin = torch.empty(B, Hkv, T, dtype=torch.float32, device=dev) if want_bfinal else None
-    rc = lib.ua_prefill_fwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q),
-                                    _ptr(a_k), _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(bfin),
-                                    _stream(stream))
+    with _on(dev):   # the library's scratch array is resolved on the current device
+        rc = lib.ua_prefill_fwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q),
+                                        _ptr(a_k), _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(bfin),
+                                        _stream(stream))
     _check("ua_prefill_fwd_noalloc", rc)
     return {"o": o, "lse": lse, "b_final": bfin}
 
@@ -255,11 +284,13 @@ def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, d_o, *, scal
     need = prefill_bwd_workspace_size(shape)
     if ws is None or _nbytes(ws) < need:
         ws = alloc_workspace(need, dev)
-    rc = lib.ua_prefill_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
-                            _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(b_final), _ptr(d_o),
-                            _ptr(gr["dq"]), _ptr(gr["dk"]), _ptr(gr["dv"]), _ptr(gr["dg"]), _ptr(gr["da_q"]),
-                            _ptr(gr["da_k"]), _ptr(gr["dalpha"]), _ptr(gr["dbeta"]), _ptr(ws),
-                            ctypes.c_size_t(_nbytes(ws)), _stream(stream))
+    _same_device(dev, o=o, lse=lse, b_final=b_final, d_o=d_o, ws=ws)
+    with _on(dev):
+        rc = lib.ua_prefill_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
+                                _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(b_final), _ptr(d_o),
+                                _ptr(gr["dq"]), _ptr(gr["dk"]), _ptr(gr["dv"]), _ptr(gr["dg"]), _ptr(gr["da_q"]),
+                                _ptr(gr["da_k"]), _ptr(gr["dalpha"]), _ptr(gr["dbeta"]), _ptr(ws),
+                                ctypes.c_size_t(_nbytes(ws)), _stream(stream))
     _check("ua_prefill_bwd", rc)
     return gr
 
@@ -300,9 +331,11 @@ class Cache:
         _need("cache.rk", self.rk, n, F32)
         _need("cache.pos", self.pos, n, I32)
         _need("cache.n_kept", self.n_kept, self.B * self.Hkv, I32)
-        return ua_cache(self.B, self.Hkv, self.d, self.capacity, _dtype_code(self.dtype),
-                        self.khat.data_ptr(), self.krope.data_ptr(), self.v.data_ptr(), self.bias.data_ptr(),
-                        self.rk.data_ptr(), self.pos.data_ptr(), self.n_kept.data_ptr())
+        names = ("khat", "krope", "v", "bias", "rk", "pos", "n_kept")
+        dev = self.khat.device
+        _same_device(dev, **{f"cache.{n}": getattr(self, n) for n in names})
+        ptrs = [_ptr(getattr(self, n)).value for n in names]
+        return ua_cache(self.B, self.Hkv, self.d, self.capacity, _dtype_code(self.dtype), *ptrs)
 
     def nbytes_per_entry(self) -> int:
         return 3 * self.d * self.khat.element_size() + 12
@@ -318,8 +351,11 @@ def cache_fill(cache: Cache, k, v, a_k, b_final, *, theta=500000.0, stream=None)
     _need("a_k", a_k, n, F32)
     _need("b_final", b_final, n, F32)
     c = cache.struct()
-    _check("ua_cache_fill", load_library().ua_cache_fill(ctypes.byref(c), T, _ptr(k), _ptr(v), _ptr(a_k),
-                                                         _ptr(b_final), float(theta), _stream(stream)))
+    dev = cache.khat.device
+    _same_device(dev, k=k, v=v, a_k=a_k, b_final=b_final)
+    with _on(dev):
+        _check("ua_cache_fill", load_library().ua_cache_fill(ctypes.byref(c), T, _ptr(k), _ptr(v), _ptr(a_k),
+                                                             _ptr(b_final), float(theta), _stream(stream)))
 
 
 def cache_compact(cache: Cache, p: float = 0.0, keep=None, kept_idx=None, stream=None):
@@ -327,8 +363,11 @@ def cache_compact(cache: Cache, p: float = 0.0, keep=None, kept_idx=None, stream
     _need("keep", keep, n, MASK)
     _need("kept_idx", kept_idx, n, I32)
     c = cache.struct()
-    _check("ua_cache_compact", load_library().ua_cache_compact(ctypes.byref(c), _ptr(keep), float(p),
-                                                               _ptr(kept_idx), _stream(stream)))
+    dev = cache.khat.device
+    _same_device(dev, keep=keep, kept_idx=kept_idx)
+    with _on(dev):
+        _check("ua_cache_compact", load_library().ua_cache_compact(ctypes.byref(c), _ptr(keep), float(p),
+                                                                   _ptr(kept_idx), _stream(stream)))
 
 
 def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: float, *, scale=None,
@@ -354,11 +393,15 @@ def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: 
     scale = float(d) ** -0.5 if scale is None else float(scale)
     o = out if out is not None else torch.empty_like(q)
     c = cache.struct()
-    rc = load_library().ua_decode_step(ctypes.byref(c), H, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q),
-                                       _ptr(a_k), _ptr(alpha), _ptr(beta), int(pos_t), float(p), scale,
-                                       float(theta), _ptr(o), _ptr(evict_bits), _ptr(kept_idx),
-                                       int(variant) | (DECODE_DEFER_COMPACT if defer_compact else 0),
-                                       _stream(stream))
+    dev = cache.khat.device
+    _same_device(dev, q=q, k=k, v=v, g=g, a_q=a_q, a_k=a_k, alpha=alpha, beta=beta, out=o,
+                 evict_bits=evict_bits, kept_idx=kept_idx)
+    with _on(dev):
+        rc = load_library().ua_decode_step(ctypes.byref(c), H, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q),
+                                           _ptr(a_k), _ptr(alpha), _ptr(beta), int(pos_t), float(p), scale,
+                                           float(theta), _ptr(o), _ptr(evict_bits), _ptr(kept_idx),
+                                           int(variant) | (DECODE_DEFER_COMPACT if defer_compact else 0),
+                                           _stream(stream))
     _check("ua_decode_step", rc)
     return o
 
@@ -367,6 +410,14 @@ def get_device_status(stream=None) -> int:
     code = ctypes.c_int(0)
     _check("ua_get_device_status", load_library().ua_get_device_status(_stream(stream), ctypes.byref(code)))
     return code.value
+
+
+WAIT_LIMIT_DEFAULT_NS = 2_000_000_000
+
+
+def set_wait_limit_ns(ns: int):
+    """ua_set_wait_limit_ns: limit of every bounded device-side wait on the current device."""
+    _check("ua_set_wait_limit_ns", load_library().ua_set_wait_limit_ns(int(ns)))
 
 
 def profile_enable(on: bool = True):

@@ -230,6 +230,23 @@ def test_binding_refuses_bad_cache_and_decode_arguments(lib):
         ua.cache_compact(c, 0.1)
 
 
+def test_binding_refuses_cache_tensors_it_cannot_pass_as_device_pointers(lib):
+    # every cache field goes through the same device / contiguity check as the other arguments
+    c = ua.Cache.empty(2, 2, 64, 40, torch.bfloat16, device="cpu")
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        c.struct()
+    # a field on another device than the rest of the cache (meta stands in for a second GPU)
+    c.rk = torch.zeros(2, 2, 40, dtype=torch.float32, device="meta")
+    with pytest.raises(ValueError, match="cache.rk: on meta"):
+        c.struct()
+
+
+def test_binding_refuses_arguments_on_another_device(lib):
+    a = _prefill_args()
+    with pytest.raises(ValueError, match="v: on meta"):
+        ua.prefill_fwd(a["q"], a["k"], a["v"].to("meta"), a["g"], a["a_q"], a["a_k"], a["alpha"], a["beta"])
+
+
 def test_binding_constants_match_the_header():
     txt = open(os.path.join(ROOT, "include", "ua.h")).read()
     defines = {n: int(v) for n, v in re.findall(r"#define\s+(UA_[A-Z_]+)\s+(\d+)", txt)}

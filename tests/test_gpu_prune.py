@@ -7,7 +7,7 @@ over the survivors and their own chunk.
 
 Eviction is a decision taken in floating point: a key whose boundary bias lies within the
 bias tolerance of log p (1e-3 on the fp32 path, 2e-2 on the bf16 tensor-core path, the
-b_final bars) may go either way, and then the rows of that chunk and KV group are not
+b_final bars, both relative to max(1, |log p|)) may go either way, and then the rows of that chunk and KV group are not
 compared.  Every other row must match; the decisions are re-taken at each boundary from the
 monotone prefix, so an in-band key touches its own chunk only."""
 import math
@@ -54,7 +54,10 @@ def compared_rows(w, lam, p):
     G = w.H // w.Hkv
     ok = np.ones((w.B, w.Hkv, w.T), bool)
     for c in range(128, w.T, 128):
-        near = np.abs(lam[:, :, c - 1, :c - 1] - math.log(p)) < BAND[w.dtype]  # [B,Hkv,c-1]
+        # the b_final bar is relative (errors against max(1, |ref|)), so at the threshold the
+        # boundary bias may be off by BAND * max(1, |log p|)
+        band = BAND[w.dtype] * max(1.0, abs(math.log(p)))
+        near = np.abs(lam[:, :, c - 1, :c - 1] - math.log(p)) < band  # [B,Hkv,c-1]
         ok[:, :, c:c + 128] &= ~near.any(axis=2)[:, :, None]
     return np.repeat(ok, G, axis=1)
 
