@@ -755,7 +755,7 @@ size_t fwd_tc_smem(int G) {
     }
 }
 
-bool fwd_tc_supported(int d, int G) { return d == 64 && G >= 1 && G <= 4; }
+bool fwd_tc_supported(int d, int G) { return (d == 64 || d == 128) && G >= 1 && G <= 4; }
 
 template <int G, bool EARLY>
 static cudaError_t fwd_tc_launch(const CUtensorMap* m, const FwdTcParams& p, cudaStream_t s) {

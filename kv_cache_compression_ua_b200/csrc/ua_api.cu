@@ -70,16 +70,21 @@ FwdWs fwd_ws_layout(const ua_shape* s) {
 
 // Workspace of the tensor-core prefill forward: bf16 rotated/normalised copies (TMA
 // sources), log2-rates and row bounds (rows padded to Tp), prefixes at 128-row query tiles.
+// head_dim 64 cuts 128-row query tiles; head_dim 128 cuts 64-row query tiles (its prefix rows
+// are then padded to whole 128-key tiles, Tpk) and counts its publications per 128-key tile.
 struct TcWs {
     size_t qr, kh, kr, lq2, lk2, mq, pb, flags, flags_bytes, total;
-    int Tp, nqt;
+    int Tp, Tpk, nqt, nkt;
 };
 
 TcWs tc_ws_layout(const ua_shape* s) {
     const size_t B = s->B, T = s->T, H = s->H, Hkv = s->Hkv, d = s->d;
     TcWs w;
     w.Tp = (int)round_up(T, 4);
-    w.nqt = (int)((T + 127) / 128);
+    const size_t bq = d == 128 ? 64 : 128;
+    w.nqt = (int)((T + bq - 1) / bq);
+    w.nkt = (int)((T + 127) / 128);
+    w.Tpk = d == 128 ? (int)round_up(T, 128) : w.Tp;
     const size_t Tp = w.Tp;
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = round_up(off + bytes, 1024); return o; };
@@ -89,8 +94,8 @@ TcWs tc_ws_layout(const ua_shape* s) {
     w.lq2 = take(B * Hkv * Tp * 4);
     w.lk2 = take(B * Hkv * Tp * 4);
     w.mq = take(B * H * Tp * 4);
-    w.pb = take(B * Hkv * (size_t)w.nqt * Tp * 4);
-    w.flags_bytes = (B * Hkv * (size_t)w.nqt * w.nqt + 4) * 4;
+    w.pb = take(B * Hkv * (size_t)w.nqt * w.Tpk * 4);
+    w.flags_bytes = (B * Hkv * (size_t)w.nqt * w.nkt + 4) * 4;
     w.flags = take(w.flags_bytes);
     w.total = off;
     return w;
@@ -98,8 +103,11 @@ TcWs tc_ws_layout(const ua_shape* s) {
 
 // The tensor-core forward evaluates the three-rate geometric mean only (its decay runs in
 // log2 units with the cube root folded in); a shape with a mechanism switched off runs SIMT.
+// The head_dim-128 kernel does not take the chunked pruned prefill (its 64-row query tiles are
+// half a pruning chunk), so such calls run SIMT too.
 bool use_tc(const ua_shape* s) {
-    return s->dtype == UA_BF16 && fwd_tc_supported(s->d, s->H / s->Hkv) && (s->variant & kVarMech) == 0;
+    return s->dtype == UA_BF16 && fwd_tc_supported(s->d, s->H / s->Hkv) && (s->variant & kVarMech) == 0 &&
+           (s->d == 64 || s->prune_p == 0.f);
 }
 
 size_t prefill_ws_bytes(const ua_shape* s) {
@@ -239,12 +247,13 @@ static ua_status prefill_fwd_tc(const ua_shape* s, const void* q, const void* k,
     // the fused forward zeroes its publication counters and ticket itself (stream-ordered)
     if ((st = cuda_status(cudaMemsetAsync(at(ws, w.flags), 0, w.flags_bytes, cs))) != UA_OK) return st;
     FwdTcLaunch L;
-    L.B = s->B; L.T = s->T; L.Tp = w.Tp; L.H = s->H; L.Hkv = s->Hkv; L.nqt = w.nqt; L.scale = s->scale;
+    L.B = s->B; L.T = s->T; L.Tp = w.Tp; L.Tpk = w.Tpk; L.H = s->H; L.Hkv = s->Hkv; L.nqt = w.nqt;
+    L.scale = s->scale;
     L.kh = pp.kh; L.kr = pp.kr; L.qr = pp.qr; L.v = v; L.lq2 = pp.lq2; L.lk2 = pp.lk2; L.mq = pp.mq;
     L.pincl = reinterpret_cast<float*>(at(ws, w.pb));
     L.flags = reinterpret_cast<unsigned*>(at(ws, w.flags));
     L.alpha = alpha; L.beta = beta; L.g = g; L.o = o; L.lse = lse; L.b_final = b_final; L.prune_thr = prune_thr(s);
-    return cuda_status(launch_fwd_tc(L, cs));
+    return cuda_status(s->d == 128 ? launch_fwd_tc128(L, cs) : launch_fwd_tc(L, cs));
 }
 
 ua_status ua_prefill_fwd(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
@@ -465,8 +474,15 @@ ua_status ua_prefill_tile_stats(const ua_shape* s, const void* ws, size_t ws_byt
                                 unsigned long long* skipped, void* stream) {
     if (!s || !tiles || !skipped) return UA_ERR_INVALID_ARG;
     if (s->B <= 0 || s->T <= 0 || s->Hkv <= 0) return UA_ERR_INVALID_ARG;
-    const unsigned long long n = (unsigned long long)((s->T + 127) / 128);
-    *tiles = (unsigned long long)s->B * s->Hkv * n * (n + 1) / 2;
+    if (s->d == 128 && (s->T + 63) / 64 > 0) {
+        // 64-row query tiles: query tile t meets key tiles 0 .. t/2
+        unsigned long long n = 0;
+        for (long long t = 0; t < (s->T + 63) / 64; ++t) n += (unsigned long long)(t / 2 + 1);
+        *tiles = (unsigned long long)s->B * s->Hkv * n;
+    } else {
+        const unsigned long long n = (unsigned long long)((s->T + 127) / 128);
+        *tiles = (unsigned long long)s->B * s->Hkv * n * (n + 1) / 2;
+    }
     *skipped = 0;
     if (!use_tc(s)) return UA_OK;
     const TcWs w = tc_ws_layout(s);
@@ -474,7 +490,7 @@ ua_status ua_prefill_tile_stats(const ua_shape* s, const void* ws, size_t ws_byt
     if (ws_bytes < w.total) return UA_ERR_WORKSPACE;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     unsigned host = 0;
-    const size_t off = w.flags + ((size_t)s->B * s->Hkv * w.nqt * w.nqt + 1) * sizeof(unsigned);
+    const size_t off = w.flags + ((size_t)s->B * s->Hkv * w.nqt * w.nkt + 1) * sizeof(unsigned);
     cudaError_t e = cudaMemcpyAsync(&host, static_cast<const uint8_t*>(ws) + off, sizeof(unsigned),
                                     cudaMemcpyDeviceToHost, cs);
     if (e == cudaSuccess) e = cudaStreamSynchronize(cs);

@@ -176,6 +176,7 @@ struct BwdParams {
 
 struct FwdTcLaunch {
     int B, T, Tp, H, Hkv, nqt;
+    int Tpk;             // row stride of pincl (head_dim 128: T rounded up to 128)
     float scale;
     const void* kh;      // [B*Hkv][T][64] bf16 khat
     const void* kr;      // [B*Hkv][T][64] bf16 RoPE(khat)
@@ -197,6 +198,9 @@ struct FwdTcLaunch {
 
 bool fwd_tc_supported(int d, int G);
 cudaError_t launch_fwd_tc(const FwdTcLaunch& L, cudaStream_t s);
+// head_dim 128: 64-row query tiles (nqt = ceil(T/64)), flags [B*Hkv][nqt][ceil(T/128)] + 4,
+// pincl [B*Hkv][nqt][Tpk]
+cudaError_t launch_fwd_tc128(const FwdTcLaunch& L, cudaStream_t s);
 
 cudaError_t launch_prep(const PrepParams& p, bool bf16_in, bool bf16_work, cudaStream_t s);
 cudaError_t launch_boundary_simt(const BoundaryParams& p, cudaStream_t s);

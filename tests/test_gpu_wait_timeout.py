@@ -21,7 +21,7 @@ def _inputs(w):
             for n, a in x.items()}
 
 
-@pytest.mark.parametrize("d", [64])
+@pytest.mark.parametrize("d", [64, 128])
 def test_zero_wait_limit_reports_timeout_and_leaves_the_context_usable(d):
     # 32 query tiles in one chain: the last CTAs wait on their predecessors' prefixes
     w = I.Workload("timeout", 1, 4096, 3 if d == 128 else 4, 1, d, "bf16", 4096 + d)
