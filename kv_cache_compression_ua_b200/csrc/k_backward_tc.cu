@@ -1,0 +1,1130 @@
+// k_backward_tc.cu -- backward of the bf16 UA prefill on the tensor cores (tcgen05 / TMEM / TMA).
+//
+// The pages describe custom training kernels with activation checkpointing: the decay mask is
+// recomputed, not stored (paperlayer.ai summary §4.2, App. C, App. H).  Here the forward's lse is
+// the only saved statistic; the decay D, Lambda, P and dS are recomputed tile by tile.
+//
+// Formulas (per KV group; s = scale, dA = dO * sigmoid(g)):
+//   P_ij = exp(s qrot_i.krot_j + Lambda_ij - lse_i);  dP_ij = dA_i . v_j;  dZ_ij = P_ij (dP_ij - Delta_i)
+//   dv_j = sum_i P_ij dA_i;  dkrot_j = s sum_i dZ_ij qrot_i;  dqrot_i = s sum_j dZ_ij krot_j
+//   dLambda_ij = sum over the G heads of dZ_ij;  dD[l,j] = -sum_{i>=l} dLambda_ij;  w = dD D / 3
+//   da_q[l] = sum_j w sigmoid(a_q)/softplus(a_q);  da_k[j] = sum_l w sigmoid(a_k)/softplus(a_k)
+//   dX = w sigmoid(X)/softplus(X), X = alpha c + beta, c = <khat_l, khat_j>
+//   dalpha = sum dX c;  dbeta = sum dX;  dkhat_l += alpha sum_j dX khat_j;  dkhat_j += alpha sum_l dX khat_l
+//
+// Passes (rows in 32-row steps, keys in 128-key tiles, everything in the forward's transposed
+// layout: one thread per key, which scans its key column in registers):
+//   k_bwd_prep_tc    dA (bf16 operand), Delta, lse in log2 units
+//   k_bwd_bound_tc   per (batch, KV head, key tile), steps top-down: the decay prefix Pb above
+//                    every step (X^T on the tensor cores)
+//   k_bwd_key_tc     per (batch, KV head, key tile), steps bottom-up: X^T, S_h^T and dP_h^T on the
+//                    tensor cores; decay, P, dZ, the dD suffix scan, w and dX per thread; dv and
+//                    dkrot accumulated in TMEM (P_h^T dA_h, dZ_h^T qrot_h); the key-side decay
+//                    sums; the row sums of w per key tile; dZ_h^T and dX^T stored as bf16 tiles
+//   k_bwd_rowgemm_tc per (batch, KV head, 128-row block, output): dqrot_h = s dZ_h krot and the
+//                    row-side dkhat = alpha dX khat, summed over key tiles in a fixed order
+//   k_bwd_keygemm_tc per (batch, KV head, key tile): the key-side dkhat = alpha dX^T khat
+//   k_bwd_post_tc    RoPE^T, the normalisation Jacobians, casts, da_q / da_k
+// Every sum runs in a fixed order (no atomics), so the result is deterministic.
+#include <cudaTypedefs.h>
+
+#include "tc_common.cuh"
+#include "ua_kernels.h"
+#include "ua_profile.h"
+
+namespace ua {
+
+using namespace tc;
+
+namespace {
+constexpr float kL2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kCbrtLn2b = 0.8849970445005177f;   // (ln 2)^(1/3), the decay's log2-unit factor
+constexpr int ST = 32;                              // rows per step
+constexpr uint32_t kTileBytes = 128 * ST * 2;       // one stored bf16 tile: 128 keys x 32 rows
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn_bwd() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// bf16 [outer][T][d], box = 64 columns x `rows` rows x 1, 128-byte swizzle.
+bool map_rows_bwd(CUtensorMap* m, const void* base, int d, int T, int outer, int rows) {
+    auto fn = encode_fn_bwd();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)outer};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)T * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// V in the caller's [B][T][Hkv][d] layout, box = 64 x 1 head x 128 tokens x 1.
+bool map_v_bwd(CUtensorMap* m, const void* base, int d, int Hkv, int T, int B) {
+    auto fn = encode_fn_bwd();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)Hkv, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)Hkv * d * 2, (cuuint64_t)T * Hkv * d * 2};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// f32 rows of logical length n, row stride ld floats (a multiple of 4), box = `box` x 1; reads
+// past n are zero-filled.
+bool map_vec_bwd(CUtensorMap* m, const void* base, int n, int ld, int outer, int box_n) {
+    auto fn = encode_fn_bwd();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)outer};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+    cuuint32_t box[2] = {(cuuint32_t)box_n, 1};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// K-major SW128 descriptor of a bf16 tile of `rows` rows x d columns stored as 64-column boxes
+// of rows*128 bytes: k-step kk (16 columns) lives in box kk/4 at byte offset (kk%4)*32.
+__device__ __forceinline__ uint64_t kdesc_rows(uint32_t tile, int rows, int kk) {
+    return smem_desc(tile + (uint32_t)(kk >> 2) * (uint32_t)(rows * 128) + (uint32_t)(kk & 3) * 32u, 16, 1024,
+                     kSwizzle128B);
+}
+
+// mbar_wait taken by every lane of a warp, with one verdict for the whole warp (a warp then
+// never diverges around its warp-collective TMEM loads or issue loops).
+__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort)) != 0;
+}
+
+// Bulk copy (no tensor map) global -> shared, completing on an mbarrier.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// First stored tile of key tile kt in the causal band (steps 4kt .. nst-1 of every key tile).
+__host__ __device__ __forceinline__ size_t band_off(int kt, int nkt) {
+    return (size_t)4 * ((size_t)kt * nkt - (size_t)kt * (kt - 1) / 2);
+}
+
+// softplus(X) / ln 2 and sigmoid(X) for t2 = X log2(e), from one exp2: e = 2^-|t2|,
+// softplus/ln2 = max(t2, 0) + log2(1 + e) (the same degree-7 fit as the forward's
+// log2_softplus_over_ln2, its argument before the final log2), sigmoid = 1/(1+e) or e/(1+e).
+__device__ __forceinline__ void softplus_sigmoid(float t2, float& sp_ln2, float& sig) {
+    const float e = ex2f(-fabsf(t2));
+    float q = -0.012319492176175117f;
+    q = fmaf(q, e, 0.06360796093940735f);
+    q = fmaf(q, e, -0.15535196661949158f);
+    q = fmaf(q, e, 0.2560097873210907f);
+    q = fmaf(q, e, -0.35339486598968506f);
+    q = fmaf(q, e, 0.48006370663642883f);
+    q = fmaf(q, e, -0.7213100790977478f);
+    q = fmaf(q, e, 1.4426947832107544f);
+    sp_ln2 = fmaf(e, q, fmaxf(t2, 0.f));
+    const float r = __frcp_rn(1.f + e);
+    sig = t2 >= 0.f ? r : e * r;
+}
+
+// sigmoid(x) / softplus(x), 0 where softplus underflows (the decay it multiplies is then 0 too).
+__device__ __forceinline__ float sig_over_sp_f(float x) {
+    const float sp = softplus_f(x);
+    return sp > 0.f ? sigmoid_f(x) / sp : 0.f;
+}
+
+// Sum over the 32 lanes of a warp of v[0..31] (lane t's 32 values), transposed: on return lane t
+// holds sum over lanes of v[t] in v[0].  A butterfly that halves the vector at every level.
+__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) {
+        const bool upper = (lane & w) != 0;
+#pragma unroll
+        for (int i = 0; i < w; ++i) {
+            // keep the half selected by this lane's bit, send the other half
+            const float send = upper ? v[i] : v[i + w];
+            const float keep = upper ? v[i + w] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        }
+    }
+    return v[0];
+}
+}  // namespace
+
+// =========================================================================== prep
+// grid (T, B), 256 threads: dA = dO * sigmoid(g) (bf16, [B*H][T][d] rows), Delta = sum_c dO*O and
+// lse * log2(e) per (b, h, t).
+template <int DH>
+__global__ void __launch_bounds__(256) k_bwd_prep_tc(BwdTcParams p) {
+    constexpr int PER = DH / 32;
+    const int t = blockIdx.x, b = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(p.o);
+    const __nv_bfloat16* dO = static_cast<const __nv_bfloat16*>(p.d_o);
+    const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(p.g);
+    __nv_bfloat16* ad = static_cast<__nv_bfloat16*>(p.ad);
+    for (int h = warp; h < p.H; h += 8) {
+        const size_t src = (((size_t)b * p.T + t) * p.H + h) * DH + lane * PER;
+        float acc = 0.f;
+        float a[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const float dv = __bfloat162float(dO[src + e]);
+            acc = fmaf(dv, __bfloat162float(o[src + e]), acc);
+            a[e] = dv * sigmoid_f(__bfloat162float(g[src + e]));
+        }
+        const size_t dst = (((size_t)b * p.H + h) * p.T + t) * DH + lane * PER;
+#pragma unroll
+        for (int e = 0; e < PER; e += 2)
+            *reinterpret_cast<__nv_bfloat162*>(ad + dst + e) = __floats2bfloat162_rn(a[e], a[e + 1]);
+#pragma unroll
+        for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+        if (lane == 0) {
+            const size_t r = ((size_t)b * p.H + h);
+            p.delta[r * p.Tp + t] = acc;
+            p.lse2[r * p.Tp + t] = p.lse[r * p.T + t] * kL2e;
+        }
+    }
+}
+
+// =========================================================================== boundary pass
+// grid (nkt, B*Hkv), 128 threads = one thread per key of the tile.  Steps s = 4kt .. nst-1 top
+// down: Pb[s][j] = sum_{j < l < 32 s} D[l, j] is written, then the step's X^T tile (tensor cores,
+// two TMEM slots so the next step's MMA overlaps this step's decay) adds its rows.
+namespace bnd {
+template <int DH>
+struct Smem {
+    alignas(1024) uint8_t khk[DH / 64][16384];      // khat of the key tile, boxes [128][64]
+    alignas(1024) uint8_t kq[2][DH / 64][4096];     // khat of the step's rows, boxes [32][64]
+    alignas(128) float lq[2][ST];
+    alignas(128) float lk[128];
+    alignas(8) uint64_t kfull, qfull[2], xfull[2];
+    uint32_t tmem;
+    int abort;
+};
+}  // namespace bnd
+
+template <int DH>
+__global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CUtensorMap tm_khk,
+                                                      const __grid_constant__ CUtensorMap tm_khq,
+                                                      const __grid_constant__ CUtensorMap tm_lq,
+                                                      const __grid_constant__ CUtensorMap tm_lk, BwdTcParams p) {
+    constexpr uint32_t ID_X = idesc_bf16(128, ST, 0, 0);
+    constexpr int NB = DH / 64;
+    extern __shared__ uint8_t smem_raw[];
+    using SM = bnd::Smem<DH>;
+    SM& S = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int kt = blockIdx.x, unit = blockIdx.y, kvh = unit % p.Hkv;
+    const int T = p.T;
+    const int s0 = 4 * kt, nsteps = p.nst - s0;
+    volatile int* abort = &S.abort;
+    if (tid == 0) {
+        mbar_init(&S.kfull, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.qfull[i], 1);
+            mbar_init(&S.xfull[i], 1);
+        }
+        S.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&S.tmem, 64);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem;
+    const bool leader = warp == 0 && elect_one();
+    auto load_step = [&](int it) {
+        const int st = it & 1, s = s0 + it;
+        mbar_expect_tx(&S.qfull[st], NB * 4096 + ST * 4);
+        for (int c = 0; c < NB; ++c) tma_load_3d(S.kq[st][c], &tm_khq, &S.qfull[st], 64 * c, s * ST, unit);
+        tma_load_2d(S.lq[st], &tm_lq, &S.qfull[st], s * ST, unit);
+    };
+    auto issue_x = [&](int it) {
+        const int st = it & 1;
+        const uint32_t a = smem_u32(S.khk[0]), bq = smem_u32(S.kq[st][0]);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+            umma_f16(tmem + st * 32, kdesc_rows(a, 128, kk), kdesc_rows(bq, ST, kk), ID_X, kk > 0);
+        umma_commit(&S.xfull[st]);
+    };
+    if (leader) {
+        mbar_expect_tx(&S.kfull, NB * 16384 + 512);
+        for (int c = 0; c < NB; ++c) tma_load_3d(S.khk[c], &tm_khk, &S.kfull, 64 * c, kt * 128, unit);
+        tma_load_2d(S.lk, &tm_lk, &S.kfull, kt * 128, unit);
+        load_step(0);
+        if (nsteps > 1) load_step(1);
+    }
+    bool ok = mbar_wait(&S.kfull, 0, abort);
+    if (leader && ok && mbar_wait(&S.qfull[0], 0, abort)) {
+        tc_fence_after();
+        issue_x(0);
+    }
+    const int j = kt * 128 + tid;
+    const float rk3 = ex2f(S.lk[tid]) * kCbrtLn2b;
+    const float al2 = p.alpha[kvh] * kL2e, be2 = p.beta[kvh] * kL2e;
+    float run = 0.f;                                  // sum of D / rk3 over the rows so far
+    float* pbrow = p.pb + (size_t)unit * p.nst * p.Tpk + (size_t)kt * 128 + tid;
+    const uint32_t tl = (uint32_t)(warp * 32) << 16;
+    for (int it = 0; it < nsteps; ++it) {
+        const int st = it & 1, s = s0 + it;
+        pbrow[(size_t)s * p.Tpk] = rk3 * run;
+        if (leader && ok && it + 1 < nsteps) {
+            if (mbar_wait(&S.qfull[(it + 1) & 1], ((it + 1) >> 1) & 1, abort)) {
+                tc_fence_after();
+                issue_x(it + 1);
+            } else {
+                ok = false;
+            }
+        }
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(&S.xfull[st], (it >> 1) & 1, abort)) != 0;
+        uint32_t x[32];
+        float lqv[32];
+        if (ok) {
+            tc_fence_after();
+            uint32_t (&x0)[16] = *reinterpret_cast<uint32_t(*)[16]>(&x[0]);
+            uint32_t (&x1)[16] = *reinterpret_cast<uint32_t(*)[16]>(&x[16]);
+            tmem_ld16_async(tmem + tl + st * 32, x0);
+            tmem_ld16_async(tmem + tl + st * 32 + 16, x1);
+            tmem_wait16(x0);
+            tmem_wait16(x1);
+#pragma unroll
+            for (int r = 0; r < 32; r += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(&S.lq[st][r]);
+                lqv[r] = v.x; lqv[r + 1] = v.y; lqv[r + 2] = v.z; lqv[r + 3] = v.w;
+            }
+        }
+        tc_fence_before();
+        ok = __syncthreads_and(ok) != 0;                // slot st and lq[st] read by everyone
+        if (leader && ok && it + 2 < nsteps) load_step(it + 2);
+        if (ok) {
+            const int l0 = s * ST;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const float dq = ex2f(fmaf(log2_softplus_over_ln2(fmaf(al2, __uint_as_float(x[r]), be2)),
+                                           0.33333334f, lqv[r]));
+                const int l = l0 + r;
+                run += (l > j && l < T) ? dq : 0.f;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*abort && tid == 0) drain_pause(10000000ull);
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 64);
+    }
+}
+
+// =========================================================================== key-major pass
+// grid (nkt, B*Hkv), 160 threads: warps 0-3 compute (thread = key j, TMEM lane), warp 4 issues
+// the TMA loads and the MMAs.  Steps s = nst-1 down to 4kt.  TMEM: dV (DH columns), dKrot (DH),
+// the X^T slot (32), two slots for the S_h^T / dP_h^T pair of a head (64 each).
+namespace key {
+template <int DH, int G>
+struct Smem {
+    alignas(1024) uint8_t khk[DH / 64][16384];   // khat / krot / v of the key tile, boxes [128][64]
+    alignas(1024) uint8_t krk[DH / 64][16384];
+    alignas(1024) uint8_t vk[DH / 64][16384];
+    alignas(1024) uint8_t kq[2][DH / 64][4096];  // khat of the step's rows, boxes [32][64], two stages
+    alignas(1024) uint8_t qh[G][DH / 64][4096];  // qrot / dA of the step's rows, per head
+    alignas(1024) uint8_t ah[G][DH / 64][4096];
+    alignas(1024) uint8_t tp[2][kTileBytes];     // P_h^T and dZ_h^T tiles (K-major, no swizzle), head parity
+    alignas(1024) uint8_t tz[2][kTileBytes];
+    alignas(128) float lq[2][ST];                // log2 rate / 3 of the step's rows (with kq)
+    alignas(128) float pbv[2][128];              // decay prefix above the step (with kq)
+    alignas(128) float lse2[G][ST];              // per head (with qh / ah)
+    alignas(128) float dlt[G][ST];
+    alignas(128) float lk[128];
+    alignas(16) float red[2][4];
+    alignas(8) uint64_t kfull, qfull[2], qempty[2], xfull, xempty, hfull[G], hdone[G], pfull[2], pempty[2],
+        tfull[2], tempty[2], accdone;
+    uint32_t tmem;
+    int abort;
+};
+}  // namespace key
+
+template <int DH, int G>
+__global__ void __launch_bounds__(160, 1)
+k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__ CUtensorMap tm_krk,
+             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_khq,
+             const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ad,
+             const __grid_constant__ CUtensorMap tm_lq, const __grid_constant__ CUtensorMap tm_lk,
+             const __grid_constant__ CUtensorMap tm_pb, const __grid_constant__ CUtensorMap tm_lse2,
+             const __grid_constant__ CUtensorMap tm_dlt, BwdTcParams p) {
+    constexpr int NB = DH / 64;
+    constexpr uint32_t ID_L = idesc_bf16(128, ST, 0, 0);      // logits: keys x rows, both K-major
+    constexpr uint32_t ID_ACC = idesc_bf16(128, DH, 0, 1);    // tile^T (K-major) x rows (MN-major)
+    constexpr uint32_t COL_DV = 0, COL_DK = DH, COL_X = 2 * DH, COL_P = 2 * DH + 32;
+    static_assert(COL_P + 128 <= 512, "TMEM budget");
+    extern __shared__ uint8_t smem_raw[];
+    using SM = key::Smem<DH, G>;
+    SM& S = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int kt = blockIdx.x, unit = blockIdx.y, kvh = unit % p.Hkv, b = unit / p.Hkv;
+    const int T = p.T;
+    const int s0 = 4 * kt, nsteps = p.nst - s0;
+    volatile int* abort = &S.abort;
+    if (tid == 0) {
+        mbar_init(&S.kfull, 1);
+        mbar_init(&S.xfull, 1);
+        mbar_init(&S.xempty, 4);
+        mbar_init(&S.accdone, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.qfull[i], 1);
+            mbar_init(&S.qempty[i], 4);
+            mbar_init(&S.pfull[i], 1);
+            mbar_init(&S.pempty[i], 4);
+            mbar_init(&S.tfull[i], 4);
+            mbar_init(&S.tempty[i], 1);
+        }
+        for (int h = 0; h < G; ++h) {
+            mbar_init(&S.hfull[h], 1);
+            mbar_init(&S.hdone[h], 1);
+        }
+        S.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&S.tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem;
+
+    if (warp == 4) {
+        // ------------------------------------------------ TMA + MMA issue (one elected lane)
+        const bool leader = elect_one();
+        bool ok = true;
+        // step it covers rows of step s = nst-1-it
+        auto load_q = [&](int it) {
+            const int st = it & 1, s = p.nst - 1 - it;
+            if (leader) {
+                mbar_expect_tx(&S.qfull[st], NB * 4096 + ST * 4 + 128 * 4);
+                for (int c = 0; c < NB; ++c) tma_load_3d(S.kq[st][c], &tm_khq, &S.qfull[st], 64 * c, s * ST, unit);
+                tma_load_2d(S.lq[st], &tm_lq, &S.qfull[st], s * ST, unit);
+                tma_load_2d(S.pbv[st], &tm_pb, &S.qfull[st], kt * 128, unit * p.nst + s);
+            }
+            __syncwarp();
+        };
+        auto load_h = [&](int it, int h) {
+            const int s = p.nst - 1 - it, row = b * p.H + kvh * G + h;
+            if (leader) {
+                mbar_expect_tx(&S.hfull[h], 2 * NB * 4096 + 2 * ST * 4);
+                for (int c = 0; c < NB; ++c) {
+                    tma_load_3d(S.qh[h][c], &tm_q, &S.hfull[h], 64 * c, s * ST, row);
+                    tma_load_3d(S.ah[h][c], &tm_ad, &S.hfull[h], 64 * c, s * ST, row);
+                }
+                tma_load_2d(S.lse2[h], &tm_lse2, &S.hfull[h], s * ST, row);
+                tma_load_2d(S.dlt[h], &tm_dlt, &S.hfull[h], s * ST, row);
+            }
+            __syncwarp();
+        };
+        if (leader) {
+            mbar_expect_tx(&S.kfull, 3 * NB * 16384 + 512);
+            for (int c = 0; c < NB; ++c) {
+                tma_load_3d(S.khk[c], &tm_khk, &S.kfull, 64 * c, kt * 128, unit);
+                tma_load_3d(S.krk[c], &tm_krk, &S.kfull, 64 * c, kt * 128, unit);
+                tma_load_4d(S.vk[c], &tm_v, &S.kfull, 64 * c, kvh, kt * 128, b);
+            }
+            tma_load_2d(S.lk, &tm_lk, &S.kfull, kt * 128, unit);
+        }
+        __syncwarp();
+        load_q(0);
+        if (nsteps > 1) load_q(1);
+        for (int h = 0; h < G; ++h) load_h(0, h);
+        ok = wwait(&S.kfull, 0, abort);
+        const uint32_t akh = smem_u32(S.khk[0]), akr = smem_u32(S.krk[0]), av = smem_u32(S.vk[0]);
+        bool first_acc = true;
+        for (int it = 0; ok && it < nsteps; ++it) {
+            const int st = it & 1;
+            // X^T of the step
+            if (!wwait(&S.qfull[st], (it >> 1) & 1, abort)) break;
+            if (it >= 1 && !wwait(&S.xempty, (it - 1) & 1, abort)) break;
+            tc_fence_after();
+            if (leader) {
+                const uint32_t bq = smem_u32(S.kq[st][0]);
+#pragma unroll
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    umma_f16(tmem + COL_X, kdesc_rows(akh, 128, kk), kdesc_rows(bq, ST, kk), ID_L, kk > 0);
+                umma_commit(&S.xfull);
+            }
+            __syncwarp();
+            // accumulation of head hh of this step: dV += P^T dA, dKrot += dZ^T qrot
+            auto accum = [&](int hh) -> bool {
+                const uint32_t v = (uint32_t)(it * G + hh), tb = v & 1;
+                if (!wwait(&S.tfull[tb], (v >> 1) & 1, abort)) return false;
+                tc_fence_after();
+                if (leader) {
+                    const uint32_t tpa = smem_u32(S.tp[tb]), tza = smem_u32(S.tz[tb]);
+                    const uint32_t ba = smem_u32(S.ah[hh][0]), bqh = smem_u32(S.qh[hh][0]);
+#pragma unroll
+                    for (int kk = 0; kk < ST / 16; ++kk) {
+                        // A: tile^T, K-major no swizzle (8 keys x 16 B core matrices; 128 B apart
+                        // along the keys, 2048 B apart along the rows); B: rows of the step,
+                        // MN-major SW128 (64-dim atoms 4096 B apart, 8-row groups 1024 B apart)
+                        const uint64_t da = smem_desc(tpa + kk * 4096u, 2048, 128, kSwizzleNone);
+                        const uint64_t dz = smem_desc(tza + kk * 4096u, 2048, 128, kSwizzleNone);
+                        const uint64_t db = smem_desc(ba + kk * 2048u, 4096, 1024, kSwizzle128B);
+                        const uint64_t dq = smem_desc(bqh + kk * 2048u, 4096, 1024, kSwizzle128B);
+                        const uint32_t acc = (first_acc && kk == 0) ? 0u : 1u;
+                        umma_f16(tmem + COL_DV, da, db, ID_ACC, acc);
+                        umma_f16(tmem + COL_DK, dz, dq, ID_ACC, acc);
+                    }
+                    umma_commit(&S.tempty[tb]);
+                    umma_commit(&S.hdone[hh]);
+                }
+                __syncwarp();
+                first_acc = false;
+                return true;
+            };
+            for (int h = 0; h < G && ok; ++h) {
+                const uint32_t u = (uint32_t)(it * G + h), pp = u & 1;
+                if (!wwait(&S.hfull[h], it & 1, abort)) { ok = false; break; }
+                if (u >= 2 && !wwait(&S.pempty[pp], ((u >> 1) - 1) & 1, abort)) { ok = false; break; }
+                tc_fence_after();
+                if (leader) {
+                    const uint32_t bqh = smem_u32(S.qh[h][0]), bah = smem_u32(S.ah[h][0]);
+#pragma unroll
+                    for (int kk = 0; kk < DH / 16; ++kk) {
+                        umma_f16(tmem + COL_P + pp * 64, kdesc_rows(akr, 128, kk), kdesc_rows(bqh, ST, kk), ID_L,
+                                 kk > 0);
+                        umma_f16(tmem + COL_P + pp * 64 + 32, kdesc_rows(av, 128, kk), kdesc_rows(bah, ST, kk),
+                                 ID_L, kk > 0);
+                    }
+                    umma_commit(&S.pfull[pp]);
+                }
+                __syncwarp();
+                if (h >= 1) {
+                    if (!accum(h - 1)) { ok = false; break; }
+                    // head h-1's operands are free once its accumulation completed: refill them
+                    if (it + 1 < nsteps) {
+                        if (!wwait(&S.hdone[h - 1], it & 1, abort)) { ok = false; break; }
+                        load_h(it + 1, h - 1);
+                    }
+                }
+            }
+            if (!ok) break;
+            if (!accum(G - 1)) break;
+            if (it + 2 < nsteps) {
+                // stage st (khat rows, lq, pb) is free once the compute warps have read it
+                if (!wwait(&S.qempty[st], (it >> 1) & 1, abort)) break;
+                load_q(it + 2);
+            }
+            if (it + 1 < nsteps) {
+                if (!wwait(&S.hdone[G - 1], it & 1, abort)) break;
+                load_h(it + 1, G - 1);
+            }
+        }
+        if (leader) umma_commit(&S.accdone);
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ compute warps: thread = key j
+        const int jl = tid;
+        const int j = kt * 128 + jl;
+        const uint32_t tl = (uint32_t)(warp * 32) << 16;
+        const float al = p.alpha[kvh], be = p.beta[kvh];
+        const float al2 = al * kL2e, be2 = be * kL2e;
+        const float sl = p.scale * kL2e;
+        bool ok = wwait(&S.kfull, 0, abort);
+        const float rk3 = ok ? ex2f(S.lk[jl]) * kCbrtLn2b : 0.f;   // r_k^(1/3) (ln 2)^(1/3)
+        float carry = 0.f;                            // sum of dLambda over the rows below (dD = -carry)
+        float dak = 0.f, dal = 0.f, dbe = 0.f;
+        const size_t tstride = (size_t)p.ntiles * kTileBytes;      // bytes per stored tile set
+        uint8_t* tile_base = static_cast<uint8_t*>(p.tiles) + (size_t)unit * (G + 1) * tstride;
+        const size_t band = band_off(kt, p.nkt);
+        for (int it = 0; ok && it < nsteps; ++it) {
+            const int st = it & 1, s = p.nst - 1 - it;
+            const int i0 = s * ST;
+            if (!wwait(&S.qfull[st], (it >> 1) & 1, abort)) { ok = false; break; }
+            const float pbj = S.pbv[st][jl];
+            if (!wwait(&S.xfull, it & 1, abort)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t x[32];
+            {
+                uint32_t (&x0)[16] = *reinterpret_cast<uint32_t(*)[16]>(&x[0]);
+                uint32_t (&x1)[16] = *reinterpret_cast<uint32_t(*)[16]>(&x[16]);
+                tmem_ld16_async(tmem + tl + COL_X, x0);
+                tmem_ld16_async(tmem + tl + COL_X + 16, x1);
+                tmem_wait16(x0);
+                tmem_wait16(x1);
+            }
+            // decay of the step's rows: Dq = D / rk3; lam = Lambda * log2(e)
+            float dqv[32], lam[32];
+            {
+                float c = 0.f;
+#pragma unroll
+                for (int r = 0; r < 32; r += 4) {
+                    const float4 lv = *reinterpret_cast<const float4*>(&S.lq[st][r]);
+                    const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int l = i0 + r + e;
+                        float dq = ex2f(fmaf(log2_softplus_over_ln2(fmaf(al2, __uint_as_float(x[r + e]), be2)),
+                                             0.33333334f, l4[e]));
+                        dq = (l > j && l < T) ? dq : 0.f;
+                        dqv[r + e] = dq;
+                        c += dq;
+                        lam[r + e] = -fmaf(rk3, c, pbj) * kL2e;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&S.xempty);
+                mbar_arrive(&S.qempty[st]);
+            }
+            float dlam[32];
+#pragma unroll
+            for (int r = 0; r < 32; ++r) dlam[r] = 0.f;
+            const bool jv = j < T;
+            for (int h = 0; h < G && ok; ++h) {
+                const uint32_t u = (uint32_t)(it * G + h), pp = u & 1;
+                if (!wwait(&S.hfull[h], it & 1, abort)) { ok = false; break; }
+                if (!wwait(&S.pfull[pp], (u >> 1) & 1, abort)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t sv[32], dpv[32];
+                {
+                    uint32_t (&a0)[16] = *reinterpret_cast<uint32_t(*)[16]>(&sv[0]);
+                    uint32_t (&a1)[16] = *reinterpret_cast<uint32_t(*)[16]>(&sv[16]);
+                    uint32_t (&b0)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dpv[0]);
+                    uint32_t (&b1)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dpv[16]);
+                    const uint32_t base = tmem + tl + COL_P + pp * 64;
+                    tmem_ld16_async(base, a0);
+                    tmem_ld16_async(base + 16, a1);
+                    tmem_ld16_async(base + 32, b0);
+                    tmem_ld16_async(base + 48, b1);
+                    tmem_wait16(a0);
+                    tmem_wait16(a1);
+                    tmem_wait16(b0);
+                    tmem_wait16(b1);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.pempty[pp]);
+                const uint32_t tb = u & 1;
+                if (u >= 2 && !wwait(&S.tempty[tb], ((u >> 1) - 1) & 1, abort)) { ok = false; break; }
+                uint8_t* ttp = S.tp[tb];
+                uint8_t* ttz = S.tz[tb];
+                uint4* gz = reinterpret_cast<uint4*>(tile_base + (size_t)h * tstride + (band + (s - s0)) * kTileBytes);
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    uint32_t wp[4], wz[4];
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        float pz[2], zz[2];
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const int r = c8 * 8 + e + q;
+                            const int i = i0 + r;
+                            const float lse2 = S.lse2[h][r], dl = S.dlt[h][r];
+                            float pv = ex2f(fmaf(__uint_as_float(sv[r]), sl, lam[r] - lse2));
+                            pv = (jv && i >= j && i < T) ? pv : 0.f;
+                            const float z = pv * (__uint_as_float(dpv[r]) - dl);
+                            dlam[r] += z;
+                            pz[q] = pv;
+                            zz[q] = z;
+                        }
+                        __nv_bfloat162 bp = __floats2bfloat162_rn(pz[0], pz[1]);
+                        __nv_bfloat162 bz = __floats2bfloat162_rn(zz[0], zz[1]);
+                        wp[e >> 1] = *reinterpret_cast<uint32_t*>(&bp);
+                        wz[e >> 1] = *reinterpret_cast<uint32_t*>(&bz);
+                    }
+                    const uint4 vp = make_uint4(wp[0], wp[1], wp[2], wp[3]);
+                    const uint4 vz = make_uint4(wz[0], wz[1], wz[2], wz[3]);
+                    // core matrix (8 keys x 8 rows): rows 8*c8.., this key's 16-byte line
+                    *reinterpret_cast<uint4*>(ttp + c8 * 2048 + jl * 16) = vp;
+                    *reinterpret_cast<uint4*>(ttz + c8 * 2048 + jl * 16) = vz;
+                    gz[c8 * 128 + jl] = vz;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.tfull[tb]);
+            }
+            if (!ok) break;
+            // dD = -(sum of dLambda over the rows at and below l), bottom up; w = dD D / 3
+            float wv[32];
+#pragma unroll
+            for (int r = 31; r >= 0; --r) {
+                carry += dlam[r];
+                wv[r] = -carry * rk3 * dqv[r] * 0.33333334f;      // zero where D was masked
+                dak += wv[r];
+            }
+            {
+                uint4* gx = reinterpret_cast<uint4*>(tile_base + (size_t)G * tstride + (band + (s - s0)) * kTileBytes);
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    uint32_t wx[4];
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        float xx[2];
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const int r = c8 * 8 + e + q;
+                            const float xs = __uint_as_float(x[r]);
+                            float sp2, sg;
+                            softplus_sigmoid(fmaf(al2, xs, be2), sp2, sg);
+                            const float ratio = sp2 > 0.f ? sg * __frcp_rn(sp2 * kLn2) : 0.f;
+                            const float dX = wv[r] * ratio;
+                            dal = fmaf(dX, xs, dal);
+                            dbe += dX;
+                            xx[q] = dX;
+                        }
+                        __nv_bfloat162 bx = __floats2bfloat162_rn(xx[0], xx[1]);
+                        wx[e >> 1] = *reinterpret_cast<uint32_t*>(&bx);
+                    }
+                    gx[c8 * 128 + jl] = make_uint4(wx[0], wx[1], wx[2], wx[3]);
+                }
+            }
+            // row sums of w over this warp's 32 keys: lane t gets row t's sum (summed over the
+            // four warps and the key tiles, in that order, by the post pass)
+            const float rs = warp_transpose_sum32(wv, lane);
+            p.daq_part[(((size_t)unit * p.nkt + kt) * 4 + warp) * p.Tpk + i0 + lane] = rs;
+        }
+        // ---- results of the key tile
+        const bool done = ok && wwait(&S.accdone, 0, abort);
+        if (done) {
+            tc_fence_after();
+            float* dv = p.dv32 + ((size_t)unit * T + j) * DH;
+            float* dk = p.dkr + ((size_t)unit * T + j) * DH;
+#pragma unroll 1
+            for (int c = 0; c < DH; c += 16) {
+                float a[16], k2[16];
+                tmem_ld16(tmem + tl + COL_DV + c, a);      // warp-collective: every lane loads
+                tmem_ld16(tmem + tl + COL_DK + c, k2);
+                if (j < T) {
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4) {
+                        *reinterpret_cast<float4*>(dv + c + e) = make_float4(a[e], a[e + 1], a[e + 2], a[e + 3]);
+                        *reinterpret_cast<float4*>(dk + c + e) = make_float4(p.scale * k2[e], p.scale * k2[e + 1],
+                                                                             p.scale * k2[e + 2], p.scale * k2[e + 3]);
+                    }
+                }
+            }
+            if (j < T) {
+                const float ak = p.a_k[((size_t)b * T + j) * p.Hkv + kvh];
+                p.dak32[(size_t)unit * T + j] = dak * sig_over_sp_f(ak);
+            }
+        }
+        // dalpha / dbeta partials of the CTA
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            dal += __shfl_xor_sync(0xffffffffu, dal, o);
+            dbe += __shfl_xor_sync(0xffffffffu, dbe, o);
+        }
+        if (lane == 0) {
+            S.red[0][warp] = dal;
+            S.red[1][warp] = dbe;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (tid == 0) {
+            const size_t o = ((size_t)unit * p.nkt + kt) * 2;
+            p.dab[o] = S.red[0][0] + S.red[0][1] + S.red[0][2] + S.red[0][3];
+            p.dab[o + 1] = S.red[1][0] + S.red[1][1] + S.red[1][2] + S.red[1][3];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*abort && tid == 0) drain_pause(10000000ull);
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// =========================================================================== GEMMs over stored tiles
+// Row side: per (128-row block rb, output o, unit): C^T[dims x 128 rows] = sum_{kt <= rb} K_kt^T T_kt,
+// with K the key tile's krot (o < G, T = dZ_o^T tiles) or khat (o = G, T = dX^T tiles); the 128
+// dims run along the TMEM lanes (head_dim 64 uses the lower 64: the upper half of the A operand
+// points at a zero block).  Key side: per (key tile kt, unit): C[128 keys x dims] = sum_{rb >= kt}
+// dX^T_(kt, rb) khat_rb.  128 threads: warp 0 loads, warp 1 issues, all four write the result.
+namespace gemm {
+constexpr int NS = 3;
+template <int DH>
+struct Smem {
+    alignas(1024) uint8_t a[NS][2][16384];       // operand tile boxes [128][64] (rows side: keys; key side: rows)
+    alignas(1024) uint8_t t[NS][4 * kTileBytes]; // four stored tiles (128 rows)
+    alignas(1024) uint8_t zero[DH == 64 ? 16384 : 16];
+    alignas(8) uint64_t full[NS], empty[NS], done;
+    uint32_t tmem;
+    int abort;
+};
+}  // namespace gemm
+
+template <int DH, bool ROWS>
+__global__ void __launch_bounds__(128, 1)
+k_bwd_gemm_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_kr, BwdTcParams p) {
+    constexpr int NB = DH / 64;
+    constexpr int NCOL = ROWS ? 128 : DH;             // accumulator columns
+    extern __shared__ uint8_t smem_raw[];
+    using SM = gemm::Smem<DH>;
+    SM& S = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int NS = gemm::NS;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int blk = blockIdx.x, unit = ROWS ? blockIdx.z : blockIdx.y;
+    const int o = ROWS ? blockIdx.y : p.G;            // output: head o's dqrot, or the dkhat part
+    const int kvh = unit % p.Hkv, b = unit / p.Hkv;
+    const int T = p.T;
+    const int n = ROWS ? blk + 1 : p.nkt - blk;       // operand pairs to sum
+    volatile int* abort = &S.abort;
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&S.full[i], 1);
+            mbar_init(&S.empty[i], 1);
+        }
+        mbar_init(&S.done, 1);
+        S.abort = 0;
+        fence_barrier_init();
+    }
+    if (DH == 64 && ROWS) {
+        uint32_t* z = reinterpret_cast<uint32_t*>(S.zero);
+        for (int i = tid; i < (int)(sizeof(S.zero) / 4); i += 128) z[i] = 0u;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0) {
+        tmem_alloc(&S.tmem, NCOL);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem;
+    const size_t tstride = (size_t)p.ntiles * kTileBytes;
+    const uint8_t* tiles = static_cast<const uint8_t*>(p.tiles) + ((size_t)unit * (p.G + 1) + o) * tstride;
+    if (warp == 0) {
+        const bool leader = elect_one();
+        for (int i = 0; i < n; ++i) {
+            const int stg = i % NS;
+            if (i >= NS && !wwait(&S.empty[stg], ((i / NS) - 1) & 1, abort)) break;
+            // rows side: key tile kt = i of row block blk; key side: row block rb = blk + i of key tile blk
+            const int kt = ROWS ? i : blk, rb = ROWS ? blk : blk + i;
+            if (leader) {
+                mbar_expect_tx(&S.full[stg], NB * 16384 + 4 * kTileBytes);
+                const CUtensorMap* m = (ROWS && o < p.G) ? &tm_kr : &tm_kh;
+                const int r0 = ROWS ? kt * 128 : rb * 128;
+                for (int c = 0; c < NB; ++c) tma_load_3d(S.a[stg][c], m, &S.full[stg], 64 * c, r0, unit);
+                const size_t ti = band_off(kt, p.nkt) + (size_t)(4 * rb - 4 * kt);
+                bulk_load(S.t[stg], tiles + ti * kTileBytes, 4 * kTileBytes, &S.full[stg]);
+            }
+            __syncwarp();
+        }
+    } else if (warp == 1) {
+        const bool leader = elect_one();
+        // rows side: A = K^T (MN-major SW128, M = dims: 64-dim atoms 16384 B apart, or the zero
+        // block), B = tiles as [128 rows x 128 keys] (MN-major no swizzle: 8-row groups 2048 B
+        // apart, 8-key groups 128 B apart); key side: A = tiles as [128 keys x 128 rows]
+        // (K-major no swizzle: 8-row groups 2048 B apart, 8-key groups 128 B apart), B = khat rows
+        // (MN-major SW128, N = dims).
+        constexpr uint32_t ID = ROWS ? idesc_bf16(128, 128, 1, 1) : idesc_bf16(128, DH, 0, 1);
+        bool ok = true;
+        for (int i = 0; i < n && ok; ++i) {
+            const int stg = i % NS;
+            if (!wwait(&S.full[stg], (i / NS) & 1, abort)) { ok = false; break; }
+            tc_fence_after();
+            if (leader) {
+                const uint32_t aa = smem_u32(S.a[stg][0]), ta = smem_u32(S.t[stg]);
+                const uint32_t lbo_a = (DH == 64) ? smem_u32(S.zero) - aa : 16384u;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+                    if (ROWS) {
+                        const uint64_t da = smem_desc(aa + kk * 2048u, lbo_a, 1024, kSwizzle128B);
+                        const uint64_t db = smem_desc(ta + kk * 256u, 2048, 128, kSwizzleNone);
+                        umma_f16(tmem, da, db, ID, acc);
+                    } else {
+                        const uint64_t da = smem_desc(ta + kk * 4096u, 2048, 128, kSwizzleNone);
+                        const uint64_t db = smem_desc(aa + kk * 2048u, 16384, 1024, kSwizzle128B);
+                        umma_f16(tmem, da, db, ID, acc);
+                    }
+                }
+                umma_commit(&S.empty[stg]);
+            }
+            __syncwarp();
+        }
+        if (leader && ok) umma_commit(&S.done);
+        __syncwarp();
+    }
+    // ---- epilogue
+    const bool ok = wwait(&S.done, 0, abort);
+    if (ok) {
+        tc_fence_after();
+        const uint32_t tl = (uint32_t)(warp * 32) << 16;
+        if (ROWS) {
+            // lane = dim d, columns = the block's 128 rows
+            const int d = warp * 32 + lane;
+            const float f = o < p.G ? p.scale : p.alpha[kvh];
+#pragma unroll 1
+            for (int c = 0; c < 128; c += 16) {
+                float v[16];
+                tmem_ld16(tmem + tl + c, v);
+                if (d < DH) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int i = blk * 128 + c + e;
+                        if (i < T) {
+                            if (o < p.G)
+                                p.dqr[(((size_t)b * p.H + kvh * p.G + o) * T + i) * DH + d] = f * v[e];
+                            else
+                                p.dkh_rows[((size_t)unit * T + i) * DH + d] = f * v[e];
+                        }
+                    }
+                }
+            }
+        } else {
+            // lane = key, columns = dims
+            const int j = blk * 128 + warp * 32 + lane;
+            const float f = p.alpha[kvh];
+#pragma unroll 1
+            for (int c = 0; c < DH; c += 16) {
+                float v[16];
+                tmem_ld16(tmem + tl + c, v);
+                if (j < T) {
+                    float* dst = p.dkh_keys + ((size_t)unit * T + j) * DH + c;
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4*>(dst + e) = make_float4(f * v[e], f * v[e + 1], f * v[e + 2], f * v[e + 3]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*abort && tid == 0) drain_pause(10000000ull);
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, NCOL);
+    }
+}
+
+// =========================================================================== post pass
+// grid (T, B), 256 threads: RoPE^T of dqrot / dkrot, the query-norm and key-normalisation
+// Jacobians (khat recomputed from the raw key in fp32), casts; dg, da_q (row sums of w over the
+// key tiles, in order), da_k.
+template <int DH>
+__global__ void __launch_bounds__(256) k_bwd_post_tc(BwdTcParams p) {
+    constexpr int HALF = DH / 2;
+    const int t = blockIdx.x, b = blockIdx.y, T = p.T;
+    __shared__ float s_cos[64], s_sin[64];
+    for (int m = threadIdx.x; m < HALF; m += blockDim.x) rope_cs((double)t, p.rf.f[m], &s_cos[m], &s_sin[m]);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    using bf = __nv_bfloat16;
+    bf* dq = static_cast<bf*>(p.dq);
+    bf* dk = static_cast<bf*>(p.dk);
+    bf* dv = static_cast<bf*>(p.dv);
+    for (int hh = warp; hh < p.H + p.Hkv; hh += 8) {
+        const bool is_q = hh < p.H;
+        const int h = is_q ? hh : hh - p.H;
+        if (is_q) {
+            const float* src = p.dqr + (((size_t)b * p.H + h) * T + t) * DH;
+            bf* dst = dq + (((size_t)b * T + t) * p.H + h) * DH;
+            float y0[2] = {0.f, 0.f}, y1[2] = {0.f, 0.f}, q0[2] = {0.f, 0.f}, q1[2] = {0.f, 0.f};
+            float ss = 0.f, qy = 0.f;
+            const bf* qraw = static_cast<const bf*>(p.q) + (((size_t)b * T + t) * p.H + h) * DH;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int m = lane + 32 * u;
+                if (m < HALF) {
+                    const float x0 = src[m], x1 = src[m + HALF], cs = s_cos[m], sn = s_sin[m];
+                    y0[u] = x0 * cs + x1 * sn;              // rotation by -angle
+                    y1[u] = x1 * cs - x0 * sn;
+                    if (p.variant & kVarQNorm) {
+                        q0[u] = __bfloat162float(qraw[m]);
+                        q1[u] = __bfloat162float(qraw[m + HALF]);
+                        ss += q0[u] * q0[u] + q1[u] * q1[u];
+                        qy += q0[u] * y0[u] + q1[u] * y1[u];
+                    }
+                }
+            }
+            float r = 1.f, k = 0.f;
+            if (p.variant & kVarQNorm) {
+                // q' = r q, r = 1/sqrt(mean(q^2) + eps): dq = r (dq' - q' <q', dq'> / d)
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                    qy += __shfl_xor_sync(0xffffffffu, qy, o);
+                }
+                r = 1.f / sqrtf(ss / (float)DH + kQNormEps);
+                k = r * r * qy / (float)DH;
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int m = lane + 32 * u;
+                if (m < HALF) {
+                    dst[m] = __float2bfloat16_rn(r * (y0[u] - q0[u] * k));
+                    dst[m + HALF] = __float2bfloat16_rn(r * (y1[u] - q1[u] * k));
+                }
+            }
+        } else {
+            const size_t u = (size_t)b * p.Hkv + h;
+            const float* rot = p.dkr + (u * T + t) * DH;
+            const float* a1 = p.dkh_keys + (u * T + t) * DH;
+            const float* a2 = p.dkh_rows + (u * T + t) * DH;
+            const bf* kraw = static_cast<const bf*>(p.k) + (((size_t)b * T + t) * p.Hkv + h) * DH;
+            float g0[2] = {0.f, 0.f}, g1[2] = {0.f, 0.f}, k0[2] = {0.f, 0.f}, k1[2] = {0.f, 0.f};
+            float proj = 0.f, ss = 0.f;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int m = lane + 32 * q;
+                if (m < HALF) {
+                    const float cs = s_cos[m], sn = s_sin[m];
+                    g0[q] = a1[m] + a2[m] + rot[m] * cs + rot[m + HALF] * sn;
+                    g1[q] = a1[m + HALF] + a2[m + HALF] + rot[m + HALF] * cs - rot[m] * sn;
+                    k0[q] = __bfloat162float(kraw[m]);
+                    k1[q] = __bfloat162float(kraw[m + HALF]);
+                    ss += k0[q] * k0[q] + k1[q] * k1[q];
+                    proj += g0[q] * k0[q] + g1[q] * k1[q];
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                proj += __shfl_xor_sync(0xffffffffu, proj, o);
+                ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            }
+            const float n = fmaxf(sqrtf(ss), 1e-12f);
+            const float inv = 1.f / n;
+            // khat = k / n:  dk = (g - khat <khat, g>) / n
+            const float pr = proj * inv * inv;
+            bf* dst = dk + (((size_t)b * T + t) * p.Hkv + h) * DH;
+            bf* dvd = dv + (((size_t)b * T + t) * p.Hkv + h) * DH;
+            const float* dvs = p.dv32 + (u * T + t) * DH;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int m = lane + 32 * q;
+                if (m < HALF) {
+                    dst[m] = __float2bfloat16_rn((g0[q] - k0[q] * pr) * inv);
+                    dst[m + HALF] = __float2bfloat16_rn((g1[q] - k1[q] * pr) * inv);
+                    dvd[m] = __float2bfloat16_rn(dvs[m]);
+                    dvd[m + HALF] = __float2bfloat16_rn(dvs[m + HALF]);
+                }
+            }
+        }
+    }
+    for (int h = threadIdx.x; h < p.Hkv; h += blockDim.x) {
+        const size_t u = (size_t)b * p.Hkv + h;
+        float sw = 0.f;
+        for (int kt = 0; kt <= t / 128; ++kt)
+            for (int w = 0; w < 4; ++w) sw += p.daq_part[((u * p.nkt + kt) * 4 + w) * p.Tpk + t];
+        const size_t src = ((size_t)b * T + t) * p.Hkv + h;
+        p.da_q[src] = sw * sig_over_sp_f(p.a_q[src]);
+        p.da_k[src] = p.dak32[u * T + t];
+    }
+    // dg = dO * O * (1 - sigmoid(g))
+    const bf* o = static_cast<const bf*>(p.o);
+    const bf* dO = static_cast<const bf*>(p.d_o);
+    const bf* g = static_cast<const bf*>(p.g);
+    bf* dg = static_cast<bf*>(p.dg);
+    const size_t base = ((size_t)b * T + t) * p.H * DH;
+    for (int e = threadIdx.x; e < p.H * DH; e += blockDim.x)
+        dg[base + e] = __float2bfloat16_rn(__bfloat162float(dO[base + e]) * __bfloat162float(o[base + e]) *
+                                           (1.f - sigmoid_f(__bfloat162float(g[base + e]))));
+}
+
+// =========================================================================== launcher
+bool bwd_tc_supported(int d, int G) { return (d == 64 || d == 128) && G >= 1 && G <= 4; }
+
+template <int DH, int G>
+static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
+    const int BH = p.B * p.H, BK = p.B * p.Hkv;
+    cudaError_t e;
+    {
+        UA_PROFILE("k_bwd_prep_tc", s);
+        k_bwd_prep_tc<DH><<<dim3(p.T, p.B), 256, 0, s>>>(p);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    CUtensorMap m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk, m_pb, m_lse2, m_dlt, m_kh128;
+    if (!map_rows_bwd(&m_khk, p.kh, DH, p.T, BK, 128) || !map_rows_bwd(&m_krk, p.kr, DH, p.T, BK, 128) ||
+        !map_v_bwd(&m_v, p.v, DH, p.Hkv, p.T, p.B) || !map_rows_bwd(&m_khq, p.kh, DH, p.T, BK, ST) ||
+        !map_rows_bwd(&m_q, p.qr, DH, p.T, BH, ST) || !map_rows_bwd(&m_ad, p.ad, DH, p.T, BH, ST) ||
+        !map_vec_bwd(&m_lq, p.lq2, p.T, p.Tp, BK, ST) || !map_vec_bwd(&m_lk, p.lk2, p.T, p.Tp, BK, 128) ||
+        !map_vec_bwd(&m_pb, p.pb, p.Tpk, p.Tpk, BK * p.nst, 128) ||
+        !map_vec_bwd(&m_lse2, p.lse2, p.T, p.Tp, BH, ST) || !map_vec_bwd(&m_dlt, p.delta, p.T, p.Tp, BH, ST) ||
+        !map_rows_bwd(&m_kh128, p.kh, DH, p.T, BK, 128))
+        return cudaErrorInvalidValue;
+    {
+        const size_t smem = sizeof(bnd::Smem<DH>) + 1024;
+        if ((e = cudaFuncSetAttribute(k_bwd_bound_tc<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess)
+            return e;
+        UA_PROFILE("k_bwd_bound_tc", s);
+        k_bwd_bound_tc<DH><<<dim3(p.nkt, BK), 128, smem, s>>>(m_khk, m_khq, m_lq, m_lk, p);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    {
+        const size_t smem = sizeof(key::Smem<DH, G>) + 1024;
+        if ((e = cudaFuncSetAttribute(k_bwd_key_tc<DH, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess)
+            return e;
+        UA_PROFILE("k_bwd_key_tc", s);
+        k_bwd_key_tc<DH, G><<<dim3(p.nkt, BK), 160, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk,
+                                                               m_pb, m_lse2, m_dlt, p);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    {
+        const size_t smem = sizeof(gemm::Smem<DH>) + 1024;
+        if ((e = cudaFuncSetAttribute(k_bwd_gemm_tc<DH, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(k_bwd_gemm_tc<DH, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        {
+            UA_PROFILE("k_bwd_rowgemm_tc", s);
+            k_bwd_gemm_tc<DH, true><<<dim3(p.nkt, G + 1, BK), 128, smem, s>>>(m_kh128, m_krk, p);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        {
+            UA_PROFILE("k_bwd_keygemm_tc", s);
+            k_bwd_gemm_tc<DH, false><<<dim3(p.nkt, BK), 128, smem, s>>>(m_kh128, m_krk, p);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        UA_PROFILE("k_bwd_post_tc", s);
+        k_bwd_post_tc<DH><<<dim3(p.T, p.B), 256, 0, s>>>(p);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    {
+        UA_PROFILE("k_bwd_dab", s);
+        k_bwd_dab<<<p.Hkv, 256, 0, s>>>(p.dab, p.B, p.Hkv, p.nkt, p.dalpha, p.dbeta);
+    }
+    return cudaGetLastError();
+}
+
+template <int DH>
+static cudaError_t bwd_tc_g(const BwdTcParams& p, cudaStream_t s) {
+    switch (p.G) {
+        case 1: return bwd_tc_inst<DH, 1>(p, s);
+        case 2: return bwd_tc_inst<DH, 2>(p, s);
+        case 3: return bwd_tc_inst<DH, 3>(p, s);
+        case 4: return bwd_tc_inst<DH, 4>(p, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_bwd_tc(const BwdTcParams& p, cudaStream_t s) {
+    return p.d == 64 ? bwd_tc_g<64>(p, s) : bwd_tc_g<128>(p, s);
+}
+
+}  // namespace ua

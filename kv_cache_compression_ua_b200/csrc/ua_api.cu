@@ -356,12 +356,104 @@ BwdWs bwd_ws_layout(const ua_shape* s) {
     return w;
 }
 
+// Workspace of the tensor-core backward: the bf16 token preparation of the tensor-core forward,
+// dA, Delta and lse in log2 units, the decay prefixes above every 32-row step, the stored bf16
+// dZ^T / dX^T tiles of the causal band, and f32 gradient intermediates.
+struct BwdTcWs {
+    size_t qr, kh, kr, lq2, lk2, mq, ad, lse2, delta, pb, tiles, daq, dab, dv32, dkr, dkh, dkh_rows, dqr, dak,
+        total, ntiles;
+    int Tp, Tpk, nkt, nst;
+};
+
+BwdTcWs bwd_tc_ws_layout(const ua_shape* s) {
+    const size_t B = s->B, T = s->T, H = s->H, Hkv = s->Hkv, d = s->d, G = s->H / s->Hkv;
+    BwdTcWs w;
+    w.Tp = (int)round_up(T, 4);
+    w.nkt = (int)((T + 127) / 128);
+    w.Tpk = w.nkt * 128;
+    w.nst = 4 * w.nkt;
+    w.ntiles = (size_t)2 * w.nkt * (w.nkt + 1);
+    const size_t Tp = w.Tp, Tpk = w.Tpk, nkt = w.nkt;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = round_up(off + bytes, 1024); return o; };
+    w.qr = take(B * H * T * d * 2);
+    w.kh = take(B * Hkv * T * d * 2);
+    w.kr = take(B * Hkv * T * d * 2);
+    w.lq2 = take(B * Hkv * Tp * 4);
+    w.lk2 = take(B * Hkv * Tp * 4);
+    w.mq = take(B * H * Tp * 4);
+    w.ad = take(B * H * T * d * 2);
+    w.lse2 = take(B * H * Tp * 4);
+    w.delta = take(B * H * Tp * 4);
+    w.pb = take(B * Hkv * (size_t)w.nst * Tpk * 4);
+    w.tiles = take(B * Hkv * (G + 1) * w.ntiles * 8192);
+    w.daq = take(B * Hkv * nkt * 4 * Tpk * 4);
+    w.dab = take(B * Hkv * nkt * 2 * 4);
+    w.dv32 = take(B * Hkv * T * d * 4);
+    w.dkr = take(B * Hkv * T * d * 4);
+    w.dkh = take(B * Hkv * T * d * 4);
+    w.dkh_rows = take(B * Hkv * T * d * 4);
+    w.dqr = take(B * H * T * d * 4);
+    w.dak = take(B * Hkv * T * 4);
+    w.total = off;
+    return w;
+}
+
+// bf16 problems of the three-rate method (or with the query norm) whose head_dim and group size
+// the tensor-core kernels take run the tensor-core backward; the others the fp32 SIMT one.
+bool use_bwd_tc(const ua_shape* s) {
+    return s->dtype == UA_BF16 && bwd_tc_supported(s->d, s->H / s->Hkv) && (s->variant & kVarMech) == 0;
+}
+
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes) {
     ua_status st = check_shape(shape);
     if (st != UA_OK) return st;
     if (!bytes || shape->prune_p != 0.f) return UA_ERR_INVALID_ARG;   // training is dense
-    *bytes = bwd_ws_layout(shape).total;
+    *bytes = use_bwd_tc(shape) ? bwd_tc_ws_layout(shape).total : bwd_ws_layout(shape).total;
     return UA_OK;
+}
+
+static ua_status prefill_bwd_tc(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
+                                const float* a_q, const float* a_k, const float* alpha, const float* beta,
+                                const void* o, const float* lse, const void* d_o, void* dq, void* dk, void* dv,
+                                void* dg, float* da_q, float* da_k, float* dalpha, float* dbeta, void* ws,
+                                cudaStream_t cs) {
+    ua_status st;
+    const BwdTcWs w = bwd_tc_ws_layout(s);
+    PrepParams pp;
+    memset(&pp, 0, sizeof(pp));
+    pp.B = s->B; pp.T = s->T; pp.H = s->H; pp.Hkv = s->Hkv; pp.d = s->d; pp.theta = s->rope_theta;
+    pp.q = q; pp.k = k; pp.a_q = a_q; pp.a_k = a_k;
+    pp.qr = at(ws, w.qr); pp.kh = at(ws, w.kh); pp.kr = at(ws, w.kr);
+    pp.rq = nullptr; pp.rk = nullptr;
+    pp.Tp = w.Tp; pp.mq_scale = s->scale * 1.4426950408889634f;
+    pp.lq2 = reinterpret_cast<float*>(at(ws, w.lq2)); pp.lk2 = reinterpret_cast<float*>(at(ws, w.lk2));
+    pp.mq = reinterpret_cast<float*>(at(ws, w.mq));
+    pp.rf = rope_freq(s->rope_theta, s->d);
+    pp.variant = s->variant;   // the query norm only: use_bwd_tc excludes the mechanism bits
+    if ((st = cuda_status(launch_prep(pp, true, true, cs))) != UA_OK) return st;
+    BwdTcParams p;
+    p.B = s->B; p.T = s->T; p.Tp = w.Tp; p.Tpk = w.Tpk; p.H = s->H; p.Hkv = s->Hkv; p.d = s->d;
+    p.G = s->H / s->Hkv; p.nkt = w.nkt; p.nst = w.nst; p.scale = s->scale; p.rf = pp.rf; p.variant = s->variant;
+    p.qr = pp.qr; p.kh = pp.kh; p.kr = pp.kr; p.lq2 = pp.lq2; p.lk2 = pp.lk2;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.o = o; p.d_o = d_o;
+    p.a_q = a_q; p.a_k = a_k; p.alpha = alpha; p.beta = beta; p.lse = lse;
+    p.ad = at(ws, w.ad);
+    p.lse2 = reinterpret_cast<float*>(at(ws, w.lse2));
+    p.delta = reinterpret_cast<float*>(at(ws, w.delta));
+    p.pb = reinterpret_cast<float*>(at(ws, w.pb));
+    p.tiles = at(ws, w.tiles);
+    p.ntiles = w.ntiles;
+    p.daq_part = reinterpret_cast<float*>(at(ws, w.daq));
+    p.dab = reinterpret_cast<float*>(at(ws, w.dab));
+    p.dv32 = reinterpret_cast<float*>(at(ws, w.dv32));
+    p.dkr = reinterpret_cast<float*>(at(ws, w.dkr));
+    p.dkh_keys = reinterpret_cast<float*>(at(ws, w.dkh));
+    p.dkh_rows = reinterpret_cast<float*>(at(ws, w.dkh_rows));
+    p.dqr = reinterpret_cast<float*>(at(ws, w.dqr));
+    p.dak32 = reinterpret_cast<float*>(at(ws, w.dak));
+    p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.da_q = da_q; p.da_k = da_k; p.dalpha = dalpha; p.dbeta = dbeta;
+    return cuda_status(launch_bwd_tc(p, cs));
 }
 
 ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
@@ -379,9 +471,14 @@ ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const 
     for (const void* p : need)
         if (!aligned(p, 16)) return UA_ERR_ALIGNMENT;
     if (!aligned(ws, 256)) return UA_ERR_ALIGNMENT;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (use_bwd_tc(s)) {
+        if (ws_bytes < bwd_tc_ws_layout(s).total) return UA_ERR_WORKSPACE;
+        return prefill_bwd_tc(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, d_o, dq, dk, dv, dg, da_q, da_k, dalpha,
+                              dbeta, ws, cs);
+    }
     const BwdWs w = bwd_ws_layout(s);
     if (ws_bytes < w.total) return UA_ERR_WORKSPACE;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const bool bf = s->dtype == UA_BF16;
 
     PrepParams pp;

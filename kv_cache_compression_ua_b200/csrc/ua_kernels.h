@@ -196,6 +196,47 @@ struct FwdTcLaunch {
     float prune_thr;     // chunked pruned prefill (chunks = the 128-row query tiles): -log p, +inf = dense
 };
 
+// Backward on the tensor cores (bf16, head_dim 64 or 128, H/Hkv <= 4, the three-rate method or
+// the query norm).  Rows are cut into 32-row steps, keys into 128-key tiles; nst = 4 * nkt steps
+// (the last ones may lie past T and are then all zero).
+struct BwdTcParams {
+    int B, T, Tp, Tpk, H, Hkv, d, G, nkt, nst;
+    float scale;
+    RopeFreq rf;
+    int variant;          // UA_VAR_QUERY_NORM or 0
+    // token preparation of the tensor-core forward (bf16 copies, log2 rates / 3)
+    const void* qr;       // [B*H][T][d] RoPE(q)
+    const void* kh;       // [B*Hkv][T][d] khat
+    const void* kr;       // [B*Hkv][T][d] RoPE(khat)
+    const float* lq2;     // [B*Hkv][Tp]
+    const float* lk2;     // [B*Hkv][Tp]
+    // the caller's tensors
+    const void* q; const void* k; const void* v; const void* g; const void* o; const void* d_o;
+    const float* a_q; const float* a_k; const float* alpha; const float* beta; const float* lse;
+    // workspace
+    void* ad;             // [B*H][T][d] bf16: dA = dO * sigmoid(g)
+    float* lse2;          // [B*H][Tp] lse * log2(e)
+    float* delta;         // [B*H][Tp] sum_c dO * O
+    float* pb;            // [B*Hkv][nst][Tpk] decay prefix above each step
+    void* tiles;          // [B*Hkv][G+1][ntiles][8 KB]: dZ^T of each head, then dX^T (bf16)
+    size_t ntiles;        // 32-row x 128-key tiles of the causal band: 2 * nkt * (nkt + 1)
+    float* daq_part;      // [B*Hkv][nkt][Tpk] row sums of w over each key tile
+    float* dab;           // [B*Hkv*nkt][2] dalpha / dbeta partials
+    float* dv32;          // [B*Hkv][T][d]
+    float* dkr;           // [B*Hkv][T][d] scale * dkrot
+    float* dkh_keys;      // [B*Hkv][T][d] key-side similarity gradient (alpha applied)
+    float* dkh_rows;      // [B*Hkv][T][d] row-side similarity gradient (alpha applied)
+    float* dqr;           // [B*H][T][d] scale * dqrot
+    float* dak32;         // [B*Hkv][T]
+    // outputs
+    void* dq; void* dk; void* dv; void* dg;
+    float* da_q; float* da_k; float* dalpha; float* dbeta;
+};
+bool bwd_tc_supported(int d, int G);
+cudaError_t launch_bwd_tc(const BwdTcParams& p, cudaStream_t s);
+// reduction of the per-CTA dalpha / dbeta partials (k_backward_simt.cu)
+__global__ void k_bwd_dab(const float* dab, int B, int Hkv, int nkt, float* dalpha, float* dbeta);
+
 bool fwd_tc_supported(int d, int G);
 cudaError_t launch_fwd_tc(const FwdTcLaunch& L, cudaStream_t s);
 // head_dim 128: 64-row query tiles (nqt = ceil(T/64)), flags [B*Hkv][nqt][ceil(T/128)] + 4,

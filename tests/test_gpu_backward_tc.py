@@ -1,0 +1,88 @@
+"""GPU parity of the tensor-core backward (bf16, head_dim 64 and 128, 1-4 query heads per KV
+head) against the analytic fp64 oracle, through the C ABI.
+
+The backward cuts rows into 32-row steps and keys into 128-key tiles; the shapes span a single
+token, ragged tails, several key tiles and every group size, and the query-norm variant.  The
+kernels that ran are checked too: the fp32 SIMT backward must not be the one that answered."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_compression_ua_b200 import inputs as I
+from kv_cache_compression_ua_b200 import ua
+from helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+GRADS = ("dq", "dk", "dv", "dg", "da_q", "da_k", "dalpha", "dbeta")
+
+
+def dev(x):
+    return {n: torch.from_numpy(np.ascontiguousarray(a)).cuda().to(
+        torch.bfloat16 if n in ("q", "k", "v", "g", "d_o") else torch.float32).contiguous() for n, a in x.items()}
+
+
+def run(w, x, variant=0):
+    d = dev(x)
+    f = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
+                       scale=w.scale, theta=w.theta, variant=variant)
+    ua.profile_reset()
+    ua.profile_enable(True)
+    try:
+        gr = ua.prefill_bwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"], f["o"],
+                            f["lse"], f["b_final"], d["d_o"], scale=w.scale, theta=w.theta, variant=variant)
+        torch.cuda.synchronize()
+    finally:
+        ua.profile_enable(False)
+    names = set(ua.profile_read())
+    assert ua.get_device_status() == 0
+    return gr, names
+
+
+SHAPES = [
+    # (B, T, H, Hkv, d)
+    (1, 1, 4, 1, 64),
+    (2, 63, 4, 2, 64),
+    (1, 129, 8, 2, 64),
+    (1, 300, 6, 2, 64),
+    (2, 200, 4, 4, 64),
+    (1, 600, 2, 1, 64),
+    (1, 257, 6, 2, 128),
+    (2, 130, 4, 2, 128),
+    (1, 400, 4, 1, 128),
+]
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,d", SHAPES)
+def test_tensor_core_backward_matches_analytic_oracle(B, T, H, Hkv, d):
+    w = I.Workload("bwdtc", B, T, H, Hkv, d, "bf16", 2300 + T + H + d, with_grad=True)
+    x = I.make_prefill_inputs(w)
+    gr, names = run(w, x)
+    assert "k_bwd_key_tc" in names and "k_bwd_keys" not in names, names
+    g = {k: v.float().cpu().numpy() for k, v in gr.items()}
+    r = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta)
+    for n in GRADS:
+        assert np.all(np.isfinite(g[n])), n
+        assert_close(n, g[n], r[n], "bf16", tensor_scale=True)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_tensor_core_backward_with_query_norm(d):
+    w = I.Workload("bwdqn", 1, 211, 6, 2, d, "bf16", 2400 + d, with_grad=True)
+    x = I.make_prefill_inputs(w)
+    x["q"] = x["q"] * 2.0
+    gr, names = run(w, x, variant=ua.VAR_QUERY_NORM)
+    assert "k_bwd_key_tc" in names, names
+    g = {k: v.float().cpu().numpy() for k, v in gr.items()}
+    r = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta, variant=ua.VAR_QUERY_NORM)
+    for n in GRADS:
+        assert_close(n, g[n], r[n], "bf16", tensor_scale=True)
+
+
+def test_tensor_core_backward_is_deterministic():
+    w = I.Workload("bwddet", 2, 333, 8, 2, 64, "bf16", 2500, with_grad=True)
+    x = I.make_prefill_inputs(w)
+    a, _ = run(w, x)
+    b, _ = run(w, x)
+    for n in GRADS:
+        assert torch.equal(a[n], b[n]), n
