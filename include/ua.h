@@ -75,11 +75,21 @@ typedef enum { UA_F32 = 0, UA_BF16 = 1 } ua_dtype;
  *     UA_ERR_INVALID_ARG.
  *   UA_VAR_QUERY_NORM RMS-normalises every query head before RoPE (Qwen3-style query norm
  *     with unit gain): q' = q / sqrt(mean(q^2) + 1e-6).  Keys keep their L2 normalisation.
+ *   UA_VAR_PER_HEAD_DECAY (prefill calls only) gives every query head its own decay: a_q, a_k
+ *     are [B,T,H], alpha, beta [H], and b_final / lambda_dbg have H heads ([B,H,T] / [B,H,T,T]).
+ *     The pages decide retention "head by head" (summary §4.2) without saying whether a head is
+ *     a query or a KV head; with per-query-head rates, query head h is exactly multi-head UA over
+ *     its group's shared keys and values, so the library repeats each KV head's keys and values
+ *     for the G heads of its group (inside the workspace), runs the per-KV-head path with one
+ *     decay unit per query head (G times the decay work), and sums dk, dv over the copies.  The
+ *     matching decode uses a cache of H heads filled from the repeated keys and values (each
+ *     query head evicts on its own bias); ua_decode_step takes no per-head bit.
  * Any other bit is UA_ERR_INVALID_ARG. */
 #define UA_VAR_NO_QUERY_DECAY 1
 #define UA_VAR_NO_KEY_DECAY 2
 #define UA_VAR_NO_SIM_DECAY 4
 #define UA_VAR_QUERY_NORM 8
+#define UA_VAR_PER_HEAD_DECAY 16
 
 /* Decode-step flag: defer compaction (see ua_decode_step). */
 #define UA_DECODE_DEFER_COMPACT 256

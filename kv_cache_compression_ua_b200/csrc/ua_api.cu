@@ -28,6 +28,7 @@ bool group_ok(int G) { return G == 1 || G == 2 || G == 3 || G == 4 || G == 8; }
 
 // Known bits only, and at least one decay mechanism left on.
 bool variant_ok(int v) { return (v & ~(kVarMech | kVarQNorm)) == 0 && (v & kVarMech) != kVarMech; }
+bool prefill_variant_ok(int v) { return variant_ok(v & ~kVarPerHead); }
 
 ua_status check_shape(const ua_shape* s) {
     if (!s) return UA_ERR_INVALID_ARG;
@@ -37,9 +38,26 @@ ua_status check_shape(const ua_shape* s) {
     if (s->d != 64 && s->d != 128) return UA_ERR_UNSUPPORTED;
     if (!group_ok(s->H / s->Hkv)) return UA_ERR_UNSUPPORTED;
     if (s->dtype != UA_F32 && s->dtype != UA_BF16) return UA_ERR_UNSUPPORTED;
-    if (!variant_ok(s->variant)) return UA_ERR_INVALID_ARG;
+    if (!prefill_variant_ok(s->variant)) return UA_ERR_INVALID_ARG;
     if (!(s->prune_p >= 0.f && s->prune_p <= 1.f)) return UA_ERR_INVALID_ARG;
     return UA_OK;
+}
+
+// Per-query-head decay runs the per-KV-head path with one decay unit per query head, on keys
+// and values repeated for the G query heads of each group (k_per_head.cu).
+bool per_head(const ua_shape* s) { return (s->variant & kVarPerHead) != 0; }
+
+ua_shape per_head_inner(const ua_shape* s) {
+    ua_shape i = *s;
+    i.Hkv = s->H;
+    i.variant = s->variant & ~kVarPerHead;
+    return i;
+}
+
+// bytes of one repeated key or value tensor [B,T,H,d], rounded to 256
+size_t rep_bytes(const ua_shape* s) {
+    const size_t e = s->dtype == UA_BF16 ? 2 : 4;
+    return ((size_t)s->B * s->T * s->H * s->d * e + 255) / 256 * 256;
 }
 
 // Chunked pruned prefill: a key is evicted when its boundary prefix Pb exceeds -log p.
@@ -173,11 +191,18 @@ const char* ua_status_string(ua_status s) {
     return "UA_ERR_UNKNOWN";
 }
 
+// Whole workspace of a forward call (per-query-head decay: two repeated tensors first).
+size_t fwd_call_ws_bytes(const ua_shape* s) {
+    if (!per_head(s)) return prefill_ws_bytes(s);
+    const ua_shape in = per_head_inner(s);
+    return 2 * rep_bytes(s) + prefill_ws_bytes(&in);
+}
+
 ua_status ua_prefill_workspace_size(const ua_shape* shape, size_t* bytes) {
     ua_status st = check_shape(shape);
     if (st != UA_OK) return st;
     if (!bytes) return UA_ERR_INVALID_ARG;
-    *bytes = prefill_ws_bytes(shape);
+    *bytes = fwd_call_ws_bytes(shape);
     return UA_OK;
 }
 
@@ -256,6 +281,29 @@ static ua_status prefill_fwd_tc(const ua_shape* s, const void* q, const void* k,
     return cuda_status(s->d == 128 ? launch_fwd_tc128(L, cs) : launch_fwd_tc(L, cs));
 }
 
+// A validated forward: per-query-head decay repeats K and V into the head of the workspace and
+// runs the per-KV-head path on the rest of it.
+static ua_status prefill_fwd_dispatch(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
+                                      const float* a_q, const float* a_k, const float* alpha, const float* beta,
+                                      void* o, float* lse, float* b_final, float* lambda_dbg, void* ws,
+                                      cudaStream_t cs) {
+    if (per_head(s)) {
+        const ua_shape in = per_head_inner(s);
+        const size_t rb = rep_bytes(s);
+        void* kr = ws;
+        void* vr = at(ws, rb);
+        const bool bf = s->dtype == UA_BF16;
+        const int G = s->H / s->Hkv;
+        ua_status st;
+        if ((st = cuda_status(launch_repeat_kv(k, kr, s->B, s->T, s->H, G, s->d, bf, cs))) != UA_OK) return st;
+        if ((st = cuda_status(launch_repeat_kv(v, vr, s->B, s->T, s->H, G, s->d, bf, cs))) != UA_OK) return st;
+        return prefill_fwd_dispatch(&in, q, kr, vr, g, a_q, a_k, alpha, beta, o, lse, b_final, lambda_dbg,
+                                    at(ws, 2 * rb), cs);
+    }
+    if (use_tc(s) && !lambda_dbg) return prefill_fwd_tc(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, ws, cs);
+    return prefill_fwd_simt(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, lambda_dbg, ws, cs);
+}
+
 ua_status ua_prefill_fwd(const ua_shape* s, const void* q, const void* k, const void* v, const void* g,
                          const float* a_q, const float* a_k, const float* alpha, const float* beta,
                          void* o, float* lse, float* b_final, float* lambda_dbg, void* ws, size_t ws_bytes,
@@ -268,10 +316,9 @@ ua_status ua_prefill_fwd(const ua_shape* s, const void* q, const void* k, const 
         if (p && !aligned(p, 16)) return UA_ERR_ALIGNMENT;
     if (!aligned(ws, 256)) return UA_ERR_ALIGNMENT;
     if (lambda_dbg && s->T > 1024) return UA_ERR_INVALID_ARG;
-    if (ws_bytes < prefill_ws_bytes(s)) return UA_ERR_WORKSPACE;
+    if (ws_bytes < fwd_call_ws_bytes(s)) return UA_ERR_WORKSPACE;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (use_tc(s) && !lambda_dbg) return prefill_fwd_tc(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, ws, cs);
-    return prefill_fwd_simt(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, lambda_dbg, ws, cs);
+    return prefill_fwd_dispatch(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, lambda_dbg, ws, cs);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -314,14 +361,13 @@ ua_status ua_prefill_fwd_noalloc(const ua_shape* s, const void* q, const void* k
     const void* ps[] = {q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final};
     for (const void* p : ps)
         if (p && !aligned(p, 16)) return UA_ERR_ALIGNMENT;
-    if (prefill_ws_bytes(s) > kNoAllocScratchBytes) return UA_ERR_WORKSPACE;
+    if (fwd_call_ws_bytes(s) > kNoAllocScratchBytes) return UA_ERR_WORKSPACE;
     void* ws = nullptr;
     if ((st = noalloc_scratch(&ws)) != UA_OK) return st;
     // Every part of the scratch is written before it is read within a call, so nothing has
     // to be cleared between calls.
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (use_tc(s)) return prefill_fwd_tc(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, ws, cs);
-    return prefill_fwd_simt(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, nullptr, ws, cs);
+    return prefill_fwd_dispatch(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, nullptr, ws, cs);
 }
 
 size_t ua_prefill_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
@@ -405,11 +451,23 @@ bool use_bwd_tc(const ua_shape* s) {
     return s->dtype == UA_BF16 && bwd_tc_supported(s->d, s->H / s->Hkv) && (s->variant & kVarMech) == 0;
 }
 
+size_t bwd_inner_ws_bytes(const ua_shape* s) {
+    return use_bwd_tc(s) ? bwd_tc_ws_layout(s).total : bwd_ws_layout(s).total;
+}
+
+// Whole workspace of a backward call (per-query-head decay: repeated K, V and their gradient
+// copies first).
+size_t bwd_call_ws_bytes(const ua_shape* s) {
+    if (!per_head(s)) return bwd_inner_ws_bytes(s);
+    const ua_shape in = per_head_inner(s);
+    return 4 * rep_bytes(s) + bwd_inner_ws_bytes(&in);
+}
+
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes) {
     ua_status st = check_shape(shape);
     if (st != UA_OK) return st;
     if (!bytes || shape->prune_p != 0.f) return UA_ERR_INVALID_ARG;   // training is dense
-    *bytes = use_bwd_tc(shape) ? bwd_tc_ws_layout(shape).total : bwd_ws_layout(shape).total;
+    *bytes = bwd_call_ws_bytes(shape);
     return UA_OK;
 }
 
@@ -471,9 +529,28 @@ ua_status ua_prefill_bwd(const ua_shape* s, const void* q, const void* k, const 
     for (const void* p : need)
         if (!aligned(p, 16)) return UA_ERR_ALIGNMENT;
     if (!aligned(ws, 256)) return UA_ERR_ALIGNMENT;
+    if (ws_bytes < bwd_call_ws_bytes(s)) return UA_ERR_WORKSPACE;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (per_head(s)) {
+        // per-query-head decay: the per-KV-head backward on repeated K and V, whose key and
+        // value gradients are then summed over each group's copies
+        const ua_shape in = per_head_inner(s);
+        const size_t rb = rep_bytes(s);
+        void* kr = ws;
+        void* vr = at(ws, rb);
+        void* dkr = at(ws, 2 * rb);
+        void* dvr = at(ws, 3 * rb);
+        const bool bfa = s->dtype == UA_BF16;
+        const int G = s->H / s->Hkv;
+        if ((st = cuda_status(launch_repeat_kv(k, kr, s->B, s->T, s->H, G, s->d, bfa, cs))) != UA_OK) return st;
+        if ((st = cuda_status(launch_repeat_kv(v, vr, s->B, s->T, s->H, G, s->d, bfa, cs))) != UA_OK) return st;
+        if ((st = ua_prefill_bwd(&in, q, kr, vr, g, a_q, a_k, alpha, beta, o, lse, b_final, d_o, dq, dkr, dvr, dg,
+                                 da_q, da_k, dalpha, dbeta, at(ws, 4 * rb), ws_bytes - 4 * rb, stream)) != UA_OK)
+            return st;
+        if ((st = cuda_status(launch_sum_copies(dkr, dk, s->B, s->T, s->Hkv, G, s->d, bfa, cs))) != UA_OK) return st;
+        return cuda_status(launch_sum_copies(dvr, dv, s->B, s->T, s->Hkv, G, s->d, bfa, cs));
+    }
     if (use_bwd_tc(s)) {
-        if (ws_bytes < bwd_tc_ws_layout(s).total) return UA_ERR_WORKSPACE;
         return prefill_bwd_tc(s, q, k, v, g, a_q, a_k, alpha, beta, o, lse, d_o, dq, dk, dv, dg, da_q, da_k, dalpha,
                               dbeta, ws, cs);
     }

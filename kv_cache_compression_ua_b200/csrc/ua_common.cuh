@@ -32,7 +32,7 @@ __device__ __forceinline__ float decay_geo(float rq, float rk, float rsim) {
 }
 
 // Variant bits of ua_shape.variant (the ablations; 0 = the method itself).
-constexpr int kVarNoQ = 1, kVarNoK = 2, kVarNoSim = 4, kVarQNorm = 8;
+constexpr int kVarNoQ = 1, kVarNoK = 2, kVarNoSim = 4, kVarQNorm = 8, kVarPerHead = 16;
 constexpr int kVarMech = kVarNoQ | kVarNoK | kVarNoSim;
 constexpr float kQNormEps = 1e-6f;
 

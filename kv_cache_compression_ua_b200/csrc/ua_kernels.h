@@ -237,6 +237,11 @@ cudaError_t launch_bwd_tc(const BwdTcParams& p, cudaStream_t s);
 // reduction of the per-CTA dalpha / dbeta partials (k_backward_simt.cu)
 __global__ void k_bwd_dab(const float* dab, int B, int Hkv, int nkt, float* dalpha, float* dbeta);
 
+// per-query-head decay: repeat K / V for the G query heads of each group; sum gradients back
+cudaError_t launch_repeat_kv(const void* in, void* out, int B, int T, int H, int G, int d, bool bf16, cudaStream_t s);
+cudaError_t launch_sum_copies(const void* in, void* out, int B, int T, int Hkv, int G, int d, bool bf16,
+                              cudaStream_t s);
+
 bool fwd_tc_supported(int d, int G);
 cudaError_t launch_fwd_tc(const FwdTcLaunch& L, cudaStream_t s);
 // head_dim 128: 64-row query tiles (nqt = ceil(T/64)), flags [B*Hkv][nqt][ceil(T/128)] + 4,

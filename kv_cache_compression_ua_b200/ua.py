@@ -37,6 +37,7 @@ class ua_shape(ctypes.Structure):
 
 # ua_shape.variant bits (UA_VAR_* in ua.h); 0 is the method itself.
 VAR_NO_QUERY_DECAY, VAR_NO_KEY_DECAY, VAR_NO_SIM_DECAY, VAR_QUERY_NORM = 1, 2, 4, 8
+VAR_PER_HEAD_DECAY = 16         # decay logits and parameters per query head: a_q, a_k [B,T,H], alpha, beta [H]
 DECODE_DEFER_COMPACT = 256      # ua_decode_step flag: leave evicted pairs in place
 
 
@@ -149,20 +150,27 @@ def _nbytes(t) -> int:
     return t.numel() * t.element_size()
 
 
-def _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out):
+def _rate_heads(H, Hkv, variant):
+    """Heads the decay logits and parameters belong to: the KV heads, or (per-query-head decay)
+    the query heads."""
+    return H if int(variant) & VAR_PER_HEAD_DECAY else Hkv
+
+
+def _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out, variant=0):
     """Checks the prefill arguments against q [B,T,H,d] and k [B,T,Hkv,d]; returns the sizes."""
     B, T, H, d = q.shape
     if k.dim() != 4 or (k.shape[0], k.shape[1], k.shape[3]) != (B, T, d):
         raise ValueError(f"k: shape {tuple(k.shape)}, expected [{B}, {T}, Hkv, {d}]")
     Hkv = k.shape[2]
+    Hr = _rate_heads(H, Hkv, variant)
     act = (q.dtype,)
     _need("k", k, B * T * Hkv * d, act)
     _need("v", v, B * T * Hkv * d, act)
     _need("g", g, B * T * H * d, act)
-    _need("a_q", a_q, B * T * Hkv, F32)
-    _need("a_k", a_k, B * T * Hkv, F32)
-    _need("alpha", alpha, Hkv, F32)
-    _need("beta", beta, Hkv, F32)
+    _need("a_q", a_q, B * T * Hr, F32)
+    _need("a_k", a_k, B * T * Hr, F32)
+    _need("alpha", alpha, Hr, F32)
+    _need("beta", beta, Hr, F32)
     _need("out", out, B * T * H * d, act)
     _same_device(q.device, k=k, v=v, g=g, a_q=a_q, a_k=a_k, alpha=alpha, beta=beta, out=out)
     return B, T, H, Hkv, d
@@ -206,9 +214,10 @@ def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0
     b_final may be given as preallocated outputs.  Returns dict(o, lse, b_final, lam) (absent
     outputs are None)."""
     lib = load_library()
-    B, T, H, Hkv, d = _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out)
+    B, T, H, Hkv, d = _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out, variant)
+    Hr = _rate_heads(H, Hkv, variant)
     _need("lse", lse, B * H * T, F32)
-    _need("b_final", b_final, B * Hkv * T, F32)
+    _need("b_final", b_final, B * Hr * T, F32)
     shape = make_shape(q, k, scale, theta, variant, prune_p)
     dev = q.device
     _same_device(dev, lse=lse, b_final=b_final)
@@ -216,9 +225,9 @@ def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0
     if lse is None and want_lse:
         lse = torch.empty(B, H, T, dtype=torch.float32, device=dev)
     if b_final is None and want_bfinal:
-        b_final = torch.empty(B, Hkv, T, dtype=torch.float32, device=dev)
+        b_final = torch.empty(B, Hr, T, dtype=torch.float32, device=dev)
     bfin = b_final
-    lam = torch.empty(B, Hkv, T, T, dtype=torch.float32, device=dev) if want_lambda else None
+    lam = torch.empty(B, Hr, T, T, dtype=torch.float32, device=dev) if want_lambda else None
     need = prefill_workspace_size(shape)
     if ws is None or _nbytes(ws) < need:
         ws = alloc_workspace(need, dev)
@@ -245,12 +254,12 @@ def prefill_fwd_noalloc(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=
     """ua_prefill_fwd_noalloc: the prefill forward using the library's fixed internal scratch
     instead of a workspace (for callers that cannot allocate device memory)."""
     lib = load_library()
-    B, T, H, Hkv, d = _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out)
+    B, T, H, Hkv, d = _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, out, variant)
     shape = make_shape(q, k, scale, theta, variant, prune_p)
     dev = q.device
     o = out if out is not None else torch.empty_like(q)
     lse = torch.empty(B, H, T, dtype=torch.float32, device=dev) if want_lse else None
-    bfin = torch.empty(B, Hkv, T, dtype=torch.float32, device=dev) if want_bfinal else None
+    bfin = torch.empty(B, _rate_heads(H, Hkv, variant), T, dtype=torch.float32, device=dev) if want_bfinal else None
     with _on(dev):   # the library's scratch array is resolved on the current device
         rc = lib.ua_prefill_fwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q),
                                         _ptr(a_k), _ptr(alpha), _ptr(beta), _ptr(o), _ptr(lse), _ptr(bfin),
@@ -271,11 +280,11 @@ def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, d_o, *, scal
     """ua_prefill_bwd (variant: the forward's VAR_* bits).  Returns dict(dq, dk, dv, dg,
     da_q, da_k, dalpha, dbeta)."""
     lib = load_library()
-    B, T, H, Hkv, d = _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, None)
+    B, T, H, Hkv, d = _prefill_dims(q, k, v, g, a_q, a_k, alpha, beta, None, variant)
     _need("o", o, B * T * H * d, (q.dtype,))
     _need("d_o", d_o, B * T * H * d, (q.dtype,))
     _need("lse", lse, B * H * T, F32)
-    _need("b_final", b_final, B * Hkv * T, F32)
+    _need("b_final", b_final, B * _rate_heads(H, Hkv, variant) * T, F32)
     shape = make_shape(q, k, scale, theta, variant)
     dev = q.device
     gr = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),

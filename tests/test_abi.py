@@ -85,7 +85,8 @@ def test_prefill_rejects_null_misaligned_and_small_workspace(lib):
     assert _fwd(lib, _shape(), ws_bytes=need.value - 1) == 4
 
 
-@pytest.mark.parametrize("variant,code", [(16, 1), (7, 1), (15, 1), (-8, 1), (1, 0), (6, 0), (8, 0), (11, 0)])
+@pytest.mark.parametrize("variant,code", [(32, 1), (7, 1), (15, 1), (23, 1), (-8, 1), (1, 0), (6, 0), (8, 0),
+                                          (11, 0), (16, 0), (24, 0)])
 def test_variant_bits_validated(lib, variant, code):
     need = ctypes.c_size_t(0)
     s = _shape(variant=variant)
@@ -254,6 +255,7 @@ def test_binding_constants_match_the_header():
     assert defines["UA_VAR_NO_KEY_DECAY"] == ua.VAR_NO_KEY_DECAY
     assert defines["UA_VAR_NO_SIM_DECAY"] == ua.VAR_NO_SIM_DECAY
     assert defines["UA_VAR_QUERY_NORM"] == ua.VAR_QUERY_NORM
+    assert defines["UA_VAR_PER_HEAD_DECAY"] == ua.VAR_PER_HEAD_DECAY
     assert defines["UA_DECODE_DEFER_COMPACT"] == ua.DECODE_DEFER_COMPACT
     assert re.search(r"UA_F32\s*=\s*0", txt) and re.search(r"UA_BF16\s*=\s*1", txt)
     assert (ua.UA_F32, ua.UA_BF16) == (0, 1)

@@ -1,0 +1,94 @@
+"""GPU parity of per-query-head decay (UA_VAR_PER_HEAD_DECAY) against the oracle's per-head
+forward and backward, through the C ABI.
+
+Every query head gets its own decay logits and similarity parameters (a_q, a_k [B,T,H];
+alpha, beta [H]); the library runs the per-KV-head path with one decay unit per query head on
+keys and values repeated for each group, and sums dk, dv over the copies.  Checked on the bf16
+tensor-core paths (head_dim 64 and 128) and the fp32 SIMT path."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_compression_ua_b200 import inputs as I
+from kv_cache_compression_ua_b200 import ua
+from helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+PH = ua.VAR_PER_HEAD_DECAY
+
+
+def per_head_inputs(w, seed):
+    """Rates per query head: each KV head's repeated over its group and perturbed (seeded), then
+    rounded like every other input."""
+    x = I.make_prefill_inputs(w)
+    G = w.H // w.Hkv
+    rng = np.random.default_rng(seed)
+    for n in ("a_q", "a_k"):
+        x[n] = (np.repeat(x[n], G, axis=2) + 0.5 * rng.standard_normal((w.B, w.T, w.H))).astype(np.float32)
+    for n in ("alpha", "beta"):
+        x[n] = (np.repeat(x[n], G) + 0.5 * rng.standard_normal(w.H)).astype(np.float32)
+    return x
+
+
+def dev(x, dtype):
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    return {n: torch.from_numpy(np.ascontiguousarray(a)).cuda().to(
+        dt if n in ("q", "k", "v", "g", "d_o") else torch.float32).contiguous() for n, a in x.items()}
+
+
+def kernels_ran(fn):
+    ua.profile_reset()
+    ua.profile_enable(True)
+    try:
+        out = fn()
+        torch.cuda.synchronize()
+    finally:
+        ua.profile_enable(False)
+    return out, set(ua.profile_read())
+
+
+CASES = [
+    # (B, T, H, Hkv, d, dtype, forward kernel)
+    (2, 200, 4, 2, 64, "bf16", "k_fwd_tc"),
+    (1, 300, 6, 2, 128, "bf16", "k_fwd_tc128"),
+    (1, 150, 4, 1, 64, "f32", "k_fwd_simt"),
+]
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,d,dtype,kernel", CASES)
+def test_per_head_forward_matches_oracle(B, T, H, Hkv, d, dtype, kernel):
+    w = I.Workload("ph", B, T, H, Hkv, d, dtype, 2600 + T)
+    x = per_head_inputs(w, 2600 + T)
+    dd = dev(x, dtype)
+    r_gpu, names = kernels_ran(lambda: ua.prefill_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["a_q"], dd["a_k"],
+                                                        dd["alpha"], dd["beta"], scale=w.scale, theta=w.theta,
+                                                        variant=PH))
+    assert kernel in names and "k_repeat_kv" in names, names
+    assert ua.get_device_status() == 0
+    assert r_gpu["b_final"].shape == (B, H, T)
+    g = {k: v.float().cpu().numpy() for k, v in r_gpu.items() if v is not None}
+    r = oracle.prefill_fwd_per_head(**x, scale=w.scale, theta=w.theta)
+    assert_close("o", g["o"], r["o"], dtype)
+    assert_close("lse", g["lse"], r["lse"], dtype, relative_max=True)
+    assert_close("b_final", g["b_final"], r["b_final"], dtype, relative_max=True)
+    # the per-head rates matter: the per-KV-head reading of the same tensors differs
+    assert np.max(np.abs(g["b_final"][:, 0] - g["b_final"][:, 1])) > 1e-3
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,d,dtype,kernel", CASES)
+def test_per_head_backward_matches_oracle(B, T, H, Hkv, d, dtype, kernel):
+    w = I.Workload("phb", B, T, H, Hkv, d, dtype, 2700 + T, with_grad=True)
+    x = per_head_inputs(w, 2700 + T)
+    dd = dev(x, dtype)
+    f = ua.prefill_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["a_q"], dd["a_k"], dd["alpha"], dd["beta"],
+                       scale=w.scale, theta=w.theta, variant=PH)
+    gr = ua.prefill_bwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["a_q"], dd["a_k"], dd["alpha"], dd["beta"], f["o"],
+                        f["lse"], f["b_final"], dd["d_o"], scale=w.scale, theta=w.theta, variant=PH)
+    torch.cuda.synchronize()
+    assert ua.get_device_status() == 0
+    assert gr["da_q"].shape == (B, T, H) and gr["dalpha"].shape == (H,) and gr["dk"].shape == (B, T, Hkv, d)
+    g = {k: v.float().cpu().numpy() for k, v in gr.items()}
+    r = oracle.prefill_bwd_per_head(**x, scale=w.scale, theta=w.theta)
+    for n in ("dq", "dk", "dv", "dg", "da_q", "da_k", "dalpha", "dbeta"):
+        assert_close(n, g[n], r[n], dtype, tensor_scale=True)
