@@ -286,13 +286,11 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     const float rq_t = (variant & kVarNoQ) ? 1.f : softplus_f(aq_t);
     const float rk_t = softplus_f(ak_t);          // stored in the cache as is
 
-    float kq[VEC], qh[G][VEC];
+    // the new key stays in registers; the rotated queries are read from shared memory per
+    // entry, which leaves the registers for the next pass's entries (loaded one pass ahead)
+    float kq[VEC];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-        kq[e] = s_kt[gl * VEC + e];
-#pragma unroll
-        for (int h = 0; h < G; ++h) qh[h][e] = s_q[h][gl * VEC + e];
-    }
+    for (int e = 0; e < VEC; ++e) kq[e] = s_kt[gl * VEC + e];
     float m_h[G], l_h[G], acc[G][VEC];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -308,6 +306,24 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     }
     int out = 0;
     const bool multi_pass = n > 4 * EPB;   // block-uniform
+    // Software pipeline: the entries of the next pass are loaded before this pass is processed,
+    // so two passes of loads are in flight.  Safe with the in-place compaction: a survivor of
+    // this pass only ever moves to a slot at or below its own, never into the next pass.
+    uint4 na = make_uint4(0, 0, 0, 0), nb = na, nv = na;
+    float nbj = 0.f, nrk = 0.f;
+    int npj = 0;
+    auto load_entry = [&](int jj) {
+        if (jj < n) {
+            const size_t e = (base + jj) * DH + gl * VEC;
+            na = *reinterpret_cast<const uint4*>(khat + e);
+            nb = *reinterpret_cast<const uint4*>(krope + e);
+            nv = *reinterpret_cast<const uint4*>(vc + e);
+            nbj = c.bias[base + jj];
+            nrk = c.rk[base + jj];
+            npj = c.pos[base + jj];
+        }
+    };
+    load_entry(gidx);
     for (int c0 = 0; c0 < n; c0 += EPB) {
         const int j = c0 + gidx;
         const bool valid = j < n;
@@ -330,18 +346,10 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
                 }
             }
         }
-        uint4 ra = make_uint4(0, 0, 0, 0), rb = ra, rv = ra;
-        float bj = 0.f, rkj = 0.f;
-        int pj = 0;
-        if (valid) {
-            const size_t e = (base + j) * DH + gl * VEC;
-            ra = *reinterpret_cast<const uint4*>(khat + e);
-            rb = *reinterpret_cast<const uint4*>(krope + e);
-            rv = *reinterpret_cast<const uint4*>(vc + e);
-            bj = c.bias[base + j];
-            rkj = c.rk[base + j];
-            pj = c.pos[base + j];
-        }
+        const uint4 ra = na, rb = nb, rv = nv;
+        const float bj = nbj, rkj = nrk;
+        const int pj = npj;
+        load_entry(j + EPB);
         float xa[VEC], xb[VEC], xv[VEC];
         Vec16<TC>::unpack(ra, xa);
         Vec16<TC>::unpack(rb, xb);
@@ -357,7 +365,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         for (int h = 0; h < G; ++h) {
             float lg = 0.f;
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) lg = fmaf(qh[h][e], xb[e], lg);
+            for (int e = 0; e < VEC; ++e) lg = fmaf(s_q[h][gl * VEC + e], xb[e], lg);
             lg = group_sum<LPE>(lg);
             if (keep) {
                 lg = fmaf(lg, p.scale, bnew);
