@@ -830,11 +830,12 @@ k_bwd_gemm_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__
         }
     } else if (warp == 1) {
         const bool leader = elect_one();
-        // rows side: A = K^T (MN-major SW128, M = dims: 64-dim atoms 16384 B apart, or the zero
-        // block), B = tiles as [128 rows x 128 keys] (MN-major no swizzle: 8-row groups 2048 B
-        // apart, 8-key groups 128 B apart); key side: A = tiles as [128 keys x 128 rows]
-        // (K-major no swizzle: 8-row groups 2048 B apart, 8-key groups 128 B apart), B = khat rows
-        // (MN-major SW128, N = dims).
+        // rows side: A = K^T (MN-major SW128, M = dims: 64-dim atoms 16384 B apart = the leading
+        // byte offset, or the zero block), B = tiles as [128 rows x 128 keys] (MN-major, no swizzle:
+        // there the leading byte offset is the K-direction step, 8-key groups 128 B apart, and the
+        // stride byte offset the MN-direction step, 8-row groups 2048 B apart); key side: A = tiles
+        // as [128 keys x 128 rows] (K-major, no swizzle: leading = K step, 8-row groups 2048 B
+        // apart; stride = M step, 8-key groups 128 B apart), B = khat rows (MN-major SW128, N = dims).
         constexpr uint32_t ID = ROWS ? idesc_bf16(128, 128, 1, 1) : idesc_bf16(128, DH, 0, 1);
         bool ok = true;
         for (int i = 0; i < n && ok; ++i) {
@@ -849,7 +850,7 @@ k_bwd_gemm_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__
                     const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
                     if (ROWS) {
                         const uint64_t da = smem_desc(aa + kk * 2048u, lbo_a, 1024, kSwizzle128B);
-                        const uint64_t db = smem_desc(ta + kk * 256u, 2048, 128, kSwizzleNone);
+                        const uint64_t db = smem_desc(ta + kk * 256u, 128, 2048, kSwizzleNone);
                         umma_f16(tmem, da, db, ID, acc);
                     } else {
                         const uint64_t da = smem_desc(ta + kk * 4096u, 2048, 128, kSwizzleNone);
