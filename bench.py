@@ -488,6 +488,63 @@ def bench_decode(args, peaks, peaks_kind):
             res[key]["ak_slow_mean"] = I.DECODE_RETAINED_AK_SLOW_MEAN
         del g, cache, snap
         torch.cuda.empty_cache()
+    # Split walk for few long caches (supplementary): one sequence (B=1, 8 KV heads, p = 0: 16.4k
+    # live pairs per head, compaction deferred) decoded by one CTA per cache and by the split step
+    # (up to 16 CTAs per cache), both graph-captured.
+    xs = {n: x[n][:1].contiguous() for n in ("k", "v", "a_k")}
+    bf1 = bfinal[:1].contiguous()
+    tk1 = {n: t[:, :1].contiguous() for n, t in tok.items()}
+    split_res = {}
+    for mode in ("one CTA per cache", "split"):
+        cache = ua.Cache.empty(1, w.Hkv, w.d, cap, torch.bfloat16)
+        ua.cache_fill(cache, xs["k"], xs["v"], xs["a_k"], bf1, theta=w.theta)
+        ua.cache_compact(cache, 0.0)
+        snap = {n: getattr(cache, n).clone() for n in ("khat", "krope", "v", "bias", "rk", "pos", "n_kept")}
+        n0 = int(cache.n_kept.sum().item())
+        o = torch.empty(steps, 1, w.H, w.d, dtype=torch.bfloat16, device="cuda")
+        ws = ua.alloc_workspace(ua.decode_workspace_size(cache, w.H), "cuda") if mode == "split" else None
+
+        def run1(stream=None):
+            for s in range(steps):
+                ua.decode_step(cache, tk1["q"][s], tk1["k"][s], tk1["v"][s], tk1["g"][s], tk1["a_q"][s],
+                               tk1["a_k"][s], x["alpha"], x["beta"], T0 + s, 0.0, scale=w.scale, theta=w.theta,
+                               out=o[s], defer_compact=True, ws=ws, stream=stream)
+
+        def restore1():
+            for n, t in snap.items():
+                getattr(cache, n).copy_(t)
+        g = torch.cuda.CUDAGraph()
+        s_cap = torch.cuda.Stream()
+        s_cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s_cap):
+            run1(s_cap)
+        torch.cuda.current_stream().wait_stream(s_cap)
+        torch.cuda.synchronize()
+        restore1()
+        with torch.cuda.graph(g, stream=s_cap):
+            run1(s_cap)
+        times = []
+        for it in range(3 + 5):
+            restore1()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            if it >= 3:
+                times.append(e0.elapsed_time(e1))
+        assert ua.get_device_status() == 0
+        ms = statistics.median(times)
+        byts = sum((n0 + w.Hkv * s) * entry_bytes + (n0 + w.Hkv * (s + 1)) * 4 for s in range(steps))
+        split_res[mode] = {"us_per_step": 1e3 * ms / steps, "tokens_per_s": steps / (ms * 1e-3),
+                           "hbm_gbs": byts / (ms * 1e-3) / 1e9,
+                           "hbm_frac": byts / (ms * 1e-3) / 1e9 / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])}
+        del g, cache, snap
+        torch.cuda.empty_cache()
+    split_res["workload"] = (f"decode_1b batch 0 only: B=1, {w.Hkv} KV heads, p=0 (16.4k live pairs per head), "
+                             f"{steps} steps, deferred compaction, graph-captured")
+    res["few_long_caches (supplementary)"] = split_res
     res["peak_source"] = f"{peaks_kind} HBM copy bandwidth"
     res["workload"] = f"decode_1b: B={w.B}, 16k prefill, {steps} steps, graph-captured"
     return res

@@ -192,8 +192,14 @@ ua_status ua_prefill_tile_stats(const ua_shape* shape, const void* ws, size_t ws
  * and is not read (the decay prefixes are recomputed).  d_o: [B,T,H,d] act.
  * Outputs: dq, dg [B,T,H,d] act; dk, dv [B,T,Hkv,d] act; da_q, da_k [B,T,Hkv] f32;
  * dalpha, dbeta [Hkv] f32 (summed over the batch).  All outputs are overwritten; the result
- * is deterministic (no atomics).  Runs as fp32 SIMT kernels.  Training is dense: a shape
- * with prune_p != 0 is UA_ERR_INVALID_ARG. */
+ * is deterministic (no atomics).  bf16 problems with d = 64 (H/Hkv <= 4) or d = 128
+ * (H/Hkv <= 3) of the three-rate method (the query norm allowed) run on the tensor cores: the
+ * decay prefixes above every 32-row step, a key-major pass that accumulates dv and the rotated
+ * key gradient in TMEM and stores the bf16 dZ / dX tiles of the causal band, and tensor-core
+ * GEMMs for the query and similarity gradients (the workspace holds the band: about
+ * (G+1) * 2 bytes per causal pair and KV head).  Similarities are formed from the unit keys
+ * split into two bf16 parts (~16 significant bits).  Other problems run as fp32 SIMT kernels.
+ * Training is dense: a shape with prune_p != 0 is UA_ERR_INVALID_ARG. */
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes);
 
 ua_status ua_prefill_bwd(const ua_shape* shape, const void* q, const void* k, const void* v,
@@ -269,6 +275,25 @@ ua_status ua_decode_step(const ua_cache* cache, int H, const void* q, const void
                          const float* alpha, const float* beta, int pos_t, float p, float scale,
                          double rope_theta, void* o, uint32_t* evict_bits, int32_t* kept_idx,
                          int flags, void* stream);
+
+/* ------------------------------------------------------------------ split decode step
+ * The same step as ua_decode_step with UA_DECODE_DEFER_COMPACT (set or not in flags), for few
+ * long caches: a cache of n live slots is walked by min(16, ceil(n / 512)) CTAs at once, each
+ * over a slice of whole 32-slot words, instead of by one (the pages' App. H asks for fused,
+ * specialised kernels for the pruned cache; a single CTA per cache leaves most of the GPU idle
+ * when B * Hkv is small and the caches long).  Each CTA updates its slots' biases in place and
+ * leaves a partial softmax state in the workspace; the last one to finish merges them with the
+ * new token, gates, writes o and appends the token at slot n.  evict_bits and kept_idx follow the
+ * deferred-compaction rules of ua_decode_step; evicted pairs stay until ua_cache_compact.
+ * ws: device workspace of ua_decode_workspace_size bytes (256-byte aligned), scratch only; calls
+ * that share a workspace must not overlap on the GPU.  A short cache (n <= 512) takes one CTA, as
+ * ua_decode_step does. */
+ua_status ua_decode_workspace_size(const ua_cache* cache, int H, size_t* bytes);
+ua_status ua_decode_step_split(const ua_cache* cache, int H, const void* q, const void* k, const void* v,
+                               const void* g, const float* a_q, const float* a_k, const float* alpha,
+                               const float* beta, int pos_t, float p, float scale, double rope_theta, void* o,
+                               uint32_t* evict_bits, int32_t* kept_idx, int flags, void* ws, size_t ws_bytes,
+                               void* stream);
 
 /* ------------------------------------------------------------------ status
  * Synchronises `stream`, returns the device status word accumulated since the last call

@@ -206,7 +206,9 @@ namespace bnd {
 template <int DH>
 struct Smem {
     alignas(1024) uint8_t khk[DH / 64][16384];      // khat of the key tile, boxes [128][64]
+    alignas(1024) uint8_t khk_lo[DH / 64][16384];   // its bf16 residual
     alignas(1024) uint8_t kq[2][DH / 64][4096];     // khat of the step's rows, boxes [32][64]
+    alignas(1024) uint8_t kq_lo[2][DH / 64][4096];  // their residual
     alignas(128) float lq[2][ST];
     alignas(128) float lk[128];
     alignas(8) uint64_t kfull, qfull[2], xfull[2];
@@ -218,6 +220,8 @@ struct Smem {
 template <int DH>
 __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CUtensorMap tm_khk,
                                                       const __grid_constant__ CUtensorMap tm_khq,
+                                                      const __grid_constant__ CUtensorMap tm_khk_lo,
+                                                      const __grid_constant__ CUtensorMap tm_khq_lo,
                                                       const __grid_constant__ CUtensorMap tm_lq,
                                                       const __grid_constant__ CUtensorMap tm_lk, BwdTcParams p) {
     constexpr uint32_t ID_X = idesc_bf16(128, ST, 0, 0);
@@ -250,21 +254,32 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
     const bool leader = warp == 0 && elect_one();
     auto load_step = [&](int it) {
         const int st = it & 1, s = s0 + it;
-        mbar_expect_tx(&S.qfull[st], NB * 4096 + ST * 4);
-        for (int c = 0; c < NB; ++c) tma_load_3d(S.kq[st][c], &tm_khq, &S.qfull[st], 64 * c, s * ST, unit);
+        mbar_expect_tx(&S.qfull[st], 2 * NB * 4096 + ST * 4);
+        for (int c = 0; c < NB; ++c) {
+            tma_load_3d(S.kq[st][c], &tm_khq, &S.qfull[st], 64 * c, s * ST, unit);
+            tma_load_3d(S.kq_lo[st][c], &tm_khq_lo, &S.qfull[st], 64 * c, s * ST, unit);
+        }
         tma_load_2d(S.lq[st], &tm_lq, &S.qfull[st], s * ST, unit);
     };
+    // X^T from the split keys: hi hi^T + hi lo^T + lo hi^T (the lo lo^T term is below fp32 rounding)
     auto issue_x = [&](int it) {
         const int st = it & 1;
-        const uint32_t a = smem_u32(S.khk[0]), bq = smem_u32(S.kq[st][0]);
+        const uint32_t a = smem_u32(S.khk[0]), al = smem_u32(S.khk_lo[0]);
+        const uint32_t bq = smem_u32(S.kq[st][0]), bl = smem_u32(S.kq_lo[st][0]);
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk)
+        for (int kk = 0; kk < DH / 16; ++kk) {
             umma_f16(tmem + st * 32, kdesc_rows(a, 128, kk), kdesc_rows(bq, ST, kk), ID_X, kk > 0);
+            umma_f16(tmem + st * 32, kdesc_rows(a, 128, kk), kdesc_rows(bl, ST, kk), ID_X, 1);
+            umma_f16(tmem + st * 32, kdesc_rows(al, 128, kk), kdesc_rows(bq, ST, kk), ID_X, 1);
+        }
         umma_commit(&S.xfull[st]);
     };
     if (leader) {
-        mbar_expect_tx(&S.kfull, NB * 16384 + 512);
-        for (int c = 0; c < NB; ++c) tma_load_3d(S.khk[c], &tm_khk, &S.kfull, 64 * c, kt * 128, unit);
+        mbar_expect_tx(&S.kfull, 2 * NB * 16384 + 512);
+        for (int c = 0; c < NB; ++c) {
+            tma_load_3d(S.khk[c], &tm_khk, &S.kfull, 64 * c, kt * 128, unit);
+            tma_load_3d(S.khk_lo[c], &tm_khk_lo, &S.kfull, 64 * c, kt * 128, unit);
+        }
         tma_load_2d(S.lk, &tm_lk, &S.kfull, kt * 128, unit);
         load_step(0);
         if (nsteps > 1) load_step(1);
@@ -339,22 +354,24 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
 namespace key {
 template <int DH, int G>
 struct Smem {
-    alignas(1024) uint8_t khk[DH / 64][16384];   // khat / krot / v of the key tile, boxes [128][64]
+    alignas(1024) uint8_t khk[DH / 64][16384];   // khat (and its bf16 residual) / krot / v of the key
+    alignas(1024) uint8_t khk_lo[DH / 64][16384];// tile, boxes [128][64]
     alignas(1024) uint8_t krk[DH / 64][16384];
     alignas(1024) uint8_t vk[DH / 64][16384];
-    alignas(1024) uint8_t kq[2][DH / 64][4096];  // khat of the step's rows, boxes [32][64], two stages
+    alignas(1024) uint8_t kq[DH / 64][4096];     // khat of the step's rows and its residual, boxes [32][64]
+    alignas(1024) uint8_t kq_lo[DH / 64][4096];
     alignas(1024) uint8_t qh[G][DH / 64][4096];  // qrot / dA of the step's rows, per head
     alignas(1024) uint8_t ah[G][DH / 64][4096];
-    alignas(1024) uint8_t tp[2][kTileBytes];     // P_h^T and dZ_h^T tiles (K-major, no swizzle), head parity
-    alignas(1024) uint8_t tz[2][kTileBytes];
-    alignas(128) float lq[2][ST];                // log2 rate / 3 of the step's rows (with kq)
-    alignas(128) float pbv[2][128];              // decay prefix above the step (with kq)
+    alignas(1024) uint8_t tp[kTileBytes];        // P_h^T and dZ_h^T tiles (K-major, no swizzle)
+    alignas(1024) uint8_t tz[kTileBytes];
+    alignas(128) float lq[ST];                   // log2 rate / 3 of the step's rows (with kq)
+    alignas(128) float pbv[128];                 // decay prefix above the step (with kq)
     alignas(128) float lse2[G][ST];              // per head (with qh / ah)
     alignas(128) float dlt[G][ST];
     alignas(128) float lk[128];
     alignas(16) float red[2][4];
-    alignas(8) uint64_t kfull, qfull[2], qempty[2], xfull, xempty, hfull[G], hdone[G], pfull[2], pempty[2],
-        tfull[2], tempty[2], accdone;
+    alignas(8) uint64_t kfull, qfull, qempty, xfull, xempty, hfull[G], hdone[G], pfull[2], pempty[2], tfull,
+        tempty, accdone;
     uint32_t tmem;
     int abort;
 };
@@ -364,6 +381,7 @@ template <int DH, int G>
 __global__ void __launch_bounds__(160, 1)
 k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__ CUtensorMap tm_krk,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_khq,
+             const __grid_constant__ CUtensorMap tm_khk_lo, const __grid_constant__ CUtensorMap tm_khq_lo,
              const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ad,
              const __grid_constant__ CUtensorMap tm_lq, const __grid_constant__ CUtensorMap tm_lk,
              const __grid_constant__ CUtensorMap tm_pb, const __grid_constant__ CUtensorMap tm_lse2,
@@ -386,13 +404,13 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         mbar_init(&S.xfull, 1);
         mbar_init(&S.xempty, 4);
         mbar_init(&S.accdone, 1);
+        mbar_init(&S.qfull, 1);
+        mbar_init(&S.qempty, 4);
+        mbar_init(&S.tfull, 4);
+        mbar_init(&S.tempty, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.qfull[i], 1);
-            mbar_init(&S.qempty[i], 4);
             mbar_init(&S.pfull[i], 1);
             mbar_init(&S.pempty[i], 4);
-            mbar_init(&S.tfull[i], 4);
-            mbar_init(&S.tempty[i], 1);
         }
         for (int h = 0; h < G; ++h) {
             mbar_init(&S.hfull[h], 1);
@@ -414,14 +432,19 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         // ------------------------------------------------ TMA + MMA issue (one elected lane)
         const bool leader = elect_one();
         bool ok = true;
-        // step it covers rows of step s = nst-1-it
+        // step it covers rows of step s = nst-1-it.  The step's khat rows (and residual), lq and
+        // the prefix vector have one buffer: X^T is the first MMA of a step, so they are free
+        // early and the next step's copy overlaps the rest of this one.
         auto load_q = [&](int it) {
-            const int st = it & 1, s = p.nst - 1 - it;
+            const int s = p.nst - 1 - it;
             if (leader) {
-                mbar_expect_tx(&S.qfull[st], NB * 4096 + ST * 4 + 128 * 4);
-                for (int c = 0; c < NB; ++c) tma_load_3d(S.kq[st][c], &tm_khq, &S.qfull[st], 64 * c, s * ST, unit);
-                tma_load_2d(S.lq[st], &tm_lq, &S.qfull[st], s * ST, unit);
-                tma_load_2d(S.pbv[st], &tm_pb, &S.qfull[st], kt * 128, unit * p.nst + s);
+                mbar_expect_tx(&S.qfull, 2 * NB * 4096 + ST * 4 + 128 * 4);
+                for (int c = 0; c < NB; ++c) {
+                    tma_load_3d(S.kq[c], &tm_khq, &S.qfull, 64 * c, s * ST, unit);
+                    tma_load_3d(S.kq_lo[c], &tm_khq_lo, &S.qfull, 64 * c, s * ST, unit);
+                }
+                tma_load_2d(S.lq, &tm_lq, &S.qfull, s * ST, unit);
+                tma_load_2d(S.pbv, &tm_pb, &S.qfull, kt * 128, unit * p.nst + s);
             }
             __syncwarp();
         };
@@ -439,9 +462,10 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             __syncwarp();
         };
         if (leader) {
-            mbar_expect_tx(&S.kfull, 3 * NB * 16384 + 512);
+            mbar_expect_tx(&S.kfull, 4 * NB * 16384 + 512);
             for (int c = 0; c < NB; ++c) {
                 tma_load_3d(S.khk[c], &tm_khk, &S.kfull, 64 * c, kt * 128, unit);
+                tma_load_3d(S.khk_lo[c], &tm_khk_lo, &S.kfull, 64 * c, kt * 128, unit);
                 tma_load_3d(S.krk[c], &tm_krk, &S.kfull, 64 * c, kt * 128, unit);
                 tma_load_4d(S.vk[c], &tm_v, &S.kfull, 64 * c, kvh, kt * 128, b);
             }
@@ -449,32 +473,35 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         }
         __syncwarp();
         load_q(0);
-        if (nsteps > 1) load_q(1);
         for (int h = 0; h < G; ++h) load_h(0, h);
         ok = wwait(&S.kfull, 0, abort);
-        const uint32_t akh = smem_u32(S.khk[0]), akr = smem_u32(S.krk[0]), av = smem_u32(S.vk[0]);
+        const uint32_t akh = smem_u32(S.khk[0]), akl = smem_u32(S.khk_lo[0]);
+        const uint32_t akr = smem_u32(S.krk[0]), av = smem_u32(S.vk[0]);
+        const uint32_t bq = smem_u32(S.kq[0]), bql = smem_u32(S.kq_lo[0]);
         bool first_acc = true;
         for (int it = 0; ok && it < nsteps; ++it) {
-            const int st = it & 1;
-            // X^T of the step
-            if (!wwait(&S.qfull[st], (it >> 1) & 1, abort)) break;
+            // X^T of the step from the split keys: hi hi^T + hi lo^T + lo hi^T, so the similarity
+            // (whose gradient dalpha sums with heavy cancellation) carries ~16 significant bits
+            if (!wwait(&S.qfull, it & 1, abort)) break;
             if (it >= 1 && !wwait(&S.xempty, (it - 1) & 1, abort)) break;
             tc_fence_after();
             if (leader) {
-                const uint32_t bq = smem_u32(S.kq[st][0]);
 #pragma unroll
-                for (int kk = 0; kk < DH / 16; ++kk)
+                for (int kk = 0; kk < DH / 16; ++kk) {
                     umma_f16(tmem + COL_X, kdesc_rows(akh, 128, kk), kdesc_rows(bq, ST, kk), ID_L, kk > 0);
+                    umma_f16(tmem + COL_X, kdesc_rows(akh, 128, kk), kdesc_rows(bql, ST, kk), ID_L, 1);
+                    umma_f16(tmem + COL_X, kdesc_rows(akl, 128, kk), kdesc_rows(bq, ST, kk), ID_L, 1);
+                }
                 umma_commit(&S.xfull);
             }
             __syncwarp();
             // accumulation of head hh of this step: dV += P^T dA, dKrot += dZ^T qrot
             auto accum = [&](int hh) -> bool {
-                const uint32_t v = (uint32_t)(it * G + hh), tb = v & 1;
-                if (!wwait(&S.tfull[tb], (v >> 1) & 1, abort)) return false;
+                const uint32_t v = (uint32_t)(it * G + hh);
+                if (!wwait(&S.tfull, v & 1, abort)) return false;
                 tc_fence_after();
                 if (leader) {
-                    const uint32_t tpa = smem_u32(S.tp[tb]), tza = smem_u32(S.tz[tb]);
+                    const uint32_t tpa = smem_u32(S.tp), tza = smem_u32(S.tz);
                     const uint32_t ba = smem_u32(S.ah[hh][0]), bqh = smem_u32(S.qh[hh][0]);
 #pragma unroll
                     for (int kk = 0; kk < ST / 16; ++kk) {
@@ -489,7 +516,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                         umma_f16(tmem + COL_DV, da, db, ID_ACC, acc);
                         umma_f16(tmem + COL_DK, dz, dq, ID_ACC, acc);
                     }
-                    umma_commit(&S.tempty[tb]);
+                    umma_commit(&S.tempty);
                     umma_commit(&S.hdone[hh]);
                 }
                 __syncwarp();
@@ -513,6 +540,12 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                     umma_commit(&S.pfull[pp]);
                 }
                 __syncwarp();
+                if (h == 0 && it + 1 < nsteps) {
+                    // the step's khat rows, lq and prefixes are free once the compute warps have
+                    // read X^T and the vectors: copy the next step's
+                    if (!wwait(&S.qempty, it & 1, abort)) { ok = false; break; }
+                    load_q(it + 1);
+                }
                 if (h >= 1) {
                     if (!accum(h - 1)) { ok = false; break; }
                     // head h-1's operands are free once its accumulation completed: refill them
@@ -524,11 +557,6 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             }
             if (!ok) break;
             if (!accum(G - 1)) break;
-            if (it + 2 < nsteps) {
-                // stage st (khat rows, lq, pb) is free once the compute warps have read it
-                if (!wwait(&S.qempty[st], (it >> 1) & 1, abort)) break;
-                load_q(it + 2);
-            }
             if (it + 1 < nsteps) {
                 if (!wwait(&S.hdone[G - 1], it & 1, abort)) break;
                 load_h(it + 1, G - 1);
@@ -552,10 +580,10 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         uint8_t* tile_base = static_cast<uint8_t*>(p.tiles) + (size_t)unit * (G + 1) * tstride;
         const size_t band = band_off(kt, p.nkt);
         for (int it = 0; ok && it < nsteps; ++it) {
-            const int st = it & 1, s = p.nst - 1 - it;
+            const int s = p.nst - 1 - it;
             const int i0 = s * ST;
-            if (!wwait(&S.qfull[st], (it >> 1) & 1, abort)) { ok = false; break; }
-            const float pbj = S.pbv[st][jl];
+            if (!wwait(&S.qfull, it & 1, abort)) { ok = false; break; }
+            const float pbj = S.pbv[jl];
             if (!wwait(&S.xfull, it & 1, abort)) { ok = false; break; }
             tc_fence_after();
             uint32_t x[32];
@@ -573,7 +601,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 float c = 0.f;
 #pragma unroll
                 for (int r = 0; r < 32; r += 4) {
-                    const float4 lv = *reinterpret_cast<const float4*>(&S.lq[st][r]);
+                    const float4 lv = *reinterpret_cast<const float4*>(&S.lq[r]);
                     const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -591,7 +619,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&S.xempty);
-                mbar_arrive(&S.qempty[st]);
+                mbar_arrive(&S.qempty);
             }
             float dlam[32];
 #pragma unroll
@@ -621,10 +649,10 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.pempty[pp]);
-                const uint32_t tb = u & 1;
-                if (u >= 2 && !wwait(&S.tempty[tb], ((u >> 1) - 1) & 1, abort)) { ok = false; break; }
-                uint8_t* ttp = S.tp[tb];
-                uint8_t* ttz = S.tz[tb];
+                // the P / dZ tiles are free once the previous head's accumulation completed
+                if (u >= 1 && !wwait(&S.tempty, (u - 1) & 1, abort)) { ok = false; break; }
+                uint8_t* ttp = S.tp;
+                uint8_t* ttz = S.tz;
                 uint4* gz = reinterpret_cast<uint4*>(tile_base + (size_t)h * tstride + (band + (s - s0)) * kTileBytes);
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
@@ -658,7 +686,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S.tfull[tb]);
+                if (lane == 0) mbar_arrive(&S.tfull);
             }
             if (!ok) break;
             // dD = -(sum of dLambda over the rows at and below l), bottom up; w = dD D / 3
@@ -1043,10 +1071,13 @@ __global__ void __launch_bounds__(256) k_bwd_post_tc(BwdTcParams p) {
 }
 
 // =========================================================================== launcher
-bool bwd_tc_supported(int d, int G) { return (d == 64 || d == 128) && G >= 1 && G <= 4; }
+// head_dim 128 with four query heads per KV head does not fit the key-major pass's shared
+// memory (the step's query and dA rows of four heads beside the key tile's four operands)
+bool bwd_tc_supported(int d, int G) { return (d == 64 && G >= 1 && G <= 4) || (d == 128 && G >= 1 && G <= 3); }
 
 template <int DH, int G>
 static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
+    static_assert(sizeof(key::Smem<DH, G>) + 1024 <= 232448, "key-major pass: shared memory budget");
     const int BH = p.B * p.H, BK = p.B * p.Hkv;
     cudaError_t e;
     {
@@ -1054,7 +1085,9 @@ static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
         k_bwd_prep_tc<DH><<<dim3(p.T, p.B), 256, 0, s>>>(p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    CUtensorMap m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk, m_pb, m_lse2, m_dlt, m_kh128;
+    CUtensorMap m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk, m_pb, m_lse2, m_dlt, m_kh128, m_khk_lo, m_khq_lo;
+    if (!map_rows_bwd(&m_khk_lo, p.kh_lo, DH, p.T, BK, 128) || !map_rows_bwd(&m_khq_lo, p.kh_lo, DH, p.T, BK, ST))
+        return cudaErrorInvalidValue;
     if (!map_rows_bwd(&m_khk, p.kh, DH, p.T, BK, 128) || !map_rows_bwd(&m_krk, p.kr, DH, p.T, BK, 128) ||
         !map_v_bwd(&m_v, p.v, DH, p.Hkv, p.T, p.B) || !map_rows_bwd(&m_khq, p.kh, DH, p.T, BK, ST) ||
         !map_rows_bwd(&m_q, p.qr, DH, p.T, BH, ST) || !map_rows_bwd(&m_ad, p.ad, DH, p.T, BH, ST) ||
@@ -1069,7 +1102,7 @@ static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
             cudaSuccess)
             return e;
         UA_PROFILE("k_bwd_bound_tc", s);
-        k_bwd_bound_tc<DH><<<dim3(p.nkt, BK), 128, smem, s>>>(m_khk, m_khq, m_lq, m_lk, p);
+        k_bwd_bound_tc<DH><<<dim3(p.nkt, BK), 128, smem, s>>>(m_khk, m_khq, m_khk_lo, m_khq_lo, m_lq, m_lk, p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {
@@ -1078,8 +1111,8 @@ static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
             cudaSuccess)
             return e;
         UA_PROFILE("k_bwd_key_tc", s);
-        k_bwd_key_tc<DH, G><<<dim3(p.nkt, BK), 160, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk,
-                                                               m_pb, m_lse2, m_dlt, p);
+        k_bwd_key_tc<DH, G><<<dim3(p.nkt, BK), 160, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_khk_lo, m_khq_lo, m_q,
+                                                               m_ad, m_lq, m_lk, m_pb, m_lse2, m_dlt, p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {
@@ -1119,7 +1152,9 @@ static cudaError_t bwd_tc_g(const BwdTcParams& p, cudaStream_t s) {
         case 1: return bwd_tc_inst<DH, 1>(p, s);
         case 2: return bwd_tc_inst<DH, 2>(p, s);
         case 3: return bwd_tc_inst<DH, 3>(p, s);
-        case 4: return bwd_tc_inst<DH, 4>(p, s);
+        case 4:
+            if constexpr (DH == 64) return bwd_tc_inst<DH, 4>(p, s);
+            return cudaErrorInvalidValue;
         default: return cudaErrorInvalidValue;
     }
 }

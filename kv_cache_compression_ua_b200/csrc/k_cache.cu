@@ -11,6 +11,8 @@
 // Layout: one structure-of-arrays cache per (batch, KV head), slots in ascending token
 // order.  An entry is read by a group of LPE lanes, each moving 16 bytes of khat, krope and v
 // (128-bit coalesced loads); dot products reduce across the group with shuffles.
+#include <algorithm>
+
 #include "ua_common.cuh"
 #include "ua_kernels.h"
 #include "ua_profile.h"
@@ -463,6 +465,257 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     }
 }
 
+// ------------------------------------------------------------------ split decode step
+// grid (kDecodeSplitMax, B*Hkv), 256 threads.  A long cache is walked by several CTAs at once:
+// slice s of S = min(kDecodeSplitMax, ceil(n / kDecodeSplitSlice)) covers pairs [lo, hi) (whole
+// 32-pair words); CTAs past S leave at once, so a short cache costs one CTA as before.  Each CTA
+// updates its pairs' biases in place, marks its evictions, and leaves its partial online-softmax
+// state (per head: maximum, sum, weighted values) in the workspace; the CTA that finishes last
+// (a counter per cache; a fence before every arrival) merges the S states with the new token's
+// own term, gates, writes o and appends the token.  Compaction is deferred: pairs keep their
+// slots, evicted ones are excluded by their bias until ua_cache_compact removes them.  No CTA
+// ever waits on another.
+template <typename TC, int DH, int G, bool VAR>
+__global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodeParams p) {
+    const int variant = VAR ? p.variant : 0;
+    using L = EntryLayout<TC, DH>;
+    constexpr int VEC = L::VEC, LPE = L::LPE, EPB = L::EPB, NW = L::NW;
+    constexpr int half = DH / 2;
+    constexpr int SS = G * (DH + 2);                  // floats of one partial state
+    __shared__ float s_kt[DH], s_ktr[DH], s_vt[DH], s_q[G][DH], s_lt[G], s_g[G * DH], s_qn[G];
+    __shared__ float s_red[NW];
+    __shared__ float s_m[EPB * G], s_l[EPB * G];
+    __shared__ int s_last;
+    extern __shared__ float dsm[];
+    float* s_acc = dsm;                               // [EPB][G][DH]
+    uint32_t* s_ev = reinterpret_cast<uint32_t*>(dsm + (size_t)EPB * G * DH);   // the slice's words
+    const CacheView& c = p.c;
+    const int words = (c.cap + 31) / 32;
+    const int unit = blockIdx.y, sl = blockIdx.x, b = unit / c.Hkv, kvh = unit % c.Hkv;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = lane / LPE, gl = lane % LPE;
+    const int gidx = warp * L::EPW + grp;
+    const size_t base = (size_t)unit * c.cap;
+    TC* khat = static_cast<TC*>(c.khat);
+    TC* krope = static_cast<TC*>(c.krope);
+    TC* vc = static_cast<TC*>(c.v);
+
+    int n = c.n_kept[unit];
+    if (n < 0 || n > c.cap) {                 // corrupt count: never read past the cache
+        if (tid == 0 && sl == 0) raise_status(UA_ERR_CAPACITY);
+        n = n < 0 ? 0 : c.cap;
+    }
+    const int nsl = min(kDecodeSplitMax, max(1, (n + kDecodeSplitSlice - 1) / kDecodeSplitSlice));
+    if (sl >= nsl) return;                            // block-uniform
+    const int chunk = (((n + nsl - 1) / nsl) + 31) & ~31;
+    const int lo = min(n, sl * chunk), hi = min(n, lo + chunk);
+    const int w0 = lo >> 5, nw = (hi - lo + 31) >> 5;
+
+    // ---- new token (every CTA of the cache forms it; only the last one uses v, g)
+    const TC* kin = static_cast<const TC*>(p.k) + (size_t)unit * DH;
+    const TC* vin = static_cast<const TC*>(p.v) + (size_t)unit * DH;
+    const TC* qin = static_cast<const TC*>(p.q) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
+    const TC* gin = static_cast<const TC*>(p.g) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
+    float kx = 0.f;
+    if (tid < DH) {
+        kx = Elem<TC>::ld(kin + tid);
+        s_vt[tid] = Elem<TC>::ld(vin + tid);
+    }
+    for (int e = tid; e < G * DH; e += blockDim.x) s_g[e] = Elem<TC>::ld(gin + e);
+    for (int w = tid; w < nw; w += blockDim.x) s_ev[w] = 0u;
+    float ss = kx * kx;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) s_red[warp] = ss;
+    __syncthreads();
+    float tot_ss = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) tot_ss += s_red[w];
+    const float den = fmaxf(sqrtf(tot_ss), 1e-12f);
+    if (tid < DH) s_kt[tid] = kx / den;
+    __syncthreads();
+    for (int e = tid; e < G * half; e += blockDim.x) {
+        const int vecid = e / half, m = e % half;
+        float cs, sn;
+        rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
+        const float qa = Elem<TC>::ld(qin + vecid * DH + m), qb = Elem<TC>::ld(qin + vecid * DH + m + half);
+        s_q[vecid][m] = qa * cs - qb * sn;
+        s_q[vecid][m + half] = qb * cs + qa * sn;
+    }
+    for (int m = tid; m < half; m += blockDim.x) {
+        float cs, sn;
+        rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
+        const float x0 = s_kt[m], x1 = s_kt[m + half];
+        s_ktr[m] = x0 * cs - x1 * sn;
+        s_ktr[m + half] = x1 * cs + x0 * sn;
+    }
+    __syncthreads();
+    if (variant & kVarQNorm) {
+        if (tid < G) {
+            float qq = 0.f;
+            for (int x = 0; x < DH; ++x) qq = fmaf(s_q[tid][x], s_q[tid][x], qq);
+            s_qn[tid] = 1.f / sqrtf(qq * (1.f / DH) + kQNormEps);
+        }
+        __syncthreads();
+        for (int e = tid; e < G * DH; e += blockDim.x) s_q[e / DH][e % DH] *= s_qn[e / DH];
+        __syncthreads();
+    }
+    if (tid < G) {
+        float a = 0.f;
+        for (int x = 0; x < DH; ++x) a = fmaf(s_q[tid][x], s_ktr[x], a);
+        s_lt[tid] = a * p.scale;
+    }
+    const float aq_t = p.a_q[unit], ak_t = p.a_k[unit];
+    const float al = p.alpha[kvh], be = p.beta[kvh];
+    const float rq_t = (variant & kVarNoQ) ? 1.f : softplus_f(aq_t);
+    float kq[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) kq[e] = s_kt[gl * VEC + e];
+    float m_h[G], l_h[G], acc[G][VEC];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        m_h[h] = -INFINITY;
+        l_h[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[h][e] = 0.f;
+    }
+
+    // ---- the slice: pairs [lo, hi), next pass loaded one pass ahead
+    uint4 na = make_uint4(0, 0, 0, 0), nb = na, nv = na;
+    float nbj = 0.f, nrk = 0.f;
+    auto load_entry = [&](int jj) {
+        if (jj < hi) {
+            const size_t e = (base + jj) * DH + gl * VEC;
+            na = *reinterpret_cast<const uint4*>(khat + e);
+            nb = *reinterpret_cast<const uint4*>(krope + e);
+            nv = *reinterpret_cast<const uint4*>(vc + e);
+            nbj = c.bias[base + jj];
+            nrk = c.rk[base + jj];
+        }
+    };
+    load_entry(lo + gidx);
+    for (int c0 = lo; c0 < hi; c0 += EPB) {
+        const int j = c0 + gidx;
+        const bool valid = j < hi;
+        const uint4 ra = na, rb = nb, rv = nv;
+        const float bj = nbj, rkj = nrk;
+        load_entry(j + EPB);
+        float xa[VEC], xb[VEC], xv[VEC];
+        Vec16<TC>::unpack(ra, xa);
+        Vec16<TC>::unpack(rb, xb);
+        Vec16<TC>::unpack(rv, xv);
+        float sim = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) sim = fmaf(kq[e], xa[e], sim);
+        sim = group_sum<LPE>(sim);
+        const float D = decay_var(rq_t, (variant & kVarNoK) ? 1.f : rkj, fmaf(al, sim, be), variant);
+        const float bnew = bj - D;
+        const bool keep = valid && (bnew >= p.logp);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float lg = 0.f;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) lg = fmaf(s_q[h][gl * VEC + e], xb[e], lg);
+            lg = group_sum<LPE>(lg);
+            if (keep) {
+                lg = fmaf(lg, p.scale, bnew);
+                const float mn = fmaxf(m_h[h], lg);
+                const float corr = expf(m_h[h] - mn);
+                const float pe = expf(lg - mn);
+                l_h[h] = l_h[h] * corr + pe;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc[h][e] = fmaf(pe, xv[e], acc[h][e] * corr);
+                m_h[h] = mn;
+            }
+        }
+        if (valid && gl == 0) {
+            c.bias[base + j] = bnew;
+            if (p.kept_idx) p.kept_idx[base + j] = j;
+            if (!keep) atomicOr(&s_ev[(j >> 5) - w0], 1u << (j & 31));
+        }
+    }
+    // ---- the CTA's partial state: merge its entry groups
+    if (gl == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            s_m[gidx * G + h] = m_h[h];
+            s_l[gidx * G + h] = l_h[h];
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) s_acc[((size_t)gidx * G + h) * DH + gl * VEC + e] = acc[h][e];
+    __syncthreads();
+    if (p.evict_bits)
+        for (int w = tid; w < nw; w += blockDim.x) p.evict_bits[(size_t)unit * words + w0 + w] = s_ev[w];
+    float* st = p.split_state + ((size_t)unit * kDecodeSplitMax + sl) * SS;
+    for (int e = tid; e < G * DH; e += blockDim.x) {
+        const int h = e / DH, x = e % DH;
+        float M = -INFINITY;
+        for (int q = 0; q < EPB; ++q) M = fmaxf(M, s_m[q * G + h]);
+        float Ls = 0.f, A = 0.f;
+        if (M > -INFINITY) {
+            for (int q = 0; q < EPB; ++q) {
+                const float w = expf(s_m[q * G + h] - M);
+                Ls = fmaf(s_l[q * G + h], w, Ls);
+                A = fmaf(s_acc[((size_t)q * G + h) * DH + x], w, A);
+            }
+        }
+        st[2 * G + e] = A;
+        if (x == 0) {
+            st[h] = M;
+            st[G + h] = Ls;
+        }
+    }
+    __threadfence();                                   // the state, biases and bits before the arrival
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(p.split_cnt + unit, 1u) == (unsigned)(nsl - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    // ---- last CTA of the cache: merge the slices with the new token, gate, append
+    TC* oout = static_cast<TC*>(p.o) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
+    const float* st0 = p.split_state + (size_t)unit * kDecodeSplitMax * SS;
+    for (int e = tid; e < G * DH; e += blockDim.x) {
+        const int h = e / DH, x = e % DH;
+        float M = s_lt[h];
+        for (int q = 0; q < nsl; ++q) M = fmaxf(M, __ldcg(st0 + (size_t)q * SS + h));
+        float Ls = expf(s_lt[h] - M);
+        float A = Ls * s_vt[x];
+        for (int q = 0; q < nsl; ++q) {
+            const float mq = __ldcg(st0 + (size_t)q * SS + h);
+            if (mq > -INFINITY) {
+                const float w = expf(mq - M);
+                Ls = fmaf(__ldcg(st0 + (size_t)q * SS + G + h), w, Ls);
+                A = fmaf(__ldcg(st0 + (size_t)q * SS + 2 * G + e), w, A);
+            }
+        }
+        Elem<TC>::st(oout + e, A / Ls * sigmoid_f(s_g[e]));
+    }
+    // words past the live pairs carry no eviction
+    if (p.evict_bits)
+        for (int w = ((n + 31) >> 5) + tid; w < words; w += blockDim.x) p.evict_bits[(size_t)unit * words + w] = 0u;
+    if (n < c.cap) {
+        const size_t e = (base + n) * DH;
+        for (int x = tid; x < DH; x += blockDim.x) {
+            Elem<TC>::st(khat + e + x, s_kt[x]);
+            Elem<TC>::st(krope + e + x, s_ktr[x]);
+            Elem<TC>::st(vc + e + x, s_vt[x]);
+        }
+        if (tid == 0) {
+            c.bias[base + n] = 0.f;
+            c.rk[base + n] = softplus_f(ak_t);
+            c.pos[base + n] = p.pos_t;
+            c.n_kept[unit] = n + 1;
+            if (p.kept_idx) p.kept_idx[base + n] = -1;
+        }
+    } else if (tid == 0) {
+        raise_status(UA_ERR_CAPACITY);
+    }
+    if (tid == 0) p.split_cnt[unit] = 0u;            // ready for the next step
+}
+
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_cache_fill(const FillParams& p, bool bf16, cudaStream_t s) {
     dim3 grid(p.T, p.c.B);
@@ -522,6 +775,41 @@ static cudaError_t decode_g(const DecodeParams& p, cudaStream_t s) {
         case 8: return decode_inst<TC, DH, 8>(p, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+template <typename TC, int DH, int G>
+static cudaError_t decode_split_inst(const DecodeParams& p, cudaStream_t s) {
+    using L = EntryLayout<TC, DH>;
+    // the largest slice: at most kDecodeSplitSlice pairs while the cache is short enough to be
+    // split into whole slices, else a kDecodeSplitMax-th of the capacity (whole 32-pair words)
+    const int max_chunk = std::max(kDecodeSplitSlice, ((p.c.cap + kDecodeSplitMax - 1) / kDecodeSplitMax + 31) & ~31);
+    const size_t smem = sizeof(float) * (size_t)L::EPB * G * DH + sizeof(uint32_t) * (size_t)(max_chunk / 32 + 1);
+    dim3 grid(kDecodeSplitMax, p.c.B * p.c.Hkv);
+    auto kern = p.variant != 0 ? k_decode_split<TC, DH, G, true> : k_decode_split<TC, DH, G, false>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    UA_PROFILE("k_decode_split", s);
+    kern<<<grid, 256, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename TC, int DH>
+static cudaError_t decode_split_g(const DecodeParams& p, cudaStream_t s) {
+    switch (p.G) {
+        case 1: return decode_split_inst<TC, DH, 1>(p, s);
+        case 2: return decode_split_inst<TC, DH, 2>(p, s);
+        case 3: return decode_split_inst<TC, DH, 3>(p, s);
+        case 4: return decode_split_inst<TC, DH, 4>(p, s);
+        case 8: return decode_split_inst<TC, DH, 8>(p, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_decode_split(const DecodeParams& p, bool bf16, cudaStream_t s) {
+    if (bf16) return p.c.d == 64 ? decode_split_g<__nv_bfloat16, 64>(p, s) : decode_split_g<__nv_bfloat16, 128>(p, s);
+    return p.c.d == 64 ? decode_split_g<float, 64>(p, s) : decode_split_g<float, 128>(p, s);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t s) {

@@ -192,9 +192,8 @@ __device__ __forceinline__ void decay16r(const uint32_t (&x)[16], const float* l
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = r4 + e;
-            // the outer exp2 on the FMA pipe: the exp2/log2 unit bounds this kernel
             const float dq =
-                exp2_fma(fmaf(log2_softplus_over_ln2(fmaf(al2, __uint_as_float(x[r]), be2)), 0.33333334f, lv[e]));
+                ex2f(fmaf(log2_softplus_over_ln2(fmaf(al2, __uint_as_float(x[r]), be2)), 0.33333334f, lv[e]));
             if (MASK) c += (r >= rlo && r < rhi) ? dq : 0.f;
             else c += dq;
             lam[r] = c;

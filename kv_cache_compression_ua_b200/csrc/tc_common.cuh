@@ -281,28 +281,5 @@ __device__ __forceinline__ float log2_softplus_over_ln2(float t2) {
 }
 
 
-// 2^x on the FMA and integer pipes, for x < 128 (the decay increments): x = n + f with
-// n = round(x) formed by the 1.5 * 2^23 rounding trick and f in [-1/2, 1/2]; 2^f from a degree-5
-// polynomial fitted for this library by Lawson's iteratively reweighted least squares on
-// Chebyshev nodes (maximum relative error 2.4e-7 evaluated in fp32 by Horner's rule, the same
-// order as ex2.approx); 2^n added into the exponent field.  x < -126 gives exactly 0 (-inf
-// included, which keeps the veto: a zero rate gives a zero decay).  No transcendental-unit op,
-// so the exp2/log2 unit is left to the other exponentials of the decay and the softmax.
-__device__ __forceinline__ float exp2_fma(float x) {
-    const float xc = fmaxf(x, -126.f);
-    const float t = xc + 12582912.f;               // 1.5 * 2^23: rounds xc to an integer in the low bits
-    const float n = t - 12582912.f;
-    const float f = xc - n;                        // in [-1/2, 1/2]
-    float p = 0.001327647129073739f;
-    p = fmaf(p, f, 0.009675540961325169f);
-    p = fmaf(p, f, 0.05550713092088699f);
-    p = fmaf(p, f, 0.24022120237350464f);
-    p = fmaf(p, f, 0.6931469440460205f);
-    p = fmaf(p, f, 1.0000001192092896f);
-    const int ni = __float_as_int(t) - 0x4B400000;   // n as an integer (t's bits minus 1.5 * 2^23's)
-    const float r = __int_as_float(__float_as_int(p) + (ni << 23));
-    return x < -126.f ? 0.f : r;
-}
-
 }  // namespace tc
 }  // namespace ua

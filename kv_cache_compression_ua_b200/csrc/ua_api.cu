@@ -406,8 +406,8 @@ BwdWs bwd_ws_layout(const ua_shape* s) {
 // dA, Delta and lse in log2 units, the decay prefixes above every 32-row step, the stored bf16
 // dZ^T / dX^T tiles of the causal band, and f32 gradient intermediates.
 struct BwdTcWs {
-    size_t qr, kh, kr, lq2, lk2, mq, ad, lse2, delta, pb, tiles, daq, dab, dv32, dkr, dkh, dkh_rows, dqr, dak,
-        total, ntiles;
+    size_t qr, kh, kh_lo, kr, lq2, lk2, mq, ad, lse2, delta, pb, tiles, daq, dab, dv32, dkr, dkh, dkh_rows, dqr,
+        dak, total, ntiles;
     int Tp, Tpk, nkt, nst;
 };
 
@@ -424,6 +424,7 @@ BwdTcWs bwd_tc_ws_layout(const ua_shape* s) {
     auto take = [&](size_t bytes) { size_t o = off; off = round_up(off + bytes, 1024); return o; };
     w.qr = take(B * H * T * d * 2);
     w.kh = take(B * Hkv * T * d * 2);
+    w.kh_lo = take(B * Hkv * T * d * 2);
     w.kr = take(B * Hkv * T * d * 2);
     w.lq2 = take(B * Hkv * Tp * 4);
     w.lk2 = take(B * Hkv * Tp * 4);
@@ -487,13 +488,14 @@ static ua_status prefill_bwd_tc(const ua_shape* s, const void* q, const void* k,
     pp.Tp = w.Tp; pp.mq_scale = s->scale * 1.4426950408889634f;
     pp.lq2 = reinterpret_cast<float*>(at(ws, w.lq2)); pp.lk2 = reinterpret_cast<float*>(at(ws, w.lk2));
     pp.mq = reinterpret_cast<float*>(at(ws, w.mq));
+    pp.kh_lo = at(ws, w.kh_lo);
     pp.rf = rope_freq(s->rope_theta, s->d);
     pp.variant = s->variant;   // the query norm only: use_bwd_tc excludes the mechanism bits
     if ((st = cuda_status(launch_prep(pp, true, true, cs))) != UA_OK) return st;
     BwdTcParams p;
     p.B = s->B; p.T = s->T; p.Tp = w.Tp; p.Tpk = w.Tpk; p.H = s->H; p.Hkv = s->Hkv; p.d = s->d;
     p.G = s->H / s->Hkv; p.nkt = w.nkt; p.nst = w.nst; p.scale = s->scale; p.rf = pp.rf; p.variant = s->variant;
-    p.qr = pp.qr; p.kh = pp.kh; p.kr = pp.kr; p.lq2 = pp.lq2; p.lk2 = pp.lk2;
+    p.qr = pp.qr; p.kh = pp.kh; p.kh_lo = pp.kh_lo; p.kr = pp.kr; p.lq2 = pp.lq2; p.lk2 = pp.lk2;
     p.q = q; p.k = k; p.v = v; p.g = g; p.o = o; p.d_o = d_o;
     p.a_q = a_q; p.a_k = a_k; p.alpha = alpha; p.beta = beta; p.lse = lse;
     p.ad = at(ws, w.ad);
@@ -641,7 +643,54 @@ ua_status ua_decode_step(const ua_cache* c, int H, const void* q, const void* k,
     dp.q = q; dp.k = k; dp.v = v; dp.g = g; dp.a_q = a_q; dp.a_k = a_k; dp.alpha = alpha; dp.beta = beta;
     dp.o = o; dp.evict_bits = evict_bits; dp.kept_idx = kept_idx;
     dp.variant = flags & ~UA_DECODE_DEFER_COMPACT; dp.defer = defer ? 1 : 0;
+    dp.split_cnt = nullptr; dp.split_state = nullptr;
     return cuda_status(launch_decode(dp, c->dtype == UA_BF16, static_cast<cudaStream_t>(stream)));
+}
+
+// Split decode: a counter per cache (256-byte block), then kDecodeSplitMax partial states of
+// G*(d+2) floats per cache.
+static size_t decode_ws_bytes(const ua_cache* c, int H) {
+    const size_t units = (size_t)c->B * c->Hkv, G = (size_t)H / c->Hkv;
+    return round_up(units * 4, 256) + units * kDecodeSplitMax * G * (c->d + 2) * 4;
+}
+
+ua_status ua_decode_workspace_size(const ua_cache* c, int H, size_t* bytes) {
+    ua_status st = check_cache(c);
+    if (st != UA_OK) return st;
+    if (!bytes || H < 1 || H % c->Hkv != 0) return UA_ERR_INVALID_ARG;
+    if (!group_ok(H / c->Hkv)) return UA_ERR_UNSUPPORTED;
+    *bytes = decode_ws_bytes(c, H);
+    return UA_OK;
+}
+
+ua_status ua_decode_step_split(const ua_cache* c, int H, const void* q, const void* k, const void* v, const void* g,
+                               const float* a_q, const float* a_k, const float* alpha, const float* beta, int pos_t,
+                               float p, float scale, double rope_theta, void* o, uint32_t* evict_bits,
+                               int32_t* kept_idx, int flags, void* ws, size_t ws_bytes, void* stream) {
+    ua_status st = check_cache(c);
+    if (st != UA_OK) return st;
+    const int var = flags & ~UA_DECODE_DEFER_COMPACT;
+    if (H < 1 || H % c->Hkv != 0 || pos_t < 0 || !variant_ok(var)) return UA_ERR_INVALID_ARG;
+    if (!group_ok(H / c->Hkv)) return UA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !g || !a_q || !a_k || !alpha || !beta || !o || !ws) return UA_ERR_INVALID_ARG;
+    if (!(p >= 0.f && p <= 1.f) || !isfinite(scale) || !(rope_theta > 0.0)) return UA_ERR_INVALID_ARG;
+    const void* ps[] = {q, k, v, g, a_q, a_k, alpha, beta, o, evict_bits, kept_idx};
+    for (const void* x : ps)
+        if (x && !aligned(x, 16)) return UA_ERR_ALIGNMENT;
+    if (!aligned(ws, 256)) return UA_ERR_ALIGNMENT;
+    if (ws_bytes < decode_ws_bytes(c, H)) return UA_ERR_WORKSPACE;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const size_t units = (size_t)c->B * c->Hkv;
+    // the per-cache arrival counters start at zero (the kernel also clears them after use)
+    if ((st = cuda_status(cudaMemsetAsync(ws, 0, units * 4, cs))) != UA_OK) return st;
+    DecodeParams dp;
+    dp.c = view(c); dp.H = H; dp.G = H / c->Hkv; dp.pos_t = pos_t; dp.scale = scale;
+    dp.logp = p > 0.f ? logf(p) : -INFINITY; dp.theta = rope_theta; dp.rf = rope_freq(rope_theta, c->d);
+    dp.q = q; dp.k = k; dp.v = v; dp.g = g; dp.a_q = a_q; dp.a_k = a_k; dp.alpha = alpha; dp.beta = beta;
+    dp.o = o; dp.evict_bits = evict_bits; dp.kept_idx = kept_idx; dp.variant = var; dp.defer = 1;
+    dp.split_cnt = static_cast<unsigned*>(ws);
+    dp.split_state = reinterpret_cast<float*>(at(ws, round_up(units * 4, 256)));
+    return cuda_status(launch_decode_split(dp, c->dtype == UA_BF16, cs));
 }
 
 ua_status ua_prefill_tile_stats(const ua_shape* s, const void* ws, size_t ws_bytes, unsigned long long* tiles,

@@ -28,6 +28,7 @@ struct PrepParams {
     float* lq2;         // [B*Hkv][Tp] log2(softplus(a_q)) / 3
     float* lk2;         // [B*Hkv][Tp] log2(softplus(a_k)) / 3
     float* mq;          // [B*H][Tp]  scale * ||q|| * log2(e): bound of every logit of the row
+    void* kh_lo;        // [B,Hkv,T,d] bf16 khat - bf16(khat), or NULL (bf16 work type only)
     RopeFreq rf;
     int variant;        // UA_VAR_* bits: query norm; rq / rk = 1 for a switched-off mechanism
 };
@@ -132,7 +133,17 @@ struct DecodeParams {
     int32_t* kept_idx;
     int variant;         // UA_VAR_* bits
     int defer;           // 1: no compaction (pairs stay in their slots; append at n_kept)
+    // split walk (launch_decode_split): per cache a counter, then per (cache, slice) the partial
+    // softmax state [G maxima][G sums][G x d weighted values]
+    unsigned* split_cnt;
+    float* split_state;
 };
+
+// Split decode step: the walk of each cache is cut into up to kDecodeSplitMax slices of at least
+// kDecodeSplitSlice pairs, one CTA each; compaction is deferred.
+constexpr int kDecodeSplitMax = 16;
+constexpr int kDecodeSplitSlice = 512;
+cudaError_t launch_decode_split(const DecodeParams& p, bool bf16, cudaStream_t s);
 
 // Backward (SIMT path).  Inputs from the f32 token preparation and boundary pass (query
 // tiles of 64 rows); f32 intermediates in the workspace; outputs in the caller's layouts.
@@ -206,7 +217,8 @@ struct BwdTcParams {
     int variant;          // UA_VAR_QUERY_NORM or 0
     // token preparation of the tensor-core forward (bf16 copies, log2 rates / 3)
     const void* qr;       // [B*H][T][d] RoPE(q)
-    const void* kh;       // [B*Hkv][T][d] khat
+    const void* kh;       // [B*Hkv][T][d] khat (bf16)
+    const void* kh_lo;    // [B*Hkv][T][d] khat - bf16(khat) (bf16): similarities to ~16 bits
     const void* kr;       // [B*Hkv][T][d] RoPE(khat)
     const float* lq2;     // [B*Hkv][Tp]
     const float* lk2;     // [B*Hkv][Tp]

@@ -52,7 +52,7 @@ EXPORTS = ("ua_prefill_workspace_size", "ua_prefill_fwd", "ua_prefill_bwd_worksp
            "ua_cache_fill", "ua_cache_compact", "ua_decode_step", "ua_get_device_status",
            "ua_profile_enable", "ua_profile_reset", "ua_profile_read", "ua_status_string", "ua_version",
            "ua_prefill_fwd_noalloc", "ua_prefill_noalloc_max_scratch", "ua_prefill_tile_stats",
-           "ua_set_wait_limit_ns")
+           "ua_set_wait_limit_ns", "ua_decode_workspace_size", "ua_decode_step_split")
 
 
 class ua_kernel_time(ctypes.Structure):
@@ -90,6 +90,8 @@ def load_library(path: str = LIB_PATH):
                                           ctypes.POINTER(ctypes.c_ulonglong), P]
     lib.ua_prefill_noalloc_max_scratch.restype = S
     lib.ua_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.ua_decode_workspace_size.argtypes = [CP, I, ctypes.POINTER(S)]
+    lib.ua_decode_step_split.argtypes = [CP, I] + [P] * 8 + [I, F, F, D, P, P, P, I, P, S, P]
     lib.ua_status_string.argtypes = [I]
     lib.ua_status_string.restype = ctypes.c_char_p
     lib.ua_version.argtypes = []
@@ -379,11 +381,22 @@ def cache_compact(cache: Cache, p: float = 0.0, keep=None, kept_idx=None, stream
                                                                    _ptr(kept_idx), _stream(stream)))
 
 
+def decode_workspace_size(cache: Cache, H: int) -> int:
+    """ua_decode_workspace_size: bytes of the split decode step's workspace."""
+    n = ctypes.c_size_t(0)
+    c = cache.struct()
+    _check("ua_decode_workspace_size", load_library().ua_decode_workspace_size(ctypes.byref(c), int(H),
+                                                                               ctypes.byref(n)))
+    return n.value
+
+
 def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: float, *, scale=None,
                 theta=500000.0, out=None, evict_bits=None, kept_idx=None, variant=0, defer_compact=False,
-                stream=None):
+                ws=None, stream=None):
     """ua_decode_step for one token per sequence (variant: the prefill's VAR_* bits;
-    defer_compact: leave evicted pairs in place until cache_compact).  Returns o [B,H,d]."""
+    defer_compact: leave evicted pairs in place until cache_compact).  With a workspace `ws`
+    (decode_workspace_size bytes) the step runs as ua_decode_step_split: long caches are walked
+    by several CTAs each and compaction is deferred.  Returns o [B,H,d]."""
     B, H, d = q.shape
     if (B, d) != (cache.B, cache.d):
         raise ValueError(f"q: shape {tuple(q.shape)}, expected [{cache.B}, H, {cache.d}]")
@@ -405,11 +418,20 @@ def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: 
     dev = cache.khat.device
     _same_device(dev, q=q, k=k, v=v, g=g, a_q=a_q, a_k=a_k, alpha=alpha, beta=beta, out=o,
                  evict_bits=evict_bits, kept_idx=kept_idx)
+    flags = int(variant) | (DECODE_DEFER_COMPACT if defer_compact else 0)
     with _on(dev):
+        if ws is not None:
+            _same_device(dev, ws=ws)
+            rc = load_library().ua_decode_step_split(ctypes.byref(c), H, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                                     _ptr(a_q), _ptr(a_k), _ptr(alpha), _ptr(beta), int(pos_t),
+                                                     float(p), scale, float(theta), _ptr(o), _ptr(evict_bits),
+                                                     _ptr(kept_idx), flags, _ptr(ws), ctypes.c_size_t(_nbytes(ws)),
+                                                     _stream(stream))
+            _check("ua_decode_step_split", rc)
+            return o
         rc = load_library().ua_decode_step(ctypes.byref(c), H, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q),
                                            _ptr(a_k), _ptr(alpha), _ptr(beta), int(pos_t), float(p), scale,
-                                           float(theta), _ptr(o), _ptr(evict_bits), _ptr(kept_idx),
-                                           int(variant) | (DECODE_DEFER_COMPACT if defer_compact else 0),
+                                           float(theta), _ptr(o), _ptr(evict_bits), _ptr(kept_idx), flags,
                                            _stream(stream))
     _check("ua_decode_step", rc)
     return o
