@@ -197,8 +197,9 @@ ua_status ua_prefill_tile_stats(const ua_shape* shape, const void* ws, size_t ws
  * decay prefixes above every 32-row step, a key-major pass that accumulates dv and the rotated
  * key gradient in TMEM and stores the bf16 dZ / dX tiles of the causal band, and tensor-core
  * GEMMs for the query and similarity gradients (the workspace holds the band: about
- * (G+1) * 2 bytes per causal pair and KV head).  Similarities are formed from the unit keys
- * split into two bf16 parts (~16 significant bits).  Other problems run as fp32 SIMT kernels.
+ * (G+1) * 2 bytes per causal pair and KV head).  Similarities are formed from the same bf16 unit
+ * keys as the tensor-core forward (whose row normalisers the probabilities are divided by).  Other
+ * problems run as fp32 SIMT kernels.
  * Training is dense: a shape with prune_p != 0 is UA_ERR_INVALID_ARG. */
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes);
 

@@ -206,9 +206,7 @@ namespace bnd {
 template <int DH>
 struct Smem {
     alignas(1024) uint8_t khk[DH / 64][16384];      // khat of the key tile, boxes [128][64]
-    alignas(1024) uint8_t khk_lo[DH / 64][16384];   // its bf16 residual
     alignas(1024) uint8_t kq[2][DH / 64][4096];     // khat of the step's rows, boxes [32][64]
-    alignas(1024) uint8_t kq_lo[2][DH / 64][4096];  // their residual
     alignas(128) float lq[2][ST];
     alignas(128) float lk[128];
     alignas(8) uint64_t kfull, qfull[2], xfull[2];
@@ -220,8 +218,6 @@ struct Smem {
 template <int DH>
 __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CUtensorMap tm_khk,
                                                       const __grid_constant__ CUtensorMap tm_khq,
-                                                      const __grid_constant__ CUtensorMap tm_khk_lo,
-                                                      const __grid_constant__ CUtensorMap tm_khq_lo,
                                                       const __grid_constant__ CUtensorMap tm_lq,
                                                       const __grid_constant__ CUtensorMap tm_lk, BwdTcParams p) {
     constexpr uint32_t ID_X = idesc_bf16(128, ST, 0, 0);
@@ -254,32 +250,21 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
     const bool leader = warp == 0 && elect_one();
     auto load_step = [&](int it) {
         const int st = it & 1, s = s0 + it;
-        mbar_expect_tx(&S.qfull[st], 2 * NB * 4096 + ST * 4);
-        for (int c = 0; c < NB; ++c) {
-            tma_load_3d(S.kq[st][c], &tm_khq, &S.qfull[st], 64 * c, s * ST, unit);
-            tma_load_3d(S.kq_lo[st][c], &tm_khq_lo, &S.qfull[st], 64 * c, s * ST, unit);
-        }
+        mbar_expect_tx(&S.qfull[st], NB * 4096 + ST * 4);
+        for (int c = 0; c < NB; ++c) tma_load_3d(S.kq[st][c], &tm_khq, &S.qfull[st], 64 * c, s * ST, unit);
         tma_load_2d(S.lq[st], &tm_lq, &S.qfull[st], s * ST, unit);
     };
-    // X^T from the split keys: hi hi^T + hi lo^T + lo hi^T (the lo lo^T term is below fp32 rounding)
     auto issue_x = [&](int it) {
         const int st = it & 1;
-        const uint32_t a = smem_u32(S.khk[0]), al = smem_u32(S.khk_lo[0]);
-        const uint32_t bq = smem_u32(S.kq[st][0]), bl = smem_u32(S.kq_lo[st][0]);
+        const uint32_t a = smem_u32(S.khk[0]), bq = smem_u32(S.kq[st][0]);
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
+        for (int kk = 0; kk < DH / 16; ++kk)
             umma_f16(tmem + st * 32, kdesc_rows(a, 128, kk), kdesc_rows(bq, ST, kk), ID_X, kk > 0);
-            umma_f16(tmem + st * 32, kdesc_rows(a, 128, kk), kdesc_rows(bl, ST, kk), ID_X, 1);
-            umma_f16(tmem + st * 32, kdesc_rows(al, 128, kk), kdesc_rows(bq, ST, kk), ID_X, 1);
-        }
         umma_commit(&S.xfull[st]);
     };
     if (leader) {
-        mbar_expect_tx(&S.kfull, 2 * NB * 16384 + 512);
-        for (int c = 0; c < NB; ++c) {
-            tma_load_3d(S.khk[c], &tm_khk, &S.kfull, 64 * c, kt * 128, unit);
-            tma_load_3d(S.khk_lo[c], &tm_khk_lo, &S.kfull, 64 * c, kt * 128, unit);
-        }
+        mbar_expect_tx(&S.kfull, NB * 16384 + 512);
+        for (int c = 0; c < NB; ++c) tma_load_3d(S.khk[c], &tm_khk, &S.kfull, 64 * c, kt * 128, unit);
         tma_load_2d(S.lk, &tm_lk, &S.kfull, kt * 128, unit);
         load_step(0);
         if (nsteps > 1) load_step(1);
@@ -354,12 +339,10 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
 namespace key {
 template <int DH, int G>
 struct Smem {
-    alignas(1024) uint8_t khk[DH / 64][16384];   // khat (and its bf16 residual) / krot / v of the key
-    alignas(1024) uint8_t khk_lo[DH / 64][16384];// tile, boxes [128][64]
+    alignas(1024) uint8_t khk[DH / 64][16384];   // khat / krot / v of the key tile, boxes [128][64]
     alignas(1024) uint8_t krk[DH / 64][16384];
     alignas(1024) uint8_t vk[DH / 64][16384];
-    alignas(1024) uint8_t kq[DH / 64][4096];     // khat of the step's rows and its residual, boxes [32][64]
-    alignas(1024) uint8_t kq_lo[DH / 64][4096];
+    alignas(1024) uint8_t kq[DH / 64][4096];     // khat of the step's rows, boxes [32][64]
     alignas(1024) uint8_t qh[G][DH / 64][4096];  // qrot / dA of the step's rows, per head
     alignas(1024) uint8_t ah[G][DH / 64][4096];
     alignas(1024) uint8_t tp[kTileBytes];        // P_h^T and dZ_h^T tiles (K-major, no swizzle)
@@ -381,7 +364,6 @@ template <int DH, int G>
 __global__ void __launch_bounds__(160, 1)
 k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__ CUtensorMap tm_krk,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_khq,
-             const __grid_constant__ CUtensorMap tm_khk_lo, const __grid_constant__ CUtensorMap tm_khq_lo,
              const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ad,
              const __grid_constant__ CUtensorMap tm_lq, const __grid_constant__ CUtensorMap tm_lk,
              const __grid_constant__ CUtensorMap tm_pb, const __grid_constant__ CUtensorMap tm_lse2,
@@ -432,17 +414,14 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         // ------------------------------------------------ TMA + MMA issue (one elected lane)
         const bool leader = elect_one();
         bool ok = true;
-        // step it covers rows of step s = nst-1-it.  The step's khat rows (and residual), lq and
-        // the prefix vector have one buffer: X^T is the first MMA of a step, so they are free
+        // step it covers rows of step s = nst-1-it.  The step's khat rows, lq and the prefix
+        // vector have one buffer: X^T is the first MMA of a step, so they are free
         // early and the next step's copy overlaps the rest of this one.
         auto load_q = [&](int it) {
             const int s = p.nst - 1 - it;
             if (leader) {
-                mbar_expect_tx(&S.qfull, 2 * NB * 4096 + ST * 4 + 128 * 4);
-                for (int c = 0; c < NB; ++c) {
-                    tma_load_3d(S.kq[c], &tm_khq, &S.qfull, 64 * c, s * ST, unit);
-                    tma_load_3d(S.kq_lo[c], &tm_khq_lo, &S.qfull, 64 * c, s * ST, unit);
-                }
+                mbar_expect_tx(&S.qfull, NB * 4096 + ST * 4 + 128 * 4);
+                for (int c = 0; c < NB; ++c) tma_load_3d(S.kq[c], &tm_khq, &S.qfull, 64 * c, s * ST, unit);
                 tma_load_2d(S.lq, &tm_lq, &S.qfull, s * ST, unit);
                 tma_load_2d(S.pbv, &tm_pb, &S.qfull, kt * 128, unit * p.nst + s);
             }
@@ -462,10 +441,9 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             __syncwarp();
         };
         if (leader) {
-            mbar_expect_tx(&S.kfull, 4 * NB * 16384 + 512);
+            mbar_expect_tx(&S.kfull, 3 * NB * 16384 + 512);
             for (int c = 0; c < NB; ++c) {
                 tma_load_3d(S.khk[c], &tm_khk, &S.kfull, 64 * c, kt * 128, unit);
-                tma_load_3d(S.khk_lo[c], &tm_khk_lo, &S.kfull, 64 * c, kt * 128, unit);
                 tma_load_3d(S.krk[c], &tm_krk, &S.kfull, 64 * c, kt * 128, unit);
                 tma_load_4d(S.vk[c], &tm_v, &S.kfull, 64 * c, kvh, kt * 128, b);
             }
@@ -475,23 +453,19 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         load_q(0);
         for (int h = 0; h < G; ++h) load_h(0, h);
         ok = wwait(&S.kfull, 0, abort);
-        const uint32_t akh = smem_u32(S.khk[0]), akl = smem_u32(S.khk_lo[0]);
-        const uint32_t akr = smem_u32(S.krk[0]), av = smem_u32(S.vk[0]);
-        const uint32_t bq = smem_u32(S.kq[0]), bql = smem_u32(S.kq_lo[0]);
+        const uint32_t akh = smem_u32(S.khk[0]), akr = smem_u32(S.krk[0]), av = smem_u32(S.vk[0]);
+        const uint32_t bq = smem_u32(S.kq[0]);
         bool first_acc = true;
         for (int it = 0; ok && it < nsteps; ++it) {
-            // X^T of the step from the split keys: hi hi^T + hi lo^T + lo hi^T, so the similarity
-            // (whose gradient dalpha sums with heavy cancellation) carries ~16 significant bits
+            // X^T of the step (the same bf16 unit keys as the forward, whose row normalisers the
+            // probabilities are divided by)
             if (!wwait(&S.qfull, it & 1, abort)) break;
             if (it >= 1 && !wwait(&S.xempty, (it - 1) & 1, abort)) break;
             tc_fence_after();
             if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < DH / 16; ++kk) {
+                for (int kk = 0; kk < DH / 16; ++kk)
                     umma_f16(tmem + COL_X, kdesc_rows(akh, 128, kk), kdesc_rows(bq, ST, kk), ID_L, kk > 0);
-                    umma_f16(tmem + COL_X, kdesc_rows(akh, 128, kk), kdesc_rows(bql, ST, kk), ID_L, 1);
-                    umma_f16(tmem + COL_X, kdesc_rows(akl, 128, kk), kdesc_rows(bq, ST, kk), ID_L, 1);
-                }
                 umma_commit(&S.xfull);
             }
             __syncwarp();
@@ -1085,9 +1059,7 @@ static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
         k_bwd_prep_tc<DH><<<dim3(p.T, p.B), 256, 0, s>>>(p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    CUtensorMap m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk, m_pb, m_lse2, m_dlt, m_kh128, m_khk_lo, m_khq_lo;
-    if (!map_rows_bwd(&m_khk_lo, p.kh_lo, DH, p.T, BK, 128) || !map_rows_bwd(&m_khq_lo, p.kh_lo, DH, p.T, BK, ST))
-        return cudaErrorInvalidValue;
+    CUtensorMap m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk, m_pb, m_lse2, m_dlt, m_kh128;
     if (!map_rows_bwd(&m_khk, p.kh, DH, p.T, BK, 128) || !map_rows_bwd(&m_krk, p.kr, DH, p.T, BK, 128) ||
         !map_v_bwd(&m_v, p.v, DH, p.Hkv, p.T, p.B) || !map_rows_bwd(&m_khq, p.kh, DH, p.T, BK, ST) ||
         !map_rows_bwd(&m_q, p.qr, DH, p.T, BH, ST) || !map_rows_bwd(&m_ad, p.ad, DH, p.T, BH, ST) ||
@@ -1102,7 +1074,7 @@ static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
             cudaSuccess)
             return e;
         UA_PROFILE("k_bwd_bound_tc", s);
-        k_bwd_bound_tc<DH><<<dim3(p.nkt, BK), 128, smem, s>>>(m_khk, m_khq, m_khk_lo, m_khq_lo, m_lq, m_lk, p);
+        k_bwd_bound_tc<DH><<<dim3(p.nkt, BK), 128, smem, s>>>(m_khk, m_khq, m_lq, m_lk, p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {
@@ -1111,8 +1083,8 @@ static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
             cudaSuccess)
             return e;
         UA_PROFILE("k_bwd_key_tc", s);
-        k_bwd_key_tc<DH, G><<<dim3(p.nkt, BK), 160, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_khk_lo, m_khq_lo, m_q,
-                                                               m_ad, m_lq, m_lk, m_pb, m_lse2, m_dlt, p);
+        k_bwd_key_tc<DH, G><<<dim3(p.nkt, BK), 160, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk,
+                                                               m_pb, m_lse2, m_dlt, p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {

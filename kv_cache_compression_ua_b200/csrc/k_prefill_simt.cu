@@ -96,18 +96,6 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p) {
             TW* dst_hat = static_cast<TW*>(p.kh) + (((size_t)b * p.Hkv + h) * T + t) * DH;
             Vec8<TW>::st(dst_hat + 8 * c, x0);
             Vec8<TW>::st(dst_hat + HALF + 8 * c, x1);
-            if (p.kh_lo) {
-                // the part of khat a bf16 copy drops: hi + lo carries ~16 significant bits
-                float r0[8], r1[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    r0[e] = x0[e] - __bfloat162float(__float2bfloat16_rn(x0[e]));
-                    r1[e] = x1[e] - __bfloat162float(__float2bfloat16_rn(x1[e]));
-                }
-                __nv_bfloat16* lo = static_cast<__nv_bfloat16*>(p.kh_lo) + (((size_t)b * p.Hkv + h) * T + t) * DH;
-                Vec8<__nv_bfloat16>::st(lo + 8 * c, r0);
-                Vec8<__nv_bfloat16>::st(lo + HALF + 8 * c, r1);
-            }
             dst_rot = static_cast<TW*>(p.kr) + (((size_t)b * p.Hkv + h) * T + t) * DH;
         }
         float y0[8], y1[8];

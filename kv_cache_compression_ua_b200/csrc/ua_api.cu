@@ -406,8 +406,8 @@ BwdWs bwd_ws_layout(const ua_shape* s) {
 // dA, Delta and lse in log2 units, the decay prefixes above every 32-row step, the stored bf16
 // dZ^T / dX^T tiles of the causal band, and f32 gradient intermediates.
 struct BwdTcWs {
-    size_t qr, kh, kh_lo, kr, lq2, lk2, mq, ad, lse2, delta, pb, tiles, daq, dab, dv32, dkr, dkh, dkh_rows, dqr,
-        dak, total, ntiles;
+    size_t qr, kh, kr, lq2, lk2, mq, ad, lse2, delta, pb, tiles, daq, dab, dv32, dkr, dkh, dkh_rows, dqr, dak,
+        total, ntiles;
     int Tp, Tpk, nkt, nst;
 };
 
@@ -424,7 +424,6 @@ BwdTcWs bwd_tc_ws_layout(const ua_shape* s) {
     auto take = [&](size_t bytes) { size_t o = off; off = round_up(off + bytes, 1024); return o; };
     w.qr = take(B * H * T * d * 2);
     w.kh = take(B * Hkv * T * d * 2);
-    w.kh_lo = take(B * Hkv * T * d * 2);
     w.kr = take(B * Hkv * T * d * 2);
     w.lq2 = take(B * Hkv * Tp * 4);
     w.lk2 = take(B * Hkv * Tp * 4);
@@ -488,14 +487,13 @@ static ua_status prefill_bwd_tc(const ua_shape* s, const void* q, const void* k,
     pp.Tp = w.Tp; pp.mq_scale = s->scale * 1.4426950408889634f;
     pp.lq2 = reinterpret_cast<float*>(at(ws, w.lq2)); pp.lk2 = reinterpret_cast<float*>(at(ws, w.lk2));
     pp.mq = reinterpret_cast<float*>(at(ws, w.mq));
-    pp.kh_lo = at(ws, w.kh_lo);
     pp.rf = rope_freq(s->rope_theta, s->d);
     pp.variant = s->variant;   // the query norm only: use_bwd_tc excludes the mechanism bits
     if ((st = cuda_status(launch_prep(pp, true, true, cs))) != UA_OK) return st;
     BwdTcParams p;
     p.B = s->B; p.T = s->T; p.Tp = w.Tp; p.Tpk = w.Tpk; p.H = s->H; p.Hkv = s->Hkv; p.d = s->d;
     p.G = s->H / s->Hkv; p.nkt = w.nkt; p.nst = w.nst; p.scale = s->scale; p.rf = pp.rf; p.variant = s->variant;
-    p.qr = pp.qr; p.kh = pp.kh; p.kh_lo = pp.kh_lo; p.kr = pp.kr; p.lq2 = pp.lq2; p.lk2 = pp.lk2;
+    p.qr = pp.qr; p.kh = pp.kh; p.kr = pp.kr; p.lq2 = pp.lq2; p.lk2 = pp.lk2;
     p.q = q; p.k = k; p.v = v; p.g = g; p.o = o; p.d_o = d_o;
     p.a_q = a_q; p.a_k = a_k; p.alpha = alpha; p.beta = beta; p.lse = lse;
     p.ad = at(ws, w.ad);

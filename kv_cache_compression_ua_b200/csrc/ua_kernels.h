@@ -28,7 +28,6 @@ struct PrepParams {
     float* lq2;         // [B*Hkv][Tp] log2(softplus(a_q)) / 3
     float* lk2;         // [B*Hkv][Tp] log2(softplus(a_k)) / 3
     float* mq;          // [B*H][Tp]  scale * ||q|| * log2(e): bound of every logit of the row
-    void* kh_lo;        // [B,Hkv,T,d] bf16 khat - bf16(khat), or NULL (bf16 work type only)
     RopeFreq rf;
     int variant;        // UA_VAR_* bits: query norm; rq / rk = 1 for a switched-off mechanism
 };
@@ -218,7 +217,6 @@ struct BwdTcParams {
     // token preparation of the tensor-core forward (bf16 copies, log2 rates / 3)
     const void* qr;       // [B*H][T][d] RoPE(q)
     const void* kh;       // [B*Hkv][T][d] khat (bf16)
-    const void* kh_lo;    // [B*Hkv][T][d] khat - bf16(khat) (bf16): similarities to ~16 bits
     const void* kr;       // [B*Hkv][T][d] RoPE(khat)
     const float* lq2;     // [B*Hkv][Tp]
     const float* lk2;     // [B*Hkv][Tp]
