@@ -377,6 +377,37 @@ def bench_e2e(args, w, x):
             "pipelining": "2 buffer sets, copy-in / compute / copy-out streams"}
 
 
+DECODE_COMPACT_EVERY = 32
+
+
+def graph_time(run, restore, reps=5, warm=3):
+    """Median device time (ms) of `run` captured in one CUDA graph and replayed, the state put
+    back by `restore` before every replay (untimed)."""
+    g = torch.cuda.CUDAGraph()
+    s_cap = torch.cuda.Stream()
+    s_cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s_cap):
+        run(s_cap)               # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(s_cap)
+    torch.cuda.synchronize()
+    restore()
+    with torch.cuda.graph(g, stream=s_cap):
+        run(s_cap)
+    times = []
+    for it in range(warm + reps):
+        restore()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        if it >= warm:
+            times.append(e0.elapsed_time(e1))
+    del g
+    return statistics.median(times)
+
+
 def bench_decode(args, peaks, peaks_kind):
     """Decode workload: B=32 caches prefilled (on the GPU) from a 16k-token draw, compacted at
     p, then 256 single-token steps captured in one CUDA graph and replayed.  Besides the
@@ -419,12 +450,12 @@ def bench_decode(args, peaks, peaks_kind):
                         ak_r, bfinal_r, tok_r))
     res = {}
     cap = T0 + steps + 1
-    entry_bytes = 3 * w.d * 2 + 12
+    entry_bytes = 2 * w.d * 2 + 12          # khat, v (bf16), bias, rk, pos: 268 B at d = 64
     for key, p, ak, bf, tk in configs:
         cache = ua.Cache.empty(w.B, w.Hkv, w.d, cap, torch.bfloat16)
         ua.cache_fill(cache, x["k"], x["v"], ak, bf, theta=w.theta)
         ua.cache_compact(cache, p)
-        snap = {n: getattr(cache, n).clone() for n in ("khat", "krope", "v", "bias", "rk", "pos", "n_kept")}
+        snap = {n: getattr(cache, n).clone() for n in ("khat", "v", "bias", "rk", "pos", "n_kept")}
         n0 = cache.n_kept.clone()
         o = torch.empty(steps, w.B, w.H, w.d, dtype=torch.bfloat16, device="cuda")
 
@@ -470,8 +501,8 @@ def bench_decode(args, peaks, peaks_kind):
             if it >= 3:
                 times.append(e0.elapsed_time(e1))
         ms = statistics.median(times)
-        # algorithmic bytes: every live entry read once per step (khat, krope, v, bias, rk,
-        # pos), its bias written back, the appended token written, and the token's q/k/v/g/o
+        # algorithmic bytes: every live entry read once per step (khat, v, bias, rk, pos), its
+        # bias written back, the appended token written, and the token's q/k/v/g/o
         tok_bytes = w.B * (3 * w.H * w.d * 2 + 2 * w.Hkv * w.d * 2 + 2 * w.Hkv * 4)
         bytes_total = sum(counts[s] * entry_bytes + counts[s + 1] * 4 + w.B * w.Hkv * entry_bytes + tok_bytes
                           for s in range(steps))
@@ -486,7 +517,30 @@ def bench_decode(args, peaks, peaks_kind):
                     "compression_x": 1.0 / kept_frac if kept_frac > 0 else None}
         if ak is not x["a_k"]:
             res[key]["ak_slow_mean"] = I.DECODE_RETAINED_AK_SLOW_MEAN
-        del g, cache, snap
+        del g
+        # the same steps through the split walk (deferred compaction; at p > 0 a compaction every
+        # DECODE_COMPACT_EVERY steps and after the last), checked against the eager outputs
+        ws = ua.alloc_workspace(ua.decode_workspace_size(cache, w.H), "cuda")
+        o_eager = o.clone()
+
+        def run_split(stream=None):
+            for s in range(steps):
+                ua.decode_step(cache, tk["q"][s], tk["k"][s], tk["v"][s], tk["g"][s], tk["a_q"][s],
+                               tk["a_k"][s], x["alpha"], x["beta"], T0 + s, p, scale=w.scale, theta=w.theta,
+                               out=o[s], ws=ws, stream=stream)
+                if p > 0 and ((s + 1) % DECODE_COMPACT_EVERY == 0 or s == steps - 1):
+                    ua.cache_compact(cache, p, stream=stream)
+        restore()
+        ms_split = graph_time(run_split, restore)
+        assert ua.get_device_status() == 0
+        diff = float((o.float() - o_eager.float()).norm() / o_eager.float().norm())
+        gbs_s = bytes_total / (ms_split * 1e-3) / 1e9
+        res[key]["split_walk"] = {
+            "us_per_step": 1e3 * ms_split / steps, "tokens_per_s": w.B * steps / (ms_split * 1e-3),
+            "hbm_gbs": gbs_s, "hbm_frac": gbs_s / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+            "compaction": (f"deferred, every {DECODE_COMPACT_EVERY} steps" if p > 0 else "none needed (p = 0)"),
+            "o_rel_l2_vs_one_cta_per_cache": diff}
+        del cache, snap, ws
         torch.cuda.empty_cache()
     # Split walk for few long caches (supplementary): one sequence (B=1, 8 KV heads, p = 0: 16.4k
     # live pairs per head, compaction deferred) decoded by one CTA per cache and by the split step
@@ -499,7 +553,7 @@ def bench_decode(args, peaks, peaks_kind):
         cache = ua.Cache.empty(1, w.Hkv, w.d, cap, torch.bfloat16)
         ua.cache_fill(cache, xs["k"], xs["v"], xs["a_k"], bf1, theta=w.theta)
         ua.cache_compact(cache, 0.0)
-        snap = {n: getattr(cache, n).clone() for n in ("khat", "krope", "v", "bias", "rk", "pos", "n_kept")}
+        snap = {n: getattr(cache, n).clone() for n in ("khat", "v", "bias", "rk", "pos", "n_kept")}
         n0 = int(cache.n_kept.sum().item())
         o = torch.empty(steps, 1, w.H, w.d, dtype=torch.bfloat16, device="cuda")
         ws = ua.alloc_workspace(ua.decode_workspace_size(cache, w.H), "cuda") if mode == "split" else None
@@ -631,6 +685,8 @@ def bench_fwdbwd(args):
     """3B layer forward + backward (B=4, T=8192, H=24, Hkv=8, d=128, bf16)."""
     from kv_cache_compression_ua_b200 import ua
     w = I.WORKLOADS["fwdbwd_3b"]
+    if args.fwdbwd_batch != w.B:
+        w = w.resized(B=args.fwdbwd_batch)
     x = I.make_prefill_inputs_torch(w, "cuda")
     args_in = (x["q"], x["k"], x["v"], x["g"], x["a_q"], x["a_k"], x["alpha"], x["beta"])
     shape = ua.make_shape(x["q"], x["k"], w.scale, w.theta)
@@ -655,7 +711,7 @@ def bench_fwdbwd(args):
     prof = ua.profile_read()
     assert ua.get_device_status() == 0
     fms, bms = e[0].elapsed_time(e[1]) / n, e[1].elapsed_time(e[2]) / n
-    return {"workload": "fwdbwd_3b: B=4 T=8192 H=24 Hkv=8 d=128 bf16", "fwd_ms": fms, "bwd_ms": bms,
+    return {"workload": f"fwdbwd_3b: B={w.B} T={w.T} H={w.H} Hkv={w.Hkv} d={w.d} bf16", "fwd_ms": fms, "bwd_ms": bms,
             "fwd_tflops": fwd_flops(w) / (fms * 1e-3) / 1e12, "bwd_tflops": bwd_flops(w) / (bms * 1e-3) / 1e12,
             "fwd_bwd_tflops": (fwd_flops(w) + bwd_flops(w)) / ((fms + bms) * 1e-3) / 1e12,
             "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / v[0]} for k, v in prof.items()}}
@@ -673,6 +729,8 @@ def main():
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-more", action="store_true", help="skip the 16k and chunked-pruned prefill lines")
     ap.add_argument("--decode-p", type=float, default=None, help="run the decode section at this p only")
+    ap.add_argument("--fwdbwd-batch", type=int, default=4,
+                    help="batch of the 3B forward+backward line (4 = the workload; smaller for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

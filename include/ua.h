@@ -214,8 +214,11 @@ ua_status ua_prefill_bwd(const ua_shape* shape, const void* q, const void* k, co
  * One cache per (batch, KV head), structure of arrays, `capacity` slots each; slot s of
  * (b, h) lives at index (b*Hkv + h)*capacity + s.  Slots [0, n_kept[b,h]) are live, in
  * ascending token order.  The cache element type follows `dtype` (f32 or bf16).
- *   khat  [B,Hkv,cap,d]  normalised key (pre-RoPE), used by the similarity rate
- *   krope [B,Hkv,cap,d]  RoPE(khat, pos), used by the attention logit
+ *   khat  [B,Hkv,cap,d]  normalised key (pre-RoPE), pair-interleaved: element 2m holds
+ *                        component m and element 2m+1 component m + d/2 (the two components
+ *                        one RoPE frequency rotates together).  The similarity rate uses it as
+ *                        is; the attention logit rotates it by the slot's pos on the fly, so
+ *                        no rotated copy is stored (2*d*elt + 12 bytes per slot)
  *   v     [B,Hkv,cap,d]  value
  *   bias  [B,Hkv,cap]    f32 running log-bias b_j (= Lambda_{t,j} at the current row t)
  *   rk    [B,Hkv,cap]    f32 key-aware rate softplus(a_k[j])
@@ -227,7 +230,6 @@ typedef struct {
     int B, Hkv, d, capacity;
     ua_dtype dtype;
     void* khat;
-    void* krope;
     void* v;
     float* bias;
     float* rk;
@@ -235,8 +237,8 @@ typedef struct {
     int32_t* n_kept;
 } ua_cache;
 
-/* Load a prefill into the cache: slot t <- token t for t < T (khat, krope, v from k and
- * v; bias = b_final; rk = softplus(a_k); pos = t) and n_kept = T.  Requires T <= capacity.
+/* Load a prefill into the cache: slot t <- token t for t < T (khat, v from k and v; bias =
+ * b_final; rk = softplus(a_k); pos = t) and n_kept = T.  Requires T <= capacity.
  * k, v: [B,T,Hkv,d] act; a_k [B,T,Hkv] f32; b_final [B,Hkv,T] f32. */
 ua_status ua_cache_fill(const ua_cache* cache, int T, const void* k, const void* v,
                         const float* a_k, const float* b_final, double rope_theta, void* stream);
@@ -253,7 +255,8 @@ ua_status ua_cache_compact(const ua_cache* cache, const uint8_t* keep, float p,
  *   1. each live pair j takes the new row's decay, b_j -= D[t,j];
  *   2. it is evicted when b_j < log p (exp(b_j) < p); p = 0 evicts nothing;
  *   3. the H query heads attend over the survivors plus the new token (bias 0) with
- *      logits scale * RoPE(q).krope_j + b_j, and the result is gated by sigmoid(g);
+ *      logits scale * RoPE(q, pos_t).RoPE(khat_j, pos_j) + b_j, and the result is gated by
+ *      sigmoid(g);
  *   4. survivors are compacted stably in place and the new token is appended (b = 0).
  * All in one pass over the cache.  q, g: [B,H,d] act; k, v: [B,Hkv,d] act;
  * a_q, a_k: [B,Hkv] f32; alpha, beta [Hkv] f32; o: [B,H,d] act (required).
@@ -287,8 +290,14 @@ ua_status ua_decode_step(const ua_cache* cache, int H, const void* q, const void
  * new token, gates, writes o and appends the token at slot n.  evict_bits and kept_idx follow the
  * deferred-compaction rules of ua_decode_step; evicted pairs stay until ua_cache_compact.
  * ws: device workspace of ua_decode_workspace_size bytes (256-byte aligned), scratch only; calls
- * that share a workspace must not overlap on the GPU.  A short cache (n <= 512) takes one CTA, as
- * ua_decode_step does. */
+ * that share a workspace must not overlap on the GPU.  A short cache (n <= 512) takes one slice.
+ * bf16 caches run on the tensor cores: per 128-entry tile one tcgen05 product gives every
+ * entry's similarity and G logits (the new key and the rotated queries enter as bf16 high parts
+ * plus residuals), a thread per entry turns them into the decay, the bias, the eviction and the
+ * probabilities, and a second product accumulates the weighted values in TMEM; the softmax shift
+ * starts at the new token's logit and is raised (with the accumulated values rescaled) whenever
+ * a tile exceeds it by more than 16, so any query norm is computed.  fp32 caches run the same
+ * step on the CUDA cores. */
 ua_status ua_decode_workspace_size(const ua_cache* cache, int H, size_t* bytes);
 ua_status ua_decode_step_split(const ua_cache* cache, int H, const void* q, const void* k, const void* v,
                                const void* g, const float* a_q, const float* a_k, const float* alpha,

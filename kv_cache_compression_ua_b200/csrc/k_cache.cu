@@ -9,8 +9,11 @@
 // pruned cache as future work (paperlayer.ai summary §6, App. H) -- this file is that part.
 //
 // Layout: one structure-of-arrays cache per (batch, KV head), slots in ascending token
-// order.  An entry is read by a group of LPE lanes, each moving 16 bytes of khat, krope and v
-// (128-bit coalesced loads); dot products reduce across the group with shuffles.
+// order.  An entry is read by a group of LPE lanes, each moving 16 bytes of khat and v
+// (128-bit coalesced loads); dot products reduce across the group with shuffles.  The cache
+// holds no rotated copy of the keys: khat is stored pair-interleaved (il_index), so each lane
+// holds whole RoPE pairs and rotates them by its entry's position while the next pass loads
+// (268 bytes per bf16 entry at d = 64 instead of 396).
 #include <algorithm>
 
 #include "ua_common.cuh"
@@ -33,6 +36,20 @@ __device__ __forceinline__ float group_sum(float x) {
 #pragma unroll
     for (int o = LPE / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
     return x;
+}
+
+// RoPE of a cached key's VEC/2 pairs (pair-interleaved khat) at its position pos, the lane's
+// frequencies given in turns (gt = f / (2 pi)).
+template <int VEC>
+__device__ __forceinline__ void rotate_pairs(const float (&xa)[VEC], float (&xb)[VEC], double pos,
+                                             const double (&gt)[VEC / 2]) {
+#pragma unroll
+    for (int i = 0; i < VEC / 2; ++i) {
+        float cs, sn;
+        rope_cs_turns(pos, gt[i], &cs, &sn);
+        xb[2 * i] = xa[2 * i] * cs - xa[2 * i + 1] * sn;
+        xb[2 * i + 1] = xa[2 * i + 1] * cs + xa[2 * i] * sn;
+    }
 }
 
 // Block-wide stable compaction bookkeeping for one pass: returns the destination of this
@@ -62,9 +79,6 @@ __global__ void __launch_bounds__(256) k_cache_fill(FillParams p) {
     const int t = blockIdx.x, b = blockIdx.y, T = p.T;
     const CacheView& c = p.c;
     constexpr int half = DH / 2;
-    __shared__ float s_cos[half], s_sin[half];
-    for (int m = threadIdx.x; m < half; m += blockDim.x) rope_cs((double)t, p.rf.f[m], &s_cos[m], &s_sin[m]);
-    __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const TC* kin = static_cast<const TC*>(p.k);
     const TC* vin = static_cast<const TC*>(p.v);
@@ -86,17 +100,13 @@ __global__ void __launch_bounds__(256) k_cache_fill(FillParams p) {
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         const float den = fmaxf(sqrtf(ss), 1e-12f);
         TC* kh = static_cast<TC*>(c.khat) + slot * DH;
-        TC* kr = static_cast<TC*>(c.krope) + slot * DH;
         TC* vv = static_cast<TC*>(c.v) + slot * DH;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int m = lane + 32 * r;
-            if (m < half) {
-                const float a = x0[r] / den, bq = x1[r] / den;
-                Elem<TC>::st(kh + m, a);
-                Elem<TC>::st(kh + m + half, bq);
-                Elem<TC>::st(kr + m, a * s_cos[m] - bq * s_sin[m]);
-                Elem<TC>::st(kr + m + half, bq * s_cos[m] + a * s_sin[m]);
+            if (m < half) {                               // the pair (m, m + half), interleaved
+                Elem<TC>::st(kh + 2 * m, x0[r] / den);
+                Elem<TC>::st(kh + 2 * m + 1, x1[r] / den);
             }
         }
         for (int x = lane; x < DH; x += 32) vv[x] = vin[src + x];
@@ -126,20 +136,18 @@ __global__ void __launch_bounds__(256) k_cache_compact(CompactParams p) {
     }
     const size_t base = (size_t)unit * c.cap;
     TC* khat = static_cast<TC*>(c.khat);
-    TC* krope = static_cast<TC*>(c.krope);
     TC* vc = static_cast<TC*>(c.v);
     int out = 0;
     for (int c0 = 0; c0 < n; c0 += L::EPB) {
         const int j = c0 + warp * L::EPW + grp;
         const bool valid = j < n;
-        uint4 a = make_uint4(0, 0, 0, 0), bq = a, vv = a;
+        uint4 a = make_uint4(0, 0, 0, 0), vv = a;
         float bj = 0.f, rkj = 0.f;
         int pj = 0;
         bool keep = false;
         if (valid) {
             const size_t e = (base + j) * DH + gl * L::VEC;
             a = *reinterpret_cast<const uint4*>(khat + e);
-            bq = *reinterpret_cast<const uint4*>(krope + e);
             vv = *reinterpret_cast<const uint4*>(vc + e);
             bj = c.bias[base + j];
             rkj = c.rk[base + j];
@@ -152,7 +160,6 @@ __global__ void __launch_bounds__(256) k_cache_compact(CompactParams p) {
             if (dst != j) {
                 const size_t e = (base + dst) * DH + gl * L::VEC;
                 *reinterpret_cast<uint4*>(khat + e) = a;
-                *reinterpret_cast<uint4*>(krope + e) = bq;
                 *reinterpret_cast<uint4*>(vc + e) = vv;
                 if (gl == 0) {
                     c.bias[base + dst] = bj;
@@ -197,7 +204,6 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     const int gidx = warp * L::EPW + grp;             // entry group index in the pass
     const size_t base = (size_t)unit * c.cap;
     TC* khat = static_cast<TC*>(c.khat);
-    TC* krope = static_cast<TC*>(c.krope);
     TC* vc = static_cast<TC*>(c.v);
 
     // ---- Every load that depends on no other goes out first (the live count, the new token,
@@ -246,8 +252,9 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
 #pragma unroll
     for (int w = 0; w < NW; ++w) tot_ss += s_red[w];
     const float den = fmaxf(sqrtf(tot_ss), 1e-12f);
+    // khat_t, RoPE(q_h) and RoPE(khat_t) are held pair-interleaved, as the cache stores keys
     if (tid < DH) {
-        s_kt[tid] = kx / den;
+        s_kt[il_index(tid, half)] = kx / den;
         s_vt[tid] = vx;
     }
     __syncthreads();
@@ -258,16 +265,16 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
             const int vecid = e / half, m = e % half;
             float cs, sn;
             rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
-            s_q[vecid][m] = qa[r] * cs - qb[r] * sn;
-            s_q[vecid][m + half] = qb[r] * cs + qa[r] * sn;
+            s_q[vecid][2 * m] = qa[r] * cs - qb[r] * sn;
+            s_q[vecid][2 * m + 1] = qb[r] * cs + qa[r] * sn;
         }
     }
     for (int m = tid; m < half; m += blockDim.x) {
         float cs, sn;
         rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
-        const float x0 = s_kt[m], x1 = s_kt[m + half];
-        s_ktr[m] = x0 * cs - x1 * sn;
-        s_ktr[m + half] = x1 * cs + x0 * sn;
+        const float x0 = s_kt[2 * m], x1 = s_kt[2 * m + 1];
+        s_ktr[2 * m] = x0 * cs - x1 * sn;
+        s_ktr[2 * m + 1] = x1 * cs + x0 * sn;
     }
     __syncthreads();
     if (variant & kVarQNorm) {                    // query RMS norm (RoPE keeps the norm)
@@ -293,6 +300,9 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     float kq[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) kq[e] = s_kt[gl * VEC + e];
+    double gt[VEC / 2];                               // this lane's RoPE frequencies / (2 pi)
+#pragma unroll
+    for (int i = 0; i < VEC / 2; ++i) gt[i] = p.rf.f[gl * (VEC / 2) + i] * 0.15915494309189535;
     float m_h[G], l_h[G], acc[G][VEC];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -311,14 +321,13 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     // Software pipeline: the entries of the next pass are loaded before this pass is processed,
     // so two passes of loads are in flight.  Safe with the in-place compaction: a survivor of
     // this pass only ever moves to a slot at or below its own, never into the next pass.
-    uint4 na = make_uint4(0, 0, 0, 0), nb = na, nv = na;
+    uint4 na = make_uint4(0, 0, 0, 0), nv = na;
     float nbj = 0.f, nrk = 0.f;
     int npj = 0;
     auto load_entry = [&](int jj) {
         if (jj < n) {
             const size_t e = (base + jj) * DH + gl * VEC;
             na = *reinterpret_cast<const uint4*>(khat + e);
-            nb = *reinterpret_cast<const uint4*>(krope + e);
             nv = *reinterpret_cast<const uint4*>(vc + e);
             nbj = c.bias[base + jj];
             nrk = c.rk[base + jj];
@@ -338,7 +347,6 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
                 if (jn < n) {
                     const size_t e = (base + jn) * DH;
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(khat + e));
-                    asm volatile("prefetch.global.L2 [%0];" ::"l"(krope + e));
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(vc + e));
                     if ((jn & 31) == 0) {
                         asm volatile("prefetch.global.L2 [%0];" ::"l"(c.bias + base + jn));
@@ -348,14 +356,14 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
                 }
             }
         }
-        const uint4 ra = na, rb = nb, rv = nv;
+        const uint4 ra = na, rv = nv;
         const float bj = nbj, rkj = nrk;
         const int pj = npj;
         load_entry(j + EPB);
         float xa[VEC], xb[VEC], xv[VEC];
         Vec16<TC>::unpack(ra, xa);
-        Vec16<TC>::unpack(rb, xb);
         Vec16<TC>::unpack(rv, xv);
+        rotate_pairs<VEC>(xa, xb, (double)pj, gt);
         float sim = 0.f;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) sim = fmaf(kq[e], xa[e], sim);
@@ -395,7 +403,6 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
             if (dst != j) {
                 const size_t e = (base + dst) * DH + gl * VEC;
                 *reinterpret_cast<uint4*>(khat + e) = ra;
-                *reinterpret_cast<uint4*>(krope + e) = rb;
                 *reinterpret_cast<uint4*>(vc + e) = rv;
                 if (gl == 0) {
                     c.rk[base + dst] = rkj;
@@ -449,7 +456,6 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         const size_t e = (base + out) * DH;
         for (int x = tid; x < DH; x += blockDim.x) {
             Elem<TC>::st(khat + e + x, s_kt[x]);
-            Elem<TC>::st(krope + e + x, s_ktr[x]);
             Elem<TC>::st(vc + e + x, s_vt[x]);
         }
         if (tid == 0) {
@@ -468,13 +474,14 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
 // ------------------------------------------------------------------ split decode step
 // grid (kDecodeSplitMax, B*Hkv), 256 threads.  A long cache is walked by several CTAs at once:
 // slice s of S = min(kDecodeSplitMax, ceil(n / kDecodeSplitSlice)) covers pairs [lo, hi) (whole
-// 32-pair words); CTAs past S leave at once, so a short cache costs one CTA as before.  Each CTA
-// updates its pairs' biases in place, marks its evictions, and leaves its partial online-softmax
-// state (per head: maximum, sum, weighted values) in the workspace; the CTA that finishes last
-// (a counter per cache; a fence before every arrival) merges the S states with the new token's
-// own term, gates, writes o and appends the token.  Compaction is deferred: pairs keep their
-// slots, evicted ones are excluded by their bias until ua_cache_compact removes them.  No CTA
-// ever waits on another.
+// 32-pair words); CTAs past S get an empty slice.  Each CTA updates its pairs' biases in place,
+// marks its evictions, and leaves its partial online-softmax state (per head: maximum, sum,
+// weighted values) in the workspace; the CTA that arrives last (a counter per cache counting
+// every CTA of the grid; a fence before every arrival) merges the states with the new token's
+// own term, gates, writes o and appends the token.  Counting every CTA, not only those with
+// pairs, means the merge -- which changes n -- happens only after all of them have read n.
+// Compaction is deferred: pairs keep their slots, evicted ones are excluded by their bias until
+// ua_cache_compact removes them.  No CTA ever waits on another.
 template <typename TC, int DH, int G, bool VAR>
 __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodeParams p) {
     const int variant = VAR ? p.variant : 0;
@@ -497,7 +504,6 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
     const int gidx = warp * L::EPW + grp;
     const size_t base = (size_t)unit * c.cap;
     TC* khat = static_cast<TC*>(c.khat);
-    TC* krope = static_cast<TC*>(c.krope);
     TC* vc = static_cast<TC*>(c.v);
 
     int n = c.n_kept[unit];
@@ -506,9 +512,9 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
         n = n < 0 ? 0 : c.cap;
     }
     const int nsl = min(kDecodeSplitMax, max(1, (n + kDecodeSplitSlice - 1) / kDecodeSplitSlice));
-    if (sl >= nsl) return;                            // block-uniform
     const int chunk = (((n + nsl - 1) / nsl) + 31) & ~31;
-    const int lo = min(n, sl * chunk), hi = min(n, lo + chunk);
+    const int lo = sl < nsl ? min(n, sl * chunk) : n;
+    const int hi = sl < nsl ? min(n, lo + chunk) : n;
     const int w0 = lo >> 5, nw = (hi - lo + 31) >> 5;
 
     // ---- new token (every CTA of the cache forms it; only the last one uses v, g)
@@ -532,22 +538,22 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
 #pragma unroll
     for (int w = 0; w < NW; ++w) tot_ss += s_red[w];
     const float den = fmaxf(sqrtf(tot_ss), 1e-12f);
-    if (tid < DH) s_kt[tid] = kx / den;
+    if (tid < DH) s_kt[il_index(tid, half)] = kx / den;     // pair-interleaved, as cached
     __syncthreads();
     for (int e = tid; e < G * half; e += blockDim.x) {
         const int vecid = e / half, m = e % half;
         float cs, sn;
         rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
         const float qa = Elem<TC>::ld(qin + vecid * DH + m), qb = Elem<TC>::ld(qin + vecid * DH + m + half);
-        s_q[vecid][m] = qa * cs - qb * sn;
-        s_q[vecid][m + half] = qb * cs + qa * sn;
+        s_q[vecid][2 * m] = qa * cs - qb * sn;
+        s_q[vecid][2 * m + 1] = qb * cs + qa * sn;
     }
     for (int m = tid; m < half; m += blockDim.x) {
         float cs, sn;
         rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
-        const float x0 = s_kt[m], x1 = s_kt[m + half];
-        s_ktr[m] = x0 * cs - x1 * sn;
-        s_ktr[m + half] = x1 * cs + x0 * sn;
+        const float x0 = s_kt[2 * m], x1 = s_kt[2 * m + 1];
+        s_ktr[2 * m] = x0 * cs - x1 * sn;
+        s_ktr[2 * m + 1] = x1 * cs + x0 * sn;
     }
     __syncthreads();
     if (variant & kVarQNorm) {
@@ -571,6 +577,9 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
     float kq[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) kq[e] = s_kt[gl * VEC + e];
+    double gt[VEC / 2];                               // this lane's RoPE frequencies / (2 pi)
+#pragma unroll
+    for (int i = 0; i < VEC / 2; ++i) gt[i] = p.rf.f[gl * (VEC / 2) + i] * 0.15915494309189535;
     float m_h[G], l_h[G], acc[G][VEC];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -581,29 +590,31 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
     }
 
     // ---- the slice: pairs [lo, hi), next pass loaded one pass ahead
-    uint4 na = make_uint4(0, 0, 0, 0), nb = na, nv = na;
+    uint4 na = make_uint4(0, 0, 0, 0), nv = na;
     float nbj = 0.f, nrk = 0.f;
+    int npj = 0;
     auto load_entry = [&](int jj) {
         if (jj < hi) {
             const size_t e = (base + jj) * DH + gl * VEC;
             na = *reinterpret_cast<const uint4*>(khat + e);
-            nb = *reinterpret_cast<const uint4*>(krope + e);
             nv = *reinterpret_cast<const uint4*>(vc + e);
             nbj = c.bias[base + jj];
             nrk = c.rk[base + jj];
+            npj = c.pos[base + jj];
         }
     };
     load_entry(lo + gidx);
     for (int c0 = lo; c0 < hi; c0 += EPB) {
         const int j = c0 + gidx;
         const bool valid = j < hi;
-        const uint4 ra = na, rb = nb, rv = nv;
+        const uint4 ra = na, rv = nv;
         const float bj = nbj, rkj = nrk;
+        const int pj = npj;
         load_entry(j + EPB);
         float xa[VEC], xb[VEC], xv[VEC];
         Vec16<TC>::unpack(ra, xa);
-        Vec16<TC>::unpack(rb, xb);
         Vec16<TC>::unpack(rv, xv);
+        rotate_pairs<VEC>(xa, xb, (double)pj, gt);
         float sim = 0.f;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) sim = fmaf(kq[e], xa[e], sim);
@@ -670,7 +681,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
     }
     __threadfence();                                   // the state, biases and bits before the arrival
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(p.split_cnt + unit, 1u) == (unsigned)(nsl - 1);
+    if (tid == 0) s_last = atomicAdd(p.split_cnt + unit, 1u) == gridDim.x - 1;
     __syncthreads();
     if (!s_last) return;
     __threadfence();
@@ -680,10 +691,10 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
     for (int e = tid; e < G * DH; e += blockDim.x) {
         const int h = e / DH, x = e % DH;
         float M = s_lt[h];
-        for (int q = 0; q < nsl; ++q) M = fmaxf(M, __ldcg(st0 + (size_t)q * SS + h));
+        for (int q = 0; q < (int)gridDim.x; ++q) M = fmaxf(M, __ldcg(st0 + (size_t)q * SS + h));
         float Ls = expf(s_lt[h] - M);
         float A = Ls * s_vt[x];
-        for (int q = 0; q < nsl; ++q) {
+        for (int q = 0; q < (int)gridDim.x; ++q) {
             const float mq = __ldcg(st0 + (size_t)q * SS + h);
             if (mq > -INFINITY) {
                 const float w = expf(mq - M);
@@ -700,7 +711,6 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
         const size_t e = (base + n) * DH;
         for (int x = tid; x < DH; x += blockDim.x) {
             Elem<TC>::st(khat + e + x, s_kt[x]);
-            Elem<TC>::st(krope + e + x, s_ktr[x]);
             Elem<TC>::st(vc + e + x, s_vt[x]);
         }
         if (tid == 0) {

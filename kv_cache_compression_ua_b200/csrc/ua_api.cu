@@ -155,8 +155,8 @@ ua_status check_cache(const ua_cache* c) {
     if (c->capacity > kMaxCapacity) return UA_ERR_UNSUPPORTED;
     if (c->d != 64 && c->d != 128) return UA_ERR_UNSUPPORTED;
     if (c->dtype != UA_F32 && c->dtype != UA_BF16) return UA_ERR_UNSUPPORTED;
-    if (!c->khat || !c->krope || !c->v || !c->bias || !c->rk || !c->pos || !c->n_kept) return UA_ERR_INVALID_ARG;
-    const void* ps[] = {c->khat, c->krope, c->v, c->bias, c->rk, c->pos, c->n_kept};
+    if (!c->khat || !c->v || !c->bias || !c->rk || !c->pos || !c->n_kept) return UA_ERR_INVALID_ARG;
+    const void* ps[] = {c->khat, c->v, c->bias, c->rk, c->pos, c->n_kept};
     for (const void* p : ps)
         if (!aligned(p, 16)) return UA_ERR_ALIGNMENT;
     return UA_OK;
@@ -165,7 +165,7 @@ ua_status check_cache(const ua_cache* c) {
 CacheView view(const ua_cache* c) {
     CacheView v;
     v.B = c->B; v.Hkv = c->Hkv; v.d = c->d; v.cap = c->capacity;
-    v.khat = c->khat; v.krope = c->krope; v.v = c->v; v.bias = c->bias; v.rk = c->rk;
+    v.khat = c->khat; v.v = c->v; v.bias = c->bias; v.rk = c->rk;
     v.pos = c->pos; v.n_kept = c->n_kept;
     return v;
 }
@@ -688,6 +688,9 @@ ua_status ua_decode_step_split(const ua_cache* c, int H, const void* q, const vo
     dp.o = o; dp.evict_bits = evict_bits; dp.kept_idx = kept_idx; dp.variant = var; dp.defer = 1;
     dp.split_cnt = static_cast<unsigned*>(ws);
     dp.split_state = reinterpret_cast<float*>(at(ws, round_up(units * 4, 256)));
+    // bf16 caches on the tensor cores (their TMA row coordinate must fit an int)
+    if (c->dtype == UA_BF16 && units * (size_t)c->capacity < (size_t)INT32_MAX)
+        return cuda_status(launch_decode_tc(dp, cs));
     return cuda_status(launch_decode_split(dp, c->dtype == UA_BF16, cs));
 }
 

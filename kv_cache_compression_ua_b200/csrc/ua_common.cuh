@@ -68,6 +68,24 @@ __device__ __forceinline__ void rope_cs(double pos, double f, float* c, float* s
     sincosf((float)r, s, c);
 }
 
+// cos / sin of the RoPE angle pos * f for a cached key, given gt = f / (2 pi) in double.  The
+// reduction works in turns: pos * gt is formed in double precision and its nearest integer
+// removed exactly, so the fraction (|r| <= 1/2) keeps ~1e-16 relative accuracy whatever the
+// position; the fp32 angle 2 pi r in [-pi, pi] then goes to the fast sine / cosine unit, whose
+// absolute error there is ~1e-6 (far below the 2^-8 relative rounding of a bf16 key).
+__device__ __forceinline__ void rope_cs_turns(double pos, double gt, float* c, float* s) {
+    const double a = pos * gt;
+    const float th = (float)(a - rint(a)) * 6.28318530717958648f;
+    __sincosf(th, s, c);
+}
+
+// Cached keys are stored pair-interleaved: element 2m holds component m and element 2m + 1
+// component m + d/2, the two components one RoPE frequency rotates together, so a lane that
+// loads 16 bytes of a key holds whole rotation pairs.
+__host__ __device__ __forceinline__ int il_index(int x, int half) {
+    return x < half ? 2 * x : 2 * (x - half) + 1;
+}
+
 // ------------------------------------------------------------------ element access
 template <typename T> struct Elem;
 template <> struct Elem<float> {

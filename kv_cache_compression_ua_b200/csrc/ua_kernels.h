@@ -86,8 +86,7 @@ cudaError_t launch_tile_qmax(const TileQmaxParams& p, cudaStream_t s);
 
 struct CacheView {
     int B, Hkv, d, cap;
-    void* khat;
-    void* krope;
+    void* khat;          // pair-interleaved unit keys (see il_index)
     void* v;
     float* bias;
     float* rk;
@@ -143,6 +142,9 @@ struct DecodeParams {
 constexpr int kDecodeSplitMax = 16;
 constexpr int kDecodeSplitSlice = 512;
 cudaError_t launch_decode_split(const DecodeParams& p, bool bf16, cudaStream_t s);
+// The split step of a bf16 cache on the tensor cores (k_decode_tc.cu): same contract and
+// workspace as launch_decode_split; group sizes 1-4 and 8.
+cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t s);
 
 // Backward (SIMT path).  Inputs from the f32 token preparation and boundary pass (query
 // tiles of 64 rows); f32 intermediates in the workspace; outputs in the caller's layouts.

@@ -43,7 +43,7 @@ DECODE_DEFER_COMPACT = 256      # ua_decode_step flag: leave evicted pairs in pl
 
 class ua_cache(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int), ("capacity", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("khat", ctypes.c_void_p), ("krope", ctypes.c_void_p),
+                ("dtype", ctypes.c_int), ("khat", ctypes.c_void_p),
                 ("v", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("rk", ctypes.c_void_p),
                 ("pos", ctypes.c_void_p), ("n_kept", ctypes.c_void_p)]
 
@@ -308,14 +308,15 @@ def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, d_o, *, scal
 
 @dataclass
 class Cache:
-    """Device tensors of one self-pruning cache set (see ua_cache in ua.h)."""
+    """Device tensors of one self-pruning cache set (see ua_cache in ua.h).  khat holds the unit
+    keys pair-interleaved (element 2m = component m, 2m+1 = component m + d/2); `khat_natural()`
+    returns them in the natural order."""
     B: int
     Hkv: int
     d: int
     capacity: int
     dtype: torch.dtype
     khat: torch.Tensor
-    krope: torch.Tensor
     v: torch.Tensor
     bias: torch.Tensor
     rk: torch.Tensor
@@ -328,7 +329,6 @@ class Cache:
         return Cache(B, Hkv, d, capacity, dtype,
                      torch.zeros(B, Hkv, capacity, d, dtype=dtype, **kw),
                      torch.zeros(B, Hkv, capacity, d, dtype=dtype, **kw),
-                     torch.zeros(B, Hkv, capacity, d, dtype=dtype, **kw),
                      torch.zeros(B, Hkv, capacity, dtype=torch.float32, **kw),
                      torch.zeros(B, Hkv, capacity, dtype=torch.float32, **kw),
                      torch.zeros(B, Hkv, capacity, dtype=torch.int32, **kw),
@@ -336,20 +336,27 @@ class Cache:
 
     def struct(self) -> ua_cache:
         n = self.B * self.Hkv * self.capacity
-        for name in ("khat", "krope", "v"):
+        for name in ("khat", "v"):
             _need(f"cache.{name}", getattr(self, name), n * self.d, (self.dtype,))
         _need("cache.bias", self.bias, n, F32)
         _need("cache.rk", self.rk, n, F32)
         _need("cache.pos", self.pos, n, I32)
         _need("cache.n_kept", self.n_kept, self.B * self.Hkv, I32)
-        names = ("khat", "krope", "v", "bias", "rk", "pos", "n_kept")
+        names = FIELDS
         dev = self.khat.device
         _same_device(dev, **{f"cache.{n}": getattr(self, n) for n in names})
         ptrs = [_ptr(getattr(self, n)).value for n in names]
         return ua_cache(self.B, self.Hkv, self.d, self.capacity, _dtype_code(self.dtype), *ptrs)
 
     def nbytes_per_entry(self) -> int:
-        return 3 * self.d * self.khat.element_size() + 12
+        return 2 * self.d * self.khat.element_size() + 12
+
+    def khat_natural(self) -> torch.Tensor:
+        """khat with the components in their natural order (a copy)."""
+        return torch.cat([self.khat[..., 0::2], self.khat[..., 1::2]], dim=-1)
+
+
+FIELDS = ("khat", "v", "bias", "rk", "pos", "n_kept")
 
 
 def cache_fill(cache: Cache, k, v, a_k, b_final, *, theta=500000.0, stream=None):

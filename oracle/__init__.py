@@ -53,7 +53,7 @@ def _load():
         lib.ora_decode_step.restype = I
         lib.ora_compact_order.argtypes = [I, P, P]
         lib.ora_compact_order.restype = I
-        lib.ora_prefill_bwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 8 + [I, I]
+        lib.ora_prefill_bwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 8 + [I, Dd, I]
         lib.ora_prefill_bwd.restype = I
         _lib = lib
     return _lib
@@ -122,9 +122,15 @@ def lambda_bruteforce(k, a_q, a_k, alpha, beta, variant=0, nthreads=None):
 
 
 def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, d_o, *, scale=None, theta=500000.0,
-                unit_mask=None, variant=0, nthreads=None):
+                unit_mask=None, variant=0, bf16_saved_model=0.0, nthreads=None):
     """Analytic fp64 gradients of sum(dO * O).  Returns a dict keyed dq, dk, dv, dg,
-    da_q, da_k, dalpha, dbeta (same shapes as the inputs)."""
+    da_q, da_k, dalpha, dbeta (same shapes as the inputs).
+
+    bf16_saved_model = c > 0: a model for tolerances, not the method.  The backward is fed what
+    a bf16 forward saves: probabilities rounded to bf16 (scaled by c <= 1 first, standing in for
+    a softmax shift above the row maximum) in the output and its normaliser, the output itself
+    rounded to bf16, and delta_i = sum_x dO_ix o_ix formed from it.  Every gradient then moves
+    by about -sum_i eps_i grad(lse_i), eps_i the resulting error of row i's (dP - delta)."""
     q, k, v, g, d_o = _f64(q), _f64(k), _f64(v), _f64(g), _f64(d_o)
     a_q, a_k, alpha, beta = _f64(a_q), _f64(a_k), _f64(alpha), _f64(beta)
     B, T, H, d = q.shape
@@ -142,7 +148,7 @@ def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, d_o, *, scale=None, theta=500
                                  _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
                                  _ptr(out["dg"]), _ptr(out["da_q"]), _ptr(out["da_k"]),
                                  _ptr(out["dalpha"]), _ptr(out["dbeta"]), int(variant),
-                                 nthreads or default_threads())
+                                 float(bf16_saved_model), nthreads or default_threads())
     if rc != 0:
         raise ValueError(f"ora_prefill_bwd rejected the shapes (code {rc})")
     return out

@@ -510,6 +510,17 @@ int ora_compact_order(int n, const uint8_t* keep, int64_t* order) {
  *   dq = r (dq' - q' <q', dq'> / d), dq' = RoPE^T dqrot.
  * Lambda and dLambda are held as packed lower-triangular T x T matrices per unit.
  * dalpha / dbeta are summed over the batch: [Hkv].
+ *
+ * Saved-output model (optional, for deriving tolerances only; model_c > 0): the backward is
+ * fed what a bf16 forward saves.  That forward rounds each unnormalised probability
+ * e_ij = c exp(s_ij - m_i) to bf16 before its PV and row-sum products (c <= 1: its softmax
+ * shift need not be the row maximum; c picks which values round up), so its normaliser is
+ * l_i = sum_j bf16(c e_ij) / c and its output o = sigmoid(g) (.) sum_j bf16(c e_ij) v_j / (c l_i),
+ * stored in bf16.  The backward recomputes P_ij = e_ij / l_i from the saved lse (rows then sum to
+ * 1 + eta_i, not 1) and forms delta_i = sum_x dO_ix o_ix from the saved output.  In exact
+ * arithmetic all of this is the method; each row's error eps_i in (dP - delta) terms moves
+ * every gradient by about -sum_i eps_i * grad(lse_i) (an extra -eps_i P_ij in dS_ij is the
+ * derivative of -eps_i lse_i), which the per-head sums dalpha, dbeta feel most.
  */
 typedef struct {
     int B, T, H, Hkv, d;
@@ -519,7 +530,22 @@ typedef struct {
     double *dq, *dk, *dv, *dg, *daq, *dak;
     double *dalpha_u, *dbeta_u; /* per unit partials [B*Hkv] */
     int variant;
+    double model_c;             /* saved-output model (see above); 0 = off */
 } bwd_ctx;
+
+/* Nearest bf16 value (8 significant bits) of x, ties to even, by way of the nearest float.
+ * Used only by the saved-output model. */
+static double round_bf16(double x) {
+    float f = (float)x;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) != 0x7f800000u) {
+        u += 0x7fffu + ((u >> 16) & 1u);
+        u &= 0xffff0000u;
+        memcpy(&f, &u, sizeof f);
+    }
+    return (double)f;
+}
 
 static size_t tri(int i, int j) { return (size_t)i * (size_t)(i + 1) / 2 + (size_t)j; }
 
@@ -580,14 +606,19 @@ static void bwd_unit(void* vctx, int unit) {
                 P[j] = s * dot(qrot, krot + (size_t)j * d, d) + lam[tri(i, j)];
                 if (P[j] > m) m = P[j];
             }
+            const double mc = c->model_c;
             double l = 0.0;
-            for (int j = 0; j <= i; ++j) { P[j] = exp(P[j] - m); l += P[j]; }
-            for (int j = 0; j <= i; ++j) P[j] /= l;
+            for (int j = 0; j <= i; ++j) {
+                P[j] = exp(P[j] - m);
+                l += mc > 0.0 ? round_bf16(mc * P[j]) / mc : P[j];
+            }
             for (int x = 0; x < d; ++x) A[x] = 0.0;
             for (int j = 0; j <= i; ++j) {
                 const double* vj = c->v + (((size_t)b * T + j) * Hkv + kvh) * d;
-                for (int x = 0; x < d; ++x) A[x] += P[j] * vj[x];
+                const double pj = (mc > 0.0 ? round_bf16(mc * P[j]) / mc : P[j]) / l;
+                for (int x = 0; x < d; ++x) A[x] += pj * vj[x];
             }
+            for (int j = 0; j <= i; ++j) P[j] /= l;
             double* dgi = c->dg + (((size_t)b * T + i) * H + h) * d;
             for (int x = 0; x < d; ++x) {
                 double sg = sigmoid(gi[x]);
@@ -599,6 +630,10 @@ static void bwd_unit(void* vctx, int unit) {
                 const double* vj = c->v + (((size_t)b * T + j) * Hkv + kvh) * d;
                 dP[j] = dot(dA, vj, d);
                 delta += P[j] * dP[j];
+            }
+            if (mc > 0.0) {
+                delta = 0.0;
+                for (int x = 0; x < d; ++x) delta += doi[x] * round_bf16(sigmoid(gi[x]) * A[x]);
             }
             for (int x = 0; x < d; ++x) dqrot[x] = 0.0;
             for (int j = 0; j <= i; ++j) {
@@ -675,13 +710,13 @@ int ora_prefill_bwd(int B, int T, int H, int Hkv, int d, double scale, double th
                     const double* aq, const double* ak, const double* alpha, const double* beta,
                     const double* dout, const uint8_t* unit_mask,
                     double* dq, double* dk, double* dv, double* dg, double* daq, double* dak,
-                    double* dalpha, double* dbeta, int variant, int nthreads) {
+                    double* dalpha, double* dbeta, int variant, double model_c, int nthreads) {
     if (B < 1 || T < 1 || H < 1 || Hkv < 1 || d < 2 || (d & 1) || H % Hkv) return 1;
     if ((variant & ~VAR_ALL) || n_active(variant) == 0) return 1;
     double* dal_u = (double*)calloc((size_t)B * Hkv, sizeof(double));
     double* dbe_u = (double*)calloc((size_t)B * Hkv, sizeof(double));
     bwd_ctx c = {B, T, H, Hkv, d, scale, theta, q, k, v, g, aq, ak, alpha, beta, dout,
-                 unit_mask, dq, dk, dv, dg, daq, dak, dal_u, dbe_u, variant};
+                 unit_mask, dq, dk, dv, dg, daq, dak, dal_u, dbe_u, variant, model_c > 0.0 ? model_c : 0.0};
     run_units(bwd_unit, &c, B * Hkv, nthreads);
     for (int h = 0; h < Hkv; ++h) {
         dalpha[h] = 0.0;

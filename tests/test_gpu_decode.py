@@ -226,7 +226,7 @@ def test_compact_with_explicit_mask_is_stable_partition():
     r = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"])
     cache = ua.Cache.empty(2, 2, 128, 1000, dt)
     ua.cache_fill(cache, d["k"], d["v"], d["a_k"], r["b_final"])
-    before = {n: getattr(cache, n).clone() for n in ("khat", "krope", "v", "bias", "rk", "pos")}
+    before = {n: getattr(cache, n).clone() for n in ("khat", "v", "bias", "rk", "pos")}
     rng = np.random.default_rng(0)
     keep = (rng.random((2, 2, 1000)) < 0.37).astype(np.uint8)
     kept = torch.full((2, 2, 1000), -7, dtype=torch.int32, device="cuda")
@@ -308,7 +308,7 @@ def test_deferred_compaction_matches_step_by_step(dtype):
     ua.cache_compact(lazy, p)
     np.testing.assert_array_equal(lazy.n_kept.cpu().numpy(), eager.n_kept.cpu().numpy())
     n_e = eager.n_kept.cpu().numpy()
-    for name in ("pos", "bias", "rk", "khat", "krope", "v"):
+    for name in ("pos", "bias", "rk", "khat", "v"):
         a, b_ = getattr(lazy, name).float().cpu().numpy(), getattr(eager, name).float().cpu().numpy()
         for b in range(w.B):
             for h in range(w.Hkv):
@@ -317,3 +317,34 @@ def test_deferred_compaction_matches_step_by_step(dtype):
                     assert_close("bias", a[b, h, :m], b_[b, h, :m], "f32", relative_max=True)
                 else:
                     np.testing.assert_array_equal(a[b, h, :m], b_[b, h, :m], err_msg=name)
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 64), ("f32", 128)])
+def test_cache_fill_layout(dtype, d):
+    """ua_cache_fill stores the unit keys pair-interleaved (no rotated copy), the values, the
+    biases, softplus(a_k) and the positions, slot t <- token t."""
+    w = I.Workload("fill", 2, 37, 2 * 2, 2, d, dtype, 91)
+    x = I.make_prefill_inputs(w, names=["k", "v", "a_k"])
+    adt = TORCH_DT[dtype]
+    k, v, ak = dev(x["k"], adt), dev(x["v"], adt), dev(x["a_k"], torch.float32)
+    bf = torch.randn(w.B, w.Hkv, w.T, device="cuda")
+    cache = ua.Cache.empty(w.B, w.Hkv, d, 50, adt)
+    ua.cache_fill(cache, k, v, ak, bf, theta=w.theta)
+    torch.cuda.synchronize()
+    assert ua.get_device_status() == 0
+    assert cache.nbytes_per_entry() == 2 * d * (2 if dtype == "bf16" else 4) + 12
+    np.testing.assert_array_equal(cache.n_kept.cpu().numpy(), np.full((w.B, w.Hkv), w.T))
+    kf = k.float()
+    khat = (kf / kf.norm(dim=-1, keepdim=True)).permute(0, 2, 1, 3)           # [B,Hkv,T,d]
+    got = cache.khat_natural()[:, :, :w.T].float()
+    tol = 4e-3 if dtype == "bf16" else 1e-6
+    assert float((got - khat).abs().max()) <= tol
+    # pair-interleaved: element 2m is component m, element 2m+1 component m + d/2
+    h = d // 2
+    assert float((cache.khat[:, :, :w.T, 2 * 3].float() - khat[..., 3]).abs().max()) <= tol
+    assert float((cache.khat[:, :, :w.T, 2 * 5 + 1].float() - khat[..., h + 5]).abs().max()) <= tol
+    assert torch.equal(cache.v[:, :, :w.T], v.permute(0, 2, 1, 3))
+    assert torch.equal(cache.bias[:, :, :w.T], bf)
+    assert torch.equal(cache.pos[:, :, :w.T].cpu(), torch.arange(w.T, dtype=torch.int32).expand(w.B, w.Hkv, w.T))
+    rk = torch.nn.functional.softplus(ak).permute(0, 2, 1)
+    assert float((cache.rk[:, :, :w.T] - rk).abs().max()) <= 1e-6

@@ -1,0 +1,124 @@
+"""GPU parity of the split decode step of bf16 caches on the tensor cores (k_decode_tc, through
+ua_decode_step_split) against the fp64 oracle in lockstep, compaction deferred.
+
+Long caches (2.2k-4.1k live pairs: 5-8 slices of whole 128-entry tiles, ragged last tiles) and a
+130-pair one over 12 steps at p = 0.15 (evictions in every slice) and p = 0; group sizes 1, 2, 3, 4
+and 8; head dims 64 and 128.  Both sides start from the oracle prefill's biases.  Eviction
+decisions must match the oracle's except within 1e-3 of log p, where the oracle adopts the GPU's
+decision; outputs and the live biases are held to the bf16 bars.  A case with large query norms
+drives the softmax shift up through the in-TMEM rescale, and a final ua_cache_compact must give
+the oracle's compacted cache."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_compression_ua_b200 import inputs as I
+from kv_cache_compression_ua_b200 import ua
+from helpers import EVICT_BAND, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def dev(a, dt):
+    return torch.from_numpy(np.ascontiguousarray(a)).to("cuda").to(dt).contiguous()
+
+
+def unpack_bits(words, n):
+    bits = np.unpackbits(np.ascontiguousarray(words, np.uint32).view(np.uint8), bitorder="little")
+    return bits[:n].astype(bool)
+
+
+def run_lockstep(w, T0, steps, p, q_gain=1.0):
+    bf = torch.bfloat16
+    x = I.make_prefill_inputs(w, T=T0, names=["q", "k", "v", "g", "a_q", "a_k", "alpha", "beta"])
+    dd = {n: dev(a, bf if n in ("k", "v", "q", "g") else torch.float32) for n, a in x.items()}
+    # both caches start from the oracle prefill's biases, so the steps are checked on their own
+    # (the prefill's b_final is checked elsewhere)
+    ob = oracle.prefill_fwd(**x, scale=w.scale, theta=w.theta, row_mask=np.zeros(T0, np.uint8))["b_final"]
+    cap = T0 + steps + 1
+    cache = ua.Cache.empty(w.B, w.Hkv, w.d, cap, bf)
+    ua.cache_fill(cache, dd["k"], dd["v"], dd["a_k"], dev(ob, torch.float32), theta=w.theta)
+    ws = ua.alloc_workspace(ua.decode_workspace_size(cache, w.H), "cuda")
+    oc = oracle.DecodeCache(w.B, w.Hkv, w.d, cap)
+    oc.fill_from_prefill(x["k"], x["v"], x["a_k"], ob)
+    logp = math.log(p) if p > 0 else -math.inf
+    words = (cap + 31) // 32
+    alpha, beta = dd["alpha"].cpu().numpy(), dd["beta"].cpu().numpy()
+    ua.profile_reset()
+    ua.profile_enable(True)
+    n_evicted = n_adopted = 0
+    try:
+        for s in range(steps):
+            tok = I.make_decode_token(w, s)
+            tok["q"] = I.round_bf16(tok["q"].astype(np.float64) * q_gain).astype(np.float32)
+            t = {n: dev(a, bf if n in ("q", "k", "v", "g") else torch.float32) for n, a in tok.items()}
+            n_before = cache.n_kept.cpu().numpy()
+            ev = torch.full((w.B, w.Hkv, words), -1, dtype=torch.int32, device="cuda")
+            kept = torch.full((w.B, w.Hkv, cap), -7, dtype=torch.int32, device="cuda")
+            o = ua.decode_step(cache, t["q"], t["k"], t["v"], t["g"], t["a_q"], t["a_k"], dd["alpha"], dd["beta"],
+                               T0 + s, p, scale=w.scale, theta=w.theta, evict_bits=ev, kept_idx=kept, ws=ws)
+            torch.cuda.synchronize()
+            assert ua.get_device_status() == 0
+            ev = ev.cpu().numpy().view(np.uint32)
+            kept = kept.cpu().numpy()
+            gpu_ev = np.zeros((w.B, w.Hkv, cap), bool)
+            for b in range(w.B):
+                for h in range(w.Hkv):
+                    m = n_before[b, h]
+                    gpu_ev[b, h, :m] = unpack_bits(ev[b, h], m)
+                    assert not unpack_bits(ev[b, h], words * 32)[m:].any(), "eviction bits past the live pairs"
+                    np.testing.assert_array_equal(kept[b, h, :m], np.arange(m))
+                    assert kept[b, h, m] == -1
+            ro = oracle.decode_step(oc, tok["q"], tok["k"], tok["v"], tok["g"], tok["a_q"], tok["a_k"], alpha,
+                                    beta, T0 + s, p, scale=w.scale, theta=w.theta, band=EVICT_BAND,
+                                    adopt_keep=(~gpu_ev).astype(np.uint8), defer=True)
+            inb = ro["in_band"].astype(bool)
+            mism = (ro["evict"].astype(bool) != gpu_ev) & ~inb
+            assert not mism.any(), f"step {s}: eviction differs outside the band at {np.argwhere(mism)[:5]}"
+            n_adopted += int(inb.sum())
+            n_evicted += int(gpu_ev.sum())
+            np.testing.assert_array_equal(cache.n_kept.cpu().numpy(), n_before + 1)
+            np.testing.assert_array_equal(oc.n, n_before + 1)
+            assert_close(f"o step {s}", o.float().cpu().numpy(), ro["o"], "bf16")
+            gb = cache.bias.cpu().numpy()
+            for b in range(w.B):
+                for h in range(w.Hkv):
+                    m = n_before[b, h] + 1
+                    live = oc.b[b, h, :m] >= logp
+                    assert_close(f"bias step {s}", gb[b, h, :m][live], oc.b[b, h, :m][live], "bf16",
+                                 relative_max=True)
+                    np.testing.assert_array_equal(cache.pos[b, h, :m].cpu().numpy(), oc.pos[b, h, :m])
+    finally:
+        ua.profile_enable(False)
+    names = set(ua.profile_read())
+    assert "k_decode_tc" in names, names
+    if p > 0:
+        assert n_evicted > 0
+        kept = torch.full((w.B, w.Hkv, cap), -7, dtype=torch.int32, device="cuda")
+        ua.cache_compact(cache, p, kept_idx=kept)
+        oc.compact(p)
+        np.testing.assert_array_equal(cache.n_kept.cpu().numpy(), oc.n)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                m = oc.n[b, h]
+                np.testing.assert_array_equal(cache.pos[b, h, :m].cpu().numpy(), oc.pos[b, h, :m])
+    return n_evicted, n_adopted
+
+
+@pytest.mark.parametrize("d,H,Hkv,T0,p", [(64, 8, 2, 2600, 0.15), (64, 4, 2, 3001, 0.15), (128, 6, 2, 4095, 0.15),
+                                          (64, 8, 1, 2500, 0.0), (64, 16, 2, 2700, 0.15), (128, 2, 2, 2222, 0.0),
+                                          (64, 3, 3, 130, 0.15)])
+def test_tensor_core_split_decode_lockstep(d, H, Hkv, T0, p):
+    w = I.Workload("dec_tc", 2, T0, H, Hkv, d, "bf16", 6100 + T0 + H, bimodal_ak=True)
+    run_lockstep(w, T0, 12, p)
+
+
+def test_tensor_core_split_decode_large_query_norms():
+    """Queries scaled so that scale*||q|| reaches ~60: the logits spread over far more than the
+    shift's 16-nat headroom, so the shift is raised (and the accumulated values rescaled in
+    TMEM) tile by tile."""
+    w = I.Workload("dec_tc_qn", 1, 2600, 8, 2, 64, "bf16", 6177, bimodal_ak=True)
+    run_lockstep(w, 2600, 6, 0.15, q_gain=60.0)

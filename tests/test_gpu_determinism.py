@@ -78,7 +78,7 @@ def test_decode_is_deterministic():
                                w.T + s, 0.15, scale=w.scale, theta=w.theta)
             os_.append(o.clone())
         torch.cuda.synchronize()
-        outs.append((os_, {n: getattr(c, n).clone() for n in ("khat", "krope", "v", "bias", "rk", "pos", "n_kept")}))
+        outs.append((os_, {n: getattr(c, n).clone() for n in ("khat", "v", "bias", "rk", "pos", "n_kept")}))
     assert ua.get_device_status() == 0
     for a, b in zip(outs[0][0], outs[1][0]):
         assert torch.equal(a, b)

@@ -14,7 +14,7 @@ import torch
 import oracle
 from kv_cache_compression_ua_b200 import inputs as I
 from kv_cache_compression_ua_b200 import ua
-from helpers import assert_close
+from helpers import assert_close, assert_grad_close, sum_model_rms
 
 pytestmark = pytest.mark.gpu
 TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -116,6 +116,8 @@ def test_backward_every_variant(variant, dtype, d):
     assert ua.get_device_status() == 0
     g = {k: v.float().cpu().numpy() for k, v in gr.items()}
     r = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta, variant=variant)
+    rms = (sum_model_rms(oracle.prefill_bwd, r, **x, scale=w.scale, theta=w.theta, variant=variant)
+           if dtype == "bf16" else None)
     off = set()
     for bit, names in OFF_GRADS.items():
         if variant & bit:
@@ -125,4 +127,4 @@ def test_backward_every_variant(variant, dtype, d):
         if n in off:
             assert np.all(g[n] == 0.0), n          # a switched-off mechanism has no gradient
             continue
-        assert_close(n, g[n], r[n], dtype, tensor_scale=True)
+        assert_grad_close(n, g[n], r[n], dtype, rms)

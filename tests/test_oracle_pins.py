@@ -410,3 +410,47 @@ def test_rope_relative_position_invariance(shift):
     np.testing.assert_array_equal(moved.n, base.n)
     np.testing.assert_array_equal(moved.pos - shift, base.pos)
     np.testing.assert_array_equal(moved.b, base.b)
+
+
+@pytest.mark.parametrize("c", [1.0, 0.9, 0.55])
+def test_bf16_saved_output_model_single_token_closed_form(c):
+    """The oracle backward's bf16 saved-output model (a tolerance model, not the method) on one
+    token, where every quantity has a closed form: the probability's bf16 rounding of c gives
+    the backward P = c / bf16(c), the output A = v, delta = sum dO * bf16(sigmoid(g) v), and at
+    position 0 RoPE is the identity, so dq = scale * P * (<dA, v> - delta) * khat,
+    dv = P * dA, dg = dO * v * sigmoid'(g); no pair, so dalpha = dbeta = 0.  The rounding is
+    torch's bf16 conversion (round to nearest even)."""
+    rng = np.random.default_rng(11)
+    d, H, Hkv = 64, 2, 1
+    x = {"q": rng.standard_normal((1, 1, H, d)), "k": rng.standard_normal((1, 1, Hkv, d)),
+         "v": rng.standard_normal((1, 1, Hkv, d)), "g": rng.standard_normal((1, 1, H, d)),
+         "a_q": rng.standard_normal((1, 1, Hkv)), "a_k": rng.standard_normal((1, 1, Hkv)),
+         "alpha": np.array([2.0]), "beta": np.array([-1.0]), "d_o": rng.standard_normal((1, 1, H, d))}
+    scale = d ** -0.5
+    ex = oracle.prefill_bwd(**x, scale=scale)
+    mo = oracle.prefill_bwd(**x, scale=scale, bf16_saved_model=c)
+    bf = lambda a: torch.tensor(np.asarray(a, np.float64)).float().bfloat16().double().numpy()
+    v = x["v"][0, 0, 0]
+    khat = x["k"][0, 0, 0] / np.linalg.norm(x["k"][0, 0, 0])
+    P = c / float(bf(c))
+    for h in range(H):
+        sg = 1.0 / (1.0 + np.exp(-x["g"][0, 0, h]))
+        dA = x["d_o"][0, 0, h] * sg
+        delta = float(np.sum(x["d_o"][0, 0, h] * bf(sg * v)))
+        dS = P * (float(dA @ v) - delta)
+        np.testing.assert_allclose(mo["dq"][0, 0, h], scale * dS * khat, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(mo["dg"][0, 0, h], x["d_o"][0, 0, h] * v * sg * (1 - sg), rtol=1e-12)
+        np.testing.assert_allclose(ex["dq"][0, 0, h], 0.0, atol=1e-14)      # exact: dS = 0 at T = 1
+    dA_sum = sum(x["d_o"][0, 0, h] / (1.0 + np.exp(-x["g"][0, 0, h])) for h in range(H))
+    np.testing.assert_allclose(mo["dv"][0, 0, 0], P * dA_sum, rtol=1e-12)
+    np.testing.assert_allclose(ex["dv"][0, 0, 0], dA_sum, rtol=1e-12)
+    assert mo["dalpha"][0] == 0.0 and mo["dbeta"][0] == 0.0
+
+
+def test_bf16_saved_output_model_off_is_the_method():
+    w = I.Workload("m0", 1, 40, 4, 2, 64, "bf16", 5, with_grad=True)
+    x = I.make_prefill_inputs(w)
+    a = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta)
+    b = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta, bf16_saved_model=0.0)
+    for n in a:
+        np.testing.assert_array_equal(a[n], b[n])
