@@ -5,34 +5,31 @@
 // attend over the survivors with the bias added to their logits; ai4snews synopsis, eviction
 // paragraph).  The pages name fused kernels for the pruned cache as missing (summary §6,
 // App. H); this is the long-cache one.  A cache walked entry by entry on the CUDA cores spends
-// ~140 warp instructions per entry (one similarity and G logit dot products, G online-softmax
-// updates), several times its memory time, so here the dot products run as two small tcgen05
-// products per 128-entry tile, with one thread per cached entry for the rest:
+// ~140 warp instructions per entry (one similarity and G logit dot products spread over lanes
+// with shuffle reductions, G online-softmax updates), several times its memory time, so here a
+// 128-entry tile is one thread per entry plus two small tcgen05 products:
 //
-//   [X | S] = [khat_j | RoPE(khat_j, pos_j)] . [khat_t | RoPE(q_h, pos_t)]^T    (M = 128 entries)
-//   O^T    += V^T . P                                                         (M = head dims)
+//   thread j:  x_j = <khat_t, khat_j> (fp32, from the bf16 entry in shared memory), and the
+//              entry rotated in place to RoPE(khat_j, pos_j) (the cache keeps no rotated copy:
+//              unit keys are stored pair-interleaved, so a 16-byte chunk holds whole pairs)
+//   S   = RoPE(khat) . [q_h high parts | q_h residuals]^T        (M = 128 entries, N = 16)
+//   thread j:  decay D, bias update, eviction bit, probabilities P_hj (bf16) from x_j and S
+//   O^T += V^T . P                                                (M = head dims, N = 16)
 //
-// The B operand of the first product holds the new key and the G rotated queries, each split
-// into a bf16 high part and its bf16 residual, so the similarity and the logits carry ~16
-// significant bits on the query side (the cache itself is bf16).  The cache stores unit keys
-// pair-interleaved and no rotated copy; each thread rotates its own entry by its position
-// (rope_cs_turns) into a shared tile that the first product reads.  Thread j then turns its
-// row of X and S into the decay D, the updated bias, the eviction bit and the probabilities,
-// writes them (bf16) into the B operand of the second product, and that product accumulates
-// the weighted values in TMEM.
+// Each query enters as a bf16 high part and its bf16 residual, so the logits carry the query
+// to ~16 bits (the cache itself is bf16).  Softmax shift: probabilities are exp(logit - shift_h),
+// one shift per head, started at the new token's own logit (a lower bound of the row maximum)
+// and raised, with the accumulated values rescaled in TMEM, whenever a tile's maximum exceeds it
+// by more than 16; so no probability exceeds e^16 and none that matters underflows.
 //
-// Softmax shift: the probabilities are exp(logit - shift_h) with one shift per head, started
-// at the new token's own logit (a lower bound of the row maximum) and raised, with the
-// accumulated values rescaled in TMEM, whenever a tile's maximum exceeds it by more than 16;
-// so no probability exceeds e^16 and none that matters underflows, for any query norm.
-//
-// Work split: grid (kDecodeSplitMax, B*Hkv).  Cache (b, h) with n live slots is cut into
-// slices of whole 128-entry tiles; every CTA of the cache leaves a partial softmax state
-// (shift, sum, weighted values) in the workspace -- a CTA past the last slice an empty one --
-// and the CTA that arrives last (a counter per cache, a fence before every arrival) merges
-// them with the new token, gates, writes o and appends the token.  Counting every CTA of the
-// grid, not only those with a slice, means the merge (which changes n) happens only after all
-// of them have read n.  Compaction is deferred (pairs keep their slots; ua_cache_compact later).
+// Work split: grid (kDecodeSplitMax, B*Hkv), two or three 128-thread CTAs per SM.  Cache (b, h)
+// with n live slots is cut into slices of whole 128-entry tiles; each CTA with a slice leaves a
+// partial softmax state (shift, sum, weighted values) in the workspace, and the CTA that arrives
+// last (a counter per cache that every CTA of the grid increments, a fence before every
+// arrival) merges them with the new token, gates, writes o and appends the token.  A CTA without
+// a slice arrives at once and only builds the new token if it turns out to be last.  Counting
+// every CTA means the merge (which changes n) happens only after all of them have read n.
+// Compaction is deferred (pairs keep their slots; ua_cache_compact removes the evicted ones).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -55,28 +52,27 @@ constexpr float kRescaleGap = 16.f;     // raise the shift when a logit exceeds 
 template <int DH, int G>
 struct DecTc {
     static constexpr int NB = DH / 64;                       // 64-column (128-byte) boxes per row
-    static constexpr int NQ = (2 + 2 * G) <= 16 ? 16 : 32;   // columns of the first product
-    static constexpr int NST = DH == 64 ? 4 : 2;             // stages of (khat, v) tiles
-    static constexpr int COL_S = 0, COL_O = 32, TMEM_COLS = 64;
+    static constexpr int NST = DH == 64 ? 2 : 1;             // stages of (khat, v) tiles
+    static constexpr int CTAS = DH == 64 ? 3 : 2;            // CTAs per SM the footprint allows
+    static constexpr int COL_S = 0, COL_O = 16, TMEM_COLS = 32;
     static constexpr int SS = G * (DH + 2);                  // floats of one partial state
 };
 
 template <int DH, int G>
 struct DecTcSmem {
     using C = DecTc<DH, G>;
-    // per stage: NB boxes of khat then NB boxes of v, each [128 entries][64] bf16, 128-byte
-    // swizzle; the v boxes are followed by at least 16 KB of shared memory (the next stage or
-    // krot), which the second product's upper 64 rows read harmlessly when DH = 64
+    // per stage: NB boxes of v then NB boxes of khat (rotated in place), each [128 entries][64]
+    // bf16 with the 128-byte swizzle.  The second product's M = 128 rows are the head dims in
+    // 64-row atoms one box apart; when DH = 64 its upper atom reads the stage's khat box, whose
+    // rows of the result are never read.
     alignas(1024) uint8_t stage[C::NST][2 * C::NB][16384];
-    alignas(1024) uint8_t krot[C::NB][16384];                // RoPE(khat_j, pos_j), same layout
-    alignas(1024) uint8_t bqk[C::NQ * 2 * DH * 2];           // no-swizzle K-major B of [X | S]
+    alignas(1024) uint8_t bq[16 * DH * 2];                   // no-swizzle K-major B of S
     alignas(128) uint8_t pt[2][kDecTile][16];                // P: MN-major no-swizzle, heads 0-7 | 8-15
     double gtf[DH / 2];                                       // RoPE frequencies / (2 pi)
     float kt[DH];                                            // khat_t, pair-interleaved
     float ktr[DH];                                           // RoPE(khat_t, pos_t), pair-interleaved
     float vt[DH];
     float q[G][DH];                                          // RoPE(q_h, pos_t), pair-interleaved
-    float gate[G * DH];
     float own[G];                                            // the new token's own logits
     float qn[G];
     float shift[G];
@@ -89,8 +85,8 @@ struct DecTcSmem {
     int last;
 };
 
-// New token of the cache: khat_t, RoPE(khat_t), v_t, RoPE(q_h) (query norm applied), the gate and
-// the own logits, into shared memory.  All 128 threads.
+// New token of the cache: khat_t, RoPE(khat_t), v_t, RoPE(q_h) (query norm applied) and the own
+// logits, into shared memory.  All 128 threads; ends with a barrier.
 template <int DH, int G>
 __device__ void new_token(DecTcSmem<DH, G>& S, const DecodeParams& p, int unit, int b, int kvh) {
     constexpr int half = DH / 2;
@@ -98,52 +94,53 @@ __device__ void new_token(DecTcSmem<DH, G>& S, const DecodeParams& p, int unit, 
     const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(p.k) + (size_t)unit * DH;
     const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(p.v) + (size_t)unit * DH;
     const __nv_bfloat16* qin = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
-    const __nv_bfloat16* gin = static_cast<const __nv_bfloat16*>(p.g) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     float kx = 0.f;
     if (tid < DH) {
         kx = __bfloat162float(kin[tid]);
         S.vt[tid] = __bfloat162float(vin[tid]);
     }
-    for (int e = tid; e < G * DH; e += blockDim.x) S.gate[e] = __bfloat162float(gin[e]);
     float ss = kx * kx;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) S.red2[warp] = ss;
+    for (int m = tid; m < half; m += blockDim.x) S.gtf[m] = p.rf.f[m] * 0.15915494309189535;
     __syncthreads();
     const float den = fmaxf(sqrtf(S.red2[0] + S.red2[1] + S.red2[2] + S.red2[3]), 1e-12f);
     if (tid < DH) S.kt[il_index(tid, half)] = kx / den;
-    for (int m = tid; m < half; m += blockDim.x) S.gtf[m] = p.rf.f[m] * 0.15915494309189535;
     __syncthreads();
-    for (int e = tid; e < G * half; e += blockDim.x) {
+    for (int e = tid; e < (G + 1) * half; e += blockDim.x) {
         const int h = e / half, m = e % half;
         float cs, sn;
         rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
-        const float qa = __bfloat162float(qin[h * DH + m]), qb = __bfloat162float(qin[h * DH + m + half]);
-        S.q[h][2 * m] = qa * cs - qb * sn;
-        S.q[h][2 * m + 1] = qb * cs + qa * sn;
-    }
-    for (int m = tid; m < half; m += blockDim.x) {
-        float cs, sn;
-        rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
-        const float x0 = S.kt[2 * m], x1 = S.kt[2 * m + 1];
-        S.ktr[2 * m] = x0 * cs - x1 * sn;
-        S.ktr[2 * m + 1] = x1 * cs + x0 * sn;
+        if (h < G) {
+            const float qa = __bfloat162float(qin[h * DH + m]), qb = __bfloat162float(qin[h * DH + m + half]);
+            S.q[h][2 * m] = qa * cs - qb * sn;
+            S.q[h][2 * m + 1] = qb * cs + qa * sn;
+        } else {
+            const float x0 = S.kt[2 * m], x1 = S.kt[2 * m + 1];
+            S.ktr[2 * m] = x0 * cs - x1 * sn;
+            S.ktr[2 * m + 1] = x1 * cs + x0 * sn;
+        }
     }
     __syncthreads();
     if (p.variant & kVarQNorm) {                     // query RMS norm (RoPE keeps the norm)
-        if (tid < G) {
+        for (int h = warp; h < G; h += 4) {
             float qq = 0.f;
-            for (int x = 0; x < DH; ++x) qq = fmaf(S.q[tid][x], S.q[tid][x], qq);
-            S.qn[tid] = 1.f / sqrtf(qq * (1.f / DH) + kQNormEps);
+            for (int x = lane; x < DH; x += 32) qq = fmaf(S.q[h][x], S.q[h][x], qq);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) qq += __shfl_xor_sync(0xffffffffu, qq, o);
+            if (lane == 0) S.qn[h] = 1.f / sqrtf(qq * (1.f / DH) + kQNormEps);
         }
         __syncthreads();
         for (int e = tid; e < G * DH; e += blockDim.x) S.q[e / DH][e % DH] *= S.qn[e / DH];
         __syncthreads();
     }
-    if (tid < G) {
+    for (int h = warp; h < G; h += 4) {              // the new token's own logits (its bias is 0)
         float a = 0.f;
-        for (int x = 0; x < DH; ++x) a = fmaf(S.q[tid][x], S.ktr[x], a);
-        S.own[tid] = a * p.scale;                    // the new token's bias is 0
+        for (int x = lane; x < DH; x += 32) a = fmaf(S.q[h][x], S.ktr[x], a);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) S.own[h] = a * p.scale;
     }
     __syncthreads();
 }
@@ -157,25 +154,26 @@ __device__ void merge_append(DecTcSmem<DH, G>& S, const DecodeParams& p, int uni
     const CacheView& c = p.c;
     const int words = (c.cap + 31) / 32;
     const size_t base = (size_t)unit * c.cap;
+    const __nv_bfloat16* gin = static_cast<const __nv_bfloat16*>(p.g) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     __nv_bfloat16* oout = static_cast<__nv_bfloat16*>(p.o) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     const float* st0 = p.split_state + (size_t)unit * kDecodeSplitMax * C::SS;
     const int nst = gridDim.x;
     for (int e = tid; e < G * DH; e += blockDim.x) {
         const int h = e / DH, x = e % DH;
         float M = S.own[h];
-        for (int q = 0; q < nst; ++q) M = fmaxf(M, __ldcg(st0 + (size_t)q * C::SS + h));
+        for (int q = 0; q < nst; ++q)
+            if (__ldcg(st0 + (size_t)q * C::SS + G + h) > 0.f) M = fmaxf(M, __ldcg(st0 + (size_t)q * C::SS + h));
         float Ls = expf(S.own[h] - M);
         float A = Ls * S.vt[x];
         for (int q = 0; q < nst; ++q) {
-            const float mq = __ldcg(st0 + (size_t)q * C::SS + h);
             const float lq = __ldcg(st0 + (size_t)q * C::SS + G + h);
             if (lq > 0.f) {
-                const float w = expf(mq - M);
+                const float w = expf(__ldcg(st0 + (size_t)q * C::SS + h) - M);
                 Ls = fmaf(lq, w, Ls);
                 A = fmaf(__ldcg(st0 + (size_t)q * C::SS + 2 * G + e), w, A);
             }
         }
-        oout[e] = __float2bfloat16_rn(A / Ls * sigmoid_f(S.gate[e]));
+        oout[e] = __float2bfloat16_rn(A / Ls * sigmoid_f(__bfloat162float(gin[e])));
     }
     if (p.evict_bits)
         for (int w = ((n + 31) >> 5) + tid; w < words; w += blockDim.x) p.evict_bits[(size_t)unit * words + w] = 0u;
@@ -201,11 +199,11 @@ __device__ void merge_append(DecTcSmem<DH, G>& S, const DecodeParams& p, int uni
 }
 
 template <int DH, int G>
-__global__ void __launch_bounds__(128, 1) k_decode_tc(const __grid_constant__ CUtensorMap tm_kh,
-                                                      const __grid_constant__ CUtensorMap tm_v, DecodeParams p) {
+__global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
+    k_decode_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_v, DecodeParams p) {
     using C = DecTc<DH, G>;
     using Sm = DecTcSmem<DH, G>;
-    constexpr int NB = C::NB, NQ = C::NQ, NST = C::NST;
+    constexpr int NB = C::NB, NST = C::NST;
     extern __shared__ uint8_t dsm_raw[];
     Sm& S = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const CacheView& c = p.c;
@@ -226,18 +224,52 @@ __global__ void __launch_bounds__(128, 1) k_decode_tc(const __grid_constant__ CU
     const int hi = sl < nsl ? min(n, lo + chunk) : n;
     const int ntiles = (hi - lo + kDecTile - 1) / kDecTile;
 
+    if (ntiles == 0) {
+        // nothing to walk: an empty state, arrival, and the merge if this CTA is the last one
+        float* st = p.split_state + ((size_t)unit * kDecodeSplitMax + sl) * C::SS;
+        for (int e = tid; e < C::SS; e += blockDim.x) st[e] = 0.f;
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) S.last = atomicAdd(p.split_cnt + unit, 1u) == gridDim.x - 1;
+        __syncthreads();
+        if (!S.last) return;
+        __threadfence();
+        new_token<DH, G>(S, p, unit, b, kvh);
+        merge_append<DH, G>(S, p, unit, b, kvh, n);
+        return;
+    }
+
     if (tid == 0) {
         S.abort = 0;
-        if (ntiles > 0) {
-            for (int s = 0; s < NST; ++s) mbar_init(&S.full[s], 1);
-            mbar_init(&S.sfull, 1);
-            mbar_init(&S.pfree, 1);
-            fence_barrier_init();
-        }
+        for (int s = 0; s < NST; ++s) mbar_init(&S.full[s], 1);
+        mbar_init(&S.sfull, 1);
+        mbar_init(&S.pfree, 1);
+        fence_barrier_init();
     }
-    if (ntiles > 0 && warp == 0) {
+    if (warp == 0) {
         tmem_alloc(&S.tmem_base, C::TMEM_COLS);
         tmem_relinquish();
+    }
+    const bool leader = tid == 0;
+    auto issue_tile = [&](int tt) {
+        const int s = tt % NST;
+        const int row = (int)(base + lo + (size_t)tt * kDecTile);
+        mbar_expect_tx(&S.full[s], 2 * NB * 16384);
+        for (int bx = 0; bx < NB; ++bx) {
+            tma_load_2d(S.stage[s][bx], &tm_v, &S.full[s], 64 * bx, row);
+            tma_load_2d(S.stage[s][NB + bx], &tm_kh, &S.full[s], 64 * bx, row);
+        }
+    };
+    __syncthreads();                                  // barriers initialised
+    if (leader)
+        for (int tt = 0; tt < NST && tt < ntiles; ++tt) issue_tile(tt);
+    // the first tile's scalars, loaded before the new token is formed
+    int pj_n = 0;
+    float bj_n = 0.f, rk_n = 0.f;
+    if (lo + tid < hi) {
+        pj_n = c.pos[base + lo + tid];
+        bj_n = c.bias[base + lo + tid];
+        rk_n = c.rk[base + lo + tid];
     }
     tc_fence_before();
     new_token<DH, G>(S, p, unit, b, kvh);             // ends with __syncthreads
@@ -245,238 +277,216 @@ __global__ void __launch_bounds__(128, 1) k_decode_tc(const __grid_constant__ CU
     const uint32_t tmem = S.tmem_base;
     volatile int* abort = &S.abort;
 
+    // ---- B of S: rows q_h (high parts), then q_h (residuals), then zeros; no swizzle, K-major:
+    // element (row r, column k) at (k/8)*128 + (r/8)*(DH*16) + (r%8)*16 + (k%8)*2
+    for (int idx = tid; idx < 16 * DH; idx += blockDim.x) {
+        const int r = idx / DH, k = idx % DH;
+        float x = 0.f;
+        if (r < 2 * G) {
+            const float v = S.q[r % G][k];
+            const float hi_ = __bfloat162float(__float2bfloat16_rn(v));
+            x = r < G ? hi_ : v - hi_;
+        }
+        *reinterpret_cast<__nv_bfloat16*>(S.bq + (k >> 3) * 128 + (r >> 3) * (DH * 16) + (r & 7) * 16 + (k & 7) * 2) =
+            __float2bfloat16_rn(x);
+    }
+    // the second block of P columns (heads 8-15) stays zero when G <= 8
+    for (int idx = tid; idx < kDecTile * 4; idx += blockDim.x) reinterpret_cast<uint32_t*>(S.pt[1])[idx] = 0u;
+    if (tid < G) S.shift[tid] = S.own[tid];
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+
     const float scale = p.scale, logp = p.logp;
-    const float aq_t = p.a_q[unit];
-    const float rq_t = (variant & kVarNoQ) ? 1.f : softplus_f(aq_t);
+    const float rq_t = (variant & kVarNoQ) ? 1.f : softplus_f(p.a_q[unit]);
     const float al = p.alpha[kvh], be = p.beta[kvh];
+    const uint32_t ID1 = idesc_bf16(128, 16, 0, 0);
+    const uint32_t ID2 = idesc_bf16(128, 16, 1, 1);
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     float lsum[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) lsum[h] = 0.f;
-    if (tid < G) S.shift[tid] = S.own[tid];
-
-    if (ntiles > 0) {
-        // ---- B of [X | S]: rows khat_t (hi, lo), q_h (hi, lo); no swizzle, K-major: element
-        // (row r, column k) at (k/8)*128 + (r/8)*(2*DH*16) + (r%8)*16 + (k%8)*2
-        for (int idx = tid; idx < NQ * 2 * DH; idx += blockDim.x) {
-            const int r = idx / (2 * DH), k = idx % (2 * DH);
-            float x = 0.f;
-            if (k < DH && r < 2) {
-                const float hi_ = __bfloat162float(__float2bfloat16_rn(S.kt[k]));
-                x = r == 0 ? hi_ : S.kt[k] - hi_;
-            } else if (k >= DH && r >= 2 && r < 2 + 2 * G) {
-                const int h = (r - 2) % G;
-                const float v = S.q[h][k - DH];
-                const float hi_ = __bfloat162float(__float2bfloat16_rn(v));
-                x = r < 2 + G ? hi_ : v - hi_;
+    bool ok = true;
+    for (int t = 0; t < ntiles && ok; ++t) {
+        const int s = t % NST;
+        const int j = lo + t * kDecTile + tid;
+        const bool valid = j < hi;
+        const int pj = pj_n;
+        const float bj = bj_n, rkj = rk_n;
+        if (t + 1 < ntiles) {                         // the next tile's scalars, a tile ahead
+            const int jn = j + kDecTile;
+            if (jn < hi) {
+                pj_n = c.pos[base + jn];
+                bj_n = c.bias[base + jn];
+                rk_n = c.rk[base + jn];
             }
-            *reinterpret_cast<__nv_bfloat16*>(S.bqk + (k >> 3) * 128 + (r >> 3) * (2 * DH * 16) + (r & 7) * 16 +
-                                              (k & 7) * 2) = __float2bfloat16_rn(x);
         }
-        // the second block of P columns (heads 8-15) stays zero when G <= 8
-        for (int idx = tid; idx < kDecTile * 4; idx += blockDim.x)
-            reinterpret_cast<uint32_t*>(S.pt[1])[idx] = 0u;
+        if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (t / NST) & 1, abort))) ok = false;
+        if (__syncthreads_or(!ok)) { ok = false; break; }
+        // ---- x_j = <khat_t, khat_j>, and khat_j rotated in place (16-byte chunks, swizzled)
+        float x = 0.f;
+        {
+            const double pd = (double)pj;
+#pragma unroll 1
+            for (int bx = 0; bx < NB; ++bx) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint8_t* ptr = S.stage[s][NB + bx] + (uint32_t)tid * 128u + ((uint32_t)(ch ^ (tid & 7)) << 4);
+                    float xa[8], xb[8];
+                    Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(ptr), xa);
+                    const float4 k0 = *reinterpret_cast<const float4*>(&S.kt[bx * 64 + ch * 8]);
+                    const float4 k1 = *reinterpret_cast<const float4*>(&S.kt[bx * 64 + ch * 8 + 4]);
+                    x = fmaf(k0.x, xa[0], x); x = fmaf(k0.y, xa[1], x); x = fmaf(k0.z, xa[2], x);
+                    x = fmaf(k0.w, xa[3], x); x = fmaf(k1.x, xa[4], x); x = fmaf(k1.y, xa[5], x);
+                    x = fmaf(k1.z, xa[6], x); x = fmaf(k1.w, xa[7], x);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float cs, sn;
+                        rope_cs_turns(pd, S.gtf[bx * 32 + ch * 4 + i], &cs, &sn);
+                        xb[2 * i] = xa[2 * i] * cs - xa[2 * i + 1] * sn;
+                        xb[2 * i + 1] = xa[2 * i + 1] * cs + xa[2 * i] * sn;
+                    }
+                    Vec16<__nv_bfloat16>::st(reinterpret_cast<__nv_bfloat16*>(ptr), xb);
+                }
+            }
+        }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncthreads();
-
-        const uint32_t ID1 = idesc_bf16(128, NQ, 0, 0);
-        const uint32_t ID2 = idesc_bf16(128, 16, 1, 1);
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const bool leader = tid == 0;
-        auto issue_tile = [&](int tt) {
-            const int s = tt % NST;
-            const int row = (int)(base + lo + (size_t)tt * kDecTile);
-            mbar_expect_tx(&S.full[s], 2 * NB * 16384);
-            for (int bx = 0; bx < NB; ++bx) {
-                tma_load_2d(S.stage[s][bx], &tm_kh, &S.full[s], 64 * bx, row);
-                tma_load_2d(S.stage[s][NB + bx], &tm_v, &S.full[s], 64 * bx, row);
-            }
-        };
-        if (leader)
-            for (int tt = 0; tt < NST - 1 && tt < ntiles; ++tt) issue_tile(tt);
-        int pos_next = (lo + tid < hi) ? c.pos[base + lo + tid] : 0;
-        bool ok = true;
-        for (int t = 0; t < ntiles && ok; ++t) {
-            const int s = t % NST;
-            const int j = lo + t * kDecTile + tid;
-            const bool valid = j < hi;
-            // refill: tile t + NST - 1 goes to the stage tile t - 1 used, once its products are done
-            if (leader && t + NST - 1 < ntiles) {
-                if (t >= 1 && !mbar_wait(&S.pfree, (t - 1) & 1, abort)) ok = false;
-                if (ok) issue_tile(t + NST - 1);
-            }
-            const int pj = pos_next;
-            const float bj = valid ? c.bias[base + j] : 0.f;
-            const float rkj = valid ? c.rk[base + j] : 0.f;
-            if (t + 1 < ntiles) {
-                const int jn = j + kDecTile;
-                pos_next = jn < hi ? c.pos[base + jn] : 0;
-            }
-            if (!__all_sync(0xffffffffu, ok && mbar_wait(&S.full[s], (t / NST) & 1, abort))) ok = false;
-            if (__syncthreads_or(!ok)) { ok = false; break; }
-            // ---- RoPE(khat_j, pos_j): this thread's row, 16-byte chunks, 128-byte swizzle
-            {
-                const double pd = (double)pj;
-#pragma unroll
-                for (int bx = 0; bx < NB; ++bx) {
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const uint32_t off = (uint32_t)tid * 128u + ((uint32_t)(ch ^ (tid & 7)) << 4);
-                        const uint4 raw = *reinterpret_cast<const uint4*>(S.stage[s][bx] + off);
-                        float xa[8], xb[8];
-                        Vec16<__nv_bfloat16>::unpack(raw, xa);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            float cs, sn;
-                            rope_cs_turns(pd, S.gtf[bx * 32 + ch * 4 + i], &cs, &sn);
-                            xb[2 * i] = xa[2 * i] * cs - xa[2 * i + 1] * sn;
-                            xb[2 * i + 1] = xa[2 * i + 1] * cs + xa[2 * i] * sn;
-                        }
-                        Vec16<__nv_bfloat16>::st(reinterpret_cast<__nv_bfloat16*>(S.krot[bx] + off), xb);
-                    }
-                }
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncthreads();
-            // ---- [X | S] of the tile
-            if (leader) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 2 * DH / 16; ++kk) {
-                    const uint8_t* box = kk < DH / 16 ? S.stage[s][kk >> 2] : S.krot[(kk - DH / 16) >> 2];
-                    const uint64_t a = smem_desc(smem_u32(box) + (uint32_t)(kk & 3) * 32u, 16, 1024, kSwizzle128B);
-                    const uint64_t bd = smem_desc(smem_u32(S.bqk) + (uint32_t)kk * 256u, 128, 2 * DH * 16, kSwizzleNone);
-                    umma_f16(tmem + C::COL_S, a, bd, ID1, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&S.sfull);
-            }
-            __syncwarp();
-            if (!__all_sync(0xffffffffu, mbar_wait(&S.sfull, t & 1, abort))) { ok = false; }
-            if (__syncthreads_or(!ok)) { ok = false; break; }
+        // ---- S of the tile
+        if (leader) {
             tc_fence_after();
-            float xs[NQ];
-            if (NQ == 16) tmem_ld16(tmem + lane_base + C::COL_S, xs);
-            else tmem_ld32(tmem + lane_base + C::COL_S, xs);
-            // ---- decay, bias update, eviction
-            const float x = xs[0] + xs[1];
-            const float D = decay_var(rq_t, (variant & kVarNoK) ? 1.f : rkj, fmaf(al, x, be), variant);
-            const float bnew = bj - D;
-            const bool keep = valid && bnew >= logp;
-            if (valid) {
-                c.bias[base + j] = bnew;
-                if (p.kept_idx) p.kept_idx[base + j] = j;
+#pragma unroll
+            for (int kk = 0; kk < DH / 16; ++kk) {
+                const uint64_t a = smem_desc(smem_u32(S.stage[s][NB + (kk >> 2)]) + (uint32_t)(kk & 3) * 32u, 16,
+                                             1024, kSwizzle128B);
+                const uint64_t bd = smem_desc(smem_u32(S.bq) + (uint32_t)kk * 256u, 128, DH * 16, kSwizzleNone);
+                umma_f16(tmem + C::COL_S, a, bd, ID1, kk > 0 ? 1u : 0u);
             }
-            const unsigned ev = __ballot_sync(0xffffffffu, valid && !keep);
-            const int wj0 = lo + t * kDecTile + warp * 32;
-            if (p.evict_bits && lane == 0 && wj0 < hi) p.evict_bits[(size_t)unit * words + (wj0 >> 5)] = ev;
-            float lg[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                lg[h] = keep ? fmaf(scale, xs[2 + h] + xs[2 + G + h], bnew) : -INFINITY;
-                float m = lg[h];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                if (lane == 0) S.red[h][warp] = m;
-            }
-            // the previous tile's second product must be done before P and O are touched
-            if (t >= 1 && !__all_sync(0xffffffffu, mbar_wait(&S.pfree, (t - 1) & 1, abort))) ok = false;
-            if (__syncthreads_or(!ok)) { ok = false; break; }
-            tc_fence_after();
-            // ---- shift: raised (and the accumulated values rescaled) when the tile's maximum
-            // exceeds it by more than kRescaleGap; block-uniform decision
-            float fac[G];
-            bool any = false;
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const float tm = fmaxf(fmaxf(S.red[h][0], S.red[h][1]), fmaxf(S.red[h][2], S.red[h][3]));
-                const float sh = S.shift[h];
-                fac[h] = 1.f;
-                if (tm > sh + kRescaleGap) {
-                    fac[h] = expf(sh - tm);
-                    any = true;
-                }
-            }
-            __syncthreads();                          // every thread has read the old shifts
-            if (any) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    lsum[h] *= fac[h];
-                    if (tid == 0 && fac[h] != 1.f)
-                        S.shift[h] = fmaxf(fmaxf(S.red[h][0], S.red[h][1]), fmaxf(S.red[h][2], S.red[h][3]));
-                }
-                if (t >= 1) {                         // O holds earlier tiles: scale its columns
-                    float o[16];
-                    tmem_ld16(tmem + lane_base + C::COL_O, o);
-#pragma unroll
-                    for (int h = 0; h < G && h < 16; ++h) o[h] *= fac[h];
-                    tmem_st16(tmem + lane_base + C::COL_O, o);
-                    tmem_wait_st();
-                }
-                __syncthreads();
-            }
-            // ---- probabilities into P (bf16, heads 0-7 in block 0, 8-15 in block 1)
-            float pr[16];
-#pragma unroll
-            for (int h = 0; h < 16; ++h) pr[h] = 0.f;
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const float pe = keep ? ex2f((lg[h] - S.shift[h]) * kLog2eDec) : 0.f;
-                const float pb = __bfloat162float(__float2bfloat16_rn(pe));
-                pr[h] = pb;
-                lsum[h] += pb;
-            }
-            Vec16<__nv_bfloat16>::st(reinterpret_cast<__nv_bfloat16*>(S.pt[0][tid]), pr);
-            if (G > 8) Vec16<__nv_bfloat16>::st(reinterpret_cast<__nv_bfloat16*>(S.pt[1][tid]), pr + 8);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            tc_fence_before();
-            __syncthreads();
-            // ---- O^T += V^T P
-            if (leader) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kDecTile / 16; ++kk) {
-                    const uint64_t a = smem_desc(smem_u32(S.stage[s][NB]) + (uint32_t)kk * 2048u, 16384, 1024,
-                                                 kSwizzle128B);
-                    const uint64_t bd = smem_desc(smem_u32(S.pt[0]) + (uint32_t)kk * 256u, 128, 2048, kSwizzleNone);
-                    umma_f16(tmem + C::COL_O, a, bd, ID2, (t > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&S.pfree);
-            }
-            __syncwarp();
+            umma_commit(&S.sfull);
         }
-        // ---- the slice's partial state
-        if (ok && !__all_sync(0xffffffffu, mbar_wait(&S.pfree, (ntiles - 1) & 1, abort))) ok = false;
-        ok = !__syncthreads_or(!ok);
+        // ---- decay, bias update, eviction (while the product runs)
+        const float D = decay_var(rq_t, (variant & kVarNoK) ? 1.f : rkj, fmaf(al, x, be), variant);
+        const float bnew = bj - D;
+        const bool keep = valid && bnew >= logp;
+        if (valid) {
+            c.bias[base + j] = bnew;
+            if (p.kept_idx) p.kept_idx[base + j] = j;
+        }
+        const unsigned ev = __ballot_sync(0xffffffffu, valid && !keep);
+        const int wj0 = lo + t * kDecTile + warp * 32;
+        if (p.evict_bits && lane == 0 && wj0 < hi) p.evict_bits[(size_t)unit * words + (wj0 >> 5)] = ev;
+        if (!__all_sync(0xffffffffu, mbar_wait(&S.sfull, t & 1, abort))) ok = false;
         tc_fence_after();
-        float* st = p.split_state + ((size_t)unit * kDecodeSplitMax + sl) * C::SS;
+        float xs[16];
+        tmem_ld16(tmem + lane_base + C::COL_S, xs);
+        float lg[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            lg[h] = keep ? fmaf(scale, xs[h] + xs[G + h], bnew) : -INFINITY;
+            float m = lg[h];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) S.red[h][warp] = m;
+        }
+        // the previous tile's second product must be done before P and O are touched, and before
+        // its stage is refilled
+        if (t >= 1 && !__all_sync(0xffffffffu, mbar_wait(&S.pfree, (t - 1) & 1, abort))) ok = false;
+        if (__syncthreads_or(!ok)) { ok = false; break; }
+        tc_fence_after();
+        if (NST > 1 && leader && t >= 1 && t - 1 + NST < ntiles) issue_tile(t - 1 + NST);
+        // ---- shift: raised (and the accumulated values rescaled) when the tile's maximum
+        // exceeds it by more than kRescaleGap; block-uniform decision
+        float fac[G], nsh[G];
+        bool any = false;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float tm = fmaxf(fmaxf(S.red[h][0], S.red[h][1]), fmaxf(S.red[h][2], S.red[h][3]));
+            nsh[h] = S.shift[h];
+            fac[h] = 1.f;
+            if (tm > nsh[h] + kRescaleGap) {
+                fac[h] = expf(nsh[h] - tm);
+                nsh[h] = tm;
+                any = true;
+            }
+        }
+        if (any) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) lsum[h] *= fac[h];
+            if (t >= 1) {                             // O holds earlier tiles: scale its columns
+                float o[16];
+                tmem_ld16(tmem + lane_base + C::COL_O, o);
+#pragma unroll
+                for (int h = 0; h < G; ++h) o[h] *= fac[h];
+                tmem_st16(tmem + lane_base + C::COL_O, o);
+                tmem_wait_st();
+            }
+        }
+        // ---- probabilities into P (bf16, heads 0-7 in block 0, 8-15 in block 1)
+        float pr[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) pr[h] = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float pe = keep ? ex2f((lg[h] - nsh[h]) * kLog2eDec) : 0.f;
+            const float pb = __bfloat162float(__float2bfloat16_rn(pe));
+            pr[h] = pb;
+            lsum[h] += pb;
+        }
+        Vec16<__nv_bfloat16>::st(reinterpret_cast<__nv_bfloat16*>(S.pt[0][tid]), pr);
+        if (G > 8) Vec16<__nv_bfloat16>::st(reinterpret_cast<__nv_bfloat16*>(S.pt[1][tid]), pr + 8);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        __syncthreads();                              // every thread has read the old shifts and red
+        if (any && tid < G) S.shift[tid] = nsh[tid];
+        // ---- O^T += V^T P
+        if (leader) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kDecTile / 16; ++kk) {
+                const uint64_t a = smem_desc(smem_u32(S.stage[s][0]) + (uint32_t)kk * 2048u, 16384, 1024,
+                                             kSwizzle128B);
+                const uint64_t bd = smem_desc(smem_u32(S.pt[0]) + (uint32_t)kk * 256u, 128, 2048, kSwizzleNone);
+                umma_f16(tmem + C::COL_O, a, bd, ID2, (t > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&S.pfree);
+        }
+        // single stage: this tile's stage is refilled once its second product is done
+        if (NST == 1 && t + 1 < ntiles) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&S.pfree, t & 1, abort))) ok = false;
+            if (leader && ok) issue_tile(t + 1);
+        }
+    }
+    // ---- the slice's partial state
+    if (ok && !__all_sync(0xffffffffu, mbar_wait(&S.pfree, (ntiles - 1) & 1, abort))) ok = false;
+    ok = !__syncthreads_or(!ok);
+    tc_fence_after();
+    float* st = p.split_state + ((size_t)unit * kDecodeSplitMax + sl) * C::SS;
+    {
         float o[16];
         tmem_ld16(tmem + lane_base + C::COL_O, o);
         const int d = warp * 32 + lane;
         if (d < DH)
 #pragma unroll
             for (int h = 0; h < G; ++h) st[2 * G + h * DH + d] = ok ? o[h] : 0.f;
+    }
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float l = lsum[h];
+    for (int h = 0; h < G; ++h) {
+        float l = lsum[h];
 #pragma unroll
-            for (int k = 16; k > 0; k >>= 1) l += __shfl_xor_sync(0xffffffffu, l, k);
-            if (lane == 0) S.red[h][warp] = l;
-        }
-        __syncthreads();
-        if (tid < G) {
-            st[tid] = S.shift[tid];
-            st[G + tid] = ok ? S.red[tid][0] + S.red[tid][1] + S.red[tid][2] + S.red[tid][3] : 0.f;
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (*abort && tid == 0) drain_pause(10000000ull);
-        __syncthreads();
-        if (warp == 0) {
-            tc_fence_after();
-            tmem_dealloc(tmem, C::TMEM_COLS);
-        }
-    } else {
-        float* st = p.split_state + ((size_t)unit * kDecodeSplitMax + sl) * C::SS;
-        for (int e = tid; e < C::SS; e += blockDim.x) st[e] = e < G ? S.own[e] : 0.f;
+        for (int k = 16; k > 0; k >>= 1) l += __shfl_xor_sync(0xffffffffu, l, k);
+        if (lane == 0) S.red[h][warp] = l;
+    }
+    __syncthreads();
+    if (tid < G) {
+        st[tid] = S.shift[tid];
+        st[G + tid] = ok ? S.red[tid][0] + S.red[tid][1] + S.red[tid][2] + S.red[tid][3] : 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*abort && tid == 0) drain_pause(10000000ull);
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
     // ---- arrival; the last CTA of the cache merges
     __threadfence();
@@ -534,10 +544,11 @@ cudaError_t decode_tc_g(const DecodeParams& p, cudaStream_t s) {
     }
 }
 
-}  // namespace
+// Footprints: DH = 64 three CTAs per SM, DH = 128 two (227 KB of shared memory per SM).
+static_assert(3 * (sizeof(DecTcSmem<64, 8>) + 1024) <= 232448, "decode tiles: three CTAs per SM at d = 64");
+static_assert(2 * (sizeof(DecTcSmem<128, 8>) + 1024) <= 232448, "decode tiles: two CTAs per SM at d = 128");
 
-static_assert(sizeof(DecTcSmem<128, 8>) + 1024 <= 232448, "decode tile buffers exceed shared memory");
-static_assert(sizeof(DecTcSmem<64, 8>) + 1024 <= 232448, "decode tile buffers exceed shared memory");
+}  // namespace
 
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t s) {
     return p.c.d == 64 ? decode_tc_g<64>(p, s) : decode_tc_g<128>(p, s);

@@ -117,8 +117,9 @@ def test_tensor_core_split_decode_lockstep(d, H, Hkv, T0, p):
 
 
 def test_tensor_core_split_decode_large_query_norms():
-    """Queries scaled so that scale*||q|| reaches ~60: the logits spread over far more than the
+    """Queries scaled so that scale*||q|| reaches ~25: the logits spread over far more than the
     shift's 16-nat headroom, so the shift is raised (and the accumulated values rescaled in
-    TMEM) tile by tile."""
+    TMEM) tile by tile.  (The bf16 keys put an error of ~2^-9 * scale*||q|| / sqrt(d) on every
+    logit, so the bf16 bar on o holds up to scale*||q|| of a few tens; at 60 it measured 6.5e-3.)"""
     w = I.Workload("dec_tc_qn", 1, 2600, 8, 2, 64, "bf16", 6177, bimodal_ak=True)
-    run_lockstep(w, 2600, 6, 0.15, q_gain=60.0)
+    run_lockstep(w, 2600, 6, 0.15, q_gain=25.0)
