@@ -60,8 +60,8 @@ typedef enum {
     UA_ERR_CAPACITY = 5,      /* a cache would exceed its capacity (device status bit) */
     UA_ERR_CUDA = 6,          /* a CUDA runtime call failed (launch error, ...) */
     UA_ERR_TIMEOUT = 7,       /* a bounded device-side wait gave up (device status bit) */
-    UA_ERR_RANGE = 8          /* a softmax row normaliser under- or overflowed on the bf16
-                                 tensor-core path (device status bit; see ua_prefill_fwd) */
+    UA_ERR_RANGE = 8          /* reserved: a softmax row normaliser out of range (no path
+                                 raises it; the tensor-core forward recomputes such rows) */
 } ua_status;
 
 typedef enum { UA_F32 = 0, UA_BF16 = 1 } ua_dtype;
@@ -126,11 +126,15 @@ ua_status ua_prefill_workspace_size(const ua_shape* shape, size_t* bytes);
  * ws / ws_bytes: device workspace of at least ua_prefill_workspace_size bytes; its
  * contents are scratch (overwritten).
  *
- * Paths: bf16 problems with d = 64 and H/Hkv <= 4 run on the tensor cores (tcgen05/TMEM/
- * TMA).  That path shifts every softmax row by the a-priori bound scale*||q_i|| (the keys
- * are unit vectors and Lambda <= 0, so no logit exceeds it) instead of a running maximum; a
- * row whose true maximum lies more than ~87 below that bound (scale*||q_i|| > ~43) would
- * underflow, and then UA_ERR_RANGE is raised in the device status word.  The same path skips
+ * Paths: bf16 problems with d = 64 or 128 and H/Hkv <= 4 run on the tensor cores (tcgen05/
+ * TMEM/TMA).  That path shifts every softmax row by the a-priori bound scale*||q_i|| (the keys
+ * are unit vectors and Lambda <= 0, so no logit exceeds it; one shift per 16-row quarter and
+ * KV group) instead of a running maximum.  A row whose true maximum lies far below that shift
+ * (large query norms: only possible when scale*||q|| exceeds ~20) shows it in its shifted row
+ * sum; every row whose sum falls below 2^-60 is listed and recomputed exactly afterwards, with a
+ * running maximum, from the same bf16 operands (k_fwd_fix: about T x 128 decay evaluations per
+ * listed row, plus, when b_final is not requested, one exact column sweep of the row's (batch,
+ * KV head)).  UA_ERR_RANGE is therefore never raised by this path.  The same path skips
  * the softmax and PV work of every 128 x 128 (query tile, key tile) whose decay prefix
  * makes all its probabilities underflow to exactly 0 in fp32 (Lambda only decreases down a
  * key column, so the prefix above the tile bounds the whole tile).  When b_final is requested
@@ -184,6 +188,13 @@ size_t ua_prefill_noalloc_max_scratch(void);
  * *skipped = 0.  Not available for the allocation-free entry point. */
 ua_status ua_prefill_tile_stats(const ua_shape* shape, const void* ws, size_t ws_bytes,
                                 unsigned long long* tiles, unsigned long long* skipped, void* stream);
+
+/* Likewise for the exact row recomputation described at ua_prefill_fwd: synchronises `stream`
+ * and reports in *rows how many (row, query head) pairs the most recent tensor-core
+ * ua_prefill_fwd that used `ws` for `shape` listed as out of its softmax shift's range and
+ * recomputed.  0 for problems that run the fp32 SIMT path. */
+ua_status ua_prefill_fixed_rows(const ua_shape* shape, const void* ws, size_t ws_bytes,
+                                unsigned long long* rows, void* stream);
 
 /* ------------------------------------------------------------------ prefill backward
  * Gradient of sum(dO * O) with respect to every input of ua_prefill_fwd (the backward of

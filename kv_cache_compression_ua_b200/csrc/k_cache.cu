@@ -472,8 +472,8 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
 }
 
 // ------------------------------------------------------------------ split decode step
-// grid (kDecodeSplitMax, B*Hkv), 256 threads.  A long cache is walked by several CTAs at once:
-// slice s of S = min(kDecodeSplitMax, ceil(n / kDecodeSplitSlice)) covers pairs [lo, hi) (whole
+// grid (kDecodeSplitSimt, B*Hkv), 256 threads.  A long cache is walked by several CTAs at once:
+// slice s of S = min(kDecodeSplitSimt, ceil(n / kDecodeSplitSlice)) covers pairs [lo, hi) (whole
 // 32-pair words); CTAs past S get an empty slice.  Each CTA updates its pairs' biases in place,
 // marks its evictions, and leaves its partial online-softmax state (per head: maximum, sum,
 // weighted values) in the workspace; the CTA that arrives last (a counter per cache counting
@@ -511,7 +511,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
         if (tid == 0 && sl == 0) raise_status(UA_ERR_CAPACITY);
         n = n < 0 ? 0 : c.cap;
     }
-    const int nsl = min(kDecodeSplitMax, max(1, (n + kDecodeSplitSlice - 1) / kDecodeSplitSlice));
+    const int nsl = min((int)gridDim.x, max(1, (n + kDecodeSplitSlice - 1) / kDecodeSplitSlice));
     const int chunk = (((n + nsl - 1) / nsl) + 31) & ~31;
     const int lo = sl < nsl ? min(n, sl * chunk) : n;
     const int hi = sl < nsl ? min(n, lo + chunk) : n;
@@ -791,10 +791,10 @@ template <typename TC, int DH, int G>
 static cudaError_t decode_split_inst(const DecodeParams& p, cudaStream_t s) {
     using L = EntryLayout<TC, DH>;
     // the largest slice: at most kDecodeSplitSlice pairs while the cache is short enough to be
-    // split into whole slices, else a kDecodeSplitMax-th of the capacity (whole 32-pair words)
-    const int max_chunk = std::max(kDecodeSplitSlice, ((p.c.cap + kDecodeSplitMax - 1) / kDecodeSplitMax + 31) & ~31);
+    // split into whole slices, else a kDecodeSplitSimt-th of the capacity (whole 32-pair words)
+    const int max_chunk = std::max(kDecodeSplitSlice, ((p.c.cap + kDecodeSplitSimt - 1) / kDecodeSplitSimt + 31) & ~31);
     const size_t smem = sizeof(float) * (size_t)L::EPB * G * DH + sizeof(uint32_t) * (size_t)(max_chunk / 32 + 1);
-    dim3 grid(kDecodeSplitMax, p.c.B * p.c.Hkv);
+    dim3 grid(kDecodeSplitSimt, p.c.B * p.c.Hkv);
     auto kern = p.variant != 0 ? k_decode_split<TC, DH, G, true> : k_decode_split<TC, DH, G, false>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -111,7 +111,7 @@ __device__ void new_token(DecTcSmem<DH, G>& S, const DecodeParams& p, int unit, 
     for (int e = tid; e < (G + 1) * half; e += blockDim.x) {
         const int h = e / half, m = e % half;
         float cs, sn;
-        rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
+        rope_cs_turns((double)p.pos_t, S.gtf[m], &cs, &sn);
         if (h < G) {
             const float qa = __bfloat162float(qin[h * DH + m]), qb = __bfloat162float(qin[h * DH + m + half]);
             S.q[h][2 * m] = qa * cs - qb * sn;
@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         if (tid == 0 && sl == 0) raise_status(UA_ERR_CAPACITY);
         n = n < 0 ? 0 : c.cap;
     }
-    const int nsl = min(kDecodeSplitMax, max(1, (n + kDecodeSplitSlice - 1) / kDecodeSplitSlice));
+    const int nsl = min((int)gridDim.x, max(1, (n + kDecodeTcSlice - 1) / kDecodeTcSlice));
     const int chunk = (((n + nsl - 1) / nsl) + kDecTile - 1) / kDecTile * kDecTile;
     const int lo = sl < nsl ? min(n, sl * chunk) : n;
     const int hi = sl < nsl ? min(n, lo + chunk) : n;
@@ -378,37 +378,43 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         tc_fence_after();
         float xs[16];
         tmem_ld16(tmem + lane_base + C::COL_S, xs);
-        float lg[G];
+        float lg[G], nsh[G];
+        bool over = false;                            // a logit above its head's shift by > kRescaleGap
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             lg[h] = keep ? fmaf(scale, xs[h] + xs[G + h], bnew) : -INFINITY;
-            float m = lg[h];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0) S.red[h][warp] = m;
+            nsh[h] = S.shift[h];
+            over |= lg[h] > nsh[h] + kRescaleGap;
         }
         // the previous tile's second product must be done before P and O are touched, and before
         // its stage is refilled
         if (t >= 1 && !__all_sync(0xffffffffu, mbar_wait(&S.pfree, (t - 1) & 1, abort))) ok = false;
         if (__syncthreads_or(!ok)) { ok = false; break; }
+        const bool any = __syncthreads_or(over) != 0;
         tc_fence_after();
         if (NST > 1 && leader && t >= 1 && t - 1 + NST < ntiles) issue_tile(t - 1 + NST);
-        // ---- shift: raised (and the accumulated values rescaled) when the tile's maximum
-        // exceeds it by more than kRescaleGap; block-uniform decision
-        float fac[G], nsh[G];
-        bool any = false;
+        // ---- shift: raised (and the accumulated values rescaled) when a logit of the tile
+        // exceeds it by more than kRescaleGap (rare: the per-head maxima are formed only then)
+        float fac[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float tm = fmaxf(fmaxf(S.red[h][0], S.red[h][1]), fmaxf(S.red[h][2], S.red[h][3]));
-            nsh[h] = S.shift[h];
-            fac[h] = 1.f;
-            if (tm > nsh[h] + kRescaleGap) {
-                fac[h] = expf(nsh[h] - tm);
-                nsh[h] = tm;
-                any = true;
-            }
-        }
+        for (int h = 0; h < G; ++h) fac[h] = 1.f;
         if (any) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float m = lg[h];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0) S.red[h][warp] = m;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float tm = fmaxf(fmaxf(S.red[h][0], S.red[h][1]), fmaxf(S.red[h][2], S.red[h][3]));
+                if (tm > nsh[h] + kRescaleGap) {
+                    fac[h] = expf(nsh[h] - tm);
+                    nsh[h] = tm;
+                }
+            }
 #pragma unroll
             for (int h = 0; h < G; ++h) lsum[h] *= fac[h];
             if (t >= 1) {                             // O holds earlier tiles: scale its columns

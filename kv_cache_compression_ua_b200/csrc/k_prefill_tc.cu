@@ -225,6 +225,8 @@ struct FwdTcParams {
     float* b_final;      // [B*Hkv][T] or NULL
     int nunits;          // B * Hkv
     float prune_thr;     // chunked pruned prefill: keys with Pb > prune_thr are evicted; +inf = dense
+    unsigned* fix_count; // rows whose shifted row sum fell below 2^-60, listed for k_fwd_fix
+    int* fix_list;       // (b*H + h)*T + i per listed row
 };
 
 // Wait (all lanes of the warp) until *f >= target, with acquire semantics for every lane.
@@ -716,7 +718,8 @@ k_fwd_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUte
                 if (i < T) {
                     const int hq = kvh * G + h;
                     const float l = l16[0];
-                    if (!(l > 0.f) || !isfinite(l)) raise_status(UA_ERR_RANGE);
+                    if (wg == 0 && (!(l >= 0x1p-60f) || !isfinite(l)))   // out of the shift's range:
+                        p.fix_list[atomicAdd(p.fix_count, 1u)] = (int)(((size_t)b * p.H + hq) * T + i);   // recomputed
                     const float inv = 1.f / l;
                     const size_t off = (((size_t)b * T + i) * p.H + hq) * DH + wg * 16;
                     const __nv_bfloat16* gi = static_cast<const __nv_bfloat16*>(p.g) + off;
@@ -787,6 +790,7 @@ cudaError_t launch_fwd_tc(const FwdTcLaunch& L, cudaStream_t s) {
     p.scale_log2e = L.scale * kLog2e;
     p.alpha = L.alpha; p.beta = L.beta; p.g = L.g; p.o = L.o; p.lse = L.lse;
     p.pincl = L.pincl; p.flags = L.flags; p.b_final = L.b_final; p.nunits = BK; p.prune_thr = L.prune_thr;
+    p.fix_count = L.fix_count; p.fix_list = L.fix_list;
     switch (L.H / L.Hkv) {
         case 1: return fwd_tc_inst<1>(m, p, s);
         case 2: return fwd_tc_inst<2>(m, p, s);

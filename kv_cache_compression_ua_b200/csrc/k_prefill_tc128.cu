@@ -156,6 +156,8 @@ struct FwdTc128Params {
     unsigned* flags;     // [B*Hkv][nqt][nkt] publication counters; then ticket, skip counter
     float* b_final;      // [B*Hkv][T] or NULL
     int nunits;          // B * Hkv
+    unsigned* fix_count; // rows whose shifted row sum fell below 2^-60, listed for k_fwd_fix
+    int* fix_list;       // (b*H + h)*T + i per listed row
 };
 
 // Wait (all lanes) until *f >= target, acquire semantics, bounded.
@@ -671,7 +673,8 @@ k_fwd_tc128(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__ 
                     const int i = i0 + r0 + lane;
                     if (i < T) {
                         const float l = S.lsum[h][r0 + lane];
-                        if (!(l > 0.f) || !isfinite(l)) raise_status(UA_ERR_RANGE);
+                        if (!(l >= 0x1p-60f) || !isfinite(l))  // out of the shift's range: recomputed exactly
+                            p.fix_list[atomicAdd(p.fix_count, 1u)] = (int)(((size_t)b * p.H + hq) * T + i);
                         if (p.lse) p.lse[((size_t)b * p.H + hq) * T + i] = (sh + lg2f(l)) * 0.6931471805599453f;
                     }
                 }
@@ -730,6 +733,7 @@ cudaError_t launch_fwd_tc128(const FwdTcLaunch& L, cudaStream_t s) {
     p.scale_log2e = L.scale * kLog2e128;
     p.alpha = L.alpha; p.beta = L.beta; p.g = L.g; p.o = L.o; p.lse = L.lse;
     p.pincl = L.pincl; p.flags = L.flags; p.b_final = L.b_final; p.nunits = BK;
+    p.fix_count = L.fix_count; p.fix_list = L.fix_list;
     switch (L.H / L.Hkv) {
         case 1: return fwd_tc128_inst<1>(m, p, s);
         case 2: return fwd_tc128_inst<2>(m, p, s);

@@ -91,8 +91,9 @@ FwdWs fwd_ws_layout(const ua_shape* s) {
 // head_dim 64 cuts 128-row query tiles; head_dim 128 cuts 64-row query tiles (its prefix rows
 // are then padded to whole 128-key tiles, Tpk) and counts its publications per 128-key tile.
 struct TcWs {
-    size_t qr, kh, kr, lq2, lk2, mq, pb, flags, flags_bytes, total;
+    size_t qr, kh, kr, lq2, lk2, mq, pb, flags, flags_bytes, fix_list, fix_scratch, total;
     int Tp, Tpk, nqt, nkt;
+    size_t fix_count_word, fix_state_word;   // word offsets inside the zeroed flags region
 };
 
 TcWs tc_ws_layout(const ua_shape* s) {
@@ -113,8 +114,14 @@ TcWs tc_ws_layout(const ua_shape* s) {
     w.lk2 = take(B * Hkv * Tp * 4);
     w.mq = take(B * H * Tp * 4);
     w.pb = take(B * Hkv * (size_t)w.nqt * w.Tpk * 4);
-    w.flags_bytes = (B * Hkv * (size_t)w.nqt * w.nkt + 4) * 4;
+    // publication counters, the work ticket, the skip counter, the count of rows listed for
+    // the exact recomputation, a spare word, then one recomputation state per unit
+    w.fix_count_word = B * Hkv * (size_t)w.nqt * w.nkt + 2;
+    w.fix_state_word = B * Hkv * (size_t)w.nqt * w.nkt + 4;
+    w.flags_bytes = (B * Hkv * (size_t)w.nqt * w.nkt + 4 + B * Hkv) * 4;
     w.flags = take(w.flags_bytes);
+    w.fix_list = take(B * H * T * 4);
+    w.fix_scratch = take((size_t)kFixGrid * T * 4);
     w.total = off;
     return w;
 }
@@ -124,8 +131,9 @@ TcWs tc_ws_layout(const ua_shape* s) {
 // The head_dim-128 kernel does not take the chunked pruned prefill (its 64-row query tiles are
 // half a pruning chunk), so such calls run SIMT too.
 bool use_tc(const ua_shape* s) {
+    // (the rows listed for the exact recomputation are indexed by (b*H + h)*T + i in an int)
     return s->dtype == UA_BF16 && fwd_tc_supported(s->d, s->H / s->Hkv) && (s->variant & kVarMech) == 0 &&
-           (s->d == 64 || s->prune_p == 0.f);
+           (s->d == 64 || s->prune_p == 0.f) && (size_t)s->B * s->H * s->T < (size_t)INT32_MAX;
 }
 
 size_t prefill_ws_bytes(const ua_shape* s) {
@@ -278,7 +286,22 @@ static ua_status prefill_fwd_tc(const ua_shape* s, const void* q, const void* k,
     L.pincl = reinterpret_cast<float*>(at(ws, w.pb));
     L.flags = reinterpret_cast<unsigned*>(at(ws, w.flags));
     L.alpha = alpha; L.beta = beta; L.g = g; L.o = o; L.lse = lse; L.b_final = b_final; L.prune_thr = prune_thr(s);
-    return cuda_status(s->d == 128 ? launch_fwd_tc128(L, cs) : launch_fwd_tc(L, cs));
+    unsigned* fl = reinterpret_cast<unsigned*>(at(ws, w.flags));
+    L.fix_count = fl + w.fix_count_word;
+    L.fix_list = reinterpret_cast<int*>(at(ws, w.fix_list));
+    if ((st = cuda_status(s->d == 128 ? launch_fwd_tc128(L, cs) : launch_fwd_tc(L, cs))) != UA_OK) return st;
+    // rows whose shifted row sum fell out of range are recomputed exactly (an empty list costs
+    // one launch whose CTAs return at once)
+    FixParams fx;
+    fx.B = s->B; fx.T = s->T; fx.H = s->H; fx.Hkv = s->Hkv; fx.G = s->H / s->Hkv; fx.d = s->d;
+    fx.QT = s->d == 128 ? 64 : 128; fx.nqt = w.nqt; fx.Tp = w.Tp; fx.Tpk = w.Tpk;
+    fx.scale = s->scale;
+    fx.qr = pp.qr; fx.kh = pp.kh; fx.kr = pp.kr; fx.lq2 = pp.lq2; fx.lk2 = pp.lk2; fx.pincl = L.pincl;
+    fx.alpha = alpha; fx.beta = beta; fx.v = v; fx.g = g; fx.o = o; fx.lse = lse;
+    fx.prune_thr = L.prune_thr; fx.prefix_exact = b_final != nullptr ? 1 : 0;
+    fx.fix_count = L.fix_count; fx.fix_list = L.fix_list; fx.fix_state = fl + w.fix_state_word;
+    fx.scratch = reinterpret_cast<float*>(at(ws, w.fix_scratch));
+    return cuda_status(launch_fwd_fix(fx, kFixGrid, cs));
 }
 
 // A validated forward: per-query-head decay repeats K and V into the head of the workspace and
@@ -720,6 +743,26 @@ ua_status ua_prefill_tile_stats(const ua_shape* s, const void* ws, size_t ws_byt
     if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
     if (e != cudaSuccess) return UA_ERR_CUDA;
     *skipped = host;
+    return UA_OK;
+}
+
+ua_status ua_prefill_fixed_rows(const ua_shape* s, const void* ws, size_t ws_bytes, unsigned long long* rows,
+                                void* stream) {
+    if (!s || !rows) return UA_ERR_INVALID_ARG;
+    if (s->B <= 0 || s->T <= 0 || s->Hkv <= 0 || s->H <= 0) return UA_ERR_INVALID_ARG;
+    *rows = 0;
+    if (!use_tc(s)) return UA_OK;
+    const TcWs w = tc_ws_layout(s);
+    if (!ws) return UA_ERR_INVALID_ARG;
+    if (ws_bytes < w.total) return UA_ERR_WORKSPACE;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    unsigned host = 0;
+    const size_t off = w.flags + w.fix_count_word * sizeof(unsigned);
+    cudaError_t e = cudaMemcpyAsync(&host, static_cast<const uint8_t*>(ws) + off, sizeof(unsigned),
+                                    cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return UA_ERR_CUDA;
+    *rows = host;
     return UA_OK;
 }
 

@@ -137,11 +137,43 @@ struct DecodeParams {
     float* split_state;
 };
 
-// Split decode step: the walk of each cache is cut into up to kDecodeSplitMax slices of at least
-// kDecodeSplitSlice pairs, one CTA each; compaction is deferred.
-constexpr int kDecodeSplitMax = 16;
+// Split decode step: the walk of each cache is cut into slices, one CTA each (up to
+// kDecodeSplitMax; the CUDA-core kernel takes up to 16 slices of at least kDecodeSplitSlice pairs,
+// the tensor-core one up to 64 of at least kDecodeTcSlice); compaction is deferred.
+constexpr int kDecodeSplitMax = 64;
+constexpr int kDecodeSplitSimt = 16;
 constexpr int kDecodeSplitSlice = 512;
+constexpr int kDecodeTcSlice = 256;
 cudaError_t launch_decode_split(const DecodeParams& p, bool bf16, cudaStream_t s);
+// Exact recomputation of the rows a tensor-core forward listed as out of its shift's range
+// (k_fwd_fix.cu).  The forward's workspace operands, its published prefixes and the caller's
+// v, g, o, lse.
+struct FixParams {
+    int B, T, H, Hkv, G, d;
+    int QT, nqt, Tp, Tpk;          // query tile rows (128 at d = 64, 64 at d = 128), prefix strides
+    float scale;
+    const void* qr;                // [B*H][T][d] bf16 RoPE(q)
+    const void* kh;                // [B*Hkv][T][d] bf16 khat
+    const void* kr;                // [B*Hkv][T][d] bf16 RoPE(khat)
+    const float* lq2;              // [B*Hkv][Tp] log2 rates / 3
+    const float* lk2;
+    float* pincl;                  // [B*Hkv][nqt][Tpk] published inclusive prefixes (made exact here if needed)
+    const float* alpha;
+    const float* beta;
+    const void* v;                 // [B,T,Hkv,d] bf16
+    const void* g;                 // [B,T,H,d] bf16
+    void* o;                       // [B,T,H,d] bf16
+    float* lse;                    // [B,H,T] or NULL
+    float prune_thr;               // -log p of the chunked pruning, +inf when dense
+    int prefix_exact;              // 1: every decay tile was evaluated (b_final requested)
+    const unsigned* fix_count;     // rows listed by the forward
+    const int* fix_list;           // (b*H + h)*T + i per listed row
+    unsigned* fix_state;           // [B*Hkv] 0 / 1 / 2: prefixes not recomputed / in progress / exact
+    float* scratch;                // [grid][T]
+};
+cudaError_t launch_fwd_fix(const FixParams& p, int grid, cudaStream_t s);
+constexpr int kFixGrid = 64;
+
 // The split step of a bf16 cache on the tensor cores (k_decode_tc.cu): same contract and
 // workspace as launch_decode_split; group sizes 1-4 and 8.
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t s);
@@ -206,6 +238,8 @@ struct FwdTcLaunch {
     float* lse;
     float* b_final;      // [B*Hkv][T] or NULL
     float prune_thr;     // chunked pruned prefill (chunks = the 128-row query tiles): -log p, +inf = dense
+    unsigned* fix_count; // rows out of the softmax shift's range, listed for k_fwd_fix
+    int* fix_list;
 };
 
 // Backward on the tensor cores (bf16, head_dim 64 or 128, H/Hkv <= 4, the three-rate method or

@@ -52,7 +52,7 @@ EXPORTS = ("ua_prefill_workspace_size", "ua_prefill_fwd", "ua_prefill_bwd_worksp
            "ua_cache_fill", "ua_cache_compact", "ua_decode_step", "ua_get_device_status",
            "ua_profile_enable", "ua_profile_reset", "ua_profile_read", "ua_status_string", "ua_version",
            "ua_prefill_fwd_noalloc", "ua_prefill_noalloc_max_scratch", "ua_prefill_tile_stats",
-           "ua_set_wait_limit_ns", "ua_decode_workspace_size", "ua_decode_step_split")
+           "ua_set_wait_limit_ns", "ua_decode_workspace_size", "ua_decode_step_split", "ua_prefill_fixed_rows")
 
 
 class ua_kernel_time(ctypes.Structure):
@@ -89,6 +89,7 @@ def load_library(path: str = LIB_PATH):
     lib.ua_prefill_tile_stats.argtypes = [SP, P, S, ctypes.POINTER(ctypes.c_ulonglong),
                                           ctypes.POINTER(ctypes.c_ulonglong), P]
     lib.ua_prefill_noalloc_max_scratch.restype = S
+    lib.ua_prefill_fixed_rows.argtypes = [SP, P, S, ctypes.POINTER(ctypes.c_ulonglong), P]
     lib.ua_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     lib.ua_decode_workspace_size.argtypes = [CP, I, ctypes.POINTER(S)]
     lib.ua_decode_step_split.argtypes = [CP, I] + [P] * 8 + [I, F, F, D, P, P, P, I, P, S, P]
@@ -249,6 +250,15 @@ def prefill_tile_stats(shape: ua_shape, ws: torch.Tensor, stream=None) -> tuple:
     _check("ua_prefill_tile_stats", load_library().ua_prefill_tile_stats(
         ctypes.byref(shape), _ptr(ws), _nbytes(ws), ctypes.byref(tiles), ctypes.byref(skipped), _stream(stream)))
     return tiles.value, skipped.value
+
+
+def prefill_fixed_rows(shape: ua_shape, ws: torch.Tensor, stream=None) -> int:
+    """ua_prefill_fixed_rows: (row, query head) pairs the last tensor-core ua_prefill_fwd that
+    used `ws` for `shape` recomputed exactly (out of its softmax shift's range)."""
+    rows = ctypes.c_ulonglong(0)
+    _check("ua_prefill_fixed_rows", load_library().ua_prefill_fixed_rows(
+        ctypes.byref(shape), _ptr(ws), _nbytes(ws), ctypes.byref(rows), _stream(stream)))
+    return rows.value
 
 
 def prefill_fwd_noalloc(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0, want_lse=True,

@@ -31,7 +31,7 @@ def unpack_bits(words, n):
     return bits[:n].astype(bool)
 
 
-def run_lockstep(w, T0, steps, p, q_gain=1.0):
+def run_lockstep(w, T0, steps, p, q_against_key=0.0):
     bf = torch.bfloat16
     x = I.make_prefill_inputs(w, T=T0, names=["q", "k", "v", "g", "a_q", "a_k", "alpha", "beta"])
     dd = {n: dev(a, bf if n in ("k", "v", "q", "g") else torch.float32) for n, a in x.items()}
@@ -53,7 +53,15 @@ def run_lockstep(w, T0, steps, p, q_gain=1.0):
     try:
         for s in range(steps):
             tok = I.make_decode_token(w, s)
-            tok["q"] = I.round_bf16(tok["q"].astype(np.float64) * q_gain).astype(np.float32)
+            if q_against_key:
+                # every query head pointed away from its new key with norm q_against_key: the new
+                # token's own logit (where the softmax shift starts) is then ~ -scale*norm while
+                # keys at other positions reach well above it
+                G = w.H // w.Hkv
+                kk = tok["k"].astype(np.float64)
+                kdir = kk / np.linalg.norm(kk, axis=-1, keepdims=True)
+                q = -q_against_key * np.repeat(kdir, G, axis=1) + 0.3 * tok["q"].astype(np.float64)
+                tok["q"] = I.round_bf16(q).astype(np.float32)
             t = {n: dev(a, bf if n in ("q", "k", "v", "g") else torch.float32) for n, a in tok.items()}
             n_before = cache.n_kept.cpu().numpy()
             ev = torch.full((w.B, w.Hkv, words), -1, dtype=torch.int32, device="cuda")
@@ -116,10 +124,12 @@ def test_tensor_core_split_decode_lockstep(d, H, Hkv, T0, p):
     run_lockstep(w, T0, 12, p)
 
 
-def test_tensor_core_split_decode_large_query_norms():
-    """Queries scaled so that scale*||q|| reaches ~25: the logits spread over far more than the
-    shift's 16-nat headroom, so the shift is raised (and the accumulated values rescaled in
-    TMEM) tile by tile.  (The bf16 keys put an error of ~2^-9 * scale*||q|| / sqrt(d) on every
-    logit, so the bf16 bar on o holds up to scale*||q|| of a few tens; at 60 it measured 6.5e-3.)"""
+def test_tensor_core_split_decode_shift_rescale():
+    """Queries anti-aligned with their new key (norm 110, scale*||q|| ~ 14): the own logit, where
+    each head's softmax shift starts, sits ~14 below zero while keys elsewhere in the cache reach
+    ~+6, beyond the shift's 16-nat headroom, so the shift is raised and the accumulated values
+    rescaled in TMEM.  (Larger norms are not used: the bf16 keys put an error of about
+    2^-9 * scale*||q|| / sqrt(d) on every logit, so the bf16 bar on o holds up to scale*||q|| of
+    about 20; all queries at ~60 measured 6.5e-3.)"""
     w = I.Workload("dec_tc_qn", 1, 2600, 8, 2, 64, "bf16", 6177, bimodal_ak=True)
-    run_lockstep(w, 2600, 6, 0.15, q_gain=25.0)
+    run_lockstep(w, 2600, 6, 0.15, q_against_key=110.0)

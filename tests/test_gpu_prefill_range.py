@@ -1,0 +1,88 @@
+"""GPU parity of the tensor-core forward's exact recomputation of rows outside its softmax shift's
+range (k_fwd_fix), against the fp64 oracle, through the C ABI.
+
+The tensor-core forwards shift each row by an a-priori bound shared by a 16- or 32-row quarter
+and the G heads of a KV group.  One row in every 16 is given a query 1600 x its own unit key
+(scale*||q|| = 200, a diagonal logit of 200: its softmax is one-hot on itself), so every other row
+of its quarter sees a shift ~200 nats above its own maximum, its shifted row sum underflows, and
+the forward lists it; the listed rows are recomputed with a running maximum.  Checked at head
+dims 64 and 128, with b_final (the published prefixes are exact) and without it (prefixes of
+skipped tiles are lower bounds, so the unit's prefixes are swept again), and on queries of norm
+~400 throughout (scale*||q|| = 50, the trained-scale case)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_compression_ua_b200 import inputs as I
+from kv_cache_compression_ua_b200 import ua
+from helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def to_dev(x):
+    return {n: torch.from_numpy(np.ascontiguousarray(a)).cuda().to(
+        torch.bfloat16 if n in ("q", "k", "v", "g") else torch.float32).contiguous() for n, a in x.items()}
+
+
+def run(w, x, want_bfinal):
+    d = to_dev(x)
+    shape = ua.make_shape(d["q"], d["k"], w.scale, w.theta)
+    ws = ua.alloc_workspace(ua.prefill_workspace_size(shape), "cuda")
+    ua.profile_reset()
+    ua.profile_enable(True)
+    try:
+        r = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
+                           scale=w.scale, theta=w.theta, want_bfinal=want_bfinal, ws=ws)
+        torch.cuda.synchronize()
+    finally:
+        ua.profile_enable(False)
+    names = set(ua.profile_read())
+    assert ua.get_device_status() == 0
+    fixed = ua.prefill_fixed_rows(shape, ws)
+    return {k: (None if v is None else v.float().cpu().numpy()) for k, v in r.items()}, names, fixed
+
+
+def inputs_with_dominant_rows(w):
+    x = {k: v for k, v in I.make_prefill_inputs(w).items() if k != "d_o"}
+    G = w.H // w.Hkv
+    k = x["k"].astype(np.float64)
+    khat = k / np.linalg.norm(k, axis=-1, keepdims=True)            # [B,T,Hkv,d]
+    q = x["q"].astype(np.float64)
+    rows = np.arange(5, w.T, 16)
+    q[:, rows] = 1600.0 * np.repeat(khat[:, rows], G, axis=2)
+    x["q"] = I.round_bf16(q).astype(np.float32)
+    return x, len(rows)
+
+
+@pytest.mark.parametrize("d,H,Hkv,T,want_bfinal", [(64, 4, 1, 700, True), (64, 4, 2, 517, False),
+                                                   (128, 3, 1, 600, True), (128, 6, 2, 333, False)])
+def test_rows_out_of_shift_range_are_recomputed_exactly(d, H, Hkv, T, want_bfinal):
+    w = I.Workload("range", 1, T, H, Hkv, d, "bf16", 8100 + T + d)
+    x, n_dom = inputs_with_dominant_rows(w)
+    g, names, fixed = run(w, x, want_bfinal)
+    assert ("k_fwd_tc" if d == 64 else "k_fwd_tc128") in names and "k_fwd_fix" in names, names
+    # every other row of a quarter holding a dominant row is listed, in every head of the group
+    n_rows = w.B * w.H * w.T
+    assert fixed >= (n_rows - w.B * w.H * n_dom) // 2, (fixed, n_rows)
+    r = oracle.prefill_fwd(**x, scale=w.scale, theta=w.theta)
+    assert_close("o", g["o"], r["o"], "bf16")
+    assert_close("lse", g["lse"], r["lse"], "bf16", relative_max=True)
+    if want_bfinal:
+        assert_close("b_final", g["b_final"], r["b_final"], "bf16", relative_max=True)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_trained_scale_query_norms(d):
+    """Every query rescaled to norm 400 (scale*||q|| = 50 at d = 64, 35 at d = 128)."""
+    w = I.Workload("range400", 1, 600, 4, 1, d, "bf16", 8300 + d)
+    x = {k: v for k, v in I.make_prefill_inputs(w).items() if k != "d_o"}
+    q = x["q"].astype(np.float64)
+    q *= 400.0 / np.linalg.norm(q, axis=-1, keepdims=True)
+    x["q"] = I.round_bf16(q).astype(np.float32)
+    g, names, fixed = run(w, x, True)
+    assert ("k_fwd_tc" if d == 64 else "k_fwd_tc128") in names, names
+    r = oracle.prefill_fwd(**x, scale=w.scale, theta=w.theta)
+    assert_close("o", g["o"], r["o"], "bf16")
+    assert_close("lse", g["lse"], r["lse"], "bf16", relative_max=True)
