@@ -240,6 +240,11 @@ ua_status ua_prefill_bwd(const ua_shape* shape, const void* q, const void* k, co
 typedef struct {
     int B, Hkv, d, capacity;
     ua_dtype dtype;
+    int kv_rep;           /* cache heads per KV head of the keys and values the cache is filled and
+                             stepped with: k, v of ua_cache_fill and the decode steps have Hkv / kv_rep
+                             heads, cache head h reading head h / kv_rep.  0 or 1: one each.  With
+                             per-query-head decay (UA_VAR_PER_HEAD_DECAY) the cache keeps one head per
+                             query head (Hkv = H, kv_rep = G), each with its own biases and evictions */
     void* khat;
     void* v;
     float* bias;
@@ -250,7 +255,7 @@ typedef struct {
 
 /* Load a prefill into the cache: slot t <- token t for t < T (khat, v from k and v; bias =
  * b_final; rk = softplus(a_k); pos = t) and n_kept = T.  Requires T <= capacity.
- * k, v: [B,T,Hkv,d] act; a_k [B,T,Hkv] f32; b_final [B,Hkv,T] f32. */
+ * k, v: [B,T,Hkv/kv_rep,d] act; a_k [B,T,Hkv] f32; b_final [B,Hkv,T] f32. */
 ua_status ua_cache_fill(const ua_cache* cache, int T, const void* k, const void* v,
                         const float* a_k, const float* b_final, double rope_theta, void* stream);
 

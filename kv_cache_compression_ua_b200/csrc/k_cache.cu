@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(256) k_cache_fill(FillParams p) {
     const TC* kin = static_cast<const TC*>(p.k);
     const TC* vin = static_cast<const TC*>(p.v);
     for (int h = warp; h < c.Hkv; h += 8) {
-        const size_t src = (((size_t)b * T + t) * c.Hkv + h) * DH;
+        const size_t src = (((size_t)b * T + t) * (c.Hkv / c.rep) + h / c.rep) * DH;
         const size_t slot = ((size_t)b * c.Hkv + h) * c.cap + t;
         float x0[2] = {0.f, 0.f}, x1[2] = {0.f, 0.f};
         float ss = 0.f;
@@ -211,8 +211,10 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     // memory round trips before its arithmetic.  (Prefetching the first pass of cache entries
     // as well was measured slower: the registers it holds cost occupancy.)
     int n = c.n_kept[unit];
-    const TC* kin = static_cast<const TC*>(p.k) + (size_t)unit * DH;
-    const TC* vin = static_cast<const TC*>(p.v) + (size_t)unit * DH;
+    // the step's key and value: head kvh / rep of [B, Hkv / rep, d]
+    const size_t tok = (size_t)b * (c.Hkv / c.rep) + kvh / c.rep;
+    const TC* kin = static_cast<const TC*>(p.k) + tok * DH;
+    const TC* vin = static_cast<const TC*>(p.v) + tok * DH;
     const TC* qin = static_cast<const TC*>(p.q) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     const TC* gin = static_cast<const TC*>(p.g) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     constexpr int QE = (G * half + 255) / 256, GE = (G * DH + 255) / 256;
@@ -518,8 +520,10 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
     const int w0 = lo >> 5, nw = (hi - lo + 31) >> 5;
 
     // ---- new token (every CTA of the cache forms it; only the last one uses v, g)
-    const TC* kin = static_cast<const TC*>(p.k) + (size_t)unit * DH;
-    const TC* vin = static_cast<const TC*>(p.v) + (size_t)unit * DH;
+    // the step's key and value: head kvh / rep of [B, Hkv / rep, d]
+    const size_t tok = (size_t)b * (c.Hkv / c.rep) + kvh / c.rep;
+    const TC* kin = static_cast<const TC*>(p.k) + tok * DH;
+    const TC* vin = static_cast<const TC*>(p.v) + tok * DH;
     const TC* qin = static_cast<const TC*>(p.q) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     const TC* gin = static_cast<const TC*>(p.g) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     float kx = 0.f;

@@ -91,8 +91,9 @@ template <int DH, int G>
 __device__ void new_token(DecTcSmem<DH, G>& S, const DecodeParams& p, int unit, int b, int kvh) {
     constexpr int half = DH / 2;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(p.k) + (size_t)unit * DH;
-    const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(p.v) + (size_t)unit * DH;
+    const size_t tok = (size_t)b * (p.c.Hkv / p.c.rep) + kvh / p.c.rep;   // head kvh / rep of the step's k, v
+    const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(p.k) + tok * DH;
+    const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(p.v) + tok * DH;
     const __nv_bfloat16* qin = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     float kx = 0.f;
     if (tid < DH) {
@@ -146,7 +147,9 @@ __device__ void new_token(DecTcSmem<DH, G>& S, const DecodeParams& p, int unit, 
 }
 
 // The last CTA of a cache: merge the partial states with the new token, gate, write o, clear
-// the eviction words past the live pairs and append the token.
+// the eviction words past the live pairs and append the token.  The states' shifts and sums are
+// gathered into shared memory in one round of loads (the stage buffers, idle by now), so the
+// merge costs a few memory round trips, not one per state.
 template <int DH, int G>
 __device__ void merge_append(DecTcSmem<DH, G>& S, const DecodeParams& p, int unit, int b, int kvh, int n) {
     using C = DecTc<DH, G>;
@@ -158,22 +161,41 @@ __device__ void merge_append(DecTcSmem<DH, G>& S, const DecodeParams& p, int uni
     __nv_bfloat16* oout = static_cast<__nv_bfloat16*>(p.o) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     const float* st0 = p.split_state + (size_t)unit * kDecodeSplitMax * C::SS;
     const int nst = gridDim.x;
+    float* s_m = reinterpret_cast<float*>(S.stage[0][0]);          // [nst][G] shifts (-inf: empty)
+    float* s_l = s_m + kDecodeSplitMax * G;                          // [nst][G] sums
+    float* s_w = s_l + kDecodeSplitMax * G;                          // [nst][G] merge weights
+    float* s_M = s_w + kDecodeSplitMax * G;                          // [G] merged shift
+    float* s_L = s_M + G;                                            // [G] merged sum
+    for (int e = tid; e < nst * G; e += blockDim.x) {
+        const int q = e / G, h = e % G;
+        const float lq = __ldcg(st0 + (size_t)q * C::SS + G + h);
+        s_m[e] = lq > 0.f ? __ldcg(st0 + (size_t)q * C::SS + h) : -INFINITY;
+        s_l[e] = lq > 0.f ? lq : 0.f;
+    }
+    __syncthreads();
+    if (tid < G) {
+        float M = S.own[tid];
+        for (int q = 0; q < nst; ++q) M = fmaxf(M, s_m[q * G + tid]);
+        s_M[tid] = M;
+    }
+    __syncthreads();
+    for (int e = tid; e < nst * G; e += blockDim.x) s_w[e] = s_l[e] > 0.f ? expf(s_m[e] - s_M[e % G]) : 0.f;
+    __syncthreads();
+    if (tid < G) {
+        float Ls = expf(S.own[tid] - s_M[tid]);
+        for (int q = 0; q < nst; ++q) Ls = fmaf(s_l[q * G + tid], s_w[q * G + tid], Ls);
+        s_L[tid] = Ls;
+    }
+    __syncthreads();
     for (int e = tid; e < G * DH; e += blockDim.x) {
         const int h = e / DH, x = e % DH;
-        float M = S.own[h];
-        for (int q = 0; q < nst; ++q)
-            if (__ldcg(st0 + (size_t)q * C::SS + G + h) > 0.f) M = fmaxf(M, __ldcg(st0 + (size_t)q * C::SS + h));
-        float Ls = expf(S.own[h] - M);
-        float A = Ls * S.vt[x];
+        float A = expf(S.own[h] - s_M[h]) * S.vt[x];
+#pragma unroll 8
         for (int q = 0; q < nst; ++q) {
-            const float lq = __ldcg(st0 + (size_t)q * C::SS + G + h);
-            if (lq > 0.f) {
-                const float w = expf(__ldcg(st0 + (size_t)q * C::SS + h) - M);
-                Ls = fmaf(lq, w, Ls);
-                A = fmaf(__ldcg(st0 + (size_t)q * C::SS + 2 * G + e), w, A);
-            }
+            const float w = s_w[q * G + h];
+            if (w != 0.f) A = fmaf(__ldcg(st0 + (size_t)q * C::SS + 2 * G + e), w, A);
         }
-        oout[e] = __float2bfloat16_rn(A / Ls * sigmoid_f(__bfloat162float(gin[e])));
+        oout[e] = __float2bfloat16_rn(A / s_L[h] * sigmoid_f(__bfloat162float(gin[e])));
     }
     if (p.evict_bits)
         for (int w = ((n + 31) >> 5) + tid; w < words; w += blockDim.x) p.evict_bits[(size_t)unit * words + w] = 0u;
@@ -524,6 +546,20 @@ bool map_cache_rows(CUtensorMap* m, const void* base, size_t rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Slices per cache: as many as keep the CTAs of all caches within about two waves of the
+// GPU's resident CTAs (a long cache then takes 64 slices when there are few caches, a handful
+// when there are hundreds), at most kDecodeSplitMax.
+int decode_tc_slices(int units, int ctas_per_sm) {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            sms = 148;
+    }
+    const int n = 2 * ctas_per_sm * sms / std::max(1, units);
+    return std::min(kDecodeSplitMax, std::max(1, n));
+}
+
 template <int DH, int G>
 cudaError_t decode_tc_inst(const DecodeParams& p, cudaStream_t s) {
     const size_t rows = (size_t)p.c.B * p.c.Hkv * p.c.cap;
@@ -534,7 +570,8 @@ cudaError_t decode_tc_inst(const DecodeParams& p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(k_decode_tc<DH, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     UA_PROFILE("k_decode_tc", s);
-    k_decode_tc<DH, G><<<dim3(kDecodeSplitMax, p.c.B * p.c.Hkv), 128, smem, s>>>(mk, mv, p);
+    const int units = p.c.B * p.c.Hkv;
+    k_decode_tc<DH, G><<<dim3(decode_tc_slices(units, DecTc<DH, G>::CTAS), units), 128, smem, s>>>(mk, mv, p);
     return cudaGetLastError();
 }
 
@@ -550,9 +587,11 @@ cudaError_t decode_tc_g(const DecodeParams& p, cudaStream_t s) {
     }
 }
 
-// Footprints: DH = 64 three CTAs per SM, DH = 128 two (227 KB of shared memory per SM).
+// Footprints: DH = 64 three CTAs per SM, DH = 128 two (227 KB of shared memory per SM); the merge
+// reuses the first stage for 3 x kDecodeSplitMax x G + 2 G floats.
 static_assert(3 * (sizeof(DecTcSmem<64, 8>) + 1024) <= 232448, "decode tiles: three CTAs per SM at d = 64");
 static_assert(2 * (sizeof(DecTcSmem<128, 8>) + 1024) <= 232448, "decode tiles: two CTAs per SM at d = 128");
+static_assert((3 * kDecodeSplitMax * 8 + 2 * 8) * 4 <= 16384, "the merge's scratch fits the first stage box");
 
 }  // namespace
 

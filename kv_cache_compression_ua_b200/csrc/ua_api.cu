@@ -163,6 +163,7 @@ ua_status check_cache(const ua_cache* c) {
     if (c->capacity > kMaxCapacity) return UA_ERR_UNSUPPORTED;
     if (c->d != 64 && c->d != 128) return UA_ERR_UNSUPPORTED;
     if (c->dtype != UA_F32 && c->dtype != UA_BF16) return UA_ERR_UNSUPPORTED;
+    if (c->kv_rep < 0 || (c->kv_rep > 1 && c->Hkv % c->kv_rep != 0)) return UA_ERR_INVALID_ARG;
     if (!c->khat || !c->v || !c->bias || !c->rk || !c->pos || !c->n_kept) return UA_ERR_INVALID_ARG;
     const void* ps[] = {c->khat, c->v, c->bias, c->rk, c->pos, c->n_kept};
     for (const void* p : ps)
@@ -172,7 +173,7 @@ ua_status check_cache(const ua_cache* c) {
 
 CacheView view(const ua_cache* c) {
     CacheView v;
-    v.B = c->B; v.Hkv = c->Hkv; v.d = c->d; v.cap = c->capacity;
+    v.B = c->B; v.Hkv = c->Hkv; v.d = c->d; v.cap = c->capacity; v.rep = c->kv_rep > 1 ? c->kv_rep : 1;
     v.khat = c->khat; v.v = c->v; v.bias = c->bias; v.rk = c->rk;
     v.pos = c->pos; v.n_kept = c->n_kept;
     return v;
@@ -650,8 +651,11 @@ ua_status ua_decode_step(const ua_cache* c, int H, const void* q, const void* k,
     ua_status st = check_cache(c);
     if (st != UA_OK) return st;
     const int defer = flags & UA_DECODE_DEFER_COMPACT;
-    if (H < 1 || H % c->Hkv != 0 || pos_t < 0 || !variant_ok(flags & ~UA_DECODE_DEFER_COMPACT))
-        return UA_ERR_INVALID_ARG;
+    // per-query-head decay: a cache of one head per query head; the kernels see the method itself
+    int var = flags & ~UA_DECODE_DEFER_COMPACT;
+    if ((var & kVarPerHead) && H != c->Hkv) return UA_ERR_INVALID_ARG;
+    var &= ~kVarPerHead;
+    if (H < 1 || H % c->Hkv != 0 || pos_t < 0 || !variant_ok(var)) return UA_ERR_INVALID_ARG;
     if (!group_ok(H / c->Hkv)) return UA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !g || !a_q || !a_k || !alpha || !beta || !o) return UA_ERR_INVALID_ARG;
     if (!(p >= 0.f && p <= 1.f) || !isfinite(scale) || !(rope_theta > 0.0)) return UA_ERR_INVALID_ARG;
@@ -663,7 +667,7 @@ ua_status ua_decode_step(const ua_cache* c, int H, const void* q, const void* k,
     dp.logp = p > 0.f ? logf(p) : -INFINITY; dp.theta = rope_theta; dp.rf = rope_freq(rope_theta, c->d);
     dp.q = q; dp.k = k; dp.v = v; dp.g = g; dp.a_q = a_q; dp.a_k = a_k; dp.alpha = alpha; dp.beta = beta;
     dp.o = o; dp.evict_bits = evict_bits; dp.kept_idx = kept_idx;
-    dp.variant = flags & ~UA_DECODE_DEFER_COMPACT; dp.defer = defer ? 1 : 0;
+    dp.variant = var; dp.defer = defer ? 1 : 0;
     dp.split_cnt = nullptr; dp.split_state = nullptr;
     return cuda_status(launch_decode(dp, c->dtype == UA_BF16, static_cast<cudaStream_t>(stream)));
 }
@@ -690,7 +694,9 @@ ua_status ua_decode_step_split(const ua_cache* c, int H, const void* q, const vo
                                int32_t* kept_idx, int flags, void* ws, size_t ws_bytes, void* stream) {
     ua_status st = check_cache(c);
     if (st != UA_OK) return st;
-    const int var = flags & ~UA_DECODE_DEFER_COMPACT;
+    int var = flags & ~UA_DECODE_DEFER_COMPACT;
+    if ((var & kVarPerHead) && H != c->Hkv) return UA_ERR_INVALID_ARG;
+    var &= ~kVarPerHead;
     if (H < 1 || H % c->Hkv != 0 || pos_t < 0 || !variant_ok(var)) return UA_ERR_INVALID_ARG;
     if (!group_ok(H / c->Hkv)) return UA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !g || !a_q || !a_k || !alpha || !beta || !o || !ws) return UA_ERR_INVALID_ARG;

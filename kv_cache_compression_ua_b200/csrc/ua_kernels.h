@@ -86,6 +86,7 @@ cudaError_t launch_tile_qmax(const TileQmaxParams& p, cudaStream_t s);
 
 struct CacheView {
     int B, Hkv, d, cap;
+    int rep;             // cache heads per KV head of the step's / prefill's k and v (>= 1)
     void* khat;          // pair-interleaved unit keys (see il_index)
     void* v;
     float* bias;

@@ -43,7 +43,7 @@ DECODE_DEFER_COMPACT = 256      # ua_decode_step flag: leave evicted pairs in pl
 
 class ua_cache(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int), ("capacity", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("khat", ctypes.c_void_p),
+                ("dtype", ctypes.c_int), ("kv_rep", ctypes.c_int), ("khat", ctypes.c_void_p),
                 ("v", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("rk", ctypes.c_void_p),
                 ("pos", ctypes.c_void_p), ("n_kept", ctypes.c_void_p)]
 
@@ -320,7 +320,8 @@ def prefill_bwd(q, k, v, g, a_q, a_k, alpha, beta, o, lse, b_final, d_o, *, scal
 class Cache:
     """Device tensors of one self-pruning cache set (see ua_cache in ua.h).  khat holds the unit
     keys pair-interleaved (element 2m = component m, 2m+1 = component m + d/2); `khat_natural()`
-    returns them in the natural order."""
+    returns them in the natural order.  kv_rep: cache heads per head of the keys and values the
+    cache is filled and stepped with (G for per-query-head decay, where Hkv = H)."""
     B: int
     Hkv: int
     d: int
@@ -332,9 +333,12 @@ class Cache:
     rk: torch.Tensor
     pos: torch.Tensor
     n_kept: torch.Tensor
+    kv_rep: int = 1
 
     @staticmethod
-    def empty(B, Hkv, d, capacity, dtype=torch.bfloat16, device="cuda"):
+    def empty(B, Hkv, d, capacity, dtype=torch.bfloat16, device="cuda", kv_rep=1):
+        if kv_rep < 1 or Hkv % kv_rep:
+            raise ValueError(f"kv_rep {kv_rep} must divide Hkv {Hkv}")
         kw = dict(device=device)
         return Cache(B, Hkv, d, capacity, dtype,
                      torch.zeros(B, Hkv, capacity, d, dtype=dtype, **kw),
@@ -342,7 +346,12 @@ class Cache:
                      torch.zeros(B, Hkv, capacity, dtype=torch.float32, **kw),
                      torch.zeros(B, Hkv, capacity, dtype=torch.float32, **kw),
                      torch.zeros(B, Hkv, capacity, dtype=torch.int32, **kw),
-                     torch.zeros(B, Hkv, dtype=torch.int32, **kw))
+                     torch.zeros(B, Hkv, dtype=torch.int32, **kw), kv_rep)
+
+    @property
+    def Hin(self) -> int:
+        """Heads of the keys and values the cache is filled and stepped with."""
+        return self.Hkv // self.kv_rep
 
     def struct(self) -> ua_cache:
         n = self.B * self.Hkv * self.capacity
@@ -356,7 +365,7 @@ class Cache:
         dev = self.khat.device
         _same_device(dev, **{f"cache.{n}": getattr(self, n) for n in names})
         ptrs = [_ptr(getattr(self, n)).value for n in names]
-        return ua_cache(self.B, self.Hkv, self.d, self.capacity, _dtype_code(self.dtype), *ptrs)
+        return ua_cache(self.B, self.Hkv, self.d, self.capacity, _dtype_code(self.dtype), int(self.kv_rep), *ptrs)
 
     def nbytes_per_entry(self) -> int:
         return 2 * self.d * self.khat.element_size() + 12
@@ -370,12 +379,12 @@ FIELDS = ("khat", "v", "bias", "rk", "pos", "n_kept")
 
 
 def cache_fill(cache: Cache, k, v, a_k, b_final, *, theta=500000.0, stream=None):
-    if k.dim() != 4 or (k.shape[0], k.shape[2], k.shape[3]) != (cache.B, cache.Hkv, cache.d):
-        raise ValueError(f"k: shape {tuple(k.shape)}, expected [{cache.B}, T, {cache.Hkv}, {cache.d}]")
+    if k.dim() != 4 or (k.shape[0], k.shape[2], k.shape[3]) != (cache.B, cache.Hin, cache.d):
+        raise ValueError(f"k: shape {tuple(k.shape)}, expected [{cache.B}, T, {cache.Hin}, {cache.d}]")
     T = k.shape[1]
     n = cache.B * T * cache.Hkv
-    _need("k", k, n * cache.d, (cache.dtype,))
-    _need("v", v, n * cache.d, (cache.dtype,))
+    _need("k", k, cache.B * T * cache.Hin * cache.d, (cache.dtype,))
+    _need("v", v, cache.B * T * cache.Hin * cache.d, (cache.dtype,))
     _need("a_k", a_k, n, F32)
     _need("b_final", b_final, n, F32)
     c = cache.struct()
@@ -419,8 +428,8 @@ def decode_step(cache: Cache, q, k, v, g, a_q, a_k, alpha, beta, pos_t: int, p: 
         raise ValueError(f"q: shape {tuple(q.shape)}, expected [{cache.B}, H, {cache.d}]")
     Hkv, act = cache.Hkv, (cache.dtype,)
     _need("q", q, B * H * d, act)
-    _need("k", k, B * Hkv * d, act)
-    _need("v", v, B * Hkv * d, act)
+    _need("k", k, B * cache.Hin * d, act)
+    _need("v", v, B * cache.Hin * d, act)
     _need("g", g, B * H * d, act)
     _need("a_q", a_q, B * Hkv, F32)
     _need("a_k", a_k, B * Hkv, F32)

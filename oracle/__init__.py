@@ -44,7 +44,7 @@ def _load():
         P = ctypes.c_void_p
         I = ctypes.c_int
         Dd = ctypes.c_double
-        lib.ora_prefill_fwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 4 + [I, Dd, I]
+        lib.ora_prefill_fwd.argtypes = [I, I, I, I, I, Dd, Dd] + [P] * 8 + [P, P] + [P] * 4 + [I, Dd, I, I]
         lib.ora_prefill_fwd.restype = I
         lib.ora_lambda_bruteforce.argtypes = [I, I, I, I, P, P, P, P, P, P, I, I]
         lib.ora_lambda_bruteforce.restype = I
@@ -77,11 +77,14 @@ VAR_NO_Q, VAR_NO_K, VAR_NO_SIM, VAR_QNORM = 1, 2, 4, 8
 
 
 def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0,
-                want_lambda=False, unit_mask=None, row_mask=None, variant=0, prune_p=0.0, nthreads=None):
+                want_lambda=False, unit_mask=None, row_mask=None, variant=0, prune_p=0.0, bf16_operands=False,
+                nthreads=None):
     """Prefill forward of UA in fp64.
 
     Shapes: q, g [B,T,H,d]; k, v [B,T,Hkv,d]; a_q, a_k [B,T,Hkv]; alpha, beta [Hkv].
     prune_p > 0: chunked pruned prefill (128-token chunks, threshold p); 0 = dense.
+    bf16_operands: a model for tolerances, not the method: the unit keys, rotated keys and
+    rotated queries are rounded to bf16 where they enter the similarity and the logits.
     Returns dict(o [B,T,H,d], lse [B,H,T], b_final [B,Hkv,T], lam [B,Hkv,T,T] or None).
     Entries outside unit_mask / row_mask are left as NaN.
     """
@@ -101,7 +104,7 @@ def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0
                                  _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(a_q), _ptr(a_k),
                                  _ptr(alpha), _ptr(beta), _ptr(um), _ptr(rm),
                                  _ptr(o), _ptr(lse), _ptr(bfin), _ptr(lam), int(variant),
-                                 float(np.log(prune_p)) if prune_p > 0 else -np.inf,
+                                 float(np.log(prune_p)) if prune_p > 0 else -np.inf, int(bool(bf16_operands)),
                                  nthreads or default_threads())
     if rc != 0:
         raise ValueError(f"ora_prefill_fwd rejected the shapes (code {rc})")
@@ -280,3 +283,12 @@ def prefill_bwd_per_head(q, k, v, g, a_q, a_k, alpha, beta, d_o, **kw):
     r["dk"] = r["dk"].reshape(B, T, Hkv, G, d).sum(axis=3)
     r["dv"] = r["dv"].reshape(B, T, Hkv, G, d).sum(axis=3)
     return r
+
+
+def decode_step_per_head(cache: DecodeCache, q, k, v, g, a_q, a_k, alpha, beta, pos_t, p, **kw):
+    """One decode step with per-query-head decay: cache holds one head per query head (filled from
+    the keys and values repeated over each group); q, g [B,H,d]; k, v [B,Hkv,d]; a_q, a_k [B,H];
+    alpha, beta [H].  Returns as decode_step."""
+    G = np.shape(q)[1] // np.shape(k)[1]
+    return decode_step(cache, q, np.repeat(_f64(k), G, axis=1), np.repeat(_f64(v), G, axis=1), g, a_q, a_k,
+                       alpha, beta, pos_t, p, **kw)

@@ -175,6 +175,25 @@ static void run_units(unit_fn fn, void* ctx, int n_units, int nthreads) {
 
 /* ------------------------------------------------------------------ prefill forward */
 
+/* Nearest bf16 value (8 significant bits) of x, ties to even, by way of the nearest float.
+ * Used only by the tolerance models (bf16 operands of the forward, saved outputs of the
+ * backward). */
+static double round_bf16(double x) {
+    float f = (float)x;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) != 0x7f800000u) {
+        u += 0x7fffu + ((u >> 16) & 1u);
+        u &= 0xffff0000u;
+        memcpy(&f, &u, sizeof f);
+    }
+    return (double)f;
+}
+
+/* Forward.  Operand model (optional, for deriving tolerances only; bf16_operands set): the
+ * unit keys, the rotated keys and the rotated queries are rounded to bf16 where they enter the
+ * similarity and the logits, as in an implementation whose products take bf16 operands; the
+ * logit error that leaves grows with scale*||q||. */
 typedef struct {
     int B, T, H, Hkv, d;
     double scale, theta;
@@ -184,6 +203,7 @@ typedef struct {
     double *o, *lse, *bfinal, *lambda;
     int variant;
     double prune_logp;        /* log p of the chunked prefill pruning, -inf = dense */
+    int bf16_operands;        /* operand model (see above) */
 } fwd_ctx;
 
 static void fwd_unit(void* vctx, int unit) {
@@ -210,6 +230,11 @@ static void fwd_unit(void* vctx, int unit) {
         l2_normalise(kt, d, khat + (size_t)t * d);
         rope(khat + (size_t)t * d, d, (double)t, c->theta, 1.0, krot + (size_t)t * d);
         rk[t] = softplus(c->ak[((size_t)b * T + t) * Hkv + kvh]);
+        if (c->bf16_operands)
+            for (int x = 0; x < d; ++x) {
+                khat[(size_t)t * d + x] = round_bf16(khat[(size_t)t * d + x]);
+                krot[(size_t)t * d + x] = round_bf16(krot[(size_t)t * d + x]);
+            }
     }
 
     for (int i = 0; i < T; ++i) {
@@ -235,6 +260,8 @@ static void fwd_unit(void* vctx, int unit) {
             int h = kvh * G + hh;
             const double* qi = c->q + (((size_t)b * T + i) * H + h) * d;
             rope_query(qi, d, (double)i, c->theta, c->variant, qtmp, qrot);
+            if (c->bf16_operands)
+                for (int x = 0; x < d; ++x) qrot[x] = round_bf16(qrot[x]);
             double m = -INFINITY;
             for (int j = 0; j <= i; ++j) {
                 /* evicted at the chunk boundary: no longer in the cache */
@@ -275,12 +302,12 @@ int ora_prefill_fwd(int B, int T, int H, int Hkv, int d, double scale, double th
                     const double* aq, const double* ak, const double* alpha, const double* beta,
                     const uint8_t* unit_mask, const uint8_t* row_mask,
                     double* o, double* lse, double* bfinal, double* lambda, int variant,
-                    double prune_logp, int nthreads) {
+                    double prune_logp, int bf16_operands, int nthreads) {
     if (B < 1 || T < 1 || H < 1 || Hkv < 1 || d < 2 || (d & 1) || H % Hkv) return 1;
     if ((variant & ~VAR_ALL) || n_active(variant) == 0) return 1;
     if (isnan(prune_logp) || prune_logp > 0.0) return 1;
     fwd_ctx c = {B, T, H, Hkv, d, scale, theta, q, k, v, g, aq, ak, alpha, beta,
-                 unit_mask, row_mask, o, lse, bfinal, lambda, variant, prune_logp};
+                 unit_mask, row_mask, o, lse, bfinal, lambda, variant, prune_logp, bf16_operands != 0};
     run_units(fwd_unit, &c, B * Hkv, nthreads);
     return 0;
 }
@@ -533,19 +560,7 @@ typedef struct {
     double model_c;             /* saved-output model (see above); 0 = off */
 } bwd_ctx;
 
-/* Nearest bf16 value (8 significant bits) of x, ties to even, by way of the nearest float.
- * Used only by the saved-output model. */
-static double round_bf16(double x) {
-    float f = (float)x;
-    uint32_t u;
-    memcpy(&u, &f, sizeof u);
-    if ((u & 0x7f800000u) != 0x7f800000u) {
-        u += 0x7fffu + ((u >> 16) & 1u);
-        u &= 0xffff0000u;
-        memcpy(&f, &u, sizeof f);
-    }
-    return (double)f;
-}
+
 
 static size_t tri(int i, int j) { return (size_t)i * (size_t)(i + 1) / 2 + (size_t)j; }
 

@@ -91,3 +91,21 @@ def assert_grad_close(name, got, ref, dtype, model_rms=None):
     err = np.abs(got - ref)
     assert np.all(err <= allow) and np.linalg.norm(got - ref) <= l2, (
         f"{name}: error {err} above {allow} (L2 {np.linalg.norm(got - ref):.3e} > {l2:.3e}?), ref {ref}")
+
+
+def assert_close_model(name, got, ref, model, dtype, factor=3.0, relative_max=False):
+    """assert_close with the bar widened to `factor` times the deviation of an oracle tolerance
+    model (the same computation with the implementation's roundings) from the exact result,
+    where that is larger: rel-L2 and max error each."""
+    rl, ma = TOL[dtype]
+    ref64 = np.asarray(ref, np.float64)
+    mdl = np.asarray(model, np.float64)
+    if relative_max:
+        den = np.linalg.norm(np.maximum(1.0, np.abs(ref64)))
+        mr = float(np.linalg.norm(mdl - ref64) / den)
+        mm = float((np.abs(mdl - ref64) / np.maximum(1.0, np.abs(ref64))).max())
+    else:
+        mr = rel_l2(mdl, ref64)
+        mm = float(np.abs(mdl - ref64).max())
+    return assert_close(name, got, ref, dtype, relative_max=relative_max,
+                        tol=(max(rl, factor * mr), max(ma, factor * mm)))

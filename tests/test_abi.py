@@ -127,22 +127,28 @@ def test_lambda_debug_limited_to_small_T(lib):
 
 def test_cache_calls_reject_bad_arguments(lib):
     P = ctypes.c_void_p
-    c = ua.ua_cache(2, 2, 64, 100, ua.UA_BF16, *([FAKE] * 6))
+    c = ua.ua_cache(2, 2, 64, 100, ua.UA_BF16, 1, *([FAKE] * 6))
     # capacity too small for the fill
     assert lib.ua_cache_fill(ctypes.byref(c), 101, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 5e5, None) == 5
     # bad p without a mask
     assert lib.ua_cache_compact(ctypes.byref(c), None, ctypes.c_float(1.5), None, None) == 1
     # misaligned cache array
-    c2 = ua.ua_cache(2, 2, 64, 100, ua.UA_BF16, *([FAKE] * 5 + [FAKE + 4]))
+    c2 = ua.ua_cache(2, 2, 64, 100, ua.UA_BF16, 1, *([FAKE] * 5 + [FAKE + 4]))
     assert lib.ua_cache_compact(ctypes.byref(c2), None, ctypes.c_float(0.1), None, None) == 3
     # decode: group size 5 unsupported, flags must be valid variant bits, head_dim 80 unsupported
     args = [P(FAKE)] * 8
     assert lib.ua_decode_step(ctypes.byref(c), 10, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
                               P(FAKE), None, None, 0, None) == 2
-    for bad in (16, 7, 15, -1, 512, 256 | 7, 256 | 16):   # unknown bits; all three decay mechanisms off
+    # unknown bits; all three decay mechanisms off; per-query-head decay on a cache that does not
+    # hold one head per query head (H = 8 != Hkv = 2)
+    for bad in (16, 7, 15, -1, 512, 256 | 7, 256 | 16):
         assert lib.ua_decode_step(ctypes.byref(c), 8, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
                                   P(FAKE), None, None, bad, None) == 1
-    c3 = ua.ua_cache(2, 2, 80, 100, ua.UA_BF16, *([FAKE] * 6))
+    # kv_rep must divide Hkv (and not be negative)
+    for rep in (3, -1):
+        cr = ua.ua_cache(2, 2, 64, 100, ua.UA_BF16, rep, *([FAKE] * 6))
+        assert lib.ua_cache_compact(ctypes.byref(cr), None, ctypes.c_float(0.1), None, None) == 1
+    c3 = ua.ua_cache(2, 2, 80, 100, ua.UA_BF16, 1, *([FAKE] * 6))
     assert lib.ua_decode_step(ctypes.byref(c3), 8, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
                               P(FAKE), None, None, 0, None) == 2
 

@@ -1,9 +1,9 @@
 """Per-query-head decay in the oracle (the alternative to decay parameters per KV head).
 
-Pins: rates that are equal across the heads of a group reproduce the per-KV-head results;
-with G = 1 the two readings coincide; the gradients (dk and dv summed over the group's
-heads) equal central differences of the per-head forward; distinct per-head rates give
-distinct heads."""
+Pins: rates that are equal across the heads of a group reproduce the per-KV-head results
+(prefill and decode); with G = 1 the two readings coincide; the gradients (dk and dv summed over
+the group's heads) equal central differences of the per-head forward; distinct per-head rates
+give distinct heads."""
 import numpy as np
 import pytest
 
@@ -86,3 +86,41 @@ def test_per_head_backward_matches_central_differences():
         assert gr[gname].shape == base.shape, gname
         err = np.max(np.abs(fd - gr[gname]))
         assert err <= 1e-6 * (1.0 + np.max(np.abs(fd))), (name, err)
+
+
+def test_shared_rates_reproduce_the_per_kv_head_decode():
+    """A cache of one head per query head, filled from the keys and values repeated over each
+    group and stepped with rates repeated over it, gives the per-KV-head decode: the same
+    outputs, and every copy of a group keeps the group's biases and evictions."""
+    w, x = case(T=30, B=2, H=4, Hkv=2, d=8, seed=11)
+    G = w.H // w.Hkv
+    xo = {k: v for k, v in x.items() if k != "d_o"}
+    ref_pf = oracle.prefill_fwd(**xo)
+    p = 0.2
+    logp = np.log(p)
+    ref = oracle.DecodeCache(w.B, w.Hkv, w.d, w.T + 8)
+    ref.fill_from_prefill(x["k"], x["v"], x["a_k"], ref_pf["b_final"], logp=logp)
+    ph = oracle.DecodeCache(w.B, w.H, w.d, w.T + 8)
+    ph.fill_from_prefill(np.repeat(x["k"], G, axis=2), np.repeat(x["v"], G, axis=2), np.repeat(x["a_k"], G, axis=2),
+                         np.repeat(ref_pf["b_final"], G, axis=1), logp=logp)
+    rng = np.random.default_rng(5)
+    evicted = 0
+    for s in range(6):
+        q = rng.standard_normal((w.B, w.H, w.d))
+        k = rng.standard_normal((w.B, w.Hkv, w.d))
+        v = rng.standard_normal((w.B, w.Hkv, w.d))
+        gt = rng.standard_normal((w.B, w.H, w.d))
+        aq = rng.standard_normal((w.B, w.Hkv)) + 1.0
+        ak = rng.standard_normal((w.B, w.Hkv))
+        r1 = oracle.decode_step(ref, q, k, v, gt, aq, ak, x["alpha"], x["beta"], w.T + s, p)
+        r2 = oracle.decode_step_per_head(ph, q, k, v, gt, np.repeat(aq, G, axis=1), np.repeat(ak, G, axis=1),
+                                         np.repeat(x["alpha"], G), np.repeat(x["beta"], G), w.T + s, p)
+        np.testing.assert_allclose(r2["o"], r1["o"], atol=1e-12, rtol=0)
+        np.testing.assert_array_equal(ph.n, np.repeat(ref.n, G, axis=1))
+        for b in range(w.B):
+            for h in range(w.H):
+                n = ref.n[b, h // G]
+                np.testing.assert_array_equal(ph.pos[b, h, :n], ref.pos[b, h // G, :n])
+                np.testing.assert_allclose(ph.b[b, h, :n], ref.b[b, h // G, :n], atol=1e-12, rtol=0)
+        evicted += int(r1["evict"].sum())
+    assert evicted > 0

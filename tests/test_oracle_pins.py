@@ -454,3 +454,29 @@ def test_bf16_saved_output_model_off_is_the_method():
     b = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta, bf16_saved_model=0.0)
     for n in a:
         np.testing.assert_array_equal(a[n], b[n])
+
+
+
+def test_bf16_operand_model_single_token_closed_form():
+    """The oracle forward's bf16-operand model (a tolerance model, not the method) on one token at
+    position 0, where RoPE is the identity and the softmax has one term: o = v * sigmoid(g) as in
+    the method, and lse = scale * <bf16(q), bf16(khat)> (torch's bf16 conversion, round to
+    nearest even); with the model off, lse = scale * <q, khat>."""
+    rng = np.random.default_rng(21)
+    d, H = 64, 2
+    x = {"q": rng.standard_normal((1, 1, H, d)) * 30, "k": rng.standard_normal((1, 1, 1, d)),
+         "v": rng.standard_normal((1, 1, 1, d)), "g": rng.standard_normal((1, 1, H, d)),
+         "a_q": rng.standard_normal((1, 1, 1)), "a_k": rng.standard_normal((1, 1, 1)),
+         "alpha": np.array([2.0]), "beta": np.array([-1.0])}
+    scale = d ** -0.5
+    ex = oracle.prefill_fwd(**x, scale=scale)
+    mo = oracle.prefill_fwd(**x, scale=scale, bf16_operands=True)
+    bf = lambda a: torch.tensor(np.asarray(a, np.float64)).float().bfloat16().double().numpy()
+    khat = x["k"][0, 0, 0] / np.linalg.norm(x["k"][0, 0, 0])
+    for h in range(H):
+        q = x["q"][0, 0, h]
+        np.testing.assert_allclose(mo["lse"][0, h, 0], scale * float(bf(q) @ bf(khat)), rtol=1e-12)
+        np.testing.assert_allclose(ex["lse"][0, h, 0], scale * float(q @ khat), rtol=1e-12)
+        gate = 1.0 / (1.0 + np.exp(-x["g"][0, 0, h]))
+        np.testing.assert_allclose(mo["o"][0, 0, h], x["v"][0, 0, 0] * gate, rtol=1e-12)
+    assert abs(mo["lse"][0, 0, 0] - ex["lse"][0, 0, 0]) > 0          # the rounding is seen
