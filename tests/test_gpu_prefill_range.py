@@ -16,7 +16,7 @@ import torch
 import oracle
 from kv_cache_compression_ua_b200 import inputs as I
 from kv_cache_compression_ua_b200 import ua
-from helpers import assert_close
+from helpers import assert_close, assert_close_model
 
 pytestmark = pytest.mark.gpu
 
@@ -75,7 +75,11 @@ def test_rows_out_of_shift_range_are_recomputed_exactly(d, H, Hkv, T, want_bfina
 
 @pytest.mark.parametrize("d", [64, 128])
 def test_trained_scale_query_norms(d):
-    """Every query rescaled to norm 400 (scale*||q|| = 50 at d = 64, 35 at d = 128)."""
+    """Every query rescaled to norm 400 (scale*||q|| = 50 at d = 64, 35 at d = 128).  The products
+    take bf16 operands (rotated queries and keys), whose rounding puts an error of about
+    2^-9 * scale*||q|| / sqrt(d) on every logit: at these norms that alone moves o by ~5e-3 (the
+    oracle's bf16-operand model: 5.2e-3 rel-L2 / 3.9e-2 max at d = 64), so o and lse are held to
+    3x that model's deviation where it exceeds the bf16 bar."""
     w = I.Workload("range400", 1, 600, 4, 1, d, "bf16", 8300 + d)
     x = {k: v for k, v in I.make_prefill_inputs(w).items() if k != "d_o"}
     q = x["q"].astype(np.float64)
@@ -84,5 +88,6 @@ def test_trained_scale_query_norms(d):
     g, names, fixed = run(w, x, True)
     assert ("k_fwd_tc" if d == 64 else "k_fwd_tc128") in names, names
     r = oracle.prefill_fwd(**x, scale=w.scale, theta=w.theta)
-    assert_close("o", g["o"], r["o"], "bf16")
-    assert_close("lse", g["lse"], r["lse"], "bf16", relative_max=True)
+    m = oracle.prefill_fwd(**x, scale=w.scale, theta=w.theta, bf16_operands=True)
+    assert_close_model("o", g["o"], r["o"], m["o"], "bf16")
+    assert_close_model("lse", g["lse"], r["lse"], m["lse"], "bf16", relative_max=True)
