@@ -78,6 +78,7 @@ struct DecTcSmem {
     float shift[G];
     float red[G][4];
     float red2[4];
+    unsigned tflag[2];                                       // per tile parity: bit 0 abort, bit 1 raise the shift
     uint64_t full[C::NST];
     uint64_t sfull, pfree;
     uint32_t tmem_base;
@@ -315,6 +316,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     // the second block of P columns (heads 8-15) stays zero when G <= 8
     for (int idx = tid; idx < kDecTile * 4; idx += blockDim.x) reinterpret_cast<uint32_t*>(S.pt[1])[idx] = 0u;
     if (tid < G) S.shift[tid] = S.own[tid];
+    if (tid == 0) S.tflag[0] = S.tflag[1] = 0u;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
 
@@ -343,10 +345,9 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
             }
         }
         if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (t / NST) & 1, abort))) ok = false;
-        if (__syncthreads_or(!ok)) { ok = false; break; }
         // ---- x_j = <khat_t, khat_j>, and khat_j rotated in place (16-byte chunks, swizzled)
         float x = 0.f;
-        {
+        if (ok) {
             const double pd = (double)pj;
 #pragma unroll 1
             for (int bx = 0; bx < NB; ++bx) {
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
             }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncthreads();
+        if (__syncthreads_or(!ok)) { ok = false; break; }
         // ---- S of the tile
         if (leader) {
             tc_fence_after();
@@ -398,8 +399,9 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         if (p.evict_bits && lane == 0 && wj0 < hi) p.evict_bits[(size_t)unit * words + (wj0 >> 5)] = ev;
         if (!__all_sync(0xffffffffu, mbar_wait(&S.sfull, t & 1, abort))) ok = false;
         tc_fence_after();
-        float xs[16];
-        tmem_ld16(tmem + lane_base + C::COL_S, xs);
+        float xs[2 * G <= 8 ? 8 : 16];
+        if (2 * G <= 8) tmem_ld8(tmem + lane_base + C::COL_S, xs);
+        else tmem_ld16(tmem + lane_base + C::COL_S, xs);
         float lg[G], nsh[G];
         bool over = false;                            // a logit above its head's shift by > kRescaleGap
 #pragma unroll
@@ -411,8 +413,16 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         // the previous tile's second product must be done before P and O are touched, and before
         // its stage is refilled
         if (t >= 1 && !__all_sync(0xffffffffu, mbar_wait(&S.pfree, (t - 1) & 1, abort))) ok = false;
-        if (__syncthreads_or(!ok)) { ok = false; break; }
-        const bool any = __syncthreads_or(over) != 0;
+        {   // one barrier for both votes: bit 0 abort, bit 1 a logit above its shift's headroom
+            const unsigned ba = __ballot_sync(0xffffffffu, !ok), bo = __ballot_sync(0xffffffffu, over);
+            if (lane == 0 && (ba | bo)) atomicOr(&S.tflag[t & 1], (ba ? 1u : 0u) | (bo ? 2u : 0u));
+        }
+        __syncthreads();
+        const unsigned fl = S.tflag[t & 1];
+        if (fl & 1u) { ok = false; break; }
+        const bool any = (fl & 2u) != 0;
+        if (tid == 0) S.tflag[(t + 1) & 1] = 0u;      // the next tile's word (its writers come after
+                                                      // this tile's last barrier)
         tc_fence_after();
         if (NST > 1 && leader && t >= 1 && t - 1 + NST < ntiles) issue_tile(t - 1 + NST);
         // ---- shift: raised (and the accumulated values rescaled) when a logit of the tile
@@ -546,18 +556,31 @@ bool map_cache_rows(CUtensorMap* m, const void* base, size_t rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Slices per cache: as many as keep the CTAs of all caches within about two waves of the
-// GPU's resident CTAs (a long cache then takes 64 slices when there are few caches, a handful
-// when there are hundreds), at most kDecodeSplitMax.
-int decode_tc_slices(int units, int ctas_per_sm) {
+// Slices per cache (the grid's x extent; a cache uses fewer when it is short): the count that
+// minimises (waves of resident CTAs) x (a CTA's fixed cost + its tiles), with the tiles taken
+// from the capacity and a CTA's fixed cost (new token, setup, arrival) counted as two tiles.
+// Few caches get many slices (up to kDecodeSplitMax), hundreds of long ones a handful, sized so
+// the last wave is nearly full.
+int decode_tc_slices(int units, int cap, int ctas_per_sm) {
     static int sms = 0;
     if (sms == 0) {
         int dev = 0;
         if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             sms = 148;
     }
-    const int n = 2 * ctas_per_sm * sms / std::max(1, units);
-    return std::min(kDecodeSplitMax, std::max(1, n));
+    const long long slots = (long long)ctas_per_sm * sms;
+    const long long tiles = (cap + kDecTile - 1) / kDecTile;
+    int best = 1;
+    long long best_cost = -1;
+    for (int n = 1; n <= kDecodeSplitMax; ++n) {
+        const long long waves = ((long long)std::max(1, units) * n + slots - 1) / slots;
+        const long long cost = waves * (2 + (tiles + n - 1) / n);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = n;
+        }
+    }
+    return best;
 }
 
 template <int DH, int G>
@@ -571,7 +594,7 @@ cudaError_t decode_tc_inst(const DecodeParams& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     UA_PROFILE("k_decode_tc", s);
     const int units = p.c.B * p.c.Hkv;
-    k_decode_tc<DH, G><<<dim3(decode_tc_slices(units, DecTc<DH, G>::CTAS), units), 128, smem, s>>>(mk, mv, p);
+    k_decode_tc<DH, G><<<dim3(decode_tc_slices(units, p.c.cap, DecTc<DH, G>::CTAS), units), 128, smem, s>>>(mk, mv, p);
     return cudaGetLastError();
 }
 
