@@ -69,6 +69,10 @@ struct DecTcSmem {
     alignas(1024) uint8_t bq[16 * DH * 2];                   // no-swizzle K-major B of S
     alignas(128) uint8_t pt[2][kDecTile][16];                // P: MN-major no-swizzle, heads 0-7 | 8-15
     double gtf[DH / 2];                                       // RoPE frequencies / (2 pi)
+    float ff[DH / 2];                                        // RoPE frequencies (fp32)
+    float bcs[2][DH / 2][2];                                 // per tile parity: cos, sin of pos_base * f_m
+    int wd[2][4];                                            // per tile parity and warp: pos_j - j, or a
+                                                             // sentinel when the warp's positions are not contiguous
     float kt[DH];                                            // khat_t, pair-interleaved
     float ktr[DH];                                           // RoPE(khat_t, pos_t), pair-interleaved
     float vt[DH];
@@ -105,7 +109,10 @@ __device__ void new_token(DecTcSmem<DH, G>& S, const DecodeParams& p, int unit, 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) S.red2[warp] = ss;
-    for (int m = tid; m < half; m += blockDim.x) S.gtf[m] = p.rf.f[m] * 0.15915494309189535;
+    for (int m = tid; m < half; m += blockDim.x) {
+        S.gtf[m] = p.rf.f[m] * 0.15915494309189535;
+        S.ff[m] = (float)p.rf.f[m];
+    }
     __syncthreads();
     const float den = fmaxf(sqrtf(S.red2[0] + S.red2[1] + S.red2[2] + S.red2[3]), 1e-12f);
     if (tid < DH) S.kt[il_index(tid, half)] = kx / den;
@@ -221,6 +228,28 @@ __device__ void merge_append(DecTcSmem<DH, G>& S, const DecodeParams& p, int uni
     if (tid == 0) p.split_cnt[unit] = 0u;            // ready for the next step
 }
 
+// Dense tiles: when a tile's positions are contiguous (pos_j = pos_base + (j - first slot), as in a
+// cache that has evicted nothing since the slots were written), an entry's rotation angle is
+// pos_base*f + tid*f, so the exact reduction (double precision) is needed once per frequency and
+// tile, and each thread adds its small offset angle tid*f (|tid*f| < 128, fp32 and the fast
+// sine/cosine unit) by the angle-addition formulas.  Each warp records pos_j - j for its entries
+// (kNotDense if they disagree); warp 0 forms cos/sin of pos_base*f for the tile.
+constexpr int kNotDense = -2147483647;
+
+template <int DH, int G>
+__device__ __forceinline__ void tile_density(DecTcSmem<DH, G>& S, int par, int pj, int j, bool valid, int warp,
+                                             int lane) {
+    const int dj = pj - j;
+    const int ref = __shfl_sync(0xffffffffu, dj, 0);             // lane 0 holds the warp's first entry
+    const bool same = __all_sync(0xffffffffu, !valid || dj == ref);
+    const bool any = __any_sync(0xffffffffu, valid);
+    if (lane == 0) S.wd[par][warp] = !any ? ref : (same ? ref : kNotDense);
+    if (warp == 0) {                                              // base angles: pos of the first slot
+        const double pb = (double)__shfl_sync(0xffffffffu, pj, 0);
+        for (int m = lane; m < DH / 2; m += 32) rope_cs_turns(pb, S.gtf[m], &S.bcs[par][m][0], &S.bcs[par][m][1]);
+    }
+}
+
 template <int DH, int G>
 __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     k_decode_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_v, DecodeParams p) {
@@ -317,6 +346,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     for (int idx = tid; idx < kDecTile * 4; idx += blockDim.x) reinterpret_cast<uint32_t*>(S.pt[1])[idx] = 0u;
     if (tid < G) S.shift[tid] = S.own[tid];
     if (tid == 0) S.tflag[0] = S.tflag[1] = 0u;
+    tile_density<DH, G>(S, 0, pj_n, lo + tid, lo + tid < hi, warp, lane);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
 
@@ -347,7 +377,41 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (t / NST) & 1, abort))) ok = false;
         // ---- x_j = <khat_t, khat_j>, and khat_j rotated in place (16-byte chunks, swizzled)
         float x = 0.f;
-        if (ok) {
+        const int par = t & 1;
+        bool dense = true;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int dw = S.wd[par][w];
+            dense = dense && (lo + t * kDecTile + w * 32 >= hi || (dw != kNotDense && dw == S.wd[par][0]));
+        }
+        if (ok && dense) {
+            const float tf = (float)tid;
+#pragma unroll 1
+            for (int bx = 0; bx < NB; ++bx) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint8_t* ptr = S.stage[s][NB + bx] + (uint32_t)tid * 128u + ((uint32_t)(ch ^ (tid & 7)) << 4);
+                    float xa[8], xb[8];
+                    Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(ptr), xa);
+                    const float4 k0 = *reinterpret_cast<const float4*>(&S.kt[bx * 64 + ch * 8]);
+                    const float4 k1 = *reinterpret_cast<const float4*>(&S.kt[bx * 64 + ch * 8 + 4]);
+                    x = fmaf(k0.x, xa[0], x); x = fmaf(k0.y, xa[1], x); x = fmaf(k0.z, xa[2], x);
+                    x = fmaf(k0.w, xa[3], x); x = fmaf(k1.x, xa[4], x); x = fmaf(k1.y, xa[5], x);
+                    x = fmaf(k1.z, xa[6], x); x = fmaf(k1.w, xa[7], x);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int m = bx * 32 + ch * 4 + i;
+                        float co, so;
+                        __sincosf(tf * S.ff[m], &so, &co);
+                        const float cb = S.bcs[par][m][0], sb = S.bcs[par][m][1];
+                        const float cs = cb * co - sb * so, sn = fmaf(sb, co, cb * so);
+                        xb[2 * i] = xa[2 * i] * cs - xa[2 * i + 1] * sn;
+                        xb[2 * i + 1] = xa[2 * i + 1] * cs + xa[2 * i] * sn;
+                    }
+                    Vec16<__nv_bfloat16>::st(reinterpret_cast<__nv_bfloat16*>(ptr), xb);
+                }
+            }
+        } else if (ok) {
             const double pd = (double)pj;
 #pragma unroll 1
             for (int bx = 0; bx < NB; ++bx) {
@@ -423,6 +487,8 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         const bool any = (fl & 2u) != 0;
         if (tid == 0) S.tflag[(t + 1) & 1] = 0u;      // the next tile's word (its writers come after
                                                       // this tile's last barrier)
+        // the next tile's contiguity and base angles (read after this tile's last barrier)
+        if (t + 1 < ntiles) tile_density<DH, G>(S, (t + 1) & 1, pj_n, j + kDecTile, j + kDecTile < hi, warp, lane);
         tc_fence_after();
         if (NST > 1 && leader && t >= 1 && t - 1 + NST < ntiles) issue_tile(t - 1 + NST);
         // ---- shift: raised (and the accumulated values rescaled) when a logit of the tile
