@@ -22,7 +22,7 @@
 // and raised, with the accumulated values rescaled in TMEM, whenever a tile's maximum exceeds it
 // by more than 16; so no probability exceeds e^16 and none that matters underflows.
 //
-// Work split: grid (kDecodeSplitMax, B*Hkv), two or three 128-thread CTAs per SM.  Cache (b, h)
+// Work split: grid (slices, B*Hkv), two or four 128-thread CTAs per SM.  Cache (b, h)
 // with n live slots is cut into slices of whole 128-entry tiles; each CTA with a slice leaves a
 // partial softmax state (shift, sum, weighted values) in the workspace, and the CTA that arrives
 // last (a counter per cache that every CTA of the grid increments, a fence before every
@@ -52,8 +52,8 @@ constexpr float kRescaleGap = 16.f;     // raise the shift when a logit exceeds 
 template <int DH, int G>
 struct DecTc {
     static constexpr int NB = DH / 64;                       // 64-column (128-byte) boxes per row
-    static constexpr int NST = DH == 64 ? 2 : 1;             // stages of (khat, v) tiles
-    static constexpr int CTAS = DH == 64 ? 3 : 2;            // CTAs per SM the footprint allows
+    static constexpr int NST = 1;                            // stages of (khat, v) tiles
+    static constexpr int CTAS = DH == 64 ? 4 : 2;            // CTAs per SM the footprint allows
     static constexpr int COL_S = 0, COL_O = 16, TMEM_COLS = 32;
     static constexpr int SS = G * (DH + 2);                  // floats of one partial state
 };
@@ -676,9 +676,9 @@ cudaError_t decode_tc_g(const DecodeParams& p, cudaStream_t s) {
     }
 }
 
-// Footprints: DH = 64 three CTAs per SM, DH = 128 two (227 KB of shared memory per SM); the merge
+// Footprints: DH = 64 four CTAs per SM, DH = 128 two (227 KB of shared memory per SM); the merge
 // reuses the first stage for 3 x kDecodeSplitMax x G + 2 G floats.
-static_assert(3 * (sizeof(DecTcSmem<64, 8>) + 1024) <= 232448, "decode tiles: three CTAs per SM at d = 64");
+static_assert(4 * (sizeof(DecTcSmem<64, 8>) + 1024) <= 232448, "decode tiles: four CTAs per SM at d = 64");
 static_assert(2 * (sizeof(DecTcSmem<128, 8>) + 1024) <= 232448, "decode tiles: two CTAs per SM at d = 128");
 static_assert((3 * kDecodeSplitMax * 8 + 2 * 8) * 4 <= 16384, "the merge's scratch fits the first stage box");
 
