@@ -266,14 +266,14 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         if (e < G * half) {
             const int vecid = e / half, m = e % half;
             float cs, sn;
-            rope_cs_turns((double)p.pos_t, p.rf.f[m] * 0.15915494309189535, &cs, &sn);
+            rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
             s_q[vecid][2 * m] = qa[r] * cs - qb[r] * sn;
             s_q[vecid][2 * m + 1] = qb[r] * cs + qa[r] * sn;
         }
     }
     for (int m = tid; m < half; m += blockDim.x) {
         float cs, sn;
-        rope_cs_turns((double)p.pos_t, p.rf.f[m] * 0.15915494309189535, &cs, &sn);
+        rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
         const float x0 = s_kt[2 * m], x1 = s_kt[2 * m + 1];
         s_ktr[2 * m] = x0 * cs - x1 * sn;
         s_ktr[2 * m + 1] = x1 * cs + x0 * sn;
@@ -289,12 +289,10 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         for (int e = tid; e < G * DH; e += blockDim.x) s_q[e / DH][e % DH] *= s_qn[e / DH];
         __syncthreads();
     }
-    for (int h = warp; h < G; h += NW) {              // new token's own logits (its bias is 0)
+    if (tid < G) {
         float a = 0.f;
-        for (int x = lane; x < DH; x += 32) a = fmaf(s_q[h][x], s_ktr[x], a);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == 0) s_lt[h] = a * p.scale;
+        for (int x = 0; x < DH; ++x) a = fmaf(s_q[tid][x], s_ktr[x], a);
+        s_lt[tid] = a * p.scale;                      // new token's own bias is 0
     }
     const float rq_t = (variant & kVarNoQ) ? 1.f : softplus_f(aq_t);
     const float rk_t = softplus_f(ak_t);          // stored in the cache as is

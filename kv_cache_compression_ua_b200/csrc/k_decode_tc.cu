@@ -375,8 +375,9 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
             }
         }
         if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (t / NST) & 1, abort))) ok = false;
-        // ---- x_j = <khat_t, khat_j>, and khat_j rotated in place (16-byte chunks, swizzled)
-        float x = 0.f;
+        // ---- x_j = <khat_t, khat_j> (four partial sums: short dependency chains), and khat_j
+        // rotated in place (16-byte chunks, swizzled)
+        float xp[4] = {0.f, 0.f, 0.f, 0.f};
         const int par = t & 1;
         bool dense = true;
 #pragma unroll
@@ -395,9 +396,10 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
                     Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(ptr), xa);
                     const float4 k0 = *reinterpret_cast<const float4*>(&S.kt[bx * 64 + ch * 8]);
                     const float4 k1 = *reinterpret_cast<const float4*>(&S.kt[bx * 64 + ch * 8 + 4]);
-                    x = fmaf(k0.x, xa[0], x); x = fmaf(k0.y, xa[1], x); x = fmaf(k0.z, xa[2], x);
-                    x = fmaf(k0.w, xa[3], x); x = fmaf(k1.x, xa[4], x); x = fmaf(k1.y, xa[5], x);
-                    x = fmaf(k1.z, xa[6], x); x = fmaf(k1.w, xa[7], x);
+                    xp[0] = fmaf(k0.x, xa[0], xp[0]); xp[1] = fmaf(k0.y, xa[1], xp[1]);
+                    xp[2] = fmaf(k0.z, xa[2], xp[2]); xp[3] = fmaf(k0.w, xa[3], xp[3]);
+                    xp[0] = fmaf(k1.x, xa[4], xp[0]); xp[1] = fmaf(k1.y, xa[5], xp[1]);
+                    xp[2] = fmaf(k1.z, xa[6], xp[2]); xp[3] = fmaf(k1.w, xa[7], xp[3]);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int m = bx * 32 + ch * 4 + i;
@@ -422,9 +424,10 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
                     Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(ptr), xa);
                     const float4 k0 = *reinterpret_cast<const float4*>(&S.kt[bx * 64 + ch * 8]);
                     const float4 k1 = *reinterpret_cast<const float4*>(&S.kt[bx * 64 + ch * 8 + 4]);
-                    x = fmaf(k0.x, xa[0], x); x = fmaf(k0.y, xa[1], x); x = fmaf(k0.z, xa[2], x);
-                    x = fmaf(k0.w, xa[3], x); x = fmaf(k1.x, xa[4], x); x = fmaf(k1.y, xa[5], x);
-                    x = fmaf(k1.z, xa[6], x); x = fmaf(k1.w, xa[7], x);
+                    xp[0] = fmaf(k0.x, xa[0], xp[0]); xp[1] = fmaf(k0.y, xa[1], xp[1]);
+                    xp[2] = fmaf(k0.z, xa[2], xp[2]); xp[3] = fmaf(k0.w, xa[3], xp[3]);
+                    xp[0] = fmaf(k1.x, xa[4], xp[0]); xp[1] = fmaf(k1.y, xa[5], xp[1]);
+                    xp[2] = fmaf(k1.z, xa[6], xp[2]); xp[3] = fmaf(k1.w, xa[7], xp[3]);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         float cs, sn;
@@ -436,6 +439,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
                 }
             }
         }
+        const float x = (xp[0] + xp[1]) + (xp[2] + xp[3]);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         if (__syncthreads_or(!ok)) { ok = false; break; }
         // ---- S of the tile
