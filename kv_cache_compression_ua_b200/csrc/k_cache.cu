@@ -242,21 +242,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     }
     const float aq_t = p.a_q[unit], ak_t = p.a_k[unit];
     const float al = p.alpha[kvh], be = p.beta[kvh];
-    // the first pass of cache entries goes to L2 while the new token is formed (no registers
-    // held): a pruned cache of one pass then reads it from L2, not HBM, after the prologue
-    {
-        const int nn = min(max(n, 0), c.cap);
-        if (gl == 0 && gidx < nn) {
-            const size_t e = (base + gidx) * DH;
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(khat + e));
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(vc + e));
-            if ((gidx & 31) == 0) {
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(c.bias + base + gidx));
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(c.rk + base + gidx));
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(c.pos + base + gidx));
-            }
-        }
-    }
+
 
     // ---- new token: khat_t, RoPE(khat_t), v_t, RoPE(q_h), rates
     float ss = kx * kx;

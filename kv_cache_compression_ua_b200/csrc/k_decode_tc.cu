@@ -52,7 +52,6 @@ constexpr float kRescaleGap = 16.f;     // raise the shift when a logit exceeds 
 template <int DH, int G>
 struct DecTc {
     static constexpr int NB = DH / 64;                       // 64-column (128-byte) boxes per row
-    static constexpr int NST = 1;                            // stages of (khat, v) tiles
     static constexpr int CTAS = DH == 64 ? 4 : 2;            // CTAs per SM the footprint allows
     static constexpr int COL_S = 0, COL_O = 16, TMEM_COLS = 32;
     static constexpr int SS = G * (DH + 2);                  // floats of one partial state
@@ -65,7 +64,7 @@ struct DecTcSmem {
     // bf16 with the 128-byte swizzle.  The second product's M = 128 rows are the head dims in
     // 64-row atoms one box apart; when DH = 64 its upper atom reads the stage's khat box, whose
     // rows of the result are never read.
-    alignas(1024) uint8_t stage[C::NST][2 * C::NB][16384];
+    alignas(1024) uint8_t stage[1][2 * C::NB][16384];
     alignas(1024) uint8_t bq[16 * DH * 2];                   // no-swizzle K-major B of S
     alignas(128) uint8_t pt[2][kDecTile][16];                // P: MN-major no-swizzle, heads 0-7 | 8-15
     double gtf[DH / 2];                                       // RoPE frequencies / (2 pi)
@@ -83,7 +82,10 @@ struct DecTcSmem {
     float red[G][4];
     float red2[4];
     unsigned tflag[2];                                       // per tile parity: bit 0 abort, bit 1 raise the shift
-    uint64_t full[C::NST];
+    int scp[2][kDecTile];                                    // per tile parity: pos, bias, r_k of the entries
+    float scb[2][kDecTile];
+    float scr[2][kDecTile];
+    uint64_t full_k, full_v;                                 // khat and v of the tile landed
     uint64_t sfull, pfree;
     uint32_t tmem_base;
     int abort;
@@ -255,7 +257,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     k_decode_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_v, DecodeParams p) {
     using C = DecTc<DH, G>;
     using Sm = DecTcSmem<DH, G>;
-    constexpr int NB = C::NB, NST = C::NST;
+    constexpr int NB = C::NB;
     extern __shared__ uint8_t dsm_raw[];
     Sm& S = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const CacheView& c = p.c;
@@ -293,7 +295,8 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
 
     if (tid == 0) {
         S.abort = 0;
-        for (int s = 0; s < NST; ++s) mbar_init(&S.full[s], 1);
+        mbar_init(&S.full_k, 1);
+        mbar_init(&S.full_v, 1);
         mbar_init(&S.sfull, 1);
         mbar_init(&S.pfree, 1);
         fence_barrier_init();
@@ -303,26 +306,36 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         tmem_relinquish();
     }
     const bool leader = tid == 0;
-    auto issue_tile = [&](int tt) {
-        const int s = tt % NST;
+    // One stage.  A tile's keys are reloaded as soon as its first product has read them (mid
+    // tile), its values once the second product is done (at the start of the next tile), so both
+    // loads overlap the work of a tile instead of following it.
+    auto issue_k = [&](int tt) {
         const int row = (int)(base + lo + (size_t)tt * kDecTile);
-        mbar_expect_tx(&S.full[s], 2 * NB * 16384);
-        for (int bx = 0; bx < NB; ++bx) {
-            tma_load_2d(S.stage[s][bx], &tm_v, &S.full[s], 64 * bx, row);
-            tma_load_2d(S.stage[s][NB + bx], &tm_kh, &S.full[s], 64 * bx, row);
+        mbar_expect_tx(&S.full_k, NB * 16384);
+        for (int bx = 0; bx < NB; ++bx) tma_load_2d(S.stage[0][NB + bx], &tm_kh, &S.full_k, 64 * bx, row);
+    };
+    auto issue_v = [&](int tt) {
+        const int row = (int)(base + lo + (size_t)tt * kDecTile);
+        mbar_expect_tx(&S.full_v, NB * 16384);
+        for (int bx = 0; bx < NB; ++bx) tma_load_2d(S.stage[0][bx], &tm_v, &S.full_v, 64 * bx, row);
+    };
+    // a tile's scalars (pos, bias, r_k) go to shared memory by asynchronous copies, a tile ahead;
+    // each thread copies and later reads only its own entry's
+    auto load_scalars = [&](int tt) {
+        const int jj = lo + tt * kDecTile + tid, par = tt & 1;
+        if (jj < hi) {
+            cp_async4(&S.scp[par][tid], c.pos + base + jj);
+            cp_async4(&S.scb[par][tid], c.bias + base + jj);
+            cp_async4(&S.scr[par][tid], c.rk + base + jj);
         }
+        cp_async_commit();
     };
     __syncthreads();                                  // barriers initialised
-    if (leader)
-        for (int tt = 0; tt < NST && tt < ntiles; ++tt) issue_tile(tt);
-    // the first tile's scalars, loaded before the new token is formed
-    int pj_n = 0;
-    float bj_n = 0.f, rk_n = 0.f;
-    if (lo + tid < hi) {
-        pj_n = c.pos[base + lo + tid];
-        bj_n = c.bias[base + lo + tid];
-        rk_n = c.rk[base + lo + tid];
+    if (leader) {
+        issue_k(0);
+        issue_v(0);
     }
+    load_scalars(0);
     tc_fence_before();
     new_token<DH, G>(S, p, unit, b, kvh);             // ends with __syncthreads
     tc_fence_after();
@@ -346,7 +359,8 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     for (int idx = tid; idx < kDecTile * 4; idx += blockDim.x) reinterpret_cast<uint32_t*>(S.pt[1])[idx] = 0u;
     if (tid < G) S.shift[tid] = S.own[tid];
     if (tid == 0) S.tflag[0] = S.tflag[1] = 0u;
-    tile_density<DH, G>(S, 0, pj_n, lo + tid, lo + tid < hi, warp, lane);
+    cp_async_wait_all();
+    tile_density<DH, G>(S, 0, S.scp[0][tid], lo + tid, lo + tid < hi, warp, lane);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
 
@@ -361,20 +375,14 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     for (int h = 0; h < G; ++h) lsum[h] = 0.f;
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
-        const int s = t % NST;
         const int j = lo + t * kDecTile + tid;
         const bool valid = j < hi;
-        const int pj = pj_n;
-        const float bj = bj_n, rkj = rk_n;
-        if (t + 1 < ntiles) {                         // the next tile's scalars, a tile ahead
-            const int jn = j + kDecTile;
-            if (jn < hi) {
-                pj_n = c.pos[base + jn];
-                bj_n = c.bias[base + jn];
-                rk_n = c.rk[base + jn];
-            }
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (t / NST) & 1, abort))) ok = false;
+        const int pj = S.scp[t & 1][tid];
+        const float bj = S.scb[t & 1][tid], rkj = S.scr[t & 1][tid];
+        if (t + 1 < ntiles) load_scalars(t + 1);
+        // values of this tile: the previous tile's second product must be done with the buffer
+        if (tid == 96 && t >= 1 && mbar_wait(&S.pfree, (t - 1) & 1, abort)) issue_v(t);
+        if (!__all_sync(0xffffffffu, mbar_wait(&S.full_k, t & 1, abort))) ok = false;
         // ---- x_j = <khat_t, khat_j> (four partial sums: short dependency chains), and khat_j
         // rotated in place (16-byte chunks, swizzled)
         float xp[4] = {0.f, 0.f, 0.f, 0.f};
@@ -391,7 +399,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
             for (int bx = 0; bx < NB; ++bx) {
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    uint8_t* ptr = S.stage[s][NB + bx] + (uint32_t)tid * 128u + ((uint32_t)(ch ^ (tid & 7)) << 4);
+                    uint8_t* ptr = S.stage[0][NB + bx] + (uint32_t)tid * 128u + ((uint32_t)(ch ^ (tid & 7)) << 4);
                     float xa[8], xb[8];
                     Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(ptr), xa);
                     const float4 k0 = *reinterpret_cast<const float4*>(&S.kt[bx * 64 + ch * 8]);
@@ -419,7 +427,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
             for (int bx = 0; bx < NB; ++bx) {
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    uint8_t* ptr = S.stage[s][NB + bx] + (uint32_t)tid * 128u + ((uint32_t)(ch ^ (tid & 7)) << 4);
+                    uint8_t* ptr = S.stage[0][NB + bx] + (uint32_t)tid * 128u + ((uint32_t)(ch ^ (tid & 7)) << 4);
                     float xa[8], xb[8];
                     Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(ptr), xa);
                     const float4 k0 = *reinterpret_cast<const float4*>(&S.kt[bx * 64 + ch * 8]);
@@ -447,7 +455,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < DH / 16; ++kk) {
-                const uint64_t a = smem_desc(smem_u32(S.stage[s][NB + (kk >> 2)]) + (uint32_t)(kk & 3) * 32u, 16,
+                const uint64_t a = smem_desc(smem_u32(S.stage[0][NB + (kk >> 2)]) + (uint32_t)(kk & 3) * 32u, 16,
                                              1024, kSwizzle128B);
                 const uint64_t bd = smem_desc(smem_u32(S.bq) + (uint32_t)kk * 256u, 128, DH * 16, kSwizzleNone);
                 umma_f16(tmem + C::COL_S, a, bd, ID1, kk > 0 ? 1u : 0u);
@@ -467,6 +475,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         if (p.evict_bits && lane == 0 && wj0 < hi) p.evict_bits[(size_t)unit * words + (wj0 >> 5)] = ev;
         if (!__all_sync(0xffffffffu, mbar_wait(&S.sfull, t & 1, abort))) ok = false;
         tc_fence_after();
+        if (leader && ok && t + 1 < ntiles) issue_k(t + 1);      // the first product has read the keys
         float xs[2 * G <= 8 ? 8 : 16];
         if (2 * G <= 8) tmem_ld8(tmem + lane_base + C::COL_S, xs);
         else tmem_ld16(tmem + lane_base + C::COL_S, xs);
@@ -492,9 +501,12 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         if (tid == 0) S.tflag[(t + 1) & 1] = 0u;      // the next tile's word (its writers come after
                                                       // this tile's last barrier)
         // the next tile's contiguity and base angles (read after this tile's last barrier)
-        if (t + 1 < ntiles) tile_density<DH, G>(S, (t + 1) & 1, pj_n, j + kDecTile, j + kDecTile < hi, warp, lane);
+        if (t + 1 < ntiles) {
+            cp_async_wait_all();
+            tile_density<DH, G>(S, (t + 1) & 1, S.scp[(t + 1) & 1][tid], j + kDecTile, j + kDecTile < hi, warp,
+                                lane);
+        }
         tc_fence_after();
-        if (NST > 1 && leader && t >= 1 && t - 1 + NST < ntiles) issue_tile(t - 1 + NST);
         // ---- shift: raised (and the accumulated values rescaled) when a logit of the tile
         // exceeds it by more than kRescaleGap (rare: the per-head maxima are formed only then)
         float fac[G];
@@ -547,20 +559,16 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         if (any && tid < G) S.shift[tid] = nsh[tid];
         // ---- O^T += V^T P
         if (leader) {
+            if (!mbar_wait(&S.full_v, t & 1, abort)) ok = false;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kDecTile / 16; ++kk) {
-                const uint64_t a = smem_desc(smem_u32(S.stage[s][0]) + (uint32_t)kk * 2048u, 16384, 1024,
+                const uint64_t a = smem_desc(smem_u32(S.stage[0][0]) + (uint32_t)kk * 2048u, 16384, 1024,
                                              kSwizzle128B);
                 const uint64_t bd = smem_desc(smem_u32(S.pt[0]) + (uint32_t)kk * 256u, 128, 2048, kSwizzleNone);
                 umma_f16(tmem + C::COL_O, a, bd, ID2, (t > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&S.pfree);
-        }
-        // single stage: this tile's stage is refilled once its second product is done
-        if (NST == 1 && t + 1 < ntiles) {
-            if (!__all_sync(0xffffffffu, mbar_wait(&S.pfree, t & 1, abort))) ok = false;
-            if (leader && ok) issue_tile(t + 1);
         }
     }
     // ---- the slice's partial state
