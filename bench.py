@@ -416,6 +416,8 @@ def bench_decode(args, peaks, peaks_kind):
     pages' 16k average share of the keys, 1/21.38 at p = 0.15)."""
     from kv_cache_compression_ua_b200 import ua
     w = I.WORKLOADS["decode_1b"]
+    if getattr(args, "decode_batch", None):
+        w = w.resized(B=args.decode_batch)         # fewer sequences (profiling captures)
     steps = I.DECODE_STEPS
     T0 = w.T
     x = I.make_prefill_inputs_torch(w, "cuda", names=["k", "v", "a_q", "a_k", "alpha", "beta"])
@@ -729,6 +731,8 @@ def main():
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-more", action="store_true", help="skip the 16k and chunked-pruned prefill lines")
     ap.add_argument("--decode-p", type=float, default=None, help="run the decode section at this p only")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="sequences of the decode section (default: the workload's 32; smaller for profiling)")
     ap.add_argument("--fwdbwd-batch", type=int, default=4,
                     help="batch of the 3B forward+backward line (4 = the workload; smaller for profiling)")
     args = ap.parse_args()

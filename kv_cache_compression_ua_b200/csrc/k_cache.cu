@@ -129,6 +129,8 @@ __global__ void __launch_bounds__(256) k_cache_compact(CompactParams p) {
     const int unit = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int grp = lane / L::LPE, gl = lane % L::LPE;
+    grid_dep_wait();
+    grid_dep_release();
     int n = c.n_kept[unit];
     if (n < 0 || n > c.cap) {                 // corrupt count: never read past the cache
         if (threadIdx.x == 0) raise_status(UA_ERR_CAPACITY);
@@ -187,8 +189,9 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     using L = EntryLayout<TC, DH>;
     constexpr int VEC = L::VEC, LPE = L::LPE, EPB = L::EPB, NW = L::NW;
     constexpr int half = DH / 2;
-    __shared__ float s_kt[DH], s_ktr[DH], s_vt[DH], s_q[G][DH], s_lt[G], s_g[G * DH], s_qn[G];
+    __shared__ float s_kt[DH], s_ktr[DH], s_vt[DH], s_q[G][DH], s_g[G * DH], s_qn[G];
     __shared__ float s_red[NW];
+    __shared__ double s_rf[DH / 2];
     __shared__ int s_wcnt[NW];
     extern __shared__ float dsm[];
     const CacheView& c = p.c;
@@ -206,11 +209,31 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     TC* khat = static_cast<TC*>(c.khat);
     TC* vc = static_cast<TC*>(c.v);
 
-    // ---- Every load that depends on no other goes out first (the live count, the new token,
-    // its gate and the rates), so a step over a pruned, tiny cache does not pay a chain of
-    // memory round trips before its arithmetic.  (Prefetching the first pass of cache entries
-    // as well was measured slower: the registers it holds cost occupancy.)
+    grid_dep_wait();
+    grid_dep_release();
+    // ---- Every load that depends on no other goes out first: the live count, the first pass
+    // of cache entries, the new token, its gate and the rates, so a step over a pruned, tiny
+    // cache pays one memory round trip before its arithmetic.  The first pass is read within
+    // the capacity whatever the count (which is still in flight); entries past the count are
+    // masked out below.
     int n = c.n_kept[unit];
+    // Software pipeline: the entries of the next pass are loaded before this pass is processed,
+    // so two passes of loads are in flight.  Safe with the in-place compaction: a survivor of
+    // this pass only ever moves to a slot at or below its own, never into the next pass.
+    uint4 na = make_uint4(0, 0, 0, 0), nv = na;
+    float nbj = 0.f, nrk = 0.f;
+    int npj = 0;
+    auto load_entry = [&](int jj, int lim) {
+        if (jj < lim) {
+            const size_t e = (base + jj) * DH + gl * VEC;
+            na = *reinterpret_cast<const uint4*>(khat + e);
+            nv = *reinterpret_cast<const uint4*>(vc + e);
+            nbj = c.bias[base + jj];
+            nrk = c.rk[base + jj];
+            npj = c.pos[base + jj];
+        }
+    };
+    load_entry(gidx, c.cap);
     // the step's key and value: head kvh / rep of [B, Hkv / rep, d]
     const size_t tok = (size_t)b * (c.Hkv / c.rep) + kvh / c.rep;
     const TC* kin = static_cast<const TC*>(p.k) + tok * DH;
@@ -250,6 +273,10 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) s_red[warp] = ss;
     for (int w = tid; w < words; w += blockDim.x) s_ev[w] = 0u;
+    // the RoPE frequencies go to shared memory once, a few per warp (a kernel-parameter array
+    // read at a different index by each lane serialises those reads)
+    static_assert(half % NW == 0, "frequencies split evenly over the warps");
+    if (lane < half / NW) s_rf[warp * (half / NW) + lane] = p.rf.f[warp * (half / NW) + lane];
     __syncthreads();
     float tot_ss = 0.f;
 #pragma unroll
@@ -267,14 +294,14 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         if (e < G * half) {
             const int vecid = e / half, m = e % half;
             float cs, sn;
-            rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
+            rope_cs((double)p.pos_t, s_rf[m], &cs, &sn);
             s_q[vecid][2 * m] = qa[r] * cs - qb[r] * sn;
             s_q[vecid][2 * m + 1] = qb[r] * cs + qa[r] * sn;
         }
     }
     for (int m = tid; m < half; m += blockDim.x) {
         float cs, sn;
-        rope_cs((double)p.pos_t, p.rf.f[m], &cs, &sn);
+        rope_cs((double)p.pos_t, s_rf[m], &cs, &sn);
         const float x0 = s_kt[2 * m], x1 = s_kt[2 * m + 1];
         s_ktr[2 * m] = x0 * cs - x1 * sn;
         s_ktr[2 * m + 1] = x1 * cs + x0 * sn;
@@ -290,11 +317,6 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         for (int e = tid; e < G * DH; e += blockDim.x) s_q[e / DH][e % DH] *= s_qn[e / DH];
         __syncthreads();
     }
-    if (tid < G) {
-        float a = 0.f;
-        for (int x = 0; x < DH; ++x) a = fmaf(s_q[tid][x], s_ktr[x], a);
-        s_lt[tid] = a * p.scale;                      // new token's own bias is 0
-    }
     const float rq_t = (variant & kVarNoQ) ? 1.f : softplus_f(aq_t);
     const float rk_t = softplus_f(ak_t);          // stored in the cache as is
 
@@ -305,7 +327,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     for (int e = 0; e < VEC; ++e) kq[e] = s_kt[gl * VEC + e];
     double gt[VEC / 2];                               // this lane's RoPE frequencies / (2 pi)
 #pragma unroll
-    for (int i = 0; i < VEC / 2; ++i) gt[i] = p.rf.f[gl * (VEC / 2) + i] * 0.15915494309189535;
+    for (int i = 0; i < VEC / 2; ++i) gt[i] = s_rf[gl * (VEC / 2) + i] * 0.15915494309189535;
     float m_h[G], l_h[G], acc[G][VEC];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -321,23 +343,6 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     }
     int out = 0;
     const bool multi_pass = n > 4 * EPB;   // block-uniform
-    // Software pipeline: the entries of the next pass are loaded before this pass is processed,
-    // so two passes of loads are in flight.  Safe with the in-place compaction: a survivor of
-    // this pass only ever moves to a slot at or below its own, never into the next pass.
-    uint4 na = make_uint4(0, 0, 0, 0), nv = na;
-    float nbj = 0.f, nrk = 0.f;
-    int npj = 0;
-    auto load_entry = [&](int jj) {
-        if (jj < n) {
-            const size_t e = (base + jj) * DH + gl * VEC;
-            na = *reinterpret_cast<const uint4*>(khat + e);
-            nv = *reinterpret_cast<const uint4*>(vc + e);
-            nbj = c.bias[base + jj];
-            nrk = c.rk[base + jj];
-            npj = c.pos[base + jj];
-        }
-    };
-    load_entry(gidx);
     for (int c0 = 0; c0 < n; c0 += EPB) {
         const int j = c0 + gidx;
         const bool valid = j < n;
@@ -362,7 +367,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         const uint4 ra = na, rv = nv;
         const float bj = nbj, rkj = nrk;
         const int pj = npj;
-        load_entry(j + EPB);
+        load_entry(j + EPB, n);
         float xa[VEC], xb[VEC], xv[VEC];
         Vec16<TC>::unpack(ra, xa);
         Vec16<TC>::unpack(rv, xv);
@@ -433,25 +438,60 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) s_acc[((size_t)gidx * G + h) * DH + gl * VEC + e] = acc[h][e];
+        for (int e = 0; e < VEC; e += 4)
+            *reinterpret_cast<float4*>(s_acc + ((size_t)gidx * G + h) * DH + gl * VEC + e) =
+                make_float4(acc[h][e], acc[h][e + 1], acc[h][e + 2], acc[h][e + 3]);
     __syncthreads();
     const int qn = min(EPB, n);                       // entry groups that saw an entry (short caches: few)
+    // Warp h merges head h's states: the common maximum with the new token's own logit, the
+    // weight of each group's state (left in s_m) and of the new token, and 1 / (the total sum).
+    static_assert(EPB <= 32, "a lane per entry group in the merge");
+    __shared__ float s_wt[G], s_inv[G];
+    if (warp < G) {
+        const int h = warp;
+        // the new token's own logit (its bias is 0)
+        float lt = 0.f;
+#pragma unroll
+        for (int x = lane; x < DH; x += 32) lt = fmaf(s_q[h][x], s_ktr[x], lt);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
+        lt *= p.scale;
+        const float mq = lane < qn ? s_m[lane * G + h] : -INFINITY;
+        float M = fmaxf(mq, lt);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float w = lane < qn ? expf(mq - M) : 0.f;
+        float L = lane < qn ? s_l[lane * G + h] * w : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        const float wt = expf(lt - M);
+        __syncwarp();
+        if (lane < qn) s_m[lane * G + h] = w;
+        if (lane == 0) {
+            s_wt[h] = wt;
+            s_inv[h] = 1.f / (L + wt);
+        }
+    }
+    __syncthreads();
     TC* oout = static_cast<TC*>(p.o) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
 #pragma unroll
     for (int r = 0; r < GE; ++r) {
         const int e = tid + 256 * r;
         if (e >= G * DH) break;
         const int h = e / DH, x = e % DH;
-        float M = s_lt[h];
-        for (int q = 0; q < qn; ++q) M = fmaxf(M, s_m[q * G + h]);
-        float Ls = expf(s_lt[h] - M);
-        float A = Ls * s_vt[x];
-        for (int q = 0; q < qn; ++q) {
-            const float w = expf(s_m[q * G + h] - M);
-            Ls = fmaf(s_l[q * G + h], w, Ls);
-            A = fmaf(s_acc[((size_t)q * G + h) * DH + x], w, A);
+        // four partial sums over the groups' states (independent loads and adds)
+        const float* ac = s_acc + (size_t)h * DH + x;     // group q at + q * G * DH
+        const float* wq = s_m + h;                         // group q at + q * G
+        float A0 = s_wt[h] * s_vt[x], A1 = 0.f, A2 = 0.f, A3 = 0.f;
+        int q = 0;
+        for (; q + 4 <= qn; q += 4) {
+            A0 = fmaf(ac[(size_t)q * G * DH], wq[q * G], A0);
+            A1 = fmaf(ac[(size_t)(q + 1) * G * DH], wq[(q + 1) * G], A1);
+            A2 = fmaf(ac[(size_t)(q + 2) * G * DH], wq[(q + 2) * G], A2);
+            A3 = fmaf(ac[(size_t)(q + 3) * G * DH], wq[(q + 3) * G], A3);
         }
-        Elem<TC>::st(oout + e, A / Ls * sigmoid_f(s_g[e]));
+        for (; q < qn; ++q) A0 = fmaf(ac[(size_t)q * G * DH], wq[q * G], A0);
+        Elem<TC>::st(oout + e, ((A0 + A1) + (A2 + A3)) * s_inv[h] * sigmoid_f(s_g[e]));
     }
     // ---- eviction bits, append the new token
     if (p.evict_bits)
@@ -510,6 +550,8 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
     TC* khat = static_cast<TC*>(c.khat);
     TC* vc = static_cast<TC*>(c.v);
 
+    grid_dep_wait();
+    grid_dep_release();
     int n = c.n_kept[unit];
     if (n < 0 || n > c.cap) {                 // corrupt count: never read past the cache
         if (tid == 0 && sl == 0) raise_status(UA_ERR_CAPACITY);
@@ -750,13 +792,12 @@ cudaError_t launch_cache_compact(const CompactParams& p, bool bf16, cudaStream_t
     dim3 grid(p.c.B * p.c.Hkv);
     UA_PROFILE("k_cache_compact", s);
     if (bf16) {
-        if (p.c.d == 64) k_cache_compact<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
-        else k_cache_compact<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
+        return p.c.d == 64 ? launch_dependent(k_cache_compact<__nv_bfloat16, 64>, grid, dim3(256), 0, s, p)
+                           : launch_dependent(k_cache_compact<__nv_bfloat16, 128>, grid, dim3(256), 0, s, p);
     } else {
-        if (p.c.d == 64) k_cache_compact<float, 64><<<grid, 256, 0, s>>>(p);
-        else k_cache_compact<float, 128><<<grid, 256, 0, s>>>(p);
+        return p.c.d == 64 ? launch_dependent(k_cache_compact<float, 64>, grid, dim3(256), 0, s, p)
+                           : launch_dependent(k_cache_compact<float, 128>, grid, dim3(256), 0, s, p);
     }
-    return cudaGetLastError();
 }
 
 template <typename TC, int DH, int G, bool DEFER, bool VAR>
@@ -767,8 +808,7 @@ static cudaError_t decode_launch(const DecodeParams& p, size_t smem, cudaStream_
         if (e != cudaSuccess) return e;
     }
     UA_PROFILE("k_decode", s);
-    k_decode<TC, DH, G, DEFER, VAR><<<p.c.B * p.c.Hkv, 256, smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_dependent(k_decode<TC, DH, G, DEFER, VAR>, dim3(p.c.B * p.c.Hkv), dim3(256), smem, s, p);
 }
 
 template <typename TC, int DH, int G>
@@ -807,8 +847,7 @@ static cudaError_t decode_split_inst(const DecodeParams& p, cudaStream_t s) {
         if (e != cudaSuccess) return e;
     }
     UA_PROFILE("k_decode_split", s);
-    kern<<<grid, 256, smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_dependent(kern, grid, dim3(256), smem, s, p);
 }
 
 template <typename TC, int DH>

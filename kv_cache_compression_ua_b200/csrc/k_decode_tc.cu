@@ -267,6 +267,8 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     const size_t base = (size_t)unit * c.cap;
     const int words = (c.cap + 31) / 32;
 
+    grid_dep_wait();
+    grid_dep_release();
     int n = c.n_kept[unit];
     if (n < 0 || n > c.cap) {                 // corrupt count: never read past the cache
         if (tid == 0 && sl == 0) raise_status(UA_ERR_CAPACITY);
@@ -672,8 +674,8 @@ cudaError_t decode_tc_inst(const DecodeParams& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     UA_PROFILE("k_decode_tc", s);
     const int units = p.c.B * p.c.Hkv;
-    k_decode_tc<DH, G><<<dim3(decode_tc_slices(units, p.c.cap, DecTc<DH, G>::CTAS), units), 128, smem, s>>>(mk, mv, p);
-    return cudaGetLastError();
+    return launch_dependent(k_decode_tc<DH, G>, dim3(decode_tc_slices(units, p.c.cap, DecTc<DH, G>::CTAS), units),
+                            dim3(128), smem, s, mk, mv, p);
 }
 
 template <int DH>

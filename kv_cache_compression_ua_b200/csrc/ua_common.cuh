@@ -19,6 +19,17 @@ __device__ __forceinline__ void raise_status(int code) { atomicCAS(&g_status, 0,
 // UA_WAIT_LIMIT_DEFAULT_NS).  Defined in ua_api.cu.
 extern __device__ unsigned long long g_wait_limit_ns;
 
+// ------------------------------------------------------------------ dependent launches
+// Kernels of the decode step are launched with programmatic stream serialisation (one decode
+// step after another, in a CUDA graph or not): the next kernel's blocks may be scheduled while
+// this one finishes.  grid_dep_wait() blocks until every kernel the grid depends on has
+// completed and its writes are visible -- each kernel calls it before its first access to
+// global memory; it returns at once for a grid launched without the attribute.
+// grid_dep_release() lets the next grid be scheduled (its blocks still wait for this grid's
+// completion before touching memory).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ scalar math
 // softplus(x) = log(1 + e^x) in its overflow-free form.
 __device__ __forceinline__ float softplus_f(float x) {

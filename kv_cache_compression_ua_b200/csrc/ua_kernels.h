@@ -5,9 +5,30 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "ua_common.cuh"
 
 namespace ua {
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled before the
+// previous kernel on the stream has finished; it must call grid_dep_wait() before touching
+// global memory (see ua_common.cuh).
+template <typename... Args, typename... Act>
+cudaError_t launch_dependent(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Act&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
+}
 
 // Token preparation: normalised keys, RoPE'd queries/keys, per-token rates.
 struct PrepParams {
