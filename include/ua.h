@@ -305,8 +305,11 @@ ua_status ua_decode_step(const ua_cache* cache, int H, const void* q, const void
  * leaves a partial softmax state in the workspace; the last one to finish merges them with the
  * new token, gates, writes o and appends the token at slot n.  evict_bits and kept_idx follow the
  * deferred-compaction rules of ua_decode_step; evicted pairs stay until ua_cache_compact.
- * ws: device workspace of ua_decode_workspace_size bytes (256-byte aligned), scratch only; calls
- * that share a workspace must not overlap on the GPU.  A short cache (n <= 512) takes one slice.
+ * ws: device workspace of ua_decode_workspace_size bytes (256-byte aligned).  Zero it once before
+ * its first use (and again after using it for anything else): its first 4 x B x Hkv bytes are
+ * per-cache arrival counters, which every step leaves zero, so consecutive steps need no memset
+ * between their kernels (a counter found already at the grid's size raises UA_ERR_INVALID_ARG in
+ * the device status).  Calls that share a workspace must not overlap on the GPU.  A short cache (n <= 512) takes one slice.
  * bf16 caches run on the tensor cores: per 128-entry tile one tcgen05 product gives every
  * entry's similarity and G logits (the new key and the rotated queries enter as bf16 high parts
  * plus residuals), a thread per entry turns them into the decay, the bias, the eviction and the

@@ -729,7 +729,11 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
     }
     __threadfence();                                   // the state, biases and bits before the arrival
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(p.split_cnt + unit, 1u) == gridDim.x - 1;
+    if (tid == 0) {
+        const unsigned old = atomicAdd(p.split_cnt + unit, 1u);
+        if (old >= gridDim.x) raise_status(UA_ERR_INVALID_ARG);   // the workspace was not zeroed
+        s_last = old == gridDim.x - 1;
+    }
     __syncthreads();
     if (!s_last) return;
     __threadfence();

@@ -92,46 +92,88 @@ struct DecTcSmem {
     int last;
 };
 
-// New token of the cache: khat_t, RoPE(khat_t), v_t, RoPE(q_h) (query norm applied) and the own
-// logits, into shared memory.  All 128 threads; ends with a barrier.
+// The new token's inputs, loaded into registers at the kernel's start (the loads go out before
+// anything waits): element tid of k_t and v_t, the two components of this thread's query pairs
+// (item e = tid + 128 r is pair m = e % (DH/2) of head e / (DH/2)), and the rates.
 template <int DH, int G>
-__device__ void new_token(DecTcSmem<DH, G>& S, const DecodeParams& p, int unit, int b, int kvh) {
+struct TokIn {
+    static constexpr int QI = (G * (DH / 2) + 127) / 128;
+    float kx, vx;
+    float qa[QI], qb[QI];
+    float aq, ak, al, be;
+};
+
+template <int DH, int G>
+__device__ __forceinline__ void load_token(TokIn<DH, G>& t, const DecodeParams& p, int unit, int b, int kvh) {
     constexpr int half = DH / 2;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x;
     const size_t tok = (size_t)b * (p.c.Hkv / p.c.rep) + kvh / p.c.rep;   // head kvh / rep of the step's k, v
     const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(p.k) + tok * DH;
     const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(p.v) + tok * DH;
     const __nv_bfloat16* qin = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
-    float kx = 0.f;
+    t.kx = t.vx = 0.f;
     if (tid < DH) {
-        kx = __bfloat162float(kin[tid]);
-        S.vt[tid] = __bfloat162float(vin[tid]);
+        t.kx = __bfloat162float(kin[tid]);
+        t.vx = __bfloat162float(vin[tid]);
     }
-    float ss = kx * kx;
+#pragma unroll
+    for (int r = 0; r < TokIn<DH, G>::QI; ++r) {
+        const int e = tid + 128 * r;
+        t.qa[r] = t.qb[r] = 0.f;
+        if (e < G * half) {
+            const int h = e / half, m = e % half;
+            t.qa[r] = __bfloat162float(qin[h * DH + m]);
+            t.qb[r] = __bfloat162float(qin[h * DH + m + half]);
+        }
+    }
+    t.aq = p.a_q[unit];
+    t.ak = p.a_k[unit];
+    t.al = p.alpha[kvh];
+    t.be = p.beta[kvh];
+}
+
+// New token of the cache: khat_t, RoPE(khat_t), v_t, RoPE(q_h) (query norm applied) and the own
+// logits, into shared memory, from the preloaded inputs.  All 128 threads; ends with a barrier.
+template <int DH, int G>
+__device__ void new_token(DecTcSmem<DH, G>& S, const DecodeParams& p, const TokIn<DH, G>& tk) {
+    constexpr int half = DH / 2;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid < DH) S.vt[tid] = tk.vx;
+    float ss = tk.kx * tk.kx;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) S.red2[warp] = ss;
-    for (int m = tid; m < half; m += blockDim.x) {
-        S.gtf[m] = p.rf.f[m] * 0.15915494309189535;
-        S.ff[m] = (float)p.rf.f[m];
+    // the RoPE frequencies, a quarter per warp (a kernel-parameter array read at a different
+    // index by each lane serialises those reads)
+    static_assert(half % 4 == 0, "frequencies split over the four warps");
+    if (lane < half / 4) {
+        const int m = warp * (half / 4) + lane;
+        const double f = p.rf.f[m];
+        S.gtf[m] = f * 0.15915494309189535;
+        S.ff[m] = (float)f;
     }
     __syncthreads();
     const float den = fmaxf(sqrtf(S.red2[0] + S.red2[1] + S.red2[2] + S.red2[3]), 1e-12f);
-    if (tid < DH) S.kt[il_index(tid, half)] = kx / den;
+    if (tid < DH) S.kt[il_index(tid, half)] = tk.kx / den;
     __syncthreads();
-    for (int e = tid; e < (G + 1) * half; e += blockDim.x) {
-        const int h = e / half, m = e % half;
-        float cs, sn;
-        rope_cs_turns((double)p.pos_t, S.gtf[m], &cs, &sn);
-        if (h < G) {
-            const float qa = __bfloat162float(qin[h * DH + m]), qb = __bfloat162float(qin[h * DH + m + half]);
-            S.q[h][2 * m] = qa * cs - qb * sn;
-            S.q[h][2 * m + 1] = qb * cs + qa * sn;
-        } else {
-            const float x0 = S.kt[2 * m], x1 = S.kt[2 * m + 1];
-            S.ktr[2 * m] = x0 * cs - x1 * sn;
-            S.ktr[2 * m + 1] = x1 * cs + x0 * sn;
+    const double pt = (double)p.pos_t;
+#pragma unroll
+    for (int r = 0; r < TokIn<DH, G>::QI; ++r) {
+        const int e = tid + 128 * r;
+        if (e < G * half) {
+            const int h = e / half, m = e % half;
+            float cs, sn;
+            rope_cs_turns(pt, S.gtf[m], &cs, &sn);
+            S.q[h][2 * m] = tk.qa[r] * cs - tk.qb[r] * sn;
+            S.q[h][2 * m + 1] = tk.qb[r] * cs + tk.qa[r] * sn;
         }
+    }
+    for (int m = tid; m < half; m += blockDim.x) {
+        float cs, sn;
+        rope_cs_turns(pt, S.gtf[m], &cs, &sn);
+        const float x0 = S.kt[2 * m], x1 = S.kt[2 * m + 1];
+        S.ktr[2 * m] = x0 * cs - x1 * sn;
+        S.ktr[2 * m + 1] = x1 * cs + x0 * sn;
     }
     __syncthreads();
     if (p.variant & kVarQNorm) {                     // query RMS norm (RoPE keeps the norm)
@@ -156,56 +198,81 @@ __device__ void new_token(DecTcSmem<DH, G>& S, const DecodeParams& p, int unit, 
     __syncthreads();
 }
 
-// The last CTA of a cache: merge the partial states with the new token, gate, write o, clear
-// the eviction words past the live pairs and append the token.  The states' shifts and sums are
-// gathered into shared memory in one round of loads (the stage buffers, idle by now), so the
-// merge costs a few memory round trips, not one per state.
+// The last CTA of a cache: merge the partial states of the nsl slices that walked pairs with the
+// new token, gate, write o, clear the eviction words past the live pairs and append the token.
+// One round of loads brings every slice's shift and sum (and the gate); a warp per head forms
+// the common shift, the weights and the normaliser; the weighted values are then read once.
 template <int DH, int G>
-__device__ void merge_append(DecTcSmem<DH, G>& S, const DecodeParams& p, int unit, int b, int kvh, int n) {
+__device__ void merge_append(DecTcSmem<DH, G>& S, const DecodeParams& p, const TokIn<DH, G>& tk, int unit, int b,
+                             int kvh, int n, int nsl) {
     using C = DecTc<DH, G>;
-    const int tid = threadIdx.x;
+    constexpr int GE = (G * DH + 127) / 128;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const CacheView& c = p.c;
     const int words = (c.cap + 31) / 32;
     const size_t base = (size_t)unit * c.cap;
     const __nv_bfloat16* gin = static_cast<const __nv_bfloat16*>(p.g) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     __nv_bfloat16* oout = static_cast<__nv_bfloat16*>(p.o) + ((size_t)b * p.H + (size_t)kvh * G) * DH;
     const float* st0 = p.split_state + (size_t)unit * kDecodeSplitMax * C::SS;
-    const int nst = gridDim.x;
-    float* s_m = reinterpret_cast<float*>(S.stage[0][0]);          // [nst][G] shifts (-inf: empty)
-    float* s_l = s_m + kDecodeSplitMax * G;                          // [nst][G] sums
-    float* s_w = s_l + kDecodeSplitMax * G;                          // [nst][G] merge weights
-    float* s_M = s_w + kDecodeSplitMax * G;                          // [G] merged shift
-    float* s_L = s_M + G;                                            // [G] merged sum
-    for (int e = tid; e < nst * G; e += blockDim.x) {
-        const int q = e / G, h = e % G;
-        const float lq = __ldcg(st0 + (size_t)q * C::SS + G + h);
-        s_m[e] = lq > 0.f ? __ldcg(st0 + (size_t)q * C::SS + h) : -INFINITY;
-        s_l[e] = lq > 0.f ? lq : 0.f;
+    float* s_ml = reinterpret_cast<float*>(S.stage[0][0]);         // [nsl][2G]: shifts, sums
+    float* s_w = s_ml + kDecodeSplitMax * 2 * G;                     // [nsl][G] merge weights
+    float* s_wt = s_w + kDecodeSplitMax * G;                         // [G] weight of the new token
+    float* s_inv = s_wt + G;                                         // [G] 1 / normaliser
+    for (int e = tid; e < nsl * 2 * G; e += blockDim.x)
+        s_ml[e] = __ldcg(st0 + (size_t)(e / (2 * G)) * C::SS + e % (2 * G));
+    float gv[GE];
+#pragma unroll
+    for (int r = 0; r < GE; ++r) {
+        const int e = tid + 128 * r;
+        gv[r] = e < G * DH ? __bfloat162float(gin[e]) : 0.f;
     }
     __syncthreads();
-    if (tid < G) {
-        float M = S.own[tid];
-        for (int q = 0; q < nst; ++q) M = fmaxf(M, s_m[q * G + tid]);
-        s_M[tid] = M;
-    }
-    __syncthreads();
-    for (int e = tid; e < nst * G; e += blockDim.x) s_w[e] = s_l[e] > 0.f ? expf(s_m[e] - s_M[e % G]) : 0.f;
-    __syncthreads();
-    if (tid < G) {
-        float Ls = expf(S.own[tid] - s_M[tid]);
-        for (int q = 0; q < nst; ++q) Ls = fmaf(s_l[q * G + tid], s_w[q * G + tid], Ls);
-        s_L[tid] = Ls;
-    }
-    __syncthreads();
-    for (int e = tid; e < G * DH; e += blockDim.x) {
-        const int h = e / DH, x = e % DH;
-        float A = expf(S.own[h] - s_M[h]) * S.vt[x];
-#pragma unroll 8
-        for (int q = 0; q < nst; ++q) {
-            const float w = s_w[q * G + h];
-            if (w != 0.f) A = fmaf(__ldcg(st0 + (size_t)q * C::SS + 2 * G + e), w, A);
+    for (int h = warp; h < G; h += 4) {
+        float mq[2], lq[2];
+        float M = S.own[h];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int q = lane + 32 * i;
+            lq[i] = q < nsl ? s_ml[q * 2 * G + G + h] : 0.f;
+            mq[i] = lq[i] > 0.f ? s_ml[q * 2 * G + h] : -INFINITY;
+            M = fmaxf(M, mq[i]);
         }
-        oout[e] = __float2bfloat16_rn(A / s_L[h] * sigmoid_f(__bfloat162float(gin[e])));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int q = lane + 32 * i;
+            const float w = lq[i] > 0.f ? expf(mq[i] - M) : 0.f;
+            if (q < nsl) s_w[q * G + h] = w;
+            L = fmaf(lq[i], w, L);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (lane == 0) {
+            const float wt = expf(S.own[h] - M);
+            s_wt[h] = wt;
+            s_inv[h] = 1.f / (L + wt);
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < GE; ++r) {
+        const int e = tid + 128 * r;
+        if (e >= G * DH) break;
+        const int h = e / DH, x = e % DH;
+        float A0 = s_wt[h] * S.vt[x], A1 = 0.f;
+        int q = 0;
+        for (; q + 2 <= nsl; q += 2) {
+            const float w0 = s_w[q * G + h], w1 = s_w[(q + 1) * G + h];
+            if (w0 != 0.f) A0 = fmaf(__ldcg(st0 + (size_t)q * C::SS + 2 * G + e), w0, A0);
+            if (w1 != 0.f) A1 = fmaf(__ldcg(st0 + (size_t)(q + 1) * C::SS + 2 * G + e), w1, A1);
+        }
+        if (q < nsl) {
+            const float w0 = s_w[q * G + h];
+            if (w0 != 0.f) A0 = fmaf(__ldcg(st0 + (size_t)q * C::SS + 2 * G + e), w0, A0);
+        }
+        oout[e] = __float2bfloat16_rn((A0 + A1) * s_inv[h] * sigmoid_f(gv[r]));
     }
     if (p.evict_bits)
         for (int w = ((n + 31) >> 5) + tid; w < words; w += blockDim.x) p.evict_bits[(size_t)unit * words + w] = 0u;
@@ -219,7 +286,7 @@ __device__ void merge_append(DecTcSmem<DH, G>& S, const DecodeParams& p, int uni
         }
         if (tid == 0) {
             c.bias[base + n] = 0.f;
-            c.rk[base + n] = softplus_f(p.a_k[unit]);
+            c.rk[base + n] = softplus_f(tk.ak);
             c.pos[base + n] = p.pos_t;
             c.n_kept[unit] = n + 1;
             if (p.kept_idx) p.kept_idx[base + n] = -1;
@@ -227,7 +294,7 @@ __device__ void merge_append(DecTcSmem<DH, G>& S, const DecodeParams& p, int uni
     } else if (tid == 0) {
         raise_status(UA_ERR_CAPACITY);
     }
-    if (tid == 0) p.split_cnt[unit] = 0u;            // ready for the next step
+    if (tid == 0) p.split_cnt[unit] = 0u;            // back to zero for the next step
 }
 
 // Dense tiles: when a tile's positions are contiguous (pos_j = pos_base + (j - first slot), as in a
@@ -269,6 +336,8 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
 
     grid_dep_wait();
     grid_dep_release();
+    TokIn<DH, G> tk;
+    load_token<DH, G>(tk, p, unit, b, kvh);
     int n = c.n_kept[unit];
     if (n < 0 || n > c.cap) {                 // corrupt count: never read past the cache
         if (tid == 0 && sl == 0) raise_status(UA_ERR_CAPACITY);
@@ -279,19 +348,27 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     const int lo = sl < nsl ? min(n, sl * chunk) : n;
     const int hi = sl < nsl ? min(n, lo + chunk) : n;
     const int ntiles = (hi - lo + kDecTile - 1) / kDecTile;
+    const int nwalk = chunk > 0 ? min(nsl, (n + chunk - 1) / chunk) : 0;   // slices 0 .. nwalk-1 hold pairs
 
+    // Arrival on the cache's counter (zero before the step; the merging CTA zeroes it again):
+    // every CTA of the grid counts, so the merge -- which changes n -- comes after all of them
+    // have read n.  A count already at the grid's size means the workspace was not zeroed.
+    auto arrive = [&]() {
+        if (tid == 0) {
+            const unsigned old = atomicAdd(p.split_cnt + unit, 1u);
+            if (old >= gridDim.x) raise_status(UA_ERR_INVALID_ARG);
+            S.last = old == gridDim.x - 1;
+        }
+        __syncthreads();
+    };
     if (ntiles == 0) {
-        // nothing to walk: an empty state, arrival, and the merge if this CTA is the last one
-        float* st = p.split_state + ((size_t)unit * kDecodeSplitMax + sl) * C::SS;
-        for (int e = tid; e < C::SS; e += blockDim.x) st[e] = 0.f;
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) S.last = atomicAdd(p.split_cnt + unit, 1u) == gridDim.x - 1;
-        __syncthreads();
+        // nothing to walk (the merge reads only the slices that walked pairs): arrival, and
+        // the merge if this CTA is the last one
+        arrive();
         if (!S.last) return;
         __threadfence();
-        new_token<DH, G>(S, p, unit, b, kvh);
-        merge_append<DH, G>(S, p, unit, b, kvh, n);
+        new_token<DH, G>(S, p, tk);
+        merge_append<DH, G>(S, p, tk, unit, b, kvh, n, nwalk);
         return;
     }
 
@@ -339,7 +416,7 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     }
     load_scalars(0);
     tc_fence_before();
-    new_token<DH, G>(S, p, unit, b, kvh);             // ends with __syncthreads
+    new_token<DH, G>(S, p, tk);                       // ends with __syncthreads
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
     volatile int* abort = &S.abort;
@@ -367,8 +444,8 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     __syncthreads();
 
     const float scale = p.scale, logp = p.logp;
-    const float rq_t = (variant & kVarNoQ) ? 1.f : softplus_f(p.a_q[unit]);
-    const float al = p.alpha[kvh], be = p.beta[kvh];
+    const float rq_t = (variant & kVarNoQ) ? 1.f : softplus_f(tk.aq);
+    const float al = tk.al, be = tk.be;
     const uint32_t ID1 = idesc_bf16(128, 16, 0, 0);
     const uint32_t ID2 = idesc_bf16(128, 16, 1, 1);
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -609,11 +686,10 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     // ---- arrival; the last CTA of the cache merges
     __threadfence();
     __syncthreads();
-    if (tid == 0) S.last = atomicAdd(p.split_cnt + unit, 1u) == gridDim.x - 1;
-    __syncthreads();
+    arrive();
     if (!S.last) return;
     __threadfence();
-    merge_append<DH, G>(S, p, unit, b, kvh, n);
+    merge_append<DH, G>(S, p, tk, unit, b, kvh, n, nwalk);
 }
 
 template <int DH>

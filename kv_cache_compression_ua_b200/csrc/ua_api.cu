@@ -708,8 +708,9 @@ ua_status ua_decode_step_split(const ua_cache* c, int H, const void* q, const vo
     if (ws_bytes < decode_ws_bytes(c, H)) return UA_ERR_WORKSPACE;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const size_t units = (size_t)c->B * c->Hkv;
-    // the per-cache arrival counters start at zero (the kernel also clears them after use)
-    if ((st = cuda_status(cudaMemsetAsync(ws, 0, units * 4, cs))) != UA_OK) return st;
+    // the per-cache arrival counters at the start of ws are zero before the first step (the
+    // caller zeroes the workspace once) and every step leaves them zero, so consecutive steps
+    // need no memset between their kernels
     DecodeParams dp;
     dp.c = view(c); dp.H = H; dp.G = H / c->Hkv; dp.pos_t = pos_t; dp.scale = scale;
     dp.logp = p > 0.f ? logf(p) : -INFINITY; dp.theta = rope_theta; dp.rf = rope_freq(rope_theta, c->d);

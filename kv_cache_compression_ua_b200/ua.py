@@ -206,8 +206,9 @@ def prefill_workspace_size(shape: ua_shape) -> int:
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
-    # torch's caching allocator returns >= 512-byte aligned blocks
-    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    # torch's caching allocator returns >= 512-byte aligned blocks; zeroed, as the split decode
+    # step's arrival counters must start at zero (the prefill's scratch needs nothing)
+    return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
 def prefill_fwd(q, k, v, g, a_q, a_k, alpha, beta, *, scale=None, theta=500000.0, want_lse=True,
