@@ -68,11 +68,11 @@ struct DecTcSmem {
     alignas(1024) uint8_t bq[16 * DH * 2];                   // no-swizzle K-major B of S
     alignas(128) uint8_t pt[2][kDecTile][16];                // P: MN-major no-swizzle, heads 0-7 | 8-15
     double gtf[DH / 2];                                       // RoPE frequencies / (2 pi)
-    float ff[DH / 2];                                        // RoPE frequencies (fp32)
+    alignas(16) float ff[DH / 2];                            // RoPE frequencies (fp32)
     float bcs[2][DH / 2][2];                                 // per tile parity: cos, sin of pos_base * f_m
     int wd[2][4];                                            // per tile parity and warp: pos_j - j, or a
                                                              // sentinel when the warp's positions are not contiguous
-    float kt[DH];                                            // khat_t, pair-interleaved
+    alignas(16) float kt[DH];                                // khat_t, pair-interleaved
     float ktr[DH];                                           // RoPE(khat_t, pos_t), pair-interleaved
     float vt[DH];
     float q[G][DH];                                          // RoPE(q_h, pos_t), pair-interleaved
@@ -618,6 +618,17 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
                 tmem_st16(tmem + lane_base + C::COL_O, o);
                 tmem_wait_st();
             }
+        }
+        if (!valid) {
+            // a ragged last tile: this row of V enters the second product with P = 0; zero it, as
+            // slots past the live pairs may hold anything and 0 x NaN would poison O
+            if (!mbar_wait(&S.full_v, t & 1, abort)) ok = false;
+#pragma unroll
+            for (int bx = 0; bx < NB; ++bx)
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(S.stage[0][bx] + (uint32_t)tid * 128u + ((uint32_t)ch << 4)) =
+                        make_uint4(0u, 0u, 0u, 0u);
         }
         // ---- probabilities into P (bf16, heads 0-7 in block 0, 8-15 in block 1)
         float pr[16];

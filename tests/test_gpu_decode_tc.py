@@ -133,3 +133,80 @@ def test_tensor_core_split_decode_shift_rescale():
     about 20; all queries at ~60 measured 6.5e-3.)"""
     w = I.Workload("dec_tc_qn", 1, 2600, 8, 2, 64, "bf16", 6177, bimodal_ak=True)
     run_lockstep(w, 2600, 6, 0.15, q_against_key=110.0)
+
+
+def _stale_pair(w, T0, fill_nan):
+    """A cache filled from a T0-token prefill whose slots past the live pairs hold zeros, or NaN
+    keys, values, biases and rates and arbitrary positions."""
+    bf = torch.bfloat16
+    x = I.make_prefill_inputs(w, T=T0, names=["q", "k", "v", "g", "a_q", "a_k", "alpha", "beta"])
+    ob = oracle.prefill_fwd(**x, scale=w.scale, theta=w.theta, row_mask=np.zeros(T0, np.uint8))["b_final"]
+    cap = T0 + 200
+    cache = ua.Cache.empty(w.B, w.Hkv, w.d, cap, bf)
+    ua.cache_fill(cache, dev(x["k"], bf), dev(x["v"], bf), dev(x["a_k"], torch.float32), dev(ob, torch.float32),
+                  theta=w.theta)
+    if fill_nan:
+        cache.khat[:, :, T0:] = float("nan")
+        cache.v[:, :, T0:] = float("nan")
+        cache.bias[:, :, T0:] = float("nan")
+        cache.rk[:, :, T0:] = float("nan")
+        cache.pos[:, :, T0:] = 123456789
+    return cache, x
+
+
+@pytest.mark.parametrize("split", [False, True])
+def test_slots_past_the_live_pairs_are_never_read_into_results(split):
+    """A ragged cache (300 live pairs: two full 128-entry tiles and 44 more) whose slots past the
+    live pairs hold NaN gives bit-identical steps to the same cache with zeros there: those slots'
+    values enter the tensor-core product only with zero probabilities, and the kernels zero them
+    first (0 x NaN would be NaN)."""
+    w = I.Workload("dec_stale", 2, 300, 8, 2, 64, "bf16", 6400, bimodal_ak=True)
+    outs = []
+    for fill_nan in (False, True):
+        cache, x = _stale_pair(w, 300, fill_nan)
+        ws = ua.alloc_workspace(ua.decode_workspace_size(cache, w.H), "cuda") if split else None
+        bf = torch.bfloat16
+        res = []
+        for s in range(3):
+            tok = I.make_decode_token(w, s)
+            t = {n: dev(a, bf if n in ("q", "k", "v", "g") else torch.float32) for n, a in tok.items()}
+            o = ua.decode_step(cache, t["q"], t["k"], t["v"], t["g"], t["a_q"], t["a_k"], dev(x["alpha"], torch.float32),
+                               dev(x["beta"], torch.float32), 300 + s, 0.15, scale=w.scale, theta=w.theta, ws=ws)
+            torch.cuda.synchronize()
+            assert ua.get_device_status() == 0
+            res.append(o.float().cpu().numpy())
+        n = cache.n_kept.cpu().numpy()
+        live = [cache.bias[b, h, :n[b, h]].cpu().numpy() for b in range(w.B) for h in range(w.Hkv)]
+        outs.append((res, n, live))
+    (r0, n0, l0), (r1, n1, l1) = outs
+    assert all(np.isfinite(a).all() for a in r1)
+    for a, b in zip(r0, r1):
+        np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(n0, n1)
+    for a, b in zip(l0, l1):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_split_step_reports_a_workspace_that_was_not_zeroed():
+    """The split step's per-cache arrival counters must start at zero (ua.alloc_workspace zeroes
+    them and every step leaves them zero).  Counters found at or past the grid's size raise
+    UA_ERR_INVALID_ARG in the device status (and no CTA merges); zeroed again, the workspace
+    works."""
+    w = I.Workload("dec_ws", 1, 700, 4, 2, 64, "bf16", 6500)
+    cache, x = _stale_pair(w, 700, False)
+    ws = ua.alloc_workspace(ua.decode_workspace_size(cache, w.H), "cuda")
+    bf = torch.bfloat16
+    tok = I.make_decode_token(w, 0)
+    t = {n: dev(a, bf if n in ("q", "k", "v", "g") else torch.float32) for n, a in tok.items()}
+    args = (t["q"], t["k"], t["v"], t["g"], t["a_q"], t["a_k"], dev(x["alpha"], torch.float32),
+            dev(x["beta"], torch.float32))
+    ua.get_device_status()
+    ws[: 4 * w.B * w.Hkv] = 0xFF
+    ua.decode_step(cache, *args, 700, 0.15, scale=w.scale, theta=w.theta, ws=ws)
+    assert ua.get_device_status() == 1                    # UA_ERR_INVALID_ARG
+    np.testing.assert_array_equal(cache.n_kept.cpu().numpy(), 700)   # no merge appended the token
+    ws.zero_()
+    ua.decode_step(cache, *args, 700, 0.15, scale=w.scale, theta=w.theta, ws=ws)
+    assert ua.get_device_status() == 0
+    np.testing.assert_array_equal(cache.n_kept.cpu().numpy(), 701)
+    assert int(ws[: 4 * w.B * w.Hkv].view(torch.int32).abs().sum().item()) == 0
