@@ -520,6 +520,8 @@ def bench_decode(args, peaks, peaks_kind):
         if ak is not x["a_k"]:
             res[key]["ak_slow_mean"] = I.DECODE_RETAINED_AK_SLOW_MEAN
         del g
+        if p > 0 and ak is x["a_k"]:
+            res[key]["paged"] = bench_decode_paged(w, cache, snap, tk, x, T0, steps, p, o, restore)
         # the same steps through the split walk (deferred compaction; at p > 0 a compaction every
         # DECODE_COMPACT_EVERY steps and after the last), checked against the eager outputs
         ws = ua.alloc_workspace(ua.decode_workspace_size(cache, w.H), "cuda")
@@ -604,6 +606,56 @@ def bench_decode(args, peaks, peaks_kind):
     res["peak_source"] = f"{peaks_kind} HBM copy bandwidth"
     res["workload"] = f"decode_1b: B={w.B}, 16k prefill, {steps} steps, graph-captured"
     return res
+
+
+def bench_decode_paged(w, cache, snap, tk, x, T0, steps, p, o_ref, restore_ref):
+    """The same graph-replayed eager steps on paged storage: the compacted caches' live pairs moved
+    to a pool of 128-slot pages that holds them and the appends of the coming steps only (pages for
+    the appends are given before capture, as a graph cannot call the host allocator between
+    steps).  Reports the step time and the pool's size against the contiguous caches'."""
+    from kv_cache_compression_ua_b200 import ua
+    ps = 128
+    restore_ref()
+    n0 = cache.n_kept.reshape(-1).cpu().numpy().astype(np.int64)
+    need = (n0 + steps + ps - 1) // ps
+    max_pages = (cache.capacity + ps - 1) // ps
+    paged = ua.Cache.paged(w.B, w.Hkv, w.d, ps, max_pages, int(need.sum()), torch.bfloat16)
+    pool = ua.PagePool(paged)
+    pool.ensure(n0 + steps)
+    # move the live pairs (setup, not timed)
+    tab = paged.page_table.long()
+    for u in range(w.B * w.Hkv):
+        n = int(n0[u])
+        if n == 0:
+            continue
+        s_idx = torch.arange(n, device="cuda")
+        dst = tab[u, s_idx // ps] * ps + s_idx % ps
+        b, h = divmod(u, w.Hkv)
+        for name in ("khat", "v", "bias", "rk", "pos"):
+            getattr(paged, name)[dst] = getattr(cache, name)[b, h, :n]
+    paged.n_kept.copy_(cache.n_kept)
+    psnap = {n: getattr(paged, n).clone() for n in ("khat", "v", "bias", "rk", "pos", "n_kept")}
+    o = torch.empty_like(o_ref)
+
+    def restore():
+        for n, t in psnap.items():
+            getattr(paged, n).copy_(t)
+
+    def run_all(stream=None):
+        for s in range(steps):
+            ua.decode_step(paged, tk["q"][s], tk["k"][s], tk["v"][s], tk["g"][s], tk["a_q"][s], tk["a_k"][s],
+                           x["alpha"], x["beta"], T0 + s, p, scale=w.scale, theta=w.theta, out=o[s], stream=stream)
+    restore()
+    run_all()
+    torch.cuda.synchronize()
+    assert ua.get_device_status() == 0
+    same = bool(torch.equal(o, o_ref))
+    ms = graph_time(run_all, restore)
+    entry = 2 * w.d * 2 + 12
+    return {"us_per_step": 1e3 * ms / steps, "page_slots": ps, "pages": int(need.sum()),
+            "pool_MB": int(need.sum()) * ps * entry / 1e6,
+            "contiguous_MB": w.B * w.Hkv * cache.capacity * entry / 1e6,
+            "outputs_identical_to_contiguous": same}
 
 
 def time_prefill(w, x, steps, warmup, prune_p=0.0, want_bfinal=True):

@@ -251,6 +251,21 @@ typedef struct {
     float* rk;
     int32_t* pos;
     int32_t* n_kept;
+    /* Paged storage (optional; page_table == NULL: one contiguous region of `capacity` slots per
+     * cache, as above).  Otherwise khat, v, bias, rk and pos are a pool of pool_pages pages of
+     * page_size slots each (khat, v [pool_pages*page_size, d]; the others [pool_pages*page_size]),
+     * and slot s of cache u = b*Hkv + h lives in page page_table[u*max_pages + s/page_size] at
+     * offset s % page_size.  page_size: a power of two, 128 <= page_size <= 2^20;
+     * capacity == max_pages*page_size; pool_pages*page_size < 2^31.  The caller owns the table:
+     * before a call, every slot the call may touch (slots [0, n_kept) and, for a decode step, the
+     * append slot n_kept) must lie in a page with an id in [0, pool_pages); the kernels check every
+     * id they use and, on one outside that range, raise UA_ERR_INVALID_ARG in the device status
+     * and skip the access (the call's outputs are then unspecified).  After a compaction, the pages
+     * past ceil(n_kept/page_size) hold no live pair and may be handed to other caches.  This is
+     * the pages' missing dynamic cache manager (summary App. H) in its plainest form: a pruned
+     * cache occupies pages for its live pairs only, not a reserved region of its longest length. */
+    int page_size, max_pages, pool_pages;
+    const int32_t* page_table;
 } ua_cache;
 
 /* Load a prefill into the cache: slot t <- token t for t < T (khat, v from k and v; bias =

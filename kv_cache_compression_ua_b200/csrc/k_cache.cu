@@ -84,7 +84,12 @@ __global__ void __launch_bounds__(256) k_cache_fill(FillParams p) {
     const TC* vin = static_cast<const TC*>(p.v);
     for (int h = warp; h < c.Hkv; h += 8) {
         const size_t src = (((size_t)b * T + t) * (c.Hkv / c.rep) + h / c.rep) * DH;
-        const size_t slot = ((size_t)b * c.Hkv + h) * c.cap + t;
+        const long long ps = phys_slot(c, b * c.Hkv + h, t);    // uniform over the warp
+        if (ps < 0) {
+            if (lane == 0 && t == 0) c.n_kept[(size_t)b * c.Hkv + h] = T;
+            continue;
+        }
+        const size_t slot = (size_t)ps;
         float x0[2] = {0.f, 0.f}, x1[2] = {0.f, 0.f};
         float ss = 0.f;
 #pragma unroll
@@ -147,26 +152,28 @@ __global__ void __launch_bounds__(256) k_cache_compact(CompactParams p) {
         float bj = 0.f, rkj = 0.f;
         int pj = 0;
         bool keep = false;
-        if (valid) {
-            const size_t e = (base + j) * DH + gl * L::VEC;
+        const long long ps = valid ? phys_slot(c, unit, j) : -1;
+        if (ps >= 0) {
+            const size_t e = (size_t)ps * DH + gl * L::VEC;
             a = *reinterpret_cast<const uint4*>(khat + e);
             vv = *reinterpret_cast<const uint4*>(vc + e);
-            bj = c.bias[base + j];
-            rkj = c.rk[base + j];
-            pj = c.pos[base + j];
+            bj = c.bias[ps];
+            rkj = c.rk[ps];
+            pj = c.pos[ps];
             keep = p.keep ? (p.keep[base + j] != 0) : (bj >= p.logp);
         }
         int tot;
         const int dst = out + pass_scan<L::LPE, L::NW>(keep, warp, lane, s_wcnt, &tot);
         if (keep) {
-            if (dst != j) {
-                const size_t e = (base + dst) * DH + gl * L::VEC;
+            const long long pd = dst != j ? phys_slot(c, unit, dst) : -1;
+            if (pd >= 0) {
+                const size_t e = (size_t)pd * DH + gl * L::VEC;
                 *reinterpret_cast<uint4*>(khat + e) = a;
                 *reinterpret_cast<uint4*>(vc + e) = vv;
                 if (gl == 0) {
-                    c.bias[base + dst] = bj;
-                    c.rk[base + dst] = rkj;
-                    c.pos[base + dst] = pj;
+                    c.bias[pd] = bj;
+                    c.rk[pd] = rkj;
+                    c.pos[pd] = pj;
                 }
             }
             if (gl == 0 && p.kept_idx) p.kept_idx[base + dst] = j;
@@ -183,7 +190,7 @@ __global__ void __launch_bounds__(256) k_cache_compact(CompactParams p) {
 // DEFER: deferred compaction (UA_DECODE_DEFER_COMPACT).  VAR: an ablation variant is set; without
 // it the variant is the constant 0 and every variant branch folds away.  Both are separate
 // instantiations so that the method's own per-step path keeps its registers and instructions.
-template <typename TC, int DH, int G, bool DEFER, bool VAR>
+template <typename TC, int DH, int G, bool DEFER, bool VAR, bool PAGED>
 __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) {
     const int variant = VAR ? p.variant : 0;
     using L = EntryLayout<TC, DH>;
@@ -223,8 +230,19 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     uint4 na = make_uint4(0, 0, 0, 0), nv = na;
     float nbj = 0.f, nrk = 0.f;
     int npj = 0;
+    long long nps = -1;                               // paged: the loaded entry's physical slot
     auto load_entry = [&](int jj, int lim) {
-        if (jj < lim) {
+        if constexpr (PAGED) {
+            nps = jj < lim ? phys_slot(c, unit, jj) : -1;
+            if (nps >= 0) {
+                const size_t e = (size_t)nps * DH + gl * VEC;
+                na = *reinterpret_cast<const uint4*>(khat + e);
+                nv = *reinterpret_cast<const uint4*>(vc + e);
+                nbj = c.bias[nps];
+                nrk = c.rk[nps];
+                npj = c.pos[nps];
+            }
+        } else if (jj < lim) {
             const size_t e = (base + jj) * DH + gl * VEC;
             na = *reinterpret_cast<const uint4*>(khat + e);
             nv = *reinterpret_cast<const uint4*>(vc + e);
@@ -233,7 +251,8 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
             npj = c.pos[base + jj];
         }
     };
-    load_entry(gidx, c.cap);
+    // (paged storage reads the first pass once the count is known: slots past it may have no page)
+    if (!PAGED) load_entry(gidx, c.cap);
     // the step's key and value: head kvh / rep of [B, Hkv / rep, d]
     const size_t tok = (size_t)b * (c.Hkv / c.rep) + kvh / c.rep;
     const TC* kin = static_cast<const TC*>(p.k) + tok * DH;
@@ -343,6 +362,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     }
     int out = 0;
     const bool multi_pass = n > 4 * EPB;   // block-uniform
+    if (PAGED) load_entry(gidx, n);
     for (int c0 = 0; c0 < n; c0 += EPB) {
         const int j = c0 + gidx;
         const bool valid = j < n;
@@ -352,7 +372,19 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
 #pragma unroll
             for (int ahead = 1; ahead <= 2; ++ahead) {
                 const int jn = j + ahead * EPB;
-                if (jn < n) {
+                if constexpr (PAGED) {
+                    const long long pn = jn < n ? phys_slot<false>(c, unit, jn) : -1;
+                    if (pn >= 0) {
+                        const size_t e = (size_t)pn * DH;
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(khat + e));
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(vc + e));
+                        if ((jn & 31) == 0) {
+                            asm volatile("prefetch.global.L2 [%0];" ::"l"(c.bias + pn));
+                            asm volatile("prefetch.global.L2 [%0];" ::"l"(c.rk + pn));
+                            asm volatile("prefetch.global.L2 [%0];" ::"l"(c.pos + pn));
+                        }
+                    }
+                } else if (jn < n) {
                     const size_t e = (base + jn) * DH;
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(khat + e));
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(vc + e));
@@ -367,6 +399,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         const uint4 ra = na, rv = nv;
         const float bj = nbj, rkj = nrk;
         const int pj = npj;
+        const long long psj = nps;                    // paged only
         load_entry(j + EPB, n);
         float xa[VEC], xb[VEC], xv[VEC];
         Vec16<TC>::unpack(ra, xa);
@@ -378,7 +411,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         sim = group_sum<LPE>(sim);
         const float D = decay_var(rq_t, (variant & kVarNoK) ? 1.f : rkj, fmaf(al, sim, be), variant);
         const float bnew = bj - D;
-        const bool keep = valid && (bnew >= p.logp);
+        const bool keep = PAGED ? valid && psj >= 0 && (bnew >= p.logp) : valid && (bnew >= p.logp);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             float lg = 0.f;
@@ -399,7 +432,11 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         if (valid && !keep && gl == 0) atomicOr(&s_ev[j >> 5], 1u << (j & 31));
         if (DEFER) {                              // every pair keeps its slot
             if (valid && gl == 0) {
-                c.bias[base + j] = bnew;
+                if constexpr (PAGED) {
+                    if (psj >= 0) c.bias[psj] = bnew;
+                } else {
+                    c.bias[base + j] = bnew;
+                }
                 if (p.kept_idx) p.kept_idx[base + j] = j;
             }
             __syncthreads();
@@ -408,18 +445,35 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
         int tot;
         const int dst = out + pass_scan<LPE, NW>(keep, warp, lane, s_wcnt, &tot);
         if (keep) {
-            if (dst != j) {
-                const size_t e = (base + dst) * DH + gl * VEC;
-                *reinterpret_cast<uint4*>(khat + e) = ra;
-                *reinterpret_cast<uint4*>(vc + e) = rv;
-                if (gl == 0) {
-                    c.rk[base + dst] = rkj;
-                    c.pos[base + dst] = pj;
+            if constexpr (PAGED) {
+                const long long pd = dst != j ? phys_slot(c, unit, dst) : psj;
+                if (pd >= 0 && dst != j) {
+                    const size_t e = (size_t)pd * DH + gl * VEC;
+                    *reinterpret_cast<uint4*>(khat + e) = ra;
+                    *reinterpret_cast<uint4*>(vc + e) = rv;
+                    if (gl == 0) {
+                        c.rk[pd] = rkj;
+                        c.pos[pd] = pj;
+                    }
                 }
-            }
-            if (gl == 0) {
-                c.bias[base + dst] = bnew;
-                if (p.kept_idx) p.kept_idx[base + dst] = j;
+                if (gl == 0) {
+                    if (pd >= 0) c.bias[pd] = bnew;
+                    if (p.kept_idx) p.kept_idx[base + dst] = j;
+                }
+            } else {
+                if (dst != j) {
+                    const size_t e = (base + dst) * DH + gl * VEC;
+                    *reinterpret_cast<uint4*>(khat + e) = ra;
+                    *reinterpret_cast<uint4*>(vc + e) = rv;
+                    if (gl == 0) {
+                        c.rk[base + dst] = rkj;
+                        c.pos[base + dst] = pj;
+                    }
+                }
+                if (gl == 0) {
+                    c.bias[base + dst] = bnew;
+                    if (p.kept_idx) p.kept_idx[base + dst] = j;
+                }
             }
         }
         out += tot;
@@ -497,17 +551,37 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode(DecodeParams p) 
     if (p.evict_bits)
         for (int w = tid; w < words; w += blockDim.x) p.evict_bits[(size_t)unit * words + w] = s_ev[w];
     if (out < c.cap) {
-        const size_t e = (base + out) * DH;
-        for (int x = tid; x < DH; x += blockDim.x) {
-            Elem<TC>::st(khat + e + x, s_kt[x]);
-            Elem<TC>::st(vc + e + x, s_vt[x]);
-        }
-        if (tid == 0) {
-            c.bias[base + out] = 0.f;
-            c.rk[base + out] = rk_t;
-            c.pos[base + out] = p.pos_t;
-            c.n_kept[unit] = out + 1;
-            if (p.kept_idx) p.kept_idx[base + out] = -1;
+        if constexpr (PAGED) {
+            const long long pa = phys_slot(c, unit, out);
+            if (pa >= 0) {
+                const size_t e = (size_t)pa * DH;
+                for (int x = tid; x < DH; x += blockDim.x) {
+                    Elem<TC>::st(khat + e + x, s_kt[x]);
+                    Elem<TC>::st(vc + e + x, s_vt[x]);
+                }
+                if (tid == 0) {
+                    c.bias[pa] = 0.f;
+                    c.rk[pa] = rk_t;
+                    c.pos[pa] = p.pos_t;
+                }
+            }
+            if (tid == 0) {
+                c.n_kept[unit] = out + 1;
+                if (p.kept_idx) p.kept_idx[base + out] = -1;
+            }
+        } else {
+            const size_t e = (base + out) * DH;
+            for (int x = tid; x < DH; x += blockDim.x) {
+                Elem<TC>::st(khat + e + x, s_kt[x]);
+                Elem<TC>::st(vc + e + x, s_vt[x]);
+            }
+            if (tid == 0) {
+                c.bias[base + out] = 0.f;
+                c.rk[base + out] = rk_t;
+                c.pos[base + out] = p.pos_t;
+                c.n_kept[unit] = out + 1;
+                if (p.kept_idx) p.kept_idx[base + out] = -1;
+            }
         }
     } else if (tid == 0) {
         c.n_kept[unit] = out;
@@ -641,14 +715,16 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
     uint4 na = make_uint4(0, 0, 0, 0), nv = na;
     float nbj = 0.f, nrk = 0.f;
     int npj = 0;
+    long long nps = -1;                               // the loaded entry's physical slot
     auto load_entry = [&](int jj) {
-        if (jj < hi) {
-            const size_t e = (base + jj) * DH + gl * VEC;
+        nps = jj < hi ? phys_slot(c, unit, jj) : -1;
+        if (nps >= 0) {
+            const size_t e = (size_t)nps * DH + gl * VEC;
             na = *reinterpret_cast<const uint4*>(khat + e);
             nv = *reinterpret_cast<const uint4*>(vc + e);
-            nbj = c.bias[base + jj];
-            nrk = c.rk[base + jj];
-            npj = c.pos[base + jj];
+            nbj = c.bias[nps];
+            nrk = c.rk[nps];
+            npj = c.pos[nps];
         }
     };
     load_entry(lo + gidx);
@@ -658,6 +734,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
         const uint4 ra = na, rv = nv;
         const float bj = nbj, rkj = nrk;
         const int pj = npj;
+        const long long psj = nps;
         load_entry(j + EPB);
         float xa[VEC], xb[VEC], xv[VEC];
         Vec16<TC>::unpack(ra, xa);
@@ -669,7 +746,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
         sim = group_sum<LPE>(sim);
         const float D = decay_var(rq_t, (variant & kVarNoK) ? 1.f : rkj, fmaf(al, sim, be), variant);
         const float bnew = bj - D;
-        const bool keep = valid && (bnew >= p.logp);
+        const bool keep = valid && psj >= 0 && (bnew >= p.logp);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             float lg = 0.f;
@@ -688,7 +765,7 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
             }
         }
         if (valid && gl == 0) {
-            c.bias[base + j] = bnew;
+            if (psj >= 0) c.bias[psj] = bnew;
             if (p.kept_idx) p.kept_idx[base + j] = j;
             if (!keep) atomicOr(&s_ev[(j >> 5) - w0], 1u << (j & 31));
         }
@@ -760,15 +837,20 @@ __global__ void __launch_bounds__(256, G <= 4 ? 2 : 1) k_decode_split(DecodePara
     if (p.evict_bits)
         for (int w = ((n + 31) >> 5) + tid; w < words; w += blockDim.x) p.evict_bits[(size_t)unit * words + w] = 0u;
     if (n < c.cap) {
-        const size_t e = (base + n) * DH;
-        for (int x = tid; x < DH; x += blockDim.x) {
-            Elem<TC>::st(khat + e + x, s_kt[x]);
-            Elem<TC>::st(vc + e + x, s_vt[x]);
+        const long long pa = phys_slot(c, unit, n);
+        if (pa >= 0) {
+            const size_t e = (size_t)pa * DH;
+            for (int x = tid; x < DH; x += blockDim.x) {
+                Elem<TC>::st(khat + e + x, s_kt[x]);
+                Elem<TC>::st(vc + e + x, s_vt[x]);
+            }
+            if (tid == 0) {
+                c.bias[pa] = 0.f;
+                c.rk[pa] = softplus_f(ak_t);
+                c.pos[pa] = p.pos_t;
+            }
         }
         if (tid == 0) {
-            c.bias[base + n] = 0.f;
-            c.rk[base + n] = softplus_f(ak_t);
-            c.pos[base + n] = p.pos_t;
             c.n_kept[unit] = n + 1;
             if (p.kept_idx) p.kept_idx[base + n] = -1;
         }
@@ -806,13 +888,13 @@ cudaError_t launch_cache_compact(const CompactParams& p, bool bf16, cudaStream_t
 
 template <typename TC, int DH, int G, bool DEFER, bool VAR>
 static cudaError_t decode_launch(const DecodeParams& p, size_t smem, cudaStream_t s) {
+    auto kern = p.c.pt != nullptr ? k_decode<TC, DH, G, DEFER, VAR, true> : k_decode<TC, DH, G, DEFER, VAR, false>;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k_decode<TC, DH, G, DEFER, VAR>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     UA_PROFILE("k_decode", s);
-    return launch_dependent(k_decode<TC, DH, G, DEFER, VAR>, dim3(p.c.B * p.c.Hkv), dim3(256), smem, s, p);
+    return launch_dependent(kern, dim3(p.c.B * p.c.Hkv), dim3(256), smem, s, p);
 }
 
 template <typename TC, int DH, int G>

@@ -279,15 +279,20 @@ __device__ void merge_append(DecTcSmem<DH, G>& S, const DecodeParams& p, const T
     __nv_bfloat16* khat = static_cast<__nv_bfloat16*>(c.khat);
     __nv_bfloat16* vc = static_cast<__nv_bfloat16*>(c.v);
     if (n < c.cap) {
-        const size_t e = (base + n) * DH;
-        for (int x = tid; x < DH; x += blockDim.x) {
-            khat[e + x] = __float2bfloat16_rn(S.kt[x]);
-            vc[e + x] = __float2bfloat16_rn(S.vt[x]);
+        const long long pa = phys_slot(c, unit, n);
+        if (pa >= 0) {
+            const size_t e = (size_t)pa * DH;
+            for (int x = tid; x < DH; x += blockDim.x) {
+                khat[e + x] = __float2bfloat16_rn(S.kt[x]);
+                vc[e + x] = __float2bfloat16_rn(S.vt[x]);
+            }
+            if (tid == 0) {
+                c.bias[pa] = 0.f;
+                c.rk[pa] = softplus_f(tk.ak);
+                c.pos[pa] = p.pos_t;
+            }
         }
         if (tid == 0) {
-            c.bias[base + n] = 0.f;
-            c.rk[base + n] = softplus_f(tk.ak);
-            c.pos[base + n] = p.pos_t;
             c.n_kept[unit] = n + 1;
             if (p.kept_idx) p.kept_idx[base + n] = -1;
         }
@@ -319,7 +324,7 @@ __device__ __forceinline__ void tile_density(DecTcSmem<DH, G>& S, int par, int p
     }
 }
 
-template <int DH, int G>
+template <int DH, int G, bool PAGED>
 __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     k_decode_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_v, DecodeParams p) {
     using C = DecTc<DH, G>;
@@ -388,13 +393,23 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     // One stage.  A tile's keys are reloaded as soon as its first product has read them (mid
     // tile), its values once the second product is done (at the start of the next tile), so both
     // loads overlap the work of a tile instead of following it.
+    // a tile's first physical row: a tile lies within one page (pages hold a power of two >= 128
+    // slots, tiles start at multiples of 128); a page outside the pool (raised) reads row 0
+    auto tile_row = [&](int tt) -> int {
+        if constexpr (PAGED) {
+            const long long r = phys_slot(c, unit, lo + tt * kDecTile);
+            return r >= 0 ? (int)r : 0;
+        } else {
+            return (int)(base + lo + (size_t)tt * kDecTile);
+        }
+    };
     auto issue_k = [&](int tt) {
-        const int row = (int)(base + lo + (size_t)tt * kDecTile);
+        const int row = tile_row(tt);
         mbar_expect_tx(&S.full_k, NB * 16384);
         for (int bx = 0; bx < NB; ++bx) tma_load_2d(S.stage[0][NB + bx], &tm_kh, &S.full_k, 64 * bx, row);
     };
     auto issue_v = [&](int tt) {
-        const int row = (int)(base + lo + (size_t)tt * kDecTile);
+        const int row = tile_row(tt);
         mbar_expect_tx(&S.full_v, NB * 16384);
         for (int bx = 0; bx < NB; ++bx) tma_load_2d(S.stage[0][bx], &tm_v, &S.full_v, 64 * bx, row);
     };
@@ -402,7 +417,14 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
     // each thread copies and later reads only its own entry's
     auto load_scalars = [&](int tt) {
         const int jj = lo + tt * kDecTile + tid, par = tt & 1;
-        if (jj < hi) {
+        if constexpr (PAGED) {
+            const long long ps = jj < hi ? phys_slot(c, unit, jj) : -1;
+            if (ps >= 0) {
+                cp_async4(&S.scp[par][tid], c.pos + ps);
+                cp_async4(&S.scb[par][tid], c.bias + ps);
+                cp_async4(&S.scr[par][tid], c.rk + ps);
+            }
+        } else if (jj < hi) {
             cp_async4(&S.scp[par][tid], c.pos + base + jj);
             cp_async4(&S.scb[par][tid], c.bias + base + jj);
             cp_async4(&S.scr[par][tid], c.rk + base + jj);
@@ -546,7 +568,12 @@ __global__ void __launch_bounds__(128, DecTc<DH, G>::CTAS)
         const float bnew = bj - D;
         const bool keep = valid && bnew >= logp;
         if (valid) {
-            c.bias[base + j] = bnew;
+            if constexpr (PAGED) {
+                const long long ps = phys_slot(c, unit, j);
+                if (ps >= 0) c.bias[ps] = bnew;
+            } else {
+                c.bias[base + j] = bnew;
+            }
             if (p.kept_idx) p.kept_idx[base + j] = j;
         }
         const unsigned ev = __ballot_sync(0xffffffffu, valid && !keep);
@@ -752,16 +779,17 @@ int decode_tc_slices(int units, int cap, int ctas_per_sm) {
 
 template <int DH, int G>
 cudaError_t decode_tc_inst(const DecodeParams& p, cudaStream_t s) {
-    const size_t rows = (size_t)p.c.B * p.c.Hkv * p.c.cap;
+    const size_t rows = p.c.pt ? (size_t)p.c.pool_pages << p.c.ps_shift : (size_t)p.c.B * p.c.Hkv * p.c.cap;
     CUtensorMap mk, mv;
     if (!map_cache_rows<DH>(&mk, p.c.khat, rows) || !map_cache_rows<DH>(&mv, p.c.v, rows))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(DecTcSmem<DH, G>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_decode_tc<DH, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = p.c.pt != nullptr ? k_decode_tc<DH, G, true> : k_decode_tc<DH, G, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     UA_PROFILE("k_decode_tc", s);
     const int units = p.c.B * p.c.Hkv;
-    return launch_dependent(k_decode_tc<DH, G>, dim3(decode_tc_slices(units, p.c.cap, DecTc<DH, G>::CTAS), units),
+    return launch_dependent(kern, dim3(decode_tc_slices(units, p.c.cap, DecTc<DH, G>::CTAS), units),
                             dim3(128), smem, s, mk, mv, p);
 }
 

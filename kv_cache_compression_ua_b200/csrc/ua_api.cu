@@ -168,6 +168,14 @@ ua_status check_cache(const ua_cache* c) {
     const void* ps[] = {c->khat, c->v, c->bias, c->rk, c->pos, c->n_kept};
     for (const void* p : ps)
         if (!aligned(p, 16)) return UA_ERR_ALIGNMENT;
+    if (c->page_table) {                      // paged storage
+        const int sz = c->page_size;
+        if (sz < 128 || sz > kMaxCapacity || (sz & (sz - 1)) != 0) return UA_ERR_INVALID_ARG;
+        if (c->max_pages < 1 || c->pool_pages < 1) return UA_ERR_INVALID_ARG;
+        if ((long long)c->max_pages * sz != c->capacity) return UA_ERR_INVALID_ARG;
+        if ((long long)c->pool_pages * sz >= (long long)INT32_MAX) return UA_ERR_UNSUPPORTED;
+        if (!aligned(c->page_table, 4)) return UA_ERR_ALIGNMENT;
+    }
     return UA_OK;
 }
 
@@ -176,6 +184,14 @@ CacheView view(const ua_cache* c) {
     v.B = c->B; v.Hkv = c->Hkv; v.d = c->d; v.cap = c->capacity; v.rep = c->kv_rep > 1 ? c->kv_rep : 1;
     v.khat = c->khat; v.v = c->v; v.bias = c->bias; v.rk = c->rk;
     v.pos = c->pos; v.n_kept = c->n_kept;
+    v.pt = c->page_table;
+    v.ps_shift = 0;
+    v.max_pages = v.pool_pages = 0;
+    if (c->page_table) {
+        while ((1 << v.ps_shift) < c->page_size) ++v.ps_shift;
+        v.max_pages = c->max_pages;
+        v.pool_pages = c->pool_pages;
+    }
     return v;
 }
 
@@ -719,7 +735,8 @@ ua_status ua_decode_step_split(const ua_cache* c, int H, const void* q, const vo
     dp.split_cnt = static_cast<unsigned*>(ws);
     dp.split_state = reinterpret_cast<float*>(at(ws, round_up(units * 4, 256)));
     // bf16 caches on the tensor cores (their TMA row coordinate must fit an int)
-    if (c->dtype == UA_BF16 && units * (size_t)c->capacity < (size_t)INT32_MAX)
+    const size_t rows = c->page_table ? (size_t)c->pool_pages * c->page_size : units * (size_t)c->capacity;
+    if (c->dtype == UA_BF16 && rows < (size_t)INT32_MAX)
         return cuda_status(launch_decode_tc(dp, cs));
     return cuda_status(launch_decode_split(dp, c->dtype == UA_BF16, cs));
 }

@@ -114,7 +114,25 @@ struct CacheView {
     float* rk;
     int32_t* pos;
     int32_t* n_kept;
+    // paged storage (pt == nullptr: cache u's slot s is at u * cap + s)
+    const int32_t* pt;   // [B*Hkv][max_pages] page ids
+    int ps_shift;        // log2(page size)
+    int max_pages, pool_pages;
 };
+
+// Physical slot (row of khat and v, index of bias, rk and pos) of slot s of cache u.  A page id
+// outside the pool gives -1: RAISE records UA_ERR_INVALID_ARG (a slot the call must touch), else
+// the caller only skips the access (a speculative read).
+template <bool RAISE = true>
+__device__ __forceinline__ long long phys_slot(const CacheView& c, int u, int s) {
+    if (c.pt == nullptr) return (long long)u * c.cap + s;
+    const int pg = __ldg(c.pt + (size_t)u * c.max_pages + (s >> c.ps_shift));
+    if ((unsigned)pg >= (unsigned)c.pool_pages) {
+        if (RAISE) raise_status(UA_ERR_INVALID_ARG);
+        return -1;
+    }
+    return ((long long)pg << c.ps_shift) | (long long)(s & ((1 << c.ps_shift) - 1));
+}
 
 struct FillParams {
     CacheView c;

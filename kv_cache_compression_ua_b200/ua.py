@@ -45,7 +45,8 @@ class ua_cache(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int), ("capacity", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("kv_rep", ctypes.c_int), ("khat", ctypes.c_void_p),
                 ("v", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("rk", ctypes.c_void_p),
-                ("pos", ctypes.c_void_p), ("n_kept", ctypes.c_void_p)]
+                ("pos", ctypes.c_void_p), ("n_kept", ctypes.c_void_p), ("page_size", ctypes.c_int),
+                ("max_pages", ctypes.c_int), ("pool_pages", ctypes.c_int), ("page_table", ctypes.c_void_p)]
 
 
 EXPORTS = ("ua_prefill_workspace_size", "ua_prefill_fwd", "ua_prefill_bwd_workspace_size", "ua_prefill_bwd",
@@ -335,6 +336,28 @@ class Cache:
     pos: torch.Tensor
     n_kept: torch.Tensor
     kv_rep: int = 1
+    # paged storage (see ua_cache.page_table): the arrays above are a pool of pool_pages pages of
+    # page_size slots, page_table [B*Hkv, max_pages] int32 maps a cache's pages to pool pages
+    page_size: int = 0
+    pool_pages: int = 0
+    page_table: torch.Tensor | None = None
+
+    @staticmethod
+    def paged(B, Hkv, d, page_size, max_pages, pool_pages, dtype=torch.bfloat16, device="cuda", kv_rep=1):
+        """A cache set on a pool of pool_pages pages of page_size slots; every cache may grow to
+        max_pages pages.  The page table starts empty (-1): give the caches pages with a PagePool."""
+        if kv_rep < 1 or Hkv % kv_rep:
+            raise ValueError(f"kv_rep {kv_rep} must divide Hkv {Hkv}")
+        if page_size < 128 or page_size & (page_size - 1):
+            raise ValueError(f"page_size {page_size} must be a power of two >= 128")
+        kw = dict(device=device)
+        slots = pool_pages * page_size
+        return Cache(B, Hkv, d, max_pages * page_size, dtype,
+                     torch.zeros(slots, d, dtype=dtype, **kw), torch.zeros(slots, d, dtype=dtype, **kw),
+                     torch.zeros(slots, dtype=torch.float32, **kw), torch.zeros(slots, dtype=torch.float32, **kw),
+                     torch.zeros(slots, dtype=torch.int32, **kw), torch.zeros(B, Hkv, dtype=torch.int32, **kw),
+                     kv_rep, page_size, pool_pages,
+                     torch.full((B * Hkv, max_pages), -1, dtype=torch.int32, **kw))
 
     @staticmethod
     def empty(B, Hkv, d, capacity, dtype=torch.bfloat16, device="cuda", kv_rep=1):
@@ -355,7 +378,8 @@ class Cache:
         return self.Hkv // self.kv_rep
 
     def struct(self) -> ua_cache:
-        n = self.B * self.Hkv * self.capacity
+        paged = self.page_table is not None
+        n = self.pool_pages * self.page_size if paged else self.B * self.Hkv * self.capacity
         for name in ("khat", "v"):
             _need(f"cache.{name}", getattr(self, name), n * self.d, (self.dtype,))
         _need("cache.bias", self.bias, n, F32)
@@ -366,7 +390,27 @@ class Cache:
         dev = self.khat.device
         _same_device(dev, **{f"cache.{n}": getattr(self, n) for n in names})
         ptrs = [_ptr(getattr(self, n)).value for n in names]
-        return ua_cache(self.B, self.Hkv, self.d, self.capacity, _dtype_code(self.dtype), int(self.kv_rep), *ptrs)
+        if not paged:
+            return ua_cache(self.B, self.Hkv, self.d, self.capacity, _dtype_code(self.dtype), int(self.kv_rep), *ptrs)
+        max_pages = self.capacity // self.page_size
+        _need("cache.page_table", self.page_table, self.B * self.Hkv * max_pages, I32)
+        _same_device(dev, **{"cache.page_table": self.page_table})
+        return ua_cache(self.B, self.Hkv, self.d, self.capacity, _dtype_code(self.dtype), int(self.kv_rep), *ptrs,
+                        self.page_size, max_pages, self.pool_pages, _ptr(self.page_table).value)
+
+    def logical(self, name: str) -> torch.Tensor:
+        """A cache array in the contiguous layout [B, Hkv, capacity(, d)] (a copy for a paged cache,
+        slots without a page read as zeros)."""
+        t = getattr(self, name)
+        if self.page_table is None:
+            return t
+        ps = self.page_size
+        s = torch.arange(self.capacity, device=t.device)
+        pg = self.page_table[:, s // ps].long()                     # [B*Hkv, capacity]
+        idx = pg * ps + (s % ps)
+        out = t[idx.clamp(min=0)]
+        out[pg < 0] = 0
+        return out.reshape(self.B, self.Hkv, self.capacity, *t.shape[1:])
 
     def nbytes_per_entry(self) -> int:
         return 2 * self.d * self.khat.element_size() + 12
@@ -377,6 +421,50 @@ class Cache:
 
 
 FIELDS = ("khat", "v", "bias", "rk", "pos", "n_kept")
+
+
+class PagePool:
+    """Host-side page allocator of a paged Cache (argument marshalling: it only edits the page
+    table).  ensure(n) gives every cache u pages for its slots [0, n[u]); release() hands the pages
+    past each cache's live pairs (ceil(n_kept / page_size)) back to the pool, as a compaction
+    leaves them empty.  Both read or write the table with one host<->device copy."""
+
+    def __init__(self, cache: Cache):
+        if cache.page_table is None:
+            raise ValueError("PagePool needs a paged Cache")
+        self.cache = cache
+        self.ps = cache.page_size
+        self.table = cache.page_table.cpu().numpy().copy()
+        used = set(int(x) for x in self.table.ravel() if x >= 0)
+        self.free = [pg for pg in range(cache.pool_pages - 1, -1, -1) if pg not in used]
+
+    def pages_in_use(self) -> int:
+        return int((self.table >= 0).sum())
+
+    def _upload(self):
+        self.cache.page_table.copy_(torch.from_numpy(self.table))
+
+    def ensure(self, n_slots):
+        """n_slots: per cache (an int for all, or [B, Hkv] / [B*Hkv]) the slots that need pages."""
+        import numpy as np
+        want = np.broadcast_to(np.asarray(n_slots, dtype=np.int64).reshape(-1), (self.table.shape[0],))
+        for u, n in enumerate(want):
+            for pg in range((int(n) + self.ps - 1) // self.ps):
+                if self.table[u, pg] < 0:
+                    if not self.free:
+                        raise RuntimeError("page pool exhausted")
+                    self.table[u, pg] = self.free.pop()
+        self._upload()
+
+    def release(self):
+        """Return the pages past each cache's live pairs (reads n_kept)."""
+        n = self.cache.n_kept.reshape(-1).cpu().numpy()
+        for u, k in enumerate(n):
+            for pg in range((int(k) + self.ps - 1) // self.ps, self.table.shape[1]):
+                if self.table[u, pg] >= 0:
+                    self.free.append(int(self.table[u, pg]))
+                    self.table[u, pg] = -1
+        self._upload()
 
 
 def cache_fill(cache: Cache, k, v, a_k, b_final, *, theta=500000.0, stream=None):

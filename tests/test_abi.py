@@ -148,6 +148,13 @@ def test_cache_calls_reject_bad_arguments(lib):
     for rep in (3, -1):
         cr = ua.ua_cache(2, 2, 64, 100, ua.UA_BF16, rep, *([FAKE] * 6))
         assert lib.ua_cache_compact(ctypes.byref(cr), None, ctypes.c_float(0.1), None, None) == 1
+    # paged storage: page size a power of two >= 128, capacity = max_pages * page_size, a pool,
+    # an aligned table
+    for ps_, mp, pp, tab, want in ((100, 1, 4, FAKE, 1), (64, 2, 4, FAKE, 1), (128, 2, 4, FAKE, 1),
+                                   (128, 1, 0, FAKE, 1), (128, 1, 4, FAKE + 2, 3)):
+        cpg = ua.ua_cache(2, 2, 64, 128 if want == 1 and mp == 2 else ps_ * mp, ua.UA_BF16, 1, *([FAKE] * 6),
+                          ps_, mp, pp, tab)
+        assert lib.ua_cache_compact(ctypes.byref(cpg), None, ctypes.c_float(0.1), None, None) == want, (ps_, mp, pp)
     c3 = ua.ua_cache(2, 2, 80, 100, ua.UA_BF16, 1, *([FAKE] * 6))
     assert lib.ua_decode_step(ctypes.byref(c3), 8, *args, 5, ctypes.c_float(0.1), ctypes.c_float(0.125), 5e5,
                               P(FAKE), None, None, 0, None) == 2
