@@ -43,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 MUFU_PER_CLK_SM = 16   # transcendental (exp2/log2) results per clock per SM: 4 per SM sub-partition
 # DRAM bytes (read + written) per launch of the dominant kernel, from the ncu capture summarised
 # in profiles/k_fwd_tc_prefill_1b.md; valid only for the kernel version that capture was taken of
-TRAFFIC_BYTES = {"k_fwd_tc": 922.77e6 + 149.78e6}   # ncu dram bytes read + written, one launch (profiles/)
+TRAFFIC_BYTES = {"k_fwd_tc": 922.77e6 + 149.78e6}   # ncu dram bytes read + written of one launch
 N_SM = 148
 
 
