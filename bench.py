@@ -692,12 +692,13 @@ def time_prefill(w, x, steps, warmup, prune_p=0.0, want_bfinal=True):
 
 def bench_prefill_more(args, peaks, peaks_kind, mhz):
     """The other prefill configurations: the 16k-token long-context prefill (B=1, bimodal a_k,
-    b_final emitted) and the chunked pruned prefill of the 1B workload at p = 0.05 and 0.15
-    (128-token chunks), each with the roofline of its fused kernel."""
+    b_final emitted), the chunked pruned prefill of the 1B workload at p = 0.05 and 0.15 and of
+    the 3B-shaped forward (head_dim 128) at p = 0.15 (128-token chunks), each with the roofline
+    of its fused kernel where it is the head_dim-64 one."""
     res = {}
     peak_t = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     peak_a = MUFU_PER_CLK_SM * N_SM * (mhz or 1965.0) * 1e6 / 1e9
-    cases = [("prefill_1b_16k", 0.0)] + [("prefill_1b", p) for p in I.DECODE_THRESHOLDS]
+    cases = [("prefill_1b_16k", 0.0)] + [("prefill_1b", p) for p in I.DECODE_THRESHOLDS] + [("fwdbwd_3b", 0.15)]
     for wname, p in cases:
         w = I.WORKLOADS[wname]
         x = I.make_prefill_inputs_torch(w, "cuda")
@@ -722,7 +723,7 @@ def bench_prefill_more(args, peaks, peaks_kind, mhz):
                 "tensor": {"achieved": f_exec / (kms * 1e-3) / 1e12, "peak": peak_t, "unit": "TFLOP/s",
                            "frac": f_exec / (kms * 1e-3) / 1e12 / peak_t,
                            "dense_equiv_frac": F / (kms * 1e-3) / 1e12 / peak_t}}
-        res[f"{wname}" + (f"_pruned_p{p:g}" if p > 0 else "")] = entry
+        res[("prefill_3b" if wname == "fwdbwd_3b" else wname) + (f"_pruned_p{p:g}" if p > 0 else "")] = entry
         del x
         torch.cuda.empty_cache()
     return res

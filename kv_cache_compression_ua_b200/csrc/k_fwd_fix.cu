@@ -159,6 +159,10 @@ __global__ void __launch_bounds__(kFixThreads) k_fwd_fix(FixParams p) {
         __syncthreads();
         const float al = p.alpha[kvh], be = p.beta[kvh];
         const float* pin = p.pincl + ((size_t)unit * p.nqt + (t > 0 ? t - 1 : 0)) * p.Tpk;
+        // chunked pruning decides at the start of the row's 128-row chunk, c0: the prefix published
+        // by the query tile that ends there (the row's own tile's Pb when the tiles are 128 rows)
+        const int c0 = (i / 128) * 128;
+        const float* pinc = p.pincl + ((size_t)unit * p.nqt + (c0 > 0 ? c0 / p.QT - 1 : 0)) * p.Tpk;
         float* sc = p.scratch + (size_t)blockIdx.x * T;
         // ---- pass 1: logits (with the row's Lambda) and their maximum
         float mx = -INFINITY;
@@ -169,7 +173,7 @@ __global__ void __launch_bounds__(kFixThreads) k_fwd_fix(FixParams p) {
             const bool before = j < r0;
             const float pb = before ? pin[j] : 0.f;
             float lg;
-            if (before && pb > p.prune_thr) {
+            if (j < c0 && pinc[j] > p.prune_thr) {
                 lg = -INFINITY;                           // evicted at the chunk boundary
             } else {
                 float a = pb;

@@ -120,6 +120,7 @@ struct Smem {
     alignas(128) float mq[G][QR];            // row bound M_i (log2 units) per head
     alignas(128) float lk[128];              // lk2 of the key tile
     alignas(16) float pb[2][128];            // boundary prefix Pb of the key tile, two stages
+    alignas(16) float pbc[2][128];           // chunked pruning: the prefix at the 128-row chunk's start
     int pbskip[2];                           // 0 compute; 1 softmax skipped; 2 decay skipped too
     alignas(16) float pinc[2][128];          // inclusive prefix handed to the publisher warp
     alignas(16) float tot[3][NWG][128];      // per-quarter column sums (without the key factor), ring of 3
@@ -156,6 +157,7 @@ struct FwdTc128Params {
     unsigned* flags;     // [B*Hkv][nqt][nkt] publication counters; then ticket, skip counter
     float* b_final;      // [B*Hkv][T] or NULL
     int nunits;          // B * Hkv
+    float prune_thr;     // chunked pruned prefill (128-row chunks): -log p, +inf = dense
     unsigned* fix_count; // rows whose shifted row sum fell below 2^-60, listed for k_fwd_fix
     int* fix_list;       // (b*H + h)*T + i per listed row
 };
@@ -372,18 +374,33 @@ k_fwd_tc128(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__ 
         auto fetch = [&](int kt) -> bool {
             const int sb = kt & 1;
             if (kt >= 2 && !mbar_wait(&S.pbempty[sb], ((kt >> 1) - 1) & 1, abort)) return false;
-            float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f), c4 = v4;
             int skip = 0;
             if (qt >= 1 && kt <= ((qt - 1) >> 1)) {      // the previous query tile covered kt
                 const size_t row = (size_t)unit * p.nqt + (qt - 1);
                 if (!wait_counter128(p.flags + row * p.nkt + kt, 1u, abort, lane)) return false;
                 v4 = __ldcg(reinterpret_cast<const float4*>(p.pincl + row * p.Tpk + (size_t)kt * 128) + lane);
+                // Chunked pruning decides at the start of the 128-row chunk: for the chunk's first
+                // 64-row tile that is Pb itself; the second reads what the tile two back published
+                // (complete: the tile before waited on it for this key tile before publishing).
+                // The chunk's own key tile (kt = qt / 2) is never pruned.
+                c4 = v4;
+                if ((qt & 1) && kt < (qt >> 1))
+                    c4 = qt >= 3 ? __ldcg(reinterpret_cast<const float4*>(
+                                       p.pincl + (row - 1) * p.Tpk + (size_t)kt * 128) + lane)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
                 float mn = fminf(fminf(v4.x, v4.y), fminf(v4.z, v4.w));
+                float mc = fminf(fminf(c4.x, c4.y), fminf(c4.z, c4.w));
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                skip = (mn * kLog2e128 >= kSkipLog2_128) ? (EARLY ? 2 : 1) : 0;
+                for (int o = 16; o > 0; o >>= 1) {
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                    mc = fminf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+                }
+                const bool pruned = kt < (qt >> 1) && mc > p.prune_thr;   // every key of the tile evicted
+                skip = (mn * kLog2e128 >= kSkipLog2_128 || pruned) ? (EARLY ? 2 : 1) : 0;
             }
             *reinterpret_cast<float4*>(&S.pb[sb][lane * 4]) = v4;
+            *reinterpret_cast<float4*>(&S.pbc[sb][lane * 4]) = c4;
             if (lane == 0) {
                 S.pbskip[sb] = skip;
                 if (skip) atomicAdd(p.flags + (size_t)p.nunits * p.nqt * p.nkt + 1, 1u);
@@ -561,10 +578,11 @@ k_fwd_tc128(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__ 
             const bool diag = (kt == ktd);
             const bool tailq = i0 + QR > T;
             int code = 0;
-            float pbj = 0.f;
+            float pbj = 0.f, pbcj = 0.f;
             auto take_pb = [&]() -> bool {
                 if (!mbar_wait(&S.pbfull[kt & 1], (kt >> 1) & 1, abort)) return false;
                 pbj = S.pb[kt & 1][jl];
+                pbcj = S.pbc[kt & 1][jl];
                 code = S.pbskip[kt & 1];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.pbempty[kt & 1]);
@@ -621,6 +639,10 @@ k_fwd_tc128(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__ 
             const float ka = -rk3 * kLog2e128, kb = -fmaf(rk3, above, pbj) * kLog2e128 - S.shift[warp];
 #pragma unroll
             for (int r = 0; r < 16; ++r) lam[r] = fmaf(lam[r], ka, kb);
+            if (!diag && pbcj > p.prune_thr) {           // key evicted at this chunk's start
+#pragma unroll
+                for (int r = 0; r < 16; ++r) lam[r] = -INFINITY;
+            }
             // ---- per head: P = 2^(S*scale*log2e + Lambda - shift), causally masked
 #pragma unroll 1
             for (int h = 0; h < G && ok; ++h) {
@@ -732,7 +754,7 @@ cudaError_t launch_fwd_tc128(const FwdTcLaunch& L, cudaStream_t s) {
     p.nkt = (L.T + 127) / 128;
     p.scale_log2e = L.scale * kLog2e128;
     p.alpha = L.alpha; p.beta = L.beta; p.g = L.g; p.o = L.o; p.lse = L.lse;
-    p.pincl = L.pincl; p.flags = L.flags; p.b_final = L.b_final; p.nunits = BK;
+    p.pincl = L.pincl; p.flags = L.flags; p.b_final = L.b_final; p.nunits = BK; p.prune_thr = L.prune_thr;
     p.fix_count = L.fix_count; p.fix_list = L.fix_list;
     switch (L.H / L.Hkv) {
         case 1: return fwd_tc128_inst<1>(m, p, s);

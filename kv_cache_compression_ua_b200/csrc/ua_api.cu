@@ -128,12 +128,10 @@ TcWs tc_ws_layout(const ua_shape* s) {
 
 // The tensor-core forward evaluates the three-rate geometric mean only (its decay runs in
 // log2 units with the cube root folded in); a shape with a mechanism switched off runs SIMT.
-// The head_dim-128 kernel does not take the chunked pruned prefill (its 64-row query tiles are
-// half a pruning chunk), so such calls run SIMT too.
 bool use_tc(const ua_shape* s) {
     // (the rows listed for the exact recomputation are indexed by (b*H + h)*T + i in an int)
     return s->dtype == UA_BF16 && fwd_tc_supported(s->d, s->H / s->Hkv) && (s->variant & kVarMech) == 0 &&
-           (s->d == 64 || s->prune_p == 0.f) && (size_t)s->B * s->H * s->T < (size_t)INT32_MAX;
+           (size_t)s->B * s->H * s->T < (size_t)INT32_MAX;
 }
 
 size_t prefill_ws_bytes(const ua_shape* s) {

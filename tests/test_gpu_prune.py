@@ -131,13 +131,18 @@ def test_bf16_pruning_skips_more_tiles():
     assert skipped[1] > skipped[0], skipped
 
 
-def test_bf16_d128_runs_simt_path():
-    w = I.Workload("prune", 1, 400, 6, 2, 128, "bf16", 1500)
+@pytest.mark.parametrize("B,T,H,Hkv,p", [(1, 400, 6, 2, 0.15), (1, 1000, 3, 1, 0.05), (2, 333, 6, 2, 0.5)])
+@pytest.mark.parametrize("want_bfinal", [True, False])
+def test_bf16_d128_tensor_core_path(B, T, H, Hkv, p, want_bfinal):
+    """head_dim 128: 64-row query tiles, so the second tile of each 128-row chunk takes its
+    eviction decisions from the prefix published by the tile two back (the chunk's start)."""
+    w = I.Workload("prune", B, T, H, Hkv, 128, "bf16", 1500 + T)
     x = I.make_prefill_inputs(w)
-    r, dense = oracle_pair(w, x, 0.15)
-    g, names = kernels_ran(lambda: run(w, x, 0.15))
-    assert "k_fwd_simt" in names
-    check(w, g, r, r["lam"], 0.15, dense["b_final"])
+    r, dense = oracle_pair(w, x, p)
+    g, names = kernels_ran(lambda: run(w, x, p, want_bfinal=want_bfinal))
+    assert "k_fwd_tc128" in names and "k_fwd_simt" not in names, names
+    assert ua.get_device_status() == 0
+    check(w, g, r, r["lam"], p, dense["b_final"])
 
 
 @pytest.mark.parametrize("dtype,variant,kernel", [("bf16", ua.VAR_QUERY_NORM, "k_fwd_tc"),
