@@ -929,9 +929,15 @@ __global__ void __launch_bounds__(256) k_bwd_post_tc(BwdTcParams p) {
     constexpr int HALF = DH / 2;
     const int t = blockIdx.x, b = blockIdx.y, T = p.T;
     __shared__ float s_cos[64], s_sin[64];
-    for (int m = threadIdx.x; m < HALF; m += blockDim.x) rope_cs((double)t, p.rf.f[m], &s_cos[m], &s_sin[m]);
-    __syncthreads();
+    __shared__ double s_f[HALF];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the RoPE frequencies, a few per warp (a kernel-parameter array read at a different index by
+    // each lane serialises those reads)
+    static_assert(HALF % 8 == 0, "frequencies split over the eight warps");
+    if (lane < HALF / 8) s_f[warp * (HALF / 8) + lane] = p.rf.f[warp * (HALF / 8) + lane];
+    __syncthreads();
+    for (int m = threadIdx.x; m < HALF; m += blockDim.x) rope_cs((double)t, s_f[m], &s_cos[m], &s_sin[m]);
+    __syncthreads();
     using bf = __nv_bfloat16;
     bf* dq = static_cast<bf*>(p.dq);
     bf* dk = static_cast<bf*>(p.dk);

@@ -15,6 +15,8 @@
 
 namespace ua {
 
+constexpr int kPrepTokens = 16;   // tokens per CTA of the token preparation
+
 // ------------------------------------------------------------------ token preparation
 // 8 consecutive activations <-> float registers (16-byte bf16 or 2 x 16-byte f32 accesses).
 template <typename T> struct Vec8;
@@ -38,13 +40,19 @@ template <> struct Vec8<float> {
 // the CH = d/16 tasks of a head sit on consecutive lanes, which reduce the head's norm.
 template <typename TI, typename TW, int DH>
 __global__ void __launch_bounds__(256) k_prep(PrepParams p) {
-    constexpr int TB = 4, HALF = DH / 2, CH = HALF / 8;
+    constexpr int TB = kPrepTokens, HALF = DH / 2, CH = HALF / 8;
     __shared__ float s_cos[TB][HALF], s_sin[TB][HALF];
+    __shared__ double s_f[HALF];
     const int t0 = blockIdx.x * TB, b = blockIdx.y, T = p.T;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // the RoPE frequencies, a few per warp (a kernel-parameter array read at a different index by
+    // each lane serialises those reads)
+    static_assert(HALF % 8 == 0, "frequencies split over the eight warps");
+    if (lane < HALF / 8) s_f[warp * (HALF / 8) + lane] = p.rf.f[warp * (HALF / 8) + lane];
+    __syncthreads();
     for (int e = tid; e < TB * HALF; e += blockDim.x) {
         const int tk = e / HALF, m = e % HALF;
-        rope_cs((double)(t0 + tk), p.rf.f[m], &s_cos[tk][m], &s_sin[tk][m]);
+        rope_cs((double)(t0 + tk), s_f[m], &s_cos[tk][m], &s_sin[tk][m]);
     }
     __syncthreads();
     const int nh = p.H + p.Hkv;
@@ -402,7 +410,7 @@ __global__ void __launch_bounds__(256) k_fwd_simt(FwdParams p) {
 // ------------------------------------------------------------------ launchers
 template <int DH>
 static void prep_inst(const PrepParams& p, bool bf16_in, bool bf16_work, cudaStream_t s) {
-    dim3 grid((p.T + 3) / 4, p.B);
+    dim3 grid((p.T + kPrepTokens - 1) / kPrepTokens, p.B);
     if (bf16_in && bf16_work) k_prep<__nv_bfloat16, __nv_bfloat16, DH><<<grid, 256, 0, s>>>(p);
     else if (bf16_in) k_prep<__nv_bfloat16, float, DH><<<grid, 256, 0, s>>>(p);
     else if (bf16_work) k_prep<float, __nv_bfloat16, DH><<<grid, 256, 0, s>>>(p);
