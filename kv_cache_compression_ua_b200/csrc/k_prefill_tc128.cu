@@ -678,17 +678,21 @@ k_fwd_tc128(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__ 
             const float sh = S.shift[4 * wg];
 #pragma unroll 1
             for (int h = 0; h < G && lok; ++h) {
-                float o[16];
-                tmem_ld16(tmem + tlane + COL_O + h * 64 + wg * 16, o);
                 const int hq = kvh * G + h;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float o[8];
+                    tmem_ld8(tmem + tlane + COL_O + h * 64 + wg * 16 + half * 8, o);
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const int i = i0 + r0 + r;
-                    if (i < T) {
-                        const float l = S.lsum[h][r0 + r];
-                        const size_t off = (((size_t)b * T + i) * p.H + hq) * 128 + jl;
-                        const float gv = __bfloat162float(static_cast<const __nv_bfloat16*>(p.g)[off]);
-                        static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(o[r] / l * sigmoid_f(gv));
+                    for (int r8 = 0; r8 < 8; ++r8) {
+                        const int r = half * 8 + r8;
+                        const int i = i0 + r0 + r;
+                        if (i < T) {
+                            const float l = S.lsum[h][r0 + r];
+                            const size_t off = (((size_t)b * T + i) * p.H + hq) * 128 + jl;
+                            const float gv = __bfloat162float(static_cast<const __nv_bfloat16*>(p.g)[off]);
+                            static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(o[r8] / l * sigmoid_f(gv));
+                        }
                     }
                 }
                 if (wq == 0 && lane < 16) {
