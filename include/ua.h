@@ -312,9 +312,11 @@ ua_status ua_decode_step(const ua_cache* cache, int H, const void* q, const void
                          int flags, void* stream);
 
 /* ------------------------------------------------------------------ split decode step
- * The same step as ua_decode_step with UA_DECODE_DEFER_COMPACT (set or not in flags), for few
- * long caches: a cache of n live slots is walked by min(16, ceil(n / 512)) CTAs at once, each
- * over a slice of whole 32-slot words, instead of by one (the pages' App. H asks for fused,
+ * The same step as ua_decode_step with UA_DECODE_DEFER_COMPACT (set or not in flags), for long
+ * caches: a cache of n live slots is walked by several CTAs at once instead of by one -- bf16
+ * caches by min(S, ceil(n / 256)) CTAs over slices of whole 128-slot tiles, S (at most 64) chosen
+ * on the host from the number of caches and their capacity; fp32 caches by min(16, ceil(n / 512))
+ * CTAs over slices of whole 32-slot words (the pages' App. H asks for fused,
  * specialised kernels for the pruned cache; a single CTA per cache leaves most of the GPU idle
  * when B * Hkv is small and the caches long).  Each CTA updates its slots' biases in place and
  * leaves a partial softmax state in the workspace; the last one to finish merges them with the
@@ -324,7 +326,7 @@ ua_status ua_decode_step(const ua_cache* cache, int H, const void* q, const void
  * its first use (and again after using it for anything else): its first 4 x B x Hkv bytes are
  * per-cache arrival counters, which every step leaves zero, so consecutive steps need no memset
  * between their kernels (a counter found already at the grid's size raises UA_ERR_INVALID_ARG in
- * the device status).  Calls that share a workspace must not overlap on the GPU.  A short cache (n <= 512) takes one slice.
+ * the device status).  Calls that share a workspace must not overlap on the GPU.
  * bf16 caches run on the tensor cores: per 128-entry tile one tcgen05 product gives every
  * entry's similarity and G logits (the new key and the rotated queries enter as bf16 high parts
  * plus residuals), a thread per entry turns them into the decay, the bias, the eviction and the
