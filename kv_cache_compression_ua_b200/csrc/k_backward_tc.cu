@@ -160,6 +160,21 @@ __device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) 
     }
     return v[0];
 }
+// 16 rows over the warp's 32 lanes: lane t gets the sum of row t % 16 over all 32 lanes (the
+// halving exchanges of warp_transpose_sum32 for bits 3..0, then the two 16-lane halves added).
+__device__ __forceinline__ float warp_transpose_sum16(float (&v)[16], int lane) {
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1) {
+        const bool upper = (lane & w) != 0;
+#pragma unroll
+        for (int i = 0; i < w; ++i) {
+            const float send = upper ? v[i] : v[i + w];
+            const float keep = upper ? v[i + w] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        }
+    }
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 16);
+}
 }  // namespace
 
 // =========================================================================== prep
@@ -333,8 +348,9 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
 }
 
 // =========================================================================== key-major pass
-// grid (nkt, B*Hkv), 160 threads: warps 0-3 compute (thread = key j, TMEM lane), warp 4 issues
-// the TMA loads and the MMAs.  Steps s = nst-1 down to 4kt.  TMEM: dV (DH columns), dKrot (DH),
+// grid (nkt, B*Hkv), 288 threads: warps 0-7 compute (two threads per key j, TMEM lane j % 128:
+// warps 0-3 the upper 16 rows of each step, warps 4-7 the lower 16), warp 8 issues the TMA loads
+// and the MMAs.  Steps s = nst-1 down to 4kt.  TMEM: dV (DH columns), dKrot (DH),
 // the X^T slot (32), two slots for the S_h^T / dP_h^T pair of a head (64 each).
 namespace key {
 template <int DH, int G>
@@ -352,16 +368,19 @@ struct Smem {
     alignas(128) float lse2[G][ST];              // per head (with qh / ah)
     alignas(128) float dlt[G][ST];
     alignas(128) float lk[128];
-    alignas(16) float red[2][4];
+    alignas(16) float red[2][8];
+    alignas(16) float ca[2][128];                // upper half's decay totals, by step parity
+    alignas(16) float tv[2][2][128];             // each half's dLambda totals, by step parity
+    alignas(16) float dakx[2][128];              // each half's d a_k sums
     alignas(8) uint64_t kfull, qfull, qempty, xfull, xempty, hfull[G], hdone[G], pfull[2], pempty[2], tfull,
-        tempty, accdone;
+        tempty, accdone, cafull[2], tvfull[2];
     uint32_t tmem;
     int abort;
 };
 }  // namespace key
 
 template <int DH, int G>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(288, 1)
 k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__ CUtensorMap tm_krk,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_khq,
              const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ad,
@@ -384,15 +403,17 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
     if (tid == 0) {
         mbar_init(&S.kfull, 1);
         mbar_init(&S.xfull, 1);
-        mbar_init(&S.xempty, 4);
+        mbar_init(&S.xempty, 8);
         mbar_init(&S.accdone, 1);
         mbar_init(&S.qfull, 1);
-        mbar_init(&S.qempty, 4);
-        mbar_init(&S.tfull, 4);
+        mbar_init(&S.qempty, 8);
+        mbar_init(&S.tfull, 8);
         mbar_init(&S.tempty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.pfull[i], 1);
-            mbar_init(&S.pempty[i], 4);
+            mbar_init(&S.pempty[i], 8);
+            mbar_init(&S.cafull[i], 4);               // the upper half's four warps
+            mbar_init(&S.tvfull[i], 8);               // every compute warp
         }
         for (int h = 0; h < G; ++h) {
             mbar_init(&S.hfull[h], 1);
@@ -410,7 +431,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = S.tmem;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------ TMA + MMA issue (one elected lane)
         const bool leader = elect_one();
         bool ok = true;
@@ -539,16 +560,20 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         if (leader) umma_commit(&S.accdone);
         __syncwarp();
     } else {
-        // ------------------------------------------------ compute warps: thread = key j
-        const int jl = tid;
+        // ------------------------------------------------ compute warps: two threads per key j
+        // (TMEM lane jl): warps 0-3 take rows 0-15 of each 32-row step, warps 4-7 rows 16-31.  Two
+        // exchanges per step join the halves: the upper half's decay total, where the lower
+        // half's prefixes start, and both halves' dLambda totals, from which each half forms its
+        // rows' suffix sums (bottom up: the lower half's rows, then the upper half's).
+        const int jl = tid & 127, hf = tid >> 7, rb = 16 * hf;   // this thread: rows rb .. rb+15
         const int j = kt * 128 + jl;
-        const uint32_t tl = (uint32_t)(warp * 32) << 16;
+        const uint32_t tl = (uint32_t)((warp & 3) * 32) << 16;
         const float al = p.alpha[kvh], be = p.beta[kvh];
         const float al2 = al * kL2e, be2 = be * kL2e;
         const float sl = p.scale * kL2e;
         bool ok = wwait(&S.kfull, 0, abort);
         const float rk3 = ok ? ex2f(S.lk[jl]) * kCbrtLn2b : 0.f;   // r_k^(1/3) (ln 2)^(1/3)
-        float carry = 0.f;                            // sum of dLambda over the rows below (dD = -carry)
+        float carry = 0.f;                            // sum of dLambda over the rows below the step
         float dak = 0.f, dal = 0.f, dbe = 0.f;
         const size_t tstride = (size_t)p.ntiles * kTileBytes;      // bytes per stored tile set
         uint8_t* tile_base = static_cast<uint8_t*>(p.tiles) + (size_t)unit * (G + 1) * tstride;
@@ -556,37 +581,31 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         for (int it = 0; ok && it < nsteps; ++it) {
             const int s = p.nst - 1 - it;
             const int i0 = s * ST;
+            const int xb = it & 1;                    // exchange buffer and its phase
+            const uint32_t xph = (uint32_t)(it >> 1) & 1u;
             if (!wwait(&S.qfull, it & 1, abort)) { ok = false; break; }
             const float pbj = S.pbv[jl];
             if (!wwait(&S.xfull, it & 1, abort)) { ok = false; break; }
             tc_fence_after();
-            uint32_t x[32];
-            {
-                uint32_t (&x0)[16] = *reinterpret_cast<uint32_t(*)[16]>(&x[0]);
-                uint32_t (&x1)[16] = *reinterpret_cast<uint32_t(*)[16]>(&x[16]);
-                tmem_ld16_async(tmem + tl + COL_X, x0);
-                tmem_ld16_async(tmem + tl + COL_X + 16, x1);
-                tmem_wait16(x0);
-                tmem_wait16(x1);
-            }
-            // decay of the step's rows: Dq = D / rk3; lam = Lambda * log2(e)
-            float dqv[32], lam[32];
-            {
-                float c = 0.f;
+            uint32_t x[16];
+            tmem_ld16_async(tmem + tl + COL_X + rb, x);
+            tmem_wait16(x);
+            // decay of this half's rows: Dq = D / rk3, and their running sum from the half's first row
+            float dqv[16], csum[16];
+            float c = 0.f;
 #pragma unroll
-                for (int r = 0; r < 32; r += 4) {
-                    const float4 lv = *reinterpret_cast<const float4*>(&S.lq[r]);
-                    const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
+            for (int r = 0; r < 16; r += 4) {
+                const float4 lv = *reinterpret_cast<const float4*>(&S.lq[rb + r]);
+                const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int l = i0 + r + e;
-                        float dq = ex2f(fmaf(log2_softplus_over_ln2(fmaf(al2, __uint_as_float(x[r + e]), be2)),
-                                             0.33333334f, l4[e]));
-                        dq = (l > j && l < T) ? dq : 0.f;
-                        dqv[r + e] = dq;
-                        c += dq;
-                        lam[r + e] = -fmaf(rk3, c, pbj) * kL2e;
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const int l = i0 + rb + r + e;
+                    float dq = ex2f(fmaf(log2_softplus_over_ln2(fmaf(al2, __uint_as_float(x[r + e]), be2)),
+                                         0.33333334f, l4[e]));
+                    dq = (l > j && l < T) ? dq : 0.f;
+                    dqv[r + e] = dq;
+                    c += dq;
+                    csum[r + e] = c;
                 }
             }
             tc_fence_before();
@@ -595,30 +614,34 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 mbar_arrive(&S.xempty);
                 mbar_arrive(&S.qempty);
             }
-            float dlam[32];
+            float cbase = 0.f;                        // the decay of the step's rows above this half
+            if (hf == 0) {
+                S.ca[xb][jl] = c;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.cafull[xb]);
+            } else {
+                if (!wwait(&S.cafull[xb], xph, abort)) { ok = false; break; }
+                cbase = S.ca[xb][jl];
+            }
+            float lam[16];                            // Lambda * log2(e)
 #pragma unroll
-            for (int r = 0; r < 32; ++r) dlam[r] = 0.f;
+            for (int r = 0; r < 16; ++r) lam[r] = -fmaf(rk3, cbase + csum[r], pbj) * kL2e;
+            float dlam[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) dlam[r] = 0.f;
             const bool jv = j < T;
             for (int h = 0; h < G && ok; ++h) {
                 const uint32_t u = (uint32_t)(it * G + h), pp = u & 1;
                 if (!wwait(&S.hfull[h], it & 1, abort)) { ok = false; break; }
                 if (!wwait(&S.pfull[pp], (u >> 1) & 1, abort)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t sv[32], dpv[32];
+                uint32_t sv[16], dpv[16];
                 {
-                    uint32_t (&a0)[16] = *reinterpret_cast<uint32_t(*)[16]>(&sv[0]);
-                    uint32_t (&a1)[16] = *reinterpret_cast<uint32_t(*)[16]>(&sv[16]);
-                    uint32_t (&b0)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dpv[0]);
-                    uint32_t (&b1)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dpv[16]);
                     const uint32_t base = tmem + tl + COL_P + pp * 64;
-                    tmem_ld16_async(base, a0);
-                    tmem_ld16_async(base + 16, a1);
-                    tmem_ld16_async(base + 32, b0);
-                    tmem_ld16_async(base + 48, b1);
-                    tmem_wait16(a0);
-                    tmem_wait16(a1);
-                    tmem_wait16(b0);
-                    tmem_wait16(b1);
+                    tmem_ld16_async(base + rb, sv);
+                    tmem_ld16_async(base + 32 + rb, dpv);
+                    tmem_wait16(sv);
+                    tmem_wait16(dpv);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -629,16 +652,17 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 uint8_t* ttz = S.tz;
                 uint4* gz = reinterpret_cast<uint4*>(tile_base + (size_t)h * tstride + (band + (s - s0)) * kTileBytes);
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int c8 = 2 * hf + c2;               // the step's rows 8*c8 .. 8*c8+7
                     uint32_t wp[4], wz[4];
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
                         float pz[2], zz[2];
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {
-                            const int r = c8 * 8 + e + q;
-                            const int i = i0 + r;
-                            const float lse2 = S.lse2[h][r], dl = S.dlt[h][r];
+                            const int r = c2 * 8 + e + q;     // this half's row r = step row rb + r
+                            const int i = i0 + rb + r;
+                            const float lse2 = S.lse2[h][rb + r], dl = S.dlt[h][rb + r];
                             float pv = ex2f(fmaf(__uint_as_float(sv[r]), sl, lam[r] - lse2));
                             pv = (jv && i >= j && i < T) ? pv : 0.f;
                             const float z = pv * (__uint_as_float(dpv[r]) - dl);
@@ -663,25 +687,38 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 if (lane == 0) mbar_arrive(&S.tfull);
             }
             if (!ok) break;
-            // dD = -(sum of dLambda over the rows at and below l), bottom up; w = dD D / 3
-            float wv[32];
+            // dD = -(sum of dLambda over the rows at and below l), bottom up; w = dD D / 3.  Each
+            // half totals its rows' dLambda; with both totals every thread of the key carries the
+            // same running sum below the step.
+            float tmine = 0.f;
 #pragma unroll
-            for (int r = 31; r >= 0; --r) {
-                carry += dlam[r];
-                wv[r] = -carry * rk3 * dqv[r] * 0.33333334f;      // zero where D was masked
+            for (int r = 15; r >= 0; --r) tmine += dlam[r];
+            S.tv[xb][hf][jl] = tmine;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.tvfull[xb]);
+            if (!wwait(&S.tvfull[xb], xph, abort)) { ok = false; break; }
+            const float tlow = S.tv[xb][1][jl], tup = S.tv[xb][0][jl];
+            float cin = hf ? carry : carry + tlow;
+            carry = (carry + tlow) + tup;
+            float wv[16];
+#pragma unroll
+            for (int r = 15; r >= 0; --r) {
+                cin += dlam[r];
+                wv[r] = -cin * rk3 * dqv[r] * 0.33333334f;      // zero where D was masked
                 dak += wv[r];
             }
             {
                 uint4* gx = reinterpret_cast<uint4*>(tile_base + (size_t)G * tstride + (band + (s - s0)) * kTileBytes);
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int c8 = 2 * hf + c2;
                     uint32_t wx[4];
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
                         float xx[2];
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {
-                            const int r = c8 * 8 + e + q;
+                            const int r = c2 * 8 + e + q;
                             const float xs = __uint_as_float(x[r]);
                             float sp2, sg;
                             softplus_sigmoid(fmaf(al2, xs, be2), sp2, sg);
@@ -697,19 +734,19 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                     gx[c8 * 128 + jl] = make_uint4(wx[0], wx[1], wx[2], wx[3]);
                 }
             }
-            // row sums of w over this warp's 32 keys: lane t gets row t's sum (summed over the
-            // four warps and the key tiles, in that order, by the post pass)
-            const float rs = warp_transpose_sum32(wv, lane);
-            p.daq_part[(((size_t)unit * p.nkt + kt) * 4 + warp) * p.Tpk + i0 + lane] = rs;
+            // row sums of w over this warp's 32 keys: lane t < 16 gets row rb + t's sum (summed over
+            // the four key quarters and the key tiles, in that order, by the post pass)
+            const float rs = warp_transpose_sum16(wv, lane);
+            if (lane < 16) p.daq_part[(((size_t)unit * p.nkt + kt) * 4 + (warp & 3)) * p.Tpk + i0 + rb + lane] = rs;
         }
-        // ---- results of the key tile
+        // ---- results of the key tile: each half reads half of the dV / dKrot columns
         const bool done = ok && wwait(&S.accdone, 0, abort);
         if (done) {
             tc_fence_after();
             float* dv = p.dv32 + ((size_t)unit * T + j) * DH;
             float* dk = p.dkr + ((size_t)unit * T + j) * DH;
 #pragma unroll 1
-            for (int c = 0; c < DH; c += 16) {
+            for (int c = hf * (DH / 2); c < (hf + 1) * (DH / 2); c += 16) {
                 float a[16], k2[16];
                 tmem_ld16(tmem + tl + COL_DV + c, a);      // warp-collective: every lane loads
                 tmem_ld16(tmem + tl + COL_DK + c, k2);
@@ -722,12 +759,9 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                     }
                 }
             }
-            if (j < T) {
-                const float ak = p.a_k[((size_t)b * T + j) * p.Hkv + kvh];
-                p.dak32[(size_t)unit * T + j] = dak * sig_over_sp_f(ak);
-            }
         }
-        // dalpha / dbeta partials of the CTA
+        // d a_k of the key (both halves' sums) and the CTA's dalpha / dbeta partials
+        S.dakx[hf][jl] = dak;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             dal += __shfl_xor_sync(0xffffffffu, dal, o);
@@ -737,11 +771,21 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             S.red[0][warp] = dal;
             S.red[1][warp] = dbe;
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (done && hf == 0 && j < T) {
+            const float ak = p.a_k[((size_t)b * T + j) * p.Hkv + kvh];
+            p.dak32[(size_t)unit * T + j] = (S.dakx[0][jl] + S.dakx[1][jl]) * sig_over_sp_f(ak);
+        }
         if (tid == 0) {
             const size_t o = ((size_t)unit * p.nkt + kt) * 2;
-            p.dab[o] = S.red[0][0] + S.red[0][1] + S.red[0][2] + S.red[0][3];
-            p.dab[o + 1] = S.red[1][0] + S.red[1][1] + S.red[1][2] + S.red[1][3];
+            float sa = 0.f, sb = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                sa += S.red[0][w];
+                sb += S.red[1][w];
+            }
+            p.dab[o] = sa;
+            p.dab[o + 1] = sb;
         }
     }
     tc_fence_before();
@@ -1089,7 +1133,7 @@ static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
             cudaSuccess)
             return e;
         UA_PROFILE("k_bwd_key_tc", s);
-        k_bwd_key_tc<DH, G><<<dim3(p.nkt, BK), 160, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk,
+        k_bwd_key_tc<DH, G><<<dim3(p.nkt, BK), 288, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk,
                                                                m_pb, m_lse2, m_dlt, p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
