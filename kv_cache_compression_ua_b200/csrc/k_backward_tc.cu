@@ -160,11 +160,11 @@ __device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) 
     }
     return v[0];
 }
-// 16 rows over the warp's 32 lanes: lane t gets the sum of row t % 16 over all 32 lanes (the
-// halving exchanges of warp_transpose_sum32 for bits 3..0, then the two 16-lane halves added).
-__device__ __forceinline__ float warp_transpose_sum16(float (&v)[16], int lane) {
+// 8 rows over the warp's 32 lanes: lane t gets the sum of row t % 8 over all 32 lanes (the
+// halving exchanges of warp_transpose_sum32 for bits 2..0, then the four 8-lane groups added).
+__device__ __forceinline__ float warp_transpose_sum8(float (&v)[8], int lane) {
 #pragma unroll
-    for (int w = 8; w >= 1; w >>= 1) {
+    for (int w = 4; w >= 1; w >>= 1) {
         const bool upper = (lane & w) != 0;
 #pragma unroll
         for (int i = 0; i < w; ++i) {
@@ -173,8 +173,12 @@ __device__ __forceinline__ float warp_transpose_sum16(float (&v)[16], int lane) 
             v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
         }
     }
-    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 16);
+    float t = v[0] + __shfl_xor_sync(0xffffffffu, v[0], 8);
+    return t + __shfl_xor_sync(0xffffffffu, t, 16);
 }
+
+// Key-major pass: threads per key (each takes kKeyRows of a step's 32 rows).
+constexpr int kKeyQ = 4, kKeyRows = 32 / kKeyQ;
 }  // namespace
 
 // =========================================================================== prep
@@ -348,9 +352,8 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
 }
 
 // =========================================================================== key-major pass
-// grid (nkt, B*Hkv), 288 threads: warps 0-7 compute (two threads per key j, TMEM lane j % 128:
-// warps 0-3 the upper 16 rows of each step, warps 4-7 the lower 16), warp 8 issues the TMA loads
-// and the MMAs.  Steps s = nst-1 down to 4kt.  TMEM: dV (DH columns), dKrot (DH),
+// grid (nkt, B*Hkv), 544 threads: warps 0-15 compute (four threads per key j, TMEM lane j % 128:
+// warps 4q .. 4q+3 rows 8q .. 8q+7 of each step), warp 16 issues the TMA loads and the MMAs.  Steps s = nst-1 down to 4kt.  TMEM: dV (DH columns), dKrot (DH),
 // the X^T slot (32), two slots for the S_h^T / dP_h^T pair of a head (64 each).
 namespace key {
 template <int DH, int G>
@@ -368,10 +371,10 @@ struct Smem {
     alignas(128) float lse2[G][ST];              // per head (with qh / ah)
     alignas(128) float dlt[G][ST];
     alignas(128) float lk[128];
-    alignas(16) float red[2][8];
-    alignas(16) float ca[2][128];                // upper half's decay totals, by step parity
-    alignas(16) float tv[2][2][128];             // each half's dLambda totals, by step parity
-    alignas(16) float dakx[2][128];              // each half's d a_k sums
+    alignas(16) float red[2][4 * kKeyQ];
+    alignas(16) float ca[2][kKeyQ][128];         // each row group's decay totals, by step parity
+    alignas(16) float tv[2][kKeyQ][128];         // each row group's dLambda totals, by step parity
+    alignas(16) float dakx[kKeyQ][128];          // each row group's d a_k sums
     alignas(8) uint64_t kfull, qfull, qempty, xfull, xempty, hfull[G], hdone[G], pfull[2], pempty[2], tfull,
         tempty, accdone, cafull[2], tvfull[2];
     uint32_t tmem;
@@ -380,7 +383,7 @@ struct Smem {
 }  // namespace key
 
 template <int DH, int G>
-__global__ void __launch_bounds__(288, 1)
+__global__ void __launch_bounds__(128 * kKeyQ + 32, 1)
 k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__ CUtensorMap tm_krk,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_khq,
              const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ad,
@@ -403,17 +406,17 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
     if (tid == 0) {
         mbar_init(&S.kfull, 1);
         mbar_init(&S.xfull, 1);
-        mbar_init(&S.xempty, 8);
+        mbar_init(&S.xempty, 4 * kKeyQ);              // every compute warp, in each of these
         mbar_init(&S.accdone, 1);
         mbar_init(&S.qfull, 1);
-        mbar_init(&S.qempty, 8);
-        mbar_init(&S.tfull, 8);
+        mbar_init(&S.qempty, 4 * kKeyQ);
+        mbar_init(&S.tfull, 4 * kKeyQ);
         mbar_init(&S.tempty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.pfull[i], 1);
-            mbar_init(&S.pempty[i], 8);
-            mbar_init(&S.cafull[i], 4);               // the upper half's four warps
-            mbar_init(&S.tvfull[i], 8);               // every compute warp
+            mbar_init(&S.pempty[i], 4 * kKeyQ);
+            mbar_init(&S.cafull[i], 4 * kKeyQ);
+            mbar_init(&S.tvfull[i], 4 * kKeyQ);
         }
         for (int h = 0; h < G; ++h) {
             mbar_init(&S.hfull[h], 1);
@@ -431,7 +434,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = S.tmem;
 
-    if (warp == 8) {
+    if (warp == 4 * kKeyQ) {
         // ------------------------------------------------ TMA + MMA issue (one elected lane)
         const bool leader = elect_one();
         bool ok = true;
@@ -560,12 +563,13 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         if (leader) umma_commit(&S.accdone);
         __syncwarp();
     } else {
-        // ------------------------------------------------ compute warps: two threads per key j
-        // (TMEM lane jl): warps 0-3 take rows 0-15 of each 32-row step, warps 4-7 rows 16-31.  Two
-        // exchanges per step join the halves: the upper half's decay total, where the lower
-        // half's prefixes start, and both halves' dLambda totals, from which each half forms its
-        // rows' suffix sums (bottom up: the lower half's rows, then the upper half's).
-        const int jl = tid & 127, hf = tid >> 7, rb = 16 * hf;   // this thread: rows rb .. rb+15
+        // ------------------------------------------------ compute warps: kKeyQ threads per key j
+        // (TMEM lane jl): warps 4q .. 4q+3 take rows kKeyRows*q .. of each 32-row step.  Two
+        // exchanges per step join them: the decay totals of the row groups above, where a
+        // group's prefixes start, and every group's dLambda total, from which each forms its
+        // rows' suffix sums (bottom up: the lowest group's rows first).
+        constexpr int RQ = kKeyRows;
+        const int jl = tid & 127, qi = tid >> 7, rb = RQ * qi;   // this thread: rows rb .. rb+RQ-1
         const int j = kt * 128 + jl;
         const uint32_t tl = (uint32_t)((warp & 3) * 32) << 16;
         const float al = p.alpha[kvh], be = p.beta[kvh];
@@ -587,14 +591,14 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             const float pbj = S.pbv[jl];
             if (!wwait(&S.xfull, it & 1, abort)) { ok = false; break; }
             tc_fence_after();
-            uint32_t x[16];
-            tmem_ld16_async(tmem + tl + COL_X + rb, x);
-            tmem_wait16(x);
-            // decay of this half's rows: Dq = D / rk3, and their running sum from the half's first row
-            float dqv[16], csum[16];
+            uint32_t x[RQ];
+            tmem_ld8_async(tmem + tl + COL_X + rb, x);
+            tmem_wait8(x);
+            // decay of this group's rows: Dq = D / rk3, and their running sum from its first row
+            float dqv[RQ], csum[RQ];
             float c = 0.f;
 #pragma unroll
-            for (int r = 0; r < 16; r += 4) {
+            for (int r = 0; r < RQ; r += 4) {
                 const float4 lv = *reinterpret_cast<const float4*>(&S.lq[rb + r]);
                 const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
@@ -614,34 +618,34 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 mbar_arrive(&S.xempty);
                 mbar_arrive(&S.qempty);
             }
-            float cbase = 0.f;                        // the decay of the step's rows above this half
-            if (hf == 0) {
-                S.ca[xb][jl] = c;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.cafull[xb]);
-            } else {
-                if (!wwait(&S.cafull[xb], xph, abort)) { ok = false; break; }
-                cbase = S.ca[xb][jl];
-            }
-            float lam[16];                            // Lambda * log2(e)
+            // the decay of the step's rows above this group: the totals of the groups above
+            S.ca[xb][qi][jl] = c;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.cafull[xb]);
+            if (!wwait(&S.cafull[xb], xph, abort)) { ok = false; break; }
+            float cbase = 0.f;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) lam[r] = -fmaf(rk3, cbase + csum[r], pbj) * kL2e;
-            float dlam[16];
+            for (int q = 0; q < kKeyQ - 1; ++q)
+                if (q < qi) cbase += S.ca[xb][q][jl];
+            float lam[RQ];                            // Lambda * log2(e)
 #pragma unroll
-            for (int r = 0; r < 16; ++r) dlam[r] = 0.f;
+            for (int r = 0; r < RQ; ++r) lam[r] = -fmaf(rk3, cbase + csum[r], pbj) * kL2e;
+            float dlam[RQ];
+#pragma unroll
+            for (int r = 0; r < RQ; ++r) dlam[r] = 0.f;
             const bool jv = j < T;
             for (int h = 0; h < G && ok; ++h) {
                 const uint32_t u = (uint32_t)(it * G + h), pp = u & 1;
                 if (!wwait(&S.hfull[h], it & 1, abort)) { ok = false; break; }
                 if (!wwait(&S.pfull[pp], (u >> 1) & 1, abort)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t sv[16], dpv[16];
+                uint32_t sv[RQ], dpv[RQ];
                 {
                     const uint32_t base = tmem + tl + COL_P + pp * 64;
-                    tmem_ld16_async(base + rb, sv);
-                    tmem_ld16_async(base + 32 + rb, dpv);
-                    tmem_wait16(sv);
-                    tmem_wait16(dpv);
+                    tmem_ld8_async(base + rb, sv);
+                    tmem_ld8_async(base + 32 + rb, dpv);
+                    tmem_wait8(sv);
+                    tmem_wait8(dpv);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -652,15 +656,15 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 uint8_t* ttz = S.tz;
                 uint4* gz = reinterpret_cast<uint4*>(tile_base + (size_t)h * tstride + (band + (s - s0)) * kTileBytes);
 #pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    const int c8 = 2 * hf + c2;               // the step's rows 8*c8 .. 8*c8+7
+                for (int c2 = 0; c2 < RQ / 8; ++c2) {
+                    const int c8 = rb / 8 + c2;               // the step's rows 8*c8 .. 8*c8+7
                     uint32_t wp[4], wz[4];
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
                         float pz[2], zz[2];
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {
-                            const int r = c2 * 8 + e + q;     // this half's row r = step row rb + r
+                            const int r = c2 * 8 + e + q;     // this group's row r = step row rb + r
                             const int i = i0 + rb + r;
                             const float lse2 = S.lse2[h][rb + r], dl = S.dlt[h][rb + r];
                             float pv = ex2f(fmaf(__uint_as_float(sv[r]), sl, lam[r] - lse2));
@@ -688,21 +692,28 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             }
             if (!ok) break;
             // dD = -(sum of dLambda over the rows at and below l), bottom up; w = dD D / 3.  Each
-            // half totals its rows' dLambda; with both totals every thread of the key carries the
-            // same running sum below the step.
+            // group totals its rows' dLambda; with every total each thread of the key carries the
+            // same running sum below the step (summed in the same order everywhere).
             float tmine = 0.f;
 #pragma unroll
-            for (int r = 15; r >= 0; --r) tmine += dlam[r];
-            S.tv[xb][hf][jl] = tmine;
+            for (int r = RQ - 1; r >= 0; --r) tmine += dlam[r];
+            S.tv[xb][qi][jl] = tmine;
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.tvfull[xb]);
             if (!wwait(&S.tvfull[xb], xph, abort)) { ok = false; break; }
-            const float tlow = S.tv[xb][1][jl], tup = S.tv[xb][0][jl];
-            float cin = hf ? carry : carry + tlow;
-            carry = (carry + tlow) + tup;
-            float wv[16];
+            float cin = carry;
+            {
+                float acc = carry;
 #pragma unroll
-            for (int r = 15; r >= 0; --r) {
+                for (int q = kKeyQ - 1; q >= 0; --q) {
+                    if (q == qi) cin = acc;
+                    acc += S.tv[xb][q][jl];
+                }
+                carry = acc;
+            }
+            float wv[RQ];
+#pragma unroll
+            for (int r = RQ - 1; r >= 0; --r) {
                 cin += dlam[r];
                 wv[r] = -cin * rk3 * dqv[r] * 0.33333334f;      // zero where D was masked
                 dak += wv[r];
@@ -710,8 +721,8 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             {
                 uint4* gx = reinterpret_cast<uint4*>(tile_base + (size_t)G * tstride + (band + (s - s0)) * kTileBytes);
 #pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    const int c8 = 2 * hf + c2;
+                for (int c2 = 0; c2 < RQ / 8; ++c2) {
+                    const int c8 = rb / 8 + c2;
                     uint32_t wx[4];
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
@@ -734,19 +745,19 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                     gx[c8 * 128 + jl] = make_uint4(wx[0], wx[1], wx[2], wx[3]);
                 }
             }
-            // row sums of w over this warp's 32 keys: lane t < 16 gets row rb + t's sum (summed over
+            // row sums of w over this warp's 32 keys: lane t < RQ gets row rb + t's sum (summed over
             // the four key quarters and the key tiles, in that order, by the post pass)
-            const float rs = warp_transpose_sum16(wv, lane);
-            if (lane < 16) p.daq_part[(((size_t)unit * p.nkt + kt) * 4 + (warp & 3)) * p.Tpk + i0 + rb + lane] = rs;
+            const float rs = warp_transpose_sum8(wv, lane);
+            if (lane < RQ) p.daq_part[(((size_t)unit * p.nkt + kt) * 4 + (warp & 3)) * p.Tpk + i0 + rb + lane] = rs;
         }
-        // ---- results of the key tile: each half reads half of the dV / dKrot columns
+        // ---- results of the key tile: each group reads DH / kKeyQ of the dV / dKrot columns
         const bool done = ok && wwait(&S.accdone, 0, abort);
         if (done) {
             tc_fence_after();
             float* dv = p.dv32 + ((size_t)unit * T + j) * DH;
             float* dk = p.dkr + ((size_t)unit * T + j) * DH;
 #pragma unroll 1
-            for (int c = hf * (DH / 2); c < (hf + 1) * (DH / 2); c += 16) {
+            for (int c = qi * (DH / kKeyQ); c < (qi + 1) * (DH / kKeyQ); c += 16) {
                 float a[16], k2[16];
                 tmem_ld16(tmem + tl + COL_DV + c, a);      // warp-collective: every lane loads
                 tmem_ld16(tmem + tl + COL_DK + c, k2);
@@ -760,8 +771,8 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 }
             }
         }
-        // d a_k of the key (both halves' sums) and the CTA's dalpha / dbeta partials
-        S.dakx[hf][jl] = dak;
+        // d a_k of the key (the groups' sums) and the CTA's dalpha / dbeta partials
+        S.dakx[qi][jl] = dak;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             dal += __shfl_xor_sync(0xffffffffu, dal, o);
@@ -771,16 +782,19 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             S.red[0][warp] = dal;
             S.red[1][warp] = dbe;
         }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (done && hf == 0 && j < T) {
+        asm volatile("bar.sync 1, %0;" ::"n"(128 * kKeyQ) : "memory");
+        if (done && qi == 0 && j < T) {
+            float dsum = 0.f;
+#pragma unroll
+            for (int q = 0; q < kKeyQ; ++q) dsum += S.dakx[q][jl];
             const float ak = p.a_k[((size_t)b * T + j) * p.Hkv + kvh];
-            p.dak32[(size_t)unit * T + j] = (S.dakx[0][jl] + S.dakx[1][jl]) * sig_over_sp_f(ak);
+            p.dak32[(size_t)unit * T + j] = dsum * sig_over_sp_f(ak);
         }
         if (tid == 0) {
             const size_t o = ((size_t)unit * p.nkt + kt) * 2;
             float sa = 0.f, sb = 0.f;
 #pragma unroll
-            for (int w = 0; w < 8; ++w) {
+            for (int w = 0; w < 4 * kKeyQ; ++w) {
                 sa += S.red[0][w];
                 sb += S.red[1][w];
             }
@@ -1133,7 +1147,7 @@ static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
             cudaSuccess)
             return e;
         UA_PROFILE("k_bwd_key_tc", s);
-        k_bwd_key_tc<DH, G><<<dim3(p.nkt, BK), 288, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk,
+        k_bwd_key_tc<DH, G><<<dim3(p.nkt, BK), 128 * kKeyQ + 32, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk,
                                                                m_pb, m_lse2, m_dlt, p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
