@@ -364,8 +364,8 @@ struct Smem {
     alignas(1024) uint8_t kq[DH / 64][4096];     // khat of the step's rows, boxes [32][64]
     alignas(1024) uint8_t qh[G][DH / 64][4096];  // qrot / dA of the step's rows, per head
     alignas(1024) uint8_t ah[G][DH / 64][4096];
-    alignas(1024) uint8_t tp[kTileBytes];        // P_h^T and dZ_h^T tiles (K-major, no swizzle)
-    alignas(1024) uint8_t tz[kTileBytes];
+    alignas(1024) uint8_t tp[2][kTileBytes];     // P_h^T and dZ_h^T tiles (K-major, no swizzle),
+    alignas(1024) uint8_t tz[2][kTileBytes];     // by head parity
     alignas(128) float lq[ST];                   // log2 rate / 3 of the step's rows (with kq)
     alignas(128) float pbv[128];                 // decay prefix above the step (with kq)
     alignas(128) float lse2[G][ST];              // per head (with qh / ah)
@@ -375,8 +375,8 @@ struct Smem {
     alignas(16) float ca[2][kKeyQ][128];         // each row group's decay totals, by step parity
     alignas(16) float tv[2][kKeyQ][128];         // each row group's dLambda totals, by step parity
     alignas(16) float dakx[kKeyQ][128];          // each row group's d a_k sums
-    alignas(8) uint64_t kfull, qfull, qempty, xfull, xempty, hfull[G], hdone[G], pfull[2], pempty[2], tfull,
-        tempty, accdone, cafull[2], tvfull[2];
+    alignas(8) uint64_t kfull, qfull, qempty, xfull, xempty, hfull[G], hdone[G], pfull[2], pempty[2],
+        tfull[2], tempty[2], accdone, cafull[2], tvfull[2];
     uint32_t tmem;
     int abort;
 };
@@ -410,9 +410,9 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         mbar_init(&S.accdone, 1);
         mbar_init(&S.qfull, 1);
         mbar_init(&S.qempty, 4 * kKeyQ);
-        mbar_init(&S.tfull, 4 * kKeyQ);
-        mbar_init(&S.tempty, 1);
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.tfull[i], 4 * kKeyQ);
+            mbar_init(&S.tempty[i], 1);
             mbar_init(&S.pfull[i], 1);
             mbar_init(&S.pempty[i], 4 * kKeyQ);
             mbar_init(&S.cafull[i], 4 * kKeyQ);
@@ -480,6 +480,18 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         const uint32_t akh = smem_u32(S.khk[0]), akr = smem_u32(S.krk[0]), av = smem_u32(S.vk[0]);
         const uint32_t bq = smem_u32(S.kq[0]);
         bool first_acc = true;
+        // Head operands of the next step are copied once the head's accumulation has completed;
+        // the copy waits until the next head's products are issued (so their round trip is not
+        // behind the accumulation's), and before that head's own products at the latest.
+        int pend = -1, pit = 0;
+        auto reload = [&]() -> bool {
+            if (pend < 0) return true;
+            const int hh = pend;
+            pend = -1;
+            if (!wwait(&S.hdone[hh], pit & 1, abort)) return false;
+            load_h(pit + 1, hh);
+            return true;
+        };
         for (int it = 0; ok && it < nsteps; ++it) {
             // X^T of the step (the same bf16 unit keys as the forward, whose row normalisers the
             // probabilities are divided by)
@@ -495,11 +507,11 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             __syncwarp();
             // accumulation of head hh of this step: dV += P^T dA, dKrot += dZ^T qrot
             auto accum = [&](int hh) -> bool {
-                const uint32_t v = (uint32_t)(it * G + hh);
-                if (!wwait(&S.tfull, v & 1, abort)) return false;
+                const uint32_t v = (uint32_t)(it * G + hh), tb = v & 1;
+                if (!wwait(&S.tfull[tb], (v >> 1) & 1, abort)) return false;
                 tc_fence_after();
                 if (leader) {
-                    const uint32_t tpa = smem_u32(S.tp), tza = smem_u32(S.tz);
+                    const uint32_t tpa = smem_u32(S.tp[tb]), tza = smem_u32(S.tz[tb]);
                     const uint32_t ba = smem_u32(S.ah[hh][0]), bqh = smem_u32(S.qh[hh][0]);
 #pragma unroll
                     for (int kk = 0; kk < ST / 16; ++kk) {
@@ -514,7 +526,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                         umma_f16(tmem + COL_DV, da, db, ID_ACC, acc);
                         umma_f16(tmem + COL_DK, dz, dq, ID_ACC, acc);
                     }
-                    umma_commit(&S.tempty);
+                    umma_commit(&S.tempty[tb]);
                     umma_commit(&S.hdone[hh]);
                 }
                 __syncwarp();
@@ -523,6 +535,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             };
             for (int h = 0; h < G && ok; ++h) {
                 const uint32_t u = (uint32_t)(it * G + h), pp = u & 1;
+                if (pend == h && !reload()) { ok = false; break; }
                 if (!wwait(&S.hfull[h], it & 1, abort)) { ok = false; break; }
                 if (u >= 2 && !wwait(&S.pempty[pp], ((u >> 1) - 1) & 1, abort)) { ok = false; break; }
                 tc_fence_after();
@@ -538,6 +551,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                     umma_commit(&S.pfull[pp]);
                 }
                 __syncwarp();
+                if (!reload()) { ok = false; break; }
                 if (h == 0 && it + 1 < nsteps) {
                     // the step's khat rows, lq and prefixes are free once the compute warps have
                     // read X^T and the vectors: copy the next step's
@@ -546,18 +560,18 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 }
                 if (h >= 1) {
                     if (!accum(h - 1)) { ok = false; break; }
-                    // head h-1's operands are free once its accumulation completed: refill them
                     if (it + 1 < nsteps) {
-                        if (!wwait(&S.hdone[h - 1], it & 1, abort)) { ok = false; break; }
-                        load_h(it + 1, h - 1);
+                        pend = h - 1;
+                        pit = it;
                     }
                 }
             }
             if (!ok) break;
+            if (!reload()) break;
             if (!accum(G - 1)) break;
             if (it + 1 < nsteps) {
-                if (!wwait(&S.hdone[G - 1], it & 1, abort)) break;
-                load_h(it + 1, G - 1);
+                pend = G - 1;
+                pit = it;
             }
         }
         if (leader) umma_commit(&S.accdone);
@@ -650,14 +664,10 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.pempty[pp]);
-                // the P / dZ tiles are free once the previous head's accumulation completed
-                if (u >= 1 && !wwait(&S.tempty, (u - 1) & 1, abort)) { ok = false; break; }
-                uint8_t* ttp = S.tp;
-                uint8_t* ttz = S.tz;
                 uint4* gz = reinterpret_cast<uint4*>(tile_base + (size_t)h * tstride + (band + (s - s0)) * kTileBytes);
+                uint4 vp[RQ / 8], vz[RQ / 8];
 #pragma unroll
                 for (int c2 = 0; c2 < RQ / 8; ++c2) {
-                    const int c8 = rb / 8 + c2;               // the step's rows 8*c8 .. 8*c8+7
                     uint32_t wp[4], wz[4];
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
@@ -679,16 +689,25 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                         wp[e >> 1] = *reinterpret_cast<uint32_t*>(&bp);
                         wz[e >> 1] = *reinterpret_cast<uint32_t*>(&bz);
                     }
-                    const uint4 vp = make_uint4(wp[0], wp[1], wp[2], wp[3]);
-                    const uint4 vz = make_uint4(wz[0], wz[1], wz[2], wz[3]);
+                    vp[c2] = make_uint4(wp[0], wp[1], wp[2], wp[3]);
+                    vz[c2] = make_uint4(wz[0], wz[1], wz[2], wz[3]);
+                    gz[(rb / 8 + c2) * 128 + jl] = vz[c2];
+                }
+                // the tile pair of this parity is free once the accumulation of head u-2 completed
+                const uint32_t tb = u & 1;
+                if (u >= 2 && !wwait(&S.tempty[tb], ((u >> 1) - 1) & 1, abort)) { ok = false; break; }
+                uint8_t* ttp = S.tp[tb];
+                uint8_t* ttz = S.tz[tb];
+#pragma unroll
+                for (int c2 = 0; c2 < RQ / 8; ++c2) {
                     // core matrix (8 keys x 8 rows): rows 8*c8.., this key's 16-byte line
-                    *reinterpret_cast<uint4*>(ttp + c8 * 2048 + jl * 16) = vp;
-                    *reinterpret_cast<uint4*>(ttz + c8 * 2048 + jl * 16) = vz;
-                    gz[c8 * 128 + jl] = vz;
+                    const int c8 = rb / 8 + c2;
+                    *reinterpret_cast<uint4*>(ttp + c8 * 2048 + jl * 16) = vp[c2];
+                    *reinterpret_cast<uint4*>(ttz + c8 * 2048 + jl * 16) = vz[c2];
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S.tfull);
+                if (lane == 0) mbar_arrive(&S.tfull[tb]);
             }
             if (!ok) break;
             // dD = -(sum of dLambda over the rows at and below l), bottom up; w = dD D / 3.  Each
