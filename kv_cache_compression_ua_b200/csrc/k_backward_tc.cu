@@ -26,6 +26,7 @@
 //   k_bwd_keygemm_tc per (batch, KV head, key tile): the key-side dkhat = alpha dX^T khat
 //   k_bwd_post_tc    RoPE^T, the normalisation Jacobians, casts, da_q / da_k
 // Every sum runs in a fixed order (no atomics), so the result is deterministic.
+#include <type_traits>
 #include <cudaTypedefs.h>
 
 #include "tc_common.cuh"
@@ -120,10 +121,19 @@ __host__ __device__ __forceinline__ size_t band_off(int kt, int nkt) {
     return (size_t)4 * ((size_t)kt * nkt - (size_t)kt * (kt - 1) / 2);
 }
 
-// softplus(X) / ln 2 and sigmoid(X) for t2 = X log2(e), from one exp2: e = 2^-|t2|,
-// softplus/ln2 = max(t2, 0) + log2(1 + e) (the same degree-7 fit as the forward's
-// log2_softplus_over_ln2, its argument before the final log2), sigmoid = 1/(1+e) or e/(1+e).
-__device__ __forceinline__ void softplus_sigmoid(float t2, float& sp_ln2, float& sig) {
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// For t2 = X log2(e): log2(softplus(X) / ln 2), the decay's inner term (the forward's
+// log2_softplus_over_ln2, same arithmetic), and sigmoid(X) / softplus(X), both from one exp2
+// e = 2^-|t2|.  softplus / ln2 = max(t2, 0) + e q(e) with q the degree-7 fit of log2(1 + e) / e;
+// sigmoid = 1 / (1 + e) for t2 >= 0 (where softplus / ln2 >= 1) and e / (1 + e) below, where
+// the factor e cancels against softplus = e q ln2.  So the ratio never divides by a tiny number
+// (its limit 1 as X -> -inf included).
+__device__ __forceinline__ float log2sp_and_ratio(float t2, float& ratio) {
     const float e = ex2f(-fabsf(t2));
     float q = -0.012319492176175117f;
     q = fmaf(q, e, 0.06360796093940735f);
@@ -133,9 +143,9 @@ __device__ __forceinline__ void softplus_sigmoid(float t2, float& sp_ln2, float&
     q = fmaf(q, e, 0.48006370663642883f);
     q = fmaf(q, e, -0.7213100790977478f);
     q = fmaf(q, e, 1.4426947832107544f);
-    sp_ln2 = fmaf(e, q, fmaxf(t2, 0.f));
-    const float r = __frcp_rn(1.f + e);
-    sig = t2 >= 0.f ? r : e * r;
+    const float sp2 = fmaf(e, q, fmaxf(t2, 0.f));
+    ratio = rcp_approx(fmaf(e, kLn2, kLn2) * (t2 >= 0.f ? sp2 : q));
+    return lg2f(sp2);
 }
 
 // sigmoid(x) / softplus(x), 0 where softplus underflows (the decay it multiplies is then 0 too).
@@ -608,24 +618,34 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             uint32_t x[RQ];
             tmem_ld8_async(tmem + tl + COL_X + rb, x);
             tmem_wait8(x);
-            // decay of this group's rows: Dq = D / rk3, and their running sum from its first row
-            float dqv[RQ], csum[RQ];
+            // Steps below the key tile's diagonal, inside the sequence, of a key tile inside it carry
+            // no causal or end mask (one uniform choice per step).
+            const bool interior = i0 >= kt * 128 + 128 && i0 + ST <= T && kt * 128 + 128 <= T;
+            // decay of this group's rows: Dq = D / rk3, and their running sum from its first row;
+            // sigmoid / softplus of X for dX
+            float dqv[RQ], csum[RQ], rto[RQ];
             float c = 0.f;
+            auto decay = [&](auto masked) {
 #pragma unroll
-            for (int r = 0; r < RQ; r += 4) {
-                const float4 lv = *reinterpret_cast<const float4*>(&S.lq[rb + r]);
-                const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
+                for (int r = 0; r < RQ; r += 4) {
+                    const float4 lv = *reinterpret_cast<const float4*>(&S.lq[rb + r]);
+                    const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int l = i0 + rb + r + e;
-                    float dq = ex2f(fmaf(log2_softplus_over_ln2(fmaf(al2, __uint_as_float(x[r + e]), be2)),
-                                         0.33333334f, l4[e]));
-                    dq = (l > j && l < T) ? dq : 0.f;
-                    dqv[r + e] = dq;
-                    c += dq;
-                    csum[r + e] = c;
+                    for (int e = 0; e < 4; ++e) {
+                        float dq = ex2f(fmaf(log2sp_and_ratio(fmaf(al2, __uint_as_float(x[r + e]), be2), rto[r + e]),
+                                             0.33333334f, l4[e]));
+                        if constexpr (decltype(masked)::value) {
+                            const int l = i0 + rb + r + e;
+                            dq = (l > j && l < T) ? dq : 0.f;
+                        }
+                        dqv[r + e] = dq;
+                        c += dq;
+                        csum[r + e] = c;
+                    }
                 }
-            }
+            };
+            if (interior) decay(std::false_type{});
+            else decay(std::true_type{});
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -666,33 +686,46 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                 if (lane == 0) mbar_arrive(&S.pempty[pp]);
                 uint4* gz = reinterpret_cast<uint4*>(tile_base + (size_t)h * tstride + (band + (s - s0)) * kTileBytes);
                 uint4 vp[RQ / 8], vz[RQ / 8];
+                auto probs = [&](auto masked) {
 #pragma unroll
-                for (int c2 = 0; c2 < RQ / 8; ++c2) {
-                    uint32_t wp[4], wz[4];
+                    for (int c2 = 0; c2 < RQ / 8; ++c2) {
+                        uint32_t wp[4], wz[4];
+                        float ls[8], dl[8];
 #pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        float pz[2], zz[2];
-#pragma unroll
-                        for (int q = 0; q < 2; ++q) {
-                            const int r = c2 * 8 + e + q;     // this group's row r = step row rb + r
-                            const int i = i0 + rb + r;
-                            const float lse2 = S.lse2[h][rb + r], dl = S.dlt[h][rb + r];
-                            float pv = ex2f(fmaf(__uint_as_float(sv[r]), sl, lam[r] - lse2));
-                            pv = (jv && i >= j && i < T) ? pv : 0.f;
-                            const float z = pv * (__uint_as_float(dpv[r]) - dl);
-                            dlam[r] += z;
-                            pz[q] = pv;
-                            zz[q] = z;
+                        for (int e = 0; e < 8; e += 4) {
+                            const float4 a4 = *reinterpret_cast<const float4*>(&S.lse2[h][rb + c2 * 8 + e]);
+                            const float4 d4 = *reinterpret_cast<const float4*>(&S.dlt[h][rb + c2 * 8 + e]);
+                            ls[e] = a4.x, ls[e + 1] = a4.y, ls[e + 2] = a4.z, ls[e + 3] = a4.w;
+                            dl[e] = d4.x, dl[e + 1] = d4.y, dl[e + 2] = d4.z, dl[e + 3] = d4.w;
                         }
-                        __nv_bfloat162 bp = __floats2bfloat162_rn(pz[0], pz[1]);
-                        __nv_bfloat162 bz = __floats2bfloat162_rn(zz[0], zz[1]);
-                        wp[e >> 1] = *reinterpret_cast<uint32_t*>(&bp);
-                        wz[e >> 1] = *reinterpret_cast<uint32_t*>(&bz);
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) {
+                            float pz[2], zz[2];
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const int r = c2 * 8 + e + q;     // this group's row r = step row rb + r
+                                float pv = ex2f(fmaf(__uint_as_float(sv[r]), sl, lam[r] - ls[e + q]));
+                                if constexpr (decltype(masked)::value) {
+                                    const int i = i0 + rb + r;
+                                    pv = (jv && i >= j && i < T) ? pv : 0.f;
+                                }
+                                const float z = pv * (__uint_as_float(dpv[r]) - dl[e + q]);
+                                dlam[r] += z;
+                                pz[q] = pv;
+                                zz[q] = z;
+                            }
+                            __nv_bfloat162 bp = __floats2bfloat162_rn(pz[0], pz[1]);
+                            __nv_bfloat162 bz = __floats2bfloat162_rn(zz[0], zz[1]);
+                            wp[e >> 1] = *reinterpret_cast<uint32_t*>(&bp);
+                            wz[e >> 1] = *reinterpret_cast<uint32_t*>(&bz);
+                        }
+                        vp[c2] = make_uint4(wp[0], wp[1], wp[2], wp[3]);
+                        vz[c2] = make_uint4(wz[0], wz[1], wz[2], wz[3]);
+                        gz[(rb / 8 + c2) * 128 + jl] = vz[c2];
                     }
-                    vp[c2] = make_uint4(wp[0], wp[1], wp[2], wp[3]);
-                    vz[c2] = make_uint4(wz[0], wz[1], wz[2], wz[3]);
-                    gz[(rb / 8 + c2) * 128 + jl] = vz[c2];
-                }
+                };
+                if (interior) probs(std::false_type{});
+                else probs(std::true_type{});
                 // the tile pair of this parity is free once the accumulation of head u-2 completed
                 const uint32_t tb = u & 1;
                 if (u >= 2 && !wwait(&S.tempty[tb], ((u >> 1) - 1) & 1, abort)) { ok = false; break; }
@@ -750,10 +783,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                         for (int q = 0; q < 2; ++q) {
                             const int r = c2 * 8 + e + q;
                             const float xs = __uint_as_float(x[r]);
-                            float sp2, sg;
-                            softplus_sigmoid(fmaf(al2, xs, be2), sp2, sg);
-                            const float ratio = sp2 > 0.f ? sg * __frcp_rn(sp2 * kLn2) : 0.f;
-                            const float dX = wv[r] * ratio;
+                            const float dX = wv[r] * rto[r];
                             dal = fmaf(dX, xs, dal);
                             dbe += dX;
                             xx[q] = dX;
