@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(256) k_bwd_prep_tc(BwdTcParams p) {
 }
 
 // =========================================================================== boundary pass
-// grid (nkt, B*Hkv), 128 threads = one thread per key of the tile.  Steps s = 4kt .. nst-1 top
+// grid (B*Hkv, nkt), 128 threads = one thread per key of the tile.  Steps s = 4kt .. nst-1 top
 // down: Pb[s][j] = sum_{j < l < 32 s} D[l, j] is written, then the step's X^T tile (tensor cores,
 // two TMEM slots so the next step's MMA overlaps this step's decay) adds its rows.
 namespace bnd {
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
     using SM = bnd::Smem<DH>;
     SM& S = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int kt = blockIdx.x, unit = blockIdx.y, kvh = unit % p.Hkv;
+    const int kt = blockIdx.y, unit = blockIdx.x, kvh = unit % p.Hkv;   // longest key tiles first
     const int T = p.T;
     const int s0 = 4 * kt, nsteps = p.nst - s0;
     volatile int* abort = &S.abort;
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
 }
 
 // =========================================================================== key-major pass
-// grid (nkt, B*Hkv), 544 threads: warps 0-15 compute (four threads per key j, TMEM lane j % 128:
+// grid (B*Hkv, nkt), 544 threads: warps 0-15 compute (four threads per key j, TMEM lane j % 128:
 // warps 4q .. 4q+3 rows 8q .. 8q+7 of each step), warp 16 issues the TMA loads and the MMAs.  Steps s = nst-1 down to 4kt.  TMEM: dV (DH columns), dKrot (DH),
 // the X^T slot (32), two slots for the S_h^T / dP_h^T pair of a head (64 each).
 namespace key {
@@ -409,7 +409,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
     using SM = key::Smem<DH, G>;
     SM& S = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int kt = blockIdx.x, unit = blockIdx.y, kvh = unit % p.Hkv, b = unit / p.Hkv;
+    const int kt = blockIdx.y, unit = blockIdx.x, kvh = unit % p.Hkv, b = unit / p.Hkv;   // longest first
     const int T = p.T;
     const int s0 = 4 * kt, nsteps = p.nst - s0;
     volatile int* abort = &S.abort;
@@ -867,6 +867,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
 // dims run along the TMEM lanes (head_dim 64 uses the lower 64: the upper half of the A operand
 // points at a zero block).  Key side: per (key tile kt, unit): C[128 keys x dims] = sum_{rb >= kt}
 // dX^T_(kt, rb) khat_rb.  128 threads: warp 0 loads, warp 1 issues, all four write the result.
+// Grids (row blocks from the last, G + 1, units) and (key tiles, units).
 namespace gemm {
 constexpr int NS = 3;
 template <int DH>
@@ -890,8 +891,9 @@ k_bwd_gemm_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__
     SM& S = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NS = gemm::NS;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int blk = blockIdx.x, unit = ROWS ? blockIdx.z : blockIdx.y;
-    const int o = ROWS ? blockIdx.y : p.G;            // output: head o's dqrot, or the dkhat part
+    // row blocks from the last (the longest sums first within each unit and output)
+    const int blk = ROWS ? p.nkt - 1 - (int)blockIdx.x : (int)blockIdx.x, unit = ROWS ? blockIdx.z : blockIdx.y;
+    const int o = ROWS ? (int)blockIdx.y : p.G;       // output: head o's dqrot, or the dkhat part
     const int kvh = unit % p.Hkv, b = unit / p.Hkv;
     const int T = p.T;
     const int n = ROWS ? blk + 1 : p.nkt - blk;       // operand pairs to sum
@@ -1187,7 +1189,7 @@ static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
             cudaSuccess)
             return e;
         UA_PROFILE("k_bwd_bound_tc", s);
-        k_bwd_bound_tc<DH><<<dim3(p.nkt, BK), 128, smem, s>>>(m_khk, m_khq, m_lq, m_lk, p);
+        k_bwd_bound_tc<DH><<<dim3(BK, p.nkt), 128, smem, s>>>(m_khk, m_khq, m_lq, m_lk, p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {
@@ -1196,7 +1198,7 @@ static cudaError_t bwd_tc_inst(const BwdTcParams& p, cudaStream_t s) {
             cudaSuccess)
             return e;
         UA_PROFILE("k_bwd_key_tc", s);
-        k_bwd_key_tc<DH, G><<<dim3(p.nkt, BK), 128 * kKeyQ + 32, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk,
+        k_bwd_key_tc<DH, G><<<dim3(BK, p.nkt), 128 * kKeyQ + 32, smem, s>>>(m_khk, m_krk, m_v, m_khq, m_q, m_ad, m_lq, m_lk,
                                                                m_pb, m_lse2, m_dlt, p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
