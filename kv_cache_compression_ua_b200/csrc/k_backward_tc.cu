@@ -154,24 +154,9 @@ __device__ __forceinline__ float sig_over_sp_f(float x) {
     return sp > 0.f ? sigmoid_f(x) / sp : 0.f;
 }
 
-// Sum over the 32 lanes of a warp of v[0..31] (lane t's 32 values), transposed: on return lane t
-// holds sum over lanes of v[t] in v[0].  A butterfly that halves the vector at every level.
-__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
-#pragma unroll
-    for (int w = 16; w >= 1; w >>= 1) {
-        const bool upper = (lane & w) != 0;
-#pragma unroll
-        for (int i = 0; i < w; ++i) {
-            // keep the half selected by this lane's bit, send the other half
-            const float send = upper ? v[i] : v[i + w];
-            const float keep = upper ? v[i + w] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
-        }
-    }
-    return v[0];
-}
-// 8 rows over the warp's 32 lanes: lane t gets the sum of row t % 8 over all 32 lanes (the
-// halving exchanges of warp_transpose_sum32 for bits 2..0, then the four 8-lane groups added).
+// Sum over the 32 lanes of a warp of v[0..7] (lane t's 8 values), transposed: lane t gets the sum
+// of v[t % 8] over all lanes.  A butterfly that halves the vector at every level (each lane keeps
+// the half its bit selects and sends the other), then the four 8-lane groups added.
 __device__ __forceinline__ float warp_transpose_sum8(float (&v)[8], int lane) {
 #pragma unroll
     for (int w = 4; w >= 1; w >>= 1) {
@@ -192,8 +177,30 @@ constexpr int kKeyQ = 4, kKeyRows = 32 / kKeyQ;
 }  // namespace
 
 // =========================================================================== prep
-// grid (T, B), 256 threads: dA = dO * sigmoid(g) (bf16, [B*H][T][d] rows), Delta = sum_c dO*O and
-// lse * log2(e) per (b, h, t).
+// N consecutive bf16 (N = 2 or 4; 4N-byte aligned) to and from fp32.
+template <int N>
+__device__ __forceinline__ void ld_bf16(const __nv_bfloat16* src, float (&f)[N]) {
+    static_assert(N == 2 || N == 4, "two or four elements");
+    if constexpr (N == 4) {
+        const uint2 v = *reinterpret_cast<const uint2*>(src);
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+        f[0] = lo.x, f[1] = lo.y, f[2] = hi.x, f[3] = hi.y;
+    } else {
+        const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src));
+        f[0] = v.x, f[1] = v.y;
+    }
+}
+template <int N>
+__device__ __forceinline__ void st_bf16(__nv_bfloat16* dst, const float (&f)[N]) {
+    static_assert(N % 2 == 0, "pairs");
+#pragma unroll
+    for (int e = 0; e < N; e += 2) *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(f[e], f[e + 1]);
+}
+
+// grid (T, B), 256 threads: dA = dO * sigmoid(g) (bf16, [B*H][T][d] rows), the gate's gradient
+// dg = dO * O * (1 - sigmoid(g)) (bf16, laid out like g), Delta = sum_c dO*O and lse * log2(e) per
+// (b, h, t).
 template <int DH>
 __global__ void __launch_bounds__(256) k_bwd_prep_tc(BwdTcParams p) {
     constexpr int PER = DH / 32;
@@ -203,20 +210,24 @@ __global__ void __launch_bounds__(256) k_bwd_prep_tc(BwdTcParams p) {
     const __nv_bfloat16* dO = static_cast<const __nv_bfloat16*>(p.d_o);
     const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(p.g);
     __nv_bfloat16* ad = static_cast<__nv_bfloat16*>(p.ad);
+    __nv_bfloat16* dg = static_cast<__nv_bfloat16*>(p.dg);
     for (int h = warp; h < p.H; h += 8) {
         const size_t src = (((size_t)b * p.T + t) * p.H + h) * DH + lane * PER;
+        float fo[PER], fd[PER], fg[PER];
+        ld_bf16<PER>(dO + src, fd);
+        ld_bf16<PER>(o + src, fo);
+        ld_bf16<PER>(g + src, fg);
         float acc = 0.f;
-        float a[PER];
+        float a[PER], dgv[PER];
 #pragma unroll
         for (int e = 0; e < PER; ++e) {
-            const float dv = __bfloat162float(dO[src + e]);
-            acc = fmaf(dv, __bfloat162float(o[src + e]), acc);
-            a[e] = dv * sigmoid_f(__bfloat162float(g[src + e]));
+            acc = fmaf(fd[e], fo[e], acc);
+            const float sg = sigmoid_f(fg[e]);
+            a[e] = fd[e] * sg;
+            dgv[e] = fd[e] * fo[e] * (1.f - sg);
         }
-        const size_t dst = (((size_t)b * p.H + h) * p.T + t) * DH + lane * PER;
-#pragma unroll
-        for (int e = 0; e < PER; e += 2)
-            *reinterpret_cast<__nv_bfloat162*>(ad + dst + e) = __floats2bfloat162_rn(a[e], a[e + 1]);
+        st_bf16<PER>(ad + (((size_t)b * p.H + h) * p.T + t) * DH + lane * PER, a);
+        st_bf16<PER>(dg + src, dgv);
 #pragma unroll
         for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
         if (lane == 0) {
@@ -794,10 +805,10 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                     gx[c8 * 128 + jl] = make_uint4(wx[0], wx[1], wx[2], wx[3]);
                 }
             }
-            // row sums of w over this warp's 32 keys: lane t < RQ gets row rb + t's sum (summed over
-            // the four key quarters and the key tiles, in that order, by the post pass)
+            // row sums of w over this warp's 32 keys: lane t < RQ gets row rb + t's sum (the post pass
+            // sums the key tiles' four quarters per row)
             const float rs = warp_transpose_sum8(wv, lane);
-            if (lane < RQ) p.daq_part[(((size_t)unit * p.nkt + kt) * 4 + (warp & 3)) * p.Tpk + i0 + rb + lane] = rs;
+            if (lane < RQ) p.daq_part[(((size_t)unit * p.Tpk + i0 + rb + lane) * p.nkt + kt) * 4 + (warp & 3)] = rs;
         }
         // ---- results of the key tile: each group reads DH / kKeyQ of the dV / dKrot columns
         const bool done = ok && wwait(&S.accdone, 0, abort);
@@ -1030,12 +1041,29 @@ k_bwd_gemm_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__
 }
 
 // =========================================================================== post pass
+// N consecutive floats (N = 1 or 2).
+template <int N>
+__device__ __forceinline__ void ld_f(const float* src, float (&f)[N]) {
+    if constexpr (N == 2) {
+        const float2 v = *reinterpret_cast<const float2*>(src);
+        f[0] = v.x, f[1] = v.y;
+    } else {
+        f[0] = src[0];
+    }
+}
+template <int N>
+__device__ __forceinline__ void st_bf(__nv_bfloat16* dst, const float (&f)[N]) {
+    if constexpr (N == 2) *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(f[0], f[1]);
+    else dst[0] = __float2bfloat16_rn(f[0]);
+}
+
 // grid (T, B), 256 threads: RoPE^T of dqrot / dkrot, the query-norm and key-normalisation
-// Jacobians (khat recomputed from the raw key in fp32), casts; dg, da_q (row sums of w over the
-// key tiles, in order), da_k.
+// Jacobians (khat recomputed from the raw key in fp32), casts; da_q (row sums of w over the key
+// tiles and their quarters), da_k.  A warp per head; lane l takes the rotation pairs
+// (m, m + d/2) for m = l*PH .. l*PH+PH-1.
 template <int DH>
 __global__ void __launch_bounds__(256) k_bwd_post_tc(BwdTcParams p) {
-    constexpr int HALF = DH / 2;
+    constexpr int HALF = DH / 2, PH = HALF / 32;
     const int t = blockIdx.x, b = blockIdx.y, T = p.T;
     __shared__ float s_cos[64], s_sin[64];
     __shared__ double s_f[HALF];
@@ -1051,33 +1079,37 @@ __global__ void __launch_bounds__(256) k_bwd_post_tc(BwdTcParams p) {
     bf* dq = static_cast<bf*>(p.dq);
     bf* dk = static_cast<bf*>(p.dk);
     bf* dv = static_cast<bf*>(p.dv);
+    const int m0 = lane * PH;
+    float cs[PH], sn[PH];
+#pragma unroll
+    for (int e = 0; e < PH; ++e) cs[e] = s_cos[m0 + e], sn[e] = s_sin[m0 + e];
     for (int hh = warp; hh < p.H + p.Hkv; hh += 8) {
         const bool is_q = hh < p.H;
         const int h = is_q ? hh : hh - p.H;
         if (is_q) {
             const float* src = p.dqr + (((size_t)b * p.H + h) * T + t) * DH;
             bf* dst = dq + (((size_t)b * T + t) * p.H + h) * DH;
-            float y0[2] = {0.f, 0.f}, y1[2] = {0.f, 0.f}, q0[2] = {0.f, 0.f}, q1[2] = {0.f, 0.f};
+            float x0[PH], x1[PH], y0[PH], y1[PH], q0[PH], q1[PH];
+            ld_f<PH>(src + m0, x0);
+            ld_f<PH>(src + m0 + HALF, x1);
             float ss = 0.f, qy = 0.f;
-            const bf* qraw = static_cast<const bf*>(p.q) + (((size_t)b * T + t) * p.H + h) * DH;
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int m = lane + 32 * u;
-                if (m < HALF) {
-                    const float x0 = src[m], x1 = src[m + HALF], cs = s_cos[m], sn = s_sin[m];
-                    y0[u] = x0 * cs + x1 * sn;              // rotation by -angle
-                    y1[u] = x1 * cs - x0 * sn;
-                    if (p.variant & kVarQNorm) {
-                        q0[u] = __bfloat162float(qraw[m]);
-                        q1[u] = __bfloat162float(qraw[m + HALF]);
-                        ss += q0[u] * q0[u] + q1[u] * q1[u];
-                        qy += q0[u] * y0[u] + q1[u] * y1[u];
-                    }
-                }
+            for (int e = 0; e < PH; ++e) {
+                y0[e] = x0[e] * cs[e] + x1[e] * sn[e];          // rotation by -angle
+                y1[e] = x1[e] * cs[e] - x0[e] * sn[e];
+                q0[e] = q1[e] = 0.f;
             }
             float r = 1.f, k = 0.f;
             if (p.variant & kVarQNorm) {
                 // q' = r q, r = 1/sqrt(mean(q^2) + eps): dq = r (dq' - q' <q', dq'> / d)
+                const bf* qraw = static_cast<const bf*>(p.q) + (((size_t)b * T + t) * p.H + h) * DH;
+#pragma unroll
+                for (int e = 0; e < PH; ++e) {
+                    q0[e] = __bfloat162float(qraw[m0 + e]);
+                    q1[e] = __bfloat162float(qraw[m0 + e + HALF]);
+                    ss += q0[e] * q0[e] + q1[e] * q1[e];
+                    qy += q0[e] * y0[e] + q1[e] * y1[e];
+                }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
                     ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -1086,34 +1118,37 @@ __global__ void __launch_bounds__(256) k_bwd_post_tc(BwdTcParams p) {
                 r = 1.f / sqrtf(ss / (float)DH + kQNormEps);
                 k = r * r * qy / (float)DH;
             }
+            float z0[PH], z1[PH];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int m = lane + 32 * u;
-                if (m < HALF) {
-                    dst[m] = __float2bfloat16_rn(r * (y0[u] - q0[u] * k));
-                    dst[m + HALF] = __float2bfloat16_rn(r * (y1[u] - q1[u] * k));
-                }
+            for (int e = 0; e < PH; ++e) {
+                z0[e] = r * (y0[e] - q0[e] * k);
+                z1[e] = r * (y1[e] - q1[e] * k);
             }
+            st_bf<PH>(dst + m0, z0);
+            st_bf<PH>(dst + m0 + HALF, z1);
         } else {
             const size_t u = (size_t)b * p.Hkv + h;
-            const float* rot = p.dkr + (u * T + t) * DH;
-            const float* a1 = p.dkh_keys + (u * T + t) * DH;
-            const float* a2 = p.dkh_rows + (u * T + t) * DH;
+            const size_t row = (u * T + t) * DH;
             const bf* kraw = static_cast<const bf*>(p.k) + (((size_t)b * T + t) * p.Hkv + h) * DH;
-            float g0[2] = {0.f, 0.f}, g1[2] = {0.f, 0.f}, k0[2] = {0.f, 0.f}, k1[2] = {0.f, 0.f};
+            float r0[PH], r1[PH], a0[PH], a1[PH], c0[PH], c1[PH], v0[PH], v1[PH];
+            ld_f<PH>(p.dkr + row + m0, r0);
+            ld_f<PH>(p.dkr + row + m0 + HALF, r1);
+            ld_f<PH>(p.dkh_keys + row + m0, a0);
+            ld_f<PH>(p.dkh_keys + row + m0 + HALF, a1);
+            ld_f<PH>(p.dkh_rows + row + m0, c0);
+            ld_f<PH>(p.dkh_rows + row + m0 + HALF, c1);
+            ld_f<PH>(p.dv32 + row + m0, v0);
+            ld_f<PH>(p.dv32 + row + m0 + HALF, v1);
+            float g0[PH], g1[PH], k0[PH], k1[PH];
             float proj = 0.f, ss = 0.f;
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int m = lane + 32 * q;
-                if (m < HALF) {
-                    const float cs = s_cos[m], sn = s_sin[m];
-                    g0[q] = a1[m] + a2[m] + rot[m] * cs + rot[m + HALF] * sn;
-                    g1[q] = a1[m + HALF] + a2[m + HALF] + rot[m + HALF] * cs - rot[m] * sn;
-                    k0[q] = __bfloat162float(kraw[m]);
-                    k1[q] = __bfloat162float(kraw[m + HALF]);
-                    ss += k0[q] * k0[q] + k1[q] * k1[q];
-                    proj += g0[q] * k0[q] + g1[q] * k1[q];
-                }
+            for (int e = 0; e < PH; ++e) {
+                g0[e] = a0[e] + c0[e] + r0[e] * cs[e] + r1[e] * sn[e];
+                g1[e] = a1[e] + c1[e] + r1[e] * cs[e] - r0[e] * sn[e];
+                k0[e] = __bfloat162float(kraw[m0 + e]);
+                k1[e] = __bfloat162float(kraw[m0 + e + HALF]);
+                ss += k0[e] * k0[e] + k1[e] * k1[e];
+                proj += g0[e] * k0[e] + g1[e] * k1[e];
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -1124,39 +1159,39 @@ __global__ void __launch_bounds__(256) k_bwd_post_tc(BwdTcParams p) {
             const float inv = 1.f / n;
             // khat = k / n:  dk = (g - khat <khat, g>) / n
             const float pr = proj * inv * inv;
+            float z0[PH], z1[PH];
+#pragma unroll
+            for (int e = 0; e < PH; ++e) {
+                z0[e] = (g0[e] - k0[e] * pr) * inv;
+                z1[e] = (g1[e] - k1[e] * pr) * inv;
+            }
             bf* dst = dk + (((size_t)b * T + t) * p.Hkv + h) * DH;
             bf* dvd = dv + (((size_t)b * T + t) * p.Hkv + h) * DH;
-            const float* dvs = p.dv32 + (u * T + t) * DH;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int m = lane + 32 * q;
-                if (m < HALF) {
-                    dst[m] = __float2bfloat16_rn((g0[q] - k0[q] * pr) * inv);
-                    dst[m + HALF] = __float2bfloat16_rn((g1[q] - k1[q] * pr) * inv);
-                    dvd[m] = __float2bfloat16_rn(dvs[m]);
-                    dvd[m + HALF] = __float2bfloat16_rn(dvs[m + HALF]);
-                }
-            }
+            st_bf<PH>(dst + m0, z0);
+            st_bf<PH>(dst + m0 + HALF, z1);
+            st_bf<PH>(dvd + m0, v0);
+            st_bf<PH>(dvd + m0 + HALF, v1);
         }
     }
-    for (int h = threadIdx.x; h < p.Hkv; h += blockDim.x) {
+    // da_q: the row sums of w over the key tiles up to the row's and their four quarters (one
+    // float4 per key tile, contiguous per row), a warp per KV head; da_k from the key pass
+    const int nk = t / 128 + 1;
+    for (int h = warp; h < p.Hkv; h += 8) {
         const size_t u = (size_t)b * p.Hkv + h;
+        const float4* part = reinterpret_cast<const float4*>(p.daq_part + (u * p.Tpk + t) * p.nkt * 4);
         float sw = 0.f;
-        for (int kt = 0; kt <= t / 128; ++kt)
-            for (int w = 0; w < 4; ++w) sw += p.daq_part[((u * p.nkt + kt) * 4 + w) * p.Tpk + t];
-        const size_t src = ((size_t)b * T + t) * p.Hkv + h;
-        p.da_q[src] = sw * sig_over_sp_f(p.a_q[src]);
-        p.da_k[src] = p.dak32[u * T + t];
+        for (int kt = lane; kt < nk; kt += 32) {
+            const float4 v = part[kt];
+            sw += (v.x + v.y) + (v.z + v.w);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, o);
+        if (lane == 0) {
+            const size_t src = ((size_t)b * T + t) * p.Hkv + h;
+            p.da_q[src] = sw * sig_over_sp_f(p.a_q[src]);
+            p.da_k[src] = p.dak32[u * T + t];
+        }
     }
-    // dg = dO * O * (1 - sigmoid(g))
-    const bf* o = static_cast<const bf*>(p.o);
-    const bf* dO = static_cast<const bf*>(p.d_o);
-    const bf* g = static_cast<const bf*>(p.g);
-    bf* dg = static_cast<bf*>(p.dg);
-    const size_t base = ((size_t)b * T + t) * p.H * DH;
-    for (int e = threadIdx.x; e < p.H * DH; e += blockDim.x)
-        dg[base + e] = __float2bfloat16_rn(__bfloat162float(dO[base + e]) * __bfloat162float(o[base + e]) *
-                                           (1.f - sigmoid_f(__bfloat162float(g[base + e]))));
 }
 
 // =========================================================================== launcher

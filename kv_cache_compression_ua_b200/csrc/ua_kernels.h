@@ -306,7 +306,7 @@ struct BwdTcParams {
     float* pb;            // [B*Hkv][nst][Tpk] decay prefix above each step
     void* tiles;          // [B*Hkv][G+1][ntiles][8 KB]: dZ^T of each head, then dX^T (bf16)
     size_t ntiles;        // 32-row x 128-key tiles of the causal band: 2 * nkt * (nkt + 1)
-    float* daq_part;      // [B*Hkv][nkt][Tpk] row sums of w over each key tile
+    float* daq_part;      // [B*Hkv][Tpk][nkt][4] row sums of w over each quarter of each key tile
     float* dab;           // [B*Hkv*nkt][2] dalpha / dbeta partials
     float* dv32;          // [B*Hkv][T][d]
     float* dkr;           // [B*Hkv][T][d] scale * dkrot
