@@ -200,7 +200,9 @@ __device__ __forceinline__ void st_bf16(__nv_bfloat16* dst, const float (&f)[N])
 
 // grid (T, B), 256 threads: dA = dO * sigmoid(g) (bf16, [B*H][T][d] rows), the gate's gradient
 // dg = dO * O * (1 - sigmoid(g)) (bf16, laid out like g), Delta = sum_c dO*O and lse * log2(e) per
-// (b, h, t).
+// (b, h, t); per (b, KV head, t) the bound c = max over the group's heads of s|qrot|(1 + 2^-6) - lse
+// on the log-probability of row t before its decay (|krot| = 1 in fp32, 1 + 2^-9 in bf16).  A
+// warp per KV group, its heads in turn.
 template <int DH>
 __global__ void __launch_bounds__(256) k_bwd_prep_tc(BwdTcParams p) {
     constexpr int PER = DH / 32;
@@ -211,30 +213,43 @@ __global__ void __launch_bounds__(256) k_bwd_prep_tc(BwdTcParams p) {
     const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(p.g);
     __nv_bfloat16* ad = static_cast<__nv_bfloat16*>(p.ad);
     __nv_bfloat16* dg = static_cast<__nv_bfloat16*>(p.dg);
-    for (int h = warp; h < p.H; h += 8) {
-        const size_t src = (((size_t)b * p.T + t) * p.H + h) * DH + lane * PER;
-        float fo[PER], fd[PER], fg[PER];
-        ld_bf16<PER>(dO + src, fd);
-        ld_bf16<PER>(o + src, fo);
-        ld_bf16<PER>(g + src, fg);
-        float acc = 0.f;
-        float a[PER], dgv[PER];
+    const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(p.qr);
+    for (int u = warp; u < p.Hkv; u += 8) {
+        float cm = -INFINITY;
+        for (int hg = 0; hg < p.G; ++hg) {
+            const int h = u * p.G + hg;
+            const size_t r = (size_t)b * p.H + h;
+            const size_t src = (((size_t)b * p.T + t) * p.H + h) * DH + lane * PER;
+            float fo[PER], fd[PER], fg[PER], fq[PER];
+            ld_bf16<PER>(dO + src, fd);
+            ld_bf16<PER>(o + src, fo);
+            ld_bf16<PER>(g + src, fg);
+            ld_bf16<PER>(qr + (r * p.T + t) * DH + lane * PER, fq);
+            float acc = 0.f, qq = 0.f;
+            float a[PER], dgv[PER];
 #pragma unroll
-        for (int e = 0; e < PER; ++e) {
-            acc = fmaf(fd[e], fo[e], acc);
-            const float sg = sigmoid_f(fg[e]);
-            a[e] = fd[e] * sg;
-            dgv[e] = fd[e] * fo[e] * (1.f - sg);
-        }
-        st_bf16<PER>(ad + (((size_t)b * p.H + h) * p.T + t) * DH + lane * PER, a);
-        st_bf16<PER>(dg + src, dgv);
+            for (int e = 0; e < PER; ++e) {
+                acc = fmaf(fd[e], fo[e], acc);
+                qq = fmaf(fq[e], fq[e], qq);
+                const float sg = sigmoid_f(fg[e]);
+                a[e] = fd[e] * sg;
+                dgv[e] = fd[e] * fo[e] * (1.f - sg);
+            }
+            st_bf16<PER>(ad + (r * p.T + t) * DH + lane * PER, a);
+            st_bf16<PER>(dg + src, dgv);
 #pragma unroll
-        for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-        if (lane == 0) {
-            const size_t r = ((size_t)b * p.H + h);
-            p.delta[r * p.Tp + t] = acc;
-            p.lse2[r * p.Tp + t] = p.lse[r * p.T + t] * kL2e;
+            for (int s = 16; s > 0; s >>= 1) {
+                acc += __shfl_xor_sync(0xffffffffu, acc, s);
+                qq += __shfl_xor_sync(0xffffffffu, qq, s);
+            }
+            const float lse = p.lse[r * p.T + t];
+            cm = fmaxf(cm, p.scale * sqrtf(qq) * (1.f + 1.f / 64.f) - lse);
+            if (lane == 0) {
+                p.delta[r * p.Tp + t] = acc;
+                p.lse2[r * p.Tp + t] = lse * kL2e;
+            }
         }
+        if (lane == 0) p.cmax[((size_t)b * p.Hkv + u) * p.Tpk + t] = cm;
     }
 }
 
@@ -242,6 +257,12 @@ __global__ void __launch_bounds__(256) k_bwd_prep_tc(BwdTcParams p) {
 // grid (B*Hkv, nkt), 128 threads = one thread per key of the tile.  Steps s = 4kt .. nst-1 top
 // down: Pb[s][j] = sum_{j < l < 32 s} D[l, j] is written, then the step's X^T tile (tensor cores,
 // two TMEM slots so the next step's MMA overlaps this step's decay) adds its rows.
+// Exact underflow: Lambda only decreases down a column, so every probability of key j in step s
+// is at most exp(c_s - Pb[s][j]), c_s the rows' bound from the prep pass.  Below -88 nats the
+// kernels' exp2 (flush to zero under 2^-126) returns exactly 0, and so do dZ, dLambda, dD, w and
+// dX for every step from there down.  The key tile's last step that fails the test (at least its
+// diagonal block) bounds the key-major pass and the GEMMs; what lies below contributes zeros.
+constexpr float kUnderflowNats = -88.f;
 namespace bnd {
 template <int DH>
 struct Smem {
@@ -252,6 +273,7 @@ struct Smem {
     alignas(8) uint64_t kfull, qfull[2], xfull[2];
     uint32_t tmem;
     int abort;
+    int last[4];
 };
 }  // namespace bnd
 
@@ -319,10 +341,20 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
     const float al2 = p.alpha[kvh] * kL2e, be2 = p.beta[kvh] * kL2e;
     float run = 0.f;                                  // sum of D / rk3 over the rows so far
     float* pbrow = p.pb + (size_t)unit * p.nst * p.Tpk + (size_t)kt * 128 + tid;
+    const float* crow = p.cmax + (size_t)unit * p.Tpk;
+    int last = min(s0 + 3, p.nst - 1);                // the diagonal block is always walked
     const uint32_t tl = (uint32_t)(warp * 32) << 16;
     for (int it = 0; it < nsteps; ++it) {
         const int st = it & 1, s = s0 + it;
-        pbrow[(size_t)s * p.Tpk] = rk3 * run;
+        const float pb = rk3 * run;
+        pbrow[(size_t)s * p.Tpk] = pb;
+        {
+            const int row = s * ST + (tid & 31);
+            float c = row < T ? crow[row] : -INFINITY;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
+            if (j < T && c - pb >= kUnderflowNats) last = s;
+        }
         if (leader && ok && it + 1 < nsteps) {
             if (mbar_wait(&S.qfull[(it + 1) & 1], ((it + 1) >> 1) & 1, abort)) {
                 tc_fence_after();
@@ -362,8 +394,12 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
             }
         }
     }
+    last = __reduce_max_sync(0xffffffffu, last);
+    if ((tid & 31) == 0) S.last[warp] = last;
     tc_fence_before();
     __syncthreads();
+    if (tid == 0)
+        p.slast[(size_t)unit * p.nkt + kt] = max(max(S.last[0], S.last[1]), max(S.last[2], S.last[3]));
     if (*abort && tid == 0) drain_pause(10000000ull);
     __syncthreads();
     if (warp == 0) {
@@ -376,6 +412,13 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
 // grid (B*Hkv, nkt), 544 threads: warps 0-15 compute (four threads per key j, TMEM lane j % 128:
 // warps 4q .. 4q+3 rows 8q .. 8q+7 of each step), warp 16 issues the TMA loads and the MMAs.  Steps s = nst-1 down to 4kt.  TMEM: dV (DH columns), dKrot (DH),
 // the X^T slot (32), two slots for the S_h^T / dP_h^T pair of a head (64 each).
+// Last step of key tile kt walked by the key-major pass and summed by the GEMMs: the boundary
+// pass's bound, kept within [the diagonal block, nst - 1].
+__device__ __forceinline__ int last_step(const BwdTcParams& p, int unit, int kt) {
+    const int sd = min(4 * kt + 3, p.nst - 1);
+    return max(min(p.slast[(size_t)unit * p.nkt + kt], p.nst - 1), sd);
+}
+
 namespace key {
 template <int DH, int G>
 struct Smem {
@@ -422,7 +465,8 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int kt = blockIdx.y, unit = blockIdx.x, kvh = unit % p.Hkv, b = unit / p.Hkv;   // longest first
     const int T = p.T;
-    const int s0 = 4 * kt, nsteps = p.nst - s0;
+    // steps sfin down to 4kt; the ones below sfin hold no nonzero probability
+    const int s0 = 4 * kt, sfin = last_step(p, unit, kt), nsteps = sfin - s0 + 1;
     volatile int* abort = &S.abort;
     if (tid == 0) {
         mbar_init(&S.kfull, 1);
@@ -463,7 +507,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         // vector have one buffer: X^T is the first MMA of a step, so they are free
         // early and the next step's copy overlaps the rest of this one.
         auto load_q = [&](int it) {
-            const int s = p.nst - 1 - it;
+            const int s = sfin - it;
             if (leader) {
                 mbar_expect_tx(&S.qfull, NB * 4096 + ST * 4 + 128 * 4);
                 for (int c = 0; c < NB; ++c) tma_load_3d(S.kq[c], &tm_khq, &S.qfull, 64 * c, s * ST, unit);
@@ -473,7 +517,7 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
             __syncwarp();
         };
         auto load_h = [&](int it, int h) {
-            const int s = p.nst - 1 - it, row = b * p.H + kvh * G + h;
+            const int s = sfin - it, row = b * p.H + kvh * G + h;
             if (leader) {
                 mbar_expect_tx(&S.hfull[h], 2 * NB * 4096 + 2 * ST * 4);
                 for (int c = 0; c < NB; ++c) {
@@ -617,8 +661,22 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         const size_t tstride = (size_t)p.ntiles * kTileBytes;      // bytes per stored tile set
         uint8_t* tile_base = static_cast<uint8_t*>(p.tiles) + (size_t)unit * (G + 1) * tstride;
         const size_t band = band_off(kt, p.nkt);
+        {
+            // below sfin: the rest of its 128-row block of stored tiles (the GEMMs sum whole blocks)
+            // and the rows' w sums (the post pass reads them) are zero
+            const int zend = min(4 * (sfin / 4) + 3, p.nst - 1);
+            const int nz = (zend - sfin) * (int)(kTileBytes / 16);
+            for (int g2 = 0; g2 <= G; ++g2) {
+                uint4* z = reinterpret_cast<uint4*>(tile_base + (size_t)g2 * tstride +
+                                                    (band + (sfin + 1 - s0)) * kTileBytes);
+                for (int i = tid; i < nz; i += 128 * kKeyQ) z[i] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            float4* dq4 = reinterpret_cast<float4*>(p.daq_part);
+            for (int r = ST * (sfin + 1) + tid; r < p.Tpk; r += 128 * kKeyQ)
+                dq4[((size_t)unit * p.Tpk + r) * p.nkt + kt] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         for (int it = 0; ok && it < nsteps; ++it) {
-            const int s = p.nst - 1 - it;
+            const int s = sfin - it;
             const int i0 = s * ST;
             const int xb = it & 1;                    // exchange buffer and its phase
             const uint32_t xph = (uint32_t)(it >> 1) & 1u;
@@ -907,7 +965,14 @@ k_bwd_gemm_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__
     const int o = ROWS ? (int)blockIdx.y : p.G;       // output: head o's dqrot, or the dkhat part
     const int kvh = unit % p.Hkv, b = unit / p.Hkv;
     const int T = p.T;
-    const int n = ROWS ? blk + 1 : p.nkt - blk;       // operand pairs to sum
+    // operand pairs to sum: key tiles kt <= blk whose walked steps reach the row block (the
+    // diagonal one always does), or row blocks blk .. the one of the key tile's last walked step
+    int n = 0;
+    if (ROWS) {
+        for (int kt = 0; kt <= blk; ++kt) n += last_step(p, unit, kt) >= 4 * blk;
+    } else {
+        n = last_step(p, unit, blk) / 4 - blk + 1;
+    }
     volatile int* abort = &S.abort;
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) {
@@ -935,11 +1000,15 @@ k_bwd_gemm_tc(const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__
     const uint8_t* tiles = static_cast<const uint8_t*>(p.tiles) + ((size_t)unit * (p.G + 1) + o) * tstride;
     if (warp == 0) {
         const bool leader = elect_one();
+        int ktn = 0;                                  // rows side: next key tile to test
         for (int i = 0; i < n; ++i) {
             const int stg = i % NS;
             if (i >= NS && !wwait(&S.empty[stg], ((i / NS) - 1) & 1, abort)) break;
-            // rows side: key tile kt = i of row block blk; key side: row block rb = blk + i of key tile blk
-            const int kt = ROWS ? i : blk, rb = ROWS ? blk : blk + i;
+            // rows side: the i-th key tile of row block blk with walked steps there; key side: row
+            // block rb = blk + i of key tile blk
+            if (ROWS)
+                while (last_step(p, unit, ktn) < 4 * blk) ++ktn;
+            const int kt = ROWS ? ktn++ : blk, rb = ROWS ? blk : blk + i;
             if (leader) {
                 mbar_expect_tx(&S.full[stg], NB * 16384 + 4 * kTileBytes);
                 const CUtensorMap* m = (ROWS && o < p.G) ? &tm_kr : &tm_kh;

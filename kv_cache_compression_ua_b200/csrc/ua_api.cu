@@ -444,8 +444,8 @@ BwdWs bwd_ws_layout(const ua_shape* s) {
 // dA, Delta and lse in log2 units, the decay prefixes above every 32-row step, the stored bf16
 // dZ^T / dX^T tiles of the causal band, and f32 gradient intermediates.
 struct BwdTcWs {
-    size_t qr, kh, kr, lq2, lk2, mq, ad, lse2, delta, pb, tiles, daq, dab, dv32, dkr, dkh, dkh_rows, dqr, dak,
-        total, ntiles;
+    size_t qr, kh, kr, lq2, lk2, mq, ad, lse2, delta, pb, tiles, daq, cmax, slast, dab, dv32, dkr, dkh, dkh_rows,
+        dqr, dak, total, ntiles;
     int Tp, Tpk, nkt, nst;
 };
 
@@ -472,6 +472,8 @@ BwdTcWs bwd_tc_ws_layout(const ua_shape* s) {
     w.pb = take(B * Hkv * (size_t)w.nst * Tpk * 4);
     w.tiles = take(B * Hkv * (G + 1) * w.ntiles * 8192);
     w.daq = take(B * Hkv * nkt * 4 * Tpk * 4);
+    w.cmax = take(B * Hkv * Tpk * 4);
+    w.slast = take(B * Hkv * nkt * 4);
     w.dab = take(B * Hkv * nkt * 2 * 4);
     w.dv32 = take(B * Hkv * T * d * 4);
     w.dkr = take(B * Hkv * T * d * 4);
@@ -541,6 +543,8 @@ static ua_status prefill_bwd_tc(const ua_shape* s, const void* q, const void* k,
     p.tiles = at(ws, w.tiles);
     p.ntiles = w.ntiles;
     p.daq_part = reinterpret_cast<float*>(at(ws, w.daq));
+    p.cmax = reinterpret_cast<float*>(at(ws, w.cmax));
+    p.slast = reinterpret_cast<int*>(at(ws, w.slast));
     p.dab = reinterpret_cast<float*>(at(ws, w.dab));
     p.dv32 = reinterpret_cast<float*>(at(ws, w.dv32));
     p.dkr = reinterpret_cast<float*>(at(ws, w.dkr));

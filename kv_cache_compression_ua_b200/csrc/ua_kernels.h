@@ -307,6 +307,8 @@ struct BwdTcParams {
     void* tiles;          // [B*Hkv][G+1][ntiles][8 KB]: dZ^T of each head, then dX^T (bf16)
     size_t ntiles;        // 32-row x 128-key tiles of the causal band: 2 * nkt * (nkt + 1)
     float* daq_part;      // [B*Hkv][Tpk][nkt][4] row sums of w over each quarter of each key tile
+    float* cmax;          // [B*Hkv][Tpk] per row: max over the group's heads of s|qrot|(1 + 2^-6) - lse (nats)
+    int* slast;           // [B*Hkv][nkt] last 32-row step of each key tile with a possibly nonzero probability
     float* dab;           // [B*Hkv*nkt][2] dalpha / dbeta partials
     float* dv32;          // [B*Hkv][T][d]
     float* dkr;           // [B*Hkv][T][d] scale * dkrot

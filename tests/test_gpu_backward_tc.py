@@ -103,3 +103,34 @@ def test_d128_four_heads_per_kv_head_runs_simt_and_matches():
     rms = sum_model_rms(oracle.prefill_bwd, r, **x, scale=w.scale, theta=w.theta)
     for n in GRADS:
         assert_grad_close(n, g[n], r[n], "bf16", rms)
+
+
+@pytest.mark.parametrize("T,H,Hkv,d", [(1500, 4, 2, 64), (1200, 3, 1, 128)])
+def test_tensor_core_backward_with_underflowing_band(T, H, Hkv, d):
+    """Strong decay rates: some hundred rows below a key every probability underflows to exactly 0,
+    so the key-major pass walks each key tile only down to its last step with a possibly nonzero
+    probability and the GEMMs skip the band below it.  That band contributes exact zeros, so the
+    gradients must still match the oracle."""
+    w = I.Workload("bwduf", 1, T, H, Hkv, d, "bf16", 2700 + T + d, with_grad=True)
+    x = I.make_prefill_inputs(w)
+    x["a_q"] = x["a_q"] + 4.0
+    x["a_k"] = x["a_k"] + 4.0
+    # the inputs do put the band past the threshold (exp(-88 nats) and the logits' bound of a few
+    # nats): Lambda(i, j) for i - j >= 256
+    k = x["k"][0, :, 0].astype(np.float64)
+    kh = k / np.linalg.norm(k, axis=1, keepdims=True)
+    sp = lambda z: np.logaddexp(0.0, z)
+    X = x["alpha"][0] * (kh @ kh.T) + x["beta"][0]
+    D = np.exp(np.log(sp(x["a_q"][0, :, 0]))[:, None] / 3 + np.log(sp(x["a_k"][0, :, 0]))[None, :] / 3
+               + np.log(sp(X)) / 3)
+    lam = -np.cumsum(np.tril(D, -1), axis=0)
+    far = np.tril(np.ones((T, T), bool), -256)
+    assert np.mean(lam[far] < -120.0) > 0.99
+    gr, names = run(w, x)
+    assert "k_bwd_key_tc" in names, names
+    g = {k: v.float().cpu().numpy() for k, v in gr.items()}
+    r = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta)
+    rms = sum_model_rms(oracle.prefill_bwd, r, **x, scale=w.scale, theta=w.theta)
+    for n in GRADS:
+        assert np.all(np.isfinite(g[n])), n
+        assert_grad_close(n, g[n], r[n], "bf16", rms)
