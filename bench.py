@@ -769,6 +769,9 @@ def bench_fwdbwd(args):
     return {"workload": f"fwdbwd_3b: B={w.B} T={w.T} H={w.H} Hkv={w.Hkv} d={w.d} bf16", "fwd_ms": fms, "bwd_ms": bms,
             "fwd_tflops": fwd_flops(w) / (fms * 1e-3) / 1e12, "bwd_tflops": bwd_flops(w) / (bms * 1e-3) / 1e12,
             "fwd_bwd_tflops": (fwd_flops(w) + bwd_flops(w)) / ((fms + bms) * 1e-3) / 1e12,
+            "flops_basis": "dense-equivalent: the whole causal triangle's FLOPs; both passes skip exactly "
+                           "underflowing tiles (the forward its softmax, the backward the band below each "
+                           "key tile's last step with a possibly nonzero probability)",
             "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / v[0]} for k, v in prof.items()}}
 
 
