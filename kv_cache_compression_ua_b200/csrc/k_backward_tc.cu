@@ -274,6 +274,7 @@ struct Smem {
     uint32_t tmem;
     int abort;
     int last[4];
+    float cw[4];
 };
 }  // namespace bnd
 
@@ -305,10 +306,20 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
         tmem_alloc(&S.tmem, 64);
         tmem_relinquish();
     }
+    // the unit's largest row bound: once every key's prefix is past it, so is every later step
+    const float* crow = p.cmax + (size_t)unit * p.Tpk;
+    {
+        float c = -INFINITY;
+        for (int r = tid; r < T; r += 128) c = fmaxf(c, crow[r]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
+        if ((tid & 31) == 0) S.cw[warp] = c;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem;
+    const float call = fmaxf(fmaxf(S.cw[0], S.cw[1]), fmaxf(S.cw[2], S.cw[3]));
     const bool leader = warp == 0 && elect_one();
     auto load_step = [&](int it) {
         const int st = it & 1, s = s0 + it;
@@ -341,7 +352,6 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
     const float al2 = p.alpha[kvh] * kL2e, be2 = p.beta[kvh] * kL2e;
     float run = 0.f;                                  // sum of D / rk3 over the rows so far
     float* pbrow = p.pb + (size_t)unit * p.nst * p.Tpk + (size_t)kt * 128 + tid;
-    const float* crow = p.cmax + (size_t)unit * p.Tpk;
     int last = min(s0 + 3, p.nst - 1);                // the diagonal block is always walked
     const uint32_t tl = (uint32_t)(warp * 32) << 16;
     for (int it = 0; it < nsteps; ++it) {
@@ -354,6 +364,15 @@ __global__ void __launch_bounds__(128) k_bwd_bound_tc(const __grid_constant__ CU
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
             if (j < T && c - pb >= kUnderflowNats) last = s;
+        }
+        // below the diagonal block, once this step and all later ones are past the threshold for
+        // every key: stop (after this step's product and the next step's copy have landed)
+        if (it >= 4 && __syncthreads_and(j >= T || call - pb < kUnderflowNats)) {
+            if (ok) {
+                ok = mbar_wait(&S.xfull[st], (it >> 1) & 1, abort);
+                if (ok && it + 1 < nsteps) ok = mbar_wait(&S.qfull[(it + 1) & 1], ((it + 1) >> 1) & 1, abort);
+            }
+            break;
         }
         if (leader && ok && it + 1 < nsteps) {
             if (mbar_wait(&S.qfull[(it + 1) & 1], ((it + 1) >> 1) & 1, abort)) {
