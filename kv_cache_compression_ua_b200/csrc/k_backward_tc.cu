@@ -201,8 +201,9 @@ __device__ __forceinline__ void st_bf16(__nv_bfloat16* dst, const float (&f)[N])
 // grid (T, B), 256 threads: dA = dO * sigmoid(g) (bf16, [B*H][T][d] rows), the gate's gradient
 // dg = dO * O * (1 - sigmoid(g)) (bf16, laid out like g), Delta = sum_c dO*O and lse * log2(e) per
 // (b, h, t); per (b, KV head, t) the bound c = max over the group's heads of s|qrot|(1 + 2^-6) - lse
-// on the log-probability of row t before its decay (|krot| = 1 in fp32, 1 + 2^-9 in bf16).  A
-// warp per KV group, its heads in turn.
+// on the log-probability of row t before its decay (|qrot| from the token preparation in fp32;
+// the bf16 copies the products read are within 1 + 2^-9 of it, and |krot| of 1).  A warp per KV
+// group, its heads in turn.
 template <int DH>
 __global__ void __launch_bounds__(256) k_bwd_prep_tc(BwdTcParams p) {
     constexpr int PER = DH / 32;
@@ -213,24 +214,21 @@ __global__ void __launch_bounds__(256) k_bwd_prep_tc(BwdTcParams p) {
     const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(p.g);
     __nv_bfloat16* ad = static_cast<__nv_bfloat16*>(p.ad);
     __nv_bfloat16* dg = static_cast<__nv_bfloat16*>(p.dg);
-    const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(p.qr);
     for (int u = warp; u < p.Hkv; u += 8) {
         float cm = -INFINITY;
         for (int hg = 0; hg < p.G; ++hg) {
             const int h = u * p.G + hg;
             const size_t r = (size_t)b * p.H + h;
             const size_t src = (((size_t)b * p.T + t) * p.H + h) * DH + lane * PER;
-            float fo[PER], fd[PER], fg[PER], fq[PER];
+            float fo[PER], fd[PER], fg[PER];
             ld_bf16<PER>(dO + src, fd);
             ld_bf16<PER>(o + src, fo);
             ld_bf16<PER>(g + src, fg);
-            ld_bf16<PER>(qr + (r * p.T + t) * DH + lane * PER, fq);
-            float acc = 0.f, qq = 0.f;
+            float acc = 0.f;
             float a[PER], dgv[PER];
 #pragma unroll
             for (int e = 0; e < PER; ++e) {
                 acc = fmaf(fd[e], fo[e], acc);
-                qq = fmaf(fq[e], fq[e], qq);
                 const float sg = sigmoid_f(fg[e]);
                 a[e] = fd[e] * sg;
                 dgv[e] = fd[e] * fo[e] * (1.f - sg);
@@ -238,12 +236,9 @@ __global__ void __launch_bounds__(256) k_bwd_prep_tc(BwdTcParams p) {
             st_bf16<PER>(ad + (r * p.T + t) * DH + lane * PER, a);
             st_bf16<PER>(dg + src, dgv);
 #pragma unroll
-            for (int s = 16; s > 0; s >>= 1) {
-                acc += __shfl_xor_sync(0xffffffffu, acc, s);
-                qq += __shfl_xor_sync(0xffffffffu, qq, s);
-            }
+            for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
             const float lse = p.lse[r * p.T + t];
-            cm = fmaxf(cm, p.scale * sqrtf(qq) * (1.f + 1.f / 64.f) - lse);
+            cm = fmaxf(cm, p.mq[r * p.Tp + t] * kLn2 * (1.f + 1.f / 64.f) - lse);
             if (lane == 0) {
                 p.delta[r * p.Tp + t] = acc;
                 p.lse2[r * p.Tp + t] = lse * kL2e;

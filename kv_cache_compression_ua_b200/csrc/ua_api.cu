@@ -533,7 +533,7 @@ static ua_status prefill_bwd_tc(const ua_shape* s, const void* q, const void* k,
     BwdTcParams p;
     p.B = s->B; p.T = s->T; p.Tp = w.Tp; p.Tpk = w.Tpk; p.H = s->H; p.Hkv = s->Hkv; p.d = s->d;
     p.G = s->H / s->Hkv; p.nkt = w.nkt; p.nst = w.nst; p.scale = s->scale; p.rf = pp.rf; p.variant = s->variant;
-    p.qr = pp.qr; p.kh = pp.kh; p.kr = pp.kr; p.lq2 = pp.lq2; p.lk2 = pp.lk2;
+    p.qr = pp.qr; p.kh = pp.kh; p.kr = pp.kr; p.lq2 = pp.lq2; p.lk2 = pp.lk2; p.mq = pp.mq;
     p.q = q; p.k = k; p.v = v; p.g = g; p.o = o; p.d_o = d_o;
     p.a_q = a_q; p.a_k = a_k; p.alpha = alpha; p.beta = beta; p.lse = lse;
     p.ad = at(ws, w.ad);

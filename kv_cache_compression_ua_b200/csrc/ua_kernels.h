@@ -296,6 +296,7 @@ struct BwdTcParams {
     const void* kr;       // [B*Hkv][T][d] RoPE(khat)
     const float* lq2;     // [B*Hkv][Tp]
     const float* lk2;     // [B*Hkv][Tp]
+    const float* mq;      // [B*H][Tp] scale * log2(e) * |qrot| (fp32, after the query norm)
     // the caller's tensors
     const void* q; const void* k; const void* v; const void* g; const void* o; const void* d_o;
     const float* a_q; const float* a_k; const float* alpha; const float* beta; const float* lse;

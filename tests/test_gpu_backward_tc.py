@@ -105,12 +105,14 @@ def test_d128_four_heads_per_kv_head_runs_simt_and_matches():
         assert_grad_close(n, g[n], r[n], "bf16", rms)
 
 
-@pytest.mark.parametrize("T,H,Hkv,d", [(1500, 4, 2, 64), (1200, 3, 1, 128)])
-def test_tensor_core_backward_with_underflowing_band(T, H, Hkv, d):
+@pytest.mark.parametrize("T,H,Hkv,d,variant", [(1500, 4, 2, 64, 0), (1200, 3, 1, 128, 0),
+                                               (1500, 4, 2, 64, ua.VAR_QUERY_NORM)])
+def test_tensor_core_backward_with_underflowing_band(T, H, Hkv, d, variant):
     """Strong decay rates: some hundred rows below a key every probability underflows to exactly 0,
     so the key-major pass walks each key tile only down to its last step with a possibly nonzero
     probability and the GEMMs skip the band below it.  That band contributes exact zeros, so the
-    gradients must still match the oracle."""
+    gradients must still match the oracle (with the query norm too: the bound uses the normalised
+    queries)."""
     w = I.Workload("bwduf", 1, T, H, Hkv, d, "bf16", 2700 + T + d, with_grad=True)
     x = I.make_prefill_inputs(w)
     x["a_q"] = x["a_q"] + 4.0
@@ -126,11 +128,11 @@ def test_tensor_core_backward_with_underflowing_band(T, H, Hkv, d):
     lam = -np.cumsum(np.tril(D, -1), axis=0)
     far = np.tril(np.ones((T, T), bool), -256)
     assert np.mean(lam[far] < -120.0) > 0.99
-    gr, names = run(w, x)
+    gr, names = run(w, x, variant=variant)
     assert "k_bwd_key_tc" in names, names
     g = {k: v.float().cpu().numpy() for k, v in gr.items()}
-    r = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta)
-    rms = sum_model_rms(oracle.prefill_bwd, r, **x, scale=w.scale, theta=w.theta)
+    r = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta, variant=variant)
+    rms = sum_model_rms(oracle.prefill_bwd, r, **x, scale=w.scale, theta=w.theta, variant=variant)
     for n in GRADS:
         assert np.all(np.isfinite(g[n])), n
         assert_grad_close(n, g[n], r[n], "bf16", rms)
