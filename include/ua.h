@@ -209,7 +209,11 @@ ua_status ua_prefill_fixed_rows(const ua_shape* shape, const void* ws, size_t ws
  * key gradient in TMEM and stores the bf16 dZ / dX tiles of the causal band, and tensor-core
  * GEMMs for the query and similarity gradients (the workspace holds the band: about
  * (G+1) * 2 bytes per causal pair and KV head).  Similarities are formed from the same bf16 unit
- * keys as the tensor-core forward (whose row normalisers the probabilities are divided by).  Other
+ * keys as the tensor-core forward (whose row normalisers the probabilities are divided by).  The
+ * band below each 128-key tile's last 32-row step whose probabilities can be nonzero is skipped
+ * exactly: Lambda only decreases down a key's column, so once s|q|(1 + 2^-6) - lse - Pb falls
+ * below -88 (the exp2 then flushes to 0) for every row of a step and every step below, its dZ,
+ * dLambda and dX contributions are exact zeros (the workspace still holds the whole band).  Other
  * problems run as fp32 SIMT kernels.
  * Training is dense: a shape with prune_p != 0 is UA_ERR_INVALID_ARG. */
 ua_status ua_prefill_bwd_workspace_size(const ua_shape* shape, size_t* bytes);
