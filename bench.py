@@ -776,7 +776,11 @@ def bench_fwdbwd(args):
     prof = ua.profile_read()
     assert ua.get_device_status() == 0
     fms, bms = e[0].elapsed_time(e[1]) / n, e[1].elapsed_time(e[2]) / n
+    steps, walked = ua.prefill_bwd_band_stats(shape, wsb)
+    band = {"steps": steps, "walked": walked, "walked_fraction": walked / steps,
+            "bwd_tflops_walked_estimate": bwd_flops(w) * walked / steps / (bms * 1e-3) / 1e12}
     return {"workload": f"fwdbwd_3b: B={w.B} T={w.T} H={w.H} Hkv={w.Hkv} d={w.d} bf16", "fwd_ms": fms, "bwd_ms": bms,
+            "bwd_band": band,
             "fwd_tflops": fwd_flops(w) / (fms * 1e-3) / 1e12, "bwd_tflops": bwd_flops(w) / (bms * 1e-3) / 1e12,
             "fwd_bwd_tflops": (fwd_flops(w) + bwd_flops(w)) / ((fms + bms) * 1e-3) / 1e12,
             "flops_basis": "dense-equivalent: the whole causal triangle's FLOPs; both passes skip exactly "

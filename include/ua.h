@@ -225,6 +225,15 @@ ua_status ua_prefill_bwd(const ua_shape* shape, const void* q, const void* k, co
                          float* da_k, float* dalpha, float* dbeta, void* ws, size_t ws_bytes,
                          void* stream);
 
+/* No counterpart on the pages: a measurement aid for the exact underflow skipping described at
+ * ua_prefill_bwd.  Synchronises `stream` and reports, for the most recent ua_prefill_bwd that
+ * used workspace `ws` for `shape`, the 32-row steps of the causal band (per KV head and batch:
+ * key tile kt meets steps 4kt .. 4*ceil(T/128)-1) in *steps, and how many of them the key-major
+ * pass walked in *walked (the rest hold no nonzero probability).  Problems that run the fp32
+ * SIMT backward report *walked = *steps.  prune_p != 0 is UA_ERR_INVALID_ARG. */
+ua_status ua_prefill_bwd_band_stats(const ua_shape* shape, const void* ws, size_t ws_bytes,
+                                    unsigned long long* steps, unsigned long long* walked, void* stream);
+
 /* ------------------------------------------------------------------ self-pruning cache
  * One cache per (batch, KV head), structure of arrays, `capacity` slots each; slot s of
  * (b, h) lives at index (b*Hkv + h)*capacity + s.  Slots [0, n_kept[b,h]) are live, in

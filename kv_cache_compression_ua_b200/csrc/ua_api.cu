@@ -1,5 +1,7 @@
 // ua_api.cu -- the C ABI of libua: argument validation, workspace carving and launches.
 // Formulas, layouts and error behaviour are documented in include/ua.h.
+#include <algorithm>
+#include <vector>
 #include <math.h>
 #include <string.h>
 
@@ -769,6 +771,49 @@ ua_status ua_prefill_tile_stats(const ua_shape* s, const void* ws, size_t ws_byt
     if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
     if (e != cudaSuccess) return UA_ERR_CUDA;
     *skipped = host;
+    return UA_OK;
+}
+
+ua_status ua_prefill_bwd_band_stats(const ua_shape* s, const void* ws, size_t ws_bytes, unsigned long long* steps,
+                                    unsigned long long* walked, void* stream) {
+    if (!s || !steps || !walked) return UA_ERR_INVALID_ARG;
+    ua_status st = check_shape(s);
+    if (st != UA_OK) return st;
+    if (s->prune_p != 0.f) return UA_ERR_INVALID_ARG;
+    if (per_head(s)) {
+        // the per-KV-head backward on repeated K and V, whose workspace follows the four copies
+        const ua_shape in = per_head_inner(s);
+        const size_t rb = 4 * rep_bytes(s);
+        if (!ws) return UA_ERR_INVALID_ARG;
+        if (ws_bytes < rb) return UA_ERR_WORKSPACE;
+        return ua_prefill_bwd_band_stats(&in, static_cast<const uint8_t*>(ws) + rb, ws_bytes - rb, steps, walked,
+                                         stream);
+    }
+    // 32-row steps of the causal band: key tile kt meets steps 4kt .. nst-1
+    const long long nkt = ((long long)s->T + 127) / 128, nst = 4 * nkt;
+    const unsigned long long per_unit = (unsigned long long)(nkt * nst - 4 * nkt * (nkt - 1) / 2);
+    *steps = (unsigned long long)s->B * s->Hkv * per_unit;
+    *walked = *steps;
+    if (!use_bwd_tc(s)) return UA_OK;                 // the SIMT backward walks the whole band
+    const BwdTcWs w = bwd_tc_ws_layout(s);
+    if (!ws) return UA_ERR_INVALID_ARG;
+    if (ws_bytes < w.total) return UA_ERR_WORKSPACE;
+    const size_t n = (size_t)s->B * s->Hkv * w.nkt;
+    std::vector<int> last(n);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(last.data(), static_cast<const uint8_t*>(ws) + w.slast, n * sizeof(int),
+                                    cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return UA_ERR_CUDA;
+    unsigned long long sum = 0;
+    for (size_t i = 0; i < n; ++i) {
+        // the bound the kernels use: at least the diagonal block, at most the last step
+        const int kt = (int)(i % w.nkt);
+        const int sd = std::min(4 * kt + 3, w.nst - 1);
+        const int sl = std::max(std::min(last[i], w.nst - 1), sd);
+        sum += (unsigned long long)(sl - 4 * kt + 1);
+    }
+    *walked = sum;
     return UA_OK;
 }
 

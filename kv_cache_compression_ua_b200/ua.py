@@ -53,7 +53,8 @@ EXPORTS = ("ua_prefill_workspace_size", "ua_prefill_fwd", "ua_prefill_bwd_worksp
            "ua_cache_fill", "ua_cache_compact", "ua_decode_step", "ua_get_device_status",
            "ua_profile_enable", "ua_profile_reset", "ua_profile_read", "ua_status_string", "ua_version",
            "ua_prefill_fwd_noalloc", "ua_prefill_noalloc_max_scratch", "ua_prefill_tile_stats",
-           "ua_set_wait_limit_ns", "ua_decode_workspace_size", "ua_decode_step_split", "ua_prefill_fixed_rows")
+           "ua_set_wait_limit_ns", "ua_decode_workspace_size", "ua_decode_step_split", "ua_prefill_fixed_rows",
+           "ua_prefill_bwd_band_stats")
 
 
 class ua_kernel_time(ctypes.Structure):
@@ -91,6 +92,8 @@ def load_library(path: str = LIB_PATH):
                                           ctypes.POINTER(ctypes.c_ulonglong), P]
     lib.ua_prefill_noalloc_max_scratch.restype = S
     lib.ua_prefill_fixed_rows.argtypes = [SP, P, S, ctypes.POINTER(ctypes.c_ulonglong), P]
+    lib.ua_prefill_bwd_band_stats.argtypes = [SP, P, S, ctypes.POINTER(ctypes.c_ulonglong),
+                                              ctypes.POINTER(ctypes.c_ulonglong), P]
     lib.ua_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     lib.ua_decode_workspace_size.argtypes = [CP, I, ctypes.POINTER(S)]
     lib.ua_decode_step_split.argtypes = [CP, I] + [P] * 8 + [I, F, F, D, P, P, P, I, P, S, P]
@@ -252,6 +255,15 @@ def prefill_tile_stats(shape: ua_shape, ws: torch.Tensor, stream=None) -> tuple:
     _check("ua_prefill_tile_stats", load_library().ua_prefill_tile_stats(
         ctypes.byref(shape), _ptr(ws), _nbytes(ws), ctypes.byref(tiles), ctypes.byref(skipped), _stream(stream)))
     return tiles.value, skipped.value
+
+
+def prefill_bwd_band_stats(shape: ua_shape, ws: torch.Tensor, stream=None) -> tuple:
+    """ua_prefill_bwd_band_stats: (32-row steps of the causal band, steps the key-major pass
+    walked) of the last ua_prefill_bwd that used `ws` for `shape`."""
+    steps, walked = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+    _check("ua_prefill_bwd_band_stats", load_library().ua_prefill_bwd_band_stats(
+        ctypes.byref(shape), _ptr(ws), _nbytes(ws), ctypes.byref(steps), ctypes.byref(walked), _stream(stream)))
+    return steps.value, walked.value
 
 
 def prefill_fixed_rows(shape: ua_shape, ws: torch.Tensor, stream=None) -> int:

@@ -22,7 +22,7 @@ def dev(x):
         torch.bfloat16 if n in ("q", "k", "v", "g", "d_o") else torch.float32).contiguous() for n, a in x.items()}
 
 
-def run(w, x, variant=0):
+def run(w, x, variant=0, ws=None):
     d = dev(x)
     f = ua.prefill_fwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"],
                        scale=w.scale, theta=w.theta, variant=variant)
@@ -30,7 +30,7 @@ def run(w, x, variant=0):
     ua.profile_enable(True)
     try:
         gr = ua.prefill_bwd(d["q"], d["k"], d["v"], d["g"], d["a_q"], d["a_k"], d["alpha"], d["beta"], f["o"],
-                            f["lse"], f["b_final"], d["d_o"], scale=w.scale, theta=w.theta, variant=variant)
+                            f["lse"], f["b_final"], d["d_o"], scale=w.scale, theta=w.theta, variant=variant, ws=ws)
         torch.cuda.synchronize()
     finally:
         ua.profile_enable(False)
@@ -96,8 +96,13 @@ def test_d128_four_heads_per_kv_head_runs_simt_and_matches():
     (four dZ/dX step tiles beside the key tile); it runs on the fp32 SIMT backward."""
     w = I.Workload("bwdg4", 1, 150, 4, 1, 128, "bf16", 2600, with_grad=True)
     x = I.make_prefill_inputs(w)
-    gr, names = run(w, x)
+    shape = ua.make_shape(torch.empty(1, 150, 4, 128, dtype=torch.bfloat16),
+                          torch.empty(1, 150, 1, 128, dtype=torch.bfloat16), w.scale, w.theta, 0)
+    ws = ua.alloc_workspace(ua.prefill_bwd_workspace_size(shape), "cuda")
+    gr, names = run(w, x, ws=ws)
     assert "k_bwd_key_tc" not in names and "k_bwd_keys" in names, names
+    steps, walked = ua.prefill_bwd_band_stats(shape, ws)
+    assert walked == steps == 8 + 4, (steps, walked)   # key tile 0: steps 0..7, key tile 1: steps 4..7
     g = {k: v.float().cpu().numpy() for k, v in gr.items()}
     r = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta)
     rms = sum_model_rms(oracle.prefill_bwd, r, **x, scale=w.scale, theta=w.theta)
@@ -128,8 +133,17 @@ def test_tensor_core_backward_with_underflowing_band(T, H, Hkv, d, variant):
     lam = -np.cumsum(np.tril(D, -1), axis=0)
     far = np.tril(np.ones((T, T), bool), -256)
     assert np.mean(lam[far] < -120.0) > 0.99
-    gr, names = run(w, x, variant=variant)
+    shape = ua.make_shape(torch.empty(1, T, H, d, dtype=torch.bfloat16), torch.empty(1, T, Hkv, d, dtype=torch.bfloat16),
+                          w.scale, w.theta, variant)
+    ws = ua.alloc_workspace(ua.prefill_bwd_workspace_size(shape), "cuda")
+    gr, names = run(w, x, variant=variant, ws=ws)
     assert "k_bwd_key_tc" in names, names
+    # the key-major pass stopped early in most key tiles (steps of 32 rows: the band below a
+    # few hundred rows underflows)
+    steps, walked = ua.prefill_bwd_band_stats(shape, ws)
+    nkt = (T + 127) // 128
+    assert steps == Hkv * (nkt * 4 * nkt - 2 * nkt * (nkt - 1))
+    assert walked < steps // 2, (walked, steps)
     g = {k: v.float().cpu().numpy() for k, v in gr.items()}
     r = oracle.prefill_bwd(**x, scale=w.scale, theta=w.theta, variant=variant)
     rms = sum_model_rms(oracle.prefill_bwd, r, **x, scale=w.scale, theta=w.theta, variant=variant)
