@@ -676,8 +676,8 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
         uint8_t* tile_base = static_cast<uint8_t*>(p.tiles) + (size_t)unit * (G + 1) * tstride;
         const size_t band = band_off(kt, p.nkt);
         {
-            // below sfin: the rest of its 128-row block of stored tiles (the GEMMs sum whole blocks)
-            // and the rows' w sums (the post pass reads them) are zero
+            // below sfin: the rest of its 128-row block of stored tiles is zero (the GEMMs sum whole
+            // blocks; the post pass reads the rows' w sums of walked steps only)
             const int zend = min(4 * (sfin / 4) + 3, p.nst - 1);
             const int nz = (zend - sfin) * (int)(kTileBytes / 16);
             for (int g2 = 0; g2 <= G; ++g2) {
@@ -685,9 +685,6 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
                                                     (band + (sfin + 1 - s0)) * kTileBytes);
                 for (int i = tid; i < nz; i += 128 * kKeyQ) z[i] = make_uint4(0u, 0u, 0u, 0u);
             }
-            float4* dq4 = reinterpret_cast<float4*>(p.daq_part);
-            for (int r = ST * (sfin + 1) + tid; r < p.Tpk; r += 128 * kKeyQ)
-                dq4[((size_t)unit * p.Tpk + r) * p.nkt + kt] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         for (int it = 0; ok && it < nsteps; ++it) {
             const int s = sfin - it;
@@ -1257,13 +1254,15 @@ __global__ void __launch_bounds__(256) k_bwd_post_tc(BwdTcParams p) {
         }
     }
     // da_q: the row sums of w over the key tiles up to the row's and their four quarters (one
-    // float4 per key tile, contiguous per row), a warp per KV head; da_k from the key pass
+    // float4 per key tile, contiguous per row), a warp per KV head; key tiles whose walked steps
+    // stop above the row contribute 0 (their entries are not written); da_k from the key pass
     const int nk = t / 128 + 1;
     for (int h = warp; h < p.Hkv; h += 8) {
         const size_t u = (size_t)b * p.Hkv + h;
         const float4* part = reinterpret_cast<const float4*>(p.daq_part + (u * p.Tpk + t) * p.nkt * 4);
         float sw = 0.f;
         for (int kt = lane; kt < nk; kt += 32) {
+            if (last_step(p, (int)u, kt) < t / ST) continue;
             const float4 v = part[kt];
             sw += (v.x + v.y) + (v.z + v.w);
         }
