@@ -279,3 +279,29 @@ def test_binding_constants_match_the_header():
     body = re.search(r"typedef struct \{([^{}]*)\} ua_cache;", re.sub(r"/\*.*?\*/", "", txt, flags=re.S), re.S).group(1)
     fields = re.findall(r"(\w+)\s*[,;]", body)
     assert fields == [f for f, _ in ua.ua_cache._fields_], fields
+
+
+def test_bwd_band_stats_host_logic(lib):
+    """ua_prefill_bwd_band_stats: argument checks, and the band's step count for problems that
+    run the fp32 SIMT backward (no device access: it walks the whole band)."""
+    steps, walked = ctypes.c_ulonglong(7), ctypes.c_ulonglong(7)
+    s = _shape(B=2, T=300, H=4, Hkv=2, d=64, dtype=ua.UA_F32)
+    assert lib.ua_prefill_bwd_band_stats(ctypes.byref(s), None, 0, ctypes.byref(steps), ctypes.byref(walked),
+                                         None) == 0
+    nkt = (300 + 127) // 128                   # key tile kt meets 32-row steps 4kt .. 4nkt-1
+    assert steps.value == 2 * 2 * sum(4 * nkt - 4 * kt for kt in range(nkt))
+    assert walked.value == steps.value
+    assert lib.ua_prefill_bwd_band_stats(ctypes.byref(s), None, 0, None, ctypes.byref(walked), None) == 1
+    assert lib.ua_prefill_bwd_band_stats(None, None, 0, ctypes.byref(steps), ctypes.byref(walked), None) == 1
+    # training is dense: a pruning threshold is refused
+    pr = _shape(prune_p=0.15)
+    assert lib.ua_prefill_bwd_band_stats(ctypes.byref(pr), None, 0, ctypes.byref(steps), ctypes.byref(walked),
+                                         None) == 1
+    # the tensor-core backward needs the workspace it ran on, whole
+    tc = _shape(B=1, T=300, H=4, Hkv=1, d=64, dtype=ua.UA_BF16)
+    assert lib.ua_prefill_bwd_band_stats(ctypes.byref(tc), None, 0, ctypes.byref(steps), ctypes.byref(walked),
+                                         None) == 1
+    need = ctypes.c_size_t(0)
+    assert lib.ua_prefill_bwd_workspace_size(ctypes.byref(tc), ctypes.byref(need)) == 0
+    assert lib.ua_prefill_bwd_band_stats(ctypes.byref(tc), ctypes.c_void_p(FAKE), ctypes.c_size_t(need.value - 1),
+                                         ctypes.byref(steps), ctypes.byref(walked), None) == 4   # UA_ERR_WORKSPACE
