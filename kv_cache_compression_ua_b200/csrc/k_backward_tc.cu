@@ -947,9 +947,12 @@ k_bwd_key_tc(const __grid_constant__ CUtensorMap tm_khk, const __grid_constant__
 // dims run along the TMEM lanes (head_dim 64 uses the lower 64: the upper half of the A operand
 // points at a zero block).  Key side: per (key tile kt, unit): C[128 keys x dims] = sum_{rb >= kt}
 // dX^T_(kt, rb) khat_rb.  128 threads: warp 0 loads, warp 1 issues, all four write the result.
-// Grids (row blocks from the last, G + 1, units) and (key tiles, units).
+// Grids (row blocks from the last, G + 1, units) and (key tiles, units).  One operand stage per
+// CTA (64 KB), so two to three CTAs share an SM and overlap each other's copies, products and
+// epilogues: most sums are short once the underflowing band is skipped, and a three-stage ring in
+// one CTA per SM was slower (row GEMM 0.92 -> 0.71 ms on the 3B workload with one stage).
 namespace gemm {
-constexpr int NS = 3;
+constexpr int NS = 1;
 template <int DH>
 struct Smem {
     alignas(1024) uint8_t a[NS][2][16384];       // operand tile boxes [128][64] (rows side: keys; key side: rows)
